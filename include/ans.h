@@ -1,0 +1,220 @@
+/*
+ * ans.h -- C ABI of the tile-granular rANS weight codec and its fused
+ *          decode + GEMM for NVIDIA B200 (sm_100a).
+ *
+ * The operations follow "Approaching Shannon Bound with Lossless LLM Weight
+ * Compression" (blog summary, marsggbo.github.io, 2026-07-22):
+ *   s2.1  "熵分析：逐层算直方图"  a layer is a sequence of discrete symbols;
+ *         its histogram gives the Shannon entropy (ans_histogram, ans_entropy);
+ *   s2.2  "为什么大家不用无损压缩？"  rANS; tiles must decode independently;
+ *         decoded weights go to shared memory, never to global memory;
+ *   s3.1  "整体执行模型"  W is cut into GEMM-shaped tiles, all tiles of a layer
+ *         share one compact codebook, each tile's start is kept in an offset
+ *         index, each tile is split into R substreams with one rANS state per
+ *         warp lane (ans_encode_tiles, ans_gemm);
+ *   s4.1  "压缩率"  frequencies are normalised to a finite precision
+ *         (ans_build_codebook);
+ *   s4.2  "kernel 层面"  the layer-level decompress-then-GEMM baseline
+ *         (ans_decode_tiles followed by a dense GEMM).
+ * The bf16 split into an entropy-coded exponent and a raw sign/mantissa byte
+ * follows the DFloat11 summary "70%大小，100%准确！...", section
+ * "无损LLM压缩框架，实现高效GPU推理" (EncodedExponent / PackedSignMantissa).
+ *
+ * Stream format (fixed by this library; the pages leave these constants open):
+ *   probability precision 12 bits (frequencies sum to 4096), 32 lanes per
+ *   tile, 32-bit lane states in [2^16, 2^32), 16-bit renormalisation words.
+ *   Tile t = rb * (K / tile_k) + kt covers W rows [rb*tile_n, +tile_n) and
+ *   columns [kt*tile_k, +tile_k).  Lane l's j-th symbol is element
+ *     row = l + 32*(4h + i), col = 16s + 8c + kk   where  g = j/8, kk = j%8,
+ *     i = g%4, c = (g/4)%2, h = (g/8)%(tile_n/128), s = g/(8*(tile_n/128)).
+ *   Tile bytes: 32 little-endian u32 final encoder states (lane order), then
+ *   the u16 words in decoder order (step by step; within a step, lanes that
+ *   need a word take the next one in increasing lane order), then zero bytes
+ *   to a 16-byte boundary.  offsets[t] = byte start of tile t (16-byte
+ *   aligned), offsets[n_tiles] = total stream bytes.
+ *   bf16 raw side stream: tile_n*tile_k bytes per tile at t*tile_n*tile_k,
+ *   the raw byte (sign << 7 | 7-bit mantissa) of lane l's j-th symbol at
+ *   (j/8)*256 + l*8 + j%8.
+ *
+ * Weight storage ("original format"), row-major N x K:
+ *   ANS_INT4       packed nibbles, element k even in the low nibble, two's
+ *                  complement code q in [-8, 7]; coded symbol q + 8 (A = 16).
+ *   ANS_BF16_SPLIT uint16 bf16 bits; coded symbol = exponent byte (A = 256).
+ *   ANS_FP8_E4M3   e4m3fn code bytes; coded symbol = the code (A = 256).
+ *
+ * Conventions.  Every buffer belongs to the caller; the library allocates no
+ * device memory.  "d_" pointers are device pointers, "h_" host pointers.  GPU
+ * calls are asynchronous and stream-ordered on `stream` (a cudaStream_t; NULL
+ * is the legacy default stream).  Argument errors are returned synchronously;
+ * launch failures return ANS_ERR_CUDA (text via ans_last_error()).  Faults
+ * found while the kernel runs (a corrupt stream, a wait that ran out) are
+ * OR-ed into the caller's device word *d_status as ANS_STATUS_* bits; read it
+ * after synchronising.  No call traps or asserts on the device.
+ */
+#ifndef ANS_H_
+#define ANS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* ans_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  ANS_OK = 0,
+  ANS_ERR_ARG = 1,              /* null pointer, bad enum, misaligned pointer */
+  ANS_ERR_SHAPE = 2,            /* tile does not divide N/K, unsupported tile */
+  ANS_ERR_ALPHABET = 3,         /* bad codebook / symbol absent from it */
+  ANS_ERR_BUFFER_TOO_SMALL = 4, /* output or workspace capacity too small */
+  ANS_ERR_CUDA = 5,             /* a CUDA runtime call failed */
+  ANS_ERR_CORRUPT = 6,          /* host-side check found a corrupt stream */
+  ANS_ERR_TIMEOUT = 7,          /* reserved for host-side waits */
+  ANS_ERR_UNSUPPORTED = 8       /* no sm_100 device, or a size the kernels refuse */
+} ans_status;
+
+/* Bits OR-ed into *d_status by the device. */
+#define ANS_STATUS_CORRUPT 0x1u     /* a tile did not end at x = 2^16 in every lane, or
+                                       its words did not end at its last byte */
+#define ANS_STATUS_TIMEOUT 0x2u     /* a bounded wait inside a kernel ran out */
+#define ANS_STATUS_BAD_OFFSETS 0x4u /* an offset was unaligned, decreasing or past the end */
+
+typedef enum { ANS_INT4 = 0, ANS_BF16_SPLIT = 1, ANS_FP8_E4M3 = 2 } ans_dtype;
+
+typedef enum {
+  ANS_SCALE_NONE = 0,
+  ANS_SCALE_ROW_BF16 = 1,  /* scales: bf16[N]; w = q * s[n]            (int4) */
+  ANS_SCALE_ROW_F32 = 2,   /* scales: f32[N];  w = value * s[n]       (fp8, int4) */
+  ANS_SCALE_GROUP_BF16 = 3 /* scales: bf16[N][K/group_k]; w = q * s[n][k/group_k] (int4) */
+} ans_scale_kind;
+
+/* Shared per-layer codebook ("Approaching Shannon Bound", s3.1 and s4.1).
+ * freq[s] > 0 exactly for the symbols present in the layer; the freq sum to
+ * 2^prob_bits; cdf[s] = sum of freq[t] for t < s, cdf[alphabet] = 2^prob_bits. */
+typedef struct {
+  uint32_t alphabet;  /* 16 (int4) or 256 */
+  uint32_t prob_bits; /* 12 for the stream format; 1..15 accepted by ans_build_codebook */
+  uint16_t freq[256];
+  uint16_t cdf[257];
+  uint16_t reserved;
+} ans_codebook;
+
+typedef struct {
+  uint32_t dtype;  /* ans_dtype */
+  uint32_t N, K;   /* W is N x K (N = output features, K = reduction) */
+  uint32_t tile_n; /* 128 or 256 */
+  uint32_t tile_k; /* multiple of 16, at most 256 */
+} ans_layout;
+
+/* A compressed layer.  For GPU calls the three pointers are device pointers;
+ * the struct itself lives on the host and is read during the call only. */
+typedef struct {
+  ans_layout layout;
+  ans_codebook codebook;
+  const uint8_t* stream;   /* offsets[n_tiles] bytes */
+  uint64_t stream_bytes;
+  const uint64_t* offsets; /* n_tiles + 1 entries */
+  const uint8_t* raw;      /* ANS_BF16_SPLIT only: N*K bytes; else NULL */
+} ans_tiles;
+
+/* Human-readable name of a status code (static storage). */
+const char* ans_status_string(ans_status s);
+
+/* Text of the last CUDA error seen by this thread (static per thread). */
+const char* ans_last_error(void);
+
+/* Number of tiles of a layout, or 0 when the layout is invalid. */
+uint64_t ans_num_tiles(const ans_layout* layout);
+
+/* Validates a layout: N, K > 0, tile_n in {128, 256}, tile_k % 16 == 0,
+ * tile_k <= 256, N % tile_n == 0, K % tile_k == 0.  Returns ANS_ERR_SHAPE
+ * (or ANS_ERR_ARG for a bad dtype / NULL). */
+ans_status ans_layout_check(const ans_layout* layout);
+
+/* GPU histogram of the coded symbols of a layer ("Approaching Shannon Bound",
+ * s2.1: empirical histogram per layer).  d_w: the N*K weights in their
+ * original format; d_hist: uint64[alphabet], overwritten (zeroed first on
+ * `stream`).  Integer counts, so the result does not depend on scheduling. */
+ans_status ans_histogram(const void* d_w, const ans_layout* layout, uint64_t* d_hist,
+                         ans_stream_t stream);
+
+/* Host counterpart of ans_histogram for offline use without a GPU: h_w the
+ * N*K weights in their original format (host memory), hist uint64[alphabet]
+ * overwritten.  Multithreaded over rows; integer counts. */
+ans_status ans_histogram_host(const void* h_w, const ans_layout* layout, uint64_t* hist);
+
+/* Shannon entropy H = -sum p log2 p of a histogram, bits per symbol
+ * (DFloat11 summary, section "实验方法").  Host. */
+ans_status ans_entropy(const uint64_t* hist, uint32_t alphabet, double* bits_per_symbol);
+
+/* Normalises a histogram to integer frequencies summing to 2^prob_bits with
+ * freq > 0 exactly for the present symbols, minimising the coded size
+ * sum_s hist[s] * log2(2^prob_bits / freq[s]) ("Approaching Shannon Bound",
+ * s4.1).  Ties are broken towards the lower symbol index.  Host.
+ * Errors: ANS_ERR_ARG (empty histogram, alphabet not 16/256, prob_bits out of
+ * 1..15), ANS_ERR_ALPHABET (more present symbols than 2^prob_bits). */
+ans_status ans_build_codebook(const uint64_t* hist, uint32_t alphabet, uint32_t prob_bits,
+                              ans_codebook* out);
+
+/* Upper bound of the stream size ans_encode_tiles can produce for a layout. */
+ans_status ans_encode_bound(const ans_layout* layout, uint64_t* max_stream_bytes);
+
+/* Offline host encoder ("Approaching Shannon Bound", s3.1): codes every tile
+ * independently against `codebook` (prob_bits must be 12), writes the stream
+ * (h_stream, capacity `cap` bytes), the offset index (h_offsets, n_tiles + 1
+ * entries) and, for ANS_BF16_SPLIT, the raw side stream (h_raw, N*K bytes;
+ * may be NULL otherwise).  Multithreaded over tiles; the output does not
+ * depend on the thread count.  *stream_bytes receives the size even when
+ * ANS_ERR_BUFFER_TOO_SMALL is returned.  ANS_ERR_ALPHABET if a weight's
+ * symbol has zero frequency. */
+ans_status ans_encode_tiles(const void* h_w, const ans_layout* layout,
+                            const ans_codebook* codebook, uint8_t* h_stream, uint64_t cap,
+                            uint64_t* stream_bytes, uint64_t* h_offsets, uint8_t* h_raw);
+
+/* Standalone GPU decode to HBM: writes the original weights (format of the
+ * layout's dtype, row-major N x K) to d_out.  One warp per tile.  This is the
+ * bit-exactness check and the first half of the layer-level two-pass baseline
+ * ("Approaching Shannon Bound", s2.2 and s4.2).  d_status: device uint32. */
+ans_status ans_decode_tiles(const ans_tiles* tiles, void* d_out, uint32_t* d_status,
+                            ans_stream_t stream);
+
+/* Bytes of device workspace ans_gemm / ans_gemm_uncompressed need for a
+ * layout, M tokens and a scale kind.  The workspace must be zero-filled once
+ * before its first use; the kernels return it to all-zero counters on
+ * completion (after a run that set *d_status, zero it again). */
+ans_status ans_gemm_workspace(const ans_layout* layout, uint32_t M, ans_scale_kind scale_kind,
+                              size_t* bytes);
+
+/* Fused decode + GEMM ("Approaching Shannon Bound", s3.1):
+ *   Y[m][n] = sum_k X[m][k] * w(n, k),  Y fp32 M x N row-major,
+ * with X bf16 M x K row-major (16-byte aligned) and w the dequantised weight:
+ *   int4: q (NONE), q * s[n] (ROW_BF16 or ROW_F32), q * s[n][k/group_k]
+ *         (GROUP_BF16, group_k a multiple of 16 dividing K);
+ *   bf16: the bf16 value (NONE);  fp8: e4m3 value (NONE) or value * s[n] (ROW_F32).
+ * W's tiles are decoded by producer warps straight into shared memory in the
+ * tensor-core operand layout and consumed by tcgen05 MMAs; they never reach
+ * global memory.  Accumulation is fp32 in a fixed order, so the result is
+ * bit-identical to ans_gemm_uncompressed on the same weights.  GROUP_BF16 runs
+ * the MMA in f16 (X and q*s are exact in f16 when |X| < 65504 and the scales
+ * lie in [2^-14, 2^12]); all other kinds run it in bf16.
+ * M == 0 is a no-op.  d_ws: ans_gemm_workspace bytes. */
+ans_status ans_gemm(const uint16_t* d_X, uint32_t M, const ans_tiles* W,
+                    ans_scale_kind scale_kind, const void* d_scales, uint32_t group_k,
+                    float* d_Y, void* d_ws, size_t ws_bytes, uint32_t* d_status,
+                    ans_stream_t stream);
+
+/* The same kernel with the decoder warps replaced by a copy of the original
+ * (uncompressed) weights d_W (format of layout->dtype, row-major N x K).
+ * Bit-exact reference for ans_gemm and the uncompressed baseline. */
+ans_status ans_gemm_uncompressed(const uint16_t* d_X, uint32_t M, const void* d_W,
+                                 const ans_layout* layout, ans_scale_kind scale_kind,
+                                 const void* d_scales, uint32_t group_k, float* d_Y, void* d_ws,
+                                 size_t ws_bytes, uint32_t* d_status, ans_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ANS_H_ */

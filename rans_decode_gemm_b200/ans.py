@@ -1,0 +1,252 @@
+"""Python binding of the C ABI in ``include/ans.h`` (ctypes; argument
+marshalling only -- every step of the codec runs in ``libans.so``).
+
+Function names follow the C ABI.  Device buffers are torch CUDA tensors
+(passed by ``data_ptr()``), host buffers are numpy arrays, streams are
+``torch.cuda.Stream`` objects (default: the current stream).  A non-OK status
+raises :class:`AnsError`.  There is no fallback: if the library cannot be
+loaded, every call fails.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import threading
+
+import numpy as np
+
+from . import build as _build
+
+INT4, BF16_SPLIT, FP8_E4M3 = 0, 1, 2
+SCALE_NONE, SCALE_ROW_BF16, SCALE_ROW_F32, SCALE_GROUP_BF16 = 0, 1, 2, 3
+STATUS_CORRUPT, STATUS_TIMEOUT, STATUS_BAD_OFFSETS = 0x1, 0x2, 0x4
+ALPHABET = {INT4: 16, BF16_SPLIT: 256, FP8_E4M3: 256}
+
+# every symbol include/ans.h declares
+EXPORTS = ["ans_status_string", "ans_last_error", "ans_num_tiles", "ans_layout_check",
+           "ans_histogram", "ans_histogram_host", "ans_entropy", "ans_build_codebook", "ans_encode_bound",
+           "ans_encode_tiles", "ans_decode_tiles", "ans_gemm_workspace", "ans_gemm",
+           "ans_gemm_uncompressed"]
+
+
+class AnsError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str = ""):
+        self.status = status
+        super().__init__(f"{where}: status {status} ({_status_text(status)})"
+                         + (f": {detail}" if detail else ""))
+
+
+class AnsCodebook(C.Structure):
+    _fields_ = [("alphabet", C.c_uint32), ("prob_bits", C.c_uint32),
+                ("freq", C.c_uint16 * 256), ("cdf", C.c_uint16 * 257), ("reserved", C.c_uint16)]
+
+    def freq_array(self) -> np.ndarray:
+        return np.ctypeslib.as_array(self.freq)[:self.alphabet].astype(np.uint32)
+
+
+class AnsLayout(C.Structure):
+    _fields_ = [("dtype", C.c_uint32), ("N", C.c_uint32), ("K", C.c_uint32),
+                ("tile_n", C.c_uint32), ("tile_k", C.c_uint32)]
+
+
+class AnsTiles(C.Structure):
+    _fields_ = [("layout", AnsLayout), ("codebook", AnsCodebook), ("stream", C.c_void_p),
+                ("stream_bytes", C.c_uint64), ("offsets", C.c_void_p), ("raw", C.c_void_p)]
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def load():
+    """Loads (building in-tree first if missing or stale) libans.so."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = _build.build()
+            L = C.CDLL(path)
+            P, u32, u64, i32, sz = C.c_void_p, C.c_uint32, C.c_uint64, C.c_int, C.c_size_t
+            L.ans_status_string.argtypes = [i32]
+            L.ans_status_string.restype = C.c_char_p
+            L.ans_last_error.argtypes = []
+            L.ans_last_error.restype = C.c_char_p
+            L.ans_num_tiles.argtypes = [P]
+            L.ans_num_tiles.restype = u64
+            L.ans_layout_check.argtypes = [P]
+            L.ans_histogram.argtypes = [P, P, P, P]
+            L.ans_histogram_host.argtypes = [P, P, P]
+            L.ans_entropy.argtypes = [P, u32, P]
+            L.ans_build_codebook.argtypes = [P, u32, u32, P]
+            L.ans_encode_bound.argtypes = [P, P]
+            L.ans_encode_tiles.argtypes = [P, P, P, P, u64, P, P, P]
+            L.ans_decode_tiles.argtypes = [P, P, P, P]
+            L.ans_gemm_workspace.argtypes = [P, u32, i32, P]
+            L.ans_gemm.argtypes = [P, u32, P, i32, P, u32, P, P, sz, P, P]
+            L.ans_gemm_uncompressed.argtypes = [P, u32, P, P, i32, P, u32, P, P, sz, P, P]
+            for name in EXPORTS:
+                if name not in ("ans_status_string", "ans_last_error", "ans_num_tiles"):
+                    getattr(L, name).restype = i32
+            _lib = L
+    return _lib
+
+
+def _status_text(st: int) -> str:
+    try:
+        return load().ans_status_string(st).decode()
+    except Exception:  # noqa: BLE001 - only used to decorate an error message
+        return "?"
+
+
+def _check(st: int, where: str):
+    if st != 0:
+        raise AnsError(st, where, load().ans_last_error().decode())
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, np.ndarray):
+        return t.ctypes.data_as(C.c_void_p)
+    return C.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return C.c_void_p(stream.cuda_stream)
+
+
+def make_layout(dtype: int, N: int, K: int, tile_n: int, tile_k: int) -> AnsLayout:
+    return AnsLayout(dtype, N, K, tile_n, tile_k)
+
+
+# ---- the C ABI, one Python function per entry point -----------------------------
+def ans_status_string(st: int) -> str:
+    return load().ans_status_string(st).decode()
+
+
+def ans_last_error() -> str:
+    return load().ans_last_error().decode()
+
+
+def ans_num_tiles(layout: AnsLayout) -> int:
+    return load().ans_num_tiles(C.byref(layout))
+
+
+def ans_layout_check(layout: AnsLayout) -> int:
+    return load().ans_layout_check(C.byref(layout))
+
+
+def ans_histogram(d_w, layout: AnsLayout, d_hist, stream=None):
+    _check(load().ans_histogram(_ptr(d_w), C.byref(layout), _ptr(d_hist), _stream(stream)),
+           "ans_histogram")
+
+
+def ans_histogram_host(h_w: np.ndarray, layout: AnsLayout) -> np.ndarray:
+    h_w = np.ascontiguousarray(h_w)
+    hist = np.zeros(ALPHABET[layout.dtype], np.uint64)
+    _check(load().ans_histogram_host(_ptr(h_w), C.byref(layout), _ptr(hist)),
+           "ans_histogram_host")
+    return hist
+
+
+def ans_entropy(hist) -> float:
+    h = np.ascontiguousarray(hist, dtype=np.uint64)
+    out = C.c_double(0)
+    _check(load().ans_entropy(_ptr(h), h.size, C.byref(out)), "ans_entropy")
+    return out.value
+
+
+def ans_build_codebook(hist, alphabet: int | None = None, prob_bits: int = 12) -> AnsCodebook:
+    h = np.ascontiguousarray(hist, dtype=np.uint64)
+    cb = AnsCodebook()
+    _check(load().ans_build_codebook(_ptr(h), alphabet or h.size, prob_bits, C.byref(cb)),
+           "ans_build_codebook")
+    return cb
+
+
+def ans_encode_bound(layout: AnsLayout) -> int:
+    out = C.c_uint64(0)
+    _check(load().ans_encode_bound(C.byref(layout), C.byref(out)), "ans_encode_bound")
+    return out.value
+
+
+def ans_encode_tiles(h_w: np.ndarray, layout: AnsLayout, codebook: AnsCodebook):
+    """Returns (stream uint8[], offsets uint64[n_tiles + 1], raw uint8[] or None)."""
+    h_w = np.ascontiguousarray(h_w)
+    cap = ans_encode_bound(layout)
+    stream = np.empty(max(cap, 16), np.uint8)
+    offsets = np.empty(ans_num_tiles(layout) + 1, np.uint64)
+    raw = np.empty(layout.N * layout.K, np.uint8) if layout.dtype == BF16_SPLIT else None
+    nbytes = C.c_uint64(0)
+    _check(load().ans_encode_tiles(_ptr(h_w), C.byref(layout), C.byref(codebook), _ptr(stream),
+                                   cap, C.byref(nbytes), _ptr(offsets), _ptr(raw)),
+           "ans_encode_tiles")
+    return stream[:nbytes.value], offsets, raw
+
+
+def ans_decode_tiles(tiles: AnsTiles, d_out, d_status, stream=None):
+    _check(load().ans_decode_tiles(C.byref(tiles), _ptr(d_out), _ptr(d_status), _stream(stream)),
+           "ans_decode_tiles")
+
+
+def ans_gemm_workspace(layout: AnsLayout, M: int, scale_kind: int = SCALE_NONE) -> int:
+    out = C.c_size_t(0)
+    _check(load().ans_gemm_workspace(C.byref(layout), M, scale_kind, C.byref(out)),
+           "ans_gemm_workspace")
+    return out.value
+
+
+def ans_gemm(d_X, M: int, tiles: AnsTiles, scale_kind: int, d_scales, group_k: int, d_Y, d_ws,
+             ws_bytes: int, d_status, stream=None):
+    _check(load().ans_gemm(_ptr(d_X), M, C.byref(tiles), scale_kind, _ptr(d_scales), group_k,
+                           _ptr(d_Y), _ptr(d_ws), ws_bytes, _ptr(d_status), _stream(stream)),
+           "ans_gemm")
+
+
+def ans_gemm_uncompressed(d_X, M: int, d_W, layout: AnsLayout, scale_kind: int, d_scales,
+                          group_k: int, d_Y, d_ws, ws_bytes: int, d_status, stream=None):
+    _check(load().ans_gemm_uncompressed(_ptr(d_X), M, _ptr(d_W), C.byref(layout), scale_kind,
+                                        _ptr(d_scales), group_k, _ptr(d_Y), _ptr(d_ws),
+                                        ws_bytes, _ptr(d_status), _stream(stream)),
+           "ans_gemm_uncompressed")
+
+
+# ---- marshalling helper: a compressed layer resident on a device -----------------
+class CompressedLayer:
+    """Host encode result uploaded to device tensors, plus the ans_tiles struct
+    pointing at them.  Holds references so the device buffers stay alive."""
+
+    def __init__(self, layout: AnsLayout, codebook: AnsCodebook, stream: np.ndarray,
+                 offsets: np.ndarray, raw: np.ndarray | None, device="cuda"):
+        import torch
+        self.layout = layout
+        self.codebook = codebook
+        self.h_stream, self.h_offsets, self.h_raw = stream, offsets, raw
+        n = max(16, (stream.size + 15) // 16 * 16)
+        self.d_stream = torch.zeros(n, dtype=torch.uint8, device=device)
+        if stream.size:
+            self.d_stream[:stream.size].copy_(torch.from_numpy(stream))
+        self.d_offsets = torch.from_numpy(offsets.view(np.int64)).to(device)
+        self.d_raw = torch.from_numpy(raw).to(device) if raw is not None else None
+        self.tiles = AnsTiles(layout, codebook, self.d_stream.data_ptr(), stream.size,
+                              self.d_offsets.data_ptr(),
+                              self.d_raw.data_ptr() if self.d_raw is not None else None)
+
+    @property
+    def compressed_bytes(self) -> int:
+        """Stream + offset index + codebook + raw side stream."""
+        cb = 2 * self.codebook.alphabet
+        return int(self.h_stream.size + self.h_offsets.size * 8 + cb +
+                   (self.h_raw.size if self.h_raw is not None else 0))
+
+    @classmethod
+    def from_weights(cls, h_w: np.ndarray, layout: AnsLayout, hist=None, device="cuda"):
+        """Offline path through the library: histogram (ans_histogram_host
+        unless given) -> ans_build_codebook -> ans_encode_tiles -> upload."""
+        if hist is None:
+            hist = ans_histogram_host(h_w, layout)
+        cb = ans_build_codebook(hist, ALPHABET[layout.dtype], 12)
+        stream, offsets, raw = ans_encode_tiles(h_w, layout, cb)
+        return cls(layout, cb, stream, offsets, raw, device)

@@ -1,0 +1,61 @@
+"""Builds the in-tree C-ABI library ``libans.so`` (host codec + sm_100a kernels)
+with nvcc.  Called by ``__graft_entry__.build()`` and, when the library is
+missing or older than its sources, by the Python binding."""
+from __future__ import annotations
+
+import glob
+import os
+import subprocess
+import sys
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+CSRC = os.path.join(PKG, "csrc")
+LIB = os.path.join(PKG, "libans.so")
+NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def sources():
+    return sorted(glob.glob(os.path.join(CSRC, "**", "*.cu"), recursive=True) +
+                  glob.glob(os.path.join(CSRC, "**", "*.cpp"), recursive=True))
+
+
+def headers():
+    return (glob.glob(os.path.join(CSRC, "**", "*.h"), recursive=True) +
+            glob.glob(os.path.join(CSRC, "**", "*.cuh"), recursive=True) +
+            [os.path.join(ROOT, "include", "ans.h")])
+
+
+def stale() -> bool:
+    if not os.path.exists(LIB):
+        return True
+    t = os.path.getmtime(LIB)
+    return any(os.path.getmtime(f) > t for f in sources() + headers() + [__file__])
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    if not force and not stale():
+        return LIB
+    build_dir = os.path.join(ROOT, "_build")
+    os.makedirs(build_dir, exist_ok=True)
+    objs = []
+    for src in sources():
+        obj = os.path.join(build_dir, os.path.relpath(src, CSRC).replace(os.sep, "_") + ".o")
+        cmd = [NVCC, *ARCH, "-lineinfo", "-O3", "-std=c++17", "-Xcompiler", "-fPIC,-pthread",
+               "-I", os.path.join(ROOT, "include"), "-I", CSRC, "-c", src, "-o", obj]
+        if src.endswith(".cu"):
+            cmd[1:1] = ["-Xptxas", "-v"] if verbose else []
+        if verbose:
+            print(" ".join(cmd), file=sys.stderr)
+        subprocess.check_call(cmd)
+        objs.append(obj)
+    tmp = LIB + f".tmp{os.getpid()}"
+    subprocess.check_call([NVCC, *ARCH, "-shared", "-Xcompiler", "-fPIC", "-o", tmp, *objs,
+                           "-lpthread"])
+    os.replace(tmp, LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))

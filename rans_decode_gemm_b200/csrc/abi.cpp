@@ -1,0 +1,329 @@
+// abi.cpp -- the extern "C" boundary declared in include/ans.h: argument
+// validation, codebook checks, and dispatch to the host codec or the CUDA
+// kernels.  No device memory is allocated here.
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/ans.h"
+#include "cuda/kernels.h"
+#include "host/codec_host.h"
+
+namespace {
+
+thread_local char g_last_error[256] = "";
+
+ans_status cuda_fail(cudaError_t e, const char* where) {
+  std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%d)", where, cudaGetErrorString(e),
+                static_cast<int>(e));
+  return ANS_ERR_CUDA;
+}
+
+uint32_t alphabet_of(uint32_t dtype) { return dtype == ANS_INT4 ? 16u : 256u; }
+
+ans_status check_layout(const ans_layout* l) {
+  if (!l) return ANS_ERR_ARG;
+  if (l->dtype > ANS_FP8_E4M3) return ANS_ERR_ARG;
+  if (!anshost::layout_valid(l->N, l->K, l->tile_n, l->tile_k)) return ANS_ERR_SHAPE;
+  return ANS_OK;
+}
+
+// Stream-format codebook: alphabet of the dtype, 12-bit precision, freq
+// summing to 4096, cdf consistent with freq.
+ans_status check_codebook(const ans_codebook* cb, uint32_t dtype) {
+  if (!cb) return ANS_ERR_ARG;
+  if (cb->alphabet != alphabet_of(dtype) || cb->prob_bits != 12) return ANS_ERR_ALPHABET;
+  uint32_t run = 0;
+  for (uint32_t s = 0; s < cb->alphabet; ++s) {
+    if (cb->cdf[s] != run) return ANS_ERR_ALPHABET;
+    run += cb->freq[s];
+  }
+  if (run != 4096 || cb->cdf[cb->alphabet] != 4096) return ANS_ERR_ALPHABET;
+  return ANS_OK;
+}
+
+ans_status device_info(int* num_sms) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  static int cached_sms[64];
+  static int cached_major[64];
+  if (dev < 0 || dev >= 64) return ANS_ERR_UNSUPPORTED;
+  if (cached_sms[dev] == 0) {
+    int sms = 0, major = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    cached_major[dev] = major;
+    cached_sms[dev] = sms;
+  }
+  if (cached_major[dev] != 10) {
+    std::snprintf(g_last_error, sizeof(g_last_error),
+                  "kernels are built for sm_100a; device major = %d", cached_major[dev]);
+    return ANS_ERR_UNSUPPORTED;
+  }
+  *num_sms = cached_sms[dev];
+  return ANS_OK;
+}
+
+void fill_layer(const ans_tiles* t, ansdev::LayerDev* L) {
+  std::memset(L, 0, sizeof(*L));
+  const ans_layout& ly = t->layout;
+  L->stream = t->stream;
+  L->offsets = t->offsets;
+  L->raw = t->raw;
+  L->stream_bytes = t->stream_bytes;
+  L->N = ly.N;
+  L->K = ly.K;
+  L->tile_n = ly.tile_n;
+  L->tile_k = ly.tile_k;
+  L->n_kt = ly.K / ly.tile_k;
+  L->n_tiles = (ly.N / ly.tile_n) * L->n_kt;
+  L->dtype = ly.dtype;
+  L->alphabet = t->codebook.alphabet;
+  L->single_symbol = ansdev::kNoSymbolHost;
+  for (uint32_t s = 0; s < t->codebook.alphabet; ++s) {
+    L->freq[s] = t->codebook.freq[s];
+    L->cdf[s] = t->codebook.cdf[s];
+    if (t->codebook.freq[s] == 4096) L->single_symbol = s;
+  }
+  L->cdf[t->codebook.alphabet] = t->codebook.cdf[t->codebook.alphabet];
+}
+
+// Layout-only LayerDev (copy mode and planning).
+void fill_layer_plain(const ans_layout* ly, ansdev::LayerDev* L) {
+  std::memset(L, 0, sizeof(*L));
+  L->N = ly->N;
+  L->K = ly->K;
+  L->tile_n = ly->tile_n;
+  L->tile_k = ly->tile_k;
+  L->n_kt = ly->K / ly->tile_k;
+  L->n_tiles = (ly->N / ly->tile_n) * L->n_kt;
+  L->dtype = ly->dtype;
+  L->alphabet = alphabet_of(ly->dtype);
+  L->single_symbol = ansdev::kNoSymbolHost;
+}
+
+ans_status check_scales(uint32_t dtype, ans_scale_kind kind, const void* scales, uint32_t group_k,
+                        const ans_layout& ly) {
+  switch (kind) {
+    case ANS_SCALE_NONE: return ANS_OK;
+    case ANS_SCALE_ROW_BF16:
+    case ANS_SCALE_ROW_F32: return scales ? ANS_OK : ANS_ERR_ARG;
+    case ANS_SCALE_GROUP_BF16:
+      if (dtype != ANS_INT4 || !scales) return ANS_ERR_ARG;
+      if (group_k == 0 || group_k % 16 != 0 || ly.K % group_k != 0) return ANS_ERR_ARG;
+      if (group_k % ly.tile_k != 0) return ANS_ERR_UNSUPPORTED;
+      return ANS_OK;
+  }
+  return ANS_ERR_ARG;
+}
+
+ans_status run_gemm(const uint16_t* d_X, uint32_t M, const ansdev::LayerDev& L, bool decode,
+                    const void* d_W, ans_scale_kind kind, const void* d_scales, uint32_t group_k,
+                    float* d_Y, void* d_ws, size_t ws_bytes, uint32_t* d_status,
+                    ans_stream_t stream) {
+  if (M == 0) return ANS_OK;
+  if (!d_X || !d_Y || !d_status || !d_ws) return ANS_ERR_ARG;
+  if (reinterpret_cast<uintptr_t>(d_X) % 16 != 0) return ANS_ERR_ARG;
+  int sms = 0;
+  ans_status st = device_info(&sms);
+  if (st != ANS_OK) return st;
+  ansdev::GemmPlan plan;
+  if (!ansdev::make_gemm_plan(L, M, kind, decode, sms, &plan)) return ANS_ERR_UNSUPPORTED;
+  if (ws_bytes < plan.ws_bytes) return ANS_ERR_BUFFER_TOO_SMALL;
+  cudaError_t e = ansdev::launch_gemm(plan, L, decode, d_W, d_X, d_scales, kind, group_k, d_Y,
+                                      d_ws, d_status, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, decode ? "ans_gemm" : "ans_gemm_uncompressed");
+  return ANS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ans_status_string(ans_status s) {
+  switch (s) {
+    case ANS_OK: return "ok";
+    case ANS_ERR_ARG: return "invalid argument";
+    case ANS_ERR_SHAPE: return "unsupported shape";
+    case ANS_ERR_ALPHABET: return "invalid codebook or symbol outside it";
+    case ANS_ERR_BUFFER_TOO_SMALL: return "buffer too small";
+    case ANS_ERR_CUDA: return "CUDA error";
+    case ANS_ERR_CORRUPT: return "corrupt stream";
+    case ANS_ERR_TIMEOUT: return "timeout";
+    case ANS_ERR_UNSUPPORTED: return "unsupported";
+  }
+  return "unknown status";
+}
+
+const char* ans_last_error(void) { return g_last_error; }
+
+uint64_t ans_num_tiles(const ans_layout* layout) {
+  if (check_layout(layout) != ANS_OK) return 0;
+  return static_cast<uint64_t>(layout->N / layout->tile_n) * (layout->K / layout->tile_k);
+}
+
+ans_status ans_layout_check(const ans_layout* layout) { return check_layout(layout); }
+
+ans_status ans_histogram(const void* d_w, const ans_layout* layout, uint64_t* d_hist,
+                         ans_stream_t stream) {
+  if (!layout || layout->dtype > ANS_FP8_E4M3) return ANS_ERR_ARG;
+  if (layout->N == 0 || layout->K == 0) return ANS_ERR_SHAPE;
+  if (layout->dtype == ANS_INT4 && layout->K % 2 != 0) return ANS_ERR_SHAPE;
+  if (!d_w || !d_hist || reinterpret_cast<uintptr_t>(d_w) % 16 != 0) return ANS_ERR_ARG;
+  int sms = 0;
+  ans_status st = device_info(&sms);
+  if (st != ANS_OK) return st;
+  const uint64_t n = static_cast<uint64_t>(layout->N) * layout->K;
+  const uint64_t bytes = layout->dtype == ANS_INT4 ? n / 2 : (layout->dtype == ANS_BF16_SPLIT ? 2 * n : n);
+  cudaError_t e = ansdev::launch_histogram(d_w, bytes, layout->dtype, d_hist,
+                                           reinterpret_cast<cudaStream_t>(stream), sms);
+  if (e != cudaSuccess) return cuda_fail(e, "ans_histogram");
+  return ANS_OK;
+}
+
+ans_status ans_histogram_host(const void* h_w, const ans_layout* layout, uint64_t* hist) {
+  if (!layout || layout->dtype > ANS_FP8_E4M3) return ANS_ERR_ARG;
+  if (layout->N == 0 || layout->K == 0) return ANS_ERR_SHAPE;
+  if (layout->dtype == ANS_INT4 && layout->K % 2 != 0) return ANS_ERR_SHAPE;
+  if (!h_w || !hist) return ANS_ERR_ARG;
+  anshost::histogram(layout->dtype, h_w, static_cast<uint64_t>(layout->N) * layout->K, hist);
+  return ANS_OK;
+}
+
+ans_status ans_entropy(const uint64_t* hist, uint32_t alphabet, double* bits_per_symbol) {
+  if (!hist || !bits_per_symbol || alphabet == 0 || alphabet > 256) return ANS_ERR_ARG;
+  *bits_per_symbol = anshost::entropy_bits(hist, alphabet);
+  return ANS_OK;
+}
+
+ans_status ans_build_codebook(const uint64_t* hist, uint32_t alphabet, uint32_t prob_bits,
+                              ans_codebook* out) {
+  if (!hist || !out || (alphabet != 16 && alphabet != 256)) return ANS_ERR_ARG;
+  uint32_t freq[256] = {0};
+  int r = anshost::normalize(hist, alphabet, prob_bits, freq);
+  if (r == 1) return ANS_ERR_ARG;
+  if (r == 3) return ANS_ERR_ALPHABET;
+  std::memset(out, 0, sizeof(*out));
+  out->alphabet = alphabet;
+  out->prob_bits = prob_bits;
+  uint32_t run = 0;
+  for (uint32_t s = 0; s < alphabet; ++s) {
+    out->freq[s] = static_cast<uint16_t>(freq[s]);
+    out->cdf[s] = static_cast<uint16_t>(run);
+    run += freq[s];
+  }
+  out->cdf[alphabet] = static_cast<uint16_t>(run);
+  return ANS_OK;
+}
+
+ans_status ans_encode_bound(const ans_layout* layout, uint64_t* max_stream_bytes) {
+  ans_status st = check_layout(layout);
+  if (st != ANS_OK) return st;
+  if (!max_stream_bytes) return ANS_ERR_ARG;
+  *max_stream_bytes = anshost::encode_bound(layout->N, layout->K, layout->tile_n, layout->tile_k);
+  return ANS_OK;
+}
+
+ans_status ans_encode_tiles(const void* h_w, const ans_layout* layout,
+                            const ans_codebook* codebook, uint8_t* h_stream, uint64_t cap,
+                            uint64_t* stream_bytes, uint64_t* h_offsets, uint8_t* h_raw) {
+  ans_status st = check_layout(layout);
+  if (st != ANS_OK) return st;
+  if (!h_w || !h_stream || !stream_bytes || !h_offsets) return ANS_ERR_ARG;
+  if (layout->dtype == ANS_BF16_SPLIT && !h_raw) return ANS_ERR_ARG;
+  st = check_codebook(codebook, layout->dtype);
+  if (st != ANS_OK) return st;
+  uint32_t freq[256] = {0};
+  for (uint32_t s = 0; s < codebook->alphabet; ++s) freq[s] = codebook->freq[s];
+  int r = anshost::encode(layout->dtype, h_w, layout->N, layout->K, layout->tile_n,
+                          layout->tile_k, freq, h_stream, cap, stream_bytes, h_offsets, h_raw);
+  if (r == 3) return ANS_ERR_ALPHABET;
+  if (r == 4) return ANS_ERR_BUFFER_TOO_SMALL;
+  return r == 0 ? ANS_OK : ANS_ERR_ARG;
+}
+
+ans_status ans_decode_tiles(const ans_tiles* tiles, void* d_out, uint32_t* d_status,
+                            ans_stream_t stream) {
+  if (!tiles || !d_out || !d_status) return ANS_ERR_ARG;
+  ans_status st = check_layout(&tiles->layout);
+  if (st != ANS_OK) return st;
+  st = check_codebook(&tiles->codebook, tiles->layout.dtype);
+  if (st != ANS_OK) return st;
+  if (!tiles->stream || !tiles->offsets) return ANS_ERR_ARG;
+  if (tiles->layout.dtype == ANS_BF16_SPLIT && !tiles->raw) return ANS_ERR_ARG;
+  if (reinterpret_cast<uintptr_t>(d_out) % 16 != 0 ||
+      reinterpret_cast<uintptr_t>(tiles->stream) % 16 != 0 ||
+      reinterpret_cast<uintptr_t>(tiles->offsets) % 8 != 0 ||
+      (tiles->raw && reinterpret_cast<uintptr_t>(tiles->raw) % 8 != 0))
+    return ANS_ERR_ARG;
+  int sms = 0;
+  st = device_info(&sms);
+  if (st != ANS_OK) return st;
+  ansdev::LayerDev L;
+  fill_layer(tiles, &L);
+  cudaError_t e = ansdev::launch_decode_tiles(L, d_out, d_status,
+                                              reinterpret_cast<cudaStream_t>(stream), sms);
+  if (e != cudaSuccess) return cuda_fail(e, "ans_decode_tiles");
+  return ANS_OK;
+}
+
+ans_status ans_gemm_workspace(const ans_layout* layout, uint32_t M, ans_scale_kind scale_kind,
+                              size_t* bytes) {
+  ans_status st = check_layout(layout);
+  if (st != ANS_OK) return st;
+  if (!bytes) return ANS_ERR_ARG;
+  if (M == 0) { *bytes = 0; return ANS_OK; }
+  int sms = 0;
+  st = device_info(&sms);
+  if (st != ANS_OK) return st;
+  ansdev::LayerDev L;
+  fill_layer_plain(layout, &L);
+  ansdev::GemmPlan plan;
+  if (!ansdev::make_gemm_plan(L, M, scale_kind, true, sms, &plan)) return ANS_ERR_UNSUPPORTED;
+  *bytes = plan.ws_bytes;
+  return ANS_OK;
+}
+
+ans_status ans_gemm(const uint16_t* d_X, uint32_t M, const ans_tiles* W,
+                    ans_scale_kind scale_kind, const void* d_scales, uint32_t group_k,
+                    float* d_Y, void* d_ws, size_t ws_bytes, uint32_t* d_status,
+                    ans_stream_t stream) {
+  if (!W) return ANS_ERR_ARG;
+  ans_status st = check_layout(&W->layout);
+  if (st != ANS_OK) return st;
+  st = check_codebook(&W->codebook, W->layout.dtype);
+  if (st != ANS_OK) return st;
+  st = check_scales(W->layout.dtype, scale_kind, d_scales, group_k, W->layout);
+  if (st != ANS_OK) return st;
+  if (!W->stream || !W->offsets) return ANS_ERR_ARG;
+  if (W->layout.dtype == ANS_BF16_SPLIT && !W->raw) return ANS_ERR_ARG;
+  if (reinterpret_cast<uintptr_t>(W->stream) % 16 != 0 ||
+      reinterpret_cast<uintptr_t>(W->offsets) % 8 != 0 ||
+      (W->raw && reinterpret_cast<uintptr_t>(W->raw) % 8 != 0))
+    return ANS_ERR_ARG;
+  ansdev::LayerDev L;
+  fill_layer(W, &L);
+  return run_gemm(d_X, M, L, true, nullptr, scale_kind, d_scales, group_k, d_Y, d_ws, ws_bytes,
+                  d_status, stream);
+}
+
+ans_status ans_gemm_uncompressed(const uint16_t* d_X, uint32_t M, const void* d_W,
+                                 const ans_layout* layout, ans_scale_kind scale_kind,
+                                 const void* d_scales, uint32_t group_k, float* d_Y, void* d_ws,
+                                 size_t ws_bytes, uint32_t* d_status, ans_stream_t stream) {
+  ans_status st = check_layout(layout);
+  if (st != ANS_OK) return st;
+  if (!d_W || reinterpret_cast<uintptr_t>(d_W) % 16 != 0) return ANS_ERR_ARG;
+  st = check_scales(layout->dtype, scale_kind, d_scales, group_k, *layout);
+  if (st != ANS_OK) return st;
+  ansdev::LayerDev L;
+  fill_layer_plain(layout, &L);
+  return run_gemm(d_X, M, L, false, d_W, scale_kind, d_scales, group_k, d_Y, d_ws, ws_bytes,
+                  d_status, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,675 @@
+// gemm.cu -- fused tile-rANS decode + GEMM on sm_100a (tcgen05 / TMEM / TMA).
+//
+// "Approaching Shannon Bound with Lossless LLM Weight Compression", s3.1
+// "整体执行模型": producer warps decode compressed weight tiles straight into
+// shared memory while other warps feed the tensor cores; decoding tile k+1
+// overlaps the MMA on tile k; shared-memory stages are released in a fixed
+// order given by the traversal, with no run-time reference counting.
+//
+// B200 design (swap-AB, Y^T = W X^T):
+//   * A operand = a 128-row x 16-column slab of W (K-major, 32-byte swizzle),
+//     written by a producer warp with 16-byte st.shared; B operand = X slab
+//     (T tokens x 16 columns) brought in by TMA; fp32 accumulators in TMEM
+//     (128 lanes = W rows, T columns = tokens).
+//   * Warp roles: 0-3 epilogue (TMEM -> registers -> Y or split-K partial),
+//     4 MMA issue (one thread), 5 X loader (TMA, one thread), 6.. producers
+//     (rANS decoders in ans_gemm, plain copies in ans_gemm_uncompressed).
+//   * Each producer owns a two-slot ring of 4 KB slabs; every pipeline edge is
+//     an mbarrier (tcgen05.commit releases slabs and X stages).
+//   * Static schedule: the tile units (token pass, W row block, K tile) are
+//     split into one contiguous range per CTA; inside a CTA, round r gives
+//     unit u_begin + r*D + d to producer d; the MMA thread consumes slabs in a
+//     fixed order, so accumulation order (hence every bit of Y) does not
+//     depend on timing and matches ans_gemm_uncompressed exactly.
+//   * A W row block split over several CTAs is reduced by the last CTA to
+//     finish it, in ascending CTA order (deterministic, no float atomics).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdlib>
+#include <cstring>
+
+#include "kernels.h"
+#include "rans_core.cuh"
+
+namespace ansdev {
+
+constexpr uint32_t kSlabBytes = 128 * 32;  // 128 rows x 16 bf16
+constexpr uint32_t kFixedWarps = 6;
+constexpr uint32_t kMaxProducers = 16;
+constexpr uint32_t kMaxThreads = (kFixedWarps + kMaxProducers) * 32;
+constexpr uint32_t kSmemLimit = 232448 - 4096;  // sm_100 per-block maximum, less static smem
+
+struct Bars {
+  uint64_t *w_full, *w_empty, *x_full, *x_empty, *acc_full, *acc_empty, *mma_done, *chunk;
+};
+
+__device__ __forceinline__ Bars carve_bars(uint8_t* base, uint32_t D, uint32_t XS) {
+  uint64_t* b = reinterpret_cast<uint64_t*>(base);
+  Bars r;
+  r.w_full = b;
+  r.w_empty = b + 2 * D;
+  r.x_full = b + 4 * D;
+  r.x_empty = b + 4 * D + XS;
+  r.acc_full = b + 4 * D + 2 * XS;
+  r.acc_empty = r.acc_full + 2;
+  r.mma_done = r.acc_empty + 2;
+  r.chunk = r.mma_done + 1;
+  return r;
+}
+
+__host__ __device__ inline uint32_t num_bars(uint32_t D, uint32_t XS) {
+  return 4 * D + 2 * XS + 5 + 4 * D;
+}
+
+__device__ __forceinline__ uint64_t cta_begin(uint64_t U, uint32_t G, uint32_t c) {
+  return U * c / G;
+}
+
+// CTA whose range contains unit u.
+__device__ __forceinline__ uint32_t cta_of(uint64_t U, uint32_t G, uint64_t u) {
+  uint32_t c = static_cast<uint32_t>(u * G / U);
+  while (c + 1 < G && cta_begin(U, G, c + 1) <= u) ++c;
+  while (c > 0 && cta_begin(U, G, c) > u) --c;
+  return c;
+}
+
+// Calls f(u, s, d) in the order the MMA thread consumes (unit, slab) pairs.
+// With two accumulator sets a round is consumed slab-major across all its
+// units; with one set, the units of each segment of the round are finished
+// before the next segment starts (so its accumulator can be drained first).
+// Either way the order within one segment is (slab, unit) ascending.
+template <class F>
+__device__ __forceinline__ void for_each_mma_step(const GemmDev& P, uint64_t u_begin,
+                                                  uint64_t u_end, F&& f) {
+  const uint32_t n_kt = P.L.n_kt;
+  for (uint64_t u0 = u_begin; u0 < u_end; u0 += P.D) {
+    const uint32_t nd = static_cast<uint32_t>(u_end - u0 < P.D ? u_end - u0 : P.D);
+    if (P.n_bufs == 2) {
+      for (uint32_t s = 0; s < P.C; ++s)
+        for (uint32_t d = 0; d < nd; ++d) f(u0 + d, s, d);
+    } else {
+      const uint64_t seg_end = (u0 / n_kt + 1) * n_kt;
+      const uint32_t nA = static_cast<uint32_t>(seg_end - u0 < nd ? seg_end - u0 : nd);
+      for (uint32_t s = 0; s < P.C; ++s)
+        for (uint32_t d = 0; d < nA; ++d) f(u0 + d, s, d);
+      for (uint32_t s = 0; s < P.C; ++s)
+        for (uint32_t d = nA; d < nd; ++d) f(u0 + d, s, d);
+    }
+  }
+}
+
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ float bf16_to_f32(uint16_t b) {
+  return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+// ---------------------------------------------------------------------------
+template <bool kDecode, uint32_t kFmt>
+__global__ void __launch_bounds__(kMaxThreads, 1)
+    fused_gemm_kernel(const __grid_constant__ GemmDev P, const __grid_constant__ CUtensorMap tmX) {
+  extern __shared__ __align__(2048) uint8_t smem[];
+  __shared__ uint32_t tmem_slot;
+  __shared__ uint32_t abort_flag;
+  __shared__ uint32_t reduce_flag;
+
+  const uint32_t warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t D = P.D, XS = P.x_stages;
+  const uint32_t G = gridDim.x;
+  const uint64_t u_begin = cta_begin(P.n_units, G, blockIdx.x);
+  const uint64_t u_end = cta_begin(P.n_units, G, blockIdx.x + 1);
+  const uint32_t n_kt = P.L.n_kt;
+
+  uint32_t* lut = reinterpret_cast<uint32_t*>(smem + P.off_lut);
+  uint8_t* wring = smem + P.off_w;
+  uint8_t* chunks = smem + P.off_chunk;
+  uint8_t* xring = smem + P.off_x;
+  Bars B = carve_bars(smem + P.off_bars, D, XS);
+  const uint32_t x_stage_bytes = P.T_pass * 32;
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (uint32_t i = 0; i < 2 * D; ++i) { mbar_init(&B.w_full[i], 1); mbar_init(&B.w_empty[i], 1); }
+    for (uint32_t i = 0; i < XS; ++i) { mbar_init(&B.x_full[i], 1); mbar_init(&B.x_empty[i], 1); }
+    for (uint32_t i = 0; i < 2; ++i) { mbar_init(&B.acc_full[i], 1); mbar_init(&B.acc_empty[i], 4); }
+    mbar_init(B.mma_done, 1);
+    for (uint32_t i = 0; i < 4 * D; ++i) mbar_init(&B.chunk[i], 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&tmem_slot, P.tmem_cols);
+    tmem_relinquish();
+  }
+  if (warp == 5 && lane == 0) prefetch_tmap(&tmX);
+  if (kDecode && P.L.single_symbol == kNoSymbol) build_lut(lut, P.L, warp, blockDim.x / 32, lane);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_slot;
+  volatile uint32_t* abort = &abort_flag;
+
+  if (warp >= kFixedWarps) {
+    // ======================= producer warps =======================
+    const uint32_t d = warp - kFixedWarps;
+    const uint32_t lt = lanemask_lt();
+    const LayerDev& L = P.L;
+    const bool single = L.single_symbol != kNoSymbol;
+    const uint32_t H = P.H;
+    const uint32_t slab_groups = 8;                 // 8 groups of 8 symbols per lane = one slab
+    const uint32_t n_slabs = P.H * P.C;
+    TileSeq seq{static_cast<uint32_t>(u_begin) + d, D, static_cast<uint32_t>(u_end), L.n_tiles};
+    ChunkPipe pipe;
+    pipe_init(pipe, chunks + d * kRingBytes, B.chunk + 4 * d);
+    uint32_t cb = 0;
+    uint32_t sc = 0;  // unit slabs produced
+    const uint32_t swz = ((lane >> 2) & 1u) << 4;
+
+    for (uint32_t r = 0; seq.has(r); ++r) {
+      const uint32_t t = seq.at(r);
+      const uint32_t n0 = (t / n_kt) * L.tile_n, k0 = (t % n_kt) * L.tile_k;
+      // ---- per-tile setup
+      uint32_t x = kStateLow, pos = 0, last = 0, nch = 0, bytes = 0;
+      bool zero_tile = false;
+      if (kDecode) {
+        uint64_t start;
+        if (!tile_extent(L, t, &start, &bytes)) {
+          zero_tile = true;
+          if (lane == 0) atomicOr(P.status, kStatusBadOffsets);
+        } else {
+          nch = (bytes + kChunkBytes - 1) / kChunkBytes;
+          last = cb + nch - 1;
+          pos = cb * kChunkBytes;
+          pipe_before_group(pipe, L, seq, pos, last, lane, abort, P.status);
+          x = *reinterpret_cast<const uint32_t*>(pipe.ring + ((pos + 4 * lane) & (kRingBytes - 1)));
+          pos += 4 * kLanes;
+        }
+      }
+      __half2 gscale[8];
+      if (kFmt == kFmtInt4F16Group) {
+        const uint32_t gk = k0 / P.group_k;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          uint32_t hh = q / 4, ii = q % 4;
+          float sv = 0.f;
+          if (hh < H) {
+            uint32_t row = n0 + lane + 32 * (4 * hh + ii);
+            sv = bf16_to_f32(__ldg(static_cast<const uint16_t*>(P.scales) +
+                                   static_cast<uint64_t>(row) * P.n_groups_k + gk));
+          }
+          gscale[q] = __float2half2_rn(sv);
+        }
+      }
+      const uint8_t* raw_tile =
+          (kFmt == kFmtBf16Split && kDecode) ? L.raw + static_cast<uint64_t>(t) * (L.tile_n * L.tile_k) + lane * 8
+                                             : nullptr;
+      uint64_t raw_next = 0;
+      if (kFmt == kFmtBf16Split && kDecode && !zero_tile)
+        raw_next = __ldg(reinterpret_cast<const unsigned long long*>(raw_tile));
+
+      for (uint32_t us = 0; us < n_slabs; ++us) {
+        const uint32_t h = us % H, s = us / H;
+        const uint32_t slot = sc & 1u;
+        if (sc >= 2) wait_live(&B.w_empty[2 * d + slot], ((sc >> 1) + 1) & 1u, abort, P.status);
+        uint8_t* slab = wring + (2 * d + slot) * kSlabBytes;
+        for (uint32_t gg = 0; gg < slab_groups; ++gg) {
+          const uint32_t g = us * slab_groups + gg;
+          const uint32_t i = gg & 3, c = gg >> 2;
+          uint32_t o[4];
+          if (kDecode) {
+            uint64_t raw8 = raw_next;
+            if (kFmt == kFmtBf16Split && !zero_tile && g + 1 < n_slabs * slab_groups)
+              raw_next = __ldg(reinterpret_cast<const unsigned long long*>(raw_tile + (g + 1) * 256));
+            uint32_t e[8];
+            if (zero_tile) {
+#pragma unroll
+              for (int k = 0; k < 8; ++k) e[k] = 0;
+            } else if (single) {
+#pragma unroll
+              for (int k = 0; k < 8; ++k) e[k] = L.single_symbol << 12;
+            } else {
+              pipe_before_group(pipe, L, seq, pos, last, lane, abort, P.status);
+#pragma unroll
+              for (int k = 0; k < 8; ++k) e[k] = decode_step(x, pos, lut, pipe.ring, lt);
+            }
+            if (kFmt == kFmtBf16Split) fmt_bf16_split(e, raw8, o);
+            else if (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
+            else if (kFmt == kFmtInt4F16Group) fmt_int4_f16_scaled(e, gscale[4 * h + i], o);
+            else fmt_fp8_f16(e, o);
+            if (zero_tile) o[0] = o[1] = o[2] = o[3] = 0;
+          } else {
+            // copy mode: read the original weights of this group
+            const uint64_t row = n0 + lane + 32 * (4 * h + i);
+            const uint64_t idx = row * L.K + k0 + 16 * s + 8 * c;
+            if (kFmt == kFmtBf16Split) {
+              uint4 v = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(P.w_plain) + idx));
+              o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+            } else {
+              uint32_t e[8];
+              if (kFmt == kFmtFp8F16) {
+                uint2 v = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(P.w_plain) + idx));
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  e[k] = ((v.x >> (8 * k)) & 0xFFu) << 12;
+                  e[k + 4] = ((v.y >> (8 * k)) & 0xFFu) << 12;
+                }
+                fmt_fp8_f16(e, o);
+              } else {
+                uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(P.w_plain) + idx / 2));
+#pragma unroll
+                for (int k = 0; k < 8; ++k) e[k] = (((v >> (4 * k)) & 0xFu) ^ 8u) << 12;
+                if (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
+                else fmt_int4_f16_scaled(e, gscale[4 * h + i], o);
+              }
+            }
+          }
+          const uint32_t rr = 32 * i + lane;
+          *reinterpret_cast<uint4*>(slab + rr * 32 + ((c << 4) ^ swz)) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&B.w_full[2 * d + slot]);
+        ++sc;
+      }
+      if (kDecode && !zero_tile) {
+        if (!single) {
+          const uint32_t used = pos - cb * kChunkBytes;
+          bool bad = (x != kStateLow) || used > bytes || bytes - used >= 16;
+          if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) atomicOr(P.status, kStatusCorrupt);
+        } else {
+          bool bad = (x != kStateLow) || bytes != 4 * kLanes;
+          if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) atomicOr(P.status, kStatusCorrupt);
+        }
+        cb += nch;
+      }
+    }
+    if (kDecode) pipe_drain(pipe, P.status);
+  } else if (warp == 4) {
+    // ======================= MMA issue (one thread) =======================
+    if (lane == 0) {
+      const uint64_t seg0 = u_begin / n_kt;
+      uint32_t fresh = 0;  // bit (buf * 2 + h): next MMA into that accumulator starts it
+      uint32_t xc = 0;
+      for_each_mma_step(P, u_begin, u_end, [&](uint64_t u, uint32_t s, uint32_t d) {
+        const uint64_t seg = u / n_kt;
+        const uint32_t lseg = static_cast<uint32_t>(seg - seg0);
+        const uint32_t buf = lseg % P.n_bufs;
+        const bool seg_first = (u == u_begin) || (u % n_kt == 0);
+        const bool seg_last = (u + 1 == u_end) || ((u + 1) % n_kt == 0);
+        if (s == 0 && seg_first) {
+          const uint32_t k = lseg / P.n_bufs;
+          if (k >= 1) wait_live(&B.acc_empty[buf], (k - 1) & 1u, abort, P.status);
+          tc_fence_after();
+          fresh |= 3u << (2 * buf);
+        }
+        const uint32_t xs = xc % XS;
+        wait_live(&B.x_full[xs], (xc / XS) & 1u, abort, P.status);
+        const uint32_t r = static_cast<uint32_t>((u - u_begin) / P.D);
+        for (uint32_t h = 0; h < P.H; ++h) {
+          const uint32_t idx = (r * P.C + s) * P.H + h;
+          const uint32_t slot = idx & 1u;
+          wait_live(&B.w_full[2 * d + slot], (idx >> 1) & 1u, abort, P.status);
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(wring + (2 * d + slot) * kSlabBytes);
+          const uint64_t adesc = sdesc_sw32(a_addr, 256);
+          const uint32_t acc_bit = 1u << (2 * buf + h);
+          const uint32_t accumulate = (fresh & acc_bit) ? 0u : 1u;
+          for (uint32_t j = 0; j < P.NT; ++j) {
+            const uint32_t b_addr = smem_u32(xring + xs * x_stage_bytes + j * P.T * 32);
+            const uint32_t col = ((buf * P.H + h) * P.NT + j) * P.T;
+            umma_f16(tmem_base + col, adesc, sdesc_sw32(b_addr, 256), P.idesc, accumulate);
+          }
+          fresh &= ~acc_bit;
+          umma_commit(&B.w_empty[2 * d + slot]);
+        }
+        umma_commit(&B.x_empty[xs]);
+        ++xc;
+        if (s == P.C - 1 && seg_last) umma_commit(&B.acc_full[buf]);
+      });
+      umma_commit(B.mma_done);
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // ======================= X loader (TMA, one thread) =======================
+    if (lane == 0) {
+      uint32_t xc = 0;
+      uint32_t last_issued[8];  // per stage: 1 + index of the last load issued into it
+#pragma unroll
+      for (int k = 0; k < 8; ++k) last_issued[k] = 0;
+      for_each_mma_step(P, u_begin, u_end, [&](uint64_t u, uint32_t s, uint32_t) {
+        const uint32_t xs = xc % XS;
+        if (xc >= XS) wait_live(&B.x_empty[xs], ((xc / XS) + 1) & 1u, abort, P.status);
+        const uint32_t p = static_cast<uint32_t>(u / P.L.n_tiles);
+        const uint32_t t = static_cast<uint32_t>(u % P.L.n_tiles);
+        const int32_t kx = static_cast<int32_t>((t % n_kt) * P.L.tile_k + 16 * s);
+        if (!*abort) {
+          mbar_arrive_expect_tx(&B.x_full[xs], P.T_pass * 32);
+          for (uint32_t j = 0; j < P.NT; ++j)
+            tma_load_2d(xring + xs * x_stage_bytes + j * P.T * 32, &tmX, kx,
+                        static_cast<int32_t>(p * P.T_pass + j * P.T), &B.x_full[xs]);
+          last_issued[xs] = xc + 1;
+        }
+        ++xc;
+      });
+      // drain: the last load issued into every stage must have landed
+      for (uint32_t k = 0; k < XS; ++k)
+        if (last_issued[k]) wait_drain(&B.x_full[k], ((last_issued[k] - 1) / XS) & 1u, P.status);
+    }
+    __syncwarp();
+  } else {
+    // ======================= epilogue (warps 0-3, 128 threads) =======================
+    const uint32_t e = threadIdx.x;  // TMEM lane = row within the 128-row half
+    const uint64_t seg_first = u_begin / n_kt, seg_last = (u_end - 1) / n_kt;
+    const uint32_t N = P.L.N;
+    for (uint64_t seg = seg_first; seg <= seg_last; ++seg) {
+      const uint32_t lseg = static_cast<uint32_t>(seg - seg_first);
+      const uint32_t buf = lseg % P.n_bufs;
+      wait_live(&B.acc_full[buf], (lseg / P.n_bufs) & 1u, abort, P.status);
+      tc_fence_after();
+      const uint32_t p = static_cast<uint32_t>(seg / P.n_rb);
+      const uint32_t rb = static_cast<uint32_t>(seg % P.n_rb);
+      const uint64_t s_lo = seg * n_kt, s_hi = s_lo + n_kt;
+      const bool complete = u_begin <= s_lo && u_end >= s_hi;
+      const uint32_t slot = (seg == seg_first) ? 0u : 1u;
+      float* part = P.partials + (static_cast<uint64_t>(blockIdx.x) * 2 + slot) * P.H * P.T_pass * 128;
+      for (uint32_t h = 0; h < P.H; ++h) {
+        const uint32_t n = rb * P.L.tile_n + h * 128 + e;
+        float scale = 1.0f;
+        if (complete) {
+          if (P.scale_kind == 1) scale = bf16_to_f32(__ldg(static_cast<const uint16_t*>(P.scales) + n));
+          else if (P.scale_kind == 2) scale = __ldg(static_cast<const float*>(P.scales) + n);
+        }
+        for (uint32_t j = 0; j < P.NT; ++j) {
+          const uint32_t col0 = ((buf * P.H + h) * P.NT + j) * P.T;
+          for (uint32_t cc = 0; cc < P.T; cc += 16) {
+            uint32_t v[16];
+            tmem_ld16(tmem_base + ((32 * warp) << 16) + col0 + cc, v);
+            tmem_ld_wait();
+            const uint32_t tok0 = j * P.T + cc;
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+              const uint32_t m = p * P.T_pass + tok0 + q;
+              const float a = __uint_as_float(v[q]);
+              if (complete) {
+                if (m < P.M) P.Y[static_cast<uint64_t>(m) * N + n] = a * scale;
+              } else {
+                part[(static_cast<uint64_t>(h) * P.T_pass + tok0 + q) * 128 + e] = a;
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&B.acc_empty[buf]);
+      if (!complete) {
+        // split-K: the last CTA to finish this segment reduces it in CTA order
+        __threadfence();
+        named_bar_sync(1, 128);
+        const uint32_t c_first = cta_of(P.n_units, G, s_lo);
+        const uint32_t c_last = cta_of(P.n_units, G, s_hi - 1);
+        if (e == 0) {
+          uint32_t old = atomicAdd(&P.counters[seg], 1u);
+          reduce_flag = (old == c_last - c_first) ? 1u : 0u;
+        }
+        named_bar_sync(1, 128);
+        if (reduce_flag) {
+          __threadfence();
+          for (uint32_t h = 0; h < P.H; ++h) {
+            const uint32_t n = rb * P.L.tile_n + h * 128 + e;
+            float scale = 1.0f;
+            if (P.scale_kind == 1) scale = bf16_to_f32(__ldg(static_cast<const uint16_t*>(P.scales) + n));
+            else if (P.scale_kind == 2) scale = __ldg(static_cast<const float*>(P.scales) + n);
+            for (uint32_t tok = 0; tok < P.T_pass; ++tok) {
+              const uint32_t m = p * P.T_pass + tok;
+              if (m >= P.M) break;
+              float acc = 0.f;
+              for (uint32_t c2 = c_first; c2 <= c_last; ++c2) {
+                const uint64_t c2_seg0 = cta_begin(P.n_units, G, c2) / n_kt;
+                const uint32_t sl = (c2_seg0 == seg) ? 0u : 1u;
+                const float* pp = P.partials + (static_cast<uint64_t>(c2) * 2 + sl) * P.H * P.T_pass * 128;
+                acc += __ldcg(pp + (static_cast<uint64_t>(h) * P.T_pass + tok) * 128 + e);
+              }
+              P.Y[static_cast<uint64_t>(m) * N + n] = acc * scale;
+            }
+          }
+          if (e == 0) P.counters[seg] = 0;
+        }
+        named_bar_sync(1, 128);
+      }
+    }
+  }
+
+  // ---- teardown: every MMA retired before TMEM is released
+  __syncthreads();
+  if (warp == 0) {
+    wait_drain(B.mma_done, 0, P.status);
+    tc_fence_after();
+    tmem_dealloc(tmem_base, P.tmem_cols);
+  }
+}
+
+__global__ void x_to_f16_kernel(const uint4* __restrict__ X, uint4* __restrict__ Xh, uint64_t n8) {
+  for (uint64_t i = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += static_cast<uint64_t>(gridDim.x) * blockDim.x) {
+    uint4 v = __ldg(X + i);
+    uint32_t in[4] = {v.x, v.y, v.z, v.w}, out[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float lo = __uint_as_float(in[k] << 16), hi = __uint_as_float(in[k] & 0xFFFF0000u);
+      __half2 h = __floats2half2_rn(lo, hi);
+      out[k] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    Xh[i] = make_uint4(out[0], out[1], out[2], out[3]);
+  }
+}
+
+// =============================== host side ===============================
+
+static uint32_t round_up(uint32_t a, uint32_t b) { return (a + b - 1) / b * b; }
+
+bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool decode, int num_sms,
+                    GemmPlan* plan) {
+  GemmPlan p;
+  std::memset(&p, 0, sizeof(p));
+  if (L.dtype == 1) p.fmt = kFmtBf16Split;
+  else if (L.dtype == 0) p.fmt = (scale_kind == 3) ? kFmtInt4F16Group : kFmtInt4Bf16;
+  else p.fmt = kFmtFp8F16;
+  p.ab_f16 = (p.fmt == kFmtInt4F16Group || p.fmt == kFmtFp8F16) ? 1 : 0;
+  p.M = M;
+  p.H = L.tile_n / 128;
+  p.C = L.tile_k / 16;
+  const uint32_t Mp = round_up(M < 1 ? 1 : M, 16);
+  const uint32_t max_cols = 512;
+  if (2 * p.H * Mp <= max_cols) {
+    p.n_bufs = 2;
+    p.T_pass = Mp;
+  } else if (p.H * Mp <= max_cols) {
+    p.n_bufs = 1;
+    p.T_pass = Mp;
+  } else {
+    p.n_bufs = 1;
+    p.T_pass = max_cols / p.H;
+  }
+  p.NT = (p.T_pass + 255) / 256;
+  p.T = round_up((p.T_pass + p.NT - 1) / p.NT, 16);
+  p.T_pass = p.T * p.NT;
+  p.n_pass = (M + p.T_pass - 1) / p.T_pass;
+  if (p.n_pass == 0) p.n_pass = 1;
+  uint32_t cols = p.n_bufs * p.H * p.T_pass;
+  p.tmem_cols = 32;
+  while (p.tmem_cols < cols) p.tmem_cols <<= 1;
+  if (p.tmem_cols > 512) return false;
+
+  p.n_units = static_cast<uint64_t>(p.n_pass) * L.n_tiles;
+  p.n_segments = p.n_pass * (L.N / L.tile_n);
+  uint64_t sms = num_sms > 0 ? static_cast<uint64_t>(num_sms) : 148;
+  // Tuning / testing knobs: cap the CTA count and the producer warps per CTA.
+  if (const char* v = std::getenv("ANS_GEMM_MAX_CTAS")) {
+    long cap = std::strtol(v, nullptr, 10);
+    if (cap > 0 && static_cast<uint64_t>(cap) < sms) sms = static_cast<uint64_t>(cap);
+  }
+  p.grid = static_cast<uint32_t>(p.n_units < sms ? p.n_units : sms);
+  uint64_t per_cta = (p.n_units + p.grid - 1) / p.grid;
+
+  // shared memory: [lut][w rings][chunk rings][x stages][barriers]
+  const uint32_t x_stage = p.T_pass * 32;
+  const uint32_t lut_bytes = decode ? kSlots * 4 : 0;
+  uint32_t D = kMaxProducers;
+  if (const char* v = std::getenv("ANS_GEMM_MAX_PRODUCERS")) {
+    long cap = std::strtol(v, nullptr, 10);
+    if (cap > 0 && static_cast<uint32_t>(cap) < D) D = static_cast<uint32_t>(cap);
+  }
+  if (D > L.n_kt) D = L.n_kt;
+  if (D > per_cta) D = static_cast<uint32_t>(per_cta);
+  uint32_t XS = x_stage <= 2048 ? 8 : (x_stage <= 8192 ? 4 : 3);
+  for (;;) {
+    uint32_t off = lut_bytes;
+    off = round_up(off, 2048);
+    uint32_t off_w = off;
+    off += D * 2 * kSlabBytes;
+    off = round_up(off, 2048);
+    uint32_t off_chunk = off;
+    off += decode ? D * kRingBytes : 0;
+    off = round_up(off, 1024);
+    uint32_t off_x = off;
+    off += XS * x_stage;
+    off = round_up(off, 8);
+    uint32_t off_bars = off;
+    off += num_bars(D, XS) * 8;
+    if (off <= kSmemLimit) {
+      p.off_lut = 0;
+      p.off_w = off_w;
+      p.off_chunk = off_chunk;
+      p.off_x = off_x;
+      p.off_bars = off_bars;
+      p.smem_bytes = off;
+      break;
+    }
+    if (XS > 2) { --XS; continue; }
+    if (D > 1) { --D; continue; }
+    return false;
+  }
+  p.D = D;
+  p.x_stages = XS;
+  p.ws_partials_bytes = static_cast<size_t>(p.grid) * 2 * p.H * p.T_pass * 128 * sizeof(float);
+  p.ws_counters_bytes = round_up(p.n_segments * 4, 256);
+  p.ws_x16_bytes = p.ab_f16 ? static_cast<size_t>(M) * L.K * 2 : 0;
+  p.ws_bytes = p.ws_counters_bytes + (p.ws_partials_bytes + 255) / 256 * 256 +
+               (p.ws_x16_bytes + 255) / 256 * 256;
+  *plan = p;
+  return true;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+template <bool kDecode, uint32_t kFmt>
+static cudaError_t launch_variant(const GemmPlan& plan, const GemmDev& P, const CUtensorMap& tm,
+                                  cudaStream_t stream) {
+  auto kern = fused_gemm_kernel<kDecode, kFmt>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(plan.smem_bytes));
+  if (e != cudaSuccess) return e;
+  kern<<<plan.grid, (kFixedWarps + plan.D) * 32, plan.smem_bytes, stream>>>(P, tm);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm(const GemmPlan& plan, const LayerDev& L, bool decode, const void* w_plain,
+                        const uint16_t* X, const void* scales, uint32_t scale_kind,
+                        uint32_t group_k, float* Y, void* ws, uint32_t* status,
+                        cudaStream_t stream) {
+  if (plan.M == 0) return cudaSuccess;
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  uint32_t* counters = reinterpret_cast<uint32_t*>(wsb);
+  float* partials = reinterpret_cast<float*>(wsb + plan.ws_counters_bytes);
+  uint16_t* x16 = reinterpret_cast<uint16_t*>(wsb + plan.ws_counters_bytes +
+                                              ((plan.ws_partials_bytes + 255) / 256) * 256);
+  const void* xsrc = X;
+  if (plan.ab_f16) {
+    uint64_t n8 = static_cast<uint64_t>(plan.M) * L.K / 8;
+    uint32_t blocks = static_cast<uint32_t>((n8 + 255) / 256);
+    if (blocks > 1184) blocks = 1184;
+    if (blocks == 0) blocks = 1;
+    x_to_f16_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<const uint4*>(X),
+                                                reinterpret_cast<uint4*>(x16), n8);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    xsrc = x16;
+  }
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return cudaErrorNotSupported;
+  CUtensorMap tm;
+  cuuint64_t gdim[2] = {L.K, plan.M};
+  cuuint64_t gstride[1] = {static_cast<cuuint64_t>(L.K) * 2};
+  cuuint32_t box[2] = {16, plan.T};
+  cuuint32_t estride[2] = {1, 1};
+  CUresult cr = enc(&tm, plan.ab_f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                    2, const_cast<void*>(xsrc), gdim, gstride, box, estride,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
+
+  GemmDev P;
+  std::memset(&P, 0, sizeof(P));
+  P.L = L;
+  P.w_plain = w_plain;
+  P.scales = scales;
+  P.Y = Y;
+  P.partials = partials;
+  P.counters = counters;
+  P.status = status;
+  P.scale_kind = scale_kind;
+  P.group_k = group_k;
+  P.n_groups_k = group_k ? L.K / group_k : 0;
+  P.M = plan.M;
+  P.T = plan.T;
+  P.NT = plan.NT;
+  P.T_pass = plan.T_pass;
+  P.n_pass = plan.n_pass;
+  P.H = plan.H;
+  P.C = plan.C;
+  P.D = plan.D;
+  P.n_bufs = plan.n_bufs;
+  P.x_stages = plan.x_stages;
+  P.tmem_cols = plan.tmem_cols;
+  P.n_rb = L.N / L.tile_n;
+  P.n_units = plan.n_units;
+  P.idesc = idesc_f16(plan.ab_f16 ? 0u : 1u, 128, plan.T);
+  P.off_lut = plan.off_lut;
+  P.off_w = plan.off_w;
+  P.off_chunk = plan.off_chunk;
+  P.off_x = plan.off_x;
+  P.off_bars = plan.off_bars;
+
+  switch (plan.fmt | (decode ? 0u : 8u)) {
+    case kFmtBf16Split: return launch_variant<true, kFmtBf16Split>(plan, P, tm, stream);
+    case kFmtInt4Bf16: return launch_variant<true, kFmtInt4Bf16>(plan, P, tm, stream);
+    case kFmtInt4F16Group: return launch_variant<true, kFmtInt4F16Group>(plan, P, tm, stream);
+    case kFmtFp8F16: return launch_variant<true, kFmtFp8F16>(plan, P, tm, stream);
+    case 8 | kFmtBf16Split: return launch_variant<false, kFmtBf16Split>(plan, P, tm, stream);
+    case 8 | kFmtInt4Bf16: return launch_variant<false, kFmtInt4Bf16>(plan, P, tm, stream);
+    case 8 | kFmtInt4F16Group: return launch_variant<false, kFmtInt4F16Group>(plan, P, tm, stream);
+    case 8 | kFmtFp8F16: return launch_variant<false, kFmtFp8F16>(plan, P, tm, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace ansdev

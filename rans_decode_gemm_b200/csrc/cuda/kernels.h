@@ -1,0 +1,84 @@
+// kernels.h -- plain structs and launch entry points shared between the C-ABI
+// layer (host C++) and the CUDA kernels.  No device code here.
+#pragma once
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace ansdev {
+
+constexpr uint32_t kNoSymbolHost = 0xFFFFFFFFu;
+
+// A compressed layer as the kernels see it (passed by value as a kernel
+// parameter; the codebook travels with it).
+struct LayerDev {
+  const uint8_t* stream;
+  const uint64_t* offsets;
+  const uint8_t* raw;
+  uint64_t stream_bytes;
+  uint32_t N, K, tile_n, tile_k;
+  uint32_t n_kt, n_tiles, dtype, alphabet;
+  uint32_t single_symbol;  // the symbol when the codebook has exactly one, else kNoSymbolHost
+  uint16_t freq[256];
+  uint16_t cdf[257];
+};
+
+// Output formats of the producer warps (what lands in the MMA operand slab).
+enum : uint32_t {
+  kFmtBf16Split = 0,   // bf16 weights: exponent symbol + raw sign/mantissa byte -> bf16
+  kFmtInt4Bf16 = 1,    // int4 code -> exact bf16 (row scale applied in the epilogue)
+  kFmtInt4F16Group = 2,// int4 code * group scale -> exact f16
+  kFmtFp8F16 = 3       // e4m3 code -> exact f16 (row scale applied in the epilogue)
+};
+
+// Static schedule of one fused GEMM launch, computed on the host.
+struct GemmPlan {
+  uint32_t fmt;        // kFmt*
+  uint32_t ab_f16;     // MMA operand type: 1 = f16, 0 = bf16
+  uint32_t M, T, NT, T_pass, n_pass;
+  uint32_t H, C;       // 128-row halves per tile, 16-column slabs per tile
+  uint32_t D;          // producer warps per CTA
+  uint32_t n_bufs;     // TMEM accumulator sets (1 or 2)
+  uint32_t x_stages;
+  uint32_t tmem_cols;
+  uint32_t grid;       // CTAs
+  uint64_t n_units;    // n_pass * n_tiles
+  uint32_t n_segments; // n_pass * (N / tile_n)
+  uint32_t smem_bytes;
+  uint32_t off_lut, off_w, off_chunk, off_x, off_bars;
+  size_t ws_partials_bytes, ws_counters_bytes, ws_x16_bytes, ws_bytes;
+};
+
+struct GemmDev {
+  LayerDev L;
+  const void* w_plain;   // copy mode: uncompressed weights
+  const void* scales;
+  float* Y;
+  float* partials;
+  uint32_t* counters;
+  uint32_t* status;
+  uint32_t scale_kind, group_k, n_groups_k;
+  uint32_t M, T, NT, T_pass, n_pass;
+  uint32_t H, C, D, n_bufs, x_stages, tmem_cols;
+  uint32_t n_rb;
+  uint64_t n_units;
+  uint32_t idesc;
+  uint32_t off_lut, off_w, off_chunk, off_x, off_bars;
+};
+
+// Fills a plan; returns false if the shape cannot be scheduled.
+bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool decode,
+                    int num_sms, GemmPlan* plan);
+
+cudaError_t launch_decode_tiles(const LayerDev& L, void* out, uint32_t* status,
+                                cudaStream_t stream, int num_sms);
+cudaError_t launch_histogram(const void* w, uint64_t n_bytes, uint32_t dtype, uint64_t* hist,
+                             cudaStream_t stream, int num_sms);
+// X: bf16 M x K.  ws must hold plan.ws_bytes (partials, counters, f16 X copy).
+cudaError_t launch_gemm(const GemmPlan& plan, const LayerDev& L, bool decode, const void* w_plain,
+                        const uint16_t* X, const void* scales, uint32_t scale_kind,
+                        uint32_t group_k, float* Y, void* ws, uint32_t* status,
+                        cudaStream_t stream);
+
+}  // namespace ansdev

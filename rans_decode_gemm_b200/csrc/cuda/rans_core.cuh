@@ -1,0 +1,270 @@
+// rans_core.cuh -- warp-parallel tile rANS decoding shared by the standalone
+// decode kernel and the fused decode + GEMM kernel.
+//
+// "Approaching Shannon Bound with Lossless LLM Weight Compression", s3.1
+// "整体执行模型": each GEMM-shaped tile is one self-contained substream set;
+// its bitstream is split into R = 32 substreams and every warp lane keeps its
+// own rANS state, so one warp decodes one tile.  Symbols are looked up in a
+// shared-memory slot table built from the layer's shared codebook.
+//
+// Per lane and step: slot = x & 4095; e = lut[slot] packs (f, symbol,
+// slot - cdf); x = f * (x >> 12) + (slot - cdf); if x < 2^16 the lane takes
+// the next 16-bit word of the tile's interleaved word stream (lanes in
+// increasing order, found with a ballot + prefix popcount).
+//
+// Compressed bytes reach shared memory through a per-warp ring of four
+// 512-byte slots filled by 1-D bulk copies (no multicast) that complete on
+// one mbarrier per slot; the ring runs up to three chunks ahead of the read
+// cursor, across tile boundaries.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <cstdint>
+
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace ansdev {
+
+constexpr uint32_t kLanes = 32;
+constexpr uint32_t kSlots = 4096;        // 2^12 probability slots
+constexpr uint32_t kStateLow = 1u << 16; // L
+constexpr uint32_t kChunkBytes = 512;
+constexpr uint32_t kRingBytes = 2048;
+constexpr uint32_t kNoSymbol = kNoSymbolHost;
+
+constexpr uint32_t kStatusCorrupt = 0x1u;
+constexpr uint32_t kStatusTimeout = 0x2u;
+constexpr uint32_t kStatusBadOffsets = 0x4u;
+
+enum : uint32_t { kDtInt4 = 0, kDtBf16Split = 1, kDtFp8 = 2 };
+
+
+// Abort-aware bounded wait.  Returns false if the wait ran out (then sets the
+// CTA's abort flag and the TIMEOUT status bit) or if the CTA already aborted.
+__device__ __forceinline__ bool wait_live(uint64_t* bar, uint32_t parity, volatile uint32_t* abort,
+                                          uint32_t* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort) return false;
+    if (clock64() - t0 > kWaitBudgetCycles) {
+      *abort = 1u;
+      atomicOr(status, kStatusTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
+// Bounded wait used when draining copies before exit; ignores the abort flag
+// (bulk copies always complete on their own).
+__device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, uint32_t* status) {
+  if (!mbar_wait(bar, parity)) atomicOr(status, kStatusTimeout);
+}
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// Slot table: entry = (f & 0xFFF) << 20 | symbol << 12 | (slot - cdf[symbol]).
+// A single-symbol codebook (f = 4096) is decoded by a separate path.
+__device__ __forceinline__ void build_lut(uint32_t* lut, const LayerDev& L, uint32_t warp,
+                                          uint32_t nwarps, uint32_t lane) {
+  for (uint32_t s = warp; s < L.alphabet; s += nwarps) {
+    uint32_t f = L.freq[s], c = L.cdf[s];
+    uint32_t hi = ((f & 0xFFFu) << 20) | (s << 12);
+    for (uint32_t k = lane; k < f; k += 32) lut[c + k] = hi | k;
+  }
+}
+
+// Byte extent of tile t, validated against the format's rules.
+__device__ __forceinline__ bool tile_extent(const LayerDev& L, uint32_t t, uint64_t* start,
+                                            uint32_t* bytes) {
+  uint64_t a = __ldg(reinterpret_cast<const unsigned long long*>(L.offsets) + t);
+  uint64_t b = __ldg(reinterpret_cast<const unsigned long long*>(L.offsets) + t + 1);
+  uint64_t max_bytes = 4ull * kLanes + 2ull * L.tile_n * L.tile_k + 16ull;
+  bool ok = (a % 16 == 0) && (b % 16 == 0) && b >= a + 4 * kLanes && b <= L.stream_bytes &&
+            (b - a) <= max_bytes;
+  *start = a;
+  *bytes = ok ? static_cast<uint32_t>(b - a) : 0u;
+  return ok;
+}
+
+// Tiles handled by one warp: units first, first + stride, ... while < end;
+// unit u is tile u % modulo (units run over several token passes).
+struct TileSeq {
+  uint32_t first, stride, end, modulo;
+  __device__ __forceinline__ bool has(uint32_t r) const {
+    return static_cast<uint64_t>(first) + static_cast<uint64_t>(r) * stride < end;
+  }
+  __device__ __forceinline__ uint32_t at(uint32_t r) const { return (first + r * stride) % modulo; }
+};
+
+// Per-warp compressed-byte pipeline.  All lanes hold the same values; lane 0
+// issues the copies.
+struct ChunkPipe {
+  uint8_t* ring;      // kRingBytes, kRingBytes-aligned shared memory
+  uint64_t* bars;     // 4 mbarriers (count 1)
+  uint32_t issued;    // chunks issued so far (global index over the warp's tiles)
+  uint32_t ready;     // chunks known to have landed
+  uint32_t it_r;      // next sequence position to issue from
+  uint32_t it_chunk, it_nch, it_bytes;
+  uint64_t it_start;
+};
+
+__device__ __forceinline__ void pipe_init(ChunkPipe& p, uint8_t* ring, uint64_t* bars) {
+  p.ring = ring;
+  p.bars = bars;
+  p.issued = p.ready = 0;
+  p.it_r = 0;
+  p.it_chunk = p.it_nch = p.it_bytes = 0;
+  p.it_start = 0;
+}
+
+// Issue chunks while issued < limit.  Tiles whose offsets are invalid
+// contribute no chunks (their consumer skips them).
+__device__ __forceinline__ void pipe_issue(ChunkPipe& p, const LayerDev& L, const TileSeq& seq,
+                                           uint32_t limit, uint32_t lane) {
+  while (p.issued < limit) {
+    if (p.it_chunk >= p.it_nch) {
+      if (!seq.has(p.it_r)) return;
+      uint32_t t = seq.at(p.it_r);
+      p.it_r++;
+      tile_extent(L, t, &p.it_start, &p.it_bytes);
+      p.it_chunk = 0;
+      p.it_nch = (p.it_bytes + kChunkBytes - 1) / kChunkBytes;
+      continue;
+    }
+    uint32_t off = p.it_chunk * kChunkBytes;
+    uint32_t n = min(kChunkBytes, p.it_bytes - off);
+    uint32_t slot = p.issued & 3u;
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&p.bars[slot], n);
+      bulk_g2s(p.ring + slot * kChunkBytes, L.stream + p.it_start + off, n, &p.bars[slot]);
+    }
+    p.it_chunk++;
+    p.issued++;
+  }
+}
+
+// Make chunks [.., need] resident (need is a global chunk index).
+__device__ __forceinline__ void pipe_wait(ChunkPipe& p, uint32_t need, volatile uint32_t* abort,
+                                          uint32_t* status) {
+  while (p.ready <= need && p.ready < p.issued) {
+    if (!wait_live(&p.bars[p.ready & 3u], (p.ready >> 2) & 1u, abort, status)) return;
+    p.ready++;
+  }
+}
+
+__device__ __forceinline__ void pipe_drain(ChunkPipe& p, uint32_t* status) {
+  while (p.ready < p.issued) {
+    wait_drain(&p.bars[p.ready & 3u], (p.ready >> 2) & 1u, status);
+    p.ready++;
+  }
+}
+
+// Keeps the ring full and the chunks that the next group can touch resident.
+// pos: read position in ring bytes (unwrapped); last_chunk: final chunk of
+// the current tile.
+__device__ __forceinline__ void pipe_before_group(ChunkPipe& p, const LayerDev& L,
+                                                  const TileSeq& seq, uint32_t pos,
+                                                  uint32_t last_chunk, uint32_t lane,
+                                                  volatile uint32_t* abort, uint32_t* status) {
+  uint32_t c = pos / kChunkBytes;
+  uint32_t limit = min(c, p.ready) + 4u;
+  if (p.issued < limit && !*abort) pipe_issue(p, L, seq, limit, lane);
+  uint32_t need = min(c + 1u, last_chunk);
+  if (p.ready <= need) pipe_wait(p, need, abort, status);
+}
+
+// One decode step for the calling lane.  x: state; pos: ring read position
+// (bytes, unwrapped; advanced by the words the warp consumed).
+__device__ __forceinline__ uint32_t decode_step(uint32_t& x, uint32_t& pos,
+                                                const uint32_t* __restrict__ lut,
+                                                const uint8_t* __restrict__ ring, uint32_t lt) {
+  uint32_t e = lut[x & (kSlots - 1)];
+  x = (e >> 20) * (x >> 12) + (e & 0xFFFu);
+  bool need = x < kStateLow;
+  uint32_t bal = __ballot_sync(0xFFFFFFFFu, need);
+  if (need) {
+    uint32_t off = (pos + 2u * __popc(bal & lt)) & (kRingBytes - 1);
+    x = (x << 16) | *reinterpret_cast<const uint16_t*>(ring + off);
+  }
+  pos += 2u * __popc(bal);
+  return e;
+}
+
+// ---- symbol -> MMA operand formatting ---------------------------------------
+// Inputs are slot-table entries (symbol at bits 12..19); outputs are packed
+// 16-bit pairs for 16-byte shared-memory stores.
+
+// bf16 split: exponent from the symbol, sign and mantissa from the raw byte.
+// raw8: 8 raw bytes for the group (byte k belongs to symbol k).
+__device__ __forceinline__ void fmt_bf16_split(const uint32_t (&e)[8], uint64_t raw8,
+                                               uint32_t (&out)[4]) {
+  uint32_t rlo = static_cast<uint32_t>(raw8), rhi = static_cast<uint32_t>(raw8 >> 32);
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    uint32_t a = e[2 * p] >> 5;        // exponent -> bits 7..14
+    uint32_t b = e[2 * p + 1] << 11;   // exponent -> bits 23..30
+    uint32_t ab = (a & 0x0000FFFFu) | (b & 0xFFFF0000u);
+    uint32_t r = (p < 2) ? rlo : rhi;
+    uint32_t sel = (p & 1) ? 0x3322u : 0x1100u;   // [r0,r0,r1,r1] of the pair
+    uint32_t rr = __byte_perm(r, 0u, sel);
+    out[p] = (ab & 0x7F807F80u) | (rr & 0x807F807Fu);
+  }
+}
+
+// int4 codes as exact bf16: bf16(128 + s) has bits 0x4300 | s; subtract 136.
+__device__ __forceinline__ void fmt_int4_bf16(const uint32_t (&e)[8], uint32_t (&out)[4]) {
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    uint32_t a = e[2 * p] >> 12, b = e[2 * p + 1] << 4;
+    uint32_t v = ((a & 0x0000FFFFu) | (b & 0xFFFF0000u)) & 0x00FF00FFu;
+    v |= 0x43004300u;
+    __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&v);
+    const __nv_bfloat162 bias = __floats2bfloat162_rn(136.0f, 136.0f);
+    h = __hsub2(h, bias);
+    out[p] = *reinterpret_cast<uint32_t*>(&h);
+  }
+}
+
+// int4 codes times a per-row scale, exact in f16: f16(1024 + s) has bits
+// 0x6400 | s; subtract 1032, multiply by the scale (|q * s| <= 11 bits).
+__device__ __forceinline__ void fmt_int4_f16_scaled(const uint32_t (&e)[8], __half2 scale,
+                                                    uint32_t (&out)[4]) {
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    uint32_t a = e[2 * p] >> 12, b = e[2 * p + 1] << 4;
+    uint32_t v = ((a & 0x0000FFFFu) | (b & 0xFFFF0000u)) & 0x00FF00FFu;
+    v |= 0x64006400u;
+    __half2 h = *reinterpret_cast<__half2*>(&v);
+    h = __hmul2(__hsub2(h, __floats2half2_rn(1032.0f, 1032.0f)), scale);
+    out[p] = *reinterpret_cast<uint32_t*>(&h);
+  }
+}
+
+// e4m3 codes to exact f16 pairs with the hardware converter.
+__device__ __forceinline__ uint32_t cvt_e4m3x2_f16x2(uint32_t two_codes) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 t;\n\t"
+      "cvt.u16.u32 t, %1;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, t;\n\t}"
+      : "=r"(r)
+      : "r"(two_codes));
+  return r;
+}
+__device__ __forceinline__ void fmt_fp8_f16(const uint32_t (&e)[8], uint32_t (&out)[4]) {
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    // low byte: code of symbol 2p, high byte: code of symbol 2p+1
+    uint32_t v = __byte_perm(e[2 * p] >> 12, e[2 * p + 1] >> 4, 0x0050u);
+    out[p] = cvt_e4m3x2_f16x2(v);
+  }
+}
+
+}  // namespace ansdev

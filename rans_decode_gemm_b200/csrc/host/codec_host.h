@@ -1,0 +1,20 @@
+// codec_host.h -- internal interface of the host-side codec (no CUDA).
+#pragma once
+#include <cstdint>
+
+namespace anshost {
+
+enum : uint32_t { kInt4 = 0, kBf16Split = 1, kFp8 = 2 };
+
+bool layout_valid(uint32_t N, uint32_t K, uint32_t tile_n, uint32_t tile_k);
+void histogram(uint32_t dtype, const void* w, uint64_t n_weights, uint64_t* hist);
+double entropy_bits(const uint64_t* hist, uint32_t alphabet);
+// 0 ok, 1 bad argument, 3 too many present symbols.
+int normalize(const uint64_t* hist, uint32_t alphabet, uint32_t prob_bits, uint32_t* freq);
+uint64_t encode_bound(uint32_t N, uint32_t K, uint32_t tile_n, uint32_t tile_k);
+// 0 ok, 3 symbol with zero frequency, 4 capacity too small (size still reported).
+int encode(uint32_t dtype, const void* w, uint32_t N, uint32_t K, uint32_t tile_n,
+           uint32_t tile_k, const uint32_t* freq, uint8_t* stream, uint64_t cap,
+           uint64_t* stream_bytes, uint64_t* offsets, uint8_t* raw);
+
+}  // namespace anshost

@@ -1,0 +1,129 @@
+"""CPU tests of the C-ABI library: it loads, exports every entry point that
+include/ans.h declares, and its host codec (histogram, entropy, codebook,
+tile encoder) agrees with the CPU oracle byte for byte."""
+import os
+import re
+
+import numpy as np
+import pytest
+
+from rans_decode_gemm_b200 import ans
+from rans_decode_gemm_b200 import workloads as WL
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"^\s*(?:const\s+)?[\w\s\*]+?\b(ans_\w+)\s*\(", text, re.M)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol(ans_lib):
+    names = declared_functions()
+    assert len(names) >= 14
+    lib = ans_lib.load()
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+    assert sorted(ans.EXPORTS) == names
+
+
+def test_status_strings_and_layout_checks(ans_lib):
+    assert ans.ans_status_string(0) == "ok"
+    assert ans.ans_layout_check(ans.make_layout(0, 512, 512, 128, 32)) == 0
+    assert ans.ans_layout_check(ans.make_layout(0, 500, 512, 128, 32)) == 2    # N % tile_n
+    assert ans.ans_layout_check(ans.make_layout(0, 512, 520, 128, 40)) == 2    # tile_k % 16
+    assert ans.ans_layout_check(ans.make_layout(0, 512, 512, 64, 32)) == 2     # tile_n
+    assert ans.ans_layout_check(ans.make_layout(7, 512, 512, 128, 32)) == 1    # dtype
+    assert ans.ans_layout_check(ans.make_layout(1, 0, 512, 128, 32)) == 2      # empty
+    assert ans.ans_num_tiles(ans.make_layout(2, 53248, 16384, 128, 128)) == 53248
+
+
+CASES = [("tiny_int4", 512, 512), ("bf16_4096", 512, 512), ("llama8b_mlp", 256, 1024),
+         ("int4_70b", 512, 512), ("fp8_405b", 256, 1024)]
+
+
+@pytest.mark.parametrize("name,N,K", CASES)
+def test_host_codec_matches_oracle(oracle, ans_lib, name, N, K):
+    cfg = WL.CONFIGS[name]
+    d = WL.make_weights(cfg, 0, N=N, K=K)
+    lay = ans.make_layout(cfg.dtype, N, K, cfg.tile_n, cfg.tile_k)
+    hist = ans.ans_histogram_host(d["w"], lay)
+    assert np.array_equal(hist, oracle.histogram(cfg.dtype, d["w"], N * K))
+    assert abs(ans.ans_entropy(hist) - oracle.entropy(hist)) < 1e-12
+    cb = ans.ans_build_codebook(hist, ans.ALPHABET[cfg.dtype], 12)
+    st, f_or = oracle.normalize(hist, 12)
+    assert st == 0 and np.array_equal(cb.freq_array(), f_or)
+    cdf = np.concatenate([[0], np.cumsum(f_or)])
+    assert np.array_equal(np.ctypeslib.as_array(cb.cdf)[:ans.ALPHABET[cfg.dtype] + 1], cdf)
+    stream, offsets, raw = ans.ans_encode_tiles(d["w"], lay, cb)
+    st, s_or, off_or, raw_or = oracle.encode(cfg.dtype, d["w"], N, K, cfg.tile_n, cfg.tile_k, f_or)
+    assert st == 0
+    assert np.array_equal(offsets, off_or)
+    assert np.array_equal(stream, s_or)
+    if raw is not None:
+        assert np.array_equal(raw, raw_or)
+    # and the oracle decodes the library's stream back to the weights
+    st, out = oracle.decode(cfg.dtype, stream, offsets, raw, N, K, cfg.tile_n, cfg.tile_k, f_or)
+    assert st == 0 and np.array_equal(out, d["w"])
+
+
+def test_codebook_matches_oracle_on_fuzzed_histograms(oracle, ans_lib):
+    rng = np.random.default_rng(21)
+    for trial in range(200):
+        A = 16 if trial % 2 else 256
+        k = int(rng.integers(1, A + 1))
+        h = np.zeros(A, np.uint64)
+        idx = rng.choice(A, size=k, replace=False)
+        h[idx] = rng.integers(1, 10 ** int(rng.integers(1, 9)), size=k).astype(np.uint64)
+        pb = int(rng.choice([8, 10, 12]))
+        st, f = oracle.normalize(h, pb)
+        if st != 0:
+            with pytest.raises(ans.AnsError):
+                ans.ans_build_codebook(h, A, pb)
+            continue
+        cb = ans.ans_build_codebook(h, A, pb)
+        assert np.array_equal(cb.freq_array(), f), trial
+
+
+def test_host_error_paths(ans_lib):
+    lay = ans.make_layout(ans.FP8_E4M3, 128, 32, 128, 32)
+    w = np.zeros(128 * 32, np.uint8)
+    w[3] = 9
+    h = np.zeros(256, np.uint64)
+    h[0] = 1
+    cb = ans.ans_build_codebook(h, 256)       # only symbol 0 present
+    with pytest.raises(ans.AnsError) as e:
+        ans.ans_encode_tiles(w, lay, cb)
+    assert e.value.status == 3
+    with pytest.raises(ans.AnsError) as e:
+        ans.ans_build_codebook(np.zeros(16, np.uint64), 16)
+    assert e.value.status == 1
+    with pytest.raises(ans.AnsError) as e:
+        ans.ans_build_codebook(np.ones(16, np.uint64), 16, prob_bits=3)
+    assert e.value.status == 3
+    bad = ans.ans_build_codebook(np.ones(256, np.uint64), 256)
+    bad.freq[0] += 1                          # freq no longer sums to 4096
+    with pytest.raises(ans.AnsError) as e:
+        ans.ans_encode_tiles(np.zeros(128 * 32, np.uint8), lay, bad)
+    assert e.value.status == 3
+    with pytest.raises(ans.AnsError) as e:
+        ans.ans_encode_tiles(w, ans.make_layout(ans.FP8_E4M3, 100, 32, 128, 32), cb)
+    assert e.value.status == 2
+
+
+def test_single_symbol_layer(oracle, ans_lib):
+    # a constant layer codes to 128 bytes per tile (states only) and decodes
+    N, K = 256, 64
+    w = np.full(N * K, 0x3C, np.uint8)
+    lay = ans.make_layout(ans.FP8_E4M3, N, K, 128, 64)
+    cb = ans.ans_build_codebook(ans.ans_histogram_host(w, lay), 256)
+    assert cb.freq[0x3C] == 4096
+    stream, offsets, _ = ans.ans_encode_tiles(w, lay, cb)
+    assert list(offsets) == [0, 128, 256]
+    assert (np.frombuffer(stream.tobytes(), np.uint32) == 65536).all()
+    st, out = oracle.decode(ans.FP8_E4M3, stream, offsets, None, N, K, 128, 64, cb.freq_array())
+    assert st == 0 and np.array_equal(out, w)

@@ -1,0 +1,126 @@
+"""GPU parity of the fused decode + GEMM (ans_gemm) through the C ABI:
+bit-exact against the same kernel fed the uncompressed weights
+(ans_gemm_uncompressed), and within a relative Frobenius error of 1e-3 of the
+oracle's fp64 GEMM (the bar the method's statement sets; fp32 accumulation
+over K <= 16384 lands near 1e-6)."""
+import numpy as np
+import pytest
+import torch
+
+from rans_decode_gemm_b200 import ans
+from rans_decode_gemm_b200 import workloads as WL
+
+from _gpu_util import make_case, rel_fro, run_gemm, status_tensor, x_dev
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-3
+
+# (config, N, K): small shapes spanning several tiles, split-K over CTAs and
+# rounds that cross W row blocks
+SMALL = [("tiny_int4", 512, 512), ("bf16_4096", 512, 1024), ("bf16_4096", 1024, 4096),
+         ("llama8b_mlp", 384, 2048), ("int4_70b", 512, 1024), ("fp8_405b", 256, 2048)]
+MS = [1, 5, 16, 17, 64, 128, 200, 300, 600]
+
+
+@pytest.fixture(scope="module")
+def cases():
+    return {}
+
+
+def _case(cases, name, N, K):
+    key = (name, N, K)
+    if key not in cases:
+        cases[key] = make_case(name, N, K)
+    return cases[key]
+
+
+@pytest.mark.parametrize("name,N,K", SMALL)
+@pytest.mark.parametrize("M", MS)
+def test_gemm_parity_small(cuda, oracle, cases, name, N, K, M):
+    cfg, d, lay, layer = _case(cases, name, N, K)
+    X = WL.make_x(cfg, M, K)
+    Y, st, _ = run_gemm(cfg, d, lay, layer, X, compressed=True)
+    Yu, stu, _ = run_gemm(cfg, d, lay, layer, X, compressed=False)
+    assert st == 0 and stu == 0
+    assert torch.equal(Y, Yu), "ans_gemm must be bit-identical to ans_gemm_uncompressed"
+    Yref = oracle.gemm(cfg.dtype, X, M, K, d["w"], N, cfg.scale_kind, d["scales"], cfg.group_k)
+    err = rel_fro(Y.cpu().numpy(), Yref)
+    assert err <= TOL, err
+
+
+@pytest.mark.parametrize("M", [1, 16, 128])
+def test_gemm_full_size_bf16_4096(cuda, oracle, cases, M):
+    # the benchmarked workload, at full size, in the launch configuration the
+    # benchmark times; the fp64 check runs on 256 sampled W rows
+    cfg, d, lay, layer = _case(cases, "bf16_4096", None, None)
+    X = WL.make_x(cfg, M)
+    Y, st, _ = run_gemm(cfg, d, lay, layer, X, compressed=True)
+    Yu, stu, _ = run_gemm(cfg, d, lay, layer, X, compressed=False)
+    assert st == 0 and stu == 0 and torch.equal(Y, Yu)
+    rows = np.random.default_rng(M).choice(lay.N, size=256, replace=False).astype(np.uint32)
+    Yref = oracle.gemm(cfg.dtype, X, M, lay.K, d["w"], lay.N, rows=rows)
+    assert rel_fro(Y.cpu().numpy()[:, rows], Yref) <= TOL
+
+
+def test_workspace_reuse_and_determinism(cuda, cases):
+    cfg, d, lay, layer = _case(cases, "bf16_4096", 1024, 4096)
+    X = WL.make_x(cfg, 16, 4096)
+    Y1, st1, ws = run_gemm(cfg, d, lay, layer, X)
+    Y2, st2, _ = run_gemm(cfg, d, lay, layer, X, ws=ws)
+    Y3, st3, _ = run_gemm(cfg, d, lay, layer, X, ws=ws)
+    assert st1 == st2 == st3 == 0
+    assert torch.equal(Y1, Y2) and torch.equal(Y1, Y3)
+    # split-K counters are back at zero
+    nseg = (lay.N // lay.tile_n)
+    assert int(ws[:4 * nseg].view(torch.int32).abs().sum().item()) == 0
+
+
+def test_gemm_argument_errors(cuda, cases):
+    cfg, d, lay, layer = _case(cases, "bf16_4096", 512, 1024)
+    X = x_dev(WL.make_x(cfg, 4, 1024))
+    Y = torch.zeros(4, 512, dtype=torch.float32, device="cuda")
+    st = status_tensor()
+    need = ans.ans_gemm_workspace(lay, 4, 0)
+    small = torch.zeros(max(1, need // 2), dtype=torch.uint8, device="cuda")
+    with pytest.raises(ans.AnsError) as e:
+        ans.ans_gemm(X, 4, layer.tiles, 0, None, 0, Y, small, small.numel(), st)
+    assert e.value.status == 4
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    Xflat = torch.zeros(4 * 1024 + 1, dtype=torch.int16, device="cuda")
+    with pytest.raises(ans.AnsError) as e:   # misaligned X
+        ans.ans_gemm(Xflat[1:], 4, layer.tiles, 0, None, 0, Y, ws, ws.numel(), st)
+    assert e.value.status == 1
+    # M == 0 is a no-op
+    ans.ans_gemm(X, 0, layer.tiles, 0, None, 0, Y, ws, ws.numel(), st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+
+
+def test_gemm_corrupt_stream_flags_status(cuda, cases):
+    cfg, d, lay, layer = _case(cases, "bf16_4096", 512, 1024)
+    bad = layer.h_stream.copy()
+    bad[200] ^= 0x10
+    bad[5000] ^= 0x01
+    broken = ans.CompressedLayer(lay, layer.codebook, bad, layer.h_offsets, layer.h_raw)
+    X = WL.make_x(cfg, 16, 1024)
+    Y, st, _ = run_gemm(cfg, d, lay, broken, X)
+    assert st & ans.STATUS_CORRUPT
+    assert not st & ans.STATUS_TIMEOUT
+
+
+@pytest.mark.parametrize("ctas,producers", [(8, 16), (5, 3), (3, 7)])
+@pytest.mark.parametrize("name,N,K,M", [("bf16_4096", 1024, 2048, 16), ("int4_70b", 512, 2048, 40),
+                                        ("fp8_405b", 512, 1024, 300), ("tiny_int4", 512, 512, 130)])
+def test_gemm_multi_round_schedules(cuda, oracle, cases, monkeypatch, ctas, producers, name, N, K, M):
+    # few CTAs and few producer warps: many rounds per CTA, rounds that cross
+    # W row blocks, slab and X rings wrapping many times, both accumulator sets
+    monkeypatch.setenv("ANS_GEMM_MAX_CTAS", str(ctas))
+    monkeypatch.setenv("ANS_GEMM_MAX_PRODUCERS", str(producers))
+    cfg, d, lay, layer = _case(cases, name, N, K)
+    X = WL.make_x(cfg, M, K)
+    Y, st, _ = run_gemm(cfg, d, lay, layer, X, compressed=True)
+    Yu, stu, _ = run_gemm(cfg, d, lay, layer, X, compressed=False)
+    assert st == 0 and stu == 0 and torch.equal(Y, Yu)
+    Yref = oracle.gemm(cfg.dtype, X, M, K, d["w"], N, cfg.scale_kind, d["scales"], cfg.group_k)
+    assert rel_fro(Y.cpu().numpy(), Yref) <= TOL
