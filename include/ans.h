@@ -199,7 +199,8 @@ ans_status ans_gemm_workspace(const ans_layout* layout, uint32_t M, ans_scale_ki
  * bit-identical to ans_gemm_uncompressed on the same weights.  GROUP_BF16 runs
  * the MMA in f16 (X and q*s are exact in f16 when |X| < 65504 and the scales
  * lie in [2^-14, 2^12]); all other kinds run it in bf16.
- * M == 0 is a no-op.  d_ws: ans_gemm_workspace bytes. */
+ * M == 0 is a no-op.  d_ws: ans_gemm_workspace bytes, 256-byte aligned; d_X,
+ * d_Y and d_scales 16-byte aligned (ANS_ERR_ARG otherwise). */
 ans_status ans_gemm(const uint16_t* d_X, uint32_t M, const ans_tiles* W,
                     ans_scale_kind scale_kind, const void* d_scales, uint32_t group_k,
                     float* d_Y, void* d_ws, size_t ws_bytes, uint32_t* d_status,

@@ -127,7 +127,10 @@ ans_status run_gemm(const uint16_t* d_X, uint32_t M, const ansdev::LayerDev& L, 
                     ans_stream_t stream) {
   if (M == 0) return ANS_OK;
   if (!d_X || !d_Y || !d_status || !d_ws) return ANS_ERR_ARG;
-  if (reinterpret_cast<uintptr_t>(d_X) % 16 != 0) return ANS_ERR_ARG;
+  if (reinterpret_cast<uintptr_t>(d_X) % 16 != 0 || reinterpret_cast<uintptr_t>(d_Y) % 16 != 0 ||
+      reinterpret_cast<uintptr_t>(d_ws) % 256 != 0 ||
+      (d_scales && reinterpret_cast<uintptr_t>(d_scales) % 16 != 0))
+    return ANS_ERR_ARG;
   int sms = 0;
   ans_status st = device_info(&sms);
   if (st != ANS_OK) return st;
@@ -325,5 +328,8 @@ ans_status ans_gemm_uncompressed(const uint16_t* d_X, uint32_t M, const void* d_
   return run_gemm(d_X, M, L, false, d_W, scale_kind, d_scales, group_k, d_Y, d_ws, ws_bytes,
                   d_status, stream);
 }
+
+// Internal profiling hook (not part of the public ABI in include/ans.h).
+void ansdev_set_trace(void* d_buf, size_t bytes) { ansdev::set_trace_buffer(d_buf, bytes); }
 
 }  // extern "C"

@@ -14,98 +14,106 @@
 
 namespace ansdev {
 
-constexpr uint32_t kDecWarps = 16;
+constexpr uint32_t kDecMaxWarps = 16;
 constexpr uint32_t kDecLutBytes = kSlots * 4;
-constexpr uint32_t kDecSmem = kDecLutBytes + kDecWarps * kRingBytes + kDecWarps * 4 * 8;
+// [lut 16 KB][align slack 2 KB][rings W x 2 KB][barriers W x 4 x 8 B]
+constexpr uint32_t kDecSmem = kDecLutBytes + kRingBytes + kDecMaxWarps * kRingBytes + kDecMaxWarps * 4 * 8;
 
-__global__ void __launch_bounds__(kDecWarps * 32, 2)
+// 8 output elements of one lane (row, 8 consecutive columns) in the original
+// storage format.
+__device__ __forceinline__ void store_group(uint32_t dtype, void* out, uint64_t idx,
+                                            const uint32_t (&e)[8], uint64_t raw8) {
+  if (dtype == kDtBf16Split) {
+    uint32_t o[4];
+    fmt_bf16_split(e, raw8, o);
+    *reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + idx) = make_uint4(o[0], o[1], o[2], o[3]);
+  } else if (dtype == kDtInt4) {
+    uint32_t w = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) w |= (((e[k] >> 12) ^ 8u) & 0xFu) << (4 * k);
+    *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(out) + idx / 2) = w;
+  } else {
+    uint32_t lo = __byte_perm(__byte_perm(e[0] >> 12, e[1] >> 4, 0x0050u),
+                              __byte_perm(e[2] >> 12, e[3] >> 4, 0x0050u), 0x5410u);
+    uint32_t hi = __byte_perm(__byte_perm(e[4] >> 12, e[5] >> 4, 0x0050u),
+                              __byte_perm(e[6] >> 12, e[7] >> 4, 0x0050u), 0x5410u);
+    *reinterpret_cast<uint2*>(static_cast<uint8_t*>(out) + idx) = make_uint2(lo, hi);
+  }
+}
+
+__global__ void __launch_bounds__(kDecMaxWarps * 32, 2)
     decode_tiles_kernel(const __grid_constant__ LayerDev L, void* __restrict__ out,
                         uint32_t* __restrict__ status) {
   extern __shared__ __align__(2048) uint8_t smem[];
   __shared__ uint32_t abort_flag;
+  const uint32_t nwarps = blockDim.x / 32;
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem);
-  uint8_t* rings = smem + kDecLutBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kDecLutBytes + kDecWarps * kRingBytes);
+  // rings on a kRingBytes-aligned shared address
+  const uint32_t ring_base_s = (smem_u32(smem + kDecLutBytes) + kRingBytes - 1) & ~(kRingBytes - 1);
+  uint8_t* rings = smem + (ring_base_s - smem_u32(smem));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kDecLutBytes + kRingBytes + kDecMaxWarps * kRingBytes);
   const uint32_t warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const bool single = L.single_symbol != kNoSymbol;
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
-    for (uint32_t i = 0; i < kDecWarps * 4; ++i) mbar_init(&bars[i], 1);
+    for (uint32_t i = 0; i < nwarps * 4; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
   }
-  if (!single) build_lut(lut, L, warp, kDecWarps, lane);
+  if (!single) build_lut(lut, L, warp, nwarps, lane);
   __syncthreads();
 
   volatile uint32_t* abort = &abort_flag;
   const uint32_t lt = lanemask_lt();
-  TileSeq seq{blockIdx.x * kDecWarps + warp, gridDim.x * kDecWarps, L.n_tiles, L.n_tiles};
+  const uint32_t lut_s = smem_u32(lut);
+  TileSeq seq{blockIdx.x * nwarps + warp, gridDim.x * nwarps, L.n_tiles, L.n_tiles};
   ChunkPipe pipe;
   pipe_init(pipe, rings + warp * kRingBytes, bars + warp * 4);
   const uint32_t H = L.tile_n / 128;
   const uint32_t groups = L.tile_n * L.tile_k / 256;
   const uint32_t S = L.tile_n * L.tile_k;
-  uint32_t cb = 0;  // first chunk of the current tile
+  const bool bf16 = L.dtype == kDtBf16Split;
+  TileCursor tc;
+  tc.cb = 0;
 
   for (uint32_t r = 0; seq.has(r); ++r) {
     const uint32_t t = seq.at(r);
-    uint64_t start;
-    uint32_t bytes;
-    if (!tile_extent(L, t, &start, &bytes)) {
+    if (!tile_begin(pipe, L, seq, t, tc, lane, abort, status)) {
       if (lane == 0) atomicOr(status, kStatusBadOffsets);
       continue;
     }
-    const uint32_t nch = (bytes + kChunkBytes - 1) / kChunkBytes;
-    const uint32_t last = cb + nch - 1;
-    uint32_t pos = cb * kChunkBytes;
-    const uint8_t* ring = pipe.ring;
-    pipe_before_group(pipe, L, seq, pos, last, lane, abort, status);
-    uint32_t x = *reinterpret_cast<const uint32_t*>(ring + ((pos + 4 * lane) & (kRingBytes - 1)));
-    pos += 4 * kLanes;
     const uint32_t n0 = (t / L.n_kt) * L.tile_n, k0 = (t % L.n_kt) * L.tile_k;
-    const uint8_t* raw_tile = L.raw + static_cast<uint64_t>(t) * S + lane * 8;
-    uint64_t raw_next = 0;
-    if (L.dtype == kDtBf16Split) raw_next = __ldg(reinterpret_cast<const unsigned long long*>(raw_tile));
-
+    const uint64_t base = static_cast<uint64_t>(n0 + lane) * L.K + k0;
+    const unsigned long long* raw_tile =
+        reinterpret_cast<const unsigned long long*>(L.raw + static_cast<uint64_t>(t) * S) + lane;
+    // raw bytes of groups g, g+1, g+2 in flight
+    uint64_t r0 = 0, r1 = 0, r2 = 0;
+    if (bf16) {
+      r0 = __ldg(raw_tile);
+      if (groups > 1) r1 = __ldg(raw_tile + 32);
+      if (groups > 2) r2 = __ldg(raw_tile + 64);
+    }
     for (uint32_t g = 0; g < groups; ++g) {
-      uint64_t raw8 = raw_next;
-      if (L.dtype == kDtBf16Split && g + 1 < groups)
-        raw_next = __ldg(reinterpret_cast<const unsigned long long*>(raw_tile + (g + 1) * 256));
+      const uint64_t raw8 = r0;
+      if (bf16) {
+        r0 = r1;
+        r1 = r2;
+        if (g + 3 < groups) r2 = __ldg(raw_tile + 32 * (g + 3));
+      }
       uint32_t e[8];
       if (single) {
 #pragma unroll
         for (int k = 0; k < 8; ++k) e[k] = L.single_symbol << 12;
       } else {
-        pipe_before_group(pipe, L, seq, pos, last, lane, abort, status);
+        tile_group(pipe, L, seq, tc, lane, abort, status);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) e[k] = decode_step(x, pos, lut, ring, lt);
+        for (int k = 0; k < 8; ++k) e[k] = decode_step(tc.x, tc.pos, lut_s, pipe.ring_s, lt);
       }
       const uint32_t i = g & 3, c = (g >> 2) & 1, h = (g >> 3) % H, s = g / (8 * H);
-      const uint64_t row = n0 + lane + 32 * (4 * h + i);
-      const uint64_t col = k0 + 16 * s + 8 * c;
-      const uint64_t idx = row * L.K + col;
-      if (L.dtype == kDtBf16Split) {
-        uint32_t o[4];
-        fmt_bf16_split(e, raw8, o);
-        *reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + idx) = make_uint4(o[0], o[1], o[2], o[3]);
-      } else if (L.dtype == kDtInt4) {
-        uint32_t w = 0;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) w |= (((e[k] >> 12) ^ 8u) & 0xFu) << (4 * k);
-        *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(out) + idx / 2) = w;
-      } else {
-        uint32_t lo = __byte_perm(__byte_perm(e[0] >> 12, e[1] >> 4, 0x0050u),
-                                  __byte_perm(e[2] >> 12, e[3] >> 4, 0x0050u), 0x5410u);
-        uint32_t hi = __byte_perm(__byte_perm(e[4] >> 12, e[5] >> 4, 0x0050u),
-                                  __byte_perm(e[6] >> 12, e[7] >> 4, 0x0050u), 0x5410u);
-        *reinterpret_cast<uint2*>(static_cast<uint8_t*>(out) + idx) = make_uint2(lo, hi);
-      }
+      const uint64_t idx = base + static_cast<uint64_t>(32 * (4 * h + i)) * L.K + 16 * s + 8 * c;
+      store_group(L.dtype, out, idx, e, raw8);
     }
-    // rANS integrity: every lane back at L, words ending within the padding.
-    const uint32_t used = pos - cb * kChunkBytes;
-    bool bad = (x != kStateLow) || used > bytes || bytes - used >= 16;
-    if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) atomicOr(status, kStatusCorrupt);
-    cb += nch;
+    if (!tile_end(tc, single) && lane == 0) atomicOr(status, kStatusCorrupt);
   }
   pipe_drain(pipe, status);
 }
@@ -170,11 +178,16 @@ cudaError_t launch_decode_tiles(const LayerDev& L, void* out, uint32_t* status,
   cudaError_t e = cudaFuncSetAttribute(decode_tiles_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem);
   if (e != cudaSuccess) return e;
-  uint32_t blocks = (L.n_tiles + kDecWarps - 1) / kDecWarps;
-  uint32_t cap = 2u * static_cast<uint32_t>(num_sms);
-  if (blocks > cap) blocks = cap;
-  if (blocks == 0) return cudaSuccess;
-  decode_tiles_kernel<<<blocks, kDecWarps * 32, kDecSmem, stream>>>(L, out, status);
+  if (L.n_tiles == 0) return cudaSuccess;
+  // One warp decodes one tile at a time, so the tiles are the unit of
+  // parallelism: spread them evenly, up to 2 blocks x 16 warps per SM.
+  const uint32_t sms = num_sms > 0 ? static_cast<uint32_t>(num_sms) : 148;
+  uint32_t warps = (L.n_tiles + sms - 1) / sms;
+  if (warps > kDecMaxWarps) warps = kDecMaxWarps;
+  if (warps < 1) warps = 1;
+  uint32_t blocks = (L.n_tiles + warps - 1) / warps;
+  if (blocks > 2 * sms) blocks = 2 * sms;
+  decode_tiles_kernel<<<blocks, warps * 32, kDecSmem, stream>>>(L, out, status);
   return cudaGetLastError();
 }
 

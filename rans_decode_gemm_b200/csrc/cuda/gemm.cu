@@ -23,7 +23,6 @@
 //     depend on timing and matches ans_gemm_uncompressed exactly.
 //   * A W row block split over several CTAs is reduced by the last CTA to
 //     finish it, in ascending CTA order (deterministic, no float atomics).
-#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdlib>
@@ -74,33 +73,67 @@ __device__ __forceinline__ uint32_t cta_of(uint64_t U, uint32_t G, uint64_t u) {
   return c;
 }
 
-// Calls f(u, s, d) in the order the MMA thread consumes (unit, slab) pairs.
-// With two accumulator sets a round is consumed slab-major across all its
-// units; with one set, the units of each segment of the round are finished
-// before the next segment starts (so its accumulator can be drained first).
-// Either way the order within one segment is (slab, unit) ascending.
+// Where a unit sits: K tile, token pass and W row-block segment, plus
+// whether it opens / closes its segment within this CTA's range.
+struct UnitInfo {
+  uint32_t kt, p, lseg;
+  bool seg_first, seg_last;
+};
+
+// Calls f(u, s, d, r, info) in the order the MMA thread consumes (unit, slab)
+// pairs.  With two accumulator sets a round is consumed slab-major across
+// all its units; with one set, the units of each segment of the round are
+// finished before the next segment starts (so its accumulator can be drained
+// first).  Either way the order within one segment is (slab, unit)
+// ascending.  Unit coordinates are tracked incrementally (two divisions per
+// round) so the single issuing threads stay cheap.
 template <class F>
-__device__ __forceinline__ void for_each_mma_step(const GemmDev& P, uint64_t u_begin,
-                                                  uint64_t u_end, F&& f) {
-  const uint32_t n_kt = P.L.n_kt;
-  for (uint64_t u0 = u_begin; u0 < u_end; u0 += P.D) {
-    const uint32_t nd = static_cast<uint32_t>(u_end - u0 < P.D ? u_end - u0 : P.D);
+__device__ __forceinline__ void for_each_mma_step(const GemmDev& P, uint32_t u_begin,
+                                                  uint32_t u_end, F&& f) {
+  const uint32_t n_kt = P.L.n_kt, n_rb = P.n_rb;
+  const uint32_t seg_begin = u_begin / n_kt;
+  uint32_t r = 0;
+  for (uint32_t u0 = u_begin; u0 < u_end; u0 += P.D, ++r) {
+    const uint32_t nd = min(P.D, u_end - u0);
+    const uint32_t seg0 = u0 / n_kt, kt0 = u0 - seg0 * n_kt;
+    const uint32_t p0 = seg0 / n_rb, p1 = (seg0 + 1) / n_rb;
+    auto info = [&](uint32_t d) {
+      UnitInfo I;
+      uint32_t kt = kt0 + d;
+      const bool wrap = kt >= n_kt;
+      kt -= wrap ? n_kt : 0;
+      const uint32_t seg = seg0 + (wrap ? 1u : 0u);
+      const uint32_t u = u0 + d;
+      I.kt = kt;
+      I.p = wrap ? p1 : p0;
+      I.lseg = seg - seg_begin;
+      I.seg_first = (u == u_begin) || (kt == 0);
+      I.seg_last = (u + 1 == u_end) || (kt + 1 == n_kt);
+      return I;
+    };
     if (P.n_bufs == 2) {
       for (uint32_t s = 0; s < P.C; ++s)
-        for (uint32_t d = 0; d < nd; ++d) f(u0 + d, s, d);
+        for (uint32_t d = 0; d < nd; ++d) f(u0 + d, s, d, r, info(d));
     } else {
-      const uint64_t seg_end = (u0 / n_kt + 1) * n_kt;
-      const uint32_t nA = static_cast<uint32_t>(seg_end - u0 < nd ? seg_end - u0 : nd);
+      const uint32_t nA = min(nd, n_kt - kt0);
       for (uint32_t s = 0; s < P.C; ++s)
-        for (uint32_t d = 0; d < nA; ++d) f(u0 + d, s, d);
+        for (uint32_t d = 0; d < nA; ++d) f(u0 + d, s, d, r, info(d));
       for (uint32_t s = 0; s < P.C; ++s)
-        for (uint32_t d = nA; d < nd; ++d) f(u0 + d, s, d);
+        for (uint32_t d = nA; d < nd; ++d) f(u0 + d, s, d, r, info(d));
     }
   }
 }
 
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void trace_mark(const GemmDev& P, uint32_t slot) {
+  if (P.trace) {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    P.trace[blockIdx.x * 64 + slot] = t;
+  }
 }
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t b) {
@@ -110,7 +143,7 @@ __device__ __forceinline__ float bf16_to_f32(uint16_t b) {
 // ---------------------------------------------------------------------------
 template <bool kDecode, uint32_t kFmt>
 __global__ void __launch_bounds__(kMaxThreads, 1)
-    fused_gemm_kernel(const __grid_constant__ GemmDev P, const __grid_constant__ CUtensorMap tmX) {
+    fused_gemm_kernel(const __grid_constant__ GemmDev P) {
   extern __shared__ __align__(2048) uint8_t smem[];
   __shared__ uint32_t tmem_slot;
   __shared__ uint32_t abort_flag;
@@ -125,7 +158,8 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
 
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem + P.off_lut);
   uint8_t* wring = smem + P.off_w;
-  uint8_t* chunks = smem + P.off_chunk;
+  // chunk rings start on a kRingBytes-aligned shared address (the plan leaves slack)
+  uint8_t* chunks = smem + (((smem_u32(smem + P.off_chunk) + kRingBytes - 1) & ~(kRingBytes - 1)) - smem_u32(smem));
   uint8_t* xring = smem + P.off_x;
   Bars B = carve_bars(smem + P.off_bars, D, XS);
   const uint32_t x_stage_bytes = P.T_pass * 32;
@@ -143,13 +177,13 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     tmem_alloc(&tmem_slot, P.tmem_cols);
     tmem_relinquish();
   }
-  if (warp == 5 && lane == 0) prefetch_tmap(&tmX);
   if (kDecode && P.L.single_symbol == kNoSymbol) build_lut(lut, P.L, warp, blockDim.x / 32, lane);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = tmem_slot;
   volatile uint32_t* abort = &abort_flag;
+  if (threadIdx.x == 0) trace_mark(P, 0);
 
   if (warp >= kFixedWarps) {
     // ======================= producer warps =======================
@@ -158,33 +192,26 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     const LayerDev& L = P.L;
     const bool single = L.single_symbol != kNoSymbol;
     const uint32_t H = P.H;
-    const uint32_t slab_groups = 8;                 // 8 groups of 8 symbols per lane = one slab
     const uint32_t n_slabs = P.H * P.C;
+    const uint32_t groups = n_slabs * 8;  // 8 groups of 8 symbols per lane fill one slab
+    const uint32_t lut_s = smem_u32(lut);
     TileSeq seq{static_cast<uint32_t>(u_begin) + d, D, static_cast<uint32_t>(u_end), L.n_tiles};
     ChunkPipe pipe;
     pipe_init(pipe, chunks + d * kRingBytes, B.chunk + 4 * d);
-    uint32_t cb = 0;
+    TileCursor tc;
+    tc.cb = 0;
     uint32_t sc = 0;  // unit slabs produced
     const uint32_t swz = ((lane >> 2) & 1u) << 4;
+    const uint32_t wslots_s = smem_u32(wring + 2 * d * kSlabBytes);
 
     for (uint32_t r = 0; seq.has(r); ++r) {
       const uint32_t t = seq.at(r);
       const uint32_t n0 = (t / n_kt) * L.tile_n, k0 = (t % n_kt) * L.tile_k;
-      // ---- per-tile setup
-      uint32_t x = kStateLow, pos = 0, last = 0, nch = 0, bytes = 0;
       bool zero_tile = false;
       if (kDecode) {
-        uint64_t start;
-        if (!tile_extent(L, t, &start, &bytes)) {
+        if (!tile_begin(pipe, L, seq, t, tc, lane, abort, P.status)) {
           zero_tile = true;
           if (lane == 0) atomicOr(P.status, kStatusBadOffsets);
-        } else {
-          nch = (bytes + kChunkBytes - 1) / kChunkBytes;
-          last = cb + nch - 1;
-          pos = cb * kChunkBytes;
-          pipe_before_group(pipe, L, seq, pos, last, lane, abort, P.status);
-          x = *reinterpret_cast<const uint32_t*>(pipe.ring + ((pos + 4 * lane) & (kRingBytes - 1)));
-          pos += 4 * kLanes;
         }
       }
       __half2 gscale[8];
@@ -192,36 +219,63 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         const uint32_t gk = k0 / P.group_k;
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-          uint32_t hh = q / 4, ii = q % 4;
+          const uint32_t hh = q / 4, ii = q % 4;
           float sv = 0.f;
           if (hh < H) {
-            uint32_t row = n0 + lane + 32 * (4 * hh + ii);
+            const uint32_t row = n0 + lane + 32 * (4 * hh + ii);
             sv = bf16_to_f32(__ldg(static_cast<const uint16_t*>(P.scales) +
                                    static_cast<uint64_t>(row) * P.n_groups_k + gk));
           }
           gscale[q] = __float2half2_rn(sv);
         }
       }
-      const uint8_t* raw_tile =
-          (kFmt == kFmtBf16Split && kDecode) ? L.raw + static_cast<uint64_t>(t) * (L.tile_n * L.tile_k) + lane * 8
-                                             : nullptr;
-      uint64_t raw_next = 0;
-      if (kFmt == kFmtBf16Split && kDecode && !zero_tile)
-        raw_next = __ldg(reinterpret_cast<const unsigned long long*>(raw_tile));
+      // raw sign/mantissa bytes of groups g, g+1, g+2 in flight (bf16, decode)
+      const unsigned long long* raw_tile = nullptr;
+      uint64_t r0 = 0, r1 = 0, r2 = 0;
+      if (kDecode && kFmt == kFmtBf16Split && !zero_tile) {
+        raw_tile = reinterpret_cast<const unsigned long long*>(
+                       L.raw + static_cast<uint64_t>(t) * (L.tile_n * L.tile_k)) + lane;
+        r0 = __ldg(raw_tile);
+        r1 = __ldg(raw_tile + 32);
+        r2 = __ldg(raw_tile + 64);
+      }
 
       for (uint32_t us = 0; us < n_slabs; ++us) {
         const uint32_t h = us % H, s = us / H;
         const uint32_t slot = sc & 1u;
-        if (sc >= 2) wait_live(&B.w_empty[2 * d + slot], ((sc >> 1) + 1) & 1u, abort, P.status);
-        uint8_t* slab = wring + (2 * d + slot) * kSlabBytes;
-        for (uint32_t gg = 0; gg < slab_groups; ++gg) {
-          const uint32_t g = us * slab_groups + gg;
+        // copy mode: fetch the slab's 8 groups before waiting for the slot
+        uint4 cp[8];
+        if (!kDecode) {
+#pragma unroll
+          for (int gg = 0; gg < 8; ++gg) {
+            const uint32_t i = gg & 3, c = gg >> 2;
+            const uint64_t row = n0 + lane + 32 * (4 * h + i);
+            const uint64_t idx = row * L.K + k0 + 16 * s + 8 * c;
+            if (kFmt == kFmtBf16Split) {
+              cp[gg] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(P.w_plain) + idx));
+            } else if (kFmt == kFmtFp8F16) {
+              uint2 v = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(P.w_plain) + idx));
+              cp[gg] = make_uint4(v.x, v.y, 0, 0);
+            } else {
+              uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(P.w_plain) + idx / 2));
+              cp[gg] = make_uint4(v, 0, 0, 0);
+            }
+          }
+        }
+        if (sc >= 2) wait_live(&B.w_empty[2 * d + slot], ((sc >> 1) + 1) & 1u, abort, P.status, 1);
+        const uint32_t slab_s = wslots_s + slot * kSlabBytes;
+#pragma unroll 1
+        for (uint32_t gg = 0; gg < 8; ++gg) {
+          const uint32_t g = us * 8 + gg;
           const uint32_t i = gg & 3, c = gg >> 2;
           uint32_t o[4];
           if (kDecode) {
-            uint64_t raw8 = raw_next;
-            if (kFmt == kFmtBf16Split && !zero_tile && g + 1 < n_slabs * slab_groups)
-              raw_next = __ldg(reinterpret_cast<const unsigned long long*>(raw_tile + (g + 1) * 256));
+            const uint64_t raw8 = r0;
+            if (kFmt == kFmtBf16Split && !zero_tile) {
+              r0 = r1;
+              r1 = r2;
+              if (g + 3 < groups) r2 = __ldg(raw_tile + 32 * (g + 3));
+            }
             uint32_t e[8];
             if (zero_tile) {
 #pragma unroll
@@ -230,9 +284,9 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
 #pragma unroll
               for (int k = 0; k < 8; ++k) e[k] = L.single_symbol << 12;
             } else {
-              pipe_before_group(pipe, L, seq, pos, last, lane, abort, P.status);
+              tile_group(pipe, L, seq, tc, lane, abort, P.status);
 #pragma unroll
-              for (int k = 0; k < 8; ++k) e[k] = decode_step(x, pos, lut, pipe.ring, lt);
+              for (int k = 0; k < 8; ++k) e[k] = decode_step(tc.x, tc.pos, lut_s, pipe.ring_s, lt);
             }
             if (kFmt == kFmtBf16Split) fmt_bf16_split(e, raw8, o);
             else if (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
@@ -240,16 +294,15 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
             else fmt_fp8_f16(e, o);
             if (zero_tile) o[0] = o[1] = o[2] = o[3] = 0;
           } else {
-            // copy mode: read the original weights of this group
-            const uint64_t row = n0 + lane + 32 * (4 * h + i);
-            const uint64_t idx = row * L.K + k0 + 16 * s + 8 * c;
+            uint4 v = cp[0];
+#pragma unroll
+            for (int q = 1; q < 8; ++q)
+              if (gg == static_cast<uint32_t>(q)) v = cp[q];
             if (kFmt == kFmtBf16Split) {
-              uint4 v = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(P.w_plain) + idx));
               o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
             } else {
               uint32_t e[8];
               if (kFmt == kFmtFp8F16) {
-                uint2 v = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(P.w_plain) + idx));
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                   e[k] = ((v.x >> (8 * k)) & 0xFFu) << 12;
@@ -257,60 +310,53 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
                 }
                 fmt_fp8_f16(e, o);
               } else {
-                uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(P.w_plain) + idx / 2));
 #pragma unroll
-                for (int k = 0; k < 8; ++k) e[k] = (((v >> (4 * k)) & 0xFu) ^ 8u) << 12;
+                for (int k = 0; k < 8; ++k) e[k] = (((v.x >> (4 * k)) & 0xFu) ^ 8u) << 12;
                 if (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
                 else fmt_int4_f16_scaled(e, gscale[4 * h + i], o);
               }
             }
           }
-          const uint32_t rr = 32 * i + lane;
-          *reinterpret_cast<uint4*>(slab + rr * 32 + ((c << 4) ^ swz)) = make_uint4(o[0], o[1], o[2], o[3]);
+          const uint32_t addr = slab_s + (32 * i + lane) * 32 + ((c << 4) ^ swz);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(o[0]), "r"(o[1]),
+                       "r"(o[2]), "r"(o[3])
+                       : "memory");
         }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&B.w_full[2 * d + slot]);
+        if (lane == 0 && sc == 0) trace_mark(P, 2 + d);
         ++sc;
       }
       if (kDecode && !zero_tile) {
-        if (!single) {
-          const uint32_t used = pos - cb * kChunkBytes;
-          bool bad = (x != kStateLow) || used > bytes || bytes - used >= 16;
-          if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) atomicOr(P.status, kStatusCorrupt);
-        } else {
-          bool bad = (x != kStateLow) || bytes != 4 * kLanes;
-          if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) atomicOr(P.status, kStatusCorrupt);
-        }
-        cb += nch;
+        if (!tile_end(tc, single) && lane == 0) atomicOr(P.status, kStatusCorrupt);
       }
     }
     if (kDecode) pipe_drain(pipe, P.status);
+    if (lane == 0) trace_mark(P, 18 + d);
   } else if (warp == 4) {
     // ======================= MMA issue (one thread) =======================
     if (lane == 0) {
-      const uint64_t seg0 = u_begin / n_kt;
+      const uint32_t ub = static_cast<uint32_t>(u_begin), ue = static_cast<uint32_t>(u_end);
       uint32_t fresh = 0;  // bit (buf * 2 + h): next MMA into that accumulator starts it
       uint32_t xc = 0;
-      for_each_mma_step(P, u_begin, u_end, [&](uint64_t u, uint32_t s, uint32_t d) {
-        const uint64_t seg = u / n_kt;
-        const uint32_t lseg = static_cast<uint32_t>(seg - seg0);
-        const uint32_t buf = lseg % P.n_bufs;
-        const bool seg_first = (u == u_begin) || (u % n_kt == 0);
-        const bool seg_last = (u + 1 == u_end) || ((u + 1) % n_kt == 0);
-        if (s == 0 && seg_first) {
-          const uint32_t k = lseg / P.n_bufs;
-          if (k >= 1) wait_live(&B.acc_empty[buf], (k - 1) & 1u, abort, P.status);
+      uint32_t nstep = 0;
+      for_each_mma_step(P, ub, ue, [&](uint32_t u, uint32_t s, uint32_t d, uint32_t r,
+                                       const UnitInfo& I) {
+        const uint32_t lseg = I.lseg;
+        const uint32_t buf = P.n_bufs == 2 ? (lseg & 1u) : 0u;
+        if (s == 0 && I.seg_first) {
+          const uint32_t k = P.n_bufs == 2 ? (lseg >> 1) : lseg;
+          if (k >= 1) wait_live(&B.acc_empty[buf], (k - 1) & 1u, abort, P.status, 4);
           tc_fence_after();
           fresh |= 3u << (2 * buf);
         }
         const uint32_t xs = xc % XS;
-        wait_live(&B.x_full[xs], (xc / XS) & 1u, abort, P.status);
-        const uint32_t r = static_cast<uint32_t>((u - u_begin) / P.D);
+        wait_live(&B.x_full[xs], (xc / XS) & 1u, abort, P.status, 2);
         for (uint32_t h = 0; h < P.H; ++h) {
           const uint32_t idx = (r * P.C + s) * P.H + h;
           const uint32_t slot = idx & 1u;
-          wait_live(&B.w_full[2 * d + slot], (idx >> 1) & 1u, abort, P.status);
+          wait_live(&B.w_full[2 * d + slot], (idx >> 1) & 1u, abort, P.status, 3);
           tc_fence_after();
           const uint32_t a_addr = smem_u32(wring + (2 * d + slot) * kSlabBytes);
           const uint64_t adesc = sdesc_sw32(a_addr, 256);
@@ -326,36 +372,42 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         }
         umma_commit(&B.x_empty[xs]);
         ++xc;
-        if (s == P.C - 1 && seg_last) umma_commit(&B.acc_full[buf]);
+        if (s == P.C - 1 && I.seg_last) umma_commit(&B.acc_full[buf]);
+        if (nstep < 16) trace_mark(P, 48 + nstep);
+        ++nstep;
       });
       umma_commit(B.mma_done);
+      trace_mark(P, 34);
     }
     __syncwarp();
   } else if (warp == 5) {
     // ======================= X loader (TMA, one thread) =======================
     if (lane == 0) {
       uint32_t xc = 0;
-      uint32_t last_issued[8];  // per stage: 1 + index of the last load issued into it
-#pragma unroll
-      for (int k = 0; k < 8; ++k) last_issued[k] = 0;
-      for_each_mma_step(P, u_begin, u_end, [&](uint64_t u, uint32_t s, uint32_t) {
+      uint32_t n_issued = 0;  // loads issued: steps [0, n_issued) (none after an abort)
+      for_each_mma_step(P, static_cast<uint32_t>(u_begin), static_cast<uint32_t>(u_end),
+                        [&](uint32_t, uint32_t s, uint32_t, uint32_t, const UnitInfo& I) {
         const uint32_t xs = xc % XS;
-        if (xc >= XS) wait_live(&B.x_empty[xs], ((xc / XS) + 1) & 1u, abort, P.status);
-        const uint32_t p = static_cast<uint32_t>(u / P.L.n_tiles);
-        const uint32_t t = static_cast<uint32_t>(u % P.L.n_tiles);
-        const int32_t kx = static_cast<int32_t>((t % n_kt) * P.L.tile_k + 16 * s);
-        if (!*abort) {
+        if (xc >= XS) wait_live(&B.x_empty[xs], ((xc / XS) + 1) & 1u, abort, P.status, 5);
+        const uint32_t p = I.p;
+        const uint32_t kx = I.kt * P.L.tile_k + 16 * s;
+        if (!*abort && n_issued == xc) {
+          // X slab (pass p, 16-column slab kx/16) is T_pass x 32 contiguous,
+          // pre-swizzled bytes in the staged copy: one bulk copy
+          const uint64_t slab = static_cast<uint64_t>(p) * (P.L.K / 16) + kx / 16;
           mbar_arrive_expect_tx(&B.x_full[xs], P.T_pass * 32);
-          for (uint32_t j = 0; j < P.NT; ++j)
-            tma_load_2d(xring + xs * x_stage_bytes + j * P.T * 32, &tmX, kx,
-                        static_cast<int32_t>(p * P.T_pass + j * P.T), &B.x_full[xs]);
-          last_issued[xs] = xc + 1;
+          bulk_g2s(xring + xs * x_stage_bytes, P.xs + slab * (P.T_pass * 32), P.T_pass * 32,
+                   &B.x_full[xs]);
+          n_issued = xc + 1;
         }
         ++xc;
       });
+      trace_mark(P, 42);
       // drain: the last load issued into every stage must have landed
-      for (uint32_t k = 0; k < XS; ++k)
-        if (last_issued[k]) wait_drain(&B.x_full[k], ((last_issued[k] - 1) / XS) & 1u, P.status);
+      const uint32_t first = n_issued > XS ? n_issued - XS : 0;
+      for (uint32_t q = first; q < n_issued; ++q)
+        wait_drain(&B.x_full[q % XS], (q / XS) & 1u, P.status);
+      trace_mark(P, 35);
     }
     __syncwarp();
   } else {
@@ -366,8 +418,9 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     for (uint64_t seg = seg_first; seg <= seg_last; ++seg) {
       const uint32_t lseg = static_cast<uint32_t>(seg - seg_first);
       const uint32_t buf = lseg % P.n_bufs;
-      wait_live(&B.acc_full[buf], (lseg / P.n_bufs) & 1u, abort, P.status);
+      wait_live(&B.acc_full[buf], (lseg / P.n_bufs) & 1u, abort, P.status, 6);
       tc_fence_after();
+      if (e == 0 && lseg < 2) trace_mark(P, 36 + lseg);
       const uint32_t p = static_cast<uint32_t>(seg / P.n_rb);
       const uint32_t rb = static_cast<uint32_t>(seg % P.n_rb);
       const uint64_t s_lo = seg * n_kt, s_hi = s_lo + n_kt;
@@ -417,25 +470,39 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         named_bar_sync(1, 128);
         if (reduce_flag) {
           __threadfence();
+          // contributors c_first..c_last; only c_first can hold this segment in
+          // its second (tail) slot, when its range started before the segment
+          const uint32_t sl_first = (cta_begin(P.n_units, G, c_first) < s_lo) ? 1u : 0u;
+          const uint64_t cta_stride = 2ull * P.H * P.T_pass * 128;
+          const uint32_t t_valid = min(P.T_pass, P.M - p * P.T_pass);
           for (uint32_t h = 0; h < P.H; ++h) {
-            const uint32_t n = rb * P.L.tile_n + h * 128 + e;
-            float scale = 1.0f;
-            if (P.scale_kind == 1) scale = bf16_to_f32(__ldg(static_cast<const uint16_t*>(P.scales) + n));
-            else if (P.scale_kind == 2) scale = __ldg(static_cast<const float*>(P.scales) + n);
-            for (uint32_t tok = 0; tok < P.T_pass; ++tok) {
-              const uint32_t m = p * P.T_pass + tok;
-              if (m >= P.M) break;
-              float acc = 0.f;
-              for (uint32_t c2 = c_first; c2 <= c_last; ++c2) {
-                const uint64_t c2_seg0 = cta_begin(P.n_units, G, c2) / n_kt;
-                const uint32_t sl = (c2_seg0 == seg) ? 0u : 1u;
-                const float* pp = P.partials + (static_cast<uint64_t>(c2) * 2 + sl) * P.H * P.T_pass * 128;
-                acc += __ldcg(pp + (static_cast<uint64_t>(h) * P.T_pass + tok) * 128 + e);
+            const uint32_t nh = rb * P.L.tile_n + h * 128;
+            for (uint32_t it = e; it < t_valid * 32; it += 128) {
+              const uint32_t tok = it >> 5, q = it & 31;
+              const uint64_t off = (static_cast<uint64_t>(h) * P.T_pass + tok) * 128 + 4 * q;
+              float4 acc = __ldcg(reinterpret_cast<const float4*>(
+                  P.partials + c_first * cta_stride + sl_first * (cta_stride / 2) + off));
+              for (uint32_t c2 = c_first + 1; c2 <= c_last; ++c2) {
+                const float4 v = __ldcg(reinterpret_cast<const float4*>(P.partials + c2 * cta_stride + off));
+                acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
               }
-              P.Y[static_cast<uint64_t>(m) * N + n] = acc * scale;
+              const uint32_t n = nh + 4 * q;
+              if (P.scale_kind == 1) {
+                const uint2 sb = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(P.scales) + n));
+                acc.x *= __uint_as_float(sb.x << 16);
+                acc.y *= __uint_as_float(sb.x & 0xFFFF0000u);
+                acc.z *= __uint_as_float(sb.y << 16);
+                acc.w *= __uint_as_float(sb.y & 0xFFFF0000u);
+              } else if (P.scale_kind == 2) {
+                const float4 sf = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(P.scales) + n));
+                acc.x *= sf.x; acc.y *= sf.y; acc.z *= sf.z; acc.w *= sf.w;
+              }
+              const uint32_t m = p * P.T_pass + tok;
+              *reinterpret_cast<float4*>(P.Y + static_cast<uint64_t>(m) * N + n) = acc;
             }
           }
           if (e == 0) P.counters[seg] = 0;
+          if (e == 0) trace_mark(P, 38);
         }
         named_bar_sync(1, 128);
       }
@@ -443,7 +510,9 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
   }
 
   // ---- teardown: every MMA retired before TMEM is released
+  if (threadIdx.x == 0) trace_mark(P, 40);
   __syncthreads();
+  if (threadIdx.x == 0) trace_mark(P, 41);
   if (warp == 0) {
     wait_drain(B.mma_done, 0, P.status);
     tc_fence_after();
@@ -451,24 +520,50 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
   }
 }
 
-__global__ void x_to_f16_kernel(const uint4* __restrict__ X, uint4* __restrict__ Xh, uint64_t n8) {
-  for (uint64_t i = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+// Stages X for the fused kernel: for every token pass p and 16-column slab
+// ks, a contiguous block of T_pass rows x 32 bytes holding X[p*T_pass + r]
+// [16 ks .. 16 ks + 15] (zero for rows >= M), its two 16-byte chunks placed
+// with the 32-byte swizzle the MMA descriptor expects (chunk c of row r at
+// c ^ ((r >> 2) & 1)); optionally converted to f16.  One thread per chunk.
+__global__ void x_stage_kernel(const uint16_t* __restrict__ X, uint8_t* __restrict__ xs,
+                               uint32_t M, uint32_t K, uint32_t T_pass, uint32_t n_pass,
+                               uint32_t to_f16) {
+  const uint64_t n_chunks = static_cast<uint64_t>(n_pass) * (K / 16) * T_pass * 2;
+  for (uint64_t i = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_chunks;
        i += static_cast<uint64_t>(gridDim.x) * blockDim.x) {
-    uint4 v = __ldg(X + i);
-    uint32_t in[4] = {v.x, v.y, v.z, v.w}, out[4];
+    const uint32_t c = static_cast<uint32_t>(i & 1);
+    const uint64_t rest = i >> 1;
+    const uint32_t r = static_cast<uint32_t>(rest % T_pass);
+    const uint64_t slab = rest / T_pass;  // p * (K / 16) + ks
+    const uint32_t ks = static_cast<uint32_t>(slab % (K / 16));
+    const uint32_t p = static_cast<uint32_t>(slab / (K / 16));
+    const uint32_t m = p * T_pass + r;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (m < M) {
+      v = __ldg(reinterpret_cast<const uint4*>(X + static_cast<uint64_t>(m) * K + 16 * ks + 8 * c));
+      if (to_f16) {
+        uint32_t in[4] = {v.x, v.y, v.z, v.w}, out[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      float lo = __uint_as_float(in[k] << 16), hi = __uint_as_float(in[k] & 0xFFFF0000u);
-      __half2 h = __floats2half2_rn(lo, hi);
-      out[k] = *reinterpret_cast<uint32_t*>(&h);
+        for (int k = 0; k < 4; ++k) {
+          __half2 h = __floats2half2_rn(__uint_as_float(in[k] << 16), __uint_as_float(in[k] & 0xFFFF0000u));
+          out[k] = *reinterpret_cast<uint32_t*>(&h);
+        }
+        v = make_uint4(out[0], out[1], out[2], out[3]);
+      }
     }
-    Xh[i] = make_uint4(out[0], out[1], out[2], out[3]);
+    const uint64_t dst = slab * (static_cast<uint64_t>(T_pass) * 32) + r * 32 + ((c ^ ((r >> 2) & 1u)) << 4);
+    *reinterpret_cast<uint4*>(xs + dst) = v;
   }
 }
 
 // =============================== host side ===============================
 
 static uint32_t round_up(uint32_t a, uint32_t b) { return (a + b - 1) / b * b; }
+
+static unsigned long long* g_trace = nullptr;
+void set_trace_buffer(void* d_buf, size_t bytes) {
+  g_trace = bytes >= 64 * sizeof(unsigned long long) ? static_cast<unsigned long long*>(d_buf) : nullptr;
+}
 
 bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool decode, int num_sms,
                     GemmPlan* plan) {
@@ -524,31 +619,35 @@ bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool dec
   }
   if (D > L.n_kt) D = L.n_kt;
   if (D > per_cta) D = static_cast<uint32_t>(per_cta);
-  uint32_t XS = x_stage <= 2048 ? 8 : (x_stage <= 8192 ? 4 : 3);
+  // X stages take whatever shared memory the producers leave (deep rings keep
+  // every X slab of a round in flight at small M), at least 2, at most 64.
+  uint32_t XS = 0;
   for (;;) {
     uint32_t off = lut_bytes;
     off = round_up(off, 2048);
-    uint32_t off_w = off;
+    const uint32_t off_w = off;
     off += D * 2 * kSlabBytes;
     off = round_up(off, 2048);
-    uint32_t off_chunk = off;
-    off += decode ? D * kRingBytes : 0;
+    const uint32_t off_chunk = off;
+    off += decode ? (D + 1) * kRingBytes : 0;
     off = round_up(off, 1024);
-    uint32_t off_x = off;
-    off += XS * x_stage;
-    off = round_up(off, 8);
-    uint32_t off_bars = off;
-    off += num_bars(D, XS) * 8;
-    if (off <= kSmemLimit) {
+    const uint32_t off_x = off;
+    const uint32_t bars_max = num_bars(D, 64) * 8;
+    const uint32_t room = kSmemLimit > off + bars_max ? kSmemLimit - off - bars_max : 0;
+    XS = room / x_stage;
+    if (XS > 64) XS = 64;
+    if (XS >= 2) {
+      off += XS * x_stage;
+      off = round_up(off, 8);
       p.off_lut = 0;
       p.off_w = off_w;
       p.off_chunk = off_chunk;
       p.off_x = off_x;
-      p.off_bars = off_bars;
+      p.off_bars = off;
+      off += num_bars(D, XS) * 8;
       p.smem_bytes = off;
       break;
     }
-    if (XS > 2) { --XS; continue; }
     if (D > 1) { --D; continue; }
     return false;
   }
@@ -556,39 +655,29 @@ bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool dec
   p.x_stages = XS;
   p.ws_partials_bytes = static_cast<size_t>(p.grid) * 2 * p.H * p.T_pass * 128 * sizeof(float);
   p.ws_counters_bytes = round_up(p.n_segments * 4, 256);
-  p.ws_x16_bytes = p.ab_f16 ? static_cast<size_t>(M) * L.K * 2 : 0;
+  p.ws_x16_bytes = static_cast<size_t>(p.n_pass) * p.T_pass * L.K * 2;  // staged X slabs
   p.ws_bytes = p.ws_counters_bytes + (p.ws_partials_bytes + 255) / 256 * 256 +
                (p.ws_x16_bytes + 255) / 256 * 256;
   *plan = p;
   return true;
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn encode_tiled_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
-  return fn;
-}
-
 template <bool kDecode, uint32_t kFmt>
-static cudaError_t launch_variant(const GemmPlan& plan, const GemmDev& P, const CUtensorMap& tm,
-                                  cudaStream_t stream) {
+static cudaError_t launch_variant(const GemmPlan& plan, const GemmDev& P, cudaStream_t stream) {
   auto kern = fused_gemm_kernel<kDecode, kFmt>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(plan.smem_bytes));
+  // the opt-in shared-memory size is a per-device function attribute: set it
+  // once per device and variant
+  static int attr_set[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  kern<<<plan.grid, (kFixedWarps + plan.D) * 32, plan.smem_bytes, stream>>>(P, tm);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = 1;
+  }
+  kern<<<plan.grid, (kFixedWarps + plan.D) * 32, plan.smem_bytes, stream>>>(P);
   return cudaGetLastError();
 }
 
@@ -602,30 +691,16 @@ cudaError_t launch_gemm(const GemmPlan& plan, const LayerDev& L, bool decode, co
   float* partials = reinterpret_cast<float*>(wsb + plan.ws_counters_bytes);
   uint16_t* x16 = reinterpret_cast<uint16_t*>(wsb + plan.ws_counters_bytes +
                                               ((plan.ws_partials_bytes + 255) / 256) * 256);
-  const void* xsrc = X;
-  if (plan.ab_f16) {
-    uint64_t n8 = static_cast<uint64_t>(plan.M) * L.K / 8;
-    uint32_t blocks = static_cast<uint32_t>((n8 + 255) / 256);
-    if (blocks > 1184) blocks = 1184;
+  {
+    const uint64_t n_chunks = static_cast<uint64_t>(plan.n_pass) * (L.K / 16) * plan.T_pass * 2;
+    uint32_t blocks = static_cast<uint32_t>((n_chunks + 255) / 256);
+    if (blocks > 4096) blocks = 4096;
     if (blocks == 0) blocks = 1;
-    x_to_f16_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<const uint4*>(X),
-                                                reinterpret_cast<uint4*>(x16), n8);
+    x_stage_kernel<<<blocks, 256, 0, stream>>>(X, reinterpret_cast<uint8_t*>(x16), plan.M, L.K,
+                                               plan.T_pass, plan.n_pass, plan.ab_f16);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    xsrc = x16;
   }
-  EncodeTiledFn enc = encode_tiled_fn();
-  if (!enc) return cudaErrorNotSupported;
-  CUtensorMap tm;
-  cuuint64_t gdim[2] = {L.K, plan.M};
-  cuuint64_t gstride[1] = {static_cast<cuuint64_t>(L.K) * 2};
-  cuuint32_t box[2] = {16, plan.T};
-  cuuint32_t estride[2] = {1, 1};
-  CUresult cr = enc(&tm, plan.ab_f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                    2, const_cast<void*>(xsrc), gdim, gstride, box, estride,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
 
   GemmDev P;
   std::memset(&P, 0, sizeof(P));
@@ -658,16 +733,18 @@ cudaError_t launch_gemm(const GemmPlan& plan, const LayerDev& L, bool decode, co
   P.off_chunk = plan.off_chunk;
   P.off_x = plan.off_x;
   P.off_bars = plan.off_bars;
+  P.trace = g_trace;
+  P.xs = reinterpret_cast<const uint8_t*>(x16);
 
   switch (plan.fmt | (decode ? 0u : 8u)) {
-    case kFmtBf16Split: return launch_variant<true, kFmtBf16Split>(plan, P, tm, stream);
-    case kFmtInt4Bf16: return launch_variant<true, kFmtInt4Bf16>(plan, P, tm, stream);
-    case kFmtInt4F16Group: return launch_variant<true, kFmtInt4F16Group>(plan, P, tm, stream);
-    case kFmtFp8F16: return launch_variant<true, kFmtFp8F16>(plan, P, tm, stream);
-    case 8 | kFmtBf16Split: return launch_variant<false, kFmtBf16Split>(plan, P, tm, stream);
-    case 8 | kFmtInt4Bf16: return launch_variant<false, kFmtInt4Bf16>(plan, P, tm, stream);
-    case 8 | kFmtInt4F16Group: return launch_variant<false, kFmtInt4F16Group>(plan, P, tm, stream);
-    case 8 | kFmtFp8F16: return launch_variant<false, kFmtFp8F16>(plan, P, tm, stream);
+    case kFmtBf16Split: return launch_variant<true, kFmtBf16Split>(plan, P, stream);
+    case kFmtInt4Bf16: return launch_variant<true, kFmtInt4Bf16>(plan, P, stream);
+    case kFmtInt4F16Group: return launch_variant<true, kFmtInt4F16Group>(plan, P, stream);
+    case kFmtFp8F16: return launch_variant<true, kFmtFp8F16>(plan, P, stream);
+    case 8 | kFmtBf16Split: return launch_variant<false, kFmtBf16Split>(plan, P, stream);
+    case 8 | kFmtInt4Bf16: return launch_variant<false, kFmtInt4Bf16>(plan, P, stream);
+    case 8 | kFmtInt4F16Group: return launch_variant<false, kFmtInt4F16Group>(plan, P, stream);
+    case 8 | kFmtFp8F16: return launch_variant<false, kFmtFp8F16>(plan, P, stream);
   }
   return cudaErrorInvalidValue;
 }

@@ -65,7 +65,13 @@ struct GemmDev {
   uint64_t n_units;
   uint32_t idesc;
   uint32_t off_lut, off_w, off_chunk, off_x, off_bars;
+  unsigned long long* trace;  // optional per-CTA event timestamps (internal profiling)
+  const uint8_t* xs;          // X staged as pre-swizzled 16-column slabs (workspace)
 };
+
+// Internal profiling hook: when set, every fused-GEMM CTA writes globaltimer
+// stamps of its phases to trace[cta * 64 + slot].
+void set_trace_buffer(void* d_buf, size_t bytes);
 
 // Fills a plan; returns false if the shape cannot be scheduled.
 bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool decode,

@@ -43,15 +43,16 @@ enum : uint32_t { kDtInt4 = 0, kDtBf16Split = 1, kDtFp8 = 2 };
 
 // Abort-aware bounded wait.  Returns false if the wait ran out (then sets the
 // CTA's abort flag and the TIMEOUT status bit) or if the CTA already aborted.
+// site: which wait (diagnostic bit 8 + site is set next to TIMEOUT).
 __device__ __forceinline__ bool wait_live(uint64_t* bar, uint32_t parity, volatile uint32_t* abort,
-                                          uint32_t* status) {
+                                          uint32_t* status, uint32_t site = 0) {
   if (mbar_try_wait(bar, parity)) return true;
   long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
     if (*abort) return false;
     if (clock64() - t0 > kWaitBudgetCycles) {
       *abort = 1u;
-      atomicOr(status, kStatusTimeout);
+      atomicOr(status, kStatusTimeout | (1u << (8 + site)));
       return false;
     }
   }
@@ -107,7 +108,8 @@ struct TileSeq {
 // Per-warp compressed-byte pipeline.  All lanes hold the same values; lane 0
 // issues the copies.
 struct ChunkPipe {
-  uint8_t* ring;      // kRingBytes, kRingBytes-aligned shared memory
+  uint8_t* ring;      // kRingBytes of shared memory (generic pointer, for copies)
+  uint32_t ring_s;    // the same ring as a kRingBytes-aligned shared address
   uint64_t* bars;     // 4 mbarriers (count 1)
   uint32_t issued;    // chunks issued so far (global index over the warp's tiles)
   uint32_t ready;     // chunks known to have landed
@@ -118,6 +120,7 @@ struct ChunkPipe {
 
 __device__ __forceinline__ void pipe_init(ChunkPipe& p, uint8_t* ring, uint64_t* bars) {
   p.ring = ring;
+  p.ring_s = smem_u32(ring);
   p.bars = bars;
   p.issued = p.ready = 0;
   p.it_r = 0;
@@ -167,33 +170,103 @@ __device__ __forceinline__ void pipe_drain(ChunkPipe& p, uint32_t* status) {
   }
 }
 
-// Keeps the ring full and the chunks that the next group can touch resident.
-// pos: read position in ring bytes (unwrapped); last_chunk: final chunk of
-// the current tile.
-__device__ __forceinline__ void pipe_before_group(ChunkPipe& p, const LayerDev& L,
-                                                  const TileSeq& seq, uint32_t pos,
-                                                  uint32_t last_chunk, uint32_t lane,
-                                                  volatile uint32_t* abort, uint32_t* status) {
-  uint32_t c = pos / kChunkBytes;
+// Keeps the ring full and the chunks that the next groups can touch
+// resident.  Called when the read position enters chunk c: afterwards chunks
+// up to min(c + 1, last_chunk) are resident (a group of 8 steps reads at most
+// 512 bytes) and up to three chunks beyond c are in flight.
+__device__ __forceinline__ void pipe_enter_chunk(ChunkPipe& p, const LayerDev& L,
+                                                 const TileSeq& seq, uint32_t c,
+                                                 uint32_t last_chunk, uint32_t lane,
+                                                 volatile uint32_t* abort, uint32_t* status) {
   uint32_t limit = min(c, p.ready) + 4u;
   if (p.issued < limit && !*abort) pipe_issue(p, L, seq, limit, lane);
   uint32_t need = min(c + 1u, last_chunk);
   if (p.ready <= need) pipe_wait(p, need, abort, status);
+  limit = min(c, p.ready) + 4u;
+  if (p.issued < limit && !*abort) pipe_issue(p, L, seq, limit, lane);
 }
 
-// One decode step for the calling lane.  x: state; pos: ring read position
-// (bytes, unwrapped; advanced by the words the warp consumed).
-__device__ __forceinline__ uint32_t decode_step(uint32_t& x, uint32_t& pos,
-                                                const uint32_t* __restrict__ lut,
-                                                const uint8_t* __restrict__ ring, uint32_t lt) {
-  uint32_t e = lut[x & (kSlots - 1)];
-  x = (e >> 20) * (x >> 12) + (e & 0xFFFu);
-  bool need = x < kStateLow;
-  uint32_t bal = __ballot_sync(0xFFFFFFFFu, need);
-  if (need) {
-    uint32_t off = (pos + 2u * __popc(bal & lt)) & (kRingBytes - 1);
-    x = (x << 16) | *reinterpret_cast<const uint16_t*>(ring + off);
+// Decode position inside the current tile of a warp.
+struct TileCursor {
+  uint32_t x;      // lane state
+  uint32_t pos;    // ring read position (bytes, unwrapped)
+  uint32_t chunk;  // chunk holding pos when the pipeline was last consulted
+  uint32_t cb;     // first chunk of the tile
+  uint32_t last;   // last chunk of the tile
+  uint32_t bytes;  // tile bytes (padded)
+};
+
+// Starts tile t: validates its extent, makes its first chunks resident and
+// loads the lane states.  Returns false for a tile with invalid offsets.
+__device__ __forceinline__ bool tile_begin(ChunkPipe& p, const LayerDev& L, const TileSeq& seq,
+                                           uint32_t t, TileCursor& tc, uint32_t lane,
+                                           volatile uint32_t* abort, uint32_t* status) {
+  uint64_t start;
+  if (!tile_extent(L, t, &start, &tc.bytes)) return false;
+  const uint32_t nch = (tc.bytes + kChunkBytes - 1) / kChunkBytes;
+  tc.last = tc.cb + nch - 1;
+  tc.pos = tc.cb * kChunkBytes;
+  tc.chunk = tc.cb;
+  pipe_enter_chunk(p, L, seq, tc.chunk, tc.last, lane, abort, status);
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];"
+               : "=r"(v)
+               : "r"(((tc.pos + 4 * lane) & (kRingBytes - 1)) + p.ring_s)
+               : "memory");
+  tc.x = v;
+  tc.pos += 4 * kLanes;
+  return true;
+}
+
+// Before each group of 8 steps: consult the pipeline when a new chunk starts.
+__device__ __forceinline__ void tile_group(ChunkPipe& p, const LayerDev& L, const TileSeq& seq,
+                                           TileCursor& tc, uint32_t lane, volatile uint32_t* abort,
+                                           uint32_t* status) {
+  const uint32_t c = tc.pos / kChunkBytes;
+  if (c != tc.chunk) {
+    tc.chunk = c;
+    pipe_enter_chunk(p, L, seq, c, tc.last, lane, abort, status);
   }
+}
+
+// Ends a tile: rANS integrity (every lane back at L, words ending inside the
+// padding; a single-symbol tile holds only its states) and advances to the
+// next tile's first chunk.
+__device__ __forceinline__ bool tile_end(TileCursor& tc, bool single) {
+  const uint32_t used = tc.pos - tc.cb * kChunkBytes;
+  bool bad = (tc.x != kStateLow) || used > tc.bytes || tc.bytes - used >= 16;
+  if (single) bad = (tc.x != kStateLow) || tc.bytes != 4 * kLanes;
+  tc.cb = tc.last + 1;
+  return !__any_sync(0xFFFFFFFFu, bad);
+}
+
+// One decode step for the calling lane, branch-free, on 32-bit shared-memory
+// addresses.  x: state; pos: ring read position (bytes, unwrapped; advanced
+// by the words the whole warp consumed); lut_s: slot-table address; ring_s:
+// ring address (kRingBytes-aligned); lt: %lanemask_lt.  Returns the slot-table
+// entry of the decoded symbol.  Every lane loads the word at its prefix
+// position (all such addresses lie in one 64-byte window, so the extra loads
+// cost no extra shared-memory wavefront); lanes that need no word discard it.
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint32_t decode_step(uint32_t& x, uint32_t& pos, uint32_t lut_s,
+                                                uint32_t ring_s, uint32_t lt) {
+  const uint32_t e = lds_u32(lut_s + ((x & (kSlots - 1)) << 2));
+  x = (e >> 20) * (x >> 12) + (e & 0xFFFu);
+  const bool need = x < kStateLow;
+  const uint32_t bal = __ballot_sync(0xFFFFFFFFu, need);
+  const uint32_t off = ((pos + 2u * __popc(bal & lt)) & (kRingBytes - 1)) + ring_s;
+  const uint32_t w = lds_u16(off);
+  x = need ? ((x << 16) | w) : x;
   pos += 2u * __popc(bal);
   return e;
 }
