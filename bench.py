@@ -1,0 +1,451 @@
+#!/usr/bin/env python3
+"""Benchmark of the fused tile-rANS decode + GEMM on one B200 per rank.
+
+Workload (the layer the headline metric is quoted on): a 4096 x 4096 bf16
+weight matrix drawn from N(0, 0.02), coded as an rANS exponent stream (one
+12-bit codebook, 128 x 64 tiles, 32 lanes) plus the raw sign/mantissa byte,
+multiplied by X (16 x 4096 bf16, N(0, 1)).  One step is one ans_gemm call
+(decode inside the GEMM, Y fp32).  Twelve copies of the compressed layer
+(together far larger than the 126 MB L2) rotate across steps, so every step
+reads its weights from HBM.
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle on
+the same workload instead.  Under torchrun every rank runs its own replica
+(no data-path collective: the layers are independent); the time is the max
+over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "bf16_4096"
+M_HEAD = 16
+N_COPIES = 12
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+KERNEL_SOURCES = ["rans_decode_gemm_b200/csrc/cuda/gemm.cu",
+                  "rans_decode_gemm_b200/csrc/cuda/rans_core.cuh",
+                  "rans_decode_gemm_b200/csrc/cuda/ptx.cuh"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10000)
+    ap.add_argument("--warmup", type=int, default=100)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--quick", action="store_true",
+                    help="skip the context sweep and the CPU baseline (profiling runs)")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            return json.load(fh), "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """dram read+write bytes per launch of the fused kernel from the committed
+    ncu summary, if it was taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "fused_gemm_bf16_4096_m16.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as fh:
+        d = json.load(fh)
+    if d.get("kernel_source_sha") != kernel_source_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        rows = []
+        with open(self.file.name) as fh:
+            for line in fh:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.file.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        under_load = sorted(sm)[len(sm) // 2:] if sm else []
+        return {"sm_mhz": statistics.median(under_load) if under_load else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def build_layers(torch, ans, WL, device):
+    cfg = WL.CONFIGS[WORKLOAD]
+    d = WL.make_weights(cfg, 0)
+    lay = ans.make_layout(cfg.dtype, d["N"], d["K"], cfg.tile_n, cfg.tile_k)
+    # offline path through the library: GPU histogram -> codebook -> host encode
+    dw = torch.from_numpy(d["w"].view(np.int16)).to(device)
+    hist = torch.zeros(256, dtype=torch.int64, device=device)
+    ans.ans_histogram(dw, lay, hist)
+    hist_h = hist.cpu().numpy().astype(np.uint64)
+    t0 = time.perf_counter()
+    cb = ans.ans_build_codebook(hist_h, 256, 12)
+    stream, offsets, raw = ans.ans_encode_tiles(d["w"], lay, cb)
+    encode_s = time.perf_counter() - t0
+    layers = [ans.CompressedLayer(lay, cb, stream, offsets, raw, device) for _ in range(N_COPIES)]
+    return cfg, d, lay, layers, hist_h, encode_s, dw
+
+
+def time_ours(args):
+    import torch
+    from rans_decode_gemm_b200 import ans
+    from rans_decode_gemm_b200 import workloads as WL
+
+    world, rank, local = dist_setup(args)
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=device)
+        pg = dist
+    cfg, d, lay, layers, hist, encode_s, dw = build_layers(torch, ans, WL, device)
+    N, K, M = lay.N, lay.K, M_HEAD
+    X_h = WL.make_x(cfg, M, K)
+    X = torch.from_numpy(X_h.view(np.int16)).to(device)
+    Y = torch.empty(M, N, dtype=torch.float32, device=device)
+    ws_bytes = ans.ans_gemm_workspace(lay, M, cfg.scale_kind)
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=device)
+    st = torch.zeros(1, dtype=torch.int32, device=device)
+    stream = torch.cuda.Stream(device=device)
+    torch.cuda.set_stream(stream)
+
+    def step(i):
+        ans.ans_gemm(X, M, layers[i % N_COPIES].tiles, cfg.scale_kind, None, 0, Y, ws,
+                     ws_bytes, st, stream)
+
+    def barrier():
+        torch.cuda.synchronize()
+        if pg is not None:
+            pg.barrier()
+        torch.cuda.synchronize()
+
+    # Each step is captured once per rotating layer copy as a CUDA graph, so
+    # the timed region measures the GPU work, not Python/ctypes launch cost.
+    for i in range(N_COPIES):          # eager warm-up: first-call attributes
+        step(i)
+    torch.cuda.synchronize()
+    graphs = []
+    for i in range(N_COPIES):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step(i)
+        graphs.append(g)
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    for i in range(args.warmup):
+        graphs[i % N_COPIES].replay()
+    barrier()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        graphs[i % N_COPIES].replay()
+    t1.record(stream)
+    barrier()
+    clocks = sampler.stop()
+    total_ms = t0.elapsed_time(t1)
+    kern_ms = total_ms / args.steps
+    status = int(st.item())
+    if pg is not None:
+        tt = torch.tensor([total_ms], device=device)
+        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    del graphs
+
+    # e2e through the same C ABI with host buffers: pinned X in, Y out per step
+    Xp = torch.from_numpy(X_h.view(np.int16)).pin_memory()
+    Yp = torch.empty(M, N, dtype=torch.float32).pin_memory()
+    Xd = torch.empty_like(X)
+
+    def e2e_step(i):
+        Xd.copy_(Xp, non_blocking=True)
+        ans.ans_gemm(Xd, M, layers[i % N_COPIES].tiles, cfg.scale_kind, None, 0, Y, ws,
+                     ws_bytes, st, stream)
+        Yp.copy_(Y, non_blocking=True)
+
+    for i in range(min(args.warmup, 20)):
+        e2e_step(i)
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    n_e2e = max(1, min(args.steps, 500))
+    e0.record(stream)
+    for i in range(n_e2e):
+        e2e_step(i)
+    e1.record(stream)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / n_e2e
+    if pg is not None:
+        tt = torch.tensor([e2e_ms], device=device)
+        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+
+    # context numbers on rank 0: other M, the two-pass baseline, uncompressed
+    extra = {}
+    if rank == 0 and not args.quick:
+        extra = context_numbers(torch, ans, WL, cfg, d, lay, layers, dw, device)
+
+    result = None
+    if rank == 0:
+        peaks, peaks_src = load_peaks()
+        weight_bytes = N * K * 2  # nominal bf16 storage of the decompressed weights
+        layer = layers[0]
+        algo_bytes = layer.compressed_bytes + 2 * M * K + 4 * M * N
+        ms_per_step = total_ms / args.steps
+        value = world * weight_bytes / (ms_per_step * 1e-3) / 1e9
+        achieved = algo_bytes / (kern_ms * 1e-3) / 1e9
+        peak = float(peaks["hbm_gbs"])
+        H_exp = ans.ans_entropy(hist)
+        bpw = 8.0 * layer.compressed_bytes / (N * K)
+        result = {
+            "metric": "fused decode-GEMM effective weight GB/s (bf16 weights, M=16)",
+            "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "bf16 split-stream 4096x4096 N(0,0.02), 128x64 tiles, 32 lanes, "
+                                   "12-bit freqs; X 16x4096 bf16 N(0,1); seed 1",
+                       "M": M, "N": N, "K": K, "global_batch": M * world,
+                       "parallelism": f"replicas x{world}",
+                       "l2": f"inputs larger than L2: {N_COPIES} rotating copies of the "
+                             f"compressed layer ({N_COPIES * layer.compressed_bytes / 1e6:.0f} MB)"},
+            "bits_per_weight": round(bpw, 4),
+            "entropy_bits": {"exponent": round(H_exp, 4), "split_bound": round(H_exp + 8, 4)},
+            "status": status,
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
+                         "unit": "GB/s", "frac": round(achieved / peak, 4),
+                         "traffic": profiled_traffic(), "peak_source": peaks_src,
+                         "algorithmic_bytes_per_launch": algo_bytes,
+                         "kernel_ms_per_launch": round(kern_ms, 6),
+                         "timing": "per-step time of the fused kernel plus its X staging "
+                                   "launch (CUDA-graph replays, events on the launch stream)"},
+            "e2e": {"value": round(world * weight_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                    "h2d_bytes_per_step": 2 * M * K, "d2h_bytes_per_step": 4 * M * N},
+            "gpu_launches": 2 * args.steps,  # per step: X staging + fused decode-GEMM
+            "clocks": clocks,
+            "offline": {"host_encode_s": round(encode_s, 3)},
+        }
+        result.update(extra)
+        if not (args.no_cpu_baseline or args.quick):
+            result["cpu_baseline"] = cpu_baseline(cfg, d, lay, layer, X_h, budget_s=20.0)
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+    return result
+
+
+def context_numbers(torch, ans, WL, cfg, d, lay, layers, dw, device):
+    """Single-GPU context: ans_gemm at the config's other M, the uncompressed
+    variant, cuBLAS on the decoded bf16 weights and the two-pass baseline
+    (ans_decode_tiles to HBM, then cuBLAS)."""
+    N, K = lay.N, lay.K
+    st = torch.zeros(1, dtype=torch.int32, device=device)
+    peaks, _ = load_peaks()
+
+    def timed(fn, iters=100, warm=10):
+        for i in range(warm):
+            fn(i)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for i in range(iters):
+            fn(i)
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / iters * 1e3  # us
+
+    W_copies = [torch.empty(N, K, dtype=torch.bfloat16, device=device) for _ in range(N_COPIES)]
+    for Wc in W_copies:
+        Wc.view(torch.int16).view(-1).copy_(dw)
+    out = {"sweep": []}
+    for M in cfg.Ms:
+        X = torch.from_numpy(WL.make_x(cfg, M, K).view(np.int16)).to(device)
+        Y = torch.empty(M, N, dtype=torch.float32, device=device)
+        nb = ans.ans_gemm_workspace(lay, M, cfg.scale_kind)
+        ws = torch.zeros(nb, dtype=torch.uint8, device=device)
+        t_f = timed(lambda i: ans.ans_gemm(X, M, layers[i % N_COPIES].tiles, 0, None, 0, Y, ws, nb, st))
+        t_u = timed(lambda i: ans.ans_gemm_uncompressed(X, M, W_copies[i % N_COPIES].view(torch.int16),
+                                                        lay, 0, None, 0, Y, ws, nb, st))
+        Xb = X.view(torch.bfloat16)
+        t_c = timed(lambda i: torch.matmul(Xb, W_copies[i % N_COPIES].t()))
+        dec = torch.empty(N, K, dtype=torch.bfloat16, device=device)
+        t_d = timed(lambda i: ans.ans_decode_tiles(layers[i % N_COPIES].tiles, dec, st))
+        t_2 = timed(lambda i: (ans.ans_decode_tiles(layers[i % N_COPIES].tiles, dec, st),
+                               torch.matmul(Xb, dec.t())))
+        algo = layers[0].compressed_bytes + 2 * M * K + 4 * M * N
+        flops = 2.0 * M * N * K
+        out["sweep"].append({
+            "M": M, "ans_gemm_us": round(t_f, 2),
+            "effective_weight_GBps": round(N * K * 2 / (t_f * 1e-6) / 1e9, 1),
+            "hbm_frac": round(algo / (t_f * 1e-6) / 1e9 / float(peaks["hbm_gbs"]), 4),
+            "tensor_frac": round(flops / (t_f * 1e-6) / 1e12 / float(peaks["bf16_tflops"]), 5),
+            "uncompressed_us": round(t_u, 2), "cublas_us": round(t_c, 2),
+            "decode_tiles_us": round(t_d, 2), "two_pass_us": round(t_2, 2),
+            "speedup_vs_two_pass": round(t_2 / t_f, 3)})
+    out["decode_tiles_Tsym_per_s"] = round(N * K / (out["sweep"][0]["decode_tiles_us"] * 1e-6) / 1e12, 4)
+    return out
+
+
+def cpu_baseline(cfg, d, lay, layer, X_h, budget_s=20.0):
+    """The CPU oracle, as it stands, on the host cores: decode of a sample of
+    whole W row blocks plus the fp64 GEMM on their rows, scaled to the metric
+    (effective weight GB/s)."""
+    from oracle import oracle as O
+    O.build()
+    cores = os.cpu_count() or 1
+    N, K, M = lay.N, lay.K, X_h.shape[0]
+    n_kt = K // lay.tile_k
+    freq = layer.codebook.freq_array()
+    rb_total = N // lay.tile_n
+    done_rb, t_spent = 0, 0.0
+    out = np.zeros(N * K, np.uint16)
+    while done_rb < rb_total and t_spent < budget_s:
+        t0 = time.perf_counter()
+        st, _ = O.decode(cfg.dtype, layer.h_stream, layer.h_offsets, layer.h_raw, N, K,
+                         lay.tile_n, lay.tile_k, freq, tile_begin=done_rb * n_kt,
+                         tile_end=(done_rb + 1) * n_kt, out=out, threads=cores)
+        rows = np.arange(done_rb * lay.tile_n, (done_rb + 1) * lay.tile_n, dtype=np.uint32)
+        O.gemm(cfg.dtype, X_h, M, K, out, N, rows=rows, threads=cores)
+        t_spent += time.perf_counter() - t0
+        done_rb += 1
+    weights = done_rb * lay.tile_n * K
+    return {"value": round(weights * 2 / t_spent / 1e9, 4), "unit": "GB/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"{done_rb} of {rb_total} row blocks of 128 rows: oracle decode of their "
+                      f"{done_rb * n_kt} tiles + fp64 GEMM of their rows with X {M}x{K}"}
+
+
+def time_reference(args):
+    world, rank, _ = dist_setup(args)
+    if rank != 0:
+        return None
+    from oracle import oracle as O
+    from rans_decode_gemm_b200 import ans
+    from rans_decode_gemm_b200 import workloads as WL
+    O.build()
+    cfg = WL.CONFIGS[WORKLOAD]
+    d = WL.make_weights(cfg, 0)
+    N, K, M = d["N"], d["K"], M_HEAD
+    counts = O.histogram(cfg.dtype, d["w"], N * K)
+    _, freq = O.normalize(counts)
+    st, stream, offsets, raw = O.encode(cfg.dtype, d["w"], N, K, cfg.tile_n, cfg.tile_k, freq)
+    X_h = WL.make_x(cfg, M, K)
+    cores = os.cpu_count() or 1
+    n_kt = K // cfg.tile_k
+    rb_total = N // cfg.tile_n
+    out = np.zeros(N * K, np.uint16)
+
+    def one(rb):
+        O.decode(cfg.dtype, stream, offsets, raw, N, K, cfg.tile_n, cfg.tile_k, freq,
+                 tile_begin=rb * n_kt, tile_end=(rb + 1) * n_kt, out=out, threads=cores)
+        rows = np.arange(rb * cfg.tile_n, (rb + 1) * cfg.tile_n, dtype=np.uint32)
+        O.gemm(cfg.dtype, X_h, M, K, out, N, rows=rows, threads=cores)
+
+    for i in range(args.warmup):
+        one(i % rb_total)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        one(i % rb_total)
+    dt = time.perf_counter() - t0
+    per_rb_s = dt / max(1, args.steps)
+    value = cfg.tile_n * K * 2 / per_rb_s / 1e9
+    sample = (f"each step: oracle decode of one 128-row block ({n_kt} tiles) + fp64 GEMM "
+              f"of its rows with X {M}x{K}")
+    return {"impl": "reference",
+            "metric": "fused decode-GEMM effective weight GB/s (bf16 weights, M=16)",
+            "value": round(value, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(per_rb_s * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": "bf16 split-stream 4096x4096 N(0,0.02), 128x64 tiles, 32 lanes, "
+                                   "12-bit freqs; X 16x4096 bf16 N(0,1); seed 1",
+                       "M": M, "N": N, "K": K},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        res = time_reference(args)
+    else:
+        res = time_ours(args)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()
