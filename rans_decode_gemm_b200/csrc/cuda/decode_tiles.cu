@@ -21,13 +21,14 @@ constexpr uint32_t kDecSmem = kDecLutBytes + kRingBytes + kDecMaxWarps * kRingBy
 
 // 8 output elements of one lane (row, 8 consecutive columns) in the original
 // storage format.
-__device__ __forceinline__ void store_group(uint32_t dtype, void* out, uint64_t idx,
-                                            const uint32_t (&e)[8], uint64_t raw8) {
-  if (dtype == kDtBf16Split) {
+template <uint32_t DT>
+__device__ __forceinline__ void store_group(void* out, uint64_t idx, const uint32_t (&e)[8],
+                                            uint64_t raw8) {
+  if (DT == kDtBf16Split) {
     uint32_t o[4];
     fmt_bf16_split(e, raw8, o);
     *reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + idx) = make_uint4(o[0], o[1], o[2], o[3]);
-  } else if (dtype == kDtInt4) {
+  } else if (DT == kDtInt4) {
     uint32_t w = 0;
 #pragma unroll
     for (int k = 0; k < 8; ++k) w |= (((e[k] >> 12) ^ 8u) & 0xFu) << (4 * k);
@@ -41,6 +42,7 @@ __device__ __forceinline__ void store_group(uint32_t dtype, void* out, uint64_t 
   }
 }
 
+template <uint32_t DT>
 __global__ void __launch_bounds__(kDecMaxWarps * 32, 2)
     decode_tiles_kernel(const __grid_constant__ LayerDev L, void* __restrict__ out,
                         uint32_t* __restrict__ status) {
@@ -54,6 +56,7 @@ __global__ void __launch_bounds__(kDecMaxWarps * 32, 2)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kDecLutBytes + kRingBytes + kDecMaxWarps * kRingBytes);
   const uint32_t warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const bool single = L.single_symbol != kNoSymbol;
+  const uint32_t single_e = L.single_symbol << 12;
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
@@ -66,15 +69,17 @@ __global__ void __launch_bounds__(kDecMaxWarps * 32, 2)
   volatile uint32_t* abort = &abort_flag;
   const uint32_t lt = lanemask_lt();
   const uint32_t lut_s = smem_u32(lut);
-  TileSeq seq{blockIdx.x * nwarps + warp, gridDim.x * nwarps, L.n_tiles, L.n_tiles};
+  const uint32_t n_tiles = L.n_tiles, n_kt = L.n_kt, K = L.K;
+  const uint32_t tile_n = L.tile_n, tile_k = L.tile_k;
+  const uint32_t H = tile_n / 128, C = tile_k / 16;
+  const uint32_t S = tile_n * tile_k;
+  const uint8_t* raw = L.raw;
+  TileSeq seq{blockIdx.x * nwarps + warp, gridDim.x * nwarps, n_tiles, n_tiles};
   ChunkPipe pipe;
   pipe_init(pipe, rings + warp * kRingBytes, bars + warp * 4);
-  const uint32_t H = L.tile_n / 128;
-  const uint32_t groups = L.tile_n * L.tile_k / 256;
-  const uint32_t S = L.tile_n * L.tile_k;
-  const bool bf16 = L.dtype == kDtBf16Split;
   TileCursor tc;
   tc.cb = 0;
+  const uint64_t row_step = 32ull * K;  // next row of the same lane
 
   for (uint32_t r = 0; seq.has(r); ++r) {
     const uint32_t t = seq.at(r);
@@ -82,36 +87,44 @@ __global__ void __launch_bounds__(kDecMaxWarps * 32, 2)
       if (lane == 0) atomicOr(status, kStatusBadOffsets);
       continue;
     }
-    const uint32_t n0 = (t / L.n_kt) * L.tile_n, k0 = (t % L.n_kt) * L.tile_k;
-    const uint64_t base = static_cast<uint64_t>(n0 + lane) * L.K + k0;
+    const uint32_t rb = t / n_kt, kt = t - rb * n_kt;
+    const uint64_t base = static_cast<uint64_t>(rb * tile_n + lane) * K + kt * tile_k;
     const unsigned long long* raw_tile =
-        reinterpret_cast<const unsigned long long*>(L.raw + static_cast<uint64_t>(t) * S) + lane;
+        reinterpret_cast<const unsigned long long*>(raw + static_cast<uint64_t>(t) * S) + lane;
+    const uint32_t groups = S / 256;
     // raw bytes of groups g, g+1, g+2 in flight
     uint64_t r0 = 0, r1 = 0, r2 = 0;
-    if (bf16) {
+    if (DT == kDtBf16Split) {
       r0 = __ldg(raw_tile);
-      if (groups > 1) r1 = __ldg(raw_tile + 32);
-      if (groups > 2) r2 = __ldg(raw_tile + 64);
+      r1 = __ldg(raw_tile + 32);
+      r2 = __ldg(raw_tile + 64);
     }
-    for (uint32_t g = 0; g < groups; ++g) {
-      const uint64_t raw8 = r0;
-      if (bf16) {
-        r0 = r1;
-        r1 = r2;
-        if (g + 3 < groups) r2 = __ldg(raw_tile + 32 * (g + 3));
-      }
-      uint32_t e[8];
-      if (single) {
+    uint32_t g = 0;
+    // group order (slab s, half h, chunk c, row i) matches the stream's lane map
+    for (uint32_t s = 0; s < C; ++s) {
+      for (uint32_t h = 0; h < H; ++h) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) e[k] = L.single_symbol << 12;
-      } else {
-        tile_group(pipe, L, seq, tc, lane, abort, status);
+        for (uint32_t ci = 0; ci < 8; ++ci, ++g) {
+          const uint32_t c = ci >> 2, i = ci & 3;
+          const uint64_t raw8 = r0;
+          if (DT == kDtBf16Split) {
+            r0 = r1;
+            r1 = r2;
+            if (g + 3 < groups) r2 = __ldg(raw_tile + 32 * (g + 3));
+          }
+          uint32_t e[8];
+          if (single) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) e[k] = decode_step(tc.x, tc.pos, lut_s, pipe.ring_s, lt);
+            for (int k = 0; k < 8; ++k) e[k] = single_e;
+          } else {
+            tile_group(pipe, L, seq, tc, lane, abort, status);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) e[k] = decode_step(tc.x, tc.pos, lut_s, pipe.ring_s, lt);
+          }
+          const uint64_t idx = base + (4 * h + i) * row_step + 16 * s + 8 * c;
+          store_group<DT>(out, idx, e, raw8);
+        }
       }
-      const uint32_t i = g & 3, c = (g >> 2) & 1, h = (g >> 3) % H, s = g / (8 * H);
-      const uint64_t idx = base + static_cast<uint64_t>(32 * (4 * h + i)) * L.K + 16 * s + 8 * c;
-      store_group(L.dtype, out, idx, e, raw8);
     }
     if (!tile_end(tc, single) && lane == 0) atomicOr(status, kStatusCorrupt);
   }
@@ -173,11 +186,18 @@ __global__ void __launch_bounds__(kHistWarps * 32)
   }
 }
 
-cudaError_t launch_decode_tiles(const LayerDev& L, void* out, uint32_t* status,
-                                cudaStream_t stream, int num_sms) {
-  cudaError_t e = cudaFuncSetAttribute(decode_tiles_kernel,
+template <uint32_t DT>
+static cudaError_t launch_decode_variant(const LayerDev& L, void* out, uint32_t* status,
+                                         cudaStream_t stream, uint32_t blocks, uint32_t warps) {
+  cudaError_t e = cudaFuncSetAttribute(decode_tiles_kernel<DT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem);
   if (e != cudaSuccess) return e;
+  decode_tiles_kernel<DT><<<blocks, warps * 32, kDecSmem, stream>>>(L, out, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_tiles(const LayerDev& L, void* out, uint32_t* status,
+                                cudaStream_t stream, int num_sms) {
   if (L.n_tiles == 0) return cudaSuccess;
   // One warp decodes one tile at a time, so the tiles are the unit of
   // parallelism: spread them evenly, up to 2 blocks x 16 warps per SM.
@@ -187,8 +207,9 @@ cudaError_t launch_decode_tiles(const LayerDev& L, void* out, uint32_t* status,
   if (warps < 1) warps = 1;
   uint32_t blocks = (L.n_tiles + warps - 1) / warps;
   if (blocks > 2 * sms) blocks = 2 * sms;
-  decode_tiles_kernel<<<blocks, warps * 32, kDecSmem, stream>>>(L, out, status);
-  return cudaGetLastError();
+  if (L.dtype == kDtBf16Split) return launch_decode_variant<kDtBf16Split>(L, out, status, stream, blocks, warps);
+  if (L.dtype == kDtInt4) return launch_decode_variant<kDtInt4>(L, out, status, stream, blocks, warps);
+  return launch_decode_variant<kDtFp8>(L, out, status, stream, blocks, warps);
 }
 
 cudaError_t launch_histogram(const void* w, uint64_t n_bytes, uint32_t dtype, uint64_t* hist,

@@ -243,6 +243,14 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
       for (uint32_t us = 0; us < n_slabs; ++us) {
         const uint32_t h = us % H, s = us / H;
         const uint32_t slot = sc & 1u;
+        // group scales of this lane's four rows in half h (int4 x group scale)
+        __half2 gs0, gs1, gs2, gs3;
+        if (kFmt == kFmtInt4F16Group) {
+          gs0 = h ? gscale[4] : gscale[0];
+          gs1 = h ? gscale[5] : gscale[1];
+          gs2 = h ? gscale[6] : gscale[2];
+          gs3 = h ? gscale[7] : gscale[3];
+        }
         // copy mode: fetch the slab's 8 groups before waiting for the slot
         uint4 cp[8];
         if (!kDecode) {
@@ -262,7 +270,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
             }
           }
         }
-        if (sc >= 2) wait_live(&B.w_empty[2 * d + slot], ((sc >> 1) + 1) & 1u, abort, P.status, 1);
+        if (sc >= 2) wait_live(&B.w_empty[2 * d + slot], ((sc >> 1) + 1) & 1u, abort, P.status, 1, 64);
         const uint32_t slab_s = wslots_s + slot * kSlabBytes;
 #pragma unroll 1
         for (uint32_t gg = 0; gg < 8; ++gg) {
@@ -290,7 +298,8 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
             }
             if (kFmt == kFmtBf16Split) fmt_bf16_split(e, raw8, o);
             else if (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
-            else if (kFmt == kFmtInt4F16Group) fmt_int4_f16_scaled(e, gscale[4 * h + i], o);
+            else if (kFmt == kFmtInt4F16Group)
+              fmt_int4_f16_scaled(e, i == 0 ? gs0 : i == 1 ? gs1 : i == 2 ? gs2 : gs3, o);
             else fmt_fp8_f16(e, o);
             if (zero_tile) o[0] = o[1] = o[2] = o[3] = 0;
           } else {
@@ -313,7 +322,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
 #pragma unroll
                 for (int k = 0; k < 8; ++k) e[k] = (((v.x >> (4 * k)) & 0xFu) ^ 8u) << 12;
                 if (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
-                else fmt_int4_f16_scaled(e, gscale[4 * h + i], o);
+                else fmt_int4_f16_scaled(e, i == 0 ? gs0 : i == 1 ? gs1 : i == 2 ? gs2 : gs3, o);
               }
             }
           }
@@ -338,44 +347,60 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     // ======================= MMA issue (one thread) =======================
     if (lane == 0) {
       const uint32_t ub = static_cast<uint32_t>(u_begin), ue = static_cast<uint32_t>(u_end);
+      const uint32_t seg_begin = ub / n_kt;
+      // descriptor fields shared by every operand: LBO 16 B, SBO 256 B,
+      // version 1, 32-byte swizzle; only the start address varies
+      const uint64_t dhi = (1ull << 16) | (16ull << 32) | (1ull << 46) | (6ull << 61);
+      const uint32_t a_base = smem_u32(wring) >> 4, x_base = smem_u32(xring) >> 4;
+      const uint32_t slab16 = kSlabBytes >> 4, xstage16 = x_stage_bytes >> 4, t16 = (P.T * 32) >> 4;
       uint32_t fresh = 0;  // bit (buf * 2 + h): next MMA into that accumulator starts it
-      uint32_t xc = 0;
-      uint32_t nstep = 0;
-      for_each_mma_step(P, ub, ue, [&](uint32_t u, uint32_t s, uint32_t d, uint32_t r,
-                                       const UnitInfo& I) {
-        const uint32_t lseg = I.lseg;
-        const uint32_t buf = P.n_bufs == 2 ? (lseg & 1u) : 0u;
-        if (s == 0 && I.seg_first) {
-          const uint32_t k = P.n_bufs == 2 ? (lseg >> 1) : lseg;
-          if (k >= 1) wait_live(&B.acc_empty[buf], (k - 1) & 1u, abort, P.status, 4);
-          tc_fence_after();
-          fresh |= 3u << (2 * buf);
-        }
-        const uint32_t xs = xc % XS;
-        wait_live(&B.x_full[xs], (xc / XS) & 1u, abort, P.status, 2);
-        for (uint32_t h = 0; h < P.H; ++h) {
-          const uint32_t idx = (r * P.C + s) * P.H + h;
-          const uint32_t slot = idx & 1u;
-          wait_live(&B.w_full[2 * d + slot], (idx >> 1) & 1u, abort, P.status, 3);
-          tc_fence_after();
-          const uint32_t a_addr = smem_u32(wring + (2 * d + slot) * kSlabBytes);
-          const uint64_t adesc = sdesc_sw32(a_addr, 256);
-          const uint32_t acc_bit = 1u << (2 * buf + h);
-          const uint32_t accumulate = (fresh & acc_bit) ? 0u : 1u;
-          for (uint32_t j = 0; j < P.NT; ++j) {
-            const uint32_t b_addr = smem_u32(xring + xs * x_stage_bytes + j * P.T * 32);
-            const uint32_t col = ((buf * P.H + h) * P.NT + j) * P.T;
-            umma_f16(tmem_base + col, adesc, sdesc_sw32(b_addr, 256), P.idesc, accumulate);
+      uint32_t xs = 0, xpar = 0;
+      uint32_t r = 0;
+      for (uint32_t u0 = ub; u0 < ue; u0 += D, ++r) {
+        const uint32_t nd = min(D, ue - u0);
+        const uint32_t seg0 = u0 / n_kt, kt0 = u0 - seg0 * n_kt;
+        const uint32_t nA = P.n_bufs == 2 ? nd : min(nd, n_kt - kt0);
+        for (uint32_t part = 0; part < 2; ++part) {
+          const uint32_t d_lo = part == 0 ? 0 : nA, d_hi = part == 0 ? nA : nd;
+          for (uint32_t s = 0; s < P.C; ++s) {
+            for (uint32_t d = d_lo; d < d_hi; ++d) {
+              const uint32_t kt = kt0 + d;
+              const bool wrap = kt >= n_kt;
+              const uint32_t ktw = wrap ? kt - n_kt : kt;
+              const uint32_t lseg = seg0 + (wrap ? 1u : 0u) - seg_begin;
+              const uint32_t buf = P.n_bufs == 2 ? (lseg & 1u) : 0u;
+              if (s == 0 && (u0 + d == ub || ktw == 0)) {
+                const uint32_t k = P.n_bufs == 2 ? (lseg >> 1) : lseg;
+                if (k >= 1) wait_live(&B.acc_empty[buf], (k - 1) & 1u, abort, P.status, 4);
+                tc_fence_after();
+                fresh |= 3u << (2 * buf);
+              }
+              wait_live(&B.x_full[xs], xpar, abort, P.status, 2);
+              for (uint32_t h = 0; h < P.H; ++h) {
+                const uint32_t idx = (r * P.C + s) * P.H + h;
+                const uint32_t slot = idx & 1u;
+                wait_live(&B.w_full[2 * d + slot], (idx >> 1) & 1u, abort, P.status, 3);
+                tc_fence_after();
+                const uint64_t adesc = dhi | (a_base + (2 * d + slot) * slab16);
+                const uint32_t acc_bit = 1u << (2 * buf + h);
+                const uint32_t accumulate = (fresh & acc_bit) ? 0u : 1u;
+                for (uint32_t j = 0; j < P.NT; ++j) {
+                  const uint64_t bdesc = dhi | (x_base + xs * xstage16 + j * t16);
+                  const uint32_t col = ((buf * P.H + h) * P.NT + j) * P.T;
+                  umma_f16(tmem_base + col, adesc, bdesc, P.idesc, accumulate);
+                }
+                fresh &= ~acc_bit;
+                umma_commit(&B.w_empty[2 * d + slot]);
+              }
+              umma_commit(&B.x_empty[xs]);
+              if (++xs == XS) { xs = 0; xpar ^= 1u; }
+              if (s == P.C - 1 && (u0 + d + 1 == ue || ktw + 1 == n_kt))
+                umma_commit(&B.acc_full[buf]);
+            }
           }
-          fresh &= ~acc_bit;
-          umma_commit(&B.w_empty[2 * d + slot]);
+          if (P.n_bufs == 2) break;  // one part: the whole round slab-major
         }
-        umma_commit(&B.x_empty[xs]);
-        ++xc;
-        if (s == P.C - 1 && I.seg_last) umma_commit(&B.acc_full[buf]);
-        if (nstep < 16) trace_mark(P, 48 + nstep);
-        ++nstep;
-      });
+      }
       umma_commit(B.mma_done);
       trace_mark(P, 34);
     }
@@ -385,10 +410,15 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     if (lane == 0) {
       uint32_t xc = 0;
       uint32_t n_issued = 0;  // loads issued: steps [0, n_issued) (none after an abort)
+      long long xw = 0, xi = 0;
+      const long long xb = clock64();
       for_each_mma_step(P, static_cast<uint32_t>(u_begin), static_cast<uint32_t>(u_end),
                         [&](uint32_t, uint32_t s, uint32_t, uint32_t, const UnitInfo& I) {
         const uint32_t xs = xc % XS;
+        long long c0 = clock64();
         if (xc >= XS) wait_live(&B.x_empty[xs], ((xc / XS) + 1) & 1u, abort, P.status, 5);
+        xw += clock64() - c0;
+        c0 = clock64();
         const uint32_t p = I.p;
         const uint32_t kx = I.kt * P.L.tile_k + 16 * s;
         if (!*abort && n_issued == xc) {
@@ -400,8 +430,15 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
                    &B.x_full[xs]);
           n_issued = xc + 1;
         }
+        xi += clock64() - c0;
         ++xc;
       });
+      if (P.trace) {
+        P.trace[blockIdx.x * 64 + 53] = xw;
+        P.trace[blockIdx.x * 64 + 54] = xi;
+        P.trace[blockIdx.x * 64 + 55] = clock64() - xb;
+        P.trace[blockIdx.x * 64 + 56] = xc;
+      }
       trace_mark(P, 42);
       // drain: the last load issued into every stage must have landed
       const uint32_t first = n_issued > XS ? n_issued - XS : 0;
@@ -418,7 +455,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     for (uint64_t seg = seg_first; seg <= seg_last; ++seg) {
       const uint32_t lseg = static_cast<uint32_t>(seg - seg_first);
       const uint32_t buf = lseg % P.n_bufs;
-      wait_live(&B.acc_full[buf], (lseg / P.n_bufs) & 1u, abort, P.status, 6);
+      wait_live(&B.acc_full[buf], (lseg / P.n_bufs) & 1u, abort, P.status, 6, 256);
       tc_fence_after();
       if (e == 0 && lseg < 2) trace_mark(P, 36 + lseg);
       const uint32_t p = static_cast<uint32_t>(seg / P.n_rb);

@@ -44,8 +44,11 @@ enum : uint32_t { kDtInt4 = 0, kDtBf16Split = 1, kDtFp8 = 2 };
 // Abort-aware bounded wait.  Returns false if the wait ran out (then sets the
 // CTA's abort flag and the TIMEOUT status bit) or if the CTA already aborted.
 // site: which wait (diagnostic bit 8 + site is set next to TIMEOUT).
+// backoff_ns > 0: sleep between polls, for waiters off the critical path, so
+// that they leave issue slots to the warps that are doing the work.
 __device__ __forceinline__ bool wait_live(uint64_t* bar, uint32_t parity, volatile uint32_t* abort,
-                                          uint32_t* status, uint32_t site = 0) {
+                                          uint32_t* status, uint32_t site = 0,
+                                          uint32_t backoff_ns = 0) {
   if (mbar_try_wait(bar, parity)) return true;
   long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
@@ -55,6 +58,7 @@ __device__ __forceinline__ bool wait_live(uint64_t* bar, uint32_t parity, volati
       atomicOr(status, kStatusTimeout | (1u << (8 + site)));
       return false;
     }
+    if (backoff_ns) __nanosleep(backoff_ns);
   }
   return true;
 }
@@ -247,27 +251,59 @@ __device__ __forceinline__ bool tile_end(TileCursor& tc, bool single) {
 // entry of the decoded symbol.  Every lane loads the word at its prefix
 // position (all such addresses lie in one 64-byte window, so the extra loads
 // cost no extra shared-memory wavefront); lanes that need no word discard it.
-__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+// Slot-table load: the table is written once before the CTA barrier and then
+// only read, so the load is an ordinary (reorderable) one.
+__device__ __forceinline__ uint32_t lds_lut(uint32_t addr) {
   uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
   return v;
 }
-__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
+// Ring-word load: volatile so it stays after the chunk waits that precede it.
+__device__ __forceinline__ uint32_t lds_ring16(uint32_t addr) {
   unsigned short v;
-  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr) : "memory");
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
   return v;
 }
 
+// One decode step of the calling lane (see the file comment), as explicit
+// PTX: slot lookup, state update, ballot of the lanes that need a word,
+// prefix-count addressing into the ring, word merge by byte permute (valid
+// because a lane needing a word has x < 2^16), predicated select.  Every lane
+// loads the word at its prefix position: those addresses all fall in one
+// 64-byte window, so lanes that need no word cost no extra wavefront.
+// Returns the slot-table entry of the decoded symbol.
 __device__ __forceinline__ uint32_t decode_step(uint32_t& x, uint32_t& pos, uint32_t lut_s,
                                                 uint32_t ring_s, uint32_t lt) {
-  const uint32_t e = lds_u32(lut_s + ((x & (kSlots - 1)) << 2));
-  x = (e >> 20) * (x >> 12) + (e & 0xFFFu);
-  const bool need = x < kStateLow;
-  const uint32_t bal = __ballot_sync(0xFFFFFFFFu, need);
-  const uint32_t off = ((pos + 2u * __popc(bal & lt)) & (kRingBytes - 1)) + ring_s;
-  const uint32_t w = lds_u16(off);
-  x = need ? ((x << 16) | w) : x;
-  pos += 2u * __popc(bal);
+  uint32_t e;
+  asm volatile(
+      "{\n\t"
+      ".reg .pred p;\n\t"
+      ".reg .b32 a, q, f, b, bal, t, pre, cnt, off, w, xs;\n\t"
+      "and.b32 a, %0, 4095;\n\t"
+      "shl.b32 a, a, 2;\n\t"
+      "add.u32 a, a, %3;\n\t"
+      "ld.shared.u32 %2, [a];\n\t"
+      "shr.u32 q, %0, 12;\n\t"
+      "shr.u32 f, %2, 20;\n\t"
+      "and.b32 b, %2, 4095;\n\t"
+      "mad.lo.u32 %0, f, q, b;\n\t"
+      "setp.lt.u32 p, %0, 65536;\n\t"
+      "vote.sync.ballot.b32 bal, p, 0xffffffff;\n\t"
+      "and.b32 t, bal, %5;\n\t"
+      "popc.b32 pre, t;\n\t"
+      "popc.b32 cnt, bal;\n\t"
+      "shl.b32 pre, pre, 1;\n\t"
+      "add.u32 off, %1, pre;\n\t"
+      "and.b32 off, off, 2047;\n\t"
+      "add.u32 off, off, %4;\n\t"
+      "ld.shared.u16 w, [off];\n\t"
+      "prmt.b32 xs, w, %0, 0x5410;\n\t"
+      "selp.b32 %0, xs, %0, p;\n\t"
+      "shl.b32 cnt, cnt, 1;\n\t"
+      "add.u32 %1, %1, cnt;\n\t"
+      "}"
+      : "+r"(x), "+r"(pos), "=&r"(e)
+      : "r"(lut_s), "r"(ring_s), "r"(lt));
   return e;
 }
 
