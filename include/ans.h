@@ -206,6 +206,25 @@ ans_status ans_gemm(const uint16_t* d_X, uint32_t M, const ans_tiles* W,
                     float* d_Y, void* d_ws, size_t ws_bytes, uint32_t* d_status,
                     ans_stream_t stream);
 
+/* Allocation-free variant of ans_gemm (no counterpart in the paper; it exists
+ * for callers of this library that cannot call cudaMalloc: code that runs
+ * while a CUDA graph is being captured, plug-ins whose host framework owns all
+ * device memory, or latency-critical paths that may not take an allocation's
+ * implicit synchronisation).  Same arguments and result as ans_gemm, without
+ * the workspace: the scratch (split-K counters and partials, staged X) lives
+ * in a fixed 16 MiB device array inside the library, which every GPU that
+ * loads the library holds until the process exits.  A shape whose
+ * ans_gemm_workspace exceeds 16 MiB returns ANS_ERR_BUFFER_TOO_SMALL (text via
+ * ans_last_error).  The first call on a device looks the array's device
+ * address up (cudaGetSymbolAddress with that device current); make that first
+ * call before any stream capture.  Each call clears the split-K counters with
+ * a memset on `stream`; it never allocates.  All calls share the one array,
+ * which keeps the last call's contents: calls that overlap on the GPU (other
+ * streams, other threads) race and must be serialised by the caller. */
+ans_status ans_gemm_noalloc(const uint16_t* d_X, uint32_t M, const ans_tiles* W,
+                            ans_scale_kind scale_kind, const void* d_scales, uint32_t group_k,
+                            float* d_Y, uint32_t* d_status, ans_stream_t stream);
+
 /* The same kernel with the decoder warps replaced by a copy of the original
  * (uncompressed) weights d_W (format of layout->dtype, row-major N x K).
  * Bit-exact reference for ans_gemm and the uncompressed baseline. */

@@ -26,7 +26,7 @@ ALPHABET = {INT4: 16, BF16_SPLIT: 256, FP8_E4M3: 256}
 EXPORTS = ["ans_status_string", "ans_last_error", "ans_num_tiles", "ans_layout_check",
            "ans_histogram", "ans_histogram_host", "ans_entropy", "ans_build_codebook", "ans_encode_bound",
            "ans_encode_tiles", "ans_decode_tiles", "ans_gemm_workspace", "ans_gemm",
-           "ans_gemm_uncompressed"]
+           "ans_gemm_noalloc", "ans_gemm_uncompressed"]
 
 
 class AnsError(RuntimeError):
@@ -82,6 +82,7 @@ def load():
             L.ans_decode_tiles.argtypes = [P, P, P, P]
             L.ans_gemm_workspace.argtypes = [P, u32, i32, P]
             L.ans_gemm.argtypes = [P, u32, P, i32, P, u32, P, P, sz, P, P]
+            L.ans_gemm_noalloc.argtypes = [P, u32, P, i32, P, u32, P, P, P]
             L.ans_gemm_uncompressed.argtypes = [P, u32, P, P, i32, P, u32, P, P, sz, P, P]
             for name in EXPORTS:
                 if name not in ("ans_status_string", "ans_last_error", "ans_num_tiles"):
@@ -203,6 +204,14 @@ def ans_gemm(d_X, M: int, tiles: AnsTiles, scale_kind: int, d_scales, group_k: i
     _check(load().ans_gemm(_ptr(d_X), M, C.byref(tiles), scale_kind, _ptr(d_scales), group_k,
                            _ptr(d_Y), _ptr(d_ws), ws_bytes, _ptr(d_status), _stream(stream)),
            "ans_gemm")
+
+
+def ans_gemm_noalloc(d_X, M: int, tiles: AnsTiles, scale_kind: int, d_scales, group_k: int, d_Y,
+                     d_status, stream=None):
+    """ans_gemm without a caller workspace (scratch inside the library)."""
+    _check(load().ans_gemm_noalloc(_ptr(d_X), M, C.byref(tiles), scale_kind, _ptr(d_scales),
+                                   group_k, _ptr(d_Y), _ptr(d_status), _stream(stream)),
+           "ans_gemm_noalloc")
 
 
 def ans_gemm_uncompressed(d_X, M: int, d_W, layout: AnsLayout, scale_kind: int, d_scales,

@@ -329,6 +329,41 @@ ans_status ans_gemm_uncompressed(const uint16_t* d_X, uint32_t M, const void* d_
                   d_status, stream);
 }
 
+ans_status ans_gemm_noalloc(const uint16_t* d_X, uint32_t M, const ans_tiles* W,
+                            ans_scale_kind scale_kind, const void* d_scales, uint32_t group_k,
+                            float* d_Y, uint32_t* d_status, ans_stream_t stream) {
+  if (!W) return ANS_ERR_ARG;
+  if (M == 0) return ANS_OK;
+  ans_status st = check_layout(&W->layout);
+  if (st != ANS_OK) return st;
+  size_t need = 0;
+  st = ans_gemm_workspace(&W->layout, M, scale_kind, &need);
+  if (st != ANS_OK) return st;
+  if (need > ansdev::kNoAllocScratchBytes) {
+    std::snprintf(g_last_error, sizeof(g_last_error),
+                  "ans_gemm_noalloc: this shape needs %zu bytes of scratch, above the fixed "
+                  "%zu-byte maximum; use ans_gemm with a caller workspace",
+                  need, ansdev::kNoAllocScratchBytes);
+    return ANS_ERR_BUFFER_TOO_SMALL;
+  }
+  void* scratch = nullptr;
+  cudaError_t e = ansdev::noalloc_scratch(&scratch);
+  if (e != cudaSuccess) return cuda_fail(e, "ans_gemm_noalloc scratch");
+  // the split-K counters must start at zero: clear them on the caller's stream
+  // (a memset, not an allocation)
+  ansdev::LayerDev L;
+  fill_layer_plain(&W->layout, &L);
+  ansdev::GemmPlan plan;
+  int sms = 0;
+  st = device_info(&sms);
+  if (st != ANS_OK) return st;
+  if (!ansdev::make_gemm_plan(L, M, scale_kind, true, sms, &plan)) return ANS_ERR_UNSUPPORTED;
+  e = cudaMemsetAsync(scratch, 0, plan.ws_counters_bytes, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "ans_gemm_noalloc clear");
+  return ans_gemm(d_X, M, W, scale_kind, d_scales, group_k, d_Y, scratch,
+                  ansdev::kNoAllocScratchBytes, d_status, stream);
+}
+
 // Internal profiling hook (not part of the public ABI in include/ans.h).
 void ansdev_set_trace(void* d_buf, size_t bytes) { ansdev::set_trace_buffer(d_buf, bytes); }
 

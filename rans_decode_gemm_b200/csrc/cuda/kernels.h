@@ -73,6 +73,12 @@ struct GemmDev {
 // stamps of its phases to trace[cta * 64 + slot].
 void set_trace_buffer(void* d_buf, size_t bytes);
 
+// Scratch capacity of the allocation-free entry point (16 MiB per device).
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
+// Device address of that scratch on the current device (looked up once per
+// device; see noalloc.cu).
+cudaError_t noalloc_scratch(void** ptr);
+
 // Fills a plan; returns false if the shape cannot be scheduled.
 bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool decode,
                     int num_sms, GemmPlan* plan);
