@@ -28,16 +28,15 @@
 #include <cstdlib>
 #include <cstring>
 
+#include "gemm_common.cuh"
 #include "kernels.h"
 #include "rans_core.cuh"
 
 namespace ansdev {
 
-constexpr uint32_t kSlabBytes = 128 * 32;  // 128 rows x 16 bf16
 constexpr uint32_t kFixedWarps = 6;
 constexpr uint32_t kMaxProducers = 16;
 constexpr uint32_t kMaxThreads = (kFixedWarps + kMaxProducers) * 32;
-constexpr uint32_t kSmemLimit = 232448 - 4096;  // sm_100 per-block maximum, less static smem
 
 struct Bars {
   uint64_t *w_full, *w_empty, *x_full, *x_empty, *acc_full, *acc_empty, *mma_done, *chunk;
@@ -59,18 +58,6 @@ __device__ __forceinline__ Bars carve_bars(uint8_t* base, uint32_t D, uint32_t X
 
 __host__ __device__ inline uint32_t num_bars(uint32_t D, uint32_t XS) {
   return 4 * D + 2 * XS + 5 + 4 * D;
-}
-
-__device__ __forceinline__ uint64_t cta_begin(uint64_t U, uint32_t G, uint32_t c) {
-  return U * c / G;
-}
-
-// CTA whose range contains unit u.
-__device__ __forceinline__ uint32_t cta_of(uint64_t U, uint32_t G, uint64_t u) {
-  uint32_t c = static_cast<uint32_t>(u * G / U);
-  while (c + 1 < G && cta_begin(U, G, c + 1) <= u) ++c;
-  while (c > 0 && cta_begin(U, G, c) > u) --c;
-  return c;
 }
 
 // Where a unit sits: K tile, token pass and W row-block segment, plus
@@ -124,22 +111,6 @@ __device__ __forceinline__ void for_each_mma_step(const GemmDev& P, uint32_t u_b
   }
 }
 
-__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void trace_mark(const GemmDev& P, uint32_t slot) {
-  if (P.trace) {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    P.trace[blockIdx.x * 64 + slot] = t;
-  }
-}
-
-__device__ __forceinline__ float bf16_to_f32(uint16_t b) {
-  return __uint_as_float(static_cast<uint32_t>(b) << 16);
-}
-
 // ---------------------------------------------------------------------------
 template <bool kDecode, uint32_t kFmt>
 __global__ void __launch_bounds__(kMaxThreads, 1)
@@ -152,8 +123,8 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
   const uint32_t warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t D = P.D, XS = P.x_stages;
   const uint32_t G = gridDim.x;
-  const uint64_t u_begin = cta_begin(P.n_units, G, blockIdx.x);
-  const uint64_t u_end = cta_begin(P.n_units, G, blockIdx.x + 1);
+  const uint32_t u_begin = cta_begin(static_cast<uint32_t>(P.n_units), G, blockIdx.x);
+  const uint32_t u_end = cta_begin(static_cast<uint32_t>(P.n_units), G, blockIdx.x + 1);
   const uint32_t n_kt = P.L.n_kt;
 
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem + P.off_lut);
@@ -450,9 +421,8 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
   } else {
     // ======================= epilogue (warps 0-3, 128 threads) =======================
     const uint32_t e = threadIdx.x;  // TMEM lane = row within the 128-row half
-    const uint64_t seg_first = u_begin / n_kt, seg_last = (u_end - 1) / n_kt;
-    const uint32_t N = P.L.N;
-    for (uint64_t seg = seg_first; seg <= seg_last; ++seg) {
+    const uint32_t seg_first = u_begin / n_kt, seg_last = (u_end - 1) / n_kt;
+    for (uint32_t seg = seg_first; seg <= seg_last; ++seg) {
       const uint32_t lseg = static_cast<uint32_t>(seg - seg_first);
       const uint32_t buf = lseg % P.n_bufs;
       wait_live(&B.acc_full[buf], (lseg / P.n_bufs) & 1u, abort, P.status, 6, 256);
@@ -460,89 +430,30 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
       if (e == 0 && lseg < 2) trace_mark(P, 36 + lseg);
       const uint32_t p = static_cast<uint32_t>(seg / P.n_rb);
       const uint32_t rb = static_cast<uint32_t>(seg % P.n_rb);
-      const uint64_t s_lo = seg * n_kt, s_hi = s_lo + n_kt;
+      const uint32_t s_lo = seg * n_kt, s_hi = s_lo + n_kt;
       const bool complete = u_begin <= s_lo && u_end >= s_hi;
       const uint32_t slot = (seg == seg_first) ? 0u : 1u;
       float* part = P.partials + (static_cast<uint64_t>(blockIdx.x) * 2 + slot) * P.H * P.T_pass * 128;
       for (uint32_t h = 0; h < P.H; ++h) {
         const uint32_t n = rb * P.L.tile_n + h * 128 + e;
-        float scale = 1.0f;
-        if (complete) {
-          if (P.scale_kind == 1) scale = bf16_to_f32(__ldg(static_cast<const uint16_t*>(P.scales) + n));
-          else if (P.scale_kind == 2) scale = __ldg(static_cast<const float*>(P.scales) + n);
-        }
+        const float scale = complete ? row_scale(P, n) : 1.0f;
         for (uint32_t j = 0; j < P.NT; ++j) {
           const uint32_t col0 = ((buf * P.H + h) * P.NT + j) * P.T;
           for (uint32_t cc = 0; cc < P.T; cc += 16) {
             uint32_t v[16];
             tmem_ld16(tmem_base + ((32 * warp) << 16) + col0 + cc, v);
             tmem_ld_wait();
-            const uint32_t tok0 = j * P.T + cc;
+            float f[16];
 #pragma unroll
-            for (int q = 0; q < 16; ++q) {
-              const uint32_t m = p * P.T_pass + tok0 + q;
-              const float a = __uint_as_float(v[q]);
-              if (complete) {
-                if (m < P.M) P.Y[static_cast<uint64_t>(m) * N + n] = a * scale;
-              } else {
-                part[(static_cast<uint64_t>(h) * P.T_pass + tok0 + q) * 128 + e] = a;
-              }
-            }
+            for (int q = 0; q < 16; ++q) f[q] = __uint_as_float(v[q]);
+            epi_emit16(P, f, complete, scale, part, p, h, j * P.T + cc, n, e);
           }
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&B.acc_empty[buf]);
-      if (!complete) {
-        // split-K: the last CTA to finish this segment reduces it in CTA order
-        __threadfence();
-        named_bar_sync(1, 128);
-        const uint32_t c_first = cta_of(P.n_units, G, s_lo);
-        const uint32_t c_last = cta_of(P.n_units, G, s_hi - 1);
-        if (e == 0) {
-          uint32_t old = atomicAdd(&P.counters[seg], 1u);
-          reduce_flag = (old == c_last - c_first) ? 1u : 0u;
-        }
-        named_bar_sync(1, 128);
-        if (reduce_flag) {
-          __threadfence();
-          // contributors c_first..c_last; only c_first can hold this segment in
-          // its second (tail) slot, when its range started before the segment
-          const uint32_t sl_first = (cta_begin(P.n_units, G, c_first) < s_lo) ? 1u : 0u;
-          const uint64_t cta_stride = 2ull * P.H * P.T_pass * 128;
-          const uint32_t t_valid = min(P.T_pass, P.M - p * P.T_pass);
-          for (uint32_t h = 0; h < P.H; ++h) {
-            const uint32_t nh = rb * P.L.tile_n + h * 128;
-            for (uint32_t it = e; it < t_valid * 32; it += 128) {
-              const uint32_t tok = it >> 5, q = it & 31;
-              const uint64_t off = (static_cast<uint64_t>(h) * P.T_pass + tok) * 128 + 4 * q;
-              float4 acc = __ldcg(reinterpret_cast<const float4*>(
-                  P.partials + c_first * cta_stride + sl_first * (cta_stride / 2) + off));
-              for (uint32_t c2 = c_first + 1; c2 <= c_last; ++c2) {
-                const float4 v = __ldcg(reinterpret_cast<const float4*>(P.partials + c2 * cta_stride + off));
-                acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-              }
-              const uint32_t n = nh + 4 * q;
-              if (P.scale_kind == 1) {
-                const uint2 sb = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(P.scales) + n));
-                acc.x *= __uint_as_float(sb.x << 16);
-                acc.y *= __uint_as_float(sb.x & 0xFFFF0000u);
-                acc.z *= __uint_as_float(sb.y << 16);
-                acc.w *= __uint_as_float(sb.y & 0xFFFF0000u);
-              } else if (P.scale_kind == 2) {
-                const float4 sf = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(P.scales) + n));
-                acc.x *= sf.x; acc.y *= sf.y; acc.z *= sf.z; acc.w *= sf.w;
-              }
-              const uint32_t m = p * P.T_pass + tok;
-              *reinterpret_cast<float4*>(P.Y + static_cast<uint64_t>(m) * N + n) = acc;
-            }
-          }
-          if (e == 0) P.counters[seg] = 0;
-          if (e == 0) trace_mark(P, 38);
-        }
-        named_bar_sync(1, 128);
-      }
+      if (!complete) splitk_finish(P, seg, p, rb, e, &reduce_flag);
     }
   }
 
@@ -602,8 +513,28 @@ void set_trace_buffer(void* d_buf, size_t bytes) {
   g_trace = bytes >= 64 * sizeof(unsigned long long) ? static_cast<unsigned long long*>(d_buf) : nullptr;
 }
 
+// Accumulator slots the local schedule needs in the busiest CTA: one per
+// (producer warp, W row-block segment) pair that holds units.
+static uint32_t local_slots(uint32_t U, uint32_t G, uint32_t D, uint32_t n_kt) {
+  uint32_t mx = 0;
+  for (uint32_t c = 0; c < G; ++c) {
+    const uint32_t ub = cta_begin(U, G, c), ue = cta_begin(U, G, c + 1);
+    uint32_t cnt = 0;
+    for (uint32_t d = 0; d < D; ++d) {
+      const uint32_t b = ub + cta_begin(ue - ub, D, d), e = ub + cta_begin(ue - ub, D, d + 1);
+      if (e > b) cnt += (e - 1) / n_kt - b / n_kt + 1;
+    }
+    if (cnt > mx) mx = cnt;
+  }
+  return mx;
+}
+
+// The schedule (grid, producers, token passes) depends only on the shape, the
+// format and the device, never on whether the weights arrive compressed, so
+// ans_gemm and ans_gemm_uncompressed add the same products in the same order.
 bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool decode, int num_sms,
                     GemmPlan* plan) {
+  (void)decode;
   GemmPlan p;
   std::memset(&p, 0, sizeof(p));
   if (L.dtype == 1) p.fmt = kFmtBf16Split;
@@ -614,6 +545,78 @@ bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool dec
   p.H = L.tile_n / 128;
   p.C = L.tile_k / 16;
   const uint32_t Mp = round_up(M < 1 ? 1 : M, 16);
+  uint64_t sms = num_sms > 0 ? static_cast<uint64_t>(num_sms) : 148;
+  // Tuning / testing knobs: cap the CTA count and the producer warps per CTA,
+  // force one of the two schedules.
+  if (const char* v = std::getenv("ANS_GEMM_MAX_CTAS")) {
+    long cap = std::strtol(v, nullptr, 10);
+    if (cap > 0 && static_cast<uint64_t>(cap) < sms) sms = static_cast<uint64_t>(cap);
+  }
+  uint32_t D_cap = kMaxProducers;
+  if (const char* v = std::getenv("ANS_GEMM_MAX_PRODUCERS")) {
+    long cap = std::strtol(v, nullptr, 10);
+    if (cap > 0 && static_cast<uint32_t>(cap) < D_cap) D_cap = static_cast<uint32_t>(cap);
+  }
+  // unit indices are 32-bit in the kernels
+  if (static_cast<uint64_t>(L.n_tiles) * ((M + 15) / 16) >= (1ull << 31)) return false;
+  bool want_local = p.H * Mp <= 32;
+  if (const char* v = std::getenv("ANS_GEMM_SCHEDULE")) {
+    if (std::strcmp(v, "central") == 0) want_local = false;
+  }
+  const uint32_t lut_bytes = kSlots * 4;
+
+  if (want_local) {
+    // ---- local schedule: every producer issues its own MMAs (gemm_local.cu)
+    p.T = p.T_pass = Mp;
+    p.NT = 1;
+    p.n_pass = 1;
+    p.n_bufs = 1;
+    p.n_units = L.n_tiles;
+    p.n_segments = L.N / L.tile_n;
+    p.grid = static_cast<uint32_t>(p.n_units < sms ? p.n_units : sms);
+    const uint64_t per_cta = (p.n_units + p.grid - 1) / p.grid;
+    uint32_t D = D_cap;
+    if (D > per_cta) D = static_cast<uint32_t>(per_cta);
+    for (; D >= 1; --D) {
+      const uint32_t slots = local_slots(static_cast<uint32_t>(p.n_units), p.grid, D, L.n_kt);
+      const uint32_t cols = slots * p.H * p.T;
+      uint32_t off = lut_bytes;
+      off = round_up(off, 1024);
+      const uint32_t off_w = off;
+      off += D * kSlabBytes;
+      off = round_up(off, 2048);
+      const uint32_t off_chunk = off;
+      off += (D + 1) * kRingBytes;
+      off = round_up(off, 1024);
+      const uint32_t off_x = off;
+      off += D * p.T * 32;
+      off = round_up(off, 8);
+      const uint32_t off_bars = off;
+      off += (5 * D + slots) * 8;
+      if (cols <= 512 && off <= kSmemLimit) {
+        p.local = 1;
+        p.D = D;
+        p.n_slots = slots;
+        p.tmem_cols = 32;
+        while (p.tmem_cols < cols) p.tmem_cols <<= 1;
+        p.off_lut = 0;
+        p.off_w = off_w;
+        p.off_chunk = off_chunk;
+        p.off_x = off_x;
+        p.off_bars = off_bars;
+        p.smem_bytes = off;
+        p.ws_partials_bytes = static_cast<size_t>(p.grid) * 2 * p.H * p.T_pass * 128 * sizeof(float);
+        p.ws_counters_bytes = round_up(p.n_segments * 4, 256);
+        p.ws_x16_bytes = 0;
+        p.ws_bytes = p.ws_counters_bytes + (p.ws_partials_bytes + 255) / 256 * 256;
+        *plan = p;
+        return true;
+      }
+    }
+    // no fit: fall through to the shared-accumulator schedule
+  }
+
+  // ---- shared-accumulator schedule: one MMA-issuing thread per CTA
   const uint32_t max_cols = 512;
   if (2 * p.H * Mp <= max_cols) {
     p.n_bufs = 2;
@@ -637,23 +640,12 @@ bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool dec
 
   p.n_units = static_cast<uint64_t>(p.n_pass) * L.n_tiles;
   p.n_segments = p.n_pass * (L.N / L.tile_n);
-  uint64_t sms = num_sms > 0 ? static_cast<uint64_t>(num_sms) : 148;
-  // Tuning / testing knobs: cap the CTA count and the producer warps per CTA.
-  if (const char* v = std::getenv("ANS_GEMM_MAX_CTAS")) {
-    long cap = std::strtol(v, nullptr, 10);
-    if (cap > 0 && static_cast<uint64_t>(cap) < sms) sms = static_cast<uint64_t>(cap);
-  }
   p.grid = static_cast<uint32_t>(p.n_units < sms ? p.n_units : sms);
   uint64_t per_cta = (p.n_units + p.grid - 1) / p.grid;
 
   // shared memory: [lut][w rings][chunk rings][x stages][barriers]
   const uint32_t x_stage = p.T_pass * 32;
-  const uint32_t lut_bytes = decode ? kSlots * 4 : 0;
-  uint32_t D = kMaxProducers;
-  if (const char* v = std::getenv("ANS_GEMM_MAX_PRODUCERS")) {
-    long cap = std::strtol(v, nullptr, 10);
-    if (cap > 0 && static_cast<uint32_t>(cap) < D) D = static_cast<uint32_t>(cap);
-  }
+  uint32_t D = D_cap;
   if (D > L.n_kt) D = L.n_kt;
   if (D > per_cta) D = static_cast<uint32_t>(per_cta);
   // X stages take whatever shared memory the producers leave (deep rings keep
@@ -666,7 +658,7 @@ bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool dec
     off += D * 2 * kSlabBytes;
     off = round_up(off, 2048);
     const uint32_t off_chunk = off;
-    off += decode ? (D + 1) * kRingBytes : 0;
+    off += (D + 1) * kRingBytes;
     off = round_up(off, 1024);
     const uint32_t off_x = off;
     const uint32_t bars_max = num_bars(D, 64) * 8;
@@ -728,7 +720,7 @@ cudaError_t launch_gemm(const GemmPlan& plan, const LayerDev& L, bool decode, co
   float* partials = reinterpret_cast<float*>(wsb + plan.ws_counters_bytes);
   uint16_t* x16 = reinterpret_cast<uint16_t*>(wsb + plan.ws_counters_bytes +
                                               ((plan.ws_partials_bytes + 255) / 256) * 256);
-  {
+  if (!plan.local) {
     const uint64_t n_chunks = static_cast<uint64_t>(plan.n_pass) * (L.K / 16) * plan.T_pass * 2;
     uint32_t blocks = static_cast<uint32_t>((n_chunks + 255) / 256);
     if (blocks > 4096) blocks = 4096;
@@ -772,6 +764,10 @@ cudaError_t launch_gemm(const GemmPlan& plan, const LayerDev& L, bool decode, co
   P.off_bars = plan.off_bars;
   P.trace = g_trace;
   P.xs = reinterpret_cast<const uint8_t*>(x16);
+  P.X = X;
+  P.x_f16 = plan.ab_f16;
+  P.n_slots = plan.n_slots;
+  if (plan.local) return launch_gemm_local(plan, P, decode, stream);
 
   switch (plan.fmt | (decode ? 0u : 8u)) {
     case kFmtBf16Split: return launch_variant<true, kFmtBf16Split>(plan, P, stream);

@@ -1,0 +1,162 @@
+// gemm_common.cuh -- pieces shared by the two schedules of the fused decode +
+// GEMM kernel (gemm.cu: one MMA-issuing thread per CTA feeding a shared
+// accumulator; gemm_local.cu: every producer warp issues its own MMAs into
+// private accumulators).  Unit ranges, the epilogue's output stores and the
+// deterministic split-K reduction live here.
+#pragma once
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "kernels.h"
+#include "rans_core.cuh"
+
+namespace ansdev {
+
+constexpr uint32_t kSlabBytes = 128 * 32;       // 128 rows x 16 bf16 (one MMA A operand)
+constexpr uint32_t kSmemLimit = 232448 - 4096;  // sm_100 per-block maximum, less static smem
+
+// Units (token pass, tile; fewer than 2^31) are split into one contiguous
+// range per CTA, the first U % G CTAs taking one unit more than the others.
+// 32-bit arithmetic only: 64-bit divisions are long software routines here.
+__host__ __device__ __forceinline__ uint32_t cta_begin(uint32_t U, uint32_t G, uint32_t c) {
+  const uint32_t q = U / G, r = U % G;
+  return q * c + (c < r ? c : r);
+}
+
+// CTA whose range contains unit u (G <= U, so q >= 1 past the longer ranges).
+__host__ __device__ __forceinline__ uint32_t cta_of(uint32_t U, uint32_t G, uint32_t u) {
+  const uint32_t q = U / G, r = U % G;
+  const uint32_t big = r * (q + 1);
+  return u < big ? u / (q + 1) : r + (u - big) / q;
+}
+
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void trace_mark(const GemmDev& P, uint32_t slot) {
+  if (P.trace) {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    P.trace[blockIdx.x * 64 + slot] = t;
+  }
+}
+
+__device__ __forceinline__ float bf16_to_f32(uint16_t b) {
+  return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+// Per-row output scale (row n of W), 1 when the format has none or applies
+// it before the MMA.
+__device__ __forceinline__ float row_scale(const GemmDev& P, uint32_t n) {
+  if (P.scale_kind == 1) return bf16_to_f32(__ldg(static_cast<const uint16_t*>(P.scales) + n));
+  if (P.scale_kind == 2) return __ldg(static_cast<const float*>(P.scales) + n);
+  return 1.0f;
+}
+
+// Epilogue output of 16 accumulator columns (tokens tok0 .. tok0 + 15 of
+// token pass p) for W row n = rb * tile_n + h * 128 + e.  A segment that this
+// CTA holds completely goes to Y (scaled); otherwise the values go to this
+// CTA's partial-sum slot for the split-K reduction.
+__device__ __forceinline__ void epi_emit16(const GemmDev& P, const float (&v)[16], bool complete,
+                                           float scale, float* part, uint32_t p, uint32_t h,
+                                           uint32_t tok0, uint32_t n, uint32_t e) {
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    const uint32_t m = p * P.T_pass + tok0 + q;
+    if (complete) {
+      if (m < P.M) P.Y[static_cast<uint64_t>(m) * P.L.N + n] = v[q] * scale;
+    } else {
+      part[(static_cast<uint64_t>(h) * P.T_pass + tok0 + q) * 128 + e] = v[q];
+    }
+  }
+}
+
+// Split-K over CTAs for segment seg (token pass p, W row block rb), run by
+// the 128 epilogue threads of every contributing CTA after its partials are
+// written: the last CTA to arrive sums the contributors' partials in
+// ascending CTA order (so the result does not depend on timing) and writes Y.
+// Only the first contributor can hold the segment in its second (tail)
+// partial slot, when its range started before the segment.
+__device__ __forceinline__ void splitk_finish(const GemmDev& P, uint32_t seg, uint32_t p,
+                                              uint32_t rb, uint32_t e,
+                                              volatile uint32_t* reduce_flag) {
+  const uint32_t G = gridDim.x, n_kt = P.L.n_kt, U = static_cast<uint32_t>(P.n_units);
+  const uint32_t s_lo = seg * n_kt, s_hi = s_lo + n_kt;
+  __threadfence();
+  named_bar_sync(1, 128);
+  const uint32_t c_first = cta_of(U, G, s_lo);
+  const uint32_t c_last = cta_of(U, G, s_hi - 1);
+  if (e == 0) {
+    const uint32_t old = atomicAdd(&P.counters[seg], 1u);
+    *reduce_flag = (old == c_last - c_first) ? 1u : 0u;
+  }
+  named_bar_sync(1, 128);
+  if (*reduce_flag) {
+    __threadfence();
+    const uint32_t sl_first = (cta_begin(U, G, c_first) < s_lo) ? 1u : 0u;
+    const uint64_t cta_stride = 2ull * P.H * P.T_pass * 128;
+    const uint32_t t_valid = min(P.T_pass, P.M - p * P.T_pass);
+    const uint32_t n_items = P.H * t_valid * 32;  // float4 items: (h, token, 4 rows)
+    const float* first = P.partials + c_first * cta_stride + sl_first * (cta_stride / 2);
+    for (uint32_t it0 = e; it0 < n_items; it0 += 4 * 128) {
+      uint64_t off[4];
+      float4 acc[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t it = min(it0 + 128u * u, n_items - 1);
+        const uint32_t q = it & 31, ht = it >> 5;
+        const uint32_t h = ht / t_valid, tok = ht - h * t_valid;
+        off[u] = (static_cast<uint64_t>(h) * P.T_pass + tok) * 128 + 4 * q;
+        acc[u] = __ldcg(reinterpret_cast<const float4*>(first + off[u]));
+      }
+      // the other contributors, two at a time with all their loads in flight
+      for (uint32_t c2 = c_first + 1; c2 <= c_last; c2 += 2) {
+        const uint32_t cb = min(c2 + 1, c_last);
+        float4 v0[4], v1[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          v0[u] = __ldcg(reinterpret_cast<const float4*>(P.partials + c2 * cta_stride + off[u]));
+          v1[u] = __ldcg(reinterpret_cast<const float4*>(P.partials + cb * cta_stride + off[u]));
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          acc[u].x += v0[u].x; acc[u].y += v0[u].y; acc[u].z += v0[u].z; acc[u].w += v0[u].w;
+        }
+        if (c2 + 1 <= c_last) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            acc[u].x += v1[u].x; acc[u].y += v1[u].y; acc[u].z += v1[u].z; acc[u].w += v1[u].w;
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t it = it0 + 128u * u;
+        if (it >= n_items) break;
+        const uint32_t q = it & 31, ht = it >> 5;
+        const uint32_t h = ht / t_valid, tok = ht - h * t_valid;
+        const uint32_t n = rb * P.L.tile_n + h * 128 + 4 * q;
+        float4 a = acc[u];
+        if (P.scale_kind == 1) {
+          const uint2 sb = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(P.scales) + n));
+          a.x *= __uint_as_float(sb.x << 16);
+          a.y *= __uint_as_float(sb.x & 0xFFFF0000u);
+          a.z *= __uint_as_float(sb.y << 16);
+          a.w *= __uint_as_float(sb.y & 0xFFFF0000u);
+        } else if (P.scale_kind == 2) {
+          const float4 sf = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(P.scales) + n));
+          a.x *= sf.x; a.y *= sf.y; a.z *= sf.z; a.w *= sf.w;
+        }
+        const uint32_t m = p * P.T_pass + tok;
+        *reinterpret_cast<float4*>(P.Y + static_cast<uint64_t>(m) * P.L.N + n) = a;
+      }
+    }
+    if (e == 0) P.counters[seg] = 0;
+    if (e == 0) trace_mark(P, 38);
+  }
+  named_bar_sync(1, 128);
+}
+
+}  // namespace ansdev

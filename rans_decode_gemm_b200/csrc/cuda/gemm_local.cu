@@ -1,0 +1,453 @@
+// gemm_local.cu -- fused tile-rANS decode + GEMM for small token counts
+// (M <= 32), where every producer warp drives the tensor core itself.
+//
+// "Approaching Shannon Bound with Lossless LLM Weight Compression", s3.1
+// "整体执行模型": decoder warps decode compressed tiles straight into shared
+// memory and the decoded tile is consumed there by the GEMM; decoding of the
+// next slab overlaps the MMA on the current one; buffers are released in an
+// order fixed by the traversal.
+//
+// Schedule (swap-AB, Y^T = W X^T, as in gemm.cu):
+//   * The units (tiles) are split into one contiguous range per CTA and,
+//     inside it, one contiguous sub-range per producer warp, so a producer
+//     streams one contiguous run of compressed bytes (RunPipe).
+//   * A producer decodes a 128 x 16 slab of W into its own shared-memory slot,
+//     writes the matching 16-column slab of X next to it, and its lane 0
+//     issues the tcgen05.mma into the producer's own TMEM accumulator; the
+//     MMA's completion (tcgen05.commit) frees the slots for the next slab.
+//   * A producer owns one accumulator per W row-block segment it touches, so
+//     an accumulator is written by one warp in a fixed order and read once;
+//     no warp waits for the epilogue.  The epilogue sums the accumulators of
+//     a segment in ascending unit order, then stores Y or takes part in the
+//     deterministic split-K reduction (gemm_common.cuh).  Every addition
+//     happens in an order fixed by the schedule, so Y is bit-identical to
+//     the same kernel fed uncompressed weights.
+// Warps: 0-3 epilogue (TMEM lanes 0-127), 4 .. 4 + D - 1 producers.
+#include <cuda_runtime.h>
+
+#include <cstring>
+
+#include "gemm_common.cuh"
+#include "kernels.h"
+#include "rans_core.cuh"
+
+namespace ansdev {
+
+constexpr uint32_t kLocalMaxProducers = 16;
+constexpr uint32_t kLocalThreads = (4 + kLocalMaxProducers) * 32;
+constexpr uint32_t kLocalMaxSlots = 32;  // 512 TMEM columns / (H * T >= 16) per accumulator
+
+// Contiguous sub-range of producer d inside the CTA's range [ub, ue) (the
+// same balanced split as the CTA ranges).
+__device__ __forceinline__ void producer_range(uint32_t ub, uint32_t ue, uint32_t D, uint32_t d,
+                                               uint32_t* b, uint32_t* e) {
+  *b = ub + cta_begin(ue - ub, D, d);
+  *e = ub + cta_begin(ue - ub, D, d + 1);
+}
+
+template <bool kDecode, uint32_t kFmt>
+__global__ void __launch_bounds__(kLocalThreads, 1)
+    fused_gemm_local_kernel(const __grid_constant__ GemmDev P) {
+  extern __shared__ __align__(2048) uint8_t smem[];
+  __shared__ uint32_t tmem_slot;
+  __shared__ uint32_t abort_flag;
+  __shared__ uint32_t reduce_flag;
+  __shared__ uint32_t slot_seg[kLocalMaxSlots];
+  __shared__ uint32_t n_cta_slots;
+
+  const uint32_t warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t D = P.D, H = P.H, C = P.C, T = P.T;
+  const uint32_t G = gridDim.x;
+  const uint32_t ub = cta_begin(static_cast<uint32_t>(P.n_units), G, blockIdx.x);
+  const uint32_t ue = cta_begin(static_cast<uint32_t>(P.n_units), G, blockIdx.x + 1);
+  const uint32_t n_kt = P.L.n_kt, n_tiles = P.L.n_tiles;
+
+  uint32_t* lut = reinterpret_cast<uint32_t*>(smem + P.off_lut);
+  uint8_t* wslots = smem + P.off_w;
+  uint8_t* chunks = smem + (((smem_u32(smem + P.off_chunk) + kRingBytes - 1) & ~(kRingBytes - 1)) - smem_u32(smem));
+  uint8_t* xslots = smem + P.off_x;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P.off_bars);
+  uint64_t* w_empty = bars;           // D: a producer's slots are free again
+  uint64_t* chunk_bars = bars + D;    // 4 per producer
+  uint64_t* acc_full = bars + 5 * D;  // one per accumulator slot
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (uint32_t i = 0; i < 5 * D + P.n_slots; ++i) mbar_init(&bars[i], 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&tmem_slot, P.tmem_cols);
+    tmem_relinquish();
+  }
+  if (kDecode && P.L.single_symbol == kNoSymbol) build_lut(lut, P.L, warp, blockDim.x / 32, lane);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_slot;
+  volatile uint32_t* abort = &abort_flag;
+  if (threadIdx.x == 0) trace_mark(P, 0);
+
+  if (warp >= 4) {
+    // ============================ producer warps ============================
+    const uint32_t d = warp - 4;
+    uint32_t pb, pe;
+    producer_range(ub, ue, D, d, &pb, &pe);
+    // accumulator slots are numbered in unit order: producer d's first slot
+    // follows the segments touched by producers 0 .. d-1
+    uint32_t slot_next = 0;
+    for (uint32_t q = 0; q < d; ++q) {
+      uint32_t b, e;
+      producer_range(ub, ue, D, q, &b, &e);
+      if (e > b) slot_next += (e - 1) / n_kt - b / n_kt + 1;
+    }
+    const LayerDev& L = P.L;
+    const bool single = L.single_symbol != kNoSymbol;
+    const uint32_t lt = lanemask_lt();
+    const uint32_t lut_s = smem_u32(lut);
+    const uint32_t swz = ((lane >> 2) & 1u) << 4;
+    const uint32_t w_s = smem_u32(wslots + d * kSlabBytes);
+    const uint32_t x_s = smem_u32(xslots + d * T * 32);
+    // descriptor fields shared by both operands: LBO 16 B, SBO 256 B,
+    // version 1, 32-byte swizzle; only the start address differs
+    const uint64_t dhi = (1ull << 16) | (16ull << 32) | (1ull << 46) | (6ull << 61);
+    const uint64_t adesc = dhi | (w_s >> 4), bdesc = dhi | (x_s >> 4);
+    const unsigned long long* offsets = reinterpret_cast<const unsigned long long*>(L.offsets);
+    const uint32_t S = L.tile_n * L.tile_k;
+    const uint32_t n_xch = T / 16;  // 16-byte X chunks per lane per slab (1 or 2)
+    RunPipe pipe;
+    rp_init(pipe, chunks + d * kRingBytes, chunk_bars + 4 * d);
+    TileCursor tc;
+    tc.x = tc.pos = tc.cb = tc.bytes = 0;
+    uint32_t nw = 0;  // slabs handed to the tensor core
+    uint32_t cur_seg = 0xFFFFFFFFu;
+    uint32_t cur_slot = 0, fresh = 0;
+
+    uint32_t u = pb;
+    while (u < pe) {
+      const uint32_t p = u / n_tiles;
+      const uint32_t run_e = min(pe, (p + 1) * n_tiles);
+      const uint32_t t0 = u - p * n_tiles;
+      const uint32_t t1 = run_e - 1 - p * n_tiles;
+      bool run_ok = true;
+      uint64_t run_start = 0, a_next = 0;
+      uint32_t run_bytes = 0, base = 0;
+      if (kDecode) {
+        run_ok = run_extent(L, t0, t1, &run_start, &run_bytes);
+        if (run_ok) base = rp_run_begin(pipe, L.stream + run_start, run_bytes);
+        a_next = run_start;
+      }
+      for (; u < run_e; ++u) {
+        const uint32_t t = u - p * n_tiles;
+        const uint32_t seg = u / n_kt;
+        if (seg != cur_seg) {
+          if (cur_seg != 0xFFFFFFFFu && lane == 0) umma_commit(&acc_full[cur_slot]);
+          cur_slot = slot_next++;
+          cur_seg = seg;
+          fresh = (1u << H) - 1u;
+        }
+        const uint32_t rb = t / n_kt, kt = t - rb * n_kt;
+        const uint32_t n0 = rb * L.tile_n, k0 = kt * L.tile_k;
+        bool zero_tile = false;
+        if (kDecode) {
+          zero_tile = !run_ok;
+          if (run_ok) {
+            const uint64_t a = a_next, b = __ldg(offsets + t + 1);
+            a_next = b;
+            if (!run_tile_begin(pipe, L, a, b, run_start, base, tc, lane, abort, P.status)) {
+              run_ok = false;
+              zero_tile = true;
+            }
+          }
+          if (zero_tile && lane == 0) atomicOr(P.status, kStatusBadOffsets);
+        }
+        __half2 gscale[8];
+        if (kFmt == kFmtInt4F16Group) {
+          const uint32_t gk = k0 / P.group_k;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const uint32_t hh = q / 4, ii = q % 4;
+            float sv = 0.f;
+            if (hh < H) {
+              const uint32_t row = n0 + lane + 32 * (4 * hh + ii);
+              sv = bf16_to_f32(__ldg(static_cast<const uint16_t*>(P.scales) +
+                                     static_cast<uint64_t>(row) * P.n_groups_k + gk));
+            }
+            gscale[q] = __float2half2_rn(sv);
+          }
+        }
+        // raw sign/mantissa bytes of groups g, g+1, g+2 in flight (bf16, decode)
+        const unsigned long long* raw_tile = nullptr;
+        uint64_t r0 = 0, r1 = 0, r2 = 0;
+        const uint32_t groups = H * C * 8;
+        if (kDecode && kFmt == kFmtBf16Split && !zero_tile) {
+          raw_tile = reinterpret_cast<const unsigned long long*>(L.raw + static_cast<uint64_t>(t) * S) + lane;
+          r0 = __ldg(raw_tile);
+          r1 = __ldg(raw_tile + 32);
+          r2 = __ldg(raw_tile + 64);
+        }
+
+        for (uint32_t us = 0; us < H * C; ++us) {
+          const uint32_t h = us % H, s = us / H;
+          __half2 gs0, gs1, gs2, gs3;
+          if (kFmt == kFmtInt4F16Group) {
+            gs0 = h ? gscale[4] : gscale[0];
+            gs1 = h ? gscale[5] : gscale[1];
+            gs2 = h ? gscale[6] : gscale[2];
+            gs3 = h ? gscale[7] : gscale[3];
+          }
+          // X slab s of this unit (T rows x 16 columns): this lane's chunks,
+          // fetched now and stored next to the W slab before the MMA
+          uint4 xv[2];
+          const bool new_x = (h == 0);
+          if (new_x) {
+#pragma unroll
+            for (uint32_t j = 0; j < 2; ++j) {
+              xv[j] = make_uint4(0, 0, 0, 0);
+              const uint32_t r = (lane >> 1) + 16 * j, c = lane & 1u;
+              const uint32_t m = p * P.T_pass + r;
+              if (j < n_xch && m < P.M)
+                xv[j] = __ldg(reinterpret_cast<const uint4*>(P.X + static_cast<uint64_t>(m) * L.K + k0 +
+                                                             16 * s + 8 * c));
+            }
+          }
+          uint4 cp[8];
+          if (!kDecode) {
+#pragma unroll
+            for (int gg = 0; gg < 8; ++gg) {
+              const uint32_t i = gg & 3, c = gg >> 2;
+              const uint64_t row = n0 + lane + 32 * (4 * h + i);
+              const uint64_t idx = row * L.K + k0 + 16 * s + 8 * c;
+              if (kFmt == kFmtBf16Split) {
+                cp[gg] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(P.w_plain) + idx));
+              } else if (kFmt == kFmtFp8F16) {
+                uint2 v = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(P.w_plain) + idx));
+                cp[gg] = make_uint4(v.x, v.y, 0, 0);
+              } else {
+                uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(P.w_plain) + idx / 2));
+                cp[gg] = make_uint4(v, 0, 0, 0);
+              }
+            }
+          }
+#pragma unroll 1
+          for (uint32_t gg = 0; gg < 8; ++gg) {
+            const uint32_t g = us * 8 + gg;
+            const uint32_t i = gg & 3, c = gg >> 2;
+            uint32_t o[4];
+            if (kDecode) {
+              const uint64_t raw8 = r0;
+              if (kFmt == kFmtBf16Split && !zero_tile) {
+                r0 = r1;
+                r1 = r2;
+                if (g + 3 < groups) r2 = __ldg(raw_tile + 32 * (g + 3));
+              }
+              uint32_t e[8];
+              if (zero_tile) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) e[k] = 0;
+              } else if (single) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) e[k] = L.single_symbol << 12;
+              } else {
+                rp_group(pipe, tc.pos, lane, abort, P.status);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) e[k] = decode_step(tc.x, tc.pos, lut_s, pipe.ring_s, lt);
+              }
+              if (kFmt == kFmtBf16Split) fmt_bf16_split(e, raw8, o);
+              else if (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
+              else if (kFmt == kFmtInt4F16Group)
+                fmt_int4_f16_scaled(e, i == 0 ? gs0 : i == 1 ? gs1 : i == 2 ? gs2 : gs3, o);
+              else fmt_fp8_f16(e, o);
+              if (zero_tile) o[0] = o[1] = o[2] = o[3] = 0;
+            } else {
+              uint4 v = cp[0];
+#pragma unroll
+              for (int q = 1; q < 8; ++q)
+                if (gg == static_cast<uint32_t>(q)) v = cp[q];
+              if (kFmt == kFmtBf16Split) {
+                o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+              } else {
+                uint32_t e[8];
+                if (kFmt == kFmtFp8F16) {
+#pragma unroll
+                  for (int k = 0; k < 4; ++k) {
+                    e[k] = ((v.x >> (8 * k)) & 0xFFu) << 12;
+                    e[k + 4] = ((v.y >> (8 * k)) & 0xFFu) << 12;
+                  }
+                  fmt_fp8_f16(e, o);
+                } else {
+#pragma unroll
+                  for (int k = 0; k < 8; ++k) e[k] = (((v.x >> (4 * k)) & 0xFu) ^ 8u) << 12;
+                  if (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
+                  else fmt_int4_f16_scaled(e, i == 0 ? gs0 : i == 1 ? gs1 : i == 2 ? gs2 : gs3, o);
+                }
+              }
+            }
+            // the slot (and the X slab) are free once the previous MMA retired
+            if (gg == 0 && nw > 0)
+              wait_live(&w_empty[d], (nw - 1) & 1u, abort, P.status, 1);
+            const uint32_t addr = w_s + (32 * i + lane) * 32 + ((c << 4) ^ swz);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(o[0]),
+                         "r"(o[1]), "r"(o[2]), "r"(o[3])
+                         : "memory");
+          }
+          if (new_x) {
+#pragma unroll
+            for (uint32_t j = 0; j < 2; ++j) {
+              if (j >= n_xch) break;
+              uint4 v = xv[j];
+              if (P.x_f16) {
+                uint32_t in[4] = {v.x, v.y, v.z, v.w}, out[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  __half2 hv = __floats2half2_rn(__uint_as_float(in[k] << 16),
+                                                 __uint_as_float(in[k] & 0xFFFF0000u));
+                  out[k] = *reinterpret_cast<uint32_t*>(&hv);
+                }
+                v = make_uint4(out[0], out[1], out[2], out[3]);
+              }
+              const uint32_t r = (lane >> 1) + 16 * j, c = lane & 1u;
+              const uint32_t addr = x_s + r * 32 + ((c ^ ((r >> 2) & 1u)) << 4);
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x),
+                           "r"(v.y), "r"(v.z), "r"(v.w)
+                           : "memory");
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tc_fence_after();
+            const uint32_t col = (cur_slot * H + h) * T;
+            umma_f16(tmem_base + col, adesc, bdesc, P.idesc, ((fresh >> h) & 1u) ? 0u : 1u);
+            umma_commit(&w_empty[d]);
+          }
+          fresh &= ~(1u << h);
+          ++nw;
+        }
+        if (kDecode && !zero_tile && !run_tile_end(tc, single) && lane == 0)
+          atomicOr(P.status, kStatusCorrupt);
+      }
+    }
+    if (cur_seg != 0xFFFFFFFFu && lane == 0) umma_commit(&acc_full[cur_slot]);
+    // the last commit's arrival lands before the warp leaves
+    if (nw > 0) wait_drain(&w_empty[d], (nw - 1) & 1u, P.status);
+    if (kDecode) rp_drain(pipe, P.status);
+    if (lane == 0) trace_mark(P, 18 + d);
+  } else {
+    // ===================== epilogue (warps 0-3, 128 threads) =====================
+    const uint32_t e = threadIdx.x;   // TMEM lane = row within the 128-row half
+    const uint32_t nck = H * T / 16;  // 16-column chunks per accumulator (1 or 2)
+    const uint32_t seg_first = ub / n_kt;
+    // W row-block segment of every accumulator slot, in slot (= unit) order
+    if (e == 0) {
+      uint32_t k = 0;
+      for (uint32_t d = 0; d < D; ++d) {
+        uint32_t b, en;
+        producer_range(ub, ue, D, d, &b, &en);
+        if (en <= b) continue;
+        for (uint32_t seg = b / n_kt; seg <= (en - 1) / n_kt && k < kLocalMaxSlots; ++seg) slot_seg[k++] = seg;
+      }
+      n_cta_slots = k;
+    }
+    named_bar_sync(1, 128);
+    const uint32_t ns = n_cta_slots;
+    uint32_t nflush = 0;
+    for (uint32_t sa = 0; sa < ns;) {
+      const uint32_t seg = slot_seg[sa];
+      uint32_t sb = sa + 1;
+      while (sb < ns && slot_seg[sb] == seg) ++sb;
+      // sum the segment's accumulators in slot order, two 16-column TMEM
+      // loads in flight per wait
+      float acc[2][16];
+      for (uint32_t k = sa; k < sb;) {
+        const uint32_t nb = (nck == 1 && k + 1 < sb) ? 2u : 1u;
+        for (uint32_t j = 0; j < nb; ++j) wait_live(&acc_full[k + j], 0, abort, P.status, 6, 64);
+        tc_fence_after();
+        uint32_t v[2][16];
+        const uint32_t taddr = tmem_base + ((32 * warp) << 16) + k * H * T;
+        tmem_ld16(taddr, v[0]);
+        if (nb == 2 || nck == 2) tmem_ld16(taddr + 16, v[1]);
+        tmem_ld_wait();
+        if (nck == 1) {
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            float x = __uint_as_float(v[0][q]);
+            if (k > sa) x = acc[0][q] + x;
+            if (nb == 2) x = x + __uint_as_float(v[1][q]);
+            acc[0][q] = x;
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            acc[0][q] = (k > sa) ? acc[0][q] + __uint_as_float(v[0][q]) : __uint_as_float(v[0][q]);
+            acc[1][q] = (k > sa) ? acc[1][q] + __uint_as_float(v[1][q]) : __uint_as_float(v[1][q]);
+          }
+        }
+        k += nb;
+      }
+      // store: Y for a segment this CTA holds whole, else split-K partials
+      const uint32_t p = seg / P.n_rb, rb = seg % P.n_rb;
+      const uint32_t s_lo = seg * n_kt, s_hi = s_lo + n_kt;
+      const bool complete = ub <= s_lo && ue >= s_hi;
+      const uint32_t pslot = (seg == seg_first) ? 0u : 1u;
+      float* part = P.partials + (static_cast<uint64_t>(blockIdx.x) * 2 + pslot) * H * P.T_pass * 128;
+#pragma unroll
+      for (uint32_t ck = 0; ck < 2; ++ck) {
+        if (ck >= nck) break;
+        const uint32_t per_h = T / 16;
+        const uint32_t h = ck / per_h, tok0 = (ck % per_h) * 16;
+        const uint32_t n = rb * P.L.tile_n + h * 128 + e;
+        const float scale = complete ? row_scale(P, n) : 1.0f;
+        epi_emit16(P, acc[ck], complete, scale, part, p, h, tok0, n, e);
+      }
+      if (e == 0) trace_mark(P, 60 + 2 * min(nflush, 1u));
+      if (!complete) splitk_finish(P, seg, p, rb, e, &reduce_flag);
+      if (e == 0) trace_mark(P, 61 + 2 * min(nflush, 1u));
+      ++nflush;
+      sa = sb;
+    }
+  }
+
+  // ---- teardown: every MMA retired (the epilogue consumed every accumulator)
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0) trace_mark(P, 41);
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, P.tmem_cols);
+  }
+}
+
+template <bool kDecode, uint32_t kFmt>
+static cudaError_t launch_local_variant(const GemmPlan& plan, const GemmDev& P, cudaStream_t stream) {
+  auto kern = fused_gemm_local_kernel<kDecode, kFmt>;
+  static int attr_set[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = 1;
+  }
+  kern<<<plan.grid, (4 + plan.D) * 32, plan.smem_bytes, stream>>>(P);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_local(const GemmPlan& plan, const GemmDev& P, bool decode,
+                              cudaStream_t stream) {
+  switch (plan.fmt | (decode ? 0u : 8u)) {
+    case kFmtBf16Split: return launch_local_variant<true, kFmtBf16Split>(plan, P, stream);
+    case kFmtInt4Bf16: return launch_local_variant<true, kFmtInt4Bf16>(plan, P, stream);
+    case kFmtInt4F16Group: return launch_local_variant<true, kFmtInt4F16Group>(plan, P, stream);
+    case kFmtFp8F16: return launch_local_variant<true, kFmtFp8F16>(plan, P, stream);
+    case 8 | kFmtBf16Split: return launch_local_variant<false, kFmtBf16Split>(plan, P, stream);
+    case 8 | kFmtInt4Bf16: return launch_local_variant<false, kFmtInt4Bf16>(plan, P, stream);
+    case 8 | kFmtInt4F16Group: return launch_local_variant<false, kFmtInt4F16Group>(plan, P, stream);
+    case 8 | kFmtFp8F16: return launch_local_variant<false, kFmtFp8F16>(plan, P, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace ansdev

@@ -42,6 +42,8 @@ struct GemmPlan {
   uint32_t n_bufs;     // TMEM accumulator sets (1 or 2)
   uint32_t x_stages;
   uint32_t tmem_cols;
+  uint32_t local;      // 1: every producer warp issues its own MMAs (gemm_local.cu)
+  uint32_t n_slots;    // local schedule: TMEM accumulators per CTA (max over CTAs)
   uint32_t grid;       // CTAs
   uint64_t n_units;    // n_pass * n_tiles
   uint32_t n_segments; // n_pass * (N / tile_n)
@@ -67,6 +69,9 @@ struct GemmDev {
   uint32_t off_lut, off_w, off_chunk, off_x, off_bars;
   unsigned long long* trace;  // optional per-CTA event timestamps (internal profiling)
   const uint8_t* xs;          // X staged as pre-swizzled 16-column slabs (workspace)
+  const uint16_t* X;          // local schedule: X as given (bf16, M x K row-major)
+  uint32_t x_f16;             // local schedule: convert X to f16 for the MMA
+  uint32_t n_slots;           // local schedule: accumulator slots (barriers) per CTA
 };
 
 // Internal profiling hook: when set, every fused-GEMM CTA writes globaltimer
@@ -78,6 +83,11 @@ constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
 // Device address of that scratch on the current device (looked up once per
 // device; see noalloc.cu).
 cudaError_t noalloc_scratch(void** ptr);
+
+// Local schedule (gemm_local.cu): launches the kernel for an already filled
+// GemmDev.
+cudaError_t launch_gemm_local(const GemmPlan& plan, const GemmDev& P, bool decode,
+                              cudaStream_t stream);
 
 // Fills a plan; returns false if the shape cannot be scheduled.
 bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool decode,

@@ -200,6 +200,141 @@ struct TileCursor {
   uint32_t bytes;  // tile bytes (padded)
 };
 
+// Per-warp pipeline over a RUN: tiles that follow one another in the stream
+// (a warp that owns a contiguous range of tiles streams one contiguous byte
+// range, so no per-tile bookkeeping is needed to keep the ring full).  Bytes
+// are addressed by an unwrapped position: a run starts on a chunk boundary
+// (run_c0 * kChunkBytes) and byte b of the run sits at that start + b; the
+// ring slot of a position is position % kRingBytes.  Same ring, chunk size
+// and barriers as ChunkPipe.
+struct RunPipe {
+  uint8_t* ring;
+  uint32_t ring_s;
+  uint64_t* bars;
+  const uint8_t* src;  // first byte of the current run in global memory
+  uint32_t run_c0;     // global chunk index of the run's first chunk
+  uint32_t run_end;    // global chunk index one past the run's last chunk
+  uint32_t run_bytes;
+  uint32_t issued, ready;  // global chunk counters
+  uint32_t cur;            // chunk the cursor was last seen in
+};
+
+__device__ __forceinline__ void rp_init(RunPipe& p, uint8_t* ring, uint64_t* bars) {
+  p.ring = ring;
+  p.ring_s = smem_u32(ring);
+  p.bars = bars;
+  p.src = nullptr;
+  p.run_c0 = p.run_end = p.run_bytes = 0;
+  p.issued = p.ready = 0;
+  p.cur = 0xFFFFFFFFu;
+}
+
+// Starts a run of `bytes` bytes at `src`; returns its base position.  Chunks
+// of earlier runs that are still in flight keep their slots until waited.
+__device__ __forceinline__ uint32_t rp_run_begin(RunPipe& p, const uint8_t* src, uint32_t bytes) {
+  p.src = src;
+  p.run_bytes = bytes;
+  p.run_c0 = p.issued;
+  p.run_end = p.issued + (bytes + kChunkBytes - 1) / kChunkBytes;
+  p.cur = 0xFFFFFFFFu;
+  return p.run_c0 * kChunkBytes;
+}
+
+// Called when the cursor enters chunk c: afterwards chunk c + 1 (or the run's
+// last chunk) has landed and chunks up to c + 3 are in flight.  A slot is
+// re-armed only after the chunk that last used it was waited for.
+__device__ __forceinline__ void rp_enter(RunPipe& p, uint32_t c, uint32_t lane,
+                                         volatile uint32_t* abort, uint32_t* status) {
+  p.cur = c;
+  const uint32_t lim = min(c + 4u, p.run_end);
+  while (p.issued < lim && !*abort) {
+    while (p.ready + 4u <= p.issued) {
+      if (!wait_live(&p.bars[p.ready & 3u], (p.ready >> 2) & 1u, abort, status)) return;
+      p.ready++;
+    }
+    const uint32_t off = (p.issued - p.run_c0) * kChunkBytes;
+    const uint32_t n = min(kChunkBytes, p.run_bytes - off);
+    const uint32_t slot = p.issued & 3u;
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&p.bars[slot], n);
+      bulk_g2s(p.ring + slot * kChunkBytes, p.src + off, n, &p.bars[slot]);
+    }
+    p.issued++;
+  }
+  const uint32_t need = min(c + 1u, p.run_end - 1u);
+  while (p.ready <= need && p.ready < p.issued) {
+    if (!wait_live(&p.bars[p.ready & 3u], (p.ready >> 2) & 1u, abort, status)) return;
+    p.ready++;
+  }
+}
+
+__device__ __forceinline__ void rp_drain(RunPipe& p, uint32_t* status) {
+  while (p.ready < p.issued) {
+    wait_drain(&p.bars[p.ready & 3u], (p.ready >> 2) & 1u, status);
+    p.ready++;
+  }
+}
+
+// Before each group of 8 steps (at most 512 bytes read): keep the chunk after
+// the cursor's resident.
+__device__ __forceinline__ void rp_group(RunPipe& p, uint32_t pos, uint32_t lane,
+                                         volatile uint32_t* abort, uint32_t* status) {
+  const uint32_t c = pos / kChunkBytes;
+  if (c != p.cur) rp_enter(p, c, lane, abort, status);
+}
+
+// Offsets of a run of tiles [t0, t1] (inclusive), validated as a whole: the
+// run's copies stay inside the stream whatever the offsets say.
+__device__ __forceinline__ bool run_extent(const LayerDev& L, uint32_t t0, uint32_t t1,
+                                           uint64_t* start, uint32_t* bytes) {
+  const unsigned long long* off = reinterpret_cast<const unsigned long long*>(L.offsets);
+  const uint64_t a = __ldg(off + t0), b = __ldg(off + t1 + 1);
+  const uint64_t max_tile = 4ull * kLanes + 2ull * L.tile_n * L.tile_k + 16ull;
+  const bool ok = (a % 16 == 0) && (b % 16 == 0) && b >= a + 4ull * kLanes * (t1 - t0 + 1) &&
+                  b <= L.stream_bytes && (b - a) <= max_tile * (t1 - t0 + 1) &&
+                  (b - a) < (1ull << 31);
+  *start = a;
+  *bytes = ok ? static_cast<uint32_t>(b - a) : 0u;
+  return ok;
+}
+
+// Tile inside a run: [a, b) are its stream offsets, run_start the run's first
+// stream offset, base the run's base position.  Checks the tile's extent
+// against the run, makes its first bytes resident and loads the lane states.
+// Returns false for a tile whose offsets are invalid (the rest of the run is
+// then skipped by the caller).
+__device__ __forceinline__ bool run_tile_begin(RunPipe& p, const LayerDev& L, uint64_t a,
+                                               uint64_t b, uint64_t run_start, uint32_t base,
+                                               TileCursor& tc, uint32_t lane,
+                                               volatile uint32_t* abort, uint32_t* status) {
+  const uint64_t max_tile = 4ull * kLanes + 2ull * L.tile_n * L.tile_k + 16ull;
+  if (b % 16 != 0 || b < a + 4ull * kLanes || b - a > max_tile || a < run_start ||
+      b > run_start + p.run_bytes)
+    return false;
+  tc.bytes = static_cast<uint32_t>(b - a);
+  tc.cb = base + static_cast<uint32_t>(a - run_start);  // tile start position
+  tc.pos = tc.cb;
+  rp_group(p, tc.pos, lane, abort, status);
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];"
+               : "=r"(v)
+               : "r"(((tc.pos + 4 * lane) & (kRingBytes - 1)) + p.ring_s)
+               : "memory");
+  tc.x = v;
+  tc.pos += 4 * kLanes;
+  return true;
+}
+
+// Ends a tile of a run (same integrity rule as tile_end).
+__device__ __forceinline__ bool run_tile_end(const TileCursor& tc, bool single) {
+  const uint32_t used = tc.pos - tc.cb;
+  bool bad = (tc.x != kStateLow) || used > tc.bytes || tc.bytes - used >= 16;
+  if (single) bad = (tc.x != kStateLow) || tc.bytes != 4 * kLanes;
+  return !__any_sync(0xFFFFFFFFu, bad);
+}
+
+
+
 // Starts tile t: validates its extent, makes its first chunks resident and
 // loads the lane states.  Returns false for a tile with invalid offsets.
 __device__ __forceinline__ bool tile_begin(ChunkPipe& p, const LayerDev& L, const TileSeq& seq,

@@ -109,12 +109,19 @@ def test_gemm_corrupt_stream_flags_status(cuda, cases):
     assert not st & ans.STATUS_TIMEOUT
 
 
+@pytest.mark.parametrize("schedule", ["local", "central"])
 @pytest.mark.parametrize("ctas,producers", [(8, 16), (5, 3), (3, 7)])
 @pytest.mark.parametrize("name,N,K,M", [("bf16_4096", 1024, 2048, 16), ("int4_70b", 512, 2048, 40),
-                                        ("fp8_405b", 512, 1024, 300), ("tiny_int4", 512, 512, 130)])
-def test_gemm_multi_round_schedules(cuda, oracle, cases, monkeypatch, ctas, producers, name, N, K, M):
-    # few CTAs and few producer warps: many rounds per CTA, rounds that cross
-    # W row blocks, slab and X rings wrapping many times, both accumulator sets
+                                        ("fp8_405b", 512, 1024, 300), ("tiny_int4", 512, 512, 130),
+                                        ("int4_70b", 512, 2048, 16), ("fp8_405b", 512, 1024, 32),
+                                        ("tiny_int4", 512, 512, 1)])
+def test_gemm_multi_round_schedules(cuda, oracle, cases, monkeypatch, schedule, ctas, producers,
+                                    name, N, K, M):
+    # few CTAs and few producer warps: many rounds (shared-accumulator
+    # schedule) or long per-warp runs crossing W row blocks (local schedule,
+    # M <= 32 only; larger M always takes the shared-accumulator schedule),
+    # slab, chunk and X rings wrapping many times
+    monkeypatch.setenv("ANS_GEMM_SCHEDULE", schedule)
     monkeypatch.setenv("ANS_GEMM_MAX_CTAS", str(ctas))
     monkeypatch.setenv("ANS_GEMM_MAX_PRODUCERS", str(producers))
     cfg, d, lay, layer = _case(cases, name, N, K)
@@ -124,3 +131,38 @@ def test_gemm_multi_round_schedules(cuda, oracle, cases, monkeypatch, ctas, prod
     assert st == 0 and stu == 0 and torch.equal(Y, Yu)
     Yref = oracle.gemm(cfg.dtype, X, M, K, d["w"], N, cfg.scale_kind, d["scales"], cfg.group_k)
     assert rel_fro(Y.cpu().numpy(), Yref) <= TOL
+
+
+@pytest.mark.parametrize("name,N,K,M", [("bf16_4096", 1024, 4096, 16), ("int4_70b", 512, 2048, 8),
+                                        ("fp8_405b", 256, 2048, 32), ("tiny_int4", 512, 512, 1)])
+def test_gemm_both_schedules_small_m(cuda, oracle, cases, monkeypatch, name, N, K, M):
+    # at M <= 32 the local schedule is the default; the shared-accumulator one
+    # must agree with the fp64 oracle too (the two add in different orders, so
+    # they agree to rounding, not bit for bit)
+    cfg, d, lay, layer = _case(cases, name, N, K)
+    X = WL.make_x(cfg, M, K)
+    Yref = oracle.gemm(cfg.dtype, X, M, K, d["w"], N, cfg.scale_kind, d["scales"], cfg.group_k)
+    out = {}
+    for schedule in ["local", "central"]:
+        monkeypatch.setenv("ANS_GEMM_SCHEDULE", schedule)
+        Y, st, _ = run_gemm(cfg, d, lay, layer, X, compressed=True)
+        Yu, stu, _ = run_gemm(cfg, d, lay, layer, X, compressed=False)
+        assert st == 0 and stu == 0 and torch.equal(Y, Yu), schedule
+        assert rel_fro(Y.cpu().numpy(), Yref) <= TOL, schedule
+        out[schedule] = Y
+    assert rel_fro(out["local"].cpu().numpy(), out["central"].cpu().numpy().astype(np.float64)) <= 1e-5
+
+
+@pytest.mark.parametrize("schedule", ["local", "central"])
+def test_gemm_bad_offsets_flag_status(cuda, cases, monkeypatch, schedule):
+    # an offset table that points past the stream: the affected tiles are
+    # skipped (treated as zero), the status says why, nothing reads outside
+    monkeypatch.setenv("ANS_GEMM_SCHEDULE", schedule)
+    cfg, d, lay, layer = _case(cases, "bf16_4096", 512, 1024)
+    off = layer.h_offsets.copy()
+    off[7] = off[-1] + 4096
+    broken = ans.CompressedLayer(lay, layer.codebook, layer.h_stream, off, layer.h_raw)
+    X = WL.make_x(cfg, 16, 1024)
+    Y, st, _ = run_gemm(cfg, d, lay, broken, X)
+    assert st & ans.STATUS_BAD_OFFSETS
+    assert not st & ans.STATUS_TIMEOUT
