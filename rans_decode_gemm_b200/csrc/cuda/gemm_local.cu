@@ -26,6 +26,7 @@
 #include <cuda_runtime.h>
 
 #include <cstring>
+#include <type_traits>
 
 #include "gemm_common.cuh"
 #include "kernels.h"
@@ -187,143 +188,149 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
           r2 = __ldg(raw_tile + 64);
         }
 
-        for (uint32_t us = 0; us < H * C; ++us) {
-          const uint32_t h = us % H, s = us / H;
-          __half2 gs0, gs1, gs2, gs3;
-          if (kFmt == kFmtInt4F16Group) {
-            gs0 = h ? gscale[4] : gscale[0];
-            gs1 = h ? gscale[5] : gscale[1];
-            gs2 = h ? gscale[6] : gscale[2];
-            gs3 = h ? gscale[7] : gscale[3];
-          }
-          // X slab s of this unit (T rows x 16 columns): this lane's chunks,
-          // fetched now and stored next to the W slab before the MMA
-          uint4 xv[2];
-          const bool new_x = (h == 0);
-          if (new_x) {
-#pragma unroll
-            for (uint32_t j = 0; j < 2; ++j) {
-              xv[j] = make_uint4(0, 0, 0, 0);
-              const uint32_t r = (lane >> 1) + 16 * j, c = lane & 1u;
-              const uint32_t m = p * P.T_pass + r;
-              if (j < n_xch && m < P.M)
-                xv[j] = __ldg(reinterpret_cast<const uint4*>(P.X + static_cast<uint64_t>(m) * L.K + k0 +
-                                                             16 * s + 8 * c));
+        // the slabs of this tile; a tile of constant symbols (single-symbol
+        // codebook, or zeros for a tile with bad offsets) takes a separate
+        // instantiation so the decoding path carries no per-group branches
+        const uint32_t const_e = zero_tile ? 0u : (single ? L.single_symbol << 12 : 0u);
+        auto run_slabs = [&](auto const_sym) {
+          constexpr bool kConst = decltype(const_sym)::value;
+          for (uint32_t us = 0; us < H * C; ++us) {
+            const uint32_t h = us % H, s = us / H;
+            __half2 gs0, gs1, gs2, gs3;
+            if (kFmt == kFmtInt4F16Group) {
+              gs0 = h ? gscale[4] : gscale[0];
+              gs1 = h ? gscale[5] : gscale[1];
+              gs2 = h ? gscale[6] : gscale[2];
+              gs3 = h ? gscale[7] : gscale[3];
             }
-          }
-          uint4 cp[8];
-          if (!kDecode) {
+            // X slab s of this unit (T rows x 16 columns): this lane's chunks,
+            // fetched now and stored next to the W slab before the MMA
+            uint4 xv[2];
+            const bool new_x = (h == 0);
+            if (new_x) {
 #pragma unroll
-            for (int gg = 0; gg < 8; ++gg) {
-              const uint32_t i = gg & 3, c = gg >> 2;
-              const uint64_t row = n0 + lane + 32 * (4 * h + i);
-              const uint64_t idx = row * L.K + k0 + 16 * s + 8 * c;
-              if (kFmt == kFmtBf16Split) {
-                cp[gg] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(P.w_plain) + idx));
-              } else if (kFmt == kFmtFp8F16) {
-                uint2 v = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(P.w_plain) + idx));
-                cp[gg] = make_uint4(v.x, v.y, 0, 0);
-              } else {
-                uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(P.w_plain) + idx / 2));
-                cp[gg] = make_uint4(v, 0, 0, 0);
+              for (uint32_t j = 0; j < 2; ++j) {
+                xv[j] = make_uint4(0, 0, 0, 0);
+                const uint32_t r = (lane >> 1) + 16 * j, c = lane & 1u;
+                const uint32_t m = p * P.T_pass + r;
+                if (j < n_xch && m < P.M)
+                  xv[j] = __ldg(reinterpret_cast<const uint4*>(P.X + static_cast<uint64_t>(m) * L.K + k0 +
+                                                               16 * s + 8 * c));
               }
             }
-          }
-#pragma unroll 1
-          for (uint32_t gg = 0; gg < 8; ++gg) {
-            const uint32_t g = us * 8 + gg;
-            const uint32_t i = gg & 3, c = gg >> 2;
-            uint32_t o[4];
-            if (kDecode) {
-              const uint64_t raw8 = r0;
-              if (kFmt == kFmtBf16Split && !zero_tile) {
-                r0 = r1;
-                r1 = r2;
-                if (g + 3 < groups) r2 = __ldg(raw_tile + 32 * (g + 3));
-              }
-              uint32_t e[8];
-              if (zero_tile) {
+            uint4 cp[8];
+            if (!kDecode) {
 #pragma unroll
-                for (int k = 0; k < 8; ++k) e[k] = 0;
-              } else if (single) {
-#pragma unroll
-                for (int k = 0; k < 8; ++k) e[k] = L.single_symbol << 12;
-              } else {
-                rp_group(pipe, tc.pos, lane, abort, P.status);
-#pragma unroll
-                for (int k = 0; k < 8; ++k) e[k] = decode_step(tc.x, tc.pos, lut_s, pipe.ring_s, lt);
-              }
-              if (kFmt == kFmtBf16Split) fmt_bf16_split(e, raw8, o);
-              else if (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
-              else if (kFmt == kFmtInt4F16Group)
-                fmt_int4_f16_scaled(e, i == 0 ? gs0 : i == 1 ? gs1 : i == 2 ? gs2 : gs3, o);
-              else fmt_fp8_f16(e, o);
-              if (zero_tile) o[0] = o[1] = o[2] = o[3] = 0;
-            } else {
-              uint4 v = cp[0];
-#pragma unroll
-              for (int q = 1; q < 8; ++q)
-                if (gg == static_cast<uint32_t>(q)) v = cp[q];
-              if (kFmt == kFmtBf16Split) {
-                o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
-              } else {
-                uint32_t e[8];
-                if (kFmt == kFmtFp8F16) {
-#pragma unroll
-                  for (int k = 0; k < 4; ++k) {
-                    e[k] = ((v.x >> (8 * k)) & 0xFFu) << 12;
-                    e[k + 4] = ((v.y >> (8 * k)) & 0xFFu) << 12;
-                  }
-                  fmt_fp8_f16(e, o);
+              for (int gg = 0; gg < 8; ++gg) {
+                const uint32_t i = gg & 3, c = gg >> 2;
+                const uint64_t row = n0 + lane + 32 * (4 * h + i);
+                const uint64_t idx = row * L.K + k0 + 16 * s + 8 * c;
+                if (kFmt == kFmtBf16Split) {
+                  cp[gg] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(P.w_plain) + idx));
+                } else if (kFmt == kFmtFp8F16) {
+                  uint2 v = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(P.w_plain) + idx));
+                  cp[gg] = make_uint4(v.x, v.y, 0, 0);
                 } else {
-#pragma unroll
-                  for (int k = 0; k < 8; ++k) e[k] = (((v.x >> (4 * k)) & 0xFu) ^ 8u) << 12;
-                  if (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
-                  else fmt_int4_f16_scaled(e, i == 0 ? gs0 : i == 1 ? gs1 : i == 2 ? gs2 : gs3, o);
+                  uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(P.w_plain) + idx / 2));
+                  cp[gg] = make_uint4(v, 0, 0, 0);
                 }
               }
             }
-            // the slot (and the X slab) are free once the previous MMA retired
-            if (gg == 0 && nw > 0)
-              wait_live(&w_empty[d], (nw - 1) & 1u, abort, P.status, 1);
-            const uint32_t addr = w_s + (32 * i + lane) * 32 + ((c << 4) ^ swz);
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(o[0]),
-                         "r"(o[1]), "r"(o[2]), "r"(o[3])
-                         : "memory");
-          }
-          if (new_x) {
-#pragma unroll
-            for (uint32_t j = 0; j < 2; ++j) {
-              if (j >= n_xch) break;
-              uint4 v = xv[j];
-              if (P.x_f16) {
-                uint32_t in[4] = {v.x, v.y, v.z, v.w}, out[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                  __half2 hv = __floats2half2_rn(__uint_as_float(in[k] << 16),
-                                                 __uint_as_float(in[k] & 0xFFFF0000u));
-                  out[k] = *reinterpret_cast<uint32_t*>(&hv);
+#pragma unroll 1
+            for (uint32_t gg = 0; gg < 8; ++gg) {
+              const uint32_t g = us * 8 + gg;
+              const uint32_t i = gg & 3, c = gg >> 2;
+              uint32_t o[4];
+              if (kDecode) {
+                const uint64_t raw8 = r0;
+                if (kFmt == kFmtBf16Split && (!kConst || !zero_tile)) {
+                  r0 = r1;
+                  r1 = r2;
+                  if (g + 3 < groups) r2 = __ldg(raw_tile + 32 * (g + 3));
                 }
-                v = make_uint4(out[0], out[1], out[2], out[3]);
+                uint32_t e[8];
+                if (kConst) {
+#pragma unroll
+                  for (int k = 0; k < 8; ++k) e[k] = const_e;
+                } else {
+                  rp_group(pipe, tc.pos, lane, abort, P.status);
+#pragma unroll
+                  for (int k = 0; k < 8; ++k) e[k] = decode_step(tc.x, tc.pos, lut_s, pipe.ring_s, lt);
+                }
+                if (kFmt == kFmtBf16Split) fmt_bf16_split(e, raw8, o);
+                else if (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
+                else if (kFmt == kFmtInt4F16Group)
+                  fmt_int4_f16_scaled(e, i == 0 ? gs0 : i == 1 ? gs1 : i == 2 ? gs2 : gs3, o);
+                else fmt_fp8_f16(e, o);
+                if (kConst && zero_tile) o[0] = o[1] = o[2] = o[3] = 0;
+              } else {
+                uint4 v = cp[0];
+#pragma unroll
+                for (int q = 1; q < 8; ++q)
+                  if (gg == static_cast<uint32_t>(q)) v = cp[q];
+                if (kFmt == kFmtBf16Split) {
+                  o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+                } else {
+                  uint32_t e[8];
+                  if (kFmt == kFmtFp8F16) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                      e[k] = ((v.x >> (8 * k)) & 0xFFu) << 12;
+                      e[k + 4] = ((v.y >> (8 * k)) & 0xFFu) << 12;
+                    }
+                    fmt_fp8_f16(e, o);
+                  } else {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) e[k] = (((v.x >> (4 * k)) & 0xFu) ^ 8u) << 12;
+                    if (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
+                    else fmt_int4_f16_scaled(e, i == 0 ? gs0 : i == 1 ? gs1 : i == 2 ? gs2 : gs3, o);
+                  }
+                }
               }
-              const uint32_t r = (lane >> 1) + 16 * j, c = lane & 1u;
-              const uint32_t addr = x_s + r * 32 + ((c ^ ((r >> 2) & 1u)) << 4);
-              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x),
-                           "r"(v.y), "r"(v.z), "r"(v.w)
+              // the slot (and the X slab) are free once the previous MMA retired
+              if (gg == 0 && nw > 0)
+                wait_live(&w_empty[d], (nw - 1) & 1u, abort, P.status, 1);
+              const uint32_t addr = w_s + (32 * i + lane) * 32 + ((c << 4) ^ swz);
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(o[0]),
+                           "r"(o[1]), "r"(o[2]), "r"(o[3])
                            : "memory");
             }
+            if (new_x) {
+#pragma unroll
+              for (uint32_t j = 0; j < 2; ++j) {
+                if (j >= n_xch) break;
+                uint4 v = xv[j];
+                if (P.x_f16) {
+                  uint32_t in[4] = {v.x, v.y, v.z, v.w}, out[4];
+#pragma unroll
+                  for (int k = 0; k < 4; ++k) {
+                    __half2 hv = __floats2half2_rn(__uint_as_float(in[k] << 16),
+                                                   __uint_as_float(in[k] & 0xFFFF0000u));
+                    out[k] = *reinterpret_cast<uint32_t*>(&hv);
+                  }
+                  v = make_uint4(out[0], out[1], out[2], out[3]);
+                }
+                const uint32_t r = (lane >> 1) + 16 * j, c = lane & 1u;
+                const uint32_t addr = x_s + r * 32 + ((c ^ ((r >> 2) & 1u)) << 4);
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x),
+                             "r"(v.y), "r"(v.z), "r"(v.w)
+                             : "memory");
+              }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tc_fence_after();
+              const uint32_t col = (cur_slot * H + h) * T;
+              umma_f16(tmem_base + col, adesc, bdesc, P.idesc, ((fresh >> h) & 1u) ? 0u : 1u);
+              umma_commit(&w_empty[d]);
+            }
+            fresh &= ~(1u << h);
+            ++nw;
           }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tc_fence_after();
-            const uint32_t col = (cur_slot * H + h) * T;
-            umma_f16(tmem_base + col, adesc, bdesc, P.idesc, ((fresh >> h) & 1u) ? 0u : 1u);
-            umma_commit(&w_empty[d]);
-          }
-          fresh &= ~(1u << h);
-          ++nw;
-        }
+        };
+        if (kDecode && (zero_tile || single)) run_slabs(std::true_type{});
+        else run_slabs(std::false_type{});
         if (kDecode && !zero_tile && !run_tile_end(tc, single) && lane == 0)
           atomicOr(P.status, kStatusCorrupt);
       }
