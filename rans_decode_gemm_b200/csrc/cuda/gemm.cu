@@ -575,7 +575,7 @@ bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool dec
     p.n_segments = L.N / L.tile_n;
     p.grid = static_cast<uint32_t>(p.n_units < sms ? p.n_units : sms);
     const uint64_t per_cta = (p.n_units + p.grid - 1) / p.grid;
-    uint32_t D = D_cap;
+    uint32_t D = D_cap < kLocalProducersMax ? D_cap : kLocalProducersMax;
     if (D > per_cta) D = static_cast<uint32_t>(per_cta);
     for (; D >= 1; --D) {
       const uint32_t slots = local_slots(static_cast<uint32_t>(p.n_units), p.grid, D, L.n_kt);
@@ -583,16 +583,16 @@ bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool dec
       uint32_t off = lut_bytes;
       off = round_up(off, 1024);
       const uint32_t off_w = off;
-      off += D * kSlabBytes;
+      off += 2 * D * kSlabBytes;  // two W slabs per producer
       off = round_up(off, 2048);
       const uint32_t off_chunk = off;
       off += (D + 1) * kRingBytes;
       off = round_up(off, 1024);
       const uint32_t off_x = off;
-      off += D * p.T * 32;
+      off += 2 * D * p.T * 32;  // two X slabs per producer
       off = round_up(off, 8);
       const uint32_t off_bars = off;
-      off += (5 * D + slots) * 8;
+      off += (8 * D + 1 + slots) * 8;
       if (cols <= 512 && off <= kSmemLimit) {
         p.local = 1;
         p.D = D;

@@ -1,5 +1,5 @@
 // gemm_local.cu -- fused tile-rANS decode + GEMM for small token counts
-// (M <= 32), where every producer warp drives the tensor core itself.
+// (M <= 32): private accumulators per producer warp, one issuing warp.
 //
 // "Approaching Shannon Bound with Lossless LLM Weight Compression", s3.1
 // "整体执行模型": decoder warps decode compressed tiles straight into shared
@@ -11,18 +11,24 @@
 //   * The units (tiles) are split into one contiguous range per CTA and,
 //     inside it, one contiguous sub-range per producer warp, so a producer
 //     streams one contiguous run of compressed bytes (RunPipe).
-//   * A producer decodes a 128 x 16 slab of W into its own shared-memory slot,
-//     writes the matching 16-column slab of X next to it, and its lane 0
-//     issues the tcgen05.mma into the producer's own TMEM accumulator; the
-//     MMA's completion (tcgen05.commit) frees the slots for the next slab.
+//   * A producer decodes a 128 x 16 slab of W into one of its two
+//     shared-memory slots, writes the matching 16-column slab of X next to
+//     it and signals the slab on an mbarrier.  The store of each group of 8
+//     decoded columns is deferred until the next group's first decode step
+//     has been issued, so it overlaps the decode chain.
+//   * One issuing warp (one lane per producer) hands every ready slab to the
+//     tensor core as soon as it is signalled -- tcgen05.mma issues are
+//     serialised per SM, so producers never wait in that queue -- into the
+//     producer's own TMEM accumulator, in that producer's slab order; the
+//     MMA's completion (tcgen05.commit) frees the slot.
 //   * A producer owns one accumulator per W row-block segment it touches, so
-//     an accumulator is written by one warp in a fixed order and read once;
-//     no warp waits for the epilogue.  The epilogue sums the accumulators of
-//     a segment in ascending unit order, then stores Y or takes part in the
-//     deterministic split-K reduction (gemm_common.cuh).  Every addition
-//     happens in an order fixed by the schedule, so Y is bit-identical to
-//     the same kernel fed uncompressed weights.
-// Warps: 0-3 epilogue (TMEM lanes 0-127), 4 .. 4 + D - 1 producers.
+//     an accumulator is written in a fixed order and read once; no warp waits
+//     for the epilogue.  The epilogue sums the accumulators of a segment in
+//     ascending unit order, then stores Y or takes part in the deterministic
+//     split-K reduction (gemm_common.cuh).  Every addition happens in an
+//     order fixed by the schedule, so Y is bit-identical to the same kernel
+//     fed uncompressed weights.
+// Warps: 0-3 epilogue (TMEM lanes 0-127), 4 MMA issue, 5 .. 5 + D - 1 producers.
 #include <cuda_runtime.h>
 
 #include <cstring>
@@ -34,8 +40,10 @@
 
 namespace ansdev {
 
-constexpr uint32_t kLocalMaxProducers = 16;
-constexpr uint32_t kLocalThreads = (4 + kLocalMaxProducers) * 32;
+// 5 + 15 = 20 warps: five per SM sub-partition leaves 96 registers a thread
+constexpr uint32_t kLocalMaxProducers = kLocalProducersMax;
+constexpr uint32_t kLocalFixedWarps = 5;
+constexpr uint32_t kLocalThreads = (kLocalFixedWarps + kLocalMaxProducers) * 32;
 constexpr uint32_t kLocalMaxSlots = 32;  // 512 TMEM columns / (H * T >= 16) per accumulator
 
 // Contiguous sub-range of producer d inside the CTA's range [ub, ue) (the
@@ -44,6 +52,25 @@ __device__ __forceinline__ void producer_range(uint32_t ub, uint32_t ue, uint32_
                                                uint32_t* b, uint32_t* e) {
   *b = ub + cta_begin(ue - ub, D, d);
   *e = ub + cta_begin(ue - ub, D, d + 1);
+}
+
+// First accumulator slot of producer d: slots are numbered in unit order, so
+// it follows the segments touched by producers 0 .. d-1.
+__device__ __forceinline__ uint32_t producer_first_slot(uint32_t ub, uint32_t ue, uint32_t D,
+                                                        uint32_t d, uint32_t n_kt) {
+  uint32_t slot = 0;
+  for (uint32_t q = 0; q < d; ++q) {
+    uint32_t b, e;
+    producer_range(ub, ue, D, q, &b, &e);
+    if (e > b) slot += (e - 1) / n_kt - b / n_kt + 1;
+  }
+  return slot;
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, const uint32_t (&o)[4]) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(o[0]), "r"(o[1]),
+               "r"(o[2]), "r"(o[3])
+               : "memory");
 }
 
 template <bool kDecode, uint32_t kFmt>
@@ -64,17 +91,19 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
   const uint32_t n_kt = P.L.n_kt, n_tiles = P.L.n_tiles;
 
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem + P.off_lut);
-  uint8_t* wslots = smem + P.off_w;
+  uint8_t* wslots = smem + P.off_w;   // 2 per producer, kSlabBytes each
   uint8_t* chunks = smem + (((smem_u32(smem + P.off_chunk) + kRingBytes - 1) & ~(kRingBytes - 1)) - smem_u32(smem));
-  uint8_t* xslots = smem + P.off_x;
+  uint8_t* xslots = smem + P.off_x;   // 2 per producer, T * 32 bytes each
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P.off_bars);
-  uint64_t* w_empty = bars;           // D: a producer's slots are free again
-  uint64_t* chunk_bars = bars + D;    // 4 per producer
-  uint64_t* acc_full = bars + 5 * D;  // one per accumulator slot
+  uint64_t* w_full = bars;                // 2 per producer: slab written
+  uint64_t* w_empty = bars + 2 * D;       // 2 per producer: slab consumed by its MMA
+  uint64_t* chunk_bars = bars + 4 * D;    // 4 per producer
+  uint64_t* mma_done = bars + 8 * D;      // every MMA of the CTA retired
+  uint64_t* acc_full = bars + 8 * D + 1;  // one per accumulator slot
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
-    for (uint32_t i = 0; i < 5 * D + P.n_slots; ++i) mbar_init(&bars[i], 1);
+    for (uint32_t i = 0; i < 8 * D + 1 + P.n_slots; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -89,30 +118,18 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
   volatile uint32_t* abort = &abort_flag;
   if (threadIdx.x == 0) trace_mark(P, 0);
 
-  if (warp >= 4) {
+  if (warp >= kLocalFixedWarps) {
     // ============================ producer warps ============================
-    const uint32_t d = warp - 4;
+    const uint32_t d = warp - kLocalFixedWarps;
     uint32_t pb, pe;
     producer_range(ub, ue, D, d, &pb, &pe);
-    // accumulator slots are numbered in unit order: producer d's first slot
-    // follows the segments touched by producers 0 .. d-1
-    uint32_t slot_next = 0;
-    for (uint32_t q = 0; q < d; ++q) {
-      uint32_t b, e;
-      producer_range(ub, ue, D, q, &b, &e);
-      if (e > b) slot_next += (e - 1) / n_kt - b / n_kt + 1;
-    }
     const LayerDev& L = P.L;
     const bool single = L.single_symbol != kNoSymbol;
     const uint32_t lt = lanemask_lt();
     const uint32_t lut_s = smem_u32(lut);
     const uint32_t swz = ((lane >> 2) & 1u) << 4;
-    const uint32_t w_s = smem_u32(wslots + d * kSlabBytes);
-    const uint32_t x_s = smem_u32(xslots + d * T * 32);
-    // descriptor fields shared by both operands: LBO 16 B, SBO 256 B,
-    // version 1, 32-byte swizzle; only the start address differs
-    const uint64_t dhi = (1ull << 16) | (16ull << 32) | (1ull << 46) | (6ull << 61);
-    const uint64_t adesc = dhi | (w_s >> 4), bdesc = dhi | (x_s >> 4);
+    const uint32_t w_s0 = smem_u32(wslots + 2 * d * kSlabBytes);
+    const uint32_t x_s0 = smem_u32(xslots + 2 * d * T * 32);
     const unsigned long long* offsets = reinterpret_cast<const unsigned long long*>(L.offsets);
     const uint32_t S = L.tile_n * L.tile_k;
     const uint32_t n_xch = T / 16;  // 16-byte X chunks per lane per slab (1 or 2)
@@ -120,9 +137,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
     rp_init(pipe, chunks + d * kRingBytes, chunk_bars + 4 * d);
     TileCursor tc;
     tc.x = tc.pos = tc.cb = tc.bytes = 0;
-    uint32_t nw = 0;  // slabs handed to the tensor core
-    uint32_t cur_seg = 0xFFFFFFFFu;
-    uint32_t cur_slot = 0, fresh = 0;
+    uint32_t nw = 0;  // slabs signalled to the issuing warp
 
     uint32_t u = pb;
     while (u < pe) {
@@ -140,13 +155,6 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
       }
       for (; u < run_e; ++u) {
         const uint32_t t = u - p * n_tiles;
-        const uint32_t seg = u / n_kt;
-        if (seg != cur_seg) {
-          if (cur_seg != 0xFFFFFFFFu && lane == 0) umma_commit(&acc_full[cur_slot]);
-          cur_slot = slot_next++;
-          cur_seg = seg;
-          fresh = (1u << H) - 1u;
-        }
         const uint32_t rb = t / n_kt, kt = t - rb * n_kt;
         const uint32_t n0 = rb * L.tile_n, k0 = kt * L.tile_k;
         bool zero_tile = false;
@@ -187,7 +195,6 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
           r1 = __ldg(raw_tile + 32);
           r2 = __ldg(raw_tile + 64);
         }
-
         // the slabs of this tile; a tile of constant symbols (single-symbol
         // codebook, or zeros for a tile with bad offsets) takes a separate
         // instantiation so the decoding path carries no per-group branches
@@ -196,27 +203,26 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
           constexpr bool kConst = decltype(const_sym)::value;
           for (uint32_t us = 0; us < H * C; ++us) {
             const uint32_t h = us % H, s = us / H;
-            __half2 gs0, gs1, gs2, gs3;
+            const uint32_t slot = nw & 1u;
+            const uint32_t w_s = w_s0 + slot * kSlabBytes, x_s = x_s0 + slot * T * 32;
+            __half2 gsc[4];
             if (kFmt == kFmtInt4F16Group) {
-              gs0 = h ? gscale[4] : gscale[0];
-              gs1 = h ? gscale[5] : gscale[1];
-              gs2 = h ? gscale[6] : gscale[2];
-              gs3 = h ? gscale[7] : gscale[3];
+              gsc[0] = h ? gscale[4] : gscale[0];
+              gsc[1] = h ? gscale[5] : gscale[1];
+              gsc[2] = h ? gscale[6] : gscale[2];
+              gsc[3] = h ? gscale[7] : gscale[3];
             }
             // X slab s of this unit (T rows x 16 columns): this lane's chunks,
-            // fetched now and stored next to the W slab before the MMA
+            // fetched now and stored next to the W slab at its end
             uint4 xv[2];
-            const bool new_x = (h == 0);
-            if (new_x) {
 #pragma unroll
-              for (uint32_t j = 0; j < 2; ++j) {
-                xv[j] = make_uint4(0, 0, 0, 0);
-                const uint32_t r = (lane >> 1) + 16 * j, c = lane & 1u;
-                const uint32_t m = p * P.T_pass + r;
-                if (j < n_xch && m < P.M)
-                  xv[j] = __ldg(reinterpret_cast<const uint4*>(P.X + static_cast<uint64_t>(m) * L.K + k0 +
-                                                               16 * s + 8 * c));
-              }
+            for (uint32_t j = 0; j < 2; ++j) {
+              xv[j] = make_uint4(0, 0, 0, 0);
+              const uint32_t r = (lane >> 1) + 16 * j, c = lane & 1u;
+              const uint32_t m = p * P.T_pass + r;
+              if (j < n_xch && m < P.M)
+                xv[j] = __ldg(reinterpret_cast<const uint4*>(P.X + static_cast<uint64_t>(m) * L.K + k0 +
+                                                             16 * s + 8 * c));
             }
             uint4 cp[8];
             if (!kDecode) {
@@ -236,10 +242,19 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
                 }
               }
             }
-#pragma unroll 1
+            // the store of group gg - 1 (deferred); the first store into the
+            // slot waits for the MMA that last read it (slab nw - 2)
+            uint32_t o_prev[4] = {0, 0, 0, 0};
+            auto store_prev = [&](uint32_t gg) {
+              if (gg == 1 && nw >= 2)
+                wait_live(&w_empty[2 * d + slot], ((nw >> 1) + 1) & 1u, abort, P.status, 1);
+              const uint32_t i = (gg - 1) & 3, c = (gg - 1) >> 2;
+              sts128(w_s + (32 * i + lane) * 32 + ((c << 4) ^ swz), o_prev);
+            };
+#pragma unroll
             for (uint32_t gg = 0; gg < 8; ++gg) {
               const uint32_t g = us * 8 + gg;
-              const uint32_t i = gg & 3, c = gg >> 2;
+              const uint32_t i = gg & 3;
               uint32_t o[4];
               if (kDecode) {
                 const uint64_t raw8 = r0;
@@ -252,22 +267,21 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
                 if (kConst) {
 #pragma unroll
                   for (int k = 0; k < 8; ++k) e[k] = const_e;
+                  if (gg > 0) store_prev(gg);
                 } else {
                   rp_group(pipe, tc.pos, lane, abort, P.status);
+                  e[0] = decode_step(tc.x, tc.pos, lut_s, pipe.ring_s, lt);
+                  if (gg > 0) store_prev(gg);
 #pragma unroll
-                  for (int k = 0; k < 8; ++k) e[k] = decode_step(tc.x, tc.pos, lut_s, pipe.ring_s, lt);
+                  for (int k = 1; k < 8; ++k) e[k] = decode_step(tc.x, tc.pos, lut_s, pipe.ring_s, lt);
                 }
                 if (kFmt == kFmtBf16Split) fmt_bf16_split(e, raw8, o);
                 else if (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
-                else if (kFmt == kFmtInt4F16Group)
-                  fmt_int4_f16_scaled(e, i == 0 ? gs0 : i == 1 ? gs1 : i == 2 ? gs2 : gs3, o);
+                else if (kFmt == kFmtInt4F16Group) fmt_int4_f16_scaled(e, gsc[i], o);
                 else fmt_fp8_f16(e, o);
                 if (kConst && zero_tile) o[0] = o[1] = o[2] = o[3] = 0;
               } else {
-                uint4 v = cp[0];
-#pragma unroll
-                for (int q = 1; q < 8; ++q)
-                  if (gg == static_cast<uint32_t>(q)) v = cp[q];
+                const uint4 v = cp[gg];
                 if (kFmt == kFmtBf16Split) {
                   o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
                 } else {
@@ -283,49 +297,37 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
 #pragma unroll
                     for (int k = 0; k < 8; ++k) e[k] = (((v.x >> (4 * k)) & 0xFu) ^ 8u) << 12;
                     if (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
-                    else fmt_int4_f16_scaled(e, i == 0 ? gs0 : i == 1 ? gs1 : i == 2 ? gs2 : gs3, o);
+                    else fmt_int4_f16_scaled(e, gsc[i], o);
                   }
                 }
+                if (gg > 0) store_prev(gg);
               }
-              // the slot (and the X slab) are free once the previous MMA retired
-              if (gg == 0 && nw > 0)
-                wait_live(&w_empty[d], (nw - 1) & 1u, abort, P.status, 1);
-              const uint32_t addr = w_s + (32 * i + lane) * 32 + ((c << 4) ^ swz);
-              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(o[0]),
-                           "r"(o[1]), "r"(o[2]), "r"(o[3])
-                           : "memory");
+#pragma unroll
+              for (int k = 0; k < 4; ++k) o_prev[k] = o[k];
             }
-            if (new_x) {
+            store_prev(8);
+            // X slab, then hand the slab to the issuing warp
 #pragma unroll
-              for (uint32_t j = 0; j < 2; ++j) {
-                if (j >= n_xch) break;
-                uint4 v = xv[j];
-                if (P.x_f16) {
-                  uint32_t in[4] = {v.x, v.y, v.z, v.w}, out[4];
+            for (uint32_t j = 0; j < 2; ++j) {
+              if (j >= n_xch) break;
+              uint4 v = xv[j];
+              if (P.x_f16) {
+                uint32_t in[4] = {v.x, v.y, v.z, v.w}, out[4];
 #pragma unroll
-                  for (int k = 0; k < 4; ++k) {
-                    __half2 hv = __floats2half2_rn(__uint_as_float(in[k] << 16),
-                                                   __uint_as_float(in[k] & 0xFFFF0000u));
-                    out[k] = *reinterpret_cast<uint32_t*>(&hv);
-                  }
-                  v = make_uint4(out[0], out[1], out[2], out[3]);
+                for (int k = 0; k < 4; ++k) {
+                  __half2 hv = __floats2half2_rn(__uint_as_float(in[k] << 16),
+                                                 __uint_as_float(in[k] & 0xFFFF0000u));
+                  out[k] = *reinterpret_cast<uint32_t*>(&hv);
                 }
-                const uint32_t r = (lane >> 1) + 16 * j, c = lane & 1u;
-                const uint32_t addr = x_s + r * 32 + ((c ^ ((r >> 2) & 1u)) << 4);
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x),
-                             "r"(v.y), "r"(v.z), "r"(v.w)
-                             : "memory");
+                v = make_uint4(out[0], out[1], out[2], out[3]);
               }
+              const uint32_t r = (lane >> 1) + 16 * j, c = lane & 1u;
+              const uint32_t xo[4] = {v.x, v.y, v.z, v.w};
+              sts128(x_s + r * 32 + ((c ^ ((r >> 2) & 1u)) << 4), xo);
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) {
-              tc_fence_after();
-              const uint32_t col = (cur_slot * H + h) * T;
-              umma_f16(tmem_base + col, adesc, bdesc, P.idesc, ((fresh >> h) & 1u) ? 0u : 1u);
-              umma_commit(&w_empty[d]);
-            }
-            fresh &= ~(1u << h);
+            if (lane == 0) mbar_arrive(&w_full[2 * d + slot]);
             ++nw;
           }
         };
@@ -335,11 +337,90 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
           atomicOr(P.status, kStatusCorrupt);
       }
     }
-    if (cur_seg != 0xFFFFFFFFu && lane == 0) umma_commit(&acc_full[cur_slot]);
-    // the last commit's arrival lands before the warp leaves
-    if (nw > 0) wait_drain(&w_empty[d], (nw - 1) & 1u, P.status);
     if (kDecode) rp_drain(pipe, P.status);
     if (lane == 0) trace_mark(P, 18 + d);
+  } else if (warp == 4) {
+    // ================== MMA issue (lane q follows producer q) ==================
+    const uint32_t q = lane;
+    uint32_t pb = 0, pe = 0;
+    if (q < D) producer_range(ub, ue, D, q, &pb, &pe);
+    uint32_t acc_slot = q < D ? producer_first_slot(ub, ue, D, q, n_kt) : 0u;
+    uint32_t u = pb, us = 0, nslab = 0;
+    uint32_t cur_seg = pb / n_kt;
+    uint32_t fresh = (1u << H) - 1u;  // bit h: next MMA into half h starts the accumulator
+    const uint32_t n_us = H * C;
+    // descriptor fields shared by both operands: LBO 16 B, SBO 256 B,
+    // version 1, 32-byte swizzle; only the start address differs
+    const uint64_t dhi = (1ull << 16) | (16ull << 32) | (1ull << 46) | (6ull << 61);
+    const uint32_t w_base = smem_u32(wslots), x_base = smem_u32(xslots);
+    long long idle_since = clock64();
+    for (;;) {
+      const bool has = q < D && u < pe;
+      if (__ballot_sync(0xFFFFFFFFu, has) == 0) break;
+      const uint32_t slot = nslab & 1u;
+      const bool ready = has && mbar_try_wait(&w_full[2 * q + slot], (nslab >> 1) & 1u);
+      uint32_t rmask = __ballot_sync(0xFFFFFFFFu, ready);
+      if (rmask == 0) {
+        if (*abort) break;
+        if (clock64() - idle_since > kWaitBudgetCycles) {
+          if (lane == 0) {
+            *abort = 1u;
+            atomicOr(P.status, kStatusTimeout | (1u << (8 + 2)));
+          }
+          break;
+        }
+        __nanosleep(32);
+        continue;
+      }
+      idle_since = clock64();
+      if (lane == 0 && P.trace) {
+        unsigned long long tnow;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(tnow));
+        if (P.trace[blockIdx.x * 64 + 36] == 0) P.trace[blockIdx.x * 64 + 36] = tnow;
+        P.trace[blockIdx.x * 64 + 37] += __popc(rmask);
+        P.trace[blockIdx.x * 64 + 39] += 1;
+      }
+      // this lane's slab: accumulator columns, accumulate flag, segment end
+      const uint32_t h = us % H;
+      const uint32_t col = (acc_slot * H + h) * T;
+      const uint32_t accum = ((fresh >> h) & 1u) ? 0u : 1u;
+      const bool seg_end = (us + 1 == n_us) && (u + 1 == pe || (u + 1) / n_kt != cur_seg);
+      const uint32_t info = slot | (accum << 1) | ((seg_end ? 1u : 0u) << 2);
+      tc_fence_after();
+      while (rmask) {
+        const uint32_t r = __ffs(rmask) - 1;
+        rmask &= rmask - 1;
+        const uint32_t c_r = __shfl_sync(0xFFFFFFFFu, col, r);
+        const uint32_t i_r = __shfl_sync(0xFFFFFFFFu, info, r);
+        const uint32_t k_r = __shfl_sync(0xFFFFFFFFu, acc_slot, r);
+        if (lane == 0) {
+          const uint32_t s_r = i_r & 1u;
+          const uint64_t adesc = dhi | ((w_base + (2 * r + s_r) * kSlabBytes) >> 4);
+          const uint64_t bdesc = dhi | ((x_base + (2 * r + s_r) * T * 32) >> 4);
+          umma_f16(tmem_base + c_r, adesc, bdesc, P.idesc, (i_r >> 1) & 1u);
+          umma_commit(&w_empty[2 * r + s_r]);
+          if (i_r & 4u) umma_commit(&acc_full[k_r]);
+        }
+        __syncwarp();
+      }
+      if (ready) {
+        fresh &= ~(1u << h);
+        ++nslab;
+        if (++us == n_us) {
+          us = 0;
+          ++u;
+          if (u < pe && u / n_kt != cur_seg) {
+            cur_seg = u / n_kt;
+            ++acc_slot;
+            fresh = (1u << H) - 1u;
+          }
+        }
+      }
+    }
+    if (lane == 0) trace_mark(P, 35);
+    // retirement of every MMA this CTA issued (waited for before TMEM is freed)
+    if (lane == 0) umma_commit(mma_done);
+    __syncwarp();
   } else {
     // ===================== epilogue (warps 0-3, 128 threads) =====================
     const uint32_t e = threadIdx.x;   // TMEM lane = row within the 128-row half
@@ -415,11 +496,12 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
     }
   }
 
-  // ---- teardown: every MMA retired (the epilogue consumed every accumulator)
+  // ---- teardown: every MMA retired before TMEM is released
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0) trace_mark(P, 41);
   if (warp == 0) {
+    wait_drain(mma_done, 0, P.status);
     tc_fence_after();
     tmem_dealloc(tmem_base, P.tmem_cols);
   }
@@ -438,7 +520,7 @@ static cudaError_t launch_local_variant(const GemmPlan& plan, const GemmDev& P, 
     if (e != cudaSuccess) return e;
     attr_set[dev] = 1;
   }
-  kern<<<plan.grid, (4 + plan.D) * 32, plan.smem_bytes, stream>>>(P);
+  kern<<<plan.grid, (kLocalFixedWarps + plan.D) * 32, plan.smem_bytes, stream>>>(P);
   return cudaGetLastError();
 }
 

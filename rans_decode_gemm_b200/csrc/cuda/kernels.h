@@ -84,6 +84,9 @@ constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
 // device; see noalloc.cu).
 cudaError_t noalloc_scratch(void** ptr);
 
+// Producer warps per CTA of the local schedule (gemm_local.cu).
+constexpr uint32_t kLocalProducersMax = 15;
+
 // Local schedule (gemm_local.cu): launches the kernel for an already filled
 // GemmDev.
 cudaError_t launch_gemm_local(const GemmPlan& plan, const GemmDev& P, bool decode,
