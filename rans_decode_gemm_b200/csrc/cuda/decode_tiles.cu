@@ -10,6 +10,7 @@
 #include <cuda_runtime.h>
 
 #include "kernels.h"
+#include "launch.h"
 #include "rans_core.cuh"
 
 namespace ansdev {
@@ -65,6 +66,10 @@ __global__ void __launch_bounds__(kDecMaxWarps * 32, 2)
   }
   if (!single) build_lut(lut, L, warp, nwarps, lane);
   __syncthreads();
+  // the prologue above read only kernel parameters: from here on global
+  // memory, after the previous grid in the stream has completed
+  griddep_wait();
+  griddep_launch_dependents();
 
   volatile uint32_t* abort = &abort_flag;
   const uint32_t lt = lanemask_lt();
@@ -192,8 +197,8 @@ static cudaError_t launch_decode_variant(const LayerDev& L, void* out, uint32_t*
   cudaError_t e = cudaFuncSetAttribute(decode_tiles_kernel<DT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem);
   if (e != cudaSuccess) return e;
-  decode_tiles_kernel<DT><<<blocks, warps * 32, kDecSmem, stream>>>(L, out, status);
-  return cudaGetLastError();
+  return launch_pdl(decode_tiles_kernel<DT>, dim3(blocks), dim3(warps * 32), kDecSmem, stream, L,
+                    out, status);
 }
 
 cudaError_t launch_decode_tiles(const LayerDev& L, void* out, uint32_t* status,

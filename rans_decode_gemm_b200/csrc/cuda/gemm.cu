@@ -30,6 +30,7 @@
 
 #include "gemm_common.cuh"
 #include "kernels.h"
+#include "launch.h"
 #include "rans_core.cuh"
 
 namespace ansdev {
@@ -119,6 +120,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
   __shared__ uint32_t tmem_slot;
   __shared__ uint32_t abort_flag;
   __shared__ uint32_t reduce_flag;
+  __shared__ uint32_t red_n, red_seg[2];  // split-K segments of this CTA
 
   const uint32_t warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t D = P.D, XS = P.x_stages;
@@ -137,6 +139,8 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
+    red_n = 0;
+    reduce_flag = 0;
     for (uint32_t i = 0; i < 2 * D; ++i) { mbar_init(&B.w_full[i], 1); mbar_init(&B.w_empty[i], 1); }
     for (uint32_t i = 0; i < XS; ++i) { mbar_init(&B.x_full[i], 1); mbar_init(&B.x_empty[i], 1); }
     for (uint32_t i = 0; i < 2; ++i) { mbar_init(&B.acc_full[i], 1); mbar_init(&B.acc_empty[i], 4); }
@@ -154,6 +158,10 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = tmem_slot;
   volatile uint32_t* abort = &abort_flag;
+  // the prologue above read only kernel parameters: from here on global
+  // memory, after the previous grid in the stream (X staging) has completed
+  griddep_wait();
+  griddep_launch_dependents();
   if (threadIdx.x == 0) trace_mark(P, 0);
 
   if (warp >= kFixedWarps) {
@@ -422,6 +430,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     // ======================= epilogue (warps 0-3, 128 threads) =======================
     const uint32_t e = threadIdx.x;  // TMEM lane = row within the 128-row half
     const uint32_t seg_first = u_begin / n_kt, seg_last = (u_end - 1) / n_kt;
+    uint32_t pend[2], npend = 0;  // segments shared with other CTAs (first, last)
     for (uint32_t seg = seg_first; seg <= seg_last; ++seg) {
       const uint32_t lseg = static_cast<uint32_t>(seg - seg_first);
       const uint32_t buf = lseg % P.n_bufs;
@@ -453,7 +462,15 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&B.acc_empty[buf]);
-      if (!complete) splitk_finish(P, seg, p, rb, e, &reduce_flag);
+      if (!complete) pend[npend++] = seg;
+    }
+    // split-K arrival once every partial of this CTA is written; the
+    // reductions this CTA owns run after the CTA barrier, on every thread
+    if (npend) splitk_arrive(P, pend, npend, e, &reduce_flag);
+    if (e == 0) {
+      red_n = npend;
+      red_seg[0] = pend[0];
+      red_seg[1] = pend[1];
     }
   }
 
@@ -466,6 +483,12 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, P.tmem_cols);
   }
+  // the split-K reductions this CTA arrived last for, on every thread
+  if (reduce_flag) {
+    __threadfence();
+    for (uint32_t k = 0; k < red_n; ++k)
+      if ((reduce_flag >> k) & 1u) splitk_reduce(P, red_seg[k], threadIdx.x, blockDim.x);
+  }
 }
 
 // Stages X for the fused kernel: for every token pass p and 16-column slab
@@ -476,6 +499,8 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
 __global__ void x_stage_kernel(const uint16_t* __restrict__ X, uint8_t* __restrict__ xs,
                                uint32_t M, uint32_t K, uint32_t T_pass, uint32_t n_pass,
                                uint32_t to_f16) {
+  griddep_wait();
+  griddep_launch_dependents();
   const uint64_t n_chunks = static_cast<uint64_t>(n_pass) * (K / 16) * T_pass * 2;
   for (uint64_t i = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_chunks;
        i += static_cast<uint64_t>(gridDim.x) * blockDim.x) {
@@ -706,8 +731,8 @@ static cudaError_t launch_variant(const GemmPlan& plan, const GemmDev& P, cudaSt
     if (e != cudaSuccess) return e;
     attr_set[dev] = 1;
   }
-  kern<<<plan.grid, (kFixedWarps + plan.D) * 32, plan.smem_bytes, stream>>>(P);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(plan.grid), dim3((kFixedWarps + plan.D) * 32), plan.smem_bytes,
+                    stream, P);
 }
 
 cudaError_t launch_gemm(const GemmPlan& plan, const LayerDev& L, bool decode, const void* w_plain,
@@ -725,9 +750,9 @@ cudaError_t launch_gemm(const GemmPlan& plan, const LayerDev& L, bool decode, co
     uint32_t blocks = static_cast<uint32_t>((n_chunks + 255) / 256);
     if (blocks > 4096) blocks = 4096;
     if (blocks == 0) blocks = 1;
-    x_stage_kernel<<<blocks, 256, 0, stream>>>(X, reinterpret_cast<uint8_t*>(x16), plan.M, L.K,
-                                               plan.T_pass, plan.n_pass, plan.ab_f16);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(x_stage_kernel, dim3(blocks), dim3(256), 0, stream, X,
+                               reinterpret_cast<uint8_t*>(x16), plan.M, L.K, plan.T_pass,
+                               plan.n_pass, plan.ab_f16);
     if (e != cudaSuccess) return e;
   }
 

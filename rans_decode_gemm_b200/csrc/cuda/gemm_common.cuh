@@ -73,45 +73,111 @@ __device__ __forceinline__ void epi_emit16(const GemmDev& P, const float (&v)[16
   }
 }
 
-// Split-K over CTAs for segment seg (token pass p, W row block rb), run by
-// the 128 epilogue threads of every contributing CTA after its partials are
-// written: the last CTA to arrive sums the contributors' partials in
-// ascending CTA order (so the result does not depend on timing) and writes Y.
-// Only the first contributor can hold the segment in its second (tail)
-// partial slot, when its range started before the segment.
-__device__ __forceinline__ void splitk_finish(const GemmDev& P, uint32_t seg, uint32_t p,
-                                              uint32_t rb, uint32_t e,
-                                              volatile uint32_t* reduce_flag) {
+// Split-K over CTAs.  A W row block's segment seg (token pass p, row block
+// rb) that spans several CTAs is summed in a fixed order: every contributor
+// writes its partial sums, then counts itself in counters[seg]; the last CTA
+// to arrive adds the contributors' partials in ascending CTA order (so the
+// result does not depend on timing) and writes Y.  A CTA holds at most two
+// such segments: its first (partial slot 0) and its last (slot 1); only the
+// first contributor of a segment can hold it in its slot 1, when its range
+// started before the segment.
+
+// Arrival: run by the 128 epilogue threads once all of this CTA's partials
+// are written.  Returns (to every thread) a bit per segment for which this
+// CTA arrived last and must reduce.
+__device__ __forceinline__ uint32_t splitk_arrive(const GemmDev& P, const uint32_t* segs,
+                                                  uint32_t n, uint32_t e,
+                                                  volatile uint32_t* reduce_flag) {
   const uint32_t G = gridDim.x, n_kt = P.L.n_kt, U = static_cast<uint32_t>(P.n_units);
-  const uint32_t s_lo = seg * n_kt, s_hi = s_lo + n_kt;
-  __threadfence();
   named_bar_sync(1, 128);
-  const uint32_t c_first = cta_of(U, G, s_lo);
-  const uint32_t c_last = cta_of(U, G, s_hi - 1);
   if (e == 0) {
-    const uint32_t old = atomicAdd(&P.counters[seg], 1u);
-    *reduce_flag = (old == c_last - c_first) ? 1u : 0u;
+    // one gpu-scope fence after the barrier covers the partials every
+    // epilogue thread wrote before it (fences are cumulative)
+    __threadfence();
+    uint32_t bits = 0;
+    for (uint32_t k = 0; k < n; ++k) {
+      const uint32_t s_lo = segs[k] * n_kt;
+      const uint32_t c_first = cta_of(U, G, s_lo), c_last = cta_of(U, G, s_lo + n_kt - 1);
+      const uint32_t old = atomicAdd(&P.counters[segs[k]], 1u);
+      if (old == c_last - c_first) bits |= 1u << k;
+    }
+    *reduce_flag = bits;
   }
   named_bar_sync(1, 128);
-  if (*reduce_flag) {
-    __threadfence();
-    const uint32_t sl_first = (cta_begin(U, G, c_first) < s_lo) ? 1u : 0u;
-    const uint64_t cta_stride = 2ull * P.H * P.T_pass * 128;
-    const uint32_t t_valid = min(P.T_pass, P.M - p * P.T_pass);
-    const uint32_t n_items = P.H * t_valid * 32;  // float4 items: (h, token, 4 rows)
-    const float* first = P.partials + c_first * cta_stride + sl_first * (cta_stride / 2);
-    for (uint32_t it0 = e; it0 < n_items; it0 += 4 * 128) {
+  return *reduce_flag;
+}
+
+// Reduction of segment seg by the CTA that arrived last, run by threads
+// tid = 0 .. nthr - 1 of that CTA (the whole CTA, once its other work is
+// done).
+__device__ __forceinline__ void splitk_reduce(const GemmDev& P, uint32_t seg, uint32_t tid,
+                                              uint32_t nthr) {
+  const uint32_t G = gridDim.x, n_kt = P.L.n_kt, U = static_cast<uint32_t>(P.n_units);
+  const uint32_t p = seg / P.n_rb, rb = seg % P.n_rb;
+  const uint32_t s_lo = seg * n_kt, s_hi = s_lo + n_kt;
+  const uint32_t c_first = cta_of(U, G, s_lo);
+  const uint32_t c_last = cta_of(U, G, s_hi - 1);
+  const uint32_t sl_first = (cta_begin(U, G, c_first) < s_lo) ? 1u : 0u;
+  const uint64_t cta_stride = 2ull * P.H * P.T_pass * 128;
+  const uint32_t t_valid = min(P.T_pass, P.M - p * P.T_pass);
+  const uint32_t n_items = P.H * t_valid * 32;  // float4 items: (h, token, 4 rows)
+  const float* first = P.partials + c_first * cta_stride + sl_first * (cta_stride / 2);
+  // an output item is 4 rows of one token (a float4).  Few items (small M):
+  // one per thread, the loads of up to 8 contributors in flight together;
+  // many items: 4 per thread and pass, 2 contributors at a time.  Either way
+  // the contributors are added in ascending CTA order.
+  auto item_off = [&](uint32_t it, uint32_t* h, uint32_t* tok, uint32_t* q) {
+    *q = it & 31;
+    const uint32_t ht = it >> 5;
+    *h = ht / t_valid;
+    *tok = ht - *h * t_valid;
+    return (static_cast<uint64_t>(*h) * P.T_pass + *tok) * 128 + 4 * *q;
+  };
+  auto store = [&](float4 acc, uint32_t h, uint32_t tok, uint32_t q) {
+    const uint32_t n = rb * P.L.tile_n + h * 128 + 4 * q;
+    if (P.scale_kind == 1) {
+      const uint2 sb = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(P.scales) + n));
+      acc.x *= __uint_as_float(sb.x << 16);
+      acc.y *= __uint_as_float(sb.x & 0xFFFF0000u);
+      acc.z *= __uint_as_float(sb.y << 16);
+      acc.w *= __uint_as_float(sb.y & 0xFFFF0000u);
+    } else if (P.scale_kind == 2) {
+      const float4 sf = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(P.scales) + n));
+      acc.x *= sf.x; acc.y *= sf.y; acc.z *= sf.z; acc.w *= sf.w;
+    }
+    const uint32_t m = p * P.T_pass + tok;
+    *reinterpret_cast<float4*>(P.Y + static_cast<uint64_t>(m) * P.L.N + n) = acc;
+  };
+  if (n_items <= nthr) {
+    for (uint32_t it = tid; it < n_items; it += nthr) {
+      uint32_t h, tok, q;
+      const uint64_t off = item_off(it, &h, &tok, &q);
+      float4 acc = __ldcg(reinterpret_cast<const float4*>(first + off));
+      for (uint32_t c0 = c_first + 1; c0 <= c_last; c0 += 8) {
+        float4 v[8];
+#pragma unroll
+        for (uint32_t k = 0; k < 8; ++k) {
+          const uint32_t cc = min(c0 + k, c_last);
+          v[k] = __ldcg(reinterpret_cast<const float4*>(P.partials + cc * cta_stride + off));
+        }
+#pragma unroll
+        for (uint32_t k = 0; k < 8; ++k) {
+          if (c0 + k > c_last) break;
+          acc.x += v[k].x; acc.y += v[k].y; acc.z += v[k].z; acc.w += v[k].w;
+        }
+      }
+      store(acc, h, tok, q);
+    }
+  } else {
+    for (uint32_t it0 = tid; it0 < n_items; it0 += 4 * nthr) {
       uint64_t off[4];
+      uint32_t hh[4], tt[4], qq[4];
       float4 acc[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const uint32_t it = min(it0 + 128u * u, n_items - 1);
-        const uint32_t q = it & 31, ht = it >> 5;
-        const uint32_t h = ht / t_valid, tok = ht - h * t_valid;
-        off[u] = (static_cast<uint64_t>(h) * P.T_pass + tok) * 128 + 4 * q;
+        off[u] = item_off(min(it0 + nthr * u, n_items - 1), &hh[u], &tt[u], &qq[u]);
         acc[u] = __ldcg(reinterpret_cast<const float4*>(first + off[u]));
       }
-      // the other contributors, two at a time with all their loads in flight
       for (uint32_t c2 = c_first + 1; c2 <= c_last; c2 += 2) {
         const uint32_t cb = min(c2 + 1, c_last);
         float4 v0[4], v1[4];
@@ -132,31 +198,12 @@ __device__ __forceinline__ void splitk_finish(const GemmDev& P, uint32_t seg, ui
         }
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const uint32_t it = it0 + 128u * u;
-        if (it >= n_items) break;
-        const uint32_t q = it & 31, ht = it >> 5;
-        const uint32_t h = ht / t_valid, tok = ht - h * t_valid;
-        const uint32_t n = rb * P.L.tile_n + h * 128 + 4 * q;
-        float4 a = acc[u];
-        if (P.scale_kind == 1) {
-          const uint2 sb = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(P.scales) + n));
-          a.x *= __uint_as_float(sb.x << 16);
-          a.y *= __uint_as_float(sb.x & 0xFFFF0000u);
-          a.z *= __uint_as_float(sb.y << 16);
-          a.w *= __uint_as_float(sb.y & 0xFFFF0000u);
-        } else if (P.scale_kind == 2) {
-          const float4 sf = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(P.scales) + n));
-          a.x *= sf.x; a.y *= sf.y; a.z *= sf.z; a.w *= sf.w;
-        }
-        const uint32_t m = p * P.T_pass + tok;
-        *reinterpret_cast<float4*>(P.Y + static_cast<uint64_t>(m) * P.L.N + n) = a;
-      }
+      for (int u = 0; u < 4; ++u)
+        if (it0 + nthr * u < n_items) store(acc[u], hh[u], tt[u], qq[u]);
     }
-    if (e == 0) P.counters[seg] = 0;
-    if (e == 0) trace_mark(P, 38);
   }
-  named_bar_sync(1, 128);
+  if (tid == 0) P.counters[seg] = 0;
+  if (tid == 0) trace_mark(P, 38);
 }
 
 }  // namespace ansdev

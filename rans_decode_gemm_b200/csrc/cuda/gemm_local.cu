@@ -36,6 +36,7 @@
 
 #include "gemm_common.cuh"
 #include "kernels.h"
+#include "launch.h"
 #include "rans_core.cuh"
 
 namespace ansdev {
@@ -80,6 +81,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
   __shared__ uint32_t tmem_slot;
   __shared__ uint32_t abort_flag;
   __shared__ uint32_t reduce_flag;
+  __shared__ uint32_t red_n, red_seg[2];  // split-K segments of this CTA
   __shared__ uint32_t slot_seg[kLocalMaxSlots];
   __shared__ uint32_t n_cta_slots;
 
@@ -103,6 +105,8 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
+    red_n = 0;
+    reduce_flag = 0;
     for (uint32_t i = 0; i < 8 * D + 1 + P.n_slots; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
   }
@@ -116,6 +120,10 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = tmem_slot;
   volatile uint32_t* abort = &abort_flag;
+  // the prologue above read only kernel parameters: from here on global
+  // memory, after the previous grid in the stream has completed
+  griddep_wait();
+  griddep_launch_dependents();
   if (threadIdx.x == 0) trace_mark(P, 0);
 
   if (warp >= kLocalFixedWarps) {
@@ -379,13 +387,17 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
         if (P.trace[blockIdx.x * 64 + 36] == 0) P.trace[blockIdx.x * 64 + 36] = tnow;
         P.trace[blockIdx.x * 64 + 37] += __popc(rmask);
         P.trace[blockIdx.x * 64 + 39] += 1;
+        P.trace[blockIdx.x * 64 + 42] = tnow;
+        P.trace[blockIdx.x * 64 + 43] = __popc(rmask);
       }
       // this lane's slab: accumulator columns, accumulate flag, segment end
       const uint32_t h = us % H;
       const uint32_t col = (acc_slot * H + h) * T;
       const uint32_t accum = ((fresh >> h) & 1u) ? 0u : 1u;
       const bool seg_end = (us + 1 == n_us) && (u + 1 == pe || (u + 1) / n_kt != cur_seg);
-      const uint32_t info = slot | (accum << 1) | ((seg_end ? 1u : 0u) << 2);
+      // the producer reuses this slot only if it has a slab nslab + 2
+      const bool reuse = nslab + 2 < (pe - pb) * n_us;
+      const uint32_t info = slot | (accum << 1) | ((seg_end ? 1u : 0u) << 2) | ((reuse ? 1u : 0u) << 3);
       tc_fence_after();
       while (rmask) {
         const uint32_t r = __ffs(rmask) - 1;
@@ -398,7 +410,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
           const uint64_t adesc = dhi | ((w_base + (2 * r + s_r) * kSlabBytes) >> 4);
           const uint64_t bdesc = dhi | ((x_base + (2 * r + s_r) * T * 32) >> 4);
           umma_f16(tmem_base + c_r, adesc, bdesc, P.idesc, (i_r >> 1) & 1u);
-          umma_commit(&w_empty[2 * r + s_r]);
+          if (i_r & 8u) umma_commit(&w_empty[2 * r + s_r]);
           if (i_r & 4u) umma_commit(&acc_full[k_r]);
         }
         __syncwarp();
@@ -440,6 +452,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
     named_bar_sync(1, 128);
     const uint32_t ns = n_cta_slots;
     uint32_t nflush = 0;
+    uint32_t pend[2], npend = 0;  // segments shared with other CTAs (first, last)
     for (uint32_t sa = 0; sa < ns;) {
       const uint32_t seg = slot_seg[sa];
       uint32_t sb = sa + 1;
@@ -488,11 +501,19 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
         const float scale = complete ? row_scale(P, n) : 1.0f;
         epi_emit16(P, acc[ck], complete, scale, part, p, h, tok0, n, e);
       }
-      if (e == 0) trace_mark(P, 60 + 2 * min(nflush, 1u));
-      if (!complete) splitk_finish(P, seg, p, rb, e, &reduce_flag);
-      if (e == 0) trace_mark(P, 61 + 2 * min(nflush, 1u));
+      if (e == 0) trace_mark(P, 60 + min(nflush, 1u));
+      if (!complete) pend[npend++] = seg;
       ++nflush;
       sa = sb;
+    }
+    // split-K arrival once every partial of this CTA is written; the
+    // reductions this CTA owns run after the CTA barrier, on every thread
+    if (npend) splitk_arrive(P, pend, npend, e, &reduce_flag);
+    if (e == 0) {
+      trace_mark(P, 62);
+      red_n = npend;
+      red_seg[0] = pend[0];
+      red_seg[1] = pend[1];
     }
   }
 
@@ -504,6 +525,12 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
     wait_drain(mma_done, 0, P.status);
     tc_fence_after();
     tmem_dealloc(tmem_base, P.tmem_cols);
+  }
+  // the split-K reductions this CTA arrived last for, on every thread
+  if (reduce_flag) {
+    __threadfence();
+    for (uint32_t k = 0; k < red_n; ++k)
+      if ((reduce_flag >> k) & 1u) splitk_reduce(P, red_seg[k], threadIdx.x, blockDim.x);
   }
 }
 
@@ -520,8 +547,8 @@ static cudaError_t launch_local_variant(const GemmPlan& plan, const GemmDev& P, 
     if (e != cudaSuccess) return e;
     attr_set[dev] = 1;
   }
-  kern<<<plan.grid, (kLocalFixedWarps + plan.D) * 32, plan.smem_bytes, stream>>>(P);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(plan.grid), dim3((kLocalFixedWarps + plan.D) * 32), plan.smem_bytes,
+                    stream, P);
 }
 
 cudaError_t launch_gemm_local(const GemmPlan& plan, const GemmDev& P, bool decode,

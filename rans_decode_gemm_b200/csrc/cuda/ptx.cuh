@@ -20,6 +20,19 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
                : "memory");
 }
 
+// Programmatic dependent launch.  griddep_wait: block until the grid that
+// precedes this one in the stream has completed and its memory operations are
+// visible (a no-op when the launch did not opt in); every global-memory access
+// of a kernel comes after it.  griddep_launch_dependents: allow the next grid
+// in the stream to start launching (its own griddep_wait still waits for this
+// grid to finish).
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void fence_mbar_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
