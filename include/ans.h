@@ -113,10 +113,10 @@ typedef struct {
 typedef struct {
   ans_layout layout;
   ans_codebook codebook;
-  const uint8_t* stream;   /* offsets[n_tiles] bytes */
+  const uint8_t* stream;   /* offsets[n_tiles] bytes, 16-byte aligned */
   uint64_t stream_bytes;
   const uint64_t* offsets; /* n_tiles + 1 entries */
-  const uint8_t* raw;      /* ANS_BF16_SPLIT only: N*K bytes; else NULL */
+  const uint8_t* raw;      /* ANS_BF16_SPLIT only: N*K bytes, 16-byte aligned; else NULL */
 } ans_tiles;
 
 /* Human-readable name of a status code (static storage). */

@@ -261,7 +261,7 @@ ans_status ans_decode_tiles(const ans_tiles* tiles, void* d_out, uint32_t* d_sta
   if (reinterpret_cast<uintptr_t>(d_out) % 16 != 0 ||
       reinterpret_cast<uintptr_t>(tiles->stream) % 16 != 0 ||
       reinterpret_cast<uintptr_t>(tiles->offsets) % 8 != 0 ||
-      (tiles->raw && reinterpret_cast<uintptr_t>(tiles->raw) % 8 != 0))
+      (tiles->raw && reinterpret_cast<uintptr_t>(tiles->raw) % 16 != 0))
     return ANS_ERR_ARG;
   int sms = 0;
   st = device_info(&sms);
@@ -306,7 +306,7 @@ ans_status ans_gemm(const uint16_t* d_X, uint32_t M, const ans_tiles* W,
   if (W->layout.dtype == ANS_BF16_SPLIT && !W->raw) return ANS_ERR_ARG;
   if (reinterpret_cast<uintptr_t>(W->stream) % 16 != 0 ||
       reinterpret_cast<uintptr_t>(W->offsets) % 8 != 0 ||
-      (W->raw && reinterpret_cast<uintptr_t>(W->raw) % 8 != 0))
+      (W->raw && reinterpret_cast<uintptr_t>(W->raw) % 16 != 0))
     return ANS_ERR_ARG;
   ansdev::LayerDev L;
   fill_layer(W, &L);

@@ -46,6 +46,7 @@ constexpr uint32_t kLocalMaxProducers = kLocalProducersMax;
 constexpr uint32_t kLocalFixedWarps = 5;
 constexpr uint32_t kLocalThreads = (kLocalFixedWarps + kLocalMaxProducers) * 32;
 constexpr uint32_t kLocalMaxSlots = 32;  // 512 TMEM columns / (H * T >= 16) per accumulator
+constexpr uint32_t kRawAhead = 3;        // raw-byte groups loaded ahead of their use
 
 // Contiguous sub-range of producer d inside the CTA's range [ub, ue) (the
 // same balanced split as the CTA ranges).
@@ -99,7 +100,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P.off_bars);
   uint64_t* w_full = bars;                // 2 per producer: slab written
   uint64_t* w_empty = bars + 2 * D;       // 2 per producer: slab consumed by its MMA
-  uint64_t* chunk_bars = bars + 4 * D;    // 4 per producer
+  uint64_t* chunk_bars = bars + 4 * D;    // 4 per producer: compressed-stream ring
   uint64_t* mma_done = bars + 8 * D;      // every MMA of the CTA retired
   uint64_t* acc_full = bars + 8 * D + 1;  // one per accumulator slot
 
@@ -158,7 +159,10 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
       uint32_t run_bytes = 0, base = 0;
       if (kDecode) {
         run_ok = run_extent(L, t0, t1, &run_start, &run_bytes);
-        if (run_ok) base = rp_run_begin(pipe, L.stream + run_start, run_bytes);
+        if (run_ok) {
+          base = rp_run_begin(pipe, L.stream + run_start, run_bytes);
+          rp_prefetch(pipe, base, lane, abort, P.status);
+        }
         a_next = run_start;
       }
       for (; u < run_e; ++u) {
@@ -193,15 +197,17 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
             gscale[q] = __float2half2_rn(sv);
           }
         }
-        // raw sign/mantissa bytes of groups g, g+1, g+2 in flight (bf16, decode)
+        // raw sign/mantissa bytes of groups g .. g + kRawAhead - 1 in flight
+        // (bf16, decode)
         const unsigned long long* raw_tile = nullptr;
-        uint64_t r0 = 0, r1 = 0, r2 = 0;
+        uint64_t rq[kRawAhead];
         const uint32_t groups = H * C * 8;
+#pragma unroll
+        for (uint32_t k = 0; k < kRawAhead; ++k) rq[k] = 0;
         if (kDecode && kFmt == kFmtBf16Split && !zero_tile) {
           raw_tile = reinterpret_cast<const unsigned long long*>(L.raw + static_cast<uint64_t>(t) * S) + lane;
-          r0 = __ldg(raw_tile);
-          r1 = __ldg(raw_tile + 32);
-          r2 = __ldg(raw_tile + 64);
+#pragma unroll
+          for (uint32_t k = 0; k < kRawAhead; ++k) rq[k] = __ldg(raw_tile + 32 * k);
         }
         // the slabs of this tile; a tile of constant symbols (single-symbol
         // codebook, or zeros for a tile with bad offsets) takes a separate
@@ -265,11 +271,11 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
               const uint32_t i = gg & 3;
               uint32_t o[4];
               if (kDecode) {
-                const uint64_t raw8 = r0;
+                const uint64_t raw8 = rq[0];
                 if (kFmt == kFmtBf16Split && (!kConst || !zero_tile)) {
-                  r0 = r1;
-                  r1 = r2;
-                  if (g + 3 < groups) r2 = __ldg(raw_tile + 32 * (g + 3));
+#pragma unroll
+                  for (uint32_t k = 0; k + 1 < kRawAhead; ++k) rq[k] = rq[k + 1];
+                  if (g + kRawAhead < groups) rq[kRawAhead - 1] = __ldg(raw_tile + 32 * (g + kRawAhead));
                 }
                 uint32_t e[8];
                 if (kConst) {

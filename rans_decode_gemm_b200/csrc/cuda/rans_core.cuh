@@ -240,13 +240,10 @@ __device__ __forceinline__ uint32_t rp_run_begin(RunPipe& p, const uint8_t* src,
   return p.run_c0 * kChunkBytes;
 }
 
-// Called when the cursor enters chunk c: afterwards chunk c + 1 (or the run's
-// last chunk) has landed and chunks up to c + 3 are in flight.  A slot is
-// re-armed only after the chunk that last used it was waited for.
-__device__ __forceinline__ void rp_enter(RunPipe& p, uint32_t c, uint32_t lane,
+// Issue chunks while fewer than lim have been issued (lim <= the run's end).
+// A slot is re-armed only after the chunk that last used it was waited for.
+__device__ __forceinline__ void rp_issue(RunPipe& p, uint32_t lim, uint32_t lane,
                                          volatile uint32_t* abort, uint32_t* status) {
-  p.cur = c;
-  const uint32_t lim = min(c + 4u, p.run_end);
   while (p.issued < lim && !*abort) {
     while (p.ready + 4u <= p.issued) {
       if (!wait_live(&p.bars[p.ready & 3u], (p.ready >> 2) & 1u, abort, status)) return;
@@ -261,6 +258,21 @@ __device__ __forceinline__ void rp_enter(RunPipe& p, uint32_t c, uint32_t lane,
     }
     p.issued++;
   }
+}
+
+// Start the copies of the chunks from position pos on (up to 4 chunks), without
+// waiting: called at the start of a run so its first bytes are in flight early.
+__device__ __forceinline__ void rp_prefetch(RunPipe& p, uint32_t pos, uint32_t lane,
+                                            volatile uint32_t* abort, uint32_t* status) {
+  rp_issue(p, min(pos / kChunkBytes + 4u, p.run_end), lane, abort, status);
+}
+
+// Called when the cursor enters chunk c: afterwards chunk c + 1 (or the run's
+// last chunk) has landed and chunks up to c + 3 are in flight.
+__device__ __forceinline__ void rp_enter(RunPipe& p, uint32_t c, uint32_t lane,
+                                         volatile uint32_t* abort, uint32_t* status) {
+  p.cur = c;
+  rp_issue(p, min(c + 4u, p.run_end), lane, abort, status);
   const uint32_t need = min(c + 1u, p.run_end - 1u);
   while (p.ready <= need && p.ready < p.issued) {
     if (!wait_live(&p.bars[p.ready & 3u], (p.ready >> 2) & 1u, abort, status)) return;

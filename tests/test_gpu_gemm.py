@@ -91,6 +91,12 @@ def test_gemm_argument_errors(cuda, cases):
     with pytest.raises(ans.AnsError) as e:   # misaligned X
         ans.ans_gemm(Xflat[1:], 4, layer.tiles, 0, None, 0, Y, ws, ws.numel(), st)
     assert e.value.status == 1
+    # the raw side stream is fetched with 16-byte bulk copies
+    shifted = ans.AnsTiles.from_buffer_copy(layer.tiles)
+    shifted.raw = layer.tiles.raw + 8
+    with pytest.raises(ans.AnsError) as e:
+        ans.ans_gemm(X, 4, shifted, 0, None, 0, Y, ws, ws.numel(), st)
+    assert e.value.status == 1
     # M == 0 is a no-op
     ans.ans_gemm(X, 0, layer.tiles, 0, None, 0, Y, ws, ws.numel(), st)
     torch.cuda.synchronize()
