@@ -18,7 +18,7 @@ namespace ansdev {
 constexpr uint32_t kDecMaxWarps = 16;
 constexpr uint32_t kDecLutBytes = kSlots * 4;
 // [lut 16 KB][align slack 2 KB][rings W x 2 KB][barriers W x 4 x 8 B]
-constexpr uint32_t kDecSmem = kDecLutBytes + kRingBytes + kDecMaxWarps * kRingBytes + kDecMaxWarps * 4 * 8;
+constexpr uint32_t kDecSmem = kDecLutBytes + 128 + kDecMaxWarps * kRingStride + kDecMaxWarps * 4 * 8;
 
 // 8 output elements of one lane (row, 8 consecutive columns) in the original
 // storage format.
@@ -51,10 +51,10 @@ __global__ void __launch_bounds__(kDecMaxWarps * 32, 2)
   __shared__ uint32_t abort_flag;
   const uint32_t nwarps = blockDim.x / 32;
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem);
-  // rings on a kRingBytes-aligned shared address
-  const uint32_t ring_base_s = (smem_u32(smem + kDecLutBytes) + kRingBytes - 1) & ~(kRingBytes - 1);
+  // rings on a 128-byte aligned shared address
+  const uint32_t ring_base_s = (smem_u32(smem + kDecLutBytes) + 127) & ~127u;
   uint8_t* rings = smem + (ring_base_s - smem_u32(smem));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kDecLutBytes + kRingBytes + kDecMaxWarps * kRingBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kDecLutBytes + 128 + kDecMaxWarps * kRingStride);
   const uint32_t warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const bool single = L.single_symbol != kNoSymbol;
   const uint32_t single_e = L.single_symbol << 12;
@@ -81,7 +81,7 @@ __global__ void __launch_bounds__(kDecMaxWarps * 32, 2)
   const uint8_t* raw = L.raw;
   TileSeq seq{blockIdx.x * nwarps + warp, gridDim.x * nwarps, n_tiles, n_tiles};
   ChunkPipe pipe;
-  pipe_init(pipe, rings + warp * kRingBytes, bars + warp * 4);
+  pipe_init(pipe, rings + warp * kRingStride, bars + warp * 4);
   TileCursor tc;
   tc.cb = 0;
   const uint64_t row_step = 32ull * K;  // next row of the same lane

@@ -131,8 +131,8 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
 
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem + P.off_lut);
   uint8_t* wring = smem + P.off_w;
-  // chunk rings start on a kRingBytes-aligned shared address (the plan leaves slack)
-  uint8_t* chunks = smem + (((smem_u32(smem + P.off_chunk) + kRingBytes - 1) & ~(kRingBytes - 1)) - smem_u32(smem));
+  // chunk rings start on a 128-byte aligned shared address (the plan leaves slack)
+  uint8_t* chunks = smem + (((smem_u32(smem + P.off_chunk) + 127) & ~127u) - smem_u32(smem));
   uint8_t* xring = smem + P.off_x;
   Bars B = carve_bars(smem + P.off_bars, D, XS);
   const uint32_t x_stage_bytes = P.T_pass * 32;
@@ -176,7 +176,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     const uint32_t lut_s = smem_u32(lut);
     TileSeq seq{static_cast<uint32_t>(u_begin) + d, D, static_cast<uint32_t>(u_end), L.n_tiles};
     ChunkPipe pipe;
-    pipe_init(pipe, chunks + d * kRingBytes, B.chunk + 4 * d);
+    pipe_init(pipe, chunks + d * kRingStride, B.chunk + 4 * d);
     TileCursor tc;
     tc.cb = 0;
     uint32_t sc = 0;  // unit slabs produced
@@ -609,9 +609,9 @@ bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool dec
       off = round_up(off, 1024);
       const uint32_t off_w = off;
       off += 2 * D * kSlabBytes;  // two W slabs per producer
-      off = round_up(off, 2048);
+      off = round_up(off, 128);
       const uint32_t off_chunk = off;
-      off += (D + 1) * kRingBytes;
+      off += D * kRingStride + 128;
       off = round_up(off, 1024);
       const uint32_t off_x = off;
       off += 2 * D * p.T * 32;  // two X slabs per producer
@@ -681,9 +681,9 @@ bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool dec
     off = round_up(off, 2048);
     const uint32_t off_w = off;
     off += D * 2 * kSlabBytes;
-    off = round_up(off, 2048);
+    off = round_up(off, 128);
     const uint32_t off_chunk = off;
-    off += (D + 1) * kRingBytes;
+    off += D * kRingStride + 128;
     off = round_up(off, 1024);
     const uint32_t off_x = off;
     const uint32_t bars_max = num_bars(D, 64) * 8;

@@ -85,6 +85,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
   __shared__ uint32_t red_n, red_seg[2];  // split-K segments of this CTA
   __shared__ uint32_t slot_seg[kLocalMaxSlots];
   __shared__ uint32_t n_cta_slots;
+  __shared__ uint4 issue_q[kLocalMaxProducers];  // MMAs posted to the issuing lane
 
   const uint32_t warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t D = P.D, H = P.H, C = P.C, T = P.T;
@@ -95,7 +96,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
 
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem + P.off_lut);
   uint8_t* wslots = smem + P.off_w;   // 2 per producer, kSlabBytes each
-  uint8_t* chunks = smem + (((smem_u32(smem + P.off_chunk) + kRingBytes - 1) & ~(kRingBytes - 1)) - smem_u32(smem));
+  uint8_t* chunks = smem + (((smem_u32(smem + P.off_chunk) + 127) & ~127u) - smem_u32(smem));
   uint8_t* xslots = smem + P.off_x;   // 2 per producer, T * 32 bytes each
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P.off_bars);
   uint64_t* w_full = bars;                // 2 per producer: slab written
@@ -143,7 +144,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
     const uint32_t S = L.tile_n * L.tile_k;
     const uint32_t n_xch = T / 16;  // 16-byte X chunks per lane per slab (1 or 2)
     RunPipe pipe;
-    rp_init(pipe, chunks + d * kRingBytes, chunk_bars + 4 * d);
+    rp_init(pipe, chunks + d * kRingStride, chunk_bars + 4 * d);
     TileCursor tc;
     tc.x = tc.pos = tc.cb = tc.bytes = 0;
     uint32_t nw = 0;  // slabs signalled to the issuing warp
@@ -404,23 +405,28 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
       // the producer reuses this slot only if it has a slab nslab + 2
       const bool reuse = nslab + 2 < (pe - pb) * n_us;
       const uint32_t info = slot | (accum << 1) | ((seg_end ? 1u : 0u) << 2) | ((reuse ? 1u : 0u) << 3);
-      tc_fence_after();
-      while (rmask) {
-        const uint32_t r = __ffs(rmask) - 1;
-        rmask &= rmask - 1;
-        const uint32_t c_r = __shfl_sync(0xFFFFFFFFu, col, r);
-        const uint32_t i_r = __shfl_sync(0xFFFFFFFFu, info, r);
-        const uint32_t k_r = __shfl_sync(0xFFFFFFFFu, acc_slot, r);
-        if (lane == 0) {
-          const uint32_t s_r = i_r & 1u;
-          const uint64_t adesc = dhi | ((w_base + (2 * r + s_r) * kSlabBytes) >> 4);
-          const uint64_t bdesc = dhi | ((x_base + (2 * r + s_r) * T * 32) >> 4);
-          umma_f16(tmem_base + c_r, adesc, bdesc, P.idesc, (i_r >> 1) & 1u);
-          if (i_r & 8u) umma_commit(&w_empty[2 * r + s_r]);
-          if (i_r & 4u) umma_commit(&acc_full[k_r]);
-        }
-        __syncwarp();
+      // each ready lane posts its MMA (accumulator address, operand start
+      // addresses, flags); lane 0 then issues the round without further warp
+      // collectives
+      if (ready) {
+        const uint32_t a_lo = (w_base + (2 * q + slot) * kSlabBytes) >> 4;
+        const uint32_t b_lo = (x_base + (2 * q + slot) * T * 32) >> 4;
+        issue_q[q] = make_uint4(tmem_base + col, a_lo | (b_lo << 16), info, acc_slot);
       }
+      __syncwarp();
+      if (lane == 0) {
+        tc_fence_after();
+        while (rmask) {
+          const uint32_t r = __ffs(rmask) - 1;
+          rmask &= rmask - 1;
+          const uint4 v = issue_q[r];
+          const uint32_t s_r = v.z & 1u;
+          umma_f16(v.x, dhi | (v.y & 0xFFFFu), dhi | (v.y >> 16), P.idesc, (v.z >> 1) & 1u);
+          if (v.z & 8u) umma_commit(&w_empty[2 * r + s_r]);
+          if (v.z & 4u) umma_commit(&acc_full[v.w]);
+        }
+      }
+      __syncwarp();
       if (ready) {
         fresh &= ~(1u << h);
         ++nslab;

@@ -32,6 +32,11 @@ constexpr uint32_t kSlots = 4096;        // 2^12 probability slots
 constexpr uint32_t kStateLow = 1u << 16; // L
 constexpr uint32_t kChunkBytes = 512;
 constexpr uint32_t kRingBytes = 2048;
+// A ring occupies kRingStride bytes: after its kRingBytes the first
+// kRingMirror bytes of slot 0 are repeated, so the words one decode step
+// reads (at most 64 bytes from the cursor) never wrap around.
+constexpr uint32_t kRingMirror = 64;
+constexpr uint32_t kRingStride = kRingBytes + kRingMirror;
 constexpr uint32_t kNoSymbol = kNoSymbolHost;
 
 constexpr uint32_t kStatusCorrupt = 0x1u;
@@ -113,7 +118,7 @@ struct TileSeq {
 // issues the copies.
 struct ChunkPipe {
   uint8_t* ring;      // kRingBytes of shared memory (generic pointer, for copies)
-  uint32_t ring_s;    // the same ring as a kRingBytes-aligned shared address
+  uint32_t ring_s;    // the same ring as a shared address (kRingStride bytes)
   uint64_t* bars;     // 4 mbarriers (count 1)
   uint32_t issued;    // chunks issued so far (global index over the warp's tiles)
   uint32_t ready;     // chunks known to have landed
@@ -150,8 +155,10 @@ __device__ __forceinline__ void pipe_issue(ChunkPipe& p, const LayerDev& L, cons
     uint32_t n = min(kChunkBytes, p.it_bytes - off);
     uint32_t slot = p.issued & 3u;
     if (lane == 0) {
-      mbar_arrive_expect_tx(&p.bars[slot], n);
+      const uint32_t nm = slot == 0 ? min(n, kRingMirror) : 0u;  // mirror of slot 0's head
+      mbar_arrive_expect_tx(&p.bars[slot], n + nm);
       bulk_g2s(p.ring + slot * kChunkBytes, L.stream + p.it_start + off, n, &p.bars[slot]);
+      if (nm) bulk_g2s(p.ring + kRingBytes, L.stream + p.it_start + off, nm, &p.bars[slot]);
     }
     p.it_chunk++;
     p.issued++;
@@ -253,8 +260,10 @@ __device__ __forceinline__ void rp_issue(RunPipe& p, uint32_t lim, uint32_t lane
     const uint32_t n = min(kChunkBytes, p.run_bytes - off);
     const uint32_t slot = p.issued & 3u;
     if (lane == 0) {
-      mbar_arrive_expect_tx(&p.bars[slot], n);
+      const uint32_t nm = slot == 0 ? min(n, kRingMirror) : 0u;  // mirror of slot 0's head
+      mbar_arrive_expect_tx(&p.bars[slot], n + nm);
       bulk_g2s(p.ring + slot * kChunkBytes, p.src + off, n, &p.bars[slot]);
+      if (nm) bulk_g2s(p.ring + kRingBytes, p.src + off, nm, &p.bars[slot]);
     }
     p.issued++;
   }
@@ -391,45 +400,31 @@ __device__ __forceinline__ bool tile_end(TileCursor& tc, bool single) {
   return !__any_sync(0xFFFFFFFFu, bad);
 }
 
-// One decode step for the calling lane, branch-free, on 32-bit shared-memory
-// addresses.  x: state; pos: ring read position (bytes, unwrapped; advanced
-// by the words the whole warp consumed); lut_s: slot-table address; ring_s:
-// ring address (kRingBytes-aligned); lt: %lanemask_lt.  Returns the slot-table
-// entry of the decoded symbol.  Every lane loads the word at its prefix
-// position (all such addresses lie in one 64-byte window, so the extra loads
-// cost no extra shared-memory wavefront); lanes that need no word discard it.
-// Slot-table load: the table is written once before the CTA barrier and then
-// only read, so the load is an ordinary (reorderable) one.
-__device__ __forceinline__ uint32_t lds_lut(uint32_t addr) {
-  uint32_t v;
-  asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
-  return v;
-}
-// Ring-word load: volatile so it stays after the chunk waits that precede it.
-__device__ __forceinline__ uint32_t lds_ring16(uint32_t addr) {
-  unsigned short v;
-  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
-  return v;
-}
-
 // One decode step of the calling lane (see the file comment), as explicit
-// PTX: slot lookup, state update, ballot of the lanes that need a word,
-// prefix-count addressing into the ring, word merge by byte permute (valid
-// because a lane needing a word has x < 2^16), predicated select.  Every lane
-// loads the word at its prefix position: those addresses all fall in one
-// 64-byte window, so lanes that need no word cost no extra wavefront.
-// Returns the slot-table entry of the decoded symbol.
+// PTX on 32-bit shared-memory addresses.  x: state; pos: ring read position
+// (bytes, unwrapped; advanced by the words the whole warp consumed); lut_s:
+// slot-table address; ring_s: ring address; lt: %lanemask_lt.  Slot lookup,
+// state update, ballot of the lanes that need a word, prefix count, word
+// merge by byte permute (valid because a lane needing a word has x < 2^16),
+// predicated select.  The ring base of the step, ring_s + pos mod 2048, is
+// computed beside the state chain; the lane's word is at base + 2 * prefix
+// with no wrap test, the mirror behind the ring covering the at most 62 bytes
+// a step can run past its end.  Every lane loads the word at its prefix
+// position (all in one 64-byte window, so lanes that need no word cost no
+// extra wavefront).  Returns the slot-table entry of the decoded symbol.
 __device__ __forceinline__ uint32_t decode_step(uint32_t& x, uint32_t& pos, uint32_t lut_s,
                                                 uint32_t ring_s, uint32_t lt) {
   uint32_t e;
   asm volatile(
       "{\n\t"
       ".reg .pred p;\n\t"
-      ".reg .b32 a, q, f, b, bal, t, pre, cnt, off, w, xs;\n\t"
+      ".reg .b32 a, q, f, b, bal, t, pre, cnt, off, w, xs, pb;\n\t"
       "and.b32 a, %0, 4095;\n\t"
       "shl.b32 a, a, 2;\n\t"
       "add.u32 a, a, %3;\n\t"
       "ld.shared.u32 %2, [a];\n\t"
+      "and.b32 pb, %1, 2047;\n\t"
+      "add.u32 pb, pb, %4;\n\t"
       "shr.u32 q, %0, 12;\n\t"
       "shr.u32 f, %2, 20;\n\t"
       "and.b32 b, %2, 4095;\n\t"
@@ -439,10 +434,7 @@ __device__ __forceinline__ uint32_t decode_step(uint32_t& x, uint32_t& pos, uint
       "and.b32 t, bal, %5;\n\t"
       "popc.b32 pre, t;\n\t"
       "popc.b32 cnt, bal;\n\t"
-      "shl.b32 pre, pre, 1;\n\t"
-      "add.u32 off, %1, pre;\n\t"
-      "and.b32 off, off, 2047;\n\t"
-      "add.u32 off, off, %4;\n\t"
+      "mad.lo.u32 off, pre, 2, pb;\n\t"
       "ld.shared.u16 w, [off];\n\t"
       "prmt.b32 xs, w, %0, 0x5410;\n\t"
       "selp.b32 %0, xs, %0, p;\n\t"
