@@ -51,6 +51,10 @@ def parse():
     ap.add_argument("--warmup", type=int, default=100)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="every workload of the pages at full size, one JSON line per point "
+                         "(instead of the benchmark line)")
+    ap.add_argument("--sweep-configs", default="", help="comma-separated subset for --sweep")
     ap.add_argument("--quick", action="store_true",
                     help="skip the context sweep and the CPU baseline (profiling runs)")
     return ap.parse_args()
@@ -377,6 +381,146 @@ def context_numbers(torch, ans, WL, cfg, d, lay, layers, dw, device):
     return out
 
 
+def dequant_bf16(torch, cfg, d, device):
+    """Dense bf16 copy of the dequantised weights (for the cuBLAS reference)."""
+    N, K = d["N"], d["K"]
+    if cfg.dtype == 1:  # bf16 bits
+        return torch.from_numpy(d["w"].view(np.int16)).to(device).view(torch.bfloat16).view(N, K)
+    if cfg.dtype == 0:  # packed int4 nibbles, element k even in the low nibble
+        b = torch.from_numpy(d["w"]).to(device)
+        nib = torch.stack([b & 0xF, b >> 4], dim=1).view(N, K).to(torch.int16)
+        q = torch.where(nib >= 8, nib - 16, nib).to(torch.float32)
+        s = torch.from_numpy(d["scales"].view(np.int16)).to(device).view(torch.bfloat16).float()
+        if s.dim() == 1:
+            return (q * s[:, None]).to(torch.bfloat16)
+        return (q * s.repeat_interleave(K // s.shape[1], dim=1)).to(torch.bfloat16)
+    codes = torch.from_numpy(d["w"]).to(device).view(torch.float8_e4m3fn).view(N, K)
+    s = torch.from_numpy(d["scales"]).to(device)
+    return (codes.float() * s[:, None]).to(torch.bfloat16)
+
+
+def sweep(args):
+    """Every workload of the pages at full size on one GPU: bits/weight against
+    the entropy bound, ans_gemm at each M of the workload, the same kernel on
+    uncompressed weights, ans_decode_tiles, cuBLAS on dense bf16 weights, the
+    two-pass baselines (decode to HBM, then ans_gemm_uncompressed on the decoded
+    weights, or cuBLAS on bf16 weights), and roofline fractions.  Weights stream from HBM (enough rotating copies
+    to exceed L2).  One JSON line per point."""
+    import torch
+    from rans_decode_gemm_b200 import ans
+    from rans_decode_gemm_b200 import workloads as WL
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    peaks, peaks_src = load_peaks()
+    nominal = {0: 0.5, 1: 2.0, 2: 1.0}
+    st = torch.zeros(1, dtype=torch.int32, device=device)
+    stream = torch.cuda.Stream(device=device)
+    torch.cuda.set_stream(stream)
+
+    def timed_graph(calls, reps):
+        """Average µs per call of `calls` (a list of closures), captured as one
+        CUDA graph and replayed `reps` times after one warm replay."""
+        for c in calls:
+            c()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for c in calls:
+                c()
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        del g
+        return a.elapsed_time(b) * 1e3 / (reps * len(calls))
+
+    only = set(args.sweep_configs.split(",")) if args.sweep_configs else None
+    for name, cfg in WL.CONFIGS.items():
+        if only and name not in only:
+            continue
+        for mi, (mname, mN, mK) in enumerate(cfg.matrices):
+            d = WL.make_weights(cfg, mi)
+            N, K = d["N"], d["K"]
+            lay = ans.make_layout(cfg.dtype, N, K, cfg.tile_n, cfg.tile_k)
+            dw = torch.from_numpy(d["w"].view(np.int16) if d["w"].dtype == np.uint16 else d["w"]).to(device)
+            A = 256 if cfg.dtype != 0 else 16
+            hist = torch.zeros(A, dtype=torch.int64, device=device)
+            ans.ans_histogram(dw, lay, hist)
+            hist_h = hist.cpu().numpy().astype(np.uint64)
+            t0 = time.perf_counter()
+            cb = ans.ans_build_codebook(hist_h, A, 12)
+            stream_h, offsets_h, raw_h = ans.ans_encode_tiles(d["w"], lay, cb)
+            encode_s = time.perf_counter() - t0
+            comp = int(stream_h.size + 8 * offsets_h.size + (raw_h.size if raw_h is not None else 0))
+            copies = int(max(1, min(12, -(-256e6 // comp))))
+            layers = [ans.CompressedLayer(lay, cb, stream_h, offsets_h, raw_h, device) for _ in range(copies)]
+            H = ans.ans_entropy(hist_h)
+            bound = H + 8.0 if cfg.dtype == 1 else H
+            bpw = 8.0 * layers[0].compressed_bytes / (N * K)
+            sc = None
+            if d["scales"] is not None:
+                s = np.ascontiguousarray(d["scales"])
+                sc = torch.from_numpy(s.view(np.int16) if s.dtype == np.uint16 else s).to(device)
+            Wb = dequant_bf16(torch, cfg, d, device)
+            wcopies = max(1, min(copies, int(-(-256e6 // (N * K * 2)))))
+            Wbs = [Wb] + [Wb.clone() for _ in range(wcopies - 1)]
+            dec = torch.empty(N * K * (2 if cfg.dtype == 1 else 1) // (2 if cfg.dtype == 0 else 1),
+                              dtype=torch.uint8, device=device)
+            rep_for = lambda us_est: max(3, min(200, int(20000 / max(us_est, 1.0))))
+            t_dec = timed_graph([lambda l=l: ans.ans_decode_tiles(l.tiles, dec, st) for l in layers], 3)
+            t_dec = timed_graph([lambda l=l: ans.ans_decode_tiles(l.tiles, dec, st) for l in layers],
+                                rep_for(t_dec * copies))
+            for M in cfg.Ms:
+                X = torch.from_numpy(WL.make_x(cfg, M, K).view(np.int16)).to(device)
+                Y = torch.empty(M, N, dtype=torch.float32, device=device)
+                Yu = torch.empty(M, N, dtype=torch.float32, device=device)
+                nb = ans.ans_gemm_workspace(lay, M, cfg.scale_kind)
+                ws = torch.zeros(max(nb, 256), dtype=torch.uint8, device=device)
+                fused = [lambda l=l: ans.ans_gemm(X, M, l.tiles, cfg.scale_kind, sc, cfg.group_k, Y, ws, nb, st)
+                         for l in layers]
+                plain = [lambda: ans.ans_gemm_uncompressed(X, M, dw, lay, cfg.scale_kind, sc, cfg.group_k,
+                                                           Yu, ws, nb, st)]
+                t_f = timed_graph(fused, 2)
+                t_f = timed_graph(fused, rep_for(t_f * copies))
+                t_u = timed_graph(plain, 2)
+                t_u = timed_graph(plain, rep_for(t_u))
+                same = bool(torch.equal(Y, Yu))
+                Xb = X.view(torch.bfloat16)
+                cub = [lambda w=w: torch.matmul(Xb, w.t()) for w in Wbs]
+                t_c = timed_graph(cub, 2)
+                t_c = timed_graph(cub, rep_for(t_c * len(cub)))
+                algo = layers[0].compressed_bytes + 2 * M * K + 4 * M * N
+                rec = {"workload": name, "matrix": mname, "N": N, "K": K, "M": M,
+                       "tile": f"{lay.tile_n}x{lay.tile_k}", "bits_per_weight": round(bpw, 4),
+                       "entropy_bound_bits": round(bound, 4), "gap_bits": round(bpw - bound, 4),
+                       "encode_s": round(encode_s, 2), "copies": copies,
+                       "ans_gemm_us": round(t_f, 2),
+                       "effective_weight_GBps": round(N * K * nominal[cfg.dtype] / (t_f * 1e-6) / 1e9, 1),
+                       "hbm_frac": round(algo / (t_f * 1e-6) / 1e9 / float(peaks["hbm_gbs"]), 4),
+                       "tensor_frac": round(2.0 * M * N * K / (t_f * 1e-6) / 1e12 / float(peaks["bf16_tflops"]), 4),
+                       "uncompressed_us": round(t_u, 2), "bit_identical_to_uncompressed": same,
+                       "decode_tiles_us": round(t_dec, 2),
+                       "decode_Tsym_per_s": round(N * K / (t_dec * 1e-6) / 1e12, 4),
+                       "two_pass_us": round(t_dec + t_u, 2),
+                       "speedup_vs_two_pass": round((t_dec + t_u) / t_f, 3),
+                       "cublas_bf16_us": round(t_c, 2),
+                       # decode to HBM, then cuBLAS on dense bf16 weights (for int4 /
+                       # fp8 this GEMM reads 2 B per weight: no cuBLAS kernel takes
+                       # those codes with a bf16 X)
+                       "two_pass_cublas_us": round(t_dec + t_c, 2),
+                       "speedup_vs_two_pass_cublas": round((t_dec + t_c) / t_f, 3),
+                       "status": int(st.item()),
+                       "peak_source": peaks_src}
+                print(json.dumps(rec), flush=True)
+                del X, Y, Yu, ws
+            del layers, Wbs, Wb, dec, dw
+            torch.cuda.empty_cache()
+
+
 def cpu_baseline(cfg, d, lay, layer, X_h, budget_s=20.0):
     """The CPU oracle, as it stands, on the host cores: decode of a sample of
     whole W row blocks plus the fp64 GEMM on their rows, scaled to the metric
@@ -459,6 +603,9 @@ def time_reference(args):
 
 def main():
     args = parse()
+    if args.sweep:
+        sweep(args)
+        return
     if args.impl == "reference":
         res = time_reference(args)
     else:
