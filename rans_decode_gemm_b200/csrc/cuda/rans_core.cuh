@@ -68,6 +68,22 @@ __device__ __forceinline__ bool wait_live(uint64_t* bar, uint32_t parity, volati
   return true;
 }
 
+// wait_live on a barrier given by its 32-bit shared-memory address.
+__device__ __forceinline__ bool wait_live_s(uint32_t bar_s, uint32_t parity, volatile uint32_t* abort,
+                                            uint32_t* status, uint32_t site = 0) {
+  if (mbar_try_wait_s(bar_s, parity)) return true;
+  long long t0 = clock64();
+  while (!mbar_try_wait_s(bar_s, parity)) {
+    if (*abort) return false;
+    if (clock64() - t0 > kWaitBudgetCycles) {
+      *abort = 1u;
+      atomicOr(status, kStatusTimeout | (1u << (8 + site)));
+      return false;
+    }
+  }
+  return true;
+}
+
 // Bounded wait used when draining copies before exit; ignores the abort flag
 // (bulk copies always complete on their own).
 __device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, uint32_t* status) {
@@ -215,9 +231,8 @@ struct TileCursor {
 // ring slot of a position is position % kRingBytes.  Same ring, chunk size
 // and barriers as ChunkPipe.
 struct RunPipe {
-  uint8_t* ring;
-  uint32_t ring_s;
-  uint64_t* bars;
+  uint32_t ring_s;     // the ring (kRingStride bytes) as a shared-memory address
+  uint32_t bars_s;     // its 4 mbarriers (count 1), shared-memory address
   const uint8_t* src;  // first byte of the current run in global memory
   uint32_t run_c0;     // global chunk index of the run's first chunk
   uint32_t run_end;    // global chunk index one past the run's last chunk
@@ -227,9 +242,8 @@ struct RunPipe {
 };
 
 __device__ __forceinline__ void rp_init(RunPipe& p, uint8_t* ring, uint64_t* bars) {
-  p.ring = ring;
   p.ring_s = smem_u32(ring);
-  p.bars = bars;
+  p.bars_s = smem_u32(bars);
   p.src = nullptr;
   p.run_c0 = p.run_end = p.run_bytes = 0;
   p.issued = p.ready = 0;
@@ -253,7 +267,7 @@ __device__ __forceinline__ void rp_issue(RunPipe& p, uint32_t lim, uint32_t lane
                                          volatile uint32_t* abort, uint32_t* status) {
   while (p.issued < lim && !*abort) {
     while (p.ready + 4u <= p.issued) {
-      if (!wait_live(&p.bars[p.ready & 3u], (p.ready >> 2) & 1u, abort, status)) return;
+      if (!wait_live_s(p.bars_s + 8 * (p.ready & 3u), (p.ready >> 2) & 1u, abort, status)) return;
       p.ready++;
     }
     const uint32_t off = (p.issued - p.run_c0) * kChunkBytes;
@@ -261,9 +275,10 @@ __device__ __forceinline__ void rp_issue(RunPipe& p, uint32_t lim, uint32_t lane
     const uint32_t slot = p.issued & 3u;
     if (lane == 0) {
       const uint32_t nm = slot == 0 ? min(n, kRingMirror) : 0u;  // mirror of slot 0's head
-      mbar_arrive_expect_tx(&p.bars[slot], n + nm);
-      bulk_g2s(p.ring + slot * kChunkBytes, p.src + off, n, &p.bars[slot]);
-      if (nm) bulk_g2s(p.ring + kRingBytes, p.src + off, nm, &p.bars[slot]);
+      const uint32_t bar = p.bars_s + 8 * slot;
+      mbar_arrive_expect_tx_s(bar, n + nm);
+      bulk_g2s_s(p.ring_s + slot * kChunkBytes, p.src + off, n, bar);
+      if (nm) bulk_g2s_s(p.ring_s + kRingBytes, p.src + off, nm, bar);
     }
     p.issued++;
   }
@@ -284,14 +299,20 @@ __device__ __forceinline__ void rp_enter(RunPipe& p, uint32_t c, uint32_t lane,
   rp_issue(p, min(c + 4u, p.run_end), lane, abort, status);
   const uint32_t need = min(c + 1u, p.run_end - 1u);
   while (p.ready <= need && p.ready < p.issued) {
-    if (!wait_live(&p.bars[p.ready & 3u], (p.ready >> 2) & 1u, abort, status)) return;
+    if (!wait_live_s(p.bars_s + 8 * (p.ready & 3u), (p.ready >> 2) & 1u, abort, status)) return;
     p.ready++;
   }
 }
 
 __device__ __forceinline__ void rp_drain(RunPipe& p, uint32_t* status) {
   while (p.ready < p.issued) {
-    wait_drain(&p.bars[p.ready & 3u], (p.ready >> 2) & 1u, status);
+    long long t0 = clock64();
+    while (!mbar_try_wait_s(p.bars_s + 8 * (p.ready & 3u), (p.ready >> 2) & 1u)) {
+      if (clock64() - t0 > kWaitBudgetCycles) {
+        atomicOr(status, kStatusTimeout);
+        break;
+      }
+    }
     p.ready++;
   }
 }

@@ -172,3 +172,39 @@ def test_gemm_bad_offsets_flag_status(cuda, cases, monkeypatch, schedule):
     Y, st, _ = run_gemm(cfg, d, lay, broken, X)
     assert st & ans.STATUS_BAD_OFFSETS
     assert not st & ans.STATUS_TIMEOUT
+
+
+@pytest.mark.parametrize("ctas", [3, 7])
+@pytest.mark.parametrize("name,N,K,M", [("bf16_4096", 1024, 2048, 16), ("int4_70b", 512, 2048, 16),
+                                        ("fp8_405b", 512, 1024, 32), ("tiny_int4", 512, 512, 1),
+                                        ("llama8b_mlp", 384, 2048, 5)])
+def test_gemm_local_long_producer_runs(cuda, oracle, cases, monkeypatch, ctas, name, N, K, M):
+    # few CTAs: every producer warp of the local schedule owns a long run of
+    # tiles crossing W row blocks (chunk rings wrap many times, several
+    # accumulators per producer); bit-identical to the uncompressed variant
+    # and within the bar of the fp64 oracle
+    monkeypatch.setenv("ANS_GEMM_MAX_CTAS", str(ctas))
+    cfg, d, lay, layer = _case(cases, name, N, K)
+    X = WL.make_x(cfg, M, K)
+    Y, st, _ = run_gemm(cfg, d, lay, layer, X, compressed=True)
+    Yu, stu, _ = run_gemm(cfg, d, lay, layer, X, compressed=False)
+    assert st == 0 and stu == 0 and torch.equal(Y, Yu)
+    Yref = oracle.gemm(cfg.dtype, X, M, K, d["w"], N, cfg.scale_kind, d["scales"], cfg.group_k)
+    assert rel_fro(Y.cpu().numpy(), Yref) <= TOL
+
+
+def test_gemm_long_runs_corrupt_and_bad_offsets(cuda, cases, monkeypatch):
+    # a corrupt or badly indexed tile in the middle of a producer's run
+    monkeypatch.setenv("ANS_GEMM_MAX_CTAS", "4")
+    cfg, d, lay, layer = _case(cases, "bf16_4096", 512, 1024)
+    X = WL.make_x(cfg, 16, 1024)
+    bad = layer.h_stream.copy()
+    bad[200] ^= 0x10
+    broken = ans.CompressedLayer(lay, layer.codebook, bad, layer.h_offsets, layer.h_raw)
+    Y, st, _ = run_gemm(cfg, d, lay, broken, X)
+    assert st & ans.STATUS_CORRUPT and not st & ans.STATUS_TIMEOUT
+    off = layer.h_offsets.copy()
+    off[9] = off[-1] + 4096
+    broken = ans.CompressedLayer(lay, layer.codebook, layer.h_stream, off, layer.h_raw)
+    Y, st, _ = run_gemm(cfg, d, lay, broken, X)
+    assert st & ans.STATUS_BAD_OFFSETS and not st & ans.STATUS_TIMEOUT
