@@ -208,3 +208,70 @@ def test_gemm_long_runs_corrupt_and_bad_offsets(cuda, cases, monkeypatch):
     broken = ans.CompressedLayer(lay, layer.codebook, layer.h_stream, off, layer.h_raw)
     Y, st, _ = run_gemm(cfg, d, lay, broken, X)
     assert st & ans.STATUS_BAD_OFFSETS and not st & ans.STATUS_TIMEOUT
+
+
+def _single_symbol_weights(dtype, N, K, rng):
+    """Weights whose coded symbol takes one value (a one-symbol codebook):
+    int4 all code 3, fp8 all 0x38, bf16 one exponent with random sign and
+    mantissa bytes."""
+    if dtype == ans.INT4:
+        return np.full(N * K // 2, 0x33, np.uint8), WL.to_bf16_bits(rng.uniform(0.005, 0.02, N))
+    if dtype == ans.FP8_E4M3:
+        return np.full(N * K, 0x38, np.uint8), rng.uniform(0.5, 2.0, N).astype(np.float32)
+    raw = rng.integers(0, 256, N * K).astype(np.uint16)
+    bits = ((raw & 0x80) << 8) | (np.uint16(0x7A) << 7) | (raw & 0x7F)
+    return bits.astype(np.uint16), None
+
+
+@pytest.mark.parametrize("dtype", [ans.INT4, ans.FP8_E4M3, ans.BF16_SPLIT])
+@pytest.mark.parametrize("M", [1, 40])
+def test_gemm_single_symbol_codebook(cuda, oracle, dtype, M):
+    # every tile is a run of one symbol: the producers take their constant
+    # path (no stream reads past the lane states) in both schedules
+    rng = np.random.default_rng(11)
+    N, K = 256, 512
+    tile_n, tile_k = (128, 64)
+    w, scales = _single_symbol_weights(dtype, N, K, rng)
+    lay = ans.make_layout(dtype, N, K, tile_n, tile_k)
+    layer = ans.CompressedLayer.from_weights(w, lay, device="cuda")
+    assert (layer.codebook.freq_array() == 4096).sum() == 1
+    scale_kind = {ans.INT4: ans.SCALE_ROW_BF16, ans.FP8_E4M3: ans.SCALE_ROW_F32, ans.BF16_SPLIT: 0}[dtype]
+    cfg = type("Cfg", (), {"scale_kind": scale_kind, "group_k": 0, "dtype": dtype})()
+    d = {"w": w, "scales": scales}
+    X = WL.make_x(WL.CONFIGS["bf16_4096"], M, K)
+    Y, st, _ = run_gemm(cfg, d, lay, layer, X, compressed=True)
+    Yu, stu, _ = run_gemm(cfg, d, lay, layer, X, compressed=False)
+    assert st == 0 and stu == 0 and torch.equal(Y, Yu)
+    Yref = oracle.gemm(dtype, X, M, K, w, N, scale_kind, scales, 0)
+    assert rel_fro(Y.cpu().numpy(), Yref) <= TOL
+
+
+@pytest.mark.parametrize("name,N,K,M", [("bf16_4096", 128, 64, 1), ("int4_70b", 256, 128, 3),
+                                        ("fp8_405b", 128, 128, 17), ("tiny_int4", 128, 32, 1),
+                                        ("bf16_4096", 4096, 64, 16), ("fp8_405b", 128, 16384, 5)])
+def test_gemm_minimal_and_extreme_shapes(cuda, oracle, cases, name, N, K, M):
+    # one tile; one K tile with many row blocks (every segment one unit);
+    # one row block with many K tiles (one segment split over every CTA)
+    cfg, d, lay, layer = _case(cases, name, N, K)
+    X = WL.make_x(cfg, M, K)
+    Y, st, _ = run_gemm(cfg, d, lay, layer, X, compressed=True)
+    Yu, stu, _ = run_gemm(cfg, d, lay, layer, X, compressed=False)
+    assert st == 0 and stu == 0 and torch.equal(Y, Yu)
+    Yref = oracle.gemm(cfg.dtype, X, M, K, d["w"], N, cfg.scale_kind, d["scales"], cfg.group_k)
+    assert rel_fro(Y.cpu().numpy(), Yref) <= TOL
+
+
+@pytest.mark.parametrize("name,M", [("int4_70b", 16), ("fp8_405b", 16)])
+def test_gemm_full_size_large_layers_sampled(cuda, oracle, cases, name, M):
+    # the largest workloads at full size in the launch configuration the
+    # sweep times; the fp64 check runs on 256 sampled W rows, bit-identity
+    # with the uncompressed variant on all of Y
+    cfg, d, lay, layer = _case(cases, name, None, None)
+    X = WL.make_x(cfg, M)
+    Y, st, _ = run_gemm(cfg, d, lay, layer, X, compressed=True)
+    Yu, stu, _ = run_gemm(cfg, d, lay, layer, X, compressed=False)
+    assert st == 0 and stu == 0 and torch.equal(Y, Yu)
+    rows = np.random.default_rng(M).choice(lay.N, size=256, replace=False).astype(np.uint32)
+    Yref = oracle.gemm(cfg.dtype, X, M, lay.K, d["w"], lay.N, cfg.scale_kind, d["scales"],
+                       cfg.group_k, rows=rows)
+    assert rel_fro(Y.cpu().numpy()[:, rows], Yref) <= TOL
