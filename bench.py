@@ -141,7 +141,26 @@ def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args is not None and world > 1 and args.gpus != world:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
     return world, rank, local
+
+
+def max_over_ranks(pg, values, device):
+    """Every rank's times -> the max over ranks of each, on every rank.  All
+    ranks call it at the same point with the same number of values."""
+    if pg is None:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return [float(v) for v in t.cpu().tolist()]
+
+
+def replica_gbs(world, bytes_per_step, ms_per_step):
+    """Whole-job throughput of `world` independent replicas, each moving
+    `bytes_per_step` per step, timed by the slowest rank at `ms_per_step`."""
+    return world * bytes_per_step / (ms_per_step * 1e-3) / 1e9
 
 
 def build_layers(torch, ans, WL, device):
@@ -237,10 +256,7 @@ def time_ours(args):
     total_ms = t0.elapsed_time(t1)
     kern_ms = total_ms / args.steps
     status = int(st.item())
-    if pg is not None:
-        tt = torch.tensor([total_ms], device=device)
-        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms, = max_over_ranks(pg, [total_ms], device)
     del g_full, g_rem
 
     # e2e through the same C ABI with host buffers: pinned X in, Y out per step
@@ -265,11 +281,7 @@ def time_ours(args):
         e2e_step(i)
     e1.record(stream)
     barrier()
-    e2e_ms = e0.elapsed_time(e1) / n_e2e
-    if pg is not None:
-        tt = torch.tensor([e2e_ms], device=device)
-        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms, = max_over_ranks(pg, [e0.elapsed_time(e1) / n_e2e], device)
 
     # context numbers on rank 0: other M, the two-pass baseline, uncompressed
     extra = {}
@@ -287,7 +299,7 @@ def time_ours(args):
         # in a second one first
         launches_per_step = 1 if ((M + 15) // 16 * 16) * (lay.tile_n // 128) <= 32 else 2
         ms_per_step = total_ms / args.steps
-        value = world * weight_bytes / (ms_per_step * 1e-3) / 1e9
+        value = replica_gbs(world, weight_bytes, ms_per_step)
         achieved = algo_bytes / (kern_ms * 1e-3) / 1e9
         peak = float(peaks["hbm_gbs"])
         H_exp = ans.ans_entropy(hist)
@@ -314,7 +326,7 @@ def time_ours(args):
                          "timing": "per-step time of the ans_gemm launch(es): CUDA graphs of "
                                    f"{N_COPIES} consecutive calls (one per layer copy), events on "
                                    "the launch stream"},
-            "e2e": {"value": round(world * weight_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "e2e": {"value": round(replica_gbs(world, weight_bytes, e2e_ms), 2), "unit": "GB/s",
                     "h2d_bytes_per_step": 2 * M * K, "d2h_bytes_per_step": 4 * M * N},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
