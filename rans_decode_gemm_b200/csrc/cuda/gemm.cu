@@ -485,7 +485,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
   }
   // the split-K reductions this CTA arrived last for, on every thread
   if (reduce_flag) {
-    __threadfence();
+    fence_acq_rel_gpu();  // acquire: the counter showed every contributor arrived
     for (uint32_t k = 0; k < red_n; ++k)
       if ((reduce_flag >> k) & 1u) splitk_reduce(P, red_seg[k], threadIdx.x, blockDim.x);
   }

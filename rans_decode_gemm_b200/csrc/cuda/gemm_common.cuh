@@ -83,24 +83,32 @@ __device__ __forceinline__ void epi_emit16(const GemmDev& P, const float (&v)[16
 // started before the segment.
 
 // Arrival: run by the 128 epilogue threads once all of this CTA's partials
-// are written.  Returns (to every thread) a bit per segment for which this
-// CTA arrived last and must reduce.
+// are written, for at most two segments.  Returns (to every thread) a bit per
+// segment for which this CTA arrived last and must reduce; the reducing CTA
+// runs fence_acq_rel_gpu() before it reads the other CTAs' partials.
 __device__ __forceinline__ uint32_t splitk_arrive(const GemmDev& P, const uint32_t* segs,
                                                   uint32_t n, uint32_t e,
                                                   volatile uint32_t* reduce_flag) {
   const uint32_t G = gridDim.x, n_kt = P.L.n_kt, U = static_cast<uint32_t>(P.n_units);
   named_bar_sync(1, 128);
   if (e == 0) {
-    // one gpu-scope fence after the barrier covers the partials every
-    // epilogue thread wrote before it (fences are cumulative)
-    __threadfence();
+    // release: one gpu-scope acq_rel fence after the barrier covers the
+    // partials every epilogue thread wrote before it (fences are cumulative);
+    // both counters are incremented before either result is looked at
+    fence_acq_rel_gpu();
     uint32_t bits = 0;
-    for (uint32_t k = 0; k < n; ++k) {
-      const uint32_t s_lo = segs[k] * n_kt;
-      const uint32_t c_first = cta_of(U, G, s_lo), c_last = cta_of(U, G, s_lo + n_kt - 1);
-      const uint32_t old = atomicAdd(&P.counters[segs[k]], 1u);
-      if (old == c_last - c_first) bits |= 1u << k;
+    uint32_t old[2] = {0, 0}, need[2] = {0, 0};
+#pragma unroll
+    for (uint32_t k = 0; k < 2; ++k) {
+      if (k < n) {
+        const uint32_t s_lo = segs[k] * n_kt;
+        need[k] = cta_of(U, G, s_lo + n_kt - 1) - cta_of(U, G, s_lo);
+        old[k] = atomicAdd(&P.counters[segs[k]], 1u);
+      }
     }
+#pragma unroll
+    for (uint32_t k = 0; k < 2; ++k)
+      if (k < n && old[k] == need[k]) bits |= 1u << k;
     *reduce_flag = bits;
   }
   named_bar_sync(1, 128);

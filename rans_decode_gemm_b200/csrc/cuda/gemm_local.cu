@@ -85,7 +85,6 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
   __shared__ uint32_t red_n, red_seg[2];  // split-K segments of this CTA
   __shared__ uint32_t slot_seg[kLocalMaxSlots];
   __shared__ uint32_t n_cta_slots;
-  __shared__ uint4 issue_q[kLocalMaxProducers];  // MMAs posted to the issuing lane
 
   const uint32_t warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t D = P.D, H = P.H, C = P.C, T = P.T;
@@ -109,7 +108,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
     abort_flag = 0;
     red_n = 0;
     reduce_flag = 0;
-    for (uint32_t i = 0; i < 8 * D + 1 + P.n_slots; ++i) mbar_init(&bars[i], 1);
+    for (uint32_t i = 0; i < 8 * D + 1 + P.n_slots; ++i) mbar_init(&bars[i], i == 8 * D ? 32u : 1u);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -356,25 +355,31 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
     if (lane == 0) trace_mark(P, 18 + d);
   } else if (warp == 4) {
     // ================== MMA issue (lane q follows producer q) ==================
+    // Every lane whose producer has a slab ready issues that slab's MMA and
+    // commits itself: the ready lanes issue in the same instructions, which
+    // the tensor core takes about twice as fast as one thread issuing them in
+    // turn.  Each producer's MMAs come from one lane, in slab order, into that
+    // producer's own accumulators, so the accumulation order is fixed.
     const uint32_t q = lane;
     uint32_t pb = 0, pe = 0;
     if (q < D) producer_range(ub, ue, D, q, &pb, &pe);
     uint32_t acc_slot = q < D ? producer_first_slot(ub, ue, D, q, n_kt) : 0u;
-    uint32_t u = pb, us = 0, nslab = 0;
+    uint32_t u = pb, us = 0, nslab = 0, n_issued = 0;
     uint32_t cur_seg = pb / n_kt;
     uint32_t fresh = (1u << H) - 1u;  // bit h: next MMA into half h starts the accumulator
     const uint32_t n_us = H * C;
     // descriptor fields shared by both operands: LBO 16 B, SBO 256 B,
     // version 1, 32-byte swizzle; only the start address differs
     const uint64_t dhi = (1ull << 16) | (16ull << 32) | (1ull << 46) | (6ull << 61);
-    const uint32_t w_base = smem_u32(wslots), x_base = smem_u32(xslots);
+    const uint32_t a_s = smem_u32(wslots) + 2 * q * kSlabBytes;
+    const uint32_t b_s = smem_u32(xslots) + 2 * q * T * 32;
     long long idle_since = clock64();
     for (;;) {
       const bool has = q < D && u < pe;
       if (__ballot_sync(0xFFFFFFFFu, has) == 0) break;
       const uint32_t slot = nslab & 1u;
       const bool ready = has && mbar_try_wait(&w_full[2 * q + slot], (nslab >> 1) & 1u);
-      uint32_t rmask = __ballot_sync(0xFFFFFFFFu, ready);
+      const uint32_t rmask = __ballot_sync(0xFFFFFFFFu, ready);
       if (rmask == 0) {
         if (*abort) break;
         if (clock64() - idle_since > kWaitBudgetCycles) {
@@ -400,34 +405,30 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
       // this lane's slab: accumulator columns, accumulate flag, segment end
       const uint32_t h = us % H;
       const uint32_t col = (acc_slot * H + h) * T;
-      const uint32_t accum = ((fresh >> h) & 1u) ? 0u : 1u;
-      const bool seg_end = (us + 1 == n_us) && (u + 1 == pe || (u + 1) / n_kt != cur_seg);
-      // the producer reuses this slot only if it has a slab nslab + 2
-      const bool reuse = nslab + 2 < (pe - pb) * n_us;
-      const uint32_t info = slot | (accum << 1) | ((seg_end ? 1u : 0u) << 2) | ((reuse ? 1u : 0u) << 3);
-      // each ready lane posts its MMA (accumulator address, operand start
-      // addresses, flags); lane 0 then issues the round without further warp
-      // collectives
-      if (ready) {
-        const uint32_t a_lo = (w_base + (2 * q + slot) * kSlabBytes) >> 4;
-        const uint32_t b_lo = (x_base + (2 * q + slot) * T * 32) >> 4;
-        issue_q[q] = make_uint4(tmem_base + col, a_lo | (b_lo << 16), info, acc_slot);
-      }
-      __syncwarp();
-      if (lane == 0) {
+      const bool accum = ((fresh >> h) & 1u) == 0u;
+      const uint32_t d_tmem = tmem_base + col;
+      const uint64_t a_desc = dhi | ((a_s + slot * kSlabBytes) >> 4);
+      const uint64_t b_desc = dhi | ((b_s + slot * T * 32) >> 4);
+      // the lanes that start an accumulator and the lanes that add to one
+      // issue in separate instructions, so that the accumulate flag of an
+      // instruction is the same on every lane issuing it
+      if (ready && !accum) {
         tc_fence_after();
-        while (rmask) {
-          const uint32_t r = __ffs(rmask) - 1;
-          rmask &= rmask - 1;
-          const uint4 v = issue_q[r];
-          const uint32_t s_r = v.z & 1u;
-          umma_f16(v.x, dhi | (v.y & 0xFFFFu), dhi | (v.y >> 16), P.idesc, (v.z >> 1) & 1u);
-          if (v.z & 8u) umma_commit(&w_empty[2 * r + s_r]);
-          if (v.z & 4u) umma_commit(&acc_full[v.w]);
-        }
+        umma_f16(d_tmem, a_desc, b_desc, P.idesc, 0u);
+      }
+      __syncwarp();
+      if (ready && accum) {
+        tc_fence_after();
+        umma_f16(d_tmem, a_desc, b_desc, P.idesc, 1u);
       }
       __syncwarp();
       if (ready) {
+        const bool seg_end = (us + 1 == n_us) && (u + 1 == pe || (u + 1) / n_kt != cur_seg);
+        // the producer reuses this slot only if it has a slab nslab + 2
+        const bool reuse = nslab + 2 < (pe - pb) * n_us;
+        if (reuse) umma_commit(&w_empty[2 * q + slot]);
+        if (seg_end) umma_commit(&acc_full[acc_slot]);
+        ++n_issued;
         fresh &= ~(1u << h);
         ++nslab;
         if (++us == n_us) {
@@ -440,10 +441,14 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
           }
         }
       }
+      __syncwarp();
     }
     if (lane == 0) trace_mark(P, 35);
-    // retirement of every MMA this CTA issued (waited for before TMEM is freed)
-    if (lane == 0) umma_commit(mma_done);
+    // retirement of every MMA this CTA issued (waited for before TMEM is
+    // freed): 32 arrivals, a commit from each lane that issued MMAs (it
+    // fires once they are done) and a plain arrival from the others
+    if (n_issued) umma_commit(mma_done);
+    else mbar_arrive(mma_done);
     __syncwarp();
   } else {
     // ===================== epilogue (warps 0-3, 128 threads) =====================
@@ -540,7 +545,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
   }
   // the split-K reductions this CTA arrived last for, on every thread
   if (reduce_flag) {
-    __threadfence();
+    fence_acq_rel_gpu();  // acquire: the counter showed every contributor arrived
     for (uint32_t k = 0; k < red_n; ++k)
       if ((reduce_flag >> k) & 1u) splitk_reduce(P, red_seg[k], threadIdx.x, blockDim.x);
   }

@@ -426,8 +426,9 @@ __device__ __forceinline__ bool tile_end(TileCursor& tc, bool single) {
 // (bytes, unwrapped; advanced by the words the whole warp consumed); lut_s:
 // slot-table address; ring_s: ring address; lt: %lanemask_lt.  Slot lookup,
 // state update, ballot of the lanes that need a word, prefix count, word
-// merge by byte permute (valid because a lane needing a word has x < 2^16),
-// predicated select.  The ring base of the step, ring_s + pos mod 2048, is
+// merge by one byte permute (x << 16 | w, valid because a lane needing a word
+// has x < 2^16, or x unchanged) whose selector is picked while the word load
+// is in flight.  The ring base of the step, ring_s + pos mod 2048, is
 // computed beside the state chain; the lane's word is at base + 2 * prefix
 // with no wrap test, the mirror behind the ring covering the at most 62 bytes
 // a step can run past its end.  Every lane loads the word at its prefix
@@ -439,7 +440,7 @@ __device__ __forceinline__ uint32_t decode_step(uint32_t& x, uint32_t& pos, uint
   asm volatile(
       "{\n\t"
       ".reg .pred p;\n\t"
-      ".reg .b32 a, q, f, b, bal, t, pre, cnt, off, w, xs, pb;\n\t"
+      ".reg .b32 a, q, f, b, bal, t, pre, cnt, off, w, sel, pb;\n\t"
       "and.b32 a, %0, 4095;\n\t"
       "shl.b32 a, a, 2;\n\t"
       "add.u32 a, a, %3;\n\t"
@@ -452,15 +453,14 @@ __device__ __forceinline__ uint32_t decode_step(uint32_t& x, uint32_t& pos, uint
       "mad.lo.u32 %0, f, q, b;\n\t"
       "setp.lt.u32 p, %0, 65536;\n\t"
       "vote.sync.ballot.b32 bal, p, 0xffffffff;\n\t"
+      "selp.b32 sel, 0x5410, 0x7654, p;\n\t"
       "and.b32 t, bal, %5;\n\t"
       "popc.b32 pre, t;\n\t"
       "popc.b32 cnt, bal;\n\t"
       "mad.lo.u32 off, pre, 2, pb;\n\t"
       "ld.shared.u16 w, [off];\n\t"
-      "prmt.b32 xs, w, %0, 0x5410;\n\t"
-      "selp.b32 %0, xs, %0, p;\n\t"
-      "shl.b32 cnt, cnt, 1;\n\t"
-      "add.u32 %1, %1, cnt;\n\t"
+      "prmt.b32 %0, w, %0, sel;\n\t"
+      "mad.lo.u32 %1, cnt, 2, %1;\n\t"
       "}"
       : "+r"(x), "+r"(pos), "=&r"(e)
       : "r"(lut_s), "r"(ring_s), "r"(lt));
