@@ -62,14 +62,21 @@ __device__ __forceinline__ float row_scale(const GemmDev& P, uint32_t n) {
 __device__ __forceinline__ void epi_emit16(const GemmDev& P, const float (&v)[16], bool complete,
                                            float scale, float* part, uint32_t p, uint32_t h,
                                            uint32_t tok0, uint32_t n, uint32_t e) {
+  // tokens past M are padding: neither stored nor reduced
+  const uint32_t m0 = p * P.T_pass + tok0;
+  const uint32_t nv = P.M > m0 ? min(16u, P.M - m0) : 0u;
+  if (complete) {
+    float* y = P.Y + static_cast<uint64_t>(m0) * P.L.N + n;
 #pragma unroll
-  for (int q = 0; q < 16; ++q) {
-    const uint32_t m = p * P.T_pass + tok0 + q;
-    if (complete) {
-      if (m < P.M) P.Y[static_cast<uint64_t>(m) * P.L.N + n] = v[q] * scale;
-    } else {
-      part[(static_cast<uint64_t>(h) * P.T_pass + tok0 + q) * 128 + e] = v[q];
+    for (uint32_t q = 0; q < 16; ++q) {
+      if (q < nv) *y = v[q] * scale;
+      y += P.L.N;
     }
+  } else {
+    float* d = part + (static_cast<uint64_t>(h) * P.T_pass + tok0) * 128 + e;
+#pragma unroll
+    for (uint32_t q = 0; q < 16; ++q)
+      if (q < nv) d[q * 128] = v[q];
   }
 }
 

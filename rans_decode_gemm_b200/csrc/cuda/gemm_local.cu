@@ -475,12 +475,16 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
       uint32_t sb = sa + 1;
       while (sb < ns && slot_seg[sb] == seg) ++sb;
       // sum the segment's accumulators in slot order, two 16-column TMEM
-      // loads in flight per wait
+      // loads in flight per wait.  The accumulators of a segment complete
+      // close together (at the end of the producers' work): the first one is
+      // polled for alone (a cheap poll while the producers still decode),
+      // then all of them are tested together with overlapping tests.
+      wait_live(&acc_full[sa], 0, abort, P.status, 6, 64);
+      wait_all_live(&acc_full[sa], sb - sa, 0, abort, P.status, 6, 32);
+      tc_fence_after();
       float acc[2][16];
       for (uint32_t k = sa; k < sb;) {
         const uint32_t nb = (nck == 1 && k + 1 < sb) ? 2u : 1u;
-        for (uint32_t j = 0; j < nb; ++j) wait_live(&acc_full[k + j], 0, abort, P.status, 6, 64);
-        tc_fence_after();
         uint32_t v[2][16];
         const uint32_t taddr = tmem_base + ((32 * warp) << 16) + k * H * T;
         tmem_ld16(taddr, v[0]);

@@ -73,6 +73,37 @@ __device__ __forceinline__ bool mbar_try_wait_s(uint32_t bar_s, uint32_t parity)
       : "memory");
   return ok != 0;
 }
+// Non-blocking test of four consecutive barriers (8 bytes apart) at once:
+// true if each has completed the phase with the given parity.  The four tests
+// are independent instructions, so their latencies overlap.
+__device__ __forceinline__ bool mbar_test4_s(uint32_t bar_s, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p0, p1, p2, p3;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p0, [%1], %2;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p1, [%1+8], %2;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p2, [%1+16], %2;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p3, [%1+24], %2;\n\t"
+      "and.pred p0, p0, p1;\n\t"
+      "and.pred p2, p2, p3;\n\t"
+      "and.pred p0, p0, p2;\n\t"
+      "selp.u32 %0, 1, 0, p0;\n\t}"
+      : "=r"(ok)
+      : "r"(bar_s), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_test_s(uint32_t bar_s, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar_s), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return mbar_try_wait_s(smem_u32(bar), parity);
 }

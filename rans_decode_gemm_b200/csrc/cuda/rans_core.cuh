@@ -84,6 +84,33 @@ __device__ __forceinline__ bool wait_live_s(uint32_t bar_s, uint32_t parity, vol
   return true;
 }
 
+// wait_live for n consecutive barriers (bars[0 .. n-1]).  Each pass tests
+// them four at a time with independent instructions instead of one dependent
+// wait after another: a test's latency is a few hundred cycles, so testing
+// barriers that are already complete one by one costs more than the work
+// that follows.
+__device__ __forceinline__ bool wait_all_live(uint64_t* bars, uint32_t n, uint32_t parity,
+                                              volatile uint32_t* abort, uint32_t* status,
+                                              uint32_t site, uint32_t backoff_ns) {
+  const uint32_t b0 = smem_u32(bars);
+  long long t0 = 0;
+  for (uint32_t pass = 0;; ++pass) {
+    bool all = true;
+    uint32_t k = 0;
+    for (; k + 4 <= n; k += 4) all = mbar_test4_s(b0 + 8 * k, parity) && all;
+    for (; k < n; ++k) all = mbar_test_s(b0 + 8 * k, parity) && all;
+    if (all) return true;
+    if (pass == 0) t0 = clock64();
+    if (*abort) return false;
+    if (clock64() - t0 > kWaitBudgetCycles) {
+      *abort = 1u;
+      atomicOr(status, kStatusTimeout | (1u << (8 + site)));
+      return false;
+    }
+    if (backoff_ns) __nanosleep(backoff_ns);
+  }
+}
+
 // Bounded wait used when draining copies before exit; ignores the abort flag
 // (bulk copies always complete on their own).
 __device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, uint32_t* status) {
