@@ -37,6 +37,17 @@
 // order), then the u16 words in decoder consumption order, then zero bytes up
 // to a 16-byte boundary.
 //
+// Wide-state variant (state_bits = 64; the same pages leave the state width
+// open): 64-bit state x in [L, L*b) with L = 2^32 and b = 2^32 (32-bit words),
+// and the renormalisation test made once per PAIR of consecutive symbols of a
+// lane (steps 2i and 2i+1) instead of once per symbol.  Decoding two symbols
+// from x >= 2^32 leaves x >= 2^8 (each step divides by at most 2^12), so one
+// 32-bit word always restores x >= L.  Encoder side, for a pair (a, b) coded
+// in reverse (b first, then a): the state must lie in
+// [(L >> 2n) f_a f_b, (L >> 2n) b f_a f_b) = [2^8 f_a f_b, 2^40 f_a f_b), so
+// one word is pushed first if x >= 2^40 f_a f_b.  Tile bytes: 32 little-endian
+// u64 final states, then the u32 words in decoder order, then zero padding.
+//
 // Build: g++ -O2 -std=c++17 -shared -fPIC -pthread ans_oracle.cpp -o liboracle.so
 
 #include <algorithm>
@@ -58,6 +69,8 @@ enum {
 const uint32_t kLanes = 32;          // substreams per tile, one per warp lane
 const uint64_t kL = 1ull << 16;      // lower bound of the state interval
 const uint32_t kWordBits = 16;       // renormalisation word width (b = 2^16)
+const uint64_t kLWide = 1ull << 32;  // wide variant: lower bound of the state interval
+const uint32_t kWideWordBits = 32;   // wide variant: renormalisation word width (b = 2^32)
 
 int alphabet_of(int dtype) { return dtype == DT_INT4 ? 16 : 256; }
 
@@ -171,9 +184,25 @@ uint64_t decode_symbol(uint64_t x, const Codebook& cb, int* sym) {
   return (uint64_t)cb.f[s] * (x >> cb.n) + slot - cb.c[s];
 }
 
+// Wide variant, one pair (a = the earlier symbol, b = the later one) coded in
+// reverse: push one 32-bit word if x >= 2^40 f_a f_b (compared in 128 bits:
+// the bound is 2^64 when f_a = f_b = 4096), then code b, then a.
+uint64_t encode_pair_wide(uint64_t x, uint32_t fa, uint32_t ca, uint32_t fb, uint32_t cb_,
+                          const Codebook& cb, std::vector<uint32_t>* pushed) {
+  unsigned __int128 x_max = ((unsigned __int128)fa * fb) << 40;
+  if ((unsigned __int128)x >= x_max) {
+    pushed->push_back((uint32_t)(x & 0xFFFFFFFFull));
+    x >>= kWideWordBits;
+  }
+  x = (x / fb) * cb.M + (x % fb) + cb_;
+  x = (x / fa) * cb.M + (x % fa) + ca;
+  return x;
+}
+
 struct Layout {
   int dtype;
   uint32_t N, K, tile_n, tile_k;
+  int state_bits;  // 32, or 64 for the wide-state variant
   uint64_t n_tiles() const { return (uint64_t)(N / tile_n) * (K / tile_k); }
   uint64_t tile_symbols() const { return (uint64_t)tile_n * tile_k; }
 };
@@ -186,29 +215,48 @@ int encode_tile(const Layout& lay, const void* w, const Codebook& cb, uint64_t t
   const uint64_t n0 = (t / kt_count) * lay.tile_n;
   const uint64_t k0 = (t % kt_count) * lay.tile_k;
   const uint32_t steps = (uint32_t)(lay.tile_symbols() / kLanes);
+  const bool wide = lay.state_bits == 64;
+  auto sym_of = [&](uint32_t l, uint32_t j) {
+    uint32_t row, col;
+    lane_map(lay.tile_n, l, j, &row, &col);
+    return symbol_at(lay.dtype, w, (n0 + row) * lay.K + (k0 + col));
+  };
   uint64_t x[kLanes];
-  for (uint32_t l = 0; l < kLanes; ++l) x[l] = kL;
+  for (uint32_t l = 0; l < kLanes; ++l) x[l] = wide ? kLWide : kL;
   std::vector<uint16_t> pushed;
+  std::vector<uint32_t> pushed32;
   // Reverse order: last step first, and inside a step the highest lane first,
   // so that the decoder (first step first, lowest lane first) meets the words
-  // in the reverse of the order in which they were pushed.
-  for (uint32_t jj = steps; jj-- > 0;) {
-    for (uint32_t ll = kLanes; ll-- > 0;) {
-      uint32_t row, col;
-      lane_map(lay.tile_n, ll, jj, &row, &col);
-      uint64_t idx = (n0 + row) * lay.K + (k0 + col);
-      uint32_t s = symbol_at(lay.dtype, w, idx);
-      if (s >= cb.f.size() || cb.f[s] == 0) return ERR_ALPHABET;
-      x[ll] = encode_step(x[ll], cb.f[s], cb.c[s], cb, &pushed);
+  // in the reverse of the order in which they were pushed.  The wide variant
+  // walks pairs of steps (2i, 2i + 1) the same way.
+  if (!wide) {
+    for (uint32_t jj = steps; jj-- > 0;) {
+      for (uint32_t ll = kLanes; ll-- > 0;) {
+        uint32_t s = sym_of(ll, jj);
+        if (s >= cb.f.size() || cb.f[s] == 0) return ERR_ALPHABET;
+        x[ll] = encode_step(x[ll], cb.f[s], cb.c[s], cb, &pushed);
+      }
+    }
+  } else {
+    for (uint32_t ii = steps / 2; ii-- > 0;) {
+      for (uint32_t ll = kLanes; ll-- > 0;) {
+        uint32_t sa = sym_of(ll, 2 * ii), sb = sym_of(ll, 2 * ii + 1);
+        if (sa >= cb.f.size() || cb.f[sa] == 0 || sb >= cb.f.size() || cb.f[sb] == 0)
+          return ERR_ALPHABET;
+        x[ll] = encode_pair_wide(x[ll], cb.f[sa], cb.c[sa], cb.f[sb], cb.c[sb], cb, &pushed32);
+      }
     }
   }
   out->clear();
+  const int state_bytes = wide ? 8 : 4;
   for (uint32_t l = 0; l < kLanes; ++l)
-    for (int b = 0; b < 4; ++b) out->push_back((uint8_t)((x[l] >> (8 * b)) & 0xFF));
+    for (int b = 0; b < state_bytes; ++b) out->push_back((uint8_t)((x[l] >> (8 * b)) & 0xFF));
   for (size_t q = pushed.size(); q-- > 0;) {
     out->push_back((uint8_t)(pushed[q] & 0xFF));
     out->push_back((uint8_t)(pushed[q] >> 8));
   }
+  for (size_t q = pushed32.size(); q-- > 0;)
+    for (int b = 0; b < 4; ++b) out->push_back((uint8_t)((pushed32[q] >> (8 * b)) & 0xFF));
   while (out->size() % 16 != 0) out->push_back(0);
   // ---- 8. raw side stream (bf16): per tile, byte of (lane l, step j) at
   //         (j / 8) * 256 + l * 8 + (j % 8).
@@ -422,13 +470,70 @@ int oracle_rans_decode_message(uint32_t state, const uint16_t* words, int n_word
   return OK;
 }
 
+// ---- Single-lane wide-state coder (state_bits = 64), for hand-checkable examples
+// len must be even (pairs).  states[i] (i even) receives the state after coding
+// the pair (msg[i], msg[i+1]), so states[0] is the final state; odd entries are
+// left 0.  Words (u32) are returned in decoder consumption order.
+int oracle_rans64_encode_message(const uint8_t* msg, int len, const uint32_t* freq, int A,
+                                 uint64_t* states, uint32_t* words, int words_cap,
+                                 int* n_words) {
+  if (len % 2 != 0) return ERR_ARG;
+  Codebook cb;
+  int st = make_codebook(freq, A, 12, &cb);
+  if (st != OK) return st;
+  uint64_t x = kLWide;
+  std::vector<uint32_t> pushed;
+  for (int i = len - 2; i >= 0; i -= 2) {
+    uint32_t a = msg[i], b = msg[i + 1];
+    if (a >= (uint32_t)A || b >= (uint32_t)A || cb.f[a] == 0 || cb.f[b] == 0) return ERR_ALPHABET;
+    x = encode_pair_wide(x, cb.f[a], cb.c[a], cb.f[b], cb.c[b], cb, &pushed);
+    states[i] = x;
+    states[i + 1] = 0;
+  }
+  if ((int)pushed.size() > words_cap) return ERR_BUFFER_TOO_SMALL;
+  *n_words = (int)pushed.size();
+  for (size_t q = 0; q < pushed.size(); ++q) words[q] = pushed[pushed.size() - 1 - q];
+  return OK;
+}
+
+// Decodes len (even) symbols; states[i] receives the state entering symbol i
+// (states[0] = the given state), states[len] the end state.  After every
+// second symbol one word is read if x < 2^32.
+int oracle_rans64_decode_message(uint64_t state, const uint32_t* words, int n_words,
+                                 const uint32_t* freq, int A, int len, uint8_t* msg,
+                                 uint64_t* states) {
+  if (len % 2 != 0) return ERR_ARG;
+  Codebook cb;
+  int st = make_codebook(freq, A, 12, &cb);
+  if (st != OK) return st;
+  uint64_t x = state;
+  int cursor = 0;
+  for (int i = 0; i < len; ++i) {
+    states[i] = x;
+    int s;
+    x = decode_symbol(x, cb, &s);
+    msg[i] = (uint8_t)s;
+    if (i % 2 == 1 && x < kLWide) {
+      if (cursor >= n_words) return ERR_CORRUPT;
+      x = (x << kWideWordBits) | words[cursor++];
+    }
+  }
+  states[len] = x;
+  if (x != kLWide || cursor != n_words) return ERR_CORRUPT;
+  return OK;
+}
+
 // Worst-case stream size: every symbol may push one word, plus states and
 // padding per tile.
-uint64_t oracle_encode_bound(uint32_t N, uint32_t K, uint32_t tile_n, uint32_t tile_k) {
+// (Wide variant: 8-byte states and at most one 4-byte word per pair of
+// symbols, so the same 2 bytes per symbol.)
+uint64_t oracle_encode_bound(uint32_t N, uint32_t K, uint32_t tile_n, uint32_t tile_k,
+                             int state_bits) {
   if (!layout_ok(N, K, tile_n, tile_k)) return 0;
+  if (state_bits != 32 && state_bits != 64) return 0;
   uint64_t S = (uint64_t)tile_n * tile_k;
   uint64_t n_tiles = (uint64_t)(N / tile_n) * (K / tile_k);
-  return n_tiles * (4 * kLanes + 2 * S + 16);
+  return n_tiles * ((uint64_t)(state_bits / 8) * kLanes + 2 * S + 16);
 }
 
 // ---- Layer encode ([SB s3.1]): tiles, one shared codebook, offset index -----
@@ -438,13 +543,15 @@ uint64_t oracle_encode_bound(uint32_t N, uint32_t K, uint32_t tile_n, uint32_t t
 int oracle_encode(int dtype, const void* w, uint32_t N, uint32_t K, uint32_t tile_n,
                   uint32_t tile_k, const uint32_t* freq, int prob_bits, uint8_t* stream,
                   uint64_t cap, uint64_t* stream_bytes, uint64_t* offsets, uint8_t* raw,
-                  int threads) {
+                  int threads, int state_bits) {
   if (dtype < 0 || dtype > 2) return ERR_ARG;
+  if (state_bits != 32 && state_bits != 64) return ERR_ARG;
   if (!layout_ok(N, K, tile_n, tile_k)) return ERR_SHAPE;
+  if (state_bits == 64 && prob_bits != 12) return ERR_ARG;  // the pair bound assumes n = 12
   Codebook cb;
   int st = make_codebook(freq, alphabet_of(dtype), prob_bits, &cb);
   if (st != OK) return st;
-  Layout lay{dtype, N, K, tile_n, tile_k};
+  Layout lay{dtype, N, K, tile_n, tile_k, state_bits};
   const uint64_t T = lay.n_tiles();
   std::vector<std::vector<uint8_t>> tiles(T);
   std::vector<int> status(T, OK);
@@ -473,13 +580,19 @@ int oracle_encode(int dtype, const void* w, uint32_t N, uint32_t K, uint32_t til
 int oracle_decode(int dtype, const uint8_t* stream, uint64_t stream_bytes,
                   const uint64_t* offsets, const uint8_t* raw, uint32_t N, uint32_t K,
                   uint32_t tile_n, uint32_t tile_k, const uint32_t* freq, int prob_bits,
-                  void* w_out, uint64_t tile_begin, uint64_t tile_end, int threads) {
+                  void* w_out, uint64_t tile_begin, uint64_t tile_end, int threads,
+                  int state_bits) {
   if (dtype < 0 || dtype > 2) return ERR_ARG;
+  if (state_bits != 32 && state_bits != 64) return ERR_ARG;
   if (!layout_ok(N, K, tile_n, tile_k)) return ERR_SHAPE;
+  if (state_bits == 64 && prob_bits != 12) return ERR_ARG;
   Codebook cb;
   int st = make_codebook(freq, alphabet_of(dtype), prob_bits, &cb);
   if (st != OK) return st;
-  Layout lay{dtype, N, K, tile_n, tile_k};
+  Layout lay{dtype, N, K, tile_n, tile_k, state_bits};
+  const bool wide = state_bits == 64;
+  const uint64_t L = wide ? kLWide : kL;
+  const uint32_t state_bytes = wide ? 8 : 4, word_bytes = wide ? 4 : 2;
   const uint64_t T = lay.n_tiles();
   if (tile_end > T) tile_end = T;
   if (tile_begin > tile_end) return ERR_ARG;
@@ -490,27 +603,33 @@ int oracle_decode(int dtype, const uint8_t* stream, uint64_t stream_bytes,
   parallel_for(tile_begin, tile_end, threads, [&](uint64_t t) {
     int& result = status[t - tile_begin];
     uint64_t a = offsets[t], b = offsets[t + 1];
-    if (b < a || b > stream_bytes || b - a < 4 * kLanes || a % 16 != 0) { result = ERR_CORRUPT; return; }
+    if (b < a || b > stream_bytes || b - a < state_bytes * kLanes || a % 16 != 0) {
+      result = ERR_CORRUPT;
+      return;
+    }
     const uint8_t* tile = stream + a;
     const uint64_t len = b - a;
     uint64_t x[kLanes];
     for (uint32_t l = 0; l < kLanes; ++l) {
-      uint32_t v = 0;
-      for (int q = 0; q < 4; ++q) v |= (uint32_t)tile[4 * l + q] << (8 * q);
+      uint64_t v = 0;
+      for (uint32_t q = 0; q < state_bytes; ++q) v |= (uint64_t)tile[state_bytes * l + q] << (8 * q);
       x[l] = v;
-      if (x[l] < kL) { result = ERR_CORRUPT; return; }
+      if (x[l] < L) { result = ERR_CORRUPT; return; }
     }
-    uint64_t cursor = 4 * kLanes;
+    uint64_t cursor = (uint64_t)state_bytes * kLanes;
     const uint64_t n0 = (t / kt_count) * tile_n, k0 = (t % kt_count) * tile_k;
     for (uint32_t j = 0; j < steps; ++j) {
       for (uint32_t l = 0; l < kLanes; ++l) {
         int s;
         x[l] = decode_symbol(x[l], cb, &s);
-        if (x[l] < kL) {
-          if (cursor + 2 > len) { result = ERR_CORRUPT; return; }
-          uint32_t word = tile[cursor] | ((uint32_t)tile[cursor + 1] << 8);
-          cursor += 2;
-          x[l] = (x[l] << kWordBits) | word;
+        // a word after every symbol (narrow), after the second of a pair (wide)
+        const bool test = !wide || (j % 2 == 1);
+        if (test && x[l] < L) {
+          if (cursor + word_bytes > len) { result = ERR_CORRUPT; return; }
+          uint64_t word = 0;
+          for (uint32_t q = 0; q < word_bytes; ++q) word |= (uint64_t)tile[cursor + q] << (8 * q);
+          cursor += word_bytes;
+          x[l] = (x[l] << (8 * word_bytes)) | word;
         }
         uint32_t row, col;
         lane_map(tile_n, l, j, &row, &col);
@@ -529,7 +648,7 @@ int oracle_decode(int dtype, const uint8_t* stream, uint64_t stream_bytes,
       }
     }
     for (uint32_t l = 0; l < kLanes; ++l)
-      if (x[l] != kL) { result = ERR_CORRUPT; return; }
+      if (x[l] != L) { result = ERR_CORRUPT; return; }
     if (len - cursor >= 16) { result = ERR_CORRUPT; return; }
     for (uint64_t q = cursor; q < len; ++q)
       if (tile[q] != 0) { result = ERR_CORRUPT; return; }

@@ -55,11 +55,14 @@ def lib():
             L.oracle_code_cost.restype = C.c_double
             L.oracle_rans_encode_message.argtypes = [P, i32, P, i32, i32, P, P, i32, P]
             L.oracle_rans_decode_message.argtypes = [u32, P, i32, P, i32, i32, i32, P, P]
-            L.oracle_encode_bound.argtypes = [u32, u32, u32, u32]
+            L.oracle_rans64_encode_message.argtypes = [P, i32, P, i32, P, P, i32, P]
+            L.oracle_rans64_decode_message.argtypes = [u64, P, i32, P, i32, i32, P, P]
+            L.oracle_encode_bound.argtypes = [u32, u32, u32, u32, i32]
             L.oracle_encode_bound.restype = u64
-            L.oracle_encode.argtypes = [i32, P, u32, u32, u32, u32, P, i32, P, u64, P, P, P, i32]
+            L.oracle_encode.argtypes = [i32, P, u32, u32, u32, u32, P, i32, P, u64, P, P, P, i32,
+                                        i32]
             L.oracle_decode.argtypes = [i32, P, u64, P, P, u32, u32, u32, u32, P, i32, P,
-                                        u64, u64, i32]
+                                        u64, u64, i32, i32]
             L.oracle_gemm.argtypes = [i32, P, u32, u32, P, u32, i32, P, u32, P, u32, P, i32]
             _lib = L
     return _lib
@@ -135,27 +138,54 @@ def decode_message(state: int, words, freq, length: int, prob_bits: int = 12):
     return st, msg[:length], states
 
 
-def encode_bound(N, K, tile_n, tile_k) -> int:
-    return lib().oracle_encode_bound(N, K, tile_n, tile_k)
+def encode_message64(msg, freq):
+    """Single-lane wide-state coder (64-bit state, 32-bit words, one test per
+    pair; 12-bit frequencies).  Returns (status, states[len] (even entries:
+    state after each pair), words[] (uint32, decoder order))."""
+    m = np.ascontiguousarray(msg, dtype=np.uint8)
+    f = np.ascontiguousarray(freq, dtype=np.uint32)
+    states = np.zeros(max(1, m.size), np.uint64)
+    words = np.zeros(max(1, m.size), np.uint32)
+    nw = C.c_int(0)
+    st = lib().oracle_rans64_encode_message(_p(m), m.size, _p(f), f.size, _p(states), _p(words),
+                                            words.size, C.byref(nw))
+    return st, states[:m.size], words[:nw.value]
 
 
-def encode(dtype, w, N, K, tile_n, tile_k, freq, prob_bits=12, threads=0):
-    """Returns (status, stream uint8[], offsets uint64[n_tiles+1], raw uint8[] or None)."""
+def decode_message64(state: int, words, freq, length: int):
+    """Single-lane wide-state decoder. Returns (status, msg[length], states[length+1])."""
+    w = np.ascontiguousarray(words, dtype=np.uint32)
+    f = np.ascontiguousarray(freq, dtype=np.uint32)
+    msg = np.zeros(max(1, length), np.uint8)
+    states = np.zeros(length + 1, np.uint64)
+    st = lib().oracle_rans64_decode_message(int(state), _p(w) if w.size else None, w.size, _p(f),
+                                            f.size, length, _p(msg), _p(states))
+    return st, msg[:length], states
+
+
+def encode_bound(N, K, tile_n, tile_k, state_bits=32) -> int:
+    return lib().oracle_encode_bound(N, K, tile_n, tile_k, state_bits)
+
+
+def encode(dtype, w, N, K, tile_n, tile_k, freq, prob_bits=12, threads=0, state_bits=32):
+    """Returns (status, stream uint8[], offsets uint64[n_tiles+1], raw uint8[] or None).
+    state_bits 64 selects the wide-state variant (64-bit states, 32-bit words,
+    one renormalisation test per pair of symbols)."""
     w = np.ascontiguousarray(w)
     f = np.ascontiguousarray(freq, dtype=np.uint32)
-    cap = encode_bound(N, K, tile_n, tile_k)
+    cap = encode_bound(N, K, tile_n, tile_k, state_bits)
     n_tiles = (N // tile_n) * (K // tile_k) if cap else 0
     stream = np.zeros(max(cap, 16), np.uint8)
     offsets = np.zeros(n_tiles + 1, np.uint64)
     raw = np.zeros(N * K, np.uint8) if dtype == BF16_SPLIT else None
     nbytes = C.c_uint64(0)
     st = lib().oracle_encode(dtype, _p(w), N, K, tile_n, tile_k, _p(f), prob_bits, _p(stream),
-                             cap, C.byref(nbytes), _p(offsets), _p(raw), threads)
+                             cap, C.byref(nbytes), _p(offsets), _p(raw), threads, state_bits)
     return st, stream[:nbytes.value].copy(), offsets, raw
 
 
 def decode(dtype, stream, offsets, raw, N, K, tile_n, tile_k, freq, prob_bits=12,
-           tile_begin=0, tile_end=None, out=None, threads=0):
+           tile_begin=0, tile_end=None, out=None, threads=0, state_bits=32):
     """Returns (status, decoded weights in the original packed format)."""
     stream = np.ascontiguousarray(stream, dtype=np.uint8)
     offsets = np.ascontiguousarray(offsets, dtype=np.uint64)
@@ -171,7 +201,7 @@ def decode(dtype, stream, offsets, raw, N, K, tile_n, tile_k, freq, prob_bits=12
         tile_end = offsets.size - 1
     st = lib().oracle_decode(dtype, _p(stream) if stream.size else None, stream.size, _p(offsets),
                              _p(raw), N, K, tile_n, tile_k, _p(f), prob_bits, _p(out),
-                             tile_begin, tile_end, threads)
+                             tile_begin, tile_end, threads, state_bits)
     return st, out
 
 

@@ -146,6 +146,149 @@ def test_equiprobable_16_is_bit_packing(oracle):
     assert ((states >= 65536) & (states < 131072)).all()
 
 
+# ---- wide-state variant (64-bit state, 32-bit words, one test per pair) ----------
+def test_rans64_hand_examples(oracle):
+    with open(os.path.join(GOLDEN, "rans64_hand_examples.json")) as fh:
+        ex = json.load(fh)["examples"]
+    for e in ex:
+        st, states, words = oracle.encode_message64(e["message"], e["freq"])
+        assert st == 0, e["name"]
+        assert [int(states[i]) for i in range(0, len(e["message"]), 2)] == e["pair_states"], e["name"]
+        assert [int(w) for w in words] == e["words"], e["name"]
+        st, msg, dstates = oracle.decode_message64(int(states[0]), words, e["freq"],
+                                                   len(e["message"]))
+        assert st == 0, e["name"]
+        assert [int(m) for m in msg] == e["message"]
+        assert [int(v) for v in dstates] == e["decode_states"], e["name"]
+
+
+def test_rans64_equiprobable_16_closed_form(oracle):
+    # f = 256 for all 16 symbols: coding s is x -> (x >> 8) << 12 | s << 8 |
+    # (x & 255), which lengthens x by exactly 4 bits; a pair adds 8 bits and a
+    # word leaves when x >= 2^40 * 256 * 256 = 2^56.  From x = 2^32 (33 bits)
+    # the state is 41, 49, 57 bits after pairs 1-3; pair 4 finds 57 bits, pushes
+    # 32 and ends at 33 bits again: one word every 4 pairs, floor(P / 4) words
+    # for P pairs, and the final state lies in [2^32, 2^33) when 4 divides P.
+    freq = np.full(16, 256, np.uint32)
+    rng = np.random.default_rng(8)
+    msg = rng.integers(0, 16, size=64).astype(np.uint8)
+    st, states, words = oracle.encode_message64(msg, freq)
+    assert st == 0 and words.size == 64 // 2 // 4
+    assert (1 << 32) <= int(states[0]) < (1 << 33)
+    x = 1 << 32
+    for i in range(len(msg) - 2, -1, -2):
+        if x >= (1 << 56):
+            x >>= 32
+        for s in (int(msg[i + 1]), int(msg[i])):
+            x = ((x >> 8) << 12) | (s << 8) | (x & 255)
+    assert x == int(states[0])
+    # tile form: 128 x 32 int4 tile (T = 128 symbols per lane, P = 64 pairs):
+    # 256 bytes of states + 32 lanes * 16 words * 4 bytes
+    N, K = 128, 32
+    codes = rng.integers(-8, 8, size=(N, K)).astype(np.int8)
+    w = WL.pack_int4(codes)
+    st, stream, offsets, _ = oracle.encode(WL.INT4, w, N, K, 128, 32, freq, state_bits=64)
+    assert st == 0
+    T = N * K // 32
+    assert int(offsets[1]) == 256 + 32 * ((T // 2) // 4) * 4
+    states = np.frombuffer(stream[:256].tobytes(), np.uint64)
+    assert ((states >= (1 << 32)) & (states < (1 << 33))).all()
+    st, out = oracle.decode(WL.INT4, stream, offsets, None, N, K, 128, 32, freq, state_bits=64)
+    assert st == 0 and np.array_equal(out, w)
+
+
+def test_rans64_single_symbol_never_moves(oracle):
+    # f = 4096: the pair bound 2^40 * 2^24 = 2^64 is above every state, and
+    # coding leaves x unchanged, so a tile is its 32 states 2^32 and nothing else.
+    freq = np.zeros(256, np.uint32)
+    freq[7] = 4096
+    w = np.full(128 * 64, 7, np.uint8)
+    st, stream, offsets, _ = oracle.encode(WL.FP8_E4M3, w, 128, 64, 128, 64, freq, state_bits=64)
+    assert st == 0 and int(offsets[1]) == 256
+    assert (np.frombuffer(stream[:256].tobytes(), np.uint64) == (1 << 32)).all()
+
+
+@pytest.mark.parametrize("name,N,K", [("tiny_int4", 512, 512), ("bf16_4096", 256, 512),
+                                      ("llama8b_mlp", 256, 512), ("int4_70b", 512, 256),
+                                      ("fp8_405b", 256, 512)])
+def test_rans64_encode_decode_identity(oracle, name, N, K):
+    cfg, d = _small(name, N, K)
+    counts = oracle.histogram(cfg.dtype, d["w"], N * K)
+    _, freq = oracle.normalize(counts)
+    st, stream, offsets, raw = oracle.encode(cfg.dtype, d["w"], N, K, cfg.tile_n, cfg.tile_k,
+                                             freq, state_bits=64)
+    assert st == 0
+    assert (offsets % 16 == 0).all() and (np.diff(offsets.astype(np.int64)) > 0).all()
+    st, out = oracle.decode(cfg.dtype, stream, offsets, raw, N, K, cfg.tile_n, cfg.tile_k, freq,
+                            state_bits=64)
+    assert st == 0 and np.array_equal(out, d["w"])
+    # the other variant's decoder does not accept the stream
+    st, _ = oracle.decode(cfg.dtype, stream, offsets, raw, N, K, cfg.tile_n, cfg.tile_k, freq)
+    assert st == 6
+
+
+def test_rans64_fuzz_identity_and_corruption(oracle):
+    rng = np.random.default_rng(12)
+    for trial in range(9):
+        dtype = [WL.INT4, WL.BF16_SPLIT, WL.FP8_E4M3][trial % 3]
+        tile_n = [128, 256][trial % 2]
+        tile_k = [16, 32, 64][trial % 3]
+        N, K = tile_n * int(rng.integers(1, 3)), tile_k * int(rng.integers(1, 4))
+        A = 16 if dtype == WL.INT4 else 256
+        k = int(rng.integers(1, A + 1))
+        support = rng.choice(A, size=k, replace=False)
+        p = rng.dirichlet(np.full(k, float(rng.choice([0.05, 0.5, 5.0]))))
+        syms = support[rng.choice(k, size=N * K, p=p)]
+        if dtype == WL.INT4:
+            w = WL.pack_int4((syms - 8).astype(np.int8))
+        elif dtype == WL.BF16_SPLIT:
+            w = ((rng.integers(0, 256, N * K) & 0x80) << 8 | (syms << 7) |
+                 rng.integers(0, 128, N * K)).astype(np.uint16)
+        else:
+            w = syms.astype(np.uint8)
+        counts = oracle.histogram(dtype, w, N * K)
+        _, freq = oracle.normalize(counts)
+        st, stream, offsets, raw = oracle.encode(dtype, w, N, K, tile_n, tile_k, freq,
+                                                 state_bits=64)
+        assert st == 0
+        st, out = oracle.decode(dtype, stream, offsets, raw, N, K, tile_n, tile_k, freq,
+                                state_bits=64)
+        assert st == 0 and np.array_equal(out, w), trial
+        # a flipped bit in a state or a word is flagged or changes the output
+        if stream.size > 256:
+            bad = stream.copy()
+            pos = int(rng.integers(0, int(offsets[1])))
+            bad[pos] ^= np.uint8(1 << int(rng.integers(0, 8)))
+            st, out = oracle.decode(dtype, bad, offsets, raw, N, K, tile_n, tile_k, freq,
+                                    state_bits=64)
+            assert st == 6 or not np.array_equal(out, w)
+
+
+@pytest.mark.parametrize("name,N,K,band", [("tiny_int4", 512, 512, 0.40),
+                                           ("bf16_4096", 512, 1024, 0.22),
+                                           ("int4_70b", 512, 1024, 0.12),
+                                           ("fp8_405b", 256, 1024, 0.12)])
+def test_rans64_size_within_band_of_entropy(oracle, name, N, K, band):
+    # The wide states end with about 32 + 1.4 bits of slack per lane instead of
+    # about 16 + 1.4 (the state interval starts at 2^32, not 2^16), so the gap
+    # to the entropy grows by about 16 bits per lane and tile: +0.125 bit/weight
+    # for 4096-symbol tiles, +0.0625 for 8192, +0.03 for 16384.  The 4096-symbol
+    # tiles leave the pages' 0.2-bit band.
+    cfg, d = _small(name, N, K)
+    counts = oracle.histogram(cfg.dtype, d["w"], N * K)
+    H = oracle.entropy(counts)
+    _, freq = oracle.normalize(counts)
+    st, s32, _, _ = oracle.encode(cfg.dtype, d["w"], N, K, cfg.tile_n, cfg.tile_k, freq)
+    st64, s64, _, _ = oracle.encode(cfg.dtype, d["w"], N, K, cfg.tile_n, cfg.tile_k, freq,
+                                    state_bits=64)
+    assert st == 0 and st64 == 0
+    gap = 8.0 * s64.size / (N * K) - H
+    assert -0.01 < gap < band, (name, gap)
+    tiles = (N // cfg.tile_n) * (K // cfg.tile_k)
+    extra = 8.0 * (s64.size - s32.size) / (tiles * 32)   # bits per lane and tile
+    assert 6 < extra < 26, (name, extra)
+
+
 # ---- e4m3 ------------------------------------------------------------------------
 def test_e4m3_matches_torch_float8(oracle):
     codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
