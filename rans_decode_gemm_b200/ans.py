@@ -46,7 +46,7 @@ class AnsCodebook(C.Structure):
 
 class AnsLayout(C.Structure):
     _fields_ = [("dtype", C.c_uint32), ("N", C.c_uint32), ("K", C.c_uint32),
-                ("tile_n", C.c_uint32), ("tile_k", C.c_uint32)]
+                ("tile_n", C.c_uint32), ("tile_k", C.c_uint32), ("state_bits", C.c_uint32)]
 
 
 class AnsTiles(C.Structure):
@@ -118,8 +118,11 @@ def _stream(stream):
     return C.c_void_p(stream.cuda_stream)
 
 
-def make_layout(dtype: int, N: int, K: int, tile_n: int, tile_k: int) -> AnsLayout:
-    return AnsLayout(dtype, N, K, tile_n, tile_k)
+def make_layout(dtype: int, N: int, K: int, tile_n: int, tile_k: int,
+                state_bits: int = 32) -> AnsLayout:
+    """state_bits 64 selects the wide-state stream variant (64-bit lane states,
+    32-bit words, one renormalisation test per pair of symbols)."""
+    return AnsLayout(dtype, N, K, tile_n, tile_k, state_bits)
 
 
 # ---- the C ABI, one Python function per entry point -----------------------------

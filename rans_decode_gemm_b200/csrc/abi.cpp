@@ -25,6 +25,7 @@ uint32_t alphabet_of(uint32_t dtype) { return dtype == ANS_INT4 ? 16u : 256u; }
 ans_status check_layout(const ans_layout* l) {
   if (!l) return ANS_ERR_ARG;
   if (l->dtype > ANS_FP8_E4M3) return ANS_ERR_ARG;
+  if (l->state_bits != 0 && l->state_bits != 32 && l->state_bits != 64) return ANS_ERR_ARG;
   if (!anshost::layout_valid(l->N, l->K, l->tile_n, l->tile_k)) return ANS_ERR_SHAPE;
   return ANS_OK;
 }
@@ -82,6 +83,7 @@ void fill_layer(const ans_tiles* t, ansdev::LayerDev* L) {
   L->n_kt = ly.K / ly.tile_k;
   L->n_tiles = (ly.N / ly.tile_n) * L->n_kt;
   L->dtype = ly.dtype;
+  L->wide = ly.state_bits == 64 ? 1u : 0u;
   L->alphabet = t->codebook.alphabet;
   L->single_symbol = ansdev::kNoSymbolHost;
   for (uint32_t s = 0; s < t->codebook.alphabet; ++s) {
@@ -227,7 +229,8 @@ ans_status ans_encode_bound(const ans_layout* layout, uint64_t* max_stream_bytes
   ans_status st = check_layout(layout);
   if (st != ANS_OK) return st;
   if (!max_stream_bytes) return ANS_ERR_ARG;
-  *max_stream_bytes = anshost::encode_bound(layout->N, layout->K, layout->tile_n, layout->tile_k);
+  *max_stream_bytes = anshost::encode_bound(layout->N, layout->K, layout->tile_n, layout->tile_k,
+                                           layout->state_bits == 64);
   return ANS_OK;
 }
 
@@ -243,7 +246,8 @@ ans_status ans_encode_tiles(const void* h_w, const ans_layout* layout,
   uint32_t freq[256] = {0};
   for (uint32_t s = 0; s < codebook->alphabet; ++s) freq[s] = codebook->freq[s];
   int r = anshost::encode(layout->dtype, h_w, layout->N, layout->K, layout->tile_n,
-                          layout->tile_k, freq, h_stream, cap, stream_bytes, h_offsets, h_raw);
+                          layout->tile_k, freq, h_stream, cap, stream_bytes, h_offsets, h_raw,
+                          layout->state_bits == 64);
   if (r == 3) return ANS_ERR_ALPHABET;
   if (r == 4) return ANS_ERR_BUFFER_TOO_SMALL;
   return r == 0 ? ANS_OK : ANS_ERR_ARG;

@@ -43,7 +43,7 @@ __device__ __forceinline__ void store_group(void* out, uint64_t idx, const uint3
   }
 }
 
-template <uint32_t DT>
+template <uint32_t DT, bool kWide>
 __global__ void __launch_bounds__(kDecMaxWarps * 32, 2)
     decode_tiles_kernel(const __grid_constant__ LayerDev L, void* __restrict__ out,
                         uint32_t* __restrict__ status) {
@@ -123,15 +123,14 @@ __global__ void __launch_bounds__(kDecMaxWarps * 32, 2)
             for (int k = 0; k < 8; ++k) e[k] = single_e;
           } else {
             tile_group(pipe, L, seq, tc, lane, abort, status);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) e[k] = decode_step(tc.x, tc.pos, lut_s, pipe.ring_s, lt);
+            decode_group<kWide>(tc, lut_s, pipe.ring_s, lt, e);
           }
           const uint64_t idx = base + (4 * h + i) * row_step + 16 * s + 8 * c;
           store_group<DT>(out, idx, e, raw8);
         }
       }
     }
-    if (!tile_end(tc, single) && lane == 0) atomicOr(status, kStatusCorrupt);
+    if (!tile_end(L, tc, single) && lane == 0) atomicOr(status, kStatusCorrupt);
   }
   pipe_drain(pipe, status);
 }
@@ -191,13 +190,13 @@ __global__ void __launch_bounds__(kHistWarps * 32)
   }
 }
 
-template <uint32_t DT>
+template <uint32_t DT, bool kWide>
 static cudaError_t launch_decode_variant(const LayerDev& L, void* out, uint32_t* status,
                                          cudaStream_t stream, uint32_t blocks, uint32_t warps) {
-  cudaError_t e = cudaFuncSetAttribute(decode_tiles_kernel<DT>,
+  cudaError_t e = cudaFuncSetAttribute(decode_tiles_kernel<DT, kWide>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(decode_tiles_kernel<DT>, dim3(blocks), dim3(warps * 32), kDecSmem, stream, L,
+  return launch_pdl(decode_tiles_kernel<DT, kWide>, dim3(blocks), dim3(warps * 32), kDecSmem, stream, L,
                     out, status);
 }
 
@@ -212,9 +211,14 @@ cudaError_t launch_decode_tiles(const LayerDev& L, void* out, uint32_t* status,
   if (warps < 1) warps = 1;
   uint32_t blocks = (L.n_tiles + warps - 1) / warps;
   if (blocks > 2 * sms) blocks = 2 * sms;
-  if (L.dtype == kDtBf16Split) return launch_decode_variant<kDtBf16Split>(L, out, status, stream, blocks, warps);
-  if (L.dtype == kDtInt4) return launch_decode_variant<kDtInt4>(L, out, status, stream, blocks, warps);
-  return launch_decode_variant<kDtFp8>(L, out, status, stream, blocks, warps);
+  if (L.wide) {
+    if (L.dtype == kDtBf16Split) return launch_decode_variant<kDtBf16Split, true>(L, out, status, stream, blocks, warps);
+    if (L.dtype == kDtInt4) return launch_decode_variant<kDtInt4, true>(L, out, status, stream, blocks, warps);
+    return launch_decode_variant<kDtFp8, true>(L, out, status, stream, blocks, warps);
+  }
+  if (L.dtype == kDtBf16Split) return launch_decode_variant<kDtBf16Split, false>(L, out, status, stream, blocks, warps);
+  if (L.dtype == kDtInt4) return launch_decode_variant<kDtInt4, false>(L, out, status, stream, blocks, warps);
+  return launch_decode_variant<kDtFp8, false>(L, out, status, stream, blocks, warps);
 }
 
 cudaError_t launch_histogram(const void* w, uint64_t n_bytes, uint32_t dtype, uint64_t* hist,

@@ -113,7 +113,7 @@ __device__ __forceinline__ void for_each_mma_step(const GemmDev& P, uint32_t u_b
 }
 
 // ---------------------------------------------------------------------------
-template <bool kDecode, uint32_t kFmt>
+template <bool kDecode, uint32_t kFmt, bool kWide>
 __global__ void __launch_bounds__(kMaxThreads, 1)
     fused_gemm_kernel(const __grid_constant__ GemmDev P) {
   extern __shared__ __align__(2048) uint8_t smem[];
@@ -272,8 +272,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
               for (int k = 0; k < 8; ++k) e[k] = L.single_symbol << 12;
             } else {
               tile_group(pipe, L, seq, tc, lane, abort, P.status);
-#pragma unroll
-              for (int k = 0; k < 8; ++k) e[k] = decode_step(tc.x, tc.pos, lut_s, pipe.ring_s, lt);
+              decode_group<kWide>(tc, lut_s, pipe.ring_s, lt, e);
             }
             if (kFmt == kFmtBf16Split) fmt_bf16_split(e, raw8, o);
             else if (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
@@ -317,7 +316,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         ++sc;
       }
       if (kDecode && !zero_tile) {
-        if (!tile_end(tc, single) && lane == 0) atomicOr(P.status, kStatusCorrupt);
+        if (!tile_end(L, tc, single) && lane == 0) atomicOr(P.status, kStatusCorrupt);
       }
     }
     if (kDecode) pipe_drain(pipe, P.status);
@@ -716,9 +715,9 @@ bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool dec
   return true;
 }
 
-template <bool kDecode, uint32_t kFmt>
+template <bool kDecode, uint32_t kFmt, bool kWide = false>
 static cudaError_t launch_variant(const GemmPlan& plan, const GemmDev& P, cudaStream_t stream) {
-  auto kern = fused_gemm_kernel<kDecode, kFmt>;
+  auto kern = fused_gemm_kernel<kDecode, kFmt, kWide>;
   // the opt-in shared-memory size is a per-device function attribute: set it
   // once per device and variant
   static int attr_set[64];
@@ -795,10 +794,18 @@ cudaError_t launch_gemm(const GemmPlan& plan, const LayerDev& L, bool decode, co
   if (plan.local) return launch_gemm_local(plan, P, decode, stream);
 
   switch (plan.fmt | (decode ? 0u : 8u)) {
-    case kFmtBf16Split: return launch_variant<true, kFmtBf16Split>(plan, P, stream);
-    case kFmtInt4Bf16: return launch_variant<true, kFmtInt4Bf16>(plan, P, stream);
-    case kFmtInt4F16Group: return launch_variant<true, kFmtInt4F16Group>(plan, P, stream);
-    case kFmtFp8F16: return launch_variant<true, kFmtFp8F16>(plan, P, stream);
+    case kFmtBf16Split:
+      return P.L.wide ? launch_variant<true, kFmtBf16Split, true>(plan, P, stream)
+                      : launch_variant<true, kFmtBf16Split>(plan, P, stream);
+    case kFmtInt4Bf16:
+      return P.L.wide ? launch_variant<true, kFmtInt4Bf16, true>(plan, P, stream)
+                      : launch_variant<true, kFmtInt4Bf16>(plan, P, stream);
+    case kFmtInt4F16Group:
+      return P.L.wide ? launch_variant<true, kFmtInt4F16Group, true>(plan, P, stream)
+                      : launch_variant<true, kFmtInt4F16Group>(plan, P, stream);
+    case kFmtFp8F16:
+      return P.L.wide ? launch_variant<true, kFmtFp8F16, true>(plan, P, stream)
+                      : launch_variant<true, kFmtFp8F16>(plan, P, stream);
     case 8 | kFmtBf16Split: return launch_variant<false, kFmtBf16Split>(plan, P, stream);
     case 8 | kFmtInt4Bf16: return launch_variant<false, kFmtInt4Bf16>(plan, P, stream);
     case 8 | kFmtInt4F16Group: return launch_variant<false, kFmtInt4F16Group>(plan, P, stream);

@@ -75,7 +75,7 @@ __device__ __forceinline__ void sts128(uint32_t addr, const uint32_t (&o)[4]) {
                : "memory");
 }
 
-template <bool kDecode, uint32_t kFmt>
+template <bool kDecode, uint32_t kFmt, bool kWide>
 __global__ void __launch_bounds__(kLocalThreads, 1)
     fused_gemm_local_kernel(const __grid_constant__ GemmDev P) {
   extern __shared__ __align__(2048) uint8_t smem[];
@@ -284,10 +284,18 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
                   if (gg > 0) store_prev(gg);
                 } else {
                   rp_group(pipe, tc.pos, lane, abort, P.status);
-                  e[0] = decode_step(tc.x, tc.pos, lut_s, pipe.ring_s, lt);
-                  if (gg > 0) store_prev(gg);
+                  if (kWide) {
+                    decode_pair(tc.xw, tc.pos, lut_s, pipe.ring_s, lt, e[0], e[1]);
+                    if (gg > 0) store_prev(gg);
 #pragma unroll
-                  for (int k = 1; k < 8; ++k) e[k] = decode_step(tc.x, tc.pos, lut_s, pipe.ring_s, lt);
+                    for (int k = 2; k < 8; k += 2)
+                      decode_pair(tc.xw, tc.pos, lut_s, pipe.ring_s, lt, e[k], e[k + 1]);
+                  } else {
+                    e[0] = decode_step(tc.x, tc.pos, lut_s, pipe.ring_s, lt);
+                    if (gg > 0) store_prev(gg);
+#pragma unroll
+                    for (int k = 1; k < 8; ++k) e[k] = decode_step(tc.x, tc.pos, lut_s, pipe.ring_s, lt);
+                  }
                 }
                 if (kFmt == kFmtBf16Split) fmt_bf16_split(e, raw8, o);
                 else if (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
@@ -347,7 +355,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
         };
         if (kDecode && (zero_tile || single)) run_slabs(std::true_type{});
         else run_slabs(std::false_type{});
-        if (kDecode && !zero_tile && !run_tile_end(tc, single) && lane == 0)
+        if (kDecode && !zero_tile && !run_tile_end(L, tc, single) && lane == 0)
           atomicOr(P.status, kStatusCorrupt);
       }
     }
@@ -555,9 +563,9 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
   }
 }
 
-template <bool kDecode, uint32_t kFmt>
+template <bool kDecode, uint32_t kFmt, bool kWide = false>
 static cudaError_t launch_local_variant(const GemmPlan& plan, const GemmDev& P, cudaStream_t stream) {
-  auto kern = fused_gemm_local_kernel<kDecode, kFmt>;
+  auto kern = fused_gemm_local_kernel<kDecode, kFmt, kWide>;
   static int attr_set[64];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -575,10 +583,18 @@ static cudaError_t launch_local_variant(const GemmPlan& plan, const GemmDev& P, 
 cudaError_t launch_gemm_local(const GemmPlan& plan, const GemmDev& P, bool decode,
                               cudaStream_t stream) {
   switch (plan.fmt | (decode ? 0u : 8u)) {
-    case kFmtBf16Split: return launch_local_variant<true, kFmtBf16Split>(plan, P, stream);
-    case kFmtInt4Bf16: return launch_local_variant<true, kFmtInt4Bf16>(plan, P, stream);
-    case kFmtInt4F16Group: return launch_local_variant<true, kFmtInt4F16Group>(plan, P, stream);
-    case kFmtFp8F16: return launch_local_variant<true, kFmtFp8F16>(plan, P, stream);
+    case kFmtBf16Split:
+      return P.L.wide ? launch_local_variant<true, kFmtBf16Split, true>(plan, P, stream)
+                      : launch_local_variant<true, kFmtBf16Split>(plan, P, stream);
+    case kFmtInt4Bf16:
+      return P.L.wide ? launch_local_variant<true, kFmtInt4Bf16, true>(plan, P, stream)
+                      : launch_local_variant<true, kFmtInt4Bf16>(plan, P, stream);
+    case kFmtInt4F16Group:
+      return P.L.wide ? launch_local_variant<true, kFmtInt4F16Group, true>(plan, P, stream)
+                      : launch_local_variant<true, kFmtInt4F16Group>(plan, P, stream);
+    case kFmtFp8F16:
+      return P.L.wide ? launch_local_variant<true, kFmtFp8F16, true>(plan, P, stream)
+                      : launch_local_variant<true, kFmtFp8F16>(plan, P, stream);
     case 8 | kFmtBf16Split: return launch_local_variant<false, kFmtBf16Split>(plan, P, stream);
     case 8 | kFmtInt4Bf16: return launch_local_variant<false, kFmtInt4Bf16>(plan, P, stream);
     case 8 | kFmtInt4F16Group: return launch_local_variant<false, kFmtInt4F16Group>(plan, P, stream);

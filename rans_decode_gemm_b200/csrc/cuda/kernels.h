@@ -20,6 +20,7 @@ struct LayerDev {
   uint32_t N, K, tile_n, tile_k;
   uint32_t n_kt, n_tiles, dtype, alphabet;
   uint32_t single_symbol;  // the symbol when the codebook has exactly one, else kNoSymbolHost
+  uint32_t wide;           // 1: wide-state variant (64-bit states, 32-bit words, pair steps)
   uint16_t freq[256];
   uint16_t cdf[257];
 };

@@ -12,6 +12,11 @@
 // the next 16-bit word of the tile's interleaved word stream (lanes in
 // increasing order, found with a ballot + prefix popcount).
 //
+// Wide-state variant (LayerDev::wide): 64-bit states in [2^32, 2^64) and
+// 32-bit words; a lane decodes two symbols (two slot lookups and updates)
+// before one renormalisation test, so the ballot, prefix count and word load
+// are made half as often.
+//
 // Compressed bytes reach shared memory through a per-warp ring of four
 // 512-byte slots filled by 1-D bulk copies (no multicast) that complete on
 // one mbarrier per slot; the ring runs up to three chunks ahead of the read
@@ -34,8 +39,9 @@ constexpr uint32_t kChunkBytes = 512;
 constexpr uint32_t kRingBytes = 2048;
 // A ring occupies kRingStride bytes: after its kRingBytes the first
 // kRingMirror bytes of slot 0 are repeated, so the words one decode step
-// reads (at most 64 bytes from the cursor) never wrap around.
-constexpr uint32_t kRingMirror = 64;
+// reads (at most 32 lanes x 4 bytes from the cursor) never wrap around.
+constexpr uint32_t kRingMirror = 128;
+constexpr uint64_t kStateLowWide = 1ull << 32;  // L of the wide-state variant
 constexpr uint32_t kRingStride = kRingBytes + kRingMirror;
 constexpr uint32_t kNoSymbol = kNoSymbolHost;
 
@@ -135,12 +141,15 @@ __device__ __forceinline__ void build_lut(uint32_t* lut, const LayerDev& L, uint
 }
 
 // Byte extent of tile t, validated against the format's rules.
+// Bytes of a tile's 32 lane states: u32 or (wide-state variant) u64 each.
+__device__ __forceinline__ uint32_t state_bytes(const LayerDev& L) { return L.wide ? 8u : 4u; }
+
 __device__ __forceinline__ bool tile_extent(const LayerDev& L, uint32_t t, uint64_t* start,
                                             uint32_t* bytes) {
   uint64_t a = __ldg(reinterpret_cast<const unsigned long long*>(L.offsets) + t);
   uint64_t b = __ldg(reinterpret_cast<const unsigned long long*>(L.offsets) + t + 1);
-  uint64_t max_bytes = 4ull * kLanes + 2ull * L.tile_n * L.tile_k + 16ull;
-  bool ok = (a % 16 == 0) && (b % 16 == 0) && b >= a + 4 * kLanes && b <= L.stream_bytes &&
+  uint64_t max_bytes = state_bytes(L) * kLanes + 2ull * L.tile_n * L.tile_k + 16ull;
+  bool ok = (a % 16 == 0) && (b % 16 == 0) && b >= a + state_bytes(L) * kLanes && b <= L.stream_bytes &&
             (b - a) <= max_bytes;
   *start = a;
   *bytes = ok ? static_cast<uint32_t>(b - a) : 0u;
@@ -243,12 +252,42 @@ __device__ __forceinline__ void pipe_enter_chunk(ChunkPipe& p, const LayerDev& L
 // Decode position inside the current tile of a warp.
 struct TileCursor {
   uint32_t x;      // lane state
+  uint64_t xw;     // lane state of the wide-state variant
   uint32_t pos;    // ring read position (bytes, unwrapped)
   uint32_t chunk;  // chunk holding pos when the pipeline was last consulted
   uint32_t cb;     // first chunk of the tile
   uint32_t last;   // last chunk of the tile
   uint32_t bytes;  // tile bytes (padded)
 };
+
+// Lane states at ring position pos (the state bytes must be resident): the
+// lane's u32, or its two u32 halves for the wide-state variant.  Each load
+// wraps on its own.  Returns the position after the states.
+__device__ __forceinline__ uint32_t load_states(const LayerDev& L, uint32_t ring_s, uint32_t pos,
+                                                uint32_t lane, TileCursor& tc) {
+  const uint32_t sb = state_bytes(L);
+  uint32_t lo, hi = 0;
+  asm volatile("ld.shared.u32 %0, [%1];"
+               : "=r"(lo)
+               : "r"(((pos + sb * lane) & (kRingBytes - 1)) + ring_s)
+               : "memory");
+  if (L.wide)
+    asm volatile("ld.shared.u32 %0, [%1];"
+                 : "=r"(hi)
+                 : "r"(((pos + sb * lane + 4) & (kRingBytes - 1)) + ring_s)
+                 : "memory");
+  tc.x = lo;
+  tc.xw = (static_cast<uint64_t>(hi) << 32) | lo;
+  return pos + sb * kLanes;
+}
+
+// A tile ends well when every lane is back at L and the cursor sits in the
+// last 16 bytes of the (padded) tile; a tile of a single-symbol codebook is
+// its states alone.
+__device__ __forceinline__ bool lanes_at_start(const LayerDev& L, const TileCursor& tc) {
+  return L.wide ? tc.xw == kStateLowWide : tc.x == kStateLow;
+}
+
 
 // Per-warp pipeline over a RUN: tiles that follow one another in the stream
 // (a warp that owns a contiguous range of tiles streams one contiguous byte
@@ -358,8 +397,8 @@ __device__ __forceinline__ bool run_extent(const LayerDev& L, uint32_t t0, uint3
                                            uint64_t* start, uint32_t* bytes) {
   const unsigned long long* off = reinterpret_cast<const unsigned long long*>(L.offsets);
   const uint64_t a = __ldg(off + t0), b = __ldg(off + t1 + 1);
-  const uint64_t max_tile = 4ull * kLanes + 2ull * L.tile_n * L.tile_k + 16ull;
-  const bool ok = (a % 16 == 0) && (b % 16 == 0) && b >= a + 4ull * kLanes * (t1 - t0 + 1) &&
+  const uint64_t max_tile = state_bytes(L) * kLanes + 2ull * L.tile_n * L.tile_k + 16ull;
+  const bool ok = (a % 16 == 0) && (b % 16 == 0) && b >= a + 1ull * state_bytes(L) * kLanes * (t1 - t0 + 1) &&
                   b <= L.stream_bytes && (b - a) <= max_tile * (t1 - t0 + 1) &&
                   (b - a) < (1ull << 31);
   *start = a;
@@ -376,29 +415,23 @@ __device__ __forceinline__ bool run_tile_begin(RunPipe& p, const LayerDev& L, ui
                                                uint64_t b, uint64_t run_start, uint32_t base,
                                                TileCursor& tc, uint32_t lane,
                                                volatile uint32_t* abort, uint32_t* status) {
-  const uint64_t max_tile = 4ull * kLanes + 2ull * L.tile_n * L.tile_k + 16ull;
-  if (b % 16 != 0 || b < a + 4ull * kLanes || b - a > max_tile || a < run_start ||
+  const uint64_t max_tile = state_bytes(L) * kLanes + 2ull * L.tile_n * L.tile_k + 16ull;
+  if (b % 16 != 0 || b < a + state_bytes(L) * kLanes || b - a > max_tile || a < run_start ||
       b > run_start + p.run_bytes)
     return false;
   tc.bytes = static_cast<uint32_t>(b - a);
   tc.cb = base + static_cast<uint32_t>(a - run_start);  // tile start position
   tc.pos = tc.cb;
   rp_group(p, tc.pos, lane, abort, status);
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];"
-               : "=r"(v)
-               : "r"(((tc.pos + 4 * lane) & (kRingBytes - 1)) + p.ring_s)
-               : "memory");
-  tc.x = v;
-  tc.pos += 4 * kLanes;
+  tc.pos = load_states(L, p.ring_s, tc.pos, lane, tc);
   return true;
 }
 
 // Ends a tile of a run (same integrity rule as tile_end).
-__device__ __forceinline__ bool run_tile_end(const TileCursor& tc, bool single) {
+__device__ __forceinline__ bool run_tile_end(const LayerDev& L, const TileCursor& tc, bool single) {
   const uint32_t used = tc.pos - tc.cb;
-  bool bad = (tc.x != kStateLow) || used > tc.bytes || tc.bytes - used >= 16;
-  if (single) bad = (tc.x != kStateLow) || tc.bytes != 4 * kLanes;
+  bool bad = !lanes_at_start(L, tc) || used > tc.bytes || tc.bytes - used >= 16;
+  if (single) bad = !lanes_at_start(L, tc) || tc.bytes != state_bytes(L) * kLanes;
   return !__any_sync(0xFFFFFFFFu, bad);
 }
 
@@ -416,13 +449,7 @@ __device__ __forceinline__ bool tile_begin(ChunkPipe& p, const LayerDev& L, cons
   tc.pos = tc.cb * kChunkBytes;
   tc.chunk = tc.cb;
   pipe_enter_chunk(p, L, seq, tc.chunk, tc.last, lane, abort, status);
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];"
-               : "=r"(v)
-               : "r"(((tc.pos + 4 * lane) & (kRingBytes - 1)) + p.ring_s)
-               : "memory");
-  tc.x = v;
-  tc.pos += 4 * kLanes;
+  tc.pos = load_states(L, p.ring_s, tc.pos, lane, tc);
   return true;
 }
 
@@ -440,10 +467,10 @@ __device__ __forceinline__ void tile_group(ChunkPipe& p, const LayerDev& L, cons
 // Ends a tile: rANS integrity (every lane back at L, words ending inside the
 // padding; a single-symbol tile holds only its states) and advances to the
 // next tile's first chunk.
-__device__ __forceinline__ bool tile_end(TileCursor& tc, bool single) {
+__device__ __forceinline__ bool tile_end(const LayerDev& L, TileCursor& tc, bool single) {
   const uint32_t used = tc.pos - tc.cb * kChunkBytes;
-  bool bad = (tc.x != kStateLow) || used > tc.bytes || tc.bytes - used >= 16;
-  if (single) bad = (tc.x != kStateLow) || tc.bytes != 4 * kLanes;
+  bool bad = !lanes_at_start(L, tc) || used > tc.bytes || tc.bytes - used >= 16;
+  if (single) bad = !lanes_at_start(L, tc) || tc.bytes != state_bytes(L) * kLanes;
   tc.cb = tc.last + 1;
   return !__any_sync(0xFFFFFFFFu, bad);
 }
@@ -492,6 +519,76 @@ __device__ __forceinline__ uint32_t decode_step(uint32_t& x, uint32_t& pos, uint
       : "+r"(x), "+r"(pos), "=&r"(e)
       : "r"(lut_s), "r"(ring_s), "r"(lt));
   return e;
+}
+
+// Two decode steps of the calling lane in the wide-state variant, then one
+// renormalisation test: slot lookup and 64-bit state update for the first
+// symbol, the same for the second, then the lanes with x < 2^32 take the next
+// 32-bit words of the shared stream in lane order (ballot, prefix count,
+// x = x << 32 | w).  Two decoded symbols from x >= 2^32 leave x >= 2^8, so one
+// word always suffices.  The ring base is computed as in decode_step; a step
+// reads at most 32 x 4 bytes past the cursor, inside the ring's mirror.
+__device__ __forceinline__ void decode_pair(uint64_t& x, uint32_t& pos, uint32_t lut_s,
+                                            uint32_t ring_s, uint32_t lt, uint32_t& e1,
+                                            uint32_t& e2) {
+  asm volatile(
+      "{\n\t"
+      ".reg .pred p;\n\t"
+      ".reg .b32 a, f, b, bal, t, pre, cnt, off, w, pb, xl, xh;\n\t"
+      ".reg .b64 q, f6, b6;\n\t"
+      "cvt.u32.u64 xl, %0;\n\t"
+      "and.b32 a, xl, 4095;\n\t"
+      "shl.b32 a, a, 2;\n\t"
+      "add.u32 a, a, %4;\n\t"
+      "ld.shared.u32 %2, [a];\n\t"
+      "and.b32 pb, %1, 2047;\n\t"
+      "add.u32 pb, pb, %5;\n\t"
+      "shr.u64 q, %0, 12;\n\t"
+      "shr.u32 f, %2, 20;\n\t"
+      "and.b32 b, %2, 4095;\n\t"
+      "cvt.u64.u32 b6, b;\n\t"
+      "cvt.u64.u32 f6, f;\n\t"
+      "mul.lo.u64 q, q, f6;\n\t"
+      "add.u64 %0, q, b6;\n\t"
+      "cvt.u32.u64 xl, %0;\n\t"
+      "and.b32 a, xl, 4095;\n\t"
+      "shl.b32 a, a, 2;\n\t"
+      "add.u32 a, a, %4;\n\t"
+      "ld.shared.u32 %3, [a];\n\t"
+      "shr.u64 q, %0, 12;\n\t"
+      "shr.u32 f, %3, 20;\n\t"
+      "and.b32 b, %3, 4095;\n\t"
+      "cvt.u64.u32 b6, b;\n\t"
+      "cvt.u64.u32 f6, f;\n\t"
+      "mul.lo.u64 q, q, f6;\n\t"
+      "add.u64 %0, q, b6;\n\t"
+      "mov.b64 {xl, xh}, %0;\n\t"
+      "setp.eq.u32 p, xh, 0;\n\t"
+      "vote.sync.ballot.b32 bal, p, 0xffffffff;\n\t"
+      "and.b32 t, bal, %6;\n\t"
+      "popc.b32 pre, t;\n\t"
+      "popc.b32 cnt, bal;\n\t"
+      "mad.lo.u32 off, pre, 4, pb;\n\t"
+      "ld.shared.u32 w, [off];\n\t"
+      "@p mov.b64 %0, {w, xl};\n\t"
+      "mad.lo.u32 %1, cnt, 4, %1;\n\t"
+      "}"
+      : "+l"(x), "+r"(pos), "=&r"(e1), "=&r"(e2)
+      : "r"(lut_s), "r"(ring_s), "r"(lt));
+}
+
+// The eight slot-table entries of one group of a lane: eight decode steps, or
+// (wide-state variant) four pair steps.
+template <bool kWide>
+__device__ __forceinline__ void decode_group(TileCursor& tc, uint32_t lut_s, uint32_t ring_s,
+                                             uint32_t lt, uint32_t (&e)[8]) {
+  if (kWide) {
+#pragma unroll
+    for (int k = 0; k < 8; k += 2) decode_pair(tc.xw, tc.pos, lut_s, ring_s, lt, e[k], e[k + 1]);
+  } else {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) e[k] = decode_step(tc.x, tc.pos, lut_s, ring_s, lt);
+  }
 }
 
 // ---- symbol -> MMA operand formatting ---------------------------------------

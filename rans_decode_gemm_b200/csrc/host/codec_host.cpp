@@ -42,6 +42,7 @@ std::vector<uint64_t> lane_order(uint32_t tile_n, uint32_t tile_k, uint64_t K) {
 }
 
 struct TileJob {
+  bool wide;  // wide-state variant: 64-bit states, 32-bit words, one test per symbol pair
   uint32_t dtype;
   const uint8_t* w;
   uint64_t K;
@@ -53,8 +54,12 @@ struct TileJob {
 
 // Codes one tile; appends its padded bytes to `out`.  Returns false if a
 // symbol has zero frequency.
+bool code_tile_wide(const TileJob& job, const std::vector<uint8_t>& sym, size_t S,
+                    std::vector<uint8_t>& out, std::vector<uint32_t>& words);
+
 bool code_tile(const TileJob& job, uint64_t t, std::vector<uint8_t>& out,
-               std::vector<uint8_t>& sym, std::vector<uint16_t>& words, uint8_t* raw_tile) {
+               std::vector<uint8_t>& sym, std::vector<uint16_t>& words,
+               std::vector<uint32_t>& words32, uint8_t* raw_tile) {
   const uint64_t origin = (t / job.n_kt) * job.tile_n * job.K + (t % job.n_kt) * job.tile_k;
   const size_t S = static_cast<size_t>(job.tile_n) * job.tile_k;
   const std::vector<uint64_t>& order = *job.order;
@@ -79,6 +84,7 @@ bool code_tile(const TileJob& job, uint64_t t, std::vector<uint8_t>& out,
     for (size_t q = 0; q < S; ++q) sym[q] = job.w[origin + order[q]];
   }
 
+  if (job.wide) return code_tile_wide(job, sym, S, out, words32);
   uint32_t x[kLanes];
   for (uint32_t l = 0; l < kLanes; ++l) x[l] = kStateLow;
   words.clear();
@@ -104,6 +110,46 @@ bool code_tile(const TileJob& job, uint64_t t, std::vector<uint8_t>& out,
     const uint16_t wv = words[words.size() - 1 - k];
     p[2 * k] = static_cast<uint8_t>(wv);
     p[2 * k + 1] = static_cast<uint8_t>(wv >> 8);
+  }
+  return true;
+}
+
+// Wide-state variant of one tile.  sym holds the tile's symbols in (step,
+// lane) order.  Pairs of steps (2p, 2p + 1) are coded last pair first and,
+// inside a pair step, highest lane first; a lane's state first gives up its low
+// 32 bits if x >= 2^40 f_a f_b (tested as x >> 40 >= f_a f_b, exact because the
+// bound is a multiple of 2^40), then takes b = step 2p + 1, then a = step 2p.
+bool code_tile_wide(const TileJob& job, const std::vector<uint8_t>& sym, size_t S,
+                    std::vector<uint8_t>& out, std::vector<uint32_t>& words) {
+  uint64_t x[kLanes];
+  for (uint32_t l = 0; l < kLanes; ++l) x[l] = 1ull << 32;
+  words.clear();
+  const size_t pairs = S / kLanes / 2;
+  for (size_t p = pairs; p-- > 0;) {
+    const uint8_t* sa = &sym[(2 * p) * kLanes];
+    const uint8_t* sb = sa + kLanes;
+    for (uint32_t l = kLanes; l-- > 0;) {
+      const uint32_t fa = job.freq[sa[l]], fb = job.freq[sb[l]];
+      if (fa == 0 || fb == 0) return false;
+      uint64_t v = x[l];
+      if ((v >> 40) >= static_cast<uint64_t>(fa) * fb) {
+        words.push_back(static_cast<uint32_t>(v));
+        v >>= 32;
+      }
+      v = (v / fb) * 4096u + (v % fb) + job.cdf[sb[l]];
+      v = (v / fa) * 4096u + (v % fa) + job.cdf[sa[l]];
+      x[l] = v;
+    }
+  }
+  const size_t base = out.size();
+  const size_t len = 8 * kLanes + 4 * words.size();
+  out.resize(base + ((len + 15) & ~static_cast<size_t>(15)), 0);
+  uint8_t* q = out.data() + base;
+  for (uint32_t l = 0; l < kLanes; ++l) std::memcpy(q + 8 * l, &x[l], 8);  // little-endian host
+  q += 8 * kLanes;
+  for (size_t k = 0; k < words.size(); ++k) {
+    const uint32_t wv = words[words.size() - 1 - k];
+    std::memcpy(q + 4 * k, &wv, 4);
   }
   return true;
 }
@@ -226,19 +272,21 @@ int normalize(const uint64_t* hist, uint32_t alphabet, uint32_t prob_bits, uint3
   return 0;
 }
 
-uint64_t encode_bound(uint32_t N, uint32_t K, uint32_t tile_n, uint32_t tile_k) {
+uint64_t encode_bound(uint32_t N, uint32_t K, uint32_t tile_n, uint32_t tile_k, bool wide) {
   if (!layout_valid(N, K, tile_n, tile_k)) return 0;
   const uint64_t tiles = static_cast<uint64_t>(N / tile_n) * (K / tile_k);
-  return tiles * (4ull * kLanes + 2ull * tile_n * tile_k + 16ull);
+  // at most one word per symbol (2 bytes) or per pair (4 bytes): 2 bytes a symbol
+  return tiles * ((wide ? 8ull : 4ull) * kLanes + 2ull * tile_n * tile_k + 16ull);
 }
 
 int encode(uint32_t dtype, const void* w, uint32_t N, uint32_t K, uint32_t tile_n,
            uint32_t tile_k, const uint32_t* freq, uint8_t* stream, uint64_t cap,
-           uint64_t* stream_bytes, uint64_t* offsets, uint8_t* raw) {
+           uint64_t* stream_bytes, uint64_t* offsets, uint8_t* raw, bool wide) {
   const uint32_t n_kt = K / tile_k;
   const uint64_t tiles = static_cast<uint64_t>(N / tile_n) * n_kt;
   const std::vector<uint64_t> order = lane_order(tile_n, tile_k, K);
   TileJob job;
+  job.wide = wide;
   job.dtype = dtype;
   job.w = static_cast<const uint8_t*>(w);
   job.K = K;
@@ -266,11 +314,12 @@ int encode(uint32_t dtype, const void* w, uint32_t N, uint32_t K, uint32_t tile_
       const uint64_t a = tiles * w_i / nw, b = tiles * (w_i + 1) / nw;
       std::vector<uint8_t> sym;
       std::vector<uint16_t> words;
+      std::vector<uint32_t> words32;
       words.reserve(S);
       for (uint64_t t = a; t < b; ++t) {
         const size_t before = bufs[w_i].size();
         uint8_t* raw_tile = (dtype == kBf16Split) ? raw + t * S : nullptr;
-        if (!code_tile(job, t, bufs[w_i], sym, words, raw_tile)) { ok[w_i] = 0; return; }
+        if (!code_tile(job, t, bufs[w_i], sym, words, words32, raw_tile)) { ok[w_i] = 0; return; }
         sizes[w_i].push_back(bufs[w_i].size() - before);
       }
     });

@@ -11,10 +11,12 @@ void histogram(uint32_t dtype, const void* w, uint64_t n_weights, uint64_t* hist
 double entropy_bits(const uint64_t* hist, uint32_t alphabet);
 // 0 ok, 1 bad argument, 3 too many present symbols.
 int normalize(const uint64_t* hist, uint32_t alphabet, uint32_t prob_bits, uint32_t* freq);
-uint64_t encode_bound(uint32_t N, uint32_t K, uint32_t tile_n, uint32_t tile_k);
+// wide: the wide-state variant (64-bit states, 32-bit words, one renormalisation
+// test per pair of symbols).
+uint64_t encode_bound(uint32_t N, uint32_t K, uint32_t tile_n, uint32_t tile_k, bool wide);
 // 0 ok, 3 symbol with zero frequency, 4 capacity too small (size still reported).
 int encode(uint32_t dtype, const void* w, uint32_t N, uint32_t K, uint32_t tile_n,
            uint32_t tile_k, const uint32_t* freq, uint8_t* stream, uint64_t cap,
-           uint64_t* stream_bytes, uint64_t* offsets, uint8_t* raw);
+           uint64_t* stream_bytes, uint64_t* offsets, uint8_t* raw, bool wide);
 
 }  // namespace anshost

@@ -40,17 +40,21 @@ def test_status_strings_and_layout_checks(ans_lib):
     assert ans.ans_layout_check(ans.make_layout(7, 512, 512, 128, 32)) == 1    # dtype
     assert ans.ans_layout_check(ans.make_layout(1, 0, 512, 128, 32)) == 2      # empty
     assert ans.ans_num_tiles(ans.make_layout(2, 53248, 16384, 128, 128)) == 53248
+    assert ans.ans_layout_check(ans.make_layout(0, 512, 512, 128, 32, 64)) == 0
+    assert ans.ans_layout_check(ans.make_layout(0, 512, 512, 128, 32, 0)) == 0    # 0 means 32
+    assert ans.ans_layout_check(ans.make_layout(0, 512, 512, 128, 32, 48)) == 1   # state width
 
 
 CASES = [("tiny_int4", 512, 512), ("bf16_4096", 512, 512), ("llama8b_mlp", 256, 1024),
          ("int4_70b", 512, 512), ("fp8_405b", 256, 1024)]
 
 
+@pytest.mark.parametrize("state_bits", [32, 64])
 @pytest.mark.parametrize("name,N,K", CASES)
-def test_host_codec_matches_oracle(oracle, ans_lib, name, N, K):
+def test_host_codec_matches_oracle(oracle, ans_lib, name, N, K, state_bits):
     cfg = WL.CONFIGS[name]
     d = WL.make_weights(cfg, 0, N=N, K=K)
-    lay = ans.make_layout(cfg.dtype, N, K, cfg.tile_n, cfg.tile_k)
+    lay = ans.make_layout(cfg.dtype, N, K, cfg.tile_n, cfg.tile_k, state_bits)
     hist = ans.ans_histogram_host(d["w"], lay)
     assert np.array_equal(hist, oracle.histogram(cfg.dtype, d["w"], N * K))
     assert abs(ans.ans_entropy(hist) - oracle.entropy(hist)) < 1e-12
@@ -60,14 +64,16 @@ def test_host_codec_matches_oracle(oracle, ans_lib, name, N, K):
     cdf = np.concatenate([[0], np.cumsum(f_or)])
     assert np.array_equal(np.ctypeslib.as_array(cb.cdf)[:ans.ALPHABET[cfg.dtype] + 1], cdf)
     stream, offsets, raw = ans.ans_encode_tiles(d["w"], lay, cb)
-    st, s_or, off_or, raw_or = oracle.encode(cfg.dtype, d["w"], N, K, cfg.tile_n, cfg.tile_k, f_or)
+    st, s_or, off_or, raw_or = oracle.encode(cfg.dtype, d["w"], N, K, cfg.tile_n, cfg.tile_k, f_or,
+                                             state_bits=state_bits)
     assert st == 0
     assert np.array_equal(offsets, off_or)
     assert np.array_equal(stream, s_or)
     if raw is not None:
         assert np.array_equal(raw, raw_or)
     # and the oracle decodes the library's stream back to the weights
-    st, out = oracle.decode(cfg.dtype, stream, offsets, raw, N, K, cfg.tile_n, cfg.tile_k, f_or)
+    st, out = oracle.decode(cfg.dtype, stream, offsets, raw, N, K, cfg.tile_n, cfg.tile_k, f_or,
+                            state_bits=state_bits)
     assert st == 0 and np.array_equal(out, d["w"])
 
 
