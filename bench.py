@@ -3,7 +3,8 @@
 
 Workload (the layer the headline metric is quoted on): a 4096 x 4096 bf16
 weight matrix drawn from N(0, 0.02), coded as an rANS exponent stream (one
-12-bit codebook, 128 x 64 tiles, 32 lanes) plus the raw sign/mantissa byte,
+12-bit codebook, 128 x 64 tiles, 32 lanes; by default the wide-state stream
+format, --state-bits 32 for 32-bit lane states) plus the raw sign/mantissa byte,
 multiplied by X (16 x 4096 bf16, N(0, 1)).  One step is one ans_gemm call
 (decode inside the GEMM, Y fp32).  Twelve copies of the compressed layer
 (together far larger than the 126 MB L2) rotate across steps, so every step
@@ -44,6 +45,13 @@ KERNEL_SOURCES = ["rans_decode_gemm_b200/csrc/cuda/gemm_local.cu",
                   "rans_decode_gemm_b200/csrc/cuda/launch.h"]
 
 
+def workload_name(state_bits):
+    fmt = ("64-bit lane states, 32-bit words, one renormalisation test per symbol pair"
+           if state_bits == 64 else "32-bit lane states, 16-bit words")
+    return ("bf16 split-stream 4096x4096 N(0,0.02), 128x64 tiles, 32 lanes, 12-bit freqs, "
+            f"{fmt}; X 16x4096 bf16 N(0,1); seed 1")
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -55,6 +63,9 @@ def parse():
                     help="every workload of the pages at full size, one JSON line per point "
                          "(instead of the benchmark line)")
     ap.add_argument("--sweep-configs", default="", help="comma-separated subset for --sweep")
+    ap.add_argument("--state-bits", type=int, default=64, choices=[32, 64],
+                    help="stream format: 64 = wide lane states (32-bit words, one "
+                         "renormalisation test per symbol pair), 32 = 32-bit states")
     ap.add_argument("--quick", action="store_true",
                     help="skip the context sweep and the CPU baseline (profiling runs)")
     return ap.parse_args()
@@ -163,10 +174,10 @@ def replica_gbs(world, bytes_per_step, ms_per_step):
     return world * bytes_per_step / (ms_per_step * 1e-3) / 1e9
 
 
-def build_layers(torch, ans, WL, device):
+def build_layers(torch, ans, WL, device, state_bits):
     cfg = WL.CONFIGS[WORKLOAD]
     d = WL.make_weights(cfg, 0)
-    lay = ans.make_layout(cfg.dtype, d["N"], d["K"], cfg.tile_n, cfg.tile_k)
+    lay = ans.make_layout(cfg.dtype, d["N"], d["K"], cfg.tile_n, cfg.tile_k, state_bits)
     # offline path through the library: GPU histogram -> codebook -> host encode
     dw = torch.from_numpy(d["w"].view(np.int16)).to(device)
     hist = torch.zeros(256, dtype=torch.int64, device=device)
@@ -195,7 +206,7 @@ def time_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=device)
         pg = dist
-    cfg, d, lay, layers, hist, encode_s, dw = build_layers(torch, ans, WL, device)
+    cfg, d, lay, layers, hist, encode_s, dw = build_layers(torch, ans, WL, device, args.state_bits)
     N, K, M = lay.N, lay.K, M_HEAD
     X_h = WL.make_x(cfg, M, K)
     X = torch.from_numpy(X_h.view(np.int16)).to(device)
@@ -309,8 +320,8 @@ def time_ours(args):
             "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "bf16 split-stream 4096x4096 N(0,0.02), 128x64 tiles, 32 lanes, "
-                                   "12-bit freqs; X 16x4096 bf16 N(0,1); seed 1",
+            "config": {"workload": workload_name(args.state_bits),
+                       "state_bits": args.state_bits,
                        "M": M, "N": N, "K": K, "global_batch": M * world,
                        "parallelism": f"replicas x{world}",
                        "l2": f"inputs larger than L2: {N_COPIES} rotating copies of the "
@@ -457,7 +468,7 @@ def sweep(args):
         for mi, (mname, mN, mK) in enumerate(cfg.matrices):
             d = WL.make_weights(cfg, mi)
             N, K = d["N"], d["K"]
-            lay = ans.make_layout(cfg.dtype, N, K, cfg.tile_n, cfg.tile_k)
+            lay = ans.make_layout(cfg.dtype, N, K, cfg.tile_n, cfg.tile_k, args.state_bits)
             dw = torch.from_numpy(d["w"].view(np.int16) if d["w"].dtype == np.uint16 else d["w"]).to(device)
             A = 256 if cfg.dtype != 0 else 16
             hist = torch.zeros(A, dtype=torch.int64, device=device)
@@ -507,6 +518,7 @@ def sweep(args):
                 t_c = timed_graph(cub, rep_for(t_c * len(cub)))
                 algo = layers[0].compressed_bytes + 2 * M * K + 4 * M * N
                 rec = {"workload": name, "matrix": mname, "N": N, "K": K, "M": M,
+                       "state_bits": args.state_bits,
                        "tile": f"{lay.tile_n}x{lay.tile_k}", "bits_per_weight": round(bpw, 4),
                        "entropy_bound_bits": round(bound, 4), "gap_bits": round(bpw - bound, 4),
                        "encode_s": round(encode_s, 2), "copies": copies,
@@ -550,7 +562,8 @@ def cpu_baseline(cfg, d, lay, layer, X_h, budget_s=20.0):
         t0 = time.perf_counter()
         st, _ = O.decode(cfg.dtype, layer.h_stream, layer.h_offsets, layer.h_raw, N, K,
                          lay.tile_n, lay.tile_k, freq, tile_begin=done_rb * n_kt,
-                         tile_end=(done_rb + 1) * n_kt, out=out, threads=cores)
+                         tile_end=(done_rb + 1) * n_kt, out=out, threads=cores,
+                         state_bits=lay.state_bits or 32)
         rows = np.arange(done_rb * lay.tile_n, (done_rb + 1) * lay.tile_n, dtype=np.uint32)
         O.gemm(cfg.dtype, X_h, M, K, out, N, rows=rows, threads=cores)
         t_spent += time.perf_counter() - t0
@@ -575,7 +588,8 @@ def time_reference(args):
     N, K, M = d["N"], d["K"], M_HEAD
     counts = O.histogram(cfg.dtype, d["w"], N * K)
     _, freq = O.normalize(counts)
-    st, stream, offsets, raw = O.encode(cfg.dtype, d["w"], N, K, cfg.tile_n, cfg.tile_k, freq)
+    st, stream, offsets, raw = O.encode(cfg.dtype, d["w"], N, K, cfg.tile_n, cfg.tile_k, freq,
+                                        state_bits=args.state_bits)
     X_h = WL.make_x(cfg, M, K)
     cores = os.cpu_count() or 1
     n_kt = K // cfg.tile_k
@@ -584,7 +598,8 @@ def time_reference(args):
 
     def one(rb):
         O.decode(cfg.dtype, stream, offsets, raw, N, K, cfg.tile_n, cfg.tile_k, freq,
-                 tile_begin=rb * n_kt, tile_end=(rb + 1) * n_kt, out=out, threads=cores)
+                 tile_begin=rb * n_kt, tile_end=(rb + 1) * n_kt, out=out, threads=cores,
+                 state_bits=args.state_bits)
         rows = np.arange(rb * cfg.tile_n, (rb + 1) * cfg.tile_n, dtype=np.uint32)
         O.gemm(cfg.dtype, X_h, M, K, out, N, rows=rows, threads=cores)
 
@@ -604,8 +619,7 @@ def time_reference(args):
             "warmup": args.warmup, "ms_per_step": round(per_rb_s * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": "bf16 split-stream 4096x4096 N(0,0.02), 128x64 tiles, 32 lanes, "
-                                   "12-bit freqs; X 16x4096 bf16 N(0,1); seed 1",
+            "config": {"workload": workload_name(args.state_bits), "state_bits": args.state_bits,
                        "M": M, "N": N, "K": K},
             "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores,
                              "kind": "oracle", "sample": sample},
