@@ -18,7 +18,7 @@
 // are made half as often.
 //
 // Compressed bytes reach shared memory through a per-warp ring of four
-// 512-byte slots filled by 1-D bulk copies (no multicast) that complete on
+// 1 KB slots filled by 1-D bulk copies (no multicast) that complete on
 // one mbarrier per slot; the ring runs up to three chunks ahead of the read
 // cursor, across tile boundaries.
 #pragma once
@@ -35,8 +35,8 @@ namespace ansdev {
 constexpr uint32_t kLanes = 32;
 constexpr uint32_t kSlots = 4096;        // 2^12 probability slots
 constexpr uint32_t kStateLow = 1u << 16; // L
-constexpr uint32_t kChunkBytes = 512;
-constexpr uint32_t kRingBytes = 2048;
+constexpr uint32_t kChunkBytes = 1024;
+constexpr uint32_t kRingBytes = 4096;
 // A ring occupies kRingStride bytes: after its kRingBytes the first
 // kRingMirror bytes of slot 0 are repeated, so the words one decode step
 // reads (at most 32 lanes x 4 bytes from the cursor) never wrap around.
@@ -482,7 +482,7 @@ __device__ __forceinline__ bool tile_end(const LayerDev& L, TileCursor& tc, bool
 // state update, ballot of the lanes that need a word, prefix count, word
 // merge by one byte permute (x << 16 | w, valid because a lane needing a word
 // has x < 2^16, or x unchanged) whose selector is picked while the word load
-// is in flight.  The ring base of the step, ring_s + pos mod 2048, is
+// is in flight.  The ring base of the step, ring_s + pos mod 4096, is
 // computed beside the state chain; the lane's word is at base + 2 * prefix
 // with no wrap test, the mirror behind the ring covering the at most 62 bytes
 // a step can run past its end.  Every lane loads the word at its prefix
@@ -499,7 +499,7 @@ __device__ __forceinline__ uint32_t decode_step(uint32_t& x, uint32_t& pos, uint
       "shl.b32 a, a, 2;\n\t"
       "add.u32 a, a, %3;\n\t"
       "ld.shared.u32 %2, [a];\n\t"
-      "and.b32 pb, %1, 2047;\n\t"
+      "and.b32 pb, %1, 4095;\n\t"
       "add.u32 pb, pb, %4;\n\t"
       "shr.u32 q, %0, 12;\n\t"
       "shr.u32 f, %2, 20;\n\t"
@@ -541,7 +541,7 @@ __device__ __forceinline__ void decode_pair(uint64_t& x, uint32_t& pos, uint32_t
       "shl.b32 a, a, 2;\n\t"
       "add.u32 a, a, %4;\n\t"
       "ld.shared.u32 %2, [a];\n\t"
-      "and.b32 pb, %1, 2047;\n\t"
+      "and.b32 pb, %1, 4095;\n\t"
       "add.u32 pb, pb, %5;\n\t"
       "shr.u64 q, %0, 12;\n\t"
       "shr.u32 f, %2, 20;\n\t"
