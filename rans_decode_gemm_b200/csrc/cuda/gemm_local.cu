@@ -558,8 +558,10 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
   // the split-K reductions this CTA arrived last for, on every thread
   if (reduce_flag) {
     fence_acq_rel_gpu();  // acquire: the counter showed every contributor arrived
-    for (uint32_t k = 0; k < red_n; ++k)
-      if ((reduce_flag >> k) & 1u) splitk_reduce(P, red_seg[k], threadIdx.x, blockDim.x);
+    const uint32_t both[2] = {red_seg[0], red_seg[1]};
+    if (!(reduce_flag == 3u && splitk_reduce2(P, both, threadIdx.x, blockDim.x)))
+      for (uint32_t k = 0; k < red_n; ++k)
+        if ((reduce_flag >> k) & 1u) splitk_reduce(P, red_seg[k], threadIdx.x, blockDim.x);
   }
 }
 
