@@ -165,6 +165,22 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
         }
         a_next = run_start;
       }
+      // raw sign/mantissa bytes (bf16, decode): groups g .. g + kRawAhead - 1
+      // of the current tile in flight.  A run's tiles are consecutive, so their
+      // raw blocks are too: the loads run on into the next tile's first groups,
+      // and the first tile's are issued here, before its first chunk is awaited.
+      const uint32_t groups = H * C * 8;
+      uint64_t rq[kRawAhead];
+#pragma unroll
+      for (uint32_t k = 0; k < kRawAhead; ++k) rq[k] = 0;
+      bool rq_ready = false;  // rq holds groups 0 .. kRawAhead - 1 of tile u
+      if (kDecode && kFmt == kFmtBf16Split && run_ok) {
+        const unsigned long long* r0 =
+            reinterpret_cast<const unsigned long long*>(L.raw + static_cast<uint64_t>(t0) * S) + lane;
+#pragma unroll
+        for (uint32_t k = 0; k < kRawAhead; ++k) rq[k] = __ldg(r0 + 32 * k);
+        rq_ready = true;
+      }
       for (; u < run_e; ++u) {
         const uint32_t t = u - p * n_tiles;
         const uint32_t rb = t / n_kt, kt = t - rb * n_kt;
@@ -197,17 +213,15 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
             gscale[q] = __float2half2_rn(sv);
           }
         }
-        // raw sign/mantissa bytes of groups g .. g + kRawAhead - 1 in flight
-        // (bf16, decode)
         const unsigned long long* raw_tile = nullptr;
-        uint64_t rq[kRawAhead];
-        const uint32_t groups = H * C * 8;
-#pragma unroll
-        for (uint32_t k = 0; k < kRawAhead; ++k) rq[k] = 0;
+        // the loads may run into the next tile's raw block while one exists
+        const uint32_t raw_lim = (t + 1 < n_tiles) ? groups + kRawAhead : groups;
         if (kDecode && kFmt == kFmtBf16Split && !zero_tile) {
           raw_tile = reinterpret_cast<const unsigned long long*>(L.raw + static_cast<uint64_t>(t) * S) + lane;
+          if (!rq_ready) {
 #pragma unroll
-          for (uint32_t k = 0; k < kRawAhead; ++k) rq[k] = __ldg(raw_tile + 32 * k);
+            for (uint32_t k = 0; k < kRawAhead; ++k) rq[k] = __ldg(raw_tile + 32 * k);
+          }
         }
         // the slabs of this tile; a tile of constant symbols (single-symbol
         // codebook, or zeros for a tile with bad offsets) takes a separate
@@ -275,7 +289,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
                 if (kFmt == kFmtBf16Split && (!kConst || !zero_tile)) {
 #pragma unroll
                   for (uint32_t k = 0; k + 1 < kRawAhead; ++k) rq[k] = rq[k + 1];
-                  if (g + kRawAhead < groups) rq[kRawAhead - 1] = __ldg(raw_tile + 32 * (g + kRawAhead));
+                  if (g + kRawAhead < raw_lim) rq[kRawAhead - 1] = __ldg(raw_tile + 32 * (g + kRawAhead));
                 }
                 uint32_t e[8];
                 if (kConst) {
@@ -355,6 +369,9 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
         };
         if (kDecode && (zero_tile || single)) run_slabs(std::true_type{});
         else run_slabs(std::false_type{});
+        // groups 0 .. kRawAhead - 1 of tile t + 1 are in rq if this tile's
+        // loads ran on into it
+        rq_ready = kDecode && kFmt == kFmtBf16Split && !zero_tile && t + 1 < n_tiles;
         if (kDecode && !zero_tile && !run_tile_end(L, tc, single) && lane == 0)
           atomicOr(P.status, kStatusCorrupt);
       }
