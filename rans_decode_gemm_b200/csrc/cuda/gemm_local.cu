@@ -165,8 +165,9 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
         }
         a_next = run_start;
       }
-      // raw sign/mantissa bytes (bf16, decode): groups g .. g + kRawAhead - 1
-      // of the current tile in flight.  A run's tiles are consecutive, so their
+      // raw sign/mantissa bytes (bf16, decode; read once, so loaded with the
+      // evict-first hint): groups g .. g + kRawAhead - 1 of the current tile in
+      // flight.  A run's tiles are consecutive, so their
       // raw blocks are too: the loads run on into the next tile's first groups,
       // and the first tile's are issued here, before its first chunk is awaited.
       const uint32_t groups = H * C * 8;
@@ -178,7 +179,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
         const unsigned long long* r0 =
             reinterpret_cast<const unsigned long long*>(L.raw + static_cast<uint64_t>(t0) * S) + lane;
 #pragma unroll
-        for (uint32_t k = 0; k < kRawAhead; ++k) rq[k] = __ldg(r0 + 32 * k);
+        for (uint32_t k = 0; k < kRawAhead; ++k) rq[k] = __ldcs(r0 + 32 * k);
         rq_ready = true;
       }
       for (; u < run_e; ++u) {
@@ -220,7 +221,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
           raw_tile = reinterpret_cast<const unsigned long long*>(L.raw + static_cast<uint64_t>(t) * S) + lane;
           if (!rq_ready) {
 #pragma unroll
-            for (uint32_t k = 0; k < kRawAhead; ++k) rq[k] = __ldg(raw_tile + 32 * k);
+            for (uint32_t k = 0; k < kRawAhead; ++k) rq[k] = __ldcs(raw_tile + 32 * k);
           }
         }
         // the slabs of this tile; a tile of constant symbols (single-symbol
@@ -289,7 +290,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
                 if (kFmt == kFmtBf16Split && (!kConst || !zero_tile)) {
 #pragma unroll
                   for (uint32_t k = 0; k + 1 < kRawAhead; ++k) rq[k] = rq[k + 1];
-                  if (g + kRawAhead < raw_lim) rq[kRawAhead - 1] = __ldg(raw_tile + 32 * (g + kRawAhead));
+                  if (g + kRawAhead < raw_lim) rq[kRawAhead - 1] = __ldcs(raw_tile + 32 * (g + kRawAhead));
                 }
                 uint32_t e[8];
                 if (kConst) {
