@@ -48,6 +48,14 @@
 // one word is pushed first if x >= 2^40 f_a f_b.  Tile bytes: 32 little-endian
 // u64 final states, then the u32 words in decoder order, then zero padding.
 //
+// int4 pairs (dtype 3; the pages call any discrete unit of a layer a symbol and
+// leave the unit open): one symbol per packed int4 byte, i.e. per pair of
+// consecutive K elements (k even, k + 1): s = (q_k + 8) | (q_{k+1} + 8) << 4,
+// which is the packed byte XOR 0x88; alphabet 256, half as many symbols per
+// tile.  Lane l's j-th pair symbol covers row l + 32 (4 h + i) and columns
+// 16 s + 2 kk, 16 s + 2 kk + 1 with g = j / 8, kk = j % 8, i = g % 4,
+// h = (g / 4) % (tile_n / 128), s = g / (4 tile_n / 128).
+//
 // Build: g++ -O2 -std=c++17 -shared -fPIC -pthread ans_oracle.cpp -o liboracle.so
 
 #include <algorithm>
@@ -59,7 +67,7 @@
 
 namespace {
 
-enum { DT_INT4 = 0, DT_BF16_SPLIT = 1, DT_FP8_E4M3 = 2 };
+enum { DT_INT4 = 0, DT_BF16_SPLIT = 1, DT_FP8_E4M3 = 2, DT_INT4_PAIRS = 3 };
 enum { SC_NONE = 0, SC_ROW_BF16 = 1, SC_ROW_F32 = 2, SC_GROUP_BF16 = 3 };
 enum {
   OK = 0, ERR_ARG = 1, ERR_SHAPE = 2, ERR_ALPHABET = 3, ERR_BUFFER_TOO_SMALL = 4,
@@ -73,6 +81,7 @@ const uint64_t kLWide = 1ull << 32;  // wide variant: lower bound of the state i
 const uint32_t kWideWordBits = 32;   // wide variant: renormalisation word width (b = 2^32)
 
 int alphabet_of(int dtype) { return dtype == DT_INT4 ? 16 : 256; }
+bool is_int4(int dtype) { return dtype == DT_INT4 || dtype == DT_INT4_PAIRS; }
 
 // ---- 1. Symbols: what is treated as "a sequence of discrete symbols" ---------
 // [SB s2.1]: a layer is a sequence of symbols (int4 value, fp8 code, ...).
@@ -89,8 +98,17 @@ int int4_code(const uint8_t* w, uint64_t idx) {
   return nib >= 8 ? nib - 16 : nib;
 }
 
+// int4 pairs (the "higher-rate" reading of a symbol): one symbol per pair of
+// consecutive K elements (idx even), low nibble = the even element's code + 8,
+// high nibble = the odd element's code + 8; alphabet 256.
+uint32_t pair_symbol_at(const void* w, uint64_t idx) {
+  uint32_t lo = (uint32_t)(int4_code((const uint8_t*)w, idx) + 8);
+  uint32_t hi = (uint32_t)(int4_code((const uint8_t*)w, idx + 1) + 8);
+  return lo | (hi << 4);
+}
 uint32_t symbol_at(int dtype, const void* w, uint64_t idx) {
   if (dtype == DT_INT4) return (uint32_t)(int4_code((const uint8_t*)w, idx) + 8);
+  if (dtype == DT_INT4_PAIRS) return pair_symbol_at(w, idx);
   if (dtype == DT_BF16_SPLIT) {
     uint16_t bits = ((const uint16_t*)w)[idx];
     return (bits >> 7) & 0xFFu;
@@ -129,6 +147,21 @@ void lane_map(uint32_t tile_n, uint32_t l, uint32_t j, uint32_t* row, uint32_t* 
   uint32_t s = g / (8 * H);
   *row = l + 32 * (4 * h + i);
   *col = 16 * s + 8 * c + kk;
+}
+
+// int4 pairs: lane l's j-th symbol covers the two elements at (row, col) and
+// (row, col + 1): g = j / 8, kk = j % 8, i = g % 4, h = (g / 4) % H,
+// s = g / (4 H); row = l + 32 (4 h + i), col = 16 s + 2 kk.  Eight symbols of a
+// lane are 16 consecutive K elements of one row, so every 32 steps a 128-row
+// x 16-column slab is complete.
+void lane_map_pairs(uint32_t tile_n, uint32_t l, uint32_t j, uint32_t* row, uint32_t* col) {
+  uint32_t g = j / 8, kk = j % 8;
+  uint32_t H = tile_n / 128;
+  uint32_t i = g % 4;
+  uint32_t h = (g / 4) % H;
+  uint32_t s = g / (4 * H);
+  *row = l + 32 * (4 * h + i);
+  *col = 16 * s + 2 * kk;
 }
 
 bool layout_ok(uint32_t N, uint32_t K, uint32_t tile_n, uint32_t tile_k) {
@@ -204,7 +237,8 @@ struct Layout {
   uint32_t N, K, tile_n, tile_k;
   int state_bits;  // 32, or 64 for the wide-state variant
   uint64_t n_tiles() const { return (uint64_t)(N / tile_n) * (K / tile_k); }
-  uint64_t tile_symbols() const { return (uint64_t)tile_n * tile_k; }
+  uint64_t tile_symbols() const { return (uint64_t)tile_n * tile_k / (dtype == DT_INT4_PAIRS ? 2 : 1); }
+  uint64_t tile_weights() const { return (uint64_t)tile_n * tile_k; }
 };
 
 // Encode one tile into `out` (states, words, padding).  Returns OK or
@@ -218,7 +252,8 @@ int encode_tile(const Layout& lay, const void* w, const Codebook& cb, uint64_t t
   const bool wide = lay.state_bits == 64;
   auto sym_of = [&](uint32_t l, uint32_t j) {
     uint32_t row, col;
-    lane_map(lay.tile_n, l, j, &row, &col);
+    if (lay.dtype == DT_INT4_PAIRS) lane_map_pairs(lay.tile_n, l, j, &row, &col);
+    else lane_map(lay.tile_n, l, j, &row, &col);
     return symbol_at(lay.dtype, w, (n0 + row) * lay.K + (k0 + col));
   };
   uint64_t x[kLanes];
@@ -329,7 +364,8 @@ double oracle_e4m3_value(uint8_t code) { return e4m3_value(code); }
 void oracle_histogram(int dtype, const void* w, uint64_t n_weights, uint64_t* counts) {
   int A = alphabet_of(dtype);
   for (int s = 0; s < A; ++s) counts[s] = 0;
-  for (uint64_t i = 0; i < n_weights; ++i) counts[symbol_at(dtype, w, i)]++;
+  const uint64_t step = dtype == DT_INT4_PAIRS ? 2 : 1;  // one pair symbol per 2 weights
+  for (uint64_t i = 0; i + step <= n_weights; i += step) counts[symbol_at(dtype, w, i)]++;
 }
 
 // Histogram of the raw sign/mantissa byte of bf16 weights (256 bins).
@@ -544,7 +580,7 @@ int oracle_encode(int dtype, const void* w, uint32_t N, uint32_t K, uint32_t til
                   uint32_t tile_k, const uint32_t* freq, int prob_bits, uint8_t* stream,
                   uint64_t cap, uint64_t* stream_bytes, uint64_t* offsets, uint8_t* raw,
                   int threads, int state_bits) {
-  if (dtype < 0 || dtype > 2) return ERR_ARG;
+  if (dtype < 0 || dtype > 3) return ERR_ARG;
   if (state_bits != 32 && state_bits != 64) return ERR_ARG;
   if (!layout_ok(N, K, tile_n, tile_k)) return ERR_SHAPE;
   if (state_bits == 64 && prob_bits != 12) return ERR_ARG;  // the pair bound assumes n = 12
@@ -582,7 +618,7 @@ int oracle_decode(int dtype, const uint8_t* stream, uint64_t stream_bytes,
                   uint32_t tile_n, uint32_t tile_k, const uint32_t* freq, int prob_bits,
                   void* w_out, uint64_t tile_begin, uint64_t tile_end, int threads,
                   int state_bits) {
-  if (dtype < 0 || dtype > 2) return ERR_ARG;
+  if (dtype < 0 || dtype > 3) return ERR_ARG;
   if (state_bits != 32 && state_bits != 64) return ERR_ARG;
   if (!layout_ok(N, K, tile_n, tile_k)) return ERR_SHAPE;
   if (state_bits == 64 && prob_bits != 12) return ERR_ARG;
@@ -632,9 +668,13 @@ int oracle_decode(int dtype, const uint8_t* stream, uint64_t stream_bytes,
           x[l] = (x[l] << (8 * word_bytes)) | word;
         }
         uint32_t row, col;
-        lane_map(tile_n, l, j, &row, &col);
+        if (dtype == DT_INT4_PAIRS) lane_map_pairs(tile_n, l, j, &row, &col);
+        else lane_map(tile_n, l, j, &row, &col);
         uint64_t idx = (n0 + row) * K + (k0 + col);
-        if (dtype == DT_INT4) {
+        if (dtype == DT_INT4_PAIRS) {
+          // idx is even: the pair is exactly one packed byte
+          ((uint8_t*)w_out)[idx / 2] = (uint8_t)(s ^ 0x88);
+        } else if (dtype == DT_INT4) {
           uint8_t* out = (uint8_t*)w_out;
           uint8_t nib = (uint8_t)((s - 8) & 0xF);
           if (idx % 2 == 0) out[idx / 2] = (uint8_t)((out[idx / 2] & 0xF0) | nib);
@@ -669,7 +709,7 @@ int oracle_decode(int dtype, const uint8_t* stream, uint64_t stream_bytes,
 int oracle_gemm(int dtype, const uint16_t* X, uint32_t M, uint32_t K, const void* W,
                 uint32_t N, int scale_kind, const void* scales, uint32_t group_k,
                 const uint32_t* rows, uint32_t n_rows, double* Y, int threads) {
-  if (dtype < 0 || dtype > 2) return ERR_ARG;
+  if (dtype < 0 || dtype > 3) return ERR_ARG;
   if (scale_kind == SC_GROUP_BF16 && (group_k == 0 || K % group_k != 0)) return ERR_ARG;
   if (scale_kind != SC_NONE && scales == nullptr) return ERR_ARG;
   if (rows == nullptr) n_rows = N;
@@ -681,7 +721,7 @@ int oracle_gemm(int dtype, const uint16_t* X, uint32_t M, uint32_t K, const void
     for (uint32_t k = 0; k < K; ++k) {
       uint64_t idx = n * K + k;
       double v;
-      if (dtype == DT_INT4) {
+      if (is_int4(dtype)) {
         v = (double)int4_code((const uint8_t*)W, idx);
         if (scale_kind == SC_ROW_BF16) v *= bf16_value(((const uint16_t*)scales)[n]);
         else if (scale_kind == SC_GROUP_BF16)

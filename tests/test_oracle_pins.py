@@ -430,6 +430,113 @@ def test_size_within_band_of_entropy(oracle, name, N, K, band):
     assert -0.01 < gap < band, (name, coded_bits, H)
 
 
+# ---- int4 pair symbols (one symbol per packed byte) ---------------------------------
+def test_pair_symbol_is_packed_byte_xor_0x88(oracle):
+    # every packed byte once: the pair histogram is one count at byte ^ 0x88
+    # (low nibble: code of the even element + 8; high nibble: odd element + 8)
+    w = np.arange(256, dtype=np.uint8)
+    counts = oracle.histogram(WL.INT4_PAIRS, w, 512)
+    assert counts.size == 256 and (counts == 1).all()
+    # hand example: byte 0x7F holds codes -1 (even) and 7 (odd): symbol 7 | 15 << 4
+    counts = oracle.histogram(WL.INT4_PAIRS, np.array([0x7F], np.uint8), 2)
+    assert int(np.argmax(counts)) == 0xF7 and counts.sum() == 1
+    # marginals of the pair histogram are the int4 histograms of even / odd elements
+    rng = np.random.default_rng(5)
+    codes = np.clip(np.rint(rng.laplace(0, 1.2, size=(64, 128))), -8, 7).astype(np.int8)
+    w = WL.pack_int4(codes)
+    pc = oracle.histogram(WL.INT4_PAIRS, w, codes.size).reshape(16, 16)   # [hi][lo]
+    even = np.bincount(codes[:, 0::2].reshape(-1) + 8, minlength=16)
+    odd = np.bincount(codes[:, 1::2].reshape(-1) + 8, minlength=16)
+    assert np.array_equal(pc.sum(axis=0), even) and np.array_equal(pc.sum(axis=1), odd)
+
+
+def _decode_equiprobable_256(stream, steps, wide):
+    """Symbols (lane, step) of one tile coded with f = 16 for all 256 symbols.
+    Then a decode step is plain bit surgery: the symbol is bits 4..11 of x and
+    x -> (x >> 12) << 4 | (x & 15); narrow states take a 16-bit word when
+    x < 2^16 after each step, wide ones a 32-bit word when x < 2^32 after each
+    odd step.  Words are shared by the 32 lanes in increasing lane order."""
+    sb, wb = (8, 4) if wide else (4, 2)
+    x = [int.from_bytes(stream[sb * l:sb * (l + 1)].tobytes(), "little") for l in range(32)]
+    pos = 32 * sb
+    out = np.zeros((32, steps), np.int64)
+    for j in range(steps):
+        for l in range(32):
+            out[l, j] = (x[l] >> 4) & 255
+            x[l] = ((x[l] >> 12) << 4) | (x[l] & 15)
+            if (not wide or j % 2 == 1) and x[l] < (1 << (8 * wb)):
+                x[l] = (x[l] << (8 * wb)) | int.from_bytes(stream[pos:pos + wb].tobytes(), "little")
+                pos += wb
+    return out
+
+
+@pytest.mark.parametrize("tile_n,tile_k", [(128, 64), (256, 32)])
+@pytest.mark.parametrize("state_bits", [32, 64])
+def test_pair_lane_map_properties(oracle, tile_n, tile_k, state_bits):
+    # Weights whose packed byte spells its own row (then its pair column) expose
+    # the (lane, step) -> (row, column pair) map of one tile; check that it is a
+    # bijection, that every 8 steps of a lane are 16 consecutive K elements of
+    # one row, and that every 32 steps complete a 128-row x 16-column slab,
+    # 128-row blocks first, then 16-column blocks.
+    freq = np.full(256, 16, np.uint32)
+    steps = tile_n * tile_k // 2 // 32
+    maps = []
+    for spell in ("row", "col"):
+        r = np.arange(tile_n)[:, None] * np.ones((1, tile_k // 2), np.int64)
+        c = np.ones((tile_n, 1), np.int64) * np.arange(tile_k // 2)[None, :]
+        byte = (r if spell == "row" else c) % 256
+        w = byte.astype(np.uint8).reshape(-1)   # packed bytes, row-major
+        st, stream, offsets, _ = oracle.encode(WL.INT4_PAIRS, w, tile_n, tile_k, tile_n, tile_k,
+                                               freq, state_bits=state_bits)
+        assert st == 0 and offsets.size == 2
+        sym = _decode_equiprobable_256(stream, steps, state_bits == 64)
+        maps.append(sym ^ 0x88)            # symbol = byte ^ 0x88
+    rows, cpairs = maps
+    seen = np.zeros((tile_n, tile_k // 2), np.int64)
+    np.add.at(seen, (rows.reshape(-1), cpairs.reshape(-1)), 1)
+    assert (seen == 1).all()
+    H = tile_n // 128
+    for j0 in range(0, steps, 8):
+        assert (rows[:, j0:j0 + 8] == rows[:, j0:j0 + 1]).all()
+        assert (cpairs[:, j0:j0 + 8] == cpairs[:, j0:j0 + 1] + np.arange(8)).all()
+    for q in range(steps // 32):
+        h, s = q % H, q // H
+        blk_r, blk_c = rows[:, 32 * q:32 * q + 32], cpairs[:, 32 * q:32 * q + 32]
+        assert set(blk_r.reshape(-1)) == set(range(128 * h, 128 * h + 128))
+        assert set(blk_c.reshape(-1)) == set(range(8 * s, 8 * s + 8))
+
+
+@pytest.mark.parametrize("name,N,K", [("tiny_int4", 512, 512), ("int4_70b", 512, 256)])
+@pytest.mark.parametrize("state_bits", [32, 64])
+def test_pair_encode_decode_identity_and_size(oracle, name, N, K, state_bits):
+    cfg, d = _small(name, N, K)
+    counts = oracle.histogram(WL.INT4_PAIRS, d["w"], N * K)
+    assert counts.sum() == N * K // 2
+    H2 = oracle.entropy(counts)                     # bits per pair
+    _, freq = oracle.normalize(counts)
+    st, stream, offsets, raw = oracle.encode(WL.INT4_PAIRS, d["w"], N, K, cfg.tile_n, cfg.tile_k,
+                                             freq, state_bits=state_bits)
+    assert st == 0 and raw is None
+    st, out = oracle.decode(WL.INT4_PAIRS, stream, offsets, None, N, K, cfg.tile_n, cfg.tile_k,
+                            freq, state_bits=state_bits)
+    assert st == 0 and np.array_equal(out, d["w"])
+    # half as many symbols as the per-element coding, each carrying two codes:
+    # the size stays within the per-element bands of the pair entropy (per
+    # weight); the wide states' extra slack per lane costs more on small tiles
+    gap = 8.0 * stream.size / (N * K) - H2 / 2
+    band = {32: 0.25, 64: 0.40}[state_bits] if name == "tiny_int4" else 0.12
+    assert -0.01 < gap < band, (name, gap)
+    # the same GEMM as the per-element reading of the same bytes
+    rng = np.random.default_rng(1)
+    X = WL.to_bf16_bits(rng.standard_normal((2, K)))
+    rows = np.arange(0, N, 37, dtype=np.uint32)
+    Yp = oracle.gemm(WL.INT4_PAIRS, X, 2, K, d["w"], N, cfg.scale_kind, d["scales"], cfg.group_k,
+                     rows=rows)
+    Y1 = oracle.gemm(WL.INT4, X, 2, K, d["w"], N, cfg.scale_kind, d["scales"], cfg.group_k,
+                     rows=rows)
+    assert np.array_equal(Yp, Y1)
+
+
 # ---- fp64 GEMM ------------------------------------------------------------------
 def test_gemm_int4_exact_integers(oracle):
     rng = np.random.default_rng(2)
