@@ -50,6 +50,13 @@
  *                  complement code q in [-8, 7]; coded symbol q + 8 (A = 16).
  *   ANS_BF16_SPLIT uint16 bf16 bits; coded symbol = exponent byte (A = 256).
  *   ANS_FP8_E4M3   e4m3fn code bytes; coded symbol = the code (A = 256).
+ *   ANS_INT4_PAIRS the same storage as ANS_INT4, coded one symbol per packed
+ *                  byte (two consecutive K elements): symbol = byte ^ 0x88,
+ *                  i.e. (q_k + 8) | (q_{k+1} + 8) << 4 (A = 256), half as
+ *                  many symbols per tile.  Lane l's j-th symbol covers row
+ *                  l + 32 (4 h + i), columns 16 s + 2 kk and 16 s + 2 kk + 1,
+ *                  with g = j / 8, kk = j % 8, i = g % 4,
+ *                  h = (g / 4) % (tile_n / 128), s = g / (4 tile_n / 128).
  *
  * Conventions.  Every buffer belongs to the caller; the library allocates no
  * device memory.  "d_" pointers are device pointers, "h_" host pointers.  GPU
@@ -91,7 +98,7 @@ typedef enum {
 #define ANS_STATUS_TIMEOUT 0x2u     /* a bounded wait inside a kernel ran out */
 #define ANS_STATUS_BAD_OFFSETS 0x4u /* an offset was unaligned, decreasing or past the end */
 
-typedef enum { ANS_INT4 = 0, ANS_BF16_SPLIT = 1, ANS_FP8_E4M3 = 2 } ans_dtype;
+typedef enum { ANS_INT4 = 0, ANS_BF16_SPLIT = 1, ANS_FP8_E4M3 = 2, ANS_INT4_PAIRS = 3 } ans_dtype;
 
 typedef enum {
   ANS_SCALE_NONE = 0,
@@ -104,7 +111,7 @@ typedef enum {
  * freq[s] > 0 exactly for the symbols present in the layer; the freq sum to
  * 2^prob_bits; cdf[s] = sum of freq[t] for t < s, cdf[alphabet] = 2^prob_bits. */
 typedef struct {
-  uint32_t alphabet;  /* 16 (int4) or 256 */
+  uint32_t alphabet;  /* 16 (ANS_INT4) or 256 */
   uint32_t prob_bits; /* 12 for the stream format; 1..15 accepted by ans_build_codebook */
   uint16_t freq[256];
   uint16_t cdf[257];

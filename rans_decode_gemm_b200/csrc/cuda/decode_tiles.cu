@@ -35,11 +35,18 @@ __device__ __forceinline__ void store_group(void* out, uint64_t idx, const uint3
     for (int k = 0; k < 8; ++k) w |= (((e[k] >> 12) ^ 8u) & 0xFu) << (4 * k);
     *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(out) + idx / 2) = w;
   } else {
+    // one byte per symbol: the e4m3 code, or the packed int4 pair (symbol ^ 0x88)
     uint32_t lo = __byte_perm(__byte_perm(e[0] >> 12, e[1] >> 4, 0x0050u),
                               __byte_perm(e[2] >> 12, e[3] >> 4, 0x0050u), 0x5410u);
     uint32_t hi = __byte_perm(__byte_perm(e[4] >> 12, e[5] >> 4, 0x0050u),
                               __byte_perm(e[6] >> 12, e[7] >> 4, 0x0050u), 0x5410u);
-    *reinterpret_cast<uint2*>(static_cast<uint8_t*>(out) + idx) = make_uint2(lo, hi);
+    if (DT == kDtInt4Pairs) {
+      lo ^= 0x88888888u;
+      hi ^= 0x88888888u;
+    }
+    // idx counts bytes for fp8 and K elements (two per byte) for int4 pairs
+    *reinterpret_cast<uint2*>(static_cast<uint8_t*>(out) + (DT == kDtInt4Pairs ? idx / 2 : idx)) =
+        make_uint2(lo, hi);
   }
 }
 
@@ -105,11 +112,13 @@ __global__ void __launch_bounds__(kDecMaxWarps * 32, 2)
       r2 = __ldg(raw_tile + 64);
     }
     uint32_t g = 0;
-    // group order (slab s, half h, chunk c, row i) matches the stream's lane map
+    // group order (slab s, half h, chunk c, row i) matches the stream's lane
+    // map; an int4 pair group covers both 8-column chunks of its row
+    constexpr uint32_t kGroups = DT == kDtInt4Pairs ? 4 : 8;
     for (uint32_t s = 0; s < C; ++s) {
       for (uint32_t h = 0; h < H; ++h) {
 #pragma unroll
-        for (uint32_t ci = 0; ci < 8; ++ci, ++g) {
+        for (uint32_t ci = 0; ci < kGroups; ++ci, ++g) {
           const uint32_t c = ci >> 2, i = ci & 3;
           const uint64_t raw8 = r0;
           if (DT == kDtBf16Split) {
@@ -157,6 +166,9 @@ __global__ void __launch_bounds__(kHistWarps * 32)
       if (dtype == kDtInt4) {
 #pragma unroll
         for (int n = 0; n < 8; ++n) atomicAdd(&mine[((u >> (4 * n)) & 0xFu) ^ 8u], 1u);
+      } else if (dtype == kDtInt4Pairs) {
+#pragma unroll
+        for (int n = 0; n < 4; ++n) atomicAdd(&mine[((u >> (8 * n)) & 0xFFu) ^ 0x88u], 1u);
       } else if (dtype == kDtBf16Split) {
         atomicAdd(&mine[(u >> 7) & 0xFFu], 1u);
         atomicAdd(&mine[(u >> 23) & 0xFFu], 1u);
@@ -173,6 +185,8 @@ __global__ void __launch_bounds__(kHistWarps * 32)
       if (dtype == kDtInt4) {
         atomicAdd(&mine[(w[b] & 0xFu) ^ 8u], 1u);
         atomicAdd(&mine[((w[b] >> 4) & 0xFu) ^ 8u], 1u);
+      } else if (dtype == kDtInt4Pairs) {
+        atomicAdd(&mine[w[b] ^ 0x88u], 1u);
       } else if (dtype == kDtBf16Split) {
         uint32_t u = w[b] | (static_cast<uint32_t>(w[b + 1]) << 8);
         atomicAdd(&mine[(u >> 7) & 0xFFu], 1u);
@@ -214,10 +228,12 @@ cudaError_t launch_decode_tiles(const LayerDev& L, void* out, uint32_t* status,
   if (L.wide) {
     if (L.dtype == kDtBf16Split) return launch_decode_variant<kDtBf16Split, true>(L, out, status, stream, blocks, warps);
     if (L.dtype == kDtInt4) return launch_decode_variant<kDtInt4, true>(L, out, status, stream, blocks, warps);
+    if (L.dtype == kDtInt4Pairs) return launch_decode_variant<kDtInt4Pairs, true>(L, out, status, stream, blocks, warps);
     return launch_decode_variant<kDtFp8, true>(L, out, status, stream, blocks, warps);
   }
   if (L.dtype == kDtBf16Split) return launch_decode_variant<kDtBf16Split, false>(L, out, status, stream, blocks, warps);
   if (L.dtype == kDtInt4) return launch_decode_variant<kDtInt4, false>(L, out, status, stream, blocks, warps);
+  if (L.dtype == kDtInt4Pairs) return launch_decode_variant<kDtInt4Pairs, false>(L, out, status, stream, blocks, warps);
   return launch_decode_variant<kDtFp8, false>(L, out, status, stream, blocks, warps);
 }
 

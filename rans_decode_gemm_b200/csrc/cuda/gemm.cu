@@ -194,7 +194,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         }
       }
       __half2 gscale[8];
-      if (kFmt == kFmtInt4F16Group) {
+      if (fmt_group(kFmt)) {
         const uint32_t gk = k0 / P.group_k;
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
@@ -224,7 +224,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         const uint32_t slot = sc & 1u;
         // group scales of this lane's four rows in half h (int4 x group scale)
         __half2 gs0, gs1, gs2, gs3;
-        if (kFmt == kFmtInt4F16Group) {
+        if (fmt_group(kFmt)) {
           gs0 = h ? gscale[4] : gscale[0];
           gs1 = h ? gscale[5] : gscale[1];
           gs2 = h ? gscale[6] : gscale[2];
@@ -251,11 +251,15 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         }
         if (sc >= 2) wait_live(&B.w_empty[2 * d + slot], ((sc >> 1) + 1) & 1u, abort, P.status, 1, 64);
         const uint32_t slab_s = wslots_s + slot * kSlabBytes;
+        // a group is 8 columns of one row, or both 8-column halves of it for
+        // int4 pair symbols (4 groups per slab)
+        constexpr bool kPair = fmt_pair(kFmt);
+        constexpr uint32_t kGroups = kPair ? 4 : 8, kOut = kPair ? 8 : 4;
 #pragma unroll 1
-        for (uint32_t gg = 0; gg < 8; ++gg) {
+        for (uint32_t gg = 0; gg < kGroups; ++gg) {
           const uint32_t g = us * 8 + gg;
           const uint32_t i = gg & 3, c = gg >> 2;
-          uint32_t o[4];
+          uint32_t o[kOut];
           if (kDecode) {
             const uint64_t raw8 = r0;
             if (kFmt == kFmtBf16Split && !zero_tile) {
@@ -274,13 +278,19 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
               tile_group(pipe, L, seq, tc, lane, abort, P.status);
               decode_group<kWide>(tc, lut_s, pipe.ring_s, lt, e);
             }
-            if (kFmt == kFmtBf16Split) fmt_bf16_split(e, raw8, o);
-            else if (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
-            else if (kFmt == kFmtInt4F16Group)
+            if constexpr (kFmt == kFmtInt4PairBf16) fmt_int4pair_bf16(e, o);
+            else if constexpr (kFmt == kFmtInt4PairF16Group)
+              fmt_int4pair_f16_scaled(e, i == 0 ? gs0 : i == 1 ? gs1 : i == 2 ? gs2 : gs3, o);
+            else if constexpr (kFmt == kFmtBf16Split) fmt_bf16_split(e, raw8, o);
+            else if constexpr (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
+            else if constexpr (kFmt == kFmtInt4F16Group)
               fmt_int4_f16_scaled(e, i == 0 ? gs0 : i == 1 ? gs1 : i == 2 ? gs2 : gs3, o);
             else fmt_fp8_f16(e, o);
-            if (zero_tile) o[0] = o[1] = o[2] = o[3] = 0;
-          } else {
+            if (zero_tile) {
+#pragma unroll
+              for (uint32_t k = 0; k < kOut; ++k) o[k] = 0;
+            }
+          } else if constexpr (!kPair) {
             uint4 v = cp[0];
 #pragma unroll
             for (int q = 1; q < 8; ++q)
@@ -304,10 +314,14 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
               }
             }
           }
-          const uint32_t addr = slab_s + (32 * i + lane) * 32 + ((c << 4) ^ swz);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(o[0]), "r"(o[1]),
-                       "r"(o[2]), "r"(o[3])
+          const uint32_t row_s = slab_s + (32 * i + lane) * 32;
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row_s + ((c << 4) ^ swz)),
+                       "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3])
                        : "memory");
+          if constexpr (kPair)
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row_s + (16u ^ swz)),
+                         "r"(o[kOut - 4]), "r"(o[kOut - 3]), "r"(o[kOut - 2]), "r"(o[kOut - 1])
+                         : "memory");
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -558,13 +572,17 @@ static uint32_t local_slots(uint32_t U, uint32_t G, uint32_t D, uint32_t n_kt) {
 // ans_gemm and ans_gemm_uncompressed add the same products in the same order.
 bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool decode, int num_sms,
                     GemmPlan* plan) {
-  (void)decode;
   GemmPlan p;
   std::memset(&p, 0, sizeof(p));
   if (L.dtype == 1) p.fmt = kFmtBf16Split;
   else if (L.dtype == 0) p.fmt = (scale_kind == 3) ? kFmtInt4F16Group : kFmtInt4Bf16;
+  else if (L.dtype == 3)
+    // int4 pair symbols fill the same slabs as per-element int4 symbols; the
+    // uncompressed weights take the per-element copy path
+    p.fmt = decode ? ((scale_kind == 3) ? kFmtInt4PairF16Group : kFmtInt4PairBf16)
+                   : ((scale_kind == 3) ? kFmtInt4F16Group : kFmtInt4Bf16);
   else p.fmt = kFmtFp8F16;
-  p.ab_f16 = (p.fmt == kFmtInt4F16Group || p.fmt == kFmtFp8F16) ? 1 : 0;
+  p.ab_f16 = (fmt_group(p.fmt) || p.fmt == kFmtFp8F16) ? 1 : 0;
   p.M = M;
   p.H = L.tile_n / 128;
   p.C = L.tile_k / 16;
@@ -803,6 +821,12 @@ cudaError_t launch_gemm(const GemmPlan& plan, const LayerDev& L, bool decode, co
     case kFmtInt4F16Group:
       return P.L.wide ? launch_variant<true, kFmtInt4F16Group, true>(plan, P, stream)
                       : launch_variant<true, kFmtInt4F16Group>(plan, P, stream);
+    case kFmtInt4PairBf16:
+      return P.L.wide ? launch_variant<true, kFmtInt4PairBf16, true>(plan, P, stream)
+                      : launch_variant<true, kFmtInt4PairBf16>(plan, P, stream);
+    case kFmtInt4PairF16Group:
+      return P.L.wide ? launch_variant<true, kFmtInt4PairF16Group, true>(plan, P, stream)
+                      : launch_variant<true, kFmtInt4PairF16Group>(plan, P, stream);
     case kFmtFp8F16:
       return P.L.wide ? launch_variant<true, kFmtFp8F16, true>(plan, P, stream)
                       : launch_variant<true, kFmtFp8F16>(plan, P, stream);

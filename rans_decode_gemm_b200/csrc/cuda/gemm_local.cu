@@ -69,10 +69,14 @@ __device__ __forceinline__ uint32_t producer_first_slot(uint32_t ub, uint32_t ue
   return slot;
 }
 
-__device__ __forceinline__ void sts128(uint32_t addr, const uint32_t (&o)[4]) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(o[0]), "r"(o[1]),
-               "r"(o[2]), "r"(o[3])
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                       uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
                : "memory");
+}
+__device__ __forceinline__ void sts128(uint32_t addr, const uint32_t (&o)[4]) {
+  sts128(addr, o[0], o[1], o[2], o[3]);
 }
 
 template <bool kDecode, uint32_t kFmt, bool kWide>
@@ -200,7 +204,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
           if (zero_tile && lane == 0) atomicOr(P.status, kStatusBadOffsets);
         }
         __half2 gscale[8];
-        if (kFmt == kFmtInt4F16Group) {
+        if (fmt_group(kFmt)) {
           const uint32_t gk = k0 / P.group_k;
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
@@ -235,7 +239,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
             const uint32_t slot = nw & 1u;
             const uint32_t w_s = w_s0 + slot * kSlabBytes, x_s = x_s0 + slot * T * 32;
             __half2 gsc[4];
-            if (kFmt == kFmtInt4F16Group) {
+            if (fmt_group(kFmt)) {
               gsc[0] = h ? gscale[4] : gscale[0];
               gsc[1] = h ? gscale[5] : gscale[1];
               gsc[2] = h ? gscale[6] : gscale[2];
@@ -272,21 +276,32 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
               }
             }
             // the store of group gg - 1 (deferred); the first store into the
-            // slot waits for the MMA that last read it (slab nw - 2)
-            uint32_t o_prev[4] = {0, 0, 0, 0};
+            // slot waits for the MMA that last read it (slab nw - 2).  A group
+            // is 8 columns of one row, or both 8-column halves of it for int4
+            // pair symbols (4 groups per slab).
+            constexpr bool kPair = fmt_pair(kFmt);
+            constexpr uint32_t kGroups = kPair ? 4 : 8, kOut = kPair ? 8 : 4;
+            uint32_t o_prev[kOut];
+#pragma unroll
+            for (uint32_t k = 0; k < kOut; ++k) o_prev[k] = 0;
             auto store_prev = [&](uint32_t gg) {
               if (gg == 1 && nw >= 2)
                 wait_live(&w_empty[2 * d + slot], ((nw >> 1) + 1) & 1u, abort, P.status, 1);
-              const uint32_t i = (gg - 1) & 3, c = (gg - 1) >> 2;
-              sts128(w_s + (32 * i + lane) * 32 + ((c << 4) ^ swz), o_prev);
+              const uint32_t row_s = w_s + (32 * ((gg - 1) & 3) + lane) * 32;
+              if constexpr (kPair) {
+                sts128(row_s + swz, o_prev[0], o_prev[1], o_prev[2], o_prev[3]);
+                sts128(row_s + (16u ^ swz), o_prev[4], o_prev[5], o_prev[6], o_prev[7]);
+              } else {
+                sts128(row_s + ((((gg - 1) >> 2) << 4) ^ swz), o_prev[0], o_prev[1], o_prev[2], o_prev[3]);
+              }
             };
 #pragma unroll
-            for (uint32_t gg = 0; gg < 8; ++gg) {
+            for (uint32_t gg = 0; gg < kGroups; ++gg) {
               const uint32_t g = us * 8 + gg;
-              const uint32_t i = gg & 3;
-              uint32_t o[4];
+              [[maybe_unused]] const uint32_t i = gg & 3;  // row quarter (group scales)
+              uint32_t o[kOut];
               if (kDecode) {
-                const uint64_t raw8 = rq[0];
+                [[maybe_unused]] const uint64_t raw8 = rq[0];
                 if (kFmt == kFmtBf16Split && (!kConst || !zero_tile)) {
 #pragma unroll
                   for (uint32_t k = 0; k + 1 < kRawAhead; ++k) rq[k] = rq[k + 1];
@@ -312,12 +327,17 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
                     for (int k = 1; k < 8; ++k) e[k] = decode_step(tc.x, tc.pos, lut_s, pipe.ring_s, lt);
                   }
                 }
-                if (kFmt == kFmtBf16Split) fmt_bf16_split(e, raw8, o);
-                else if (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
-                else if (kFmt == kFmtInt4F16Group) fmt_int4_f16_scaled(e, gsc[i], o);
+                if constexpr (kFmt == kFmtInt4PairBf16) fmt_int4pair_bf16(e, o);
+                else if constexpr (kFmt == kFmtInt4PairF16Group) fmt_int4pair_f16_scaled(e, gsc[i], o);
+                else if constexpr (kFmt == kFmtBf16Split) fmt_bf16_split(e, raw8, o);
+                else if constexpr (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
+                else if constexpr (kFmt == kFmtInt4F16Group) fmt_int4_f16_scaled(e, gsc[i], o);
                 else fmt_fp8_f16(e, o);
-                if (kConst && zero_tile) o[0] = o[1] = o[2] = o[3] = 0;
-              } else {
+                if (kConst && zero_tile) {
+#pragma unroll
+                  for (uint32_t k = 0; k < kOut; ++k) o[k] = 0;
+                }
+              } else if constexpr (!kPair) {
                 const uint4 v = cp[gg];
                 if (kFmt == kFmtBf16Split) {
                   o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
@@ -340,9 +360,9 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
                 if (gg > 0) store_prev(gg);
               }
 #pragma unroll
-              for (int k = 0; k < 4; ++k) o_prev[k] = o[k];
+              for (uint32_t k = 0; k < kOut; ++k) o_prev[k] = o[k];
             }
-            store_prev(8);
+            store_prev(kGroups);
             // X slab, then hand the slab to the issuing warp
 #pragma unroll
             for (uint32_t j = 0; j < 2; ++j) {
@@ -612,6 +632,12 @@ cudaError_t launch_gemm_local(const GemmPlan& plan, const GemmDev& P, bool decod
     case kFmtInt4F16Group:
       return P.L.wide ? launch_local_variant<true, kFmtInt4F16Group, true>(plan, P, stream)
                       : launch_local_variant<true, kFmtInt4F16Group>(plan, P, stream);
+    case kFmtInt4PairBf16:
+      return P.L.wide ? launch_local_variant<true, kFmtInt4PairBf16, true>(plan, P, stream)
+                      : launch_local_variant<true, kFmtInt4PairBf16>(plan, P, stream);
+    case kFmtInt4PairF16Group:
+      return P.L.wide ? launch_local_variant<true, kFmtInt4PairF16Group, true>(plan, P, stream)
+                      : launch_local_variant<true, kFmtInt4PairF16Group>(plan, P, stream);
     case kFmtFp8F16:
       return P.L.wide ? launch_local_variant<true, kFmtFp8F16, true>(plan, P, stream)
                       : launch_local_variant<true, kFmtFp8F16>(plan, P, stream);

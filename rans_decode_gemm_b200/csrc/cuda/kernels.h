@@ -30,8 +30,14 @@ enum : uint32_t {
   kFmtBf16Split = 0,   // bf16 weights: exponent symbol + raw sign/mantissa byte -> bf16
   kFmtInt4Bf16 = 1,    // int4 code -> exact bf16 (row scale applied in the epilogue)
   kFmtInt4F16Group = 2,// int4 code * group scale -> exact f16
-  kFmtFp8F16 = 3       // e4m3 code -> exact f16 (row scale applied in the epilogue)
+  kFmtFp8F16 = 3,      // e4m3 code -> exact f16 (row scale applied in the epilogue)
+  kFmtInt4PairBf16 = 4,     // int4 pair symbol -> two exact bf16 (row scale in the epilogue)
+  kFmtInt4PairF16Group = 5  // int4 pair symbol * group scale -> two exact f16
 };
+// int4 pair symbols: 8 symbols of a lane fill 16 columns of one slab row
+__host__ __device__ constexpr bool fmt_pair(uint32_t f) { return f == kFmtInt4PairBf16 || f == kFmtInt4PairF16Group; }
+// a per-(row, K group) scale is applied while the slab is written
+__host__ __device__ constexpr bool fmt_group(uint32_t f) { return f == kFmtInt4F16Group || f == kFmtInt4PairF16Group; }
 
 // Static schedule of one fused GEMM launch, computed on the host.
 struct GemmPlan {

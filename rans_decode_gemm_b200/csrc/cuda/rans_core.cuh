@@ -49,7 +49,7 @@ constexpr uint32_t kStatusCorrupt = 0x1u;
 constexpr uint32_t kStatusTimeout = 0x2u;
 constexpr uint32_t kStatusBadOffsets = 0x4u;
 
-enum : uint32_t { kDtInt4 = 0, kDtBf16Split = 1, kDtFp8 = 2 };
+enum : uint32_t { kDtInt4 = 0, kDtBf16Split = 1, kDtFp8 = 2, kDtInt4Pairs = 3 };
 
 
 // Abort-aware bounded wait.  Returns false if the wait ran out (then sets the
@@ -623,6 +623,32 @@ __device__ __forceinline__ void fmt_int4_bf16(const uint32_t (&e)[8], uint32_t (
     const __nv_bfloat162 bias = __floats2bfloat162_rn(136.0f, 136.0f);
     h = __hsub2(h, bias);
     out[p] = *reinterpret_cast<uint32_t*>(&h);
+  }
+}
+
+// int4 pair symbols (symbol = (q_even + 8) | (q_odd + 8) << 4, in bits 12..19 of
+// the entry) as two exact bf16: the even code's nibble goes to the low half,
+// the odd one's (already at bits 16..19) to the high half.  8 symbols -> 16
+// consecutive K elements.
+__device__ __forceinline__ void fmt_int4pair_bf16(const uint32_t (&e)[8], uint32_t (&out)[8]) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    uint32_t v = ((e[k] >> 12) & 0x0000000Fu) | (e[k] & 0x000F0000u) | 0x43004300u;
+    __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&v);
+    h = __hsub2(h, __floats2bfloat162_rn(136.0f, 136.0f));
+    out[k] = *reinterpret_cast<uint32_t*>(&h);
+  }
+}
+
+// int4 pair symbols times a per-row group scale, exact in f16.
+__device__ __forceinline__ void fmt_int4pair_f16_scaled(const uint32_t (&e)[8], __half2 scale,
+                                                        uint32_t (&out)[8]) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    uint32_t v = ((e[k] >> 12) & 0x0000000Fu) | (e[k] & 0x000F0000u) | 0x64006400u;
+    __half2 h = *reinterpret_cast<__half2*>(&v);
+    h = __hmul2(__hsub2(h, __floats2half2_rn(1032.0f, 1032.0f)), scale);
+    out[k] = *reinterpret_cast<uint32_t*>(&h);
   }
 }
 

@@ -41,6 +41,25 @@ std::vector<uint64_t> lane_order(uint32_t tile_n, uint32_t tile_k, uint64_t K) {
   return off;
 }
 
+// int4 pairs: element offset of the even element of every (step j, lane l)
+// pair symbol, stored at j * 32 + l.  Eight steps of a lane cover 16
+// consecutive columns of one row.
+std::vector<uint64_t> lane_order_pairs(uint32_t tile_n, uint32_t tile_k, uint64_t K) {
+  const uint32_t halves = tile_n / 128;
+  const uint32_t steps = tile_n * tile_k / 2 / kLanes;
+  std::vector<uint64_t> off(static_cast<size_t>(steps) * kLanes);
+  for (uint32_t j = 0; j < steps; ++j) {
+    const uint32_t g = j >> 3, kk = j & 7;
+    const uint32_t i = g & 3, h = (g >> 2) % halves, s = g / (4 * halves);
+    for (uint32_t l = 0; l < kLanes; ++l) {
+      const uint64_t row = l + 32 * (4 * h + i);
+      const uint64_t col = 16 * s + 2 * kk;
+      off[static_cast<size_t>(j) * kLanes + l] = row * K + col;
+    }
+  }
+  return off;
+}
+
 struct TileJob {
   bool wide;  // wide-state variant: 64-bit states, 32-bit words, one test per symbol pair
   uint32_t dtype;
@@ -61,10 +80,12 @@ bool code_tile(const TileJob& job, uint64_t t, std::vector<uint8_t>& out,
                std::vector<uint8_t>& sym, std::vector<uint16_t>& words,
                std::vector<uint32_t>& words32, uint8_t* raw_tile) {
   const uint64_t origin = (t / job.n_kt) * job.tile_n * job.K + (t % job.n_kt) * job.tile_k;
-  const size_t S = static_cast<size_t>(job.tile_n) * job.tile_k;
+  const size_t S = static_cast<size_t>(job.tile_n) * job.tile_k / (job.dtype == kInt4Pairs ? 2 : 1);
   const std::vector<uint64_t>& order = *job.order;
   sym.resize(S);
-  if (job.dtype == kInt4) {
+  if (job.dtype == kInt4Pairs) {
+    for (size_t q = 0; q < S; ++q) sym[q] = static_cast<uint8_t>(job.w[(origin + order[q]) >> 1] ^ 0x88);
+  } else if (job.dtype == kInt4) {
     for (size_t q = 0; q < S; ++q) {
       const uint64_t e = origin + order[q];
       const uint8_t b = job.w[e >> 1];
@@ -170,7 +191,7 @@ bool layout_valid(uint32_t N, uint32_t K, uint32_t tile_n, uint32_t tile_k) {
 
 void histogram(uint32_t dtype, const void* w, uint64_t n_weights, uint64_t* hist) {
   const uint32_t A = dtype == kInt4 ? 16 : 256;
-  const uint64_t units = dtype == kInt4 ? n_weights / 2 : n_weights;  // bytes or u16 words
+  const uint64_t units = (dtype == kInt4 || dtype == kInt4Pairs) ? n_weights / 2 : n_weights;  // bytes or u16 words
   const unsigned nw = worker_count(units / 65536 + 1);
   std::vector<std::vector<uint64_t>> part(nw, std::vector<uint64_t>(256, 0));
   std::vector<std::thread> pool;
@@ -181,6 +202,9 @@ void histogram(uint32_t dtype, const void* w, uint64_t n_weights, uint64_t* hist
       if (dtype == kInt4) {
         const uint8_t* p = static_cast<const uint8_t*>(w);
         for (uint64_t i = a; i < b; ++i) { h[(p[i] & 15) ^ 8]++; h[(p[i] >> 4) ^ 8]++; }
+      } else if (dtype == kInt4Pairs) {
+        const uint8_t* p = static_cast<const uint8_t*>(w);
+        for (uint64_t i = a; i < b; ++i) h[p[i] ^ 0x88]++;
       } else if (dtype == kBf16Split) {
         const uint16_t* p = static_cast<const uint16_t*>(w);
         for (uint64_t i = a; i < b; ++i) h[(p[i] >> 7) & 0xFF]++;
@@ -284,7 +308,8 @@ int encode(uint32_t dtype, const void* w, uint32_t N, uint32_t K, uint32_t tile_
            uint64_t* stream_bytes, uint64_t* offsets, uint8_t* raw, bool wide) {
   const uint32_t n_kt = K / tile_k;
   const uint64_t tiles = static_cast<uint64_t>(N / tile_n) * n_kt;
-  const std::vector<uint64_t> order = lane_order(tile_n, tile_k, K);
+  const std::vector<uint64_t> order =
+      dtype == kInt4Pairs ? lane_order_pairs(tile_n, tile_k, K) : lane_order(tile_n, tile_k, K);
   TileJob job;
   job.wide = wide;
   job.dtype = dtype;
@@ -302,7 +327,7 @@ int encode(uint32_t dtype, const void* w, uint32_t N, uint32_t K, uint32_t tile_
     run += job.freq[s];
   }
   job.cdf[256] = run;
-  const size_t S = static_cast<size_t>(tile_n) * tile_k;
+  const size_t S = static_cast<size_t>(tile_n) * tile_k;  // raw bytes per tile (bf16)
 
   const unsigned nw = worker_count(tiles);
   std::vector<std::vector<uint8_t>> bufs(nw);

@@ -7,10 +7,13 @@ from rans_decode_gemm_b200 import ans
 from rans_decode_gemm_b200 import workloads as WL
 
 
-def make_case(name, N=None, K=None, matrix=0, state_bits=32):
+def make_case(name, N=None, K=None, matrix=0, state_bits=32, dtype=None):
+    """dtype: the coded symbol kind when it differs from the workload's storage
+    dtype (int4 weights coded as pair symbols)."""
     cfg = WL.CONFIGS[name]
     d = WL.make_weights(cfg, matrix, N=N, K=K)
-    lay = ans.make_layout(cfg.dtype, d["N"], d["K"], cfg.tile_n, cfg.tile_k, state_bits)
+    lay = ans.make_layout(cfg.dtype if dtype is None else dtype, d["N"], d["K"], cfg.tile_n,
+                          cfg.tile_k, state_bits)
     layer = ans.CompressedLayer.from_weights(d["w"], lay, device="cuda")
     return cfg, d, lay, layer
 

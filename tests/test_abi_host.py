@@ -38,6 +38,8 @@ def test_status_strings_and_layout_checks(ans_lib):
     assert ans.ans_layout_check(ans.make_layout(0, 512, 520, 128, 40)) == 2    # tile_k % 16
     assert ans.ans_layout_check(ans.make_layout(0, 512, 512, 64, 32)) == 2     # tile_n
     assert ans.ans_layout_check(ans.make_layout(7, 512, 512, 128, 32)) == 1    # dtype
+    assert ans.ans_layout_check(ans.make_layout(4, 512, 512, 128, 32)) == 1    # dtype
+    assert ans.ans_layout_check(ans.make_layout(3, 512, 512, 128, 32)) == 0    # int4 pairs
     assert ans.ans_layout_check(ans.make_layout(1, 0, 512, 128, 32)) == 2      # empty
     assert ans.ans_num_tiles(ans.make_layout(2, 53248, 16384, 128, 128)) == 53248
     assert ans.ans_layout_check(ans.make_layout(0, 512, 512, 128, 32, 64)) == 0
@@ -49,11 +51,16 @@ CASES = [("tiny_int4", 512, 512), ("bf16_4096", 512, 512), ("llama8b_mlp", 256, 
          ("int4_70b", 512, 512), ("fp8_405b", 256, 1024)]
 
 
+@pytest.mark.parametrize("pairs", [False, True])
 @pytest.mark.parametrize("state_bits", [32, 64])
 @pytest.mark.parametrize("name,N,K", CASES)
-def test_host_codec_matches_oracle(oracle, ans_lib, name, N, K, state_bits):
+def test_host_codec_matches_oracle(oracle, ans_lib, name, N, K, state_bits, pairs):
     cfg = WL.CONFIGS[name]
-    d = WL.make_weights(cfg, 0, N=N, K=K)
+    if pairs:
+        if cfg.dtype != WL.INT4:
+            pytest.skip("pair symbols are an int4 coding")
+        cfg = WL.Config(**{**cfg.__dict__, "dtype": WL.INT4_PAIRS})
+    d = WL.make_weights(WL.CONFIGS[name], 0, N=N, K=K)
     lay = ans.make_layout(cfg.dtype, N, K, cfg.tile_n, cfg.tile_k, state_bits)
     hist = ans.ans_histogram_host(d["w"], lay)
     assert np.array_equal(hist, oracle.histogram(cfg.dtype, d["w"], N * K))
