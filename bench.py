@@ -66,6 +66,9 @@ def parse():
     ap.add_argument("--state-bits", type=int, default=64, choices=[32, 64],
                     help="stream format: 64 = wide lane states (32-bit words, one "
                          "renormalisation test per symbol pair), 32 = 32-bit states")
+    ap.add_argument("--int4-symbols", default="pairs", choices=["pairs", "element"],
+                    help="--sweep: code int4 weights one symbol per packed byte (two K "
+                         "elements) or one per element")
     ap.add_argument("--quick", action="store_true",
                     help="skip the context sweep and the CPU baseline (profiling runs)")
     return ap.parse_args()
@@ -468,9 +471,11 @@ def sweep(args):
         for mi, (mname, mN, mK) in enumerate(cfg.matrices):
             d = WL.make_weights(cfg, mi)
             N, K = d["N"], d["K"]
-            lay = ans.make_layout(cfg.dtype, N, K, cfg.tile_n, cfg.tile_k, args.state_bits)
+            pairs = cfg.dtype == WL.INT4 and args.int4_symbols == "pairs"
+            coded = WL.INT4_PAIRS if pairs else cfg.dtype
+            lay = ans.make_layout(coded, N, K, cfg.tile_n, cfg.tile_k, args.state_bits)
             dw = torch.from_numpy(d["w"].view(np.int16) if d["w"].dtype == np.uint16 else d["w"]).to(device)
-            A = 256 if cfg.dtype != 0 else 16
+            A = ans.ALPHABET[coded]
             hist = torch.zeros(A, dtype=torch.int64, device=device)
             ans.ans_histogram(dw, lay, hist)
             hist_h = hist.cpu().numpy().astype(np.uint64)
@@ -482,7 +487,8 @@ def sweep(args):
             copies = int(max(1, min(12, -(-256e6 // comp))))
             layers = [ans.CompressedLayer(lay, cb, stream_h, offsets_h, raw_h, device) for _ in range(copies)]
             H = ans.ans_entropy(hist_h)
-            bound = H + 8.0 if cfg.dtype == 1 else H
+            # per weight: + the raw byte (bf16); a pair symbol carries two weights
+            bound = H + 8.0 if cfg.dtype == 1 else (H / 2 if pairs else H)
             bpw = 8.0 * layers[0].compressed_bytes / (N * K)
             sc = None
             if d["scales"] is not None:
@@ -519,6 +525,7 @@ def sweep(args):
                 algo = layers[0].compressed_bytes + 2 * M * K + 4 * M * N
                 rec = {"workload": name, "matrix": mname, "N": N, "K": K, "M": M,
                        "state_bits": args.state_bits,
+                       **({"int4_symbols": args.int4_symbols} if cfg.dtype == WL.INT4 else {}),
                        "tile": f"{lay.tile_n}x{lay.tile_k}", "bits_per_weight": round(bpw, 4),
                        "entropy_bound_bits": round(bound, 4), "gap_bits": round(bpw - bound, 4),
                        "encode_s": round(encode_s, 2), "copies": copies,

@@ -71,7 +71,13 @@ __global__ void __launch_bounds__(kDecMaxWarps * 32, 2)
     for (uint32_t i = 0; i < nwarps * 4; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
   }
-  if (!single) build_lut(lut, L, warp, nwarps, lane);
+  // slot table; the cdf is staged in its own array: staged in the ring area,
+  // which bulk copies fill next, the decode read wrong words even with a
+  // proxy fence and a CTA barrier between the two
+  __shared__ uint32_t cdf_s[257];
+  if (!single) lut_stage_cdf(cdf_s, L, threadIdx.x, blockDim.x);
+  __syncthreads();
+  if (!single) lut_fill(lut, cdf_s, L.alphabet, threadIdx.x, blockDim.x);
   __syncthreads();
   // the prologue above read only kernel parameters: from here on global
   // memory, after the previous grid in the stream has completed

@@ -137,22 +137,26 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
   Bars B = carve_bars(smem + P.off_bars, D, XS);
   const uint32_t x_stage_bytes = P.T_pass * 32;
 
+  // barriers initialised by all threads, TMEM allocated by warp 0 while the
+  // other warps build the slot table (see the local schedule's prologue)
   if (threadIdx.x == 0) {
     abort_flag = 0;
     red_n = 0;
     reduce_flag = 0;
-    for (uint32_t i = 0; i < 2 * D; ++i) { mbar_init(&B.w_full[i], 1); mbar_init(&B.w_empty[i], 1); }
-    for (uint32_t i = 0; i < XS; ++i) { mbar_init(&B.x_full[i], 1); mbar_init(&B.x_empty[i], 1); }
-    for (uint32_t i = 0; i < 2; ++i) { mbar_init(&B.acc_full[i], 1); mbar_init(&B.acc_empty[i], 4); }
-    mbar_init(B.mma_done, 1);
-    for (uint32_t i = 0; i < 4 * D; ++i) mbar_init(&B.chunk[i], 1);
-    fence_mbar_init();
+  }
+  {
+    uint64_t* b0 = B.w_full;  // the barriers are one array, in carve_bars order
+    const uint32_t n_bars = num_bars(D, XS);
+    for (uint32_t i = threadIdx.x; i < n_bars; i += blockDim.x)
+      mbar_init(&b0[i], (b0 + i >= B.acc_empty && b0 + i < B.acc_empty + 2) ? 4u : 1u);
+    if (threadIdx.x < n_bars) fence_mbar_init();
   }
   if (warp == 0) {
     tmem_alloc(&tmem_slot, P.tmem_cols);
     tmem_relinquish();
+  } else if (kDecode && P.L.single_symbol == kNoSymbol) {
+    build_lut(lut, P.L, warp - 1, blockDim.x / 32 - 1, lane);
   }
-  if (kDecode && P.L.single_symbol == kNoSymbol) build_lut(lut, P.L, warp, blockDim.x / 32, lane);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

@@ -108,18 +108,24 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
   uint64_t* mma_done = bars + 8 * D;      // every MMA of the CTA retired
   uint64_t* acc_full = bars + 8 * D + 1;  // one per accumulator slot
 
+  // Prologue, on the critical path of every CTA that starts after a CTA of
+  // the previous launch left its SM: the barriers are initialised by all
+  // threads (one thread initialising them in turn took ~3,300 cycles), warp 0
+  // allocates TMEM while the other warps build the slot table.
   if (threadIdx.x == 0) {
     abort_flag = 0;
     red_n = 0;
     reduce_flag = 0;
-    for (uint32_t i = 0; i < 8 * D + 1 + P.n_slots; ++i) mbar_init(&bars[i], i == 8 * D ? 32u : 1u);
-    fence_mbar_init();
   }
+  const uint32_t n_bars = 8 * D + 1 + P.n_slots;
+  for (uint32_t i = threadIdx.x; i < n_bars; i += blockDim.x) mbar_init(&bars[i], i == 8 * D ? 32u : 1u);
+  if (threadIdx.x < n_bars) fence_mbar_init();
   if (warp == 0) {
     tmem_alloc(&tmem_slot, P.tmem_cols);
     tmem_relinquish();
+  } else if (kDecode && P.L.single_symbol == kNoSymbol) {
+    build_lut(lut, P.L, warp - 1, blockDim.x / 32 - 1, lane);
   }
-  if (kDecode && P.L.single_symbol == kNoSymbol) build_lut(lut, P.L, warp, blockDim.x / 32, lane);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

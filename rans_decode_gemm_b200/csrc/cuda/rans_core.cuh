@@ -131,12 +131,49 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
 
 // Slot table: entry = (f & 0xFFF) << 20 | symbol << 12 | (slot - cdf[symbol]).
 // A single-symbol codebook (f = 4096) is decoded by a separate path.
+// Per-symbol build: warp w of nwarps fills the slots of symbols w, w + nwarps,
+// ... (no barrier needed; used where a warp of the CTA has other prologue work).
 __device__ __forceinline__ void build_lut(uint32_t* lut, const LayerDev& L, uint32_t warp,
                                           uint32_t nwarps, uint32_t lane) {
   for (uint32_t s = warp; s < L.alphabet; s += nwarps) {
     uint32_t f = L.freq[s], c = L.cdf[s];
     uint32_t hi = ((f & 0xFFFu) << 20) | (s << 12);
     for (uint32_t k = lane; k < f; k += 32) lut[c + k] = hi | k;
+  }
+}
+
+// Search build, in two phases around a CTA barrier, from the kernel parameters only:
+// lut_stage_cdf copies cdf[0 .. alphabet] into shared scratch; lut_fill gives
+// thread tid the slots tid, tid + nthr, ... and finds the symbol of each by a
+// binary search of the cdf for the largest s with cdf[s] <= slot (a symbol of
+// zero frequency is never the largest), four searches in flight per thread.
+// Every thread does the same few steps, whatever the frequencies: no loop
+// over the alphabet, no warp left with the most frequent symbols.
+__device__ __forceinline__ void lut_stage_cdf(uint32_t* cdf_s, const LayerDev& L, uint32_t tid,
+                                              uint32_t nthr) {
+  for (uint32_t s = tid; s <= L.alphabet; s += nthr) cdf_s[s] = L.cdf[s];
+}
+
+__device__ __forceinline__ void lut_fill(uint32_t* lut, const uint32_t* cdf_s, uint32_t alphabet,
+                                         uint32_t tid, uint32_t nthr) {
+  for (uint32_t base = tid; base < kSlots; base += 4 * nthr) {
+    uint32_t lo[4] = {0, 0, 0, 0};
+    // the answer stays in [lo, lo + n); n shrinks to ceil(n / 2) each step
+    for (uint32_t n = alphabet; n > 1;) {
+      const uint32_t half = n >> 1;
+#pragma unroll
+      for (uint32_t q = 0; q < 4; ++q)
+        if (cdf_s[lo[q] + half] <= base + q * nthr) lo[q] += half;
+      n -= half;
+    }
+#pragma unroll
+    for (uint32_t q = 0; q < 4; ++q) {
+      const uint32_t slot = base + q * nthr;
+      if (slot < kSlots) {
+        const uint32_t c = cdf_s[lo[q]], f = cdf_s[lo[q] + 1] - c;
+        lut[slot] = ((f & 0xFFFu) << 20) | (lo[q] << 12) | (slot - c);
+      }
+    }
   }
 }
 
