@@ -251,6 +251,43 @@ ans_status ans_gemm_uncompressed(const uint16_t* d_X, uint32_t M, const void* d_
                                  const void* d_scales, uint32_t group_k, float* d_Y, void* d_ws,
                                  size_t ws_bytes, uint32_t* d_status, ans_stream_t stream);
 
+/* One layer of a batched call: its X (bf16 M x K, 16-byte aligned), its
+ * compressed weights, its scales (as for ans_gemm) and its Y (fp32 M x N,
+ * 16-byte aligned).  The structs and the ans_tiles they point to are read
+ * during the call only. */
+typedef struct {
+  const uint16_t* d_X;
+  const ans_tiles* W;
+  const void* d_scales;
+  float* d_Y;
+} ans_gemm_job;
+
+#define ANS_MAX_BATCH 8
+
+/* Bytes of device workspace for ans_gemm_batched over n_jobs layers of the
+ * layout of jobs[0] (same conditions as ans_gemm_workspace). */
+ans_status ans_gemm_batched_workspace(const ans_gemm_job* jobs, uint32_t n_jobs, uint32_t M,
+                                      ans_scale_kind scale_kind, size_t* bytes);
+
+/* Several independent layers in one launch (the gate and up projections of
+ * an MLP, say; "Approaching Shannon Bound", s3.1 applied to a list of
+ * layers): Y_j = X_j * dequant(W_j)^T for j < n_jobs, with M, scale_kind and
+ * group_k shared.  1 <= n_jobs <= ANS_MAX_BATCH; every W_j must have the same
+ * layout (dtype, N, K, tile shape, state width; ANS_ERR_SHAPE otherwise) and
+ * its own codebook.  When the shape takes the small-M schedule on an equal
+ * share of the SMs (M up to 32 for 128-row tiles, 16 for 256-row tiles) the
+ * layers share one kernel launch, each on its share, so one kernel tail
+ * serves them all; otherwise they run as consecutive ans_gemm launches.  Each
+ * Y_j is deterministic and within the error bound of ans_gemm; in one launch
+ * it is bit-identical to ans_gemm on the same layer confined to the same
+ * number of SMs (the split-K partition depends on the SM count, so it may
+ * differ from ans_gemm's in the last bits).  d_ws: ans_gemm_batched_workspace
+ * bytes, zero-filled once before first use (the kernels leave it that way);
+ * d_status as for ans_gemm. */
+ans_status ans_gemm_batched(const ans_gemm_job* jobs, uint32_t n_jobs, uint32_t M,
+                            ans_scale_kind scale_kind, uint32_t group_k, void* d_ws,
+                            size_t ws_bytes, uint32_t* d_status, ans_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -26,7 +26,9 @@ ALPHABET = {INT4: 16, BF16_SPLIT: 256, FP8_E4M3: 256, INT4_PAIRS: 256}
 EXPORTS = ["ans_status_string", "ans_last_error", "ans_num_tiles", "ans_layout_check",
            "ans_histogram", "ans_histogram_host", "ans_entropy", "ans_build_codebook", "ans_encode_bound",
            "ans_encode_tiles", "ans_decode_tiles", "ans_gemm_workspace", "ans_gemm",
-           "ans_gemm_noalloc", "ans_gemm_uncompressed"]
+           "ans_gemm_noalloc", "ans_gemm_uncompressed", "ans_gemm_batched_workspace",
+           "ans_gemm_batched"]
+MAX_BATCH = 8
 
 
 class AnsError(RuntimeError):
@@ -52,6 +54,11 @@ class AnsLayout(C.Structure):
 class AnsTiles(C.Structure):
     _fields_ = [("layout", AnsLayout), ("codebook", AnsCodebook), ("stream", C.c_void_p),
                 ("stream_bytes", C.c_uint64), ("offsets", C.c_void_p), ("raw", C.c_void_p)]
+
+
+class AnsGemmJob(C.Structure):
+    _fields_ = [("d_X", C.c_void_p), ("W", C.c_void_p), ("d_scales", C.c_void_p),
+                ("d_Y", C.c_void_p)]
 
 
 _lib = None
@@ -84,6 +91,8 @@ def load():
             L.ans_gemm.argtypes = [P, u32, P, i32, P, u32, P, P, sz, P, P]
             L.ans_gemm_noalloc.argtypes = [P, u32, P, i32, P, u32, P, P, P]
             L.ans_gemm_uncompressed.argtypes = [P, u32, P, P, i32, P, u32, P, P, sz, P, P]
+            L.ans_gemm_batched_workspace.argtypes = [P, u32, u32, i32, P]
+            L.ans_gemm_batched.argtypes = [P, u32, u32, i32, u32, P, sz, P, P]
             for name in EXPORTS:
                 if name not in ("ans_status_string", "ans_last_error", "ans_num_tiles"):
                     getattr(L, name).restype = i32
@@ -223,6 +232,37 @@ def ans_gemm_uncompressed(d_X, M: int, d_W, layout: AnsLayout, scale_kind: int, 
                                         _ptr(d_scales), group_k, _ptr(d_Y), _ptr(d_ws),
                                         ws_bytes, _ptr(d_status), _stream(stream)),
            "ans_gemm_uncompressed")
+
+
+def _jobs(jobs):
+    """jobs: sequence of (d_X, tiles, d_scales, d_Y) -> a ctypes array (the
+    AnsTiles structs must stay alive for the call)."""
+    def addr(t):
+        return None if t is None else _ptr(t).value
+    arr = (AnsGemmJob * len(jobs))()
+    for j, (x, tiles, sc, y) in enumerate(jobs):
+        arr[j].d_X = addr(x)
+        arr[j].W = C.addressof(tiles)
+        arr[j].d_scales = addr(sc)
+        arr[j].d_Y = addr(y)
+    return arr
+
+
+def ans_gemm_batched_workspace(jobs, M: int, scale_kind: int) -> int:
+    out = C.c_size_t(0)
+    arr = _jobs(jobs)
+    _check(load().ans_gemm_batched_workspace(arr, len(jobs), M, scale_kind, C.byref(out)),
+           "ans_gemm_batched_workspace")
+    return out.value
+
+
+def ans_gemm_batched(jobs, M: int, scale_kind: int, group_k: int, d_ws, ws_bytes: int, d_status,
+                     stream=None):
+    """Several layers of one layout in one call: jobs = [(d_X, tiles, d_scales, d_Y), ...]."""
+    arr = _jobs(jobs)
+    _check(load().ans_gemm_batched(arr, len(jobs), M, scale_kind, group_k, _ptr(d_ws), ws_bytes,
+                                   _ptr(d_status), _stream(stream)),
+           "ans_gemm_batched")
 
 
 # ---- marshalling helper: a compressed layer resident on a device -----------------

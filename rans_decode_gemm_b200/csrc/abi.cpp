@@ -374,3 +374,121 @@ ans_status ans_gemm_noalloc(const uint16_t* d_X, uint32_t M, const ans_tiles* W,
 void ansdev_set_trace(void* d_buf, size_t bytes) { ansdev::set_trace_buffer(d_buf, bytes); }
 
 }  // extern "C"
+
+namespace {
+
+// Shared checks of a batch; on success *sms is the device's SM count.
+ans_status check_batch(const ans_gemm_job* jobs, uint32_t n_jobs, uint32_t M,
+                       ans_scale_kind scale_kind, int* sms) {
+  if (!jobs || n_jobs == 0 || n_jobs > ANS_MAX_BATCH) return ANS_ERR_ARG;
+  for (uint32_t j = 0; j < n_jobs; ++j) {
+    if (!jobs[j].W) return ANS_ERR_ARG;
+    ans_status st = check_layout(&jobs[j].W->layout);
+    if (st != ANS_OK) return st;
+    const ans_layout& a = jobs[0].W->layout;
+    const ans_layout& b = jobs[j].W->layout;
+    if (a.dtype != b.dtype || a.N != b.N || a.K != b.K || a.tile_n != b.tile_n ||
+        a.tile_k != b.tile_k || (a.state_bits == 64) != (b.state_bits == 64))
+      return ANS_ERR_SHAPE;
+  }
+  (void)M;
+  (void)scale_kind;
+  return device_info(sms);
+}
+
+// Plans of a batch: *share for one job on its share of the SMs (used when
+// it takes the small-M schedule, all jobs in one launch), *full for one job
+// on all SMs (consecutive launches otherwise); *ws_job the workspace bytes of
+// one job, enough for either.
+ans_status batch_plan(const ans_gemm_job* jobs, uint32_t n_jobs, uint32_t M,
+                      ans_scale_kind scale_kind, int sms, ansdev::GemmPlan* share,
+                      ansdev::GemmPlan* full, size_t* ws_job) {
+  ansdev::LayerDev L;
+  fill_layer_plain(&jobs[0].W->layout, &L);
+  const int part = sms / static_cast<int>(n_jobs) > 0 ? sms / static_cast<int>(n_jobs) : 1;
+  if (!ansdev::make_gemm_plan(L, M, scale_kind, true, part, share)) return ANS_ERR_UNSUPPORTED;
+  if (!ansdev::make_gemm_plan(L, M, scale_kind, true, sms, full)) return ANS_ERR_UNSUPPORTED;
+  const size_t a = share->ws_bytes > full->ws_bytes ? share->ws_bytes : full->ws_bytes;
+  *ws_job = ((a + 255) / 256) * 256;
+  return ANS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+ans_status ans_gemm_batched_workspace(const ans_gemm_job* jobs, uint32_t n_jobs, uint32_t M,
+                                      ans_scale_kind scale_kind, size_t* bytes) {
+  if (!bytes) return ANS_ERR_ARG;
+  int sms = 0;
+  ans_status st = check_batch(jobs, n_jobs, M, scale_kind, &sms);
+  if (st != ANS_OK) return st;
+  if (M == 0) { *bytes = 0; return ANS_OK; }
+  ansdev::GemmPlan share, full;
+  size_t ws_job = 0;
+  st = batch_plan(jobs, n_jobs, M, scale_kind, sms, &share, &full, &ws_job);
+  if (st != ANS_OK) return st;
+  *bytes = n_jobs * ws_job;
+  return ANS_OK;
+}
+
+ans_status ans_gemm_batched(const ans_gemm_job* jobs, uint32_t n_jobs, uint32_t M,
+                            ans_scale_kind scale_kind, uint32_t group_k, void* d_ws,
+                            size_t ws_bytes, uint32_t* d_status, ans_stream_t stream) {
+  int sms = 0;
+  ans_status st = check_batch(jobs, n_jobs, M, scale_kind, &sms);
+  if (st != ANS_OK) return st;
+  ansdev::LayerDev Ls[ANS_MAX_BATCH];
+  const ansdev::LayerDev* Lp[ANS_MAX_BATCH];
+  const uint16_t* Xs[ANS_MAX_BATCH];
+  const void* Ss[ANS_MAX_BATCH];
+  float* Ys[ANS_MAX_BATCH];
+  for (uint32_t j = 0; j < n_jobs; ++j) {
+    const ans_tiles* W = jobs[j].W;
+    st = check_codebook(&W->codebook, W->layout.dtype);
+    if (st != ANS_OK) return st;
+    st = check_scales(W->layout.dtype, scale_kind, jobs[j].d_scales, group_k, W->layout);
+    if (st != ANS_OK) return st;
+    if (!W->stream || !W->offsets) return ANS_ERR_ARG;
+    if (W->layout.dtype == ANS_BF16_SPLIT && !W->raw) return ANS_ERR_ARG;
+    if (reinterpret_cast<uintptr_t>(W->stream) % 16 != 0 ||
+        reinterpret_cast<uintptr_t>(W->offsets) % 8 != 0 ||
+        (W->raw && reinterpret_cast<uintptr_t>(W->raw) % 16 != 0))
+      return ANS_ERR_ARG;
+    if (M > 0) {
+      if (!jobs[j].d_X || !jobs[j].d_Y) return ANS_ERR_ARG;
+      if (reinterpret_cast<uintptr_t>(jobs[j].d_X) % 16 != 0 ||
+          reinterpret_cast<uintptr_t>(jobs[j].d_Y) % 16 != 0 ||
+          (jobs[j].d_scales && reinterpret_cast<uintptr_t>(jobs[j].d_scales) % 16 != 0))
+        return ANS_ERR_ARG;
+    }
+    fill_layer(W, &Ls[j]);
+    Lp[j] = &Ls[j];
+    Xs[j] = jobs[j].d_X;
+    Ss[j] = jobs[j].d_scales;
+    Ys[j] = jobs[j].d_Y;
+  }
+  if (M == 0) return ANS_OK;
+  if (!d_status || !d_ws || reinterpret_cast<uintptr_t>(d_ws) % 256 != 0) return ANS_ERR_ARG;
+  ansdev::GemmPlan share, full;
+  size_t ws_job = 0;
+  st = batch_plan(jobs, n_jobs, M, scale_kind, sms, &share, &full, &ws_job);
+  if (st != ANS_OK) return st;
+  if (ws_bytes < n_jobs * ws_job) return ANS_ERR_BUFFER_TOO_SMALL;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (share.local) {
+    cudaError_t e = ansdev::launch_gemm_batched(share, n_jobs, Lp, Xs, Ss, scale_kind, group_k, Ys,
+                                                d_ws, d_status, s);
+    if (e != cudaSuccess) return cuda_fail(e, "ans_gemm_batched");
+    return ANS_OK;
+  }
+  for (uint32_t j = 0; j < n_jobs; ++j) {
+    cudaError_t e = ansdev::launch_gemm(full, Ls[j], true, nullptr, Xs[j], Ss[j], scale_kind,
+                                        group_k, Ys[j], static_cast<uint8_t*>(d_ws) + j * ws_job,
+                                        d_status, s);
+    if (e != cudaSuccess) return cuda_fail(e, "ans_gemm_batched");
+  }
+  return ANS_OK;
+}
+
+}  // extern "C"

@@ -483,7 +483,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     }
     // split-K arrival once every partial of this CTA is written; the
     // reductions this CTA owns run after the CTA barrier, on every thread
-    if (npend) splitk_arrive(P, pend, npend, e, &reduce_flag);
+    if (npend) splitk_arrive(P, G, pend, npend, e, &reduce_flag);
     if (e == 0) {
       red_n = npend;
       red_seg[0] = pend[0];
@@ -504,7 +504,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
   if (reduce_flag) {
     fence_acq_rel_gpu();  // acquire: the counter showed every contributor arrived
     for (uint32_t k = 0; k < red_n; ++k)
-      if ((reduce_flag >> k) & 1u) splitk_reduce(P, red_seg[k], threadIdx.x, blockDim.x);
+      if ((reduce_flag >> k) & 1u) splitk_reduce(P, G, red_seg[k], threadIdx.x, blockDim.x);
   }
 }
 
@@ -756,35 +756,20 @@ static cudaError_t launch_variant(const GemmPlan& plan, const GemmDev& P, cudaSt
                     stream, P);
 }
 
-cudaError_t launch_gemm(const GemmPlan& plan, const LayerDev& L, bool decode, const void* w_plain,
-                        const uint16_t* X, const void* scales, uint32_t scale_kind,
-                        uint32_t group_k, float* Y, void* ws, uint32_t* status,
-                        cudaStream_t stream) {
-  if (plan.M == 0) return cudaSuccess;
+// Kernel parameters of one layer's launch; ws is that layer's workspace.
+static GemmDev make_gemm_dev(const GemmPlan& plan, const LayerDev& L, const void* w_plain,
+                             const uint16_t* X, const void* scales, uint32_t scale_kind,
+                             uint32_t group_k, float* Y, void* ws, uint32_t* status) {
   uint8_t* wsb = static_cast<uint8_t*>(ws);
-  uint32_t* counters = reinterpret_cast<uint32_t*>(wsb);
-  float* partials = reinterpret_cast<float*>(wsb + plan.ws_counters_bytes);
-  uint16_t* x16 = reinterpret_cast<uint16_t*>(wsb + plan.ws_counters_bytes +
-                                              ((plan.ws_partials_bytes + 255) / 256) * 256);
-  if (!plan.local) {
-    const uint64_t n_chunks = static_cast<uint64_t>(plan.n_pass) * (L.K / 16) * plan.T_pass * 2;
-    uint32_t blocks = static_cast<uint32_t>((n_chunks + 255) / 256);
-    if (blocks > 4096) blocks = 4096;
-    if (blocks == 0) blocks = 1;
-    cudaError_t e = launch_pdl(x_stage_kernel, dim3(blocks), dim3(256), 0, stream, X,
-                               reinterpret_cast<uint8_t*>(x16), plan.M, L.K, plan.T_pass,
-                               plan.n_pass, plan.ab_f16);
-    if (e != cudaSuccess) return e;
-  }
-
   GemmDev P;
   std::memset(&P, 0, sizeof(P));
   P.L = L;
   P.w_plain = w_plain;
   P.scales = scales;
   P.Y = Y;
-  P.partials = partials;
-  P.counters = counters;
+  P.counters = reinterpret_cast<uint32_t*>(wsb);
+  P.partials = reinterpret_cast<float*>(wsb + plan.ws_counters_bytes);
+  P.xs = wsb + plan.ws_counters_bytes + ((plan.ws_partials_bytes + 255) / 256) * 256;
   P.status = status;
   P.scale_kind = scale_kind;
   P.group_k = group_k;
@@ -809,10 +794,30 @@ cudaError_t launch_gemm(const GemmPlan& plan, const LayerDev& L, bool decode, co
   P.off_x = plan.off_x;
   P.off_bars = plan.off_bars;
   P.trace = g_trace;
-  P.xs = reinterpret_cast<const uint8_t*>(x16);
   P.X = X;
   P.x_f16 = plan.ab_f16;
   P.n_slots = plan.n_slots;
+  P.n_cta = plan.grid;
+  P.cta0 = 0;
+  return P;
+}
+
+cudaError_t launch_gemm(const GemmPlan& plan, const LayerDev& L, bool decode, const void* w_plain,
+                        const uint16_t* X, const void* scales, uint32_t scale_kind,
+                        uint32_t group_k, float* Y, void* ws, uint32_t* status,
+                        cudaStream_t stream) {
+  if (plan.M == 0) return cudaSuccess;
+  const GemmDev P = make_gemm_dev(plan, L, w_plain, X, scales, scale_kind, group_k, Y, ws, status);
+  if (!plan.local) {
+    const uint64_t n_chunks = static_cast<uint64_t>(plan.n_pass) * (L.K / 16) * plan.T_pass * 2;
+    uint32_t blocks = static_cast<uint32_t>((n_chunks + 255) / 256);
+    if (blocks > 4096) blocks = 4096;
+    if (blocks == 0) blocks = 1;
+    cudaError_t e = launch_pdl(x_stage_kernel, dim3(blocks), dim3(256), 0, stream, X,
+                               const_cast<uint8_t*>(P.xs), plan.M, L.K, plan.T_pass,
+                               plan.n_pass, plan.ab_f16);
+    if (e != cudaSuccess) return e;
+  }
   if (plan.local) return launch_gemm_local(plan, P, decode, stream);
 
   switch (plan.fmt | (decode ? 0u : 8u)) {
@@ -840,6 +845,25 @@ cudaError_t launch_gemm(const GemmPlan& plan, const LayerDev& L, bool decode, co
     case 8 | kFmtFp8F16: return launch_variant<false, kFmtFp8F16>(plan, P, stream);
   }
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_gemm_batched(const GemmPlan& plan, uint32_t n, const LayerDev* const* Ls,
+                                const uint16_t* const* Xs, const void* const* scales,
+                                uint32_t scale_kind, uint32_t group_k, float* const* Ys, void* ws,
+                                uint32_t* status, cudaStream_t stream) {
+  if (plan.M == 0 || n == 0) return cudaSuccess;
+  if (!plan.local || n > kMaxBatch) return cudaErrorInvalidValue;
+  static_assert(sizeof(BatchDev) <= 32000, "kernel parameter limit");
+  BatchDev B;
+  std::memset(&B, 0, sizeof(B));
+  B.n_jobs = n;
+  const size_t ws_job = ((plan.ws_bytes + 255) / 256) * 256;
+  for (uint32_t j = 0; j < n; ++j) {
+    B.job[j] = make_gemm_dev(plan, *Ls[j], nullptr, Xs[j], scales[j], scale_kind, group_k, Ys[j],
+                             static_cast<uint8_t*>(ws) + j * ws_job, status);
+    B.job[j].cta0 = j * plan.grid;
+  }
+  return launch_gemm_local_batch(plan, B, n * plan.grid, stream);
 }
 
 }  // namespace ansdev

@@ -93,10 +93,10 @@ __device__ __forceinline__ void epi_emit16(const GemmDev& P, const float (&v)[16
 // are written, for at most two segments.  Returns (to every thread) a bit per
 // segment for which this CTA arrived last and must reduce; the reducing CTA
 // runs fence_acq_rel_gpu() before it reads the other CTAs' partials.
-__device__ __forceinline__ uint32_t splitk_arrive(const GemmDev& P, const uint32_t* segs,
+__device__ __forceinline__ uint32_t splitk_arrive(const GemmDev& P, uint32_t G, const uint32_t* segs,
                                                   uint32_t n, uint32_t e,
                                                   volatile uint32_t* reduce_flag) {
-  const uint32_t G = gridDim.x, n_kt = P.L.n_kt, U = static_cast<uint32_t>(P.n_units);
+  const uint32_t n_kt = P.L.n_kt, U = static_cast<uint32_t>(P.n_units);
   named_bar_sync(1, 128);
   if (e == 0) {
     // release: one gpu-scope acq_rel fence after the barrier covers the
@@ -125,9 +125,9 @@ __device__ __forceinline__ uint32_t splitk_arrive(const GemmDev& P, const uint32
 // Reduction of segment seg by the CTA that arrived last, run by threads
 // tid = 0 .. nthr - 1 of that CTA (the whole CTA, once its other work is
 // done).
-__device__ __forceinline__ void splitk_reduce(const GemmDev& P, uint32_t seg, uint32_t tid,
+__device__ __forceinline__ void splitk_reduce(const GemmDev& P, uint32_t G, uint32_t seg, uint32_t tid,
                                               uint32_t nthr) {
-  const uint32_t G = gridDim.x, n_kt = P.L.n_kt, U = static_cast<uint32_t>(P.n_units);
+  const uint32_t n_kt = P.L.n_kt, U = static_cast<uint32_t>(P.n_units);
   const uint32_t p = seg / P.n_rb, rb = seg % P.n_rb;
   const uint32_t s_lo = seg * n_kt, s_hi = s_lo + n_kt;
   const uint32_t c_first = cta_of(U, G, s_lo);
@@ -226,9 +226,9 @@ __device__ __forceinline__ void splitk_reduce(const GemmDev& P, uint32_t seg, ui
 // loads of up to 8 contributors of each in flight together, so both
 // reductions cost one round trip instead of two.  The additions per item are
 // the same, in the same order, as in splitk_reduce.
-__device__ __forceinline__ bool splitk_reduce2(const GemmDev& P, const uint32_t (&seg)[2],
+__device__ __forceinline__ bool splitk_reduce2(const GemmDev& P, uint32_t G, const uint32_t (&seg)[2],
                                                uint32_t tid, uint32_t nthr) {
-  const uint32_t G = gridDim.x, n_kt = P.L.n_kt, U = static_cast<uint32_t>(P.n_units);
+  const uint32_t n_kt = P.L.n_kt, U = static_cast<uint32_t>(P.n_units);
   const uint64_t cta_stride = 2ull * P.H * P.T_pass * 128;
   uint32_t p[2], rb[2], c_first[2], c_last[2], t_valid[2], n_items[2];
   const float* first[2];

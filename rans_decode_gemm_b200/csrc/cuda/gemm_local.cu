@@ -79,9 +79,10 @@ __device__ __forceinline__ void sts128(uint32_t addr, const uint32_t (&o)[4]) {
   sts128(addr, o[0], o[1], o[2], o[3]);
 }
 
-template <bool kDecode, uint32_t kFmt, bool kWide>
-__global__ void __launch_bounds__(kLocalThreads, 1)
-    fused_gemm_local_kernel(const __grid_constant__ GemmDev P) {
+// One CTA of the launch that P describes: CTA blockIdx.x - P.cta0 of the
+// P.n_cta that share P's layer (kBatch), or of the whole grid.
+template <bool kDecode, uint32_t kFmt, bool kWide, bool kBatch>
+__device__ __forceinline__ void local_cta(const GemmDev& P) {
   extern __shared__ __align__(2048) uint8_t smem[];
   __shared__ uint32_t tmem_slot;
   __shared__ uint32_t abort_flag;
@@ -92,9 +93,10 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
 
   const uint32_t warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t D = P.D, H = P.H, C = P.C, T = P.T;
-  const uint32_t G = gridDim.x;
-  const uint32_t ub = cta_begin(static_cast<uint32_t>(P.n_units), G, blockIdx.x);
-  const uint32_t ue = cta_begin(static_cast<uint32_t>(P.n_units), G, blockIdx.x + 1);
+  const uint32_t G = kBatch ? P.n_cta : gridDim.x;
+  const uint32_t cta = kBatch ? blockIdx.x - P.cta0 : blockIdx.x;
+  const uint32_t ub = cta_begin(static_cast<uint32_t>(P.n_units), G, cta);
+  const uint32_t ue = cta_begin(static_cast<uint32_t>(P.n_units), G, cta + 1);
   const uint32_t n_kt = P.L.n_kt, n_tiles = P.L.n_tiles;
 
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem + P.off_lut);
@@ -564,7 +566,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
       const uint32_t s_lo = seg * n_kt, s_hi = s_lo + n_kt;
       const bool complete = ub <= s_lo && ue >= s_hi;
       const uint32_t pslot = (seg == seg_first) ? 0u : 1u;
-      float* part = P.partials + (static_cast<uint64_t>(blockIdx.x) * 2 + pslot) * H * P.T_pass * 128;
+      float* part = P.partials + (static_cast<uint64_t>(cta) * 2 + pslot) * H * P.T_pass * 128;
 #pragma unroll
       for (uint32_t ck = 0; ck < 2; ++ck) {
         if (ck >= nck) break;
@@ -581,7 +583,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
     }
     // split-K arrival once every partial of this CTA is written; the
     // reductions this CTA owns run after the CTA barrier, on every thread
-    if (npend) splitk_arrive(P, pend, npend, e, &reduce_flag);
+    if (npend) splitk_arrive(P, G, pend, npend, e, &reduce_flag);
     if (e == 0) {
       trace_mark(P, 62);
       red_n = npend;
@@ -603,10 +605,26 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
   if (reduce_flag) {
     fence_acq_rel_gpu();  // acquire: the counter showed every contributor arrived
     const uint32_t both[2] = {red_seg[0], red_seg[1]};
-    if (!(reduce_flag == 3u && splitk_reduce2(P, both, threadIdx.x, blockDim.x)))
+    if (!(reduce_flag == 3u && splitk_reduce2(P, G, both, threadIdx.x, blockDim.x)))
       for (uint32_t k = 0; k < red_n; ++k)
-        if ((reduce_flag >> k) & 1u) splitk_reduce(P, red_seg[k], threadIdx.x, blockDim.x);
+        if ((reduce_flag >> k) & 1u) splitk_reduce(P, G, red_seg[k], threadIdx.x, blockDim.x);
   }
+}
+
+template <bool kDecode, uint32_t kFmt, bool kWide>
+__global__ void __launch_bounds__(kLocalThreads, 1)
+    fused_gemm_local_kernel(const __grid_constant__ GemmDev P) {
+  local_cta<kDecode, kFmt, kWide, false>(P);
+}
+
+// Several layers of one shape in one launch (decode only): the CTAs of job j
+// run the kernel above on job j's layer.
+template <uint32_t kFmt, bool kWide>
+__global__ void __launch_bounds__(kLocalThreads, 1)
+    fused_gemm_local_batch_kernel(const __grid_constant__ BatchDev B) {
+  uint32_t j = 0;
+  while (j + 1 < B.n_jobs && blockIdx.x >= B.job[j + 1].cta0) ++j;
+  local_cta<true, kFmt, kWide, true>(B.job[j]);
 }
 
 template <bool kDecode, uint32_t kFmt, bool kWide = false>
@@ -651,6 +669,50 @@ cudaError_t launch_gemm_local(const GemmPlan& plan, const GemmDev& P, bool decod
     case 8 | kFmtInt4Bf16: return launch_local_variant<false, kFmtInt4Bf16>(plan, P, stream);
     case 8 | kFmtInt4F16Group: return launch_local_variant<false, kFmtInt4F16Group>(plan, P, stream);
     case 8 | kFmtFp8F16: return launch_local_variant<false, kFmtFp8F16>(plan, P, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <uint32_t kFmt, bool kWide>
+static cudaError_t launch_local_batch_variant(const GemmPlan& plan, const BatchDev& B, uint32_t grid,
+                                              cudaStream_t stream) {
+  auto kern = fused_gemm_local_batch_kernel<kFmt, kWide>;
+  static int attr_set[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = 1;
+  }
+  return launch_pdl(kern, dim3(grid), dim3((kLocalFixedWarps + plan.D) * 32), plan.smem_bytes,
+                    stream, B);
+}
+
+cudaError_t launch_gemm_local_batch(const GemmPlan& plan, const BatchDev& B, uint32_t grid,
+                                    cudaStream_t stream) {
+  const bool wide = B.job[0].L.wide != 0;
+  switch (plan.fmt) {
+    case kFmtBf16Split:
+      return wide ? launch_local_batch_variant<kFmtBf16Split, true>(plan, B, grid, stream)
+                  : launch_local_batch_variant<kFmtBf16Split, false>(plan, B, grid, stream);
+    case kFmtInt4Bf16:
+      return wide ? launch_local_batch_variant<kFmtInt4Bf16, true>(plan, B, grid, stream)
+                  : launch_local_batch_variant<kFmtInt4Bf16, false>(plan, B, grid, stream);
+    case kFmtInt4F16Group:
+      return wide ? launch_local_batch_variant<kFmtInt4F16Group, true>(plan, B, grid, stream)
+                  : launch_local_batch_variant<kFmtInt4F16Group, false>(plan, B, grid, stream);
+    case kFmtInt4PairBf16:
+      return wide ? launch_local_batch_variant<kFmtInt4PairBf16, true>(plan, B, grid, stream)
+                  : launch_local_batch_variant<kFmtInt4PairBf16, false>(plan, B, grid, stream);
+    case kFmtInt4PairF16Group:
+      return wide ? launch_local_batch_variant<kFmtInt4PairF16Group, true>(plan, B, grid, stream)
+                  : launch_local_batch_variant<kFmtInt4PairF16Group, false>(plan, B, grid, stream);
+    case kFmtFp8F16:
+      return wide ? launch_local_batch_variant<kFmtFp8F16, true>(plan, B, grid, stream)
+                  : launch_local_batch_variant<kFmtFp8F16, false>(plan, B, grid, stream);
   }
   return cudaErrorInvalidValue;
 }

@@ -79,6 +79,17 @@ struct GemmDev {
   const uint16_t* X;          // local schedule: X as given (bf16, M x K row-major)
   uint32_t x_f16;             // local schedule: convert X to f16 for the MMA
   uint32_t n_slots;           // local schedule: accumulator slots (barriers) per CTA
+  uint32_t n_cta;             // CTAs that share this layer's units (the grid, or a batch job's share)
+  uint32_t cta0;              // first CTA of this layer in the grid (0 unless batched)
+};
+
+// Several layers of one shape in one launch of the local schedule: job j
+// owns CTAs [job[j].cta0, job[j].cta0 + job[j].n_cta).  Passed by value as
+// the kernel parameter (well under the 32 KB parameter limit).
+constexpr uint32_t kMaxBatch = 8;
+struct BatchDev {
+  uint32_t n_jobs;
+  GemmDev job[kMaxBatch];
 };
 
 // Internal profiling hook: when set, every fused-GEMM CTA writes globaltimer
@@ -99,6 +110,10 @@ constexpr uint32_t kLocalProducersMax = 15;
 cudaError_t launch_gemm_local(const GemmPlan& plan, const GemmDev& P, bool decode,
                               cudaStream_t stream);
 
+// Local schedule, batched: one launch of grid CTAs over B's jobs.
+cudaError_t launch_gemm_local_batch(const GemmPlan& plan, const BatchDev& B, uint32_t grid,
+                                    cudaStream_t stream);
+
 // Fills a plan; returns false if the shape cannot be scheduled.
 bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool decode,
                     int num_sms, GemmPlan* plan);
@@ -112,5 +127,12 @@ cudaError_t launch_gemm(const GemmPlan& plan, const LayerDev& L, bool decode, co
                         const uint16_t* X, const void* scales, uint32_t scale_kind,
                         uint32_t group_k, float* Y, void* ws, uint32_t* status,
                         cudaStream_t stream);
+// n layers of one shape (plan made for one of them with a CTA cap of grid / n;
+// plan.local), each with its own X, scales and Y, in one launch; ws holds n
+// consecutive workspaces of round_up(plan.ws_bytes, 256) bytes.
+cudaError_t launch_gemm_batched(const GemmPlan& plan, uint32_t n, const LayerDev* const* Ls,
+                                const uint16_t* const* Xs, const void* const* scales,
+                                uint32_t scale_kind, uint32_t group_k, float* const* Ys, void* ws,
+                                uint32_t* status, cudaStream_t stream);
 
 }  // namespace ansdev

@@ -140,3 +140,25 @@ def test_single_symbol_layer(oracle, ans_lib):
     assert (np.frombuffer(stream.tobytes(), np.uint32) == 65536).all()
     st, out = oracle.decode(ans.FP8_E4M3, stream, offsets, None, N, K, 128, 64, cb.freq_array())
     assert st == 0 and np.array_equal(out, w)
+
+
+def test_batched_argument_checks(ans_lib):
+    # argument and layout errors are reported before any device is touched
+    a = ans.make_layout(ans.BF16_SPLIT, 256, 128, 128, 64)
+    b = ans.make_layout(ans.BF16_SPLIT, 128, 128, 128, 64)
+    cb = ans.AnsCodebook()
+    ta, tb = ans.AnsTiles(a, cb, None, 0, None, None), ans.AnsTiles(b, cb, None, 0, None, None)
+    with pytest.raises(ans.AnsError) as e:
+        ans.ans_gemm_batched_workspace([], 16, 0)
+    assert e.value.status == 1
+    with pytest.raises(ans.AnsError) as e:
+        ans.ans_gemm_batched_workspace([(None, ta, None, None)] * (ans.MAX_BATCH + 1), 16, 0)
+    assert e.value.status == 1
+    with pytest.raises(ans.AnsError) as e:
+        ans.ans_gemm_batched_workspace([(None, ta, None, None), (None, tb, None, None)], 16, 0)
+    assert e.value.status == 2
+    wide = ans.AnsTiles(ans.make_layout(ans.BF16_SPLIT, 256, 128, 128, 64, 64), cb, None, 0, None,
+                        None)
+    lib = ans.load()
+    arr = ans._jobs([(None, ta, None, None), (None, wide, None, None)])
+    assert lib.ans_gemm_batched(arr, 2, 16, 0, 0, None, 0, None, None) == 2   # state widths differ
