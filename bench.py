@@ -550,6 +550,42 @@ def sweep(args):
                 del X, Y, Yu, ws
             del layers, Wbs, Wb, dec, dw
             torch.cuda.empty_cache()
+    if not only or "llama8b_mlp" in only:
+        sweep_batched(args, torch, ans, WL, device, stream, st, timed_graph)
+
+
+def sweep_batched(args, torch, ans, WL, device, stream, st, timed_graph):
+    """The Llama MLP's gate and up projections (same layout, same X): two
+    ans_gemm calls against one ans_gemm_batched call, weights from HBM."""
+    cfg = WL.CONFIGS["llama8b_mlp"]
+    mats = []
+    for mi in (0, 1):
+        d = WL.make_weights(cfg, mi)
+        lay = ans.make_layout(cfg.dtype, d["N"], d["K"], cfg.tile_n, cfg.tile_k, args.state_bits)
+        l0 = ans.CompressedLayer.from_weights(d["w"], lay, device=device)
+        copies = [l0] + [ans.CompressedLayer(lay, l0.codebook, l0.h_stream, l0.h_offsets, l0.h_raw,
+                                             device) for _ in range(3)]
+        mats.append((lay, copies))
+    lay = mats[0][0]
+    for M in (1, 8, 16, 32):
+        X = torch.from_numpy(WL.make_x(cfg, M, lay.K).view(np.int16)).to(device)
+        Ys = [torch.empty(M, lay.N, dtype=torch.float32, device=device) for _ in range(2)]
+        nb1 = ans.ans_gemm_workspace(lay, M, 0)
+        ws1 = torch.zeros(max(nb1, 256), dtype=torch.uint8, device=device)
+        jobs = [[(X, mats[j][1][c].tiles, None, Ys[j]) for j in range(2)] for c in range(4)]
+        nb2 = ans.ans_gemm_batched_workspace(jobs[0], M, 0)
+        ws2 = torch.zeros(max(nb2, 256), dtype=torch.uint8, device=device)
+        two = [lambda c=c, j=j: ans.ans_gemm(X, M, mats[j][1][c].tiles, 0, None, 0, Ys[j], ws1, nb1, st)
+               for c in range(4) for j in range(2)]
+        one = [lambda c=c: ans.ans_gemm_batched(jobs[c], M, 0, 0, ws2, nb2, st) for c in range(4)]
+        t2 = timed_graph(two, 20) * 2   # per pair of layers
+        t1 = timed_graph(one, 20)
+        rec = {"workload": "llama8b_mlp", "matrix": "gate+up", "N": 2 * lay.N, "K": lay.K, "M": M,
+               "state_bits": args.state_bits, "two_ans_gemm_us": round(t2, 2),
+               "ans_gemm_batched_us": round(t1, 2), "speedup": round(t2 / t1, 3),
+               "effective_weight_GBps": round(2 * lay.N * lay.K * 2 / (t1 * 1e-6) / 1e9, 1),
+               "status": int(st.item())}
+        print(json.dumps(rec), flush=True)
 
 
 def cpu_baseline(cfg, d, lay, layer, X_h, budget_s=20.0):
