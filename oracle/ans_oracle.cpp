@@ -48,6 +48,10 @@
 // one word is pushed first if x >= 2^40 f_a f_b.  Tile bytes: 32 little-endian
 // u64 final states, then the u32 words in decoder order, then zero padding.
 //
+// int8 (dtype 4; [SB] s2.1 lists int8 among the seven formats measured): one byte per
+// weight, two's complement q in [-128, 127], symbol q + 128, alphabet 256;
+// value q times an optional per-row scale.
+//
 // int4 pairs (dtype 3; the pages call any discrete unit of a layer a symbol and
 // leave the unit open): one symbol per packed int4 byte, i.e. per pair of
 // consecutive K elements (k even, k + 1): s = (q_k + 8) | (q_{k+1} + 8) << 4,
@@ -67,7 +71,7 @@
 
 namespace {
 
-enum { DT_INT4 = 0, DT_BF16_SPLIT = 1, DT_FP8_E4M3 = 2, DT_INT4_PAIRS = 3 };
+enum { DT_INT4 = 0, DT_BF16_SPLIT = 1, DT_FP8_E4M3 = 2, DT_INT4_PAIRS = 3, DT_INT8 = 4 };
 enum { SC_NONE = 0, SC_ROW_BF16 = 1, SC_ROW_F32 = 2, SC_GROUP_BF16 = 3 };
 enum {
   OK = 0, ERR_ARG = 1, ERR_SHAPE = 2, ERR_ALPHABET = 3, ERR_BUFFER_TOO_SMALL = 4,
@@ -109,6 +113,9 @@ uint32_t pair_symbol_at(const void* w, uint64_t idx) {
 uint32_t symbol_at(int dtype, const void* w, uint64_t idx) {
   if (dtype == DT_INT4) return (uint32_t)(int4_code((const uint8_t*)w, idx) + 8);
   if (dtype == DT_INT4_PAIRS) return pair_symbol_at(w, idx);
+  // int8: two's complement code q in [-128, 127]; symbol q + 128 (the byte
+  // with its top bit flipped)
+  if (dtype == DT_INT8) return (uint32_t)((int)(int8_t)((const uint8_t*)w)[idx] + 128);
   if (dtype == DT_BF16_SPLIT) {
     uint16_t bits = ((const uint16_t*)w)[idx];
     return (bits >> 7) & 0xFFu;
@@ -580,7 +587,7 @@ int oracle_encode(int dtype, const void* w, uint32_t N, uint32_t K, uint32_t til
                   uint32_t tile_k, const uint32_t* freq, int prob_bits, uint8_t* stream,
                   uint64_t cap, uint64_t* stream_bytes, uint64_t* offsets, uint8_t* raw,
                   int threads, int state_bits) {
-  if (dtype < 0 || dtype > 3) return ERR_ARG;
+  if (dtype < 0 || dtype > 4) return ERR_ARG;
   if (state_bits != 32 && state_bits != 64) return ERR_ARG;
   if (!layout_ok(N, K, tile_n, tile_k)) return ERR_SHAPE;
   if (state_bits == 64 && prob_bits != 12) return ERR_ARG;  // the pair bound assumes n = 12
@@ -618,7 +625,7 @@ int oracle_decode(int dtype, const uint8_t* stream, uint64_t stream_bytes,
                   uint32_t tile_n, uint32_t tile_k, const uint32_t* freq, int prob_bits,
                   void* w_out, uint64_t tile_begin, uint64_t tile_end, int threads,
                   int state_bits) {
-  if (dtype < 0 || dtype > 3) return ERR_ARG;
+  if (dtype < 0 || dtype > 4) return ERR_ARG;
   if (state_bits != 32 && state_bits != 64) return ERR_ARG;
   if (!layout_ok(N, K, tile_n, tile_k)) return ERR_SHAPE;
   if (state_bits == 64 && prob_bits != 12) return ERR_ARG;
@@ -679,6 +686,8 @@ int oracle_decode(int dtype, const uint8_t* stream, uint64_t stream_bytes,
           uint8_t nib = (uint8_t)((s - 8) & 0xF);
           if (idx % 2 == 0) out[idx / 2] = (uint8_t)((out[idx / 2] & 0xF0) | nib);
           else out[idx / 2] = (uint8_t)((out[idx / 2] & 0x0F) | (nib << 4));
+        } else if (dtype == DT_INT8) {
+          ((uint8_t*)w_out)[idx] = (uint8_t)(int8_t)(s - 128);
         } else if (dtype == DT_BF16_SPLIT) {
           uint8_t r = raw[t * lay.tile_symbols() + (j / 8) * 256 + l * 8 + (j % 8)];
           ((uint16_t*)w_out)[idx] = bf16_from_parts((uint32_t)s, r);
@@ -705,11 +714,12 @@ int oracle_decode(int dtype, const uint8_t* stream, uint64_t stream_bytes,
 //          q * s[n][k / group_k] (SC_GROUP_BF16, s bf16[N][K/group_k])
 //   bf16 : the bf16 value (no scale)
 //   fp8  : e4m3_value(code) (SC_NONE) or e4m3_value(code) * s_n (SC_ROW_F32)
+//   int8 : q (SC_NONE) or q * s_n (SC_ROW_F32 or SC_ROW_BF16)
 // Y is M x n_rows row-major doubles.
 int oracle_gemm(int dtype, const uint16_t* X, uint32_t M, uint32_t K, const void* W,
                 uint32_t N, int scale_kind, const void* scales, uint32_t group_k,
                 const uint32_t* rows, uint32_t n_rows, double* Y, int threads) {
-  if (dtype < 0 || dtype > 3) return ERR_ARG;
+  if (dtype < 0 || dtype > 4) return ERR_ARG;
   if (scale_kind == SC_GROUP_BF16 && (group_k == 0 || K % group_k != 0)) return ERR_ARG;
   if (scale_kind != SC_NONE && scales == nullptr) return ERR_ARG;
   if (rows == nullptr) n_rows = N;
@@ -727,6 +737,10 @@ int oracle_gemm(int dtype, const uint16_t* X, uint32_t M, uint32_t K, const void
         else if (scale_kind == SC_GROUP_BF16)
           v *= bf16_value(((const uint16_t*)scales)[n * (K / group_k) + k / group_k]);
         else if (scale_kind == SC_ROW_F32) v *= f32_value(scales, n);
+      } else if (dtype == DT_INT8) {
+        v = (double)(int8_t)((const uint8_t*)W)[idx];
+        if (scale_kind == SC_ROW_F32) v *= f32_value(scales, n);
+        else if (scale_kind == SC_ROW_BF16) v *= bf16_value(((const uint16_t*)scales)[n]);
       } else if (dtype == DT_BF16_SPLIT) {
         v = bf16_value(((const uint16_t*)W)[idx]);
         if (scale_kind == SC_ROW_BF16) v *= bf16_value(((const uint16_t*)scales)[n]);

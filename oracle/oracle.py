@@ -17,7 +17,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "ans_oracle.cpp")
 LIB = os.path.join(HERE, "liboracle.so")
 
-INT4, BF16_SPLIT, FP8_E4M3, INT4_PAIRS = 0, 1, 2, 3
+INT4, BF16_SPLIT, FP8_E4M3, INT4_PAIRS, INT8 = 0, 1, 2, 3, 4
 SCALE_NONE, SCALE_ROW_BF16, SCALE_ROW_F32, SCALE_GROUP_BF16 = 0, 1, 2, 3
 OK, ERR_ARG, ERR_SHAPE, ERR_ALPHABET, ERR_BUFFER_TOO_SMALL, ERR_CORRUPT = 0, 1, 2, 3, 4, 6
 

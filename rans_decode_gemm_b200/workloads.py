@@ -27,7 +27,7 @@ from dataclasses import dataclass, field
 import numpy as np
 import torch
 
-INT4, BF16_SPLIT, FP8_E4M3, INT4_PAIRS = 0, 1, 2, 3
+INT4, BF16_SPLIT, FP8_E4M3, INT4_PAIRS, INT8 = 0, 1, 2, 3, 4
 SCALE_NONE, SCALE_ROW_BF16, SCALE_ROW_F32, SCALE_GROUP_BF16 = 0, 1, 2, 3
 
 
@@ -57,6 +57,8 @@ CONFIGS = {
                        [1, 2, 4, 8, 16, 32, 64, 128, 256, 512, 1024], 3),
     "fp8_405b": Config("fp8_405b", FP8_E4M3, 53248, 16384, 128, 128, SCALE_ROW_F32, 0,
                        [1, 4, 16, 64, 256, 2048], 4),
+    # int8 (absmax per row) of a Llama-8B-shaped MLP projection
+    "int8_8b": Config("int8_8b", INT8, 14336, 4096, 128, 64, SCALE_ROW_F32, 0, [1, 16, 128], 5),
 }
 
 
@@ -111,6 +113,15 @@ def make_weights(cfg: Config, matrix: int = 0, N: int | None = None, K: int | No
                 lo, hi = np.searchsorted(outliers, [r0 * K, r1 * K])
                 v[outliers[lo:hi] - r0 * K] *= 20.0
             w[r0 * K:r1 * K] = to_bf16_bits(v)
+    elif cfg.dtype == INT8:
+        w = np.empty(N * K, np.uint8)
+        scales = np.empty(N, np.float32)
+        for r0, r1 in _rows_chunks(N, K):
+            v = (rng.standard_normal((r1 - r0, K)) * 0.02).astype(np.float32)
+            s = (np.abs(v).max(axis=1) / 127.0).astype(np.float32)
+            scales[r0:r1] = s
+            q = np.clip(np.rint(v / s[:, None]), -127, 127).astype(np.int8)
+            w[r0 * K:r1 * K] = q.view(np.uint8).reshape(-1)
     else:
         w = np.empty(N * K, np.uint8)
         scales = np.empty(N, np.float32)

@@ -537,6 +537,50 @@ def test_pair_encode_decode_identity_and_size(oracle, name, N, K, state_bits):
     assert np.array_equal(Yp, Y1)
 
 
+# ---- int8 symbols -------------------------------------------------------------------
+def test_int8_symbol_is_code_plus_128(oracle):
+    # every byte once: one count at byte ^ 0x80 = q + 128 for the two's complement q
+    counts = oracle.histogram(WL.INT8, np.arange(256, dtype=np.uint8), 256)
+    assert counts.size == 256 and (counts == 1).all()
+    for byte, sym in ((0xFF, 127), (0x80, 0), (0x7F, 255), (0x00, 128)):
+        c = oracle.histogram(WL.INT8, np.array([byte], np.uint8), 1)
+        assert int(np.argmax(c)) == sym and c.sum() == 1
+
+
+@pytest.mark.parametrize("state_bits,band", [(32, 0.15), (64, 0.25)])
+def test_int8_encode_decode_identity_and_size(oracle, state_bits, band):
+    cfg, d = _small("int8_8b", 512, 1024)
+    counts = oracle.histogram(WL.INT8, d["w"], 512 * 1024)
+    H = oracle.entropy(counts)
+    _, freq = oracle.normalize(counts)
+    st, stream, offsets, raw = oracle.encode(WL.INT8, d["w"], 512, 1024, cfg.tile_n, cfg.tile_k,
+                                             freq, state_bits=state_bits)
+    assert st == 0 and raw is None
+    st, out = oracle.decode(WL.INT8, stream, offsets, None, 512, 1024, cfg.tile_n, cfg.tile_k,
+                            freq, state_bits=state_bits)
+    assert st == 0 and np.array_equal(out, d["w"])
+    gap = 8.0 * stream.size / (512 * 1024) - H
+    assert -0.01 < gap < band, gap
+    # absmax-per-row int8 of Gaussian weights: entropy near log2(sigma / s * sqrt(2 pi e))
+    # with sigma / s = 127 / E[max |z| of 1024 normals] (about 3.2): 7.0-7.4 bits
+    assert 6.9 < H < 7.5
+
+
+def test_gemm_int8_exact_integers(oracle):
+    rng = np.random.default_rng(12)
+    M, N, K = 4, 40, 96
+    q = rng.integers(-128, 128, size=(N, K)).astype(np.int64)
+    xi = rng.integers(-20, 21, size=(M, K)).astype(np.int64)
+    Xb = WL.to_bf16_bits(xi.astype(np.float32))
+    W = q.astype(np.int8).view(np.uint8).reshape(-1)
+    Y = oracle.gemm(WL.INT8, Xb.reshape(M, K), M, K, W, N)
+    assert np.array_equal(Y, (xi @ q.T).astype(np.float64))
+    # row scales 2^-r (fp32) keep it exact
+    s = np.array([2.0 ** -(n % 5) for n in range(N)], np.float32)
+    Ys = oracle.gemm(WL.INT8, Xb, M, K, W, N, WL.SCALE_ROW_F32, s)
+    assert np.array_equal(Ys, (xi @ q.T).astype(np.float64) * s.astype(np.float64)[None, :])
+
+
 # ---- fp64 GEMM ------------------------------------------------------------------
 def test_gemm_int4_exact_integers(oracle):
     rng = np.random.default_rng(2)
