@@ -420,6 +420,10 @@ def dequant_bf16(torch, cfg, d, device):
         if s.dim() == 1:
             return (q * s[:, None]).to(torch.bfloat16)
         return (q * s.repeat_interleave(K // s.shape[1], dim=1)).to(torch.bfloat16)
+    if cfg.dtype == 4:  # int8 codes, fp32 row scales
+        q = torch.from_numpy(d["w"].view(np.int8)).to(device).view(N, K).float()
+        s = torch.from_numpy(d["scales"]).to(device)
+        return (q * s[:, None]).to(torch.bfloat16)
     codes = torch.from_numpy(d["w"]).to(device).view(torch.float8_e4m3fn).view(N, K)
     s = torch.from_numpy(d["scales"]).to(device)
     return (codes.float() * s[:, None]).to(torch.bfloat16)
@@ -438,7 +442,7 @@ def sweep(args):
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
     peaks, peaks_src = load_peaks()
-    nominal = {0: 0.5, 1: 2.0, 2: 1.0}
+    nominal = {0: 0.5, 1: 2.0, 2: 1.0, 4: 1.0}
     st = torch.zeros(1, dtype=torch.int32, device=device)
     stream = torch.cuda.Stream(device=device)
     torch.cuda.set_stream(stream)

@@ -50,6 +50,8 @@
  *                  complement code q in [-8, 7]; coded symbol q + 8 (A = 16).
  *   ANS_BF16_SPLIT uint16 bf16 bits; coded symbol = exponent byte (A = 256).
  *   ANS_FP8_E4M3   e4m3fn code bytes; coded symbol = the code (A = 256).
+ *   ANS_INT8       int8 code bytes q in [-128, 127]; coded symbol q + 128,
+ *                  i.e. the byte XOR 0x80 (A = 256).
  *   ANS_INT4_PAIRS the same storage as ANS_INT4, coded one symbol per packed
  *                  byte (two consecutive K elements): symbol = byte ^ 0x88,
  *                  i.e. (q_k + 8) | (q_{k+1} + 8) << 4 (A = 256), half as
@@ -98,7 +100,13 @@ typedef enum {
 #define ANS_STATUS_TIMEOUT 0x2u     /* a bounded wait inside a kernel ran out */
 #define ANS_STATUS_BAD_OFFSETS 0x4u /* an offset was unaligned, decreasing or past the end */
 
-typedef enum { ANS_INT4 = 0, ANS_BF16_SPLIT = 1, ANS_FP8_E4M3 = 2, ANS_INT4_PAIRS = 3 } ans_dtype;
+typedef enum {
+  ANS_INT4 = 0,
+  ANS_BF16_SPLIT = 1,
+  ANS_FP8_E4M3 = 2,
+  ANS_INT4_PAIRS = 3,
+  ANS_INT8 = 4
+} ans_dtype;
 
 typedef enum {
   ANS_SCALE_NONE = 0,
@@ -210,13 +218,16 @@ ans_status ans_gemm_workspace(const ans_layout* layout, uint32_t M, ans_scale_ki
  * with X bf16 M x K row-major (16-byte aligned) and w the dequantised weight:
  *   int4: q (NONE), q * s[n] (ROW_BF16 or ROW_F32), q * s[n][k/group_k]
  *         (GROUP_BF16, group_k a multiple of 16 dividing K);
- *   bf16: the bf16 value (NONE);  fp8: e4m3 value (NONE) or value * s[n] (ROW_F32).
+ *   bf16: the bf16 value (NONE);  fp8: e4m3 value (NONE) or value * s[n] (ROW_F32);
+ *   int8: q (NONE) or q * s[n] (ROW_BF16 or ROW_F32).
  * W's tiles are decoded by producer warps straight into shared memory in the
  * tensor-core operand layout and consumed by tcgen05 MMAs; they never reach
  * global memory.  Accumulation is fp32 in a fixed order, so the result is
  * bit-identical to ans_gemm_uncompressed on the same weights.  GROUP_BF16 runs
  * the MMA in f16 (X and q*s are exact in f16 when |X| < 65504 and the scales
- * lie in [2^-14, 2^12]); all other kinds run it in bf16.
+ * lie in [2^-14, 2^12]), and so do fp8 and int8 (their codes are exact in
+ * f16, the row scale is applied to the fp32 accumulator); the other kinds run
+ * it in bf16.
  * M == 0 is a no-op.  d_ws: ans_gemm_workspace bytes, 256-byte aligned; d_X,
  * d_Y and d_scales 16-byte aligned (ANS_ERR_ARG otherwise). */
 ans_status ans_gemm(const uint16_t* d_X, uint32_t M, const ans_tiles* W,

@@ -26,7 +26,7 @@ bool is_int4(uint32_t dtype) { return dtype == ANS_INT4 || dtype == ANS_INT4_PAI
 
 ans_status check_layout(const ans_layout* l) {
   if (!l) return ANS_ERR_ARG;
-  if (l->dtype > ANS_INT4_PAIRS) return ANS_ERR_ARG;
+  if (l->dtype > ANS_INT8) return ANS_ERR_ARG;
   if (l->state_bits != 0 && l->state_bits != 32 && l->state_bits != 64) return ANS_ERR_ARG;
   if (!anshost::layout_valid(l->N, l->K, l->tile_n, l->tile_k)) return ANS_ERR_SHAPE;
   return ANS_OK;
@@ -177,7 +177,7 @@ ans_status ans_layout_check(const ans_layout* layout) { return check_layout(layo
 
 ans_status ans_histogram(const void* d_w, const ans_layout* layout, uint64_t* d_hist,
                          ans_stream_t stream) {
-  if (!layout || layout->dtype > ANS_INT4_PAIRS) return ANS_ERR_ARG;
+  if (!layout || layout->dtype > ANS_INT8) return ANS_ERR_ARG;
   if (layout->N == 0 || layout->K == 0) return ANS_ERR_SHAPE;
   if (is_int4(layout->dtype) && layout->K % 2 != 0) return ANS_ERR_SHAPE;
   if (!d_w || !d_hist || reinterpret_cast<uintptr_t>(d_w) % 16 != 0) return ANS_ERR_ARG;
@@ -193,7 +193,7 @@ ans_status ans_histogram(const void* d_w, const ans_layout* layout, uint64_t* d_
 }
 
 ans_status ans_histogram_host(const void* h_w, const ans_layout* layout, uint64_t* hist) {
-  if (!layout || layout->dtype > ANS_INT4_PAIRS) return ANS_ERR_ARG;
+  if (!layout || layout->dtype > ANS_INT8) return ANS_ERR_ARG;
   if (layout->N == 0 || layout->K == 0) return ANS_ERR_SHAPE;
   if (is_int4(layout->dtype) && layout->K % 2 != 0) return ANS_ERR_SHAPE;
   if (!h_w || !hist) return ANS_ERR_ARG;

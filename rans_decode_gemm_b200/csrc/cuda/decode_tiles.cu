@@ -35,7 +35,8 @@ __device__ __forceinline__ void store_group(void* out, uint64_t idx, const uint3
     for (int k = 0; k < 8; ++k) w |= (((e[k] >> 12) ^ 8u) & 0xFu) << (4 * k);
     *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(out) + idx / 2) = w;
   } else {
-    // one byte per symbol: the e4m3 code, or the packed int4 pair (symbol ^ 0x88)
+    // one byte per symbol: the e4m3 code, the int8 code (symbol ^ 0x80) or the
+    // packed int4 pair (symbol ^ 0x88)
     uint32_t lo = __byte_perm(__byte_perm(e[0] >> 12, e[1] >> 4, 0x0050u),
                               __byte_perm(e[2] >> 12, e[3] >> 4, 0x0050u), 0x5410u);
     uint32_t hi = __byte_perm(__byte_perm(e[4] >> 12, e[5] >> 4, 0x0050u),
@@ -43,6 +44,9 @@ __device__ __forceinline__ void store_group(void* out, uint64_t idx, const uint3
     if (DT == kDtInt4Pairs) {
       lo ^= 0x88888888u;
       hi ^= 0x88888888u;
+    } else if (DT == kDtInt8) {
+      lo ^= 0x80808080u;
+      hi ^= 0x80808080u;
     }
     // idx counts bytes for fp8 and K elements (two per byte) for int4 pairs
     *reinterpret_cast<uint2*>(static_cast<uint8_t*>(out) + (DT == kDtInt4Pairs ? idx / 2 : idx)) =
@@ -172,9 +176,10 @@ __global__ void __launch_bounds__(kHistWarps * 32)
       if (dtype == kDtInt4) {
 #pragma unroll
         for (int n = 0; n < 8; ++n) atomicAdd(&mine[((u >> (4 * n)) & 0xFu) ^ 8u], 1u);
-      } else if (dtype == kDtInt4Pairs) {
+      } else if (dtype == kDtInt4Pairs || dtype == kDtInt8) {
+        const uint32_t flip = dtype == kDtInt8 ? 0x80u : 0x88u;
 #pragma unroll
-        for (int n = 0; n < 4; ++n) atomicAdd(&mine[((u >> (8 * n)) & 0xFFu) ^ 0x88u], 1u);
+        for (int n = 0; n < 4; ++n) atomicAdd(&mine[((u >> (8 * n)) & 0xFFu) ^ flip], 1u);
       } else if (dtype == kDtBf16Split) {
         atomicAdd(&mine[(u >> 7) & 0xFFu], 1u);
         atomicAdd(&mine[(u >> 23) & 0xFFu], 1u);
@@ -191,8 +196,8 @@ __global__ void __launch_bounds__(kHistWarps * 32)
       if (dtype == kDtInt4) {
         atomicAdd(&mine[(w[b] & 0xFu) ^ 8u], 1u);
         atomicAdd(&mine[((w[b] >> 4) & 0xFu) ^ 8u], 1u);
-      } else if (dtype == kDtInt4Pairs) {
-        atomicAdd(&mine[w[b] ^ 0x88u], 1u);
+      } else if (dtype == kDtInt4Pairs || dtype == kDtInt8) {
+        atomicAdd(&mine[w[b] ^ (dtype == kDtInt8 ? 0x80u : 0x88u)], 1u);
       } else if (dtype == kDtBf16Split) {
         uint32_t u = w[b] | (static_cast<uint32_t>(w[b + 1]) << 8);
         atomicAdd(&mine[(u >> 7) & 0xFFu], 1u);
@@ -235,11 +240,13 @@ cudaError_t launch_decode_tiles(const LayerDev& L, void* out, uint32_t* status,
     if (L.dtype == kDtBf16Split) return launch_decode_variant<kDtBf16Split, true>(L, out, status, stream, blocks, warps);
     if (L.dtype == kDtInt4) return launch_decode_variant<kDtInt4, true>(L, out, status, stream, blocks, warps);
     if (L.dtype == kDtInt4Pairs) return launch_decode_variant<kDtInt4Pairs, true>(L, out, status, stream, blocks, warps);
+    if (L.dtype == kDtInt8) return launch_decode_variant<kDtInt8, true>(L, out, status, stream, blocks, warps);
     return launch_decode_variant<kDtFp8, true>(L, out, status, stream, blocks, warps);
   }
   if (L.dtype == kDtBf16Split) return launch_decode_variant<kDtBf16Split, false>(L, out, status, stream, blocks, warps);
   if (L.dtype == kDtInt4) return launch_decode_variant<kDtInt4, false>(L, out, status, stream, blocks, warps);
   if (L.dtype == kDtInt4Pairs) return launch_decode_variant<kDtInt4Pairs, false>(L, out, status, stream, blocks, warps);
+  if (L.dtype == kDtInt8) return launch_decode_variant<kDtInt8, false>(L, out, status, stream, blocks, warps);
   return launch_decode_variant<kDtFp8, false>(L, out, status, stream, blocks, warps);
 }
 

@@ -244,7 +244,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
             const uint64_t idx = row * L.K + k0 + 16 * s + 8 * c;
             if (kFmt == kFmtBf16Split) {
               cp[gg] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(P.w_plain) + idx));
-            } else if (kFmt == kFmtFp8F16) {
+            } else if (kFmt == kFmtFp8F16 || kFmt == kFmtInt8F16) {
               uint2 v = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(P.w_plain) + idx));
               cp[gg] = make_uint4(v.x, v.y, 0, 0);
             } else {
@@ -289,6 +289,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
             else if constexpr (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
             else if constexpr (kFmt == kFmtInt4F16Group)
               fmt_int4_f16_scaled(e, i == 0 ? gs0 : i == 1 ? gs1 : i == 2 ? gs2 : gs3, o);
+            else if constexpr (kFmt == kFmtInt8F16) fmt_int8_f16(e, o);
             else fmt_fp8_f16(e, o);
             if (zero_tile) {
 #pragma unroll
@@ -303,13 +304,15 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
               o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
             } else {
               uint32_t e[8];
-              if (kFmt == kFmtFp8F16) {
+              if (kFmt == kFmtFp8F16 || kFmt == kFmtInt8F16) {
+                  const uint32_t flip = kFmt == kFmtInt8F16 ? 0x80u : 0u;  // int8: symbol = byte ^ 0x80
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                  e[k] = ((v.x >> (8 * k)) & 0xFFu) << 12;
-                  e[k + 4] = ((v.y >> (8 * k)) & 0xFFu) << 12;
+                  e[k] = (((v.x >> (8 * k)) & 0xFFu) ^ flip) << 12;
+                  e[k + 4] = (((v.y >> (8 * k)) & 0xFFu) ^ flip) << 12;
                 }
-                fmt_fp8_f16(e, o);
+                if constexpr (kFmt == kFmtInt8F16) fmt_int8_f16(e, o);
+                else fmt_fp8_f16(e, o);
               } else {
 #pragma unroll
                 for (int k = 0; k < 8; ++k) e[k] = (((v.x >> (4 * k)) & 0xFu) ^ 8u) << 12;
@@ -585,8 +588,9 @@ bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool dec
     // uncompressed weights take the per-element copy path
     p.fmt = decode ? ((scale_kind == 3) ? kFmtInt4PairF16Group : kFmtInt4PairBf16)
                    : ((scale_kind == 3) ? kFmtInt4F16Group : kFmtInt4Bf16);
+  else if (L.dtype == 4) p.fmt = kFmtInt8F16;
   else p.fmt = kFmtFp8F16;
-  p.ab_f16 = (fmt_group(p.fmt) || p.fmt == kFmtFp8F16) ? 1 : 0;
+  p.ab_f16 = (fmt_group(p.fmt) || p.fmt == kFmtFp8F16 || p.fmt == kFmtInt8F16) ? 1 : 0;
   p.M = M;
   p.H = L.tile_n / 128;
   p.C = L.tile_k / 16;
@@ -839,10 +843,14 @@ cudaError_t launch_gemm(const GemmPlan& plan, const LayerDev& L, bool decode, co
     case kFmtFp8F16:
       return P.L.wide ? launch_variant<true, kFmtFp8F16, true>(plan, P, stream)
                       : launch_variant<true, kFmtFp8F16>(plan, P, stream);
+    case kFmtInt8F16:
+      return P.L.wide ? launch_variant<true, kFmtInt8F16, true>(plan, P, stream)
+                      : launch_variant<true, kFmtInt8F16>(plan, P, stream);
     case 8 | kFmtBf16Split: return launch_variant<false, kFmtBf16Split>(plan, P, stream);
     case 8 | kFmtInt4Bf16: return launch_variant<false, kFmtInt4Bf16>(plan, P, stream);
     case 8 | kFmtInt4F16Group: return launch_variant<false, kFmtInt4F16Group>(plan, P, stream);
     case 8 | kFmtFp8F16: return launch_variant<false, kFmtFp8F16>(plan, P, stream);
+    case 8 | kFmtInt8F16: return launch_variant<false, kFmtInt8F16>(plan, P, stream);
   }
   return cudaErrorInvalidValue;
 }

@@ -274,7 +274,7 @@ __device__ __forceinline__ void local_cta(const GemmDev& P) {
                 const uint64_t idx = row * L.K + k0 + 16 * s + 8 * c;
                 if (kFmt == kFmtBf16Split) {
                   cp[gg] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(P.w_plain) + idx));
-                } else if (kFmt == kFmtFp8F16) {
+                } else if (kFmt == kFmtFp8F16 || kFmt == kFmtInt8F16) {
                   uint2 v = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(P.w_plain) + idx));
                   cp[gg] = make_uint4(v.x, v.y, 0, 0);
                 } else {
@@ -340,6 +340,7 @@ __device__ __forceinline__ void local_cta(const GemmDev& P) {
                 else if constexpr (kFmt == kFmtBf16Split) fmt_bf16_split(e, raw8, o);
                 else if constexpr (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
                 else if constexpr (kFmt == kFmtInt4F16Group) fmt_int4_f16_scaled(e, gsc[i], o);
+                else if constexpr (kFmt == kFmtInt8F16) fmt_int8_f16(e, o);
                 else fmt_fp8_f16(e, o);
                 if (kConst && zero_tile) {
 #pragma unroll
@@ -351,13 +352,15 @@ __device__ __forceinline__ void local_cta(const GemmDev& P) {
                   o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
                 } else {
                   uint32_t e[8];
-                  if (kFmt == kFmtFp8F16) {
+                  if (kFmt == kFmtFp8F16 || kFmt == kFmtInt8F16) {
+                  const uint32_t flip = kFmt == kFmtInt8F16 ? 0x80u : 0u;  // int8: symbol = byte ^ 0x80
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                      e[k] = ((v.x >> (8 * k)) & 0xFFu) << 12;
-                      e[k + 4] = ((v.y >> (8 * k)) & 0xFFu) << 12;
+                      e[k] = (((v.x >> (8 * k)) & 0xFFu) ^ flip) << 12;
+                      e[k + 4] = (((v.y >> (8 * k)) & 0xFFu) ^ flip) << 12;
                     }
-                    fmt_fp8_f16(e, o);
+                    if constexpr (kFmt == kFmtInt8F16) fmt_int8_f16(e, o);
+                    else fmt_fp8_f16(e, o);
                   } else {
 #pragma unroll
                     for (int k = 0; k < 8; ++k) e[k] = (((v.x >> (4 * k)) & 0xFu) ^ 8u) << 12;
@@ -665,10 +668,14 @@ cudaError_t launch_gemm_local(const GemmPlan& plan, const GemmDev& P, bool decod
     case kFmtFp8F16:
       return P.L.wide ? launch_local_variant<true, kFmtFp8F16, true>(plan, P, stream)
                       : launch_local_variant<true, kFmtFp8F16>(plan, P, stream);
+    case kFmtInt8F16:
+      return P.L.wide ? launch_local_variant<true, kFmtInt8F16, true>(plan, P, stream)
+                      : launch_local_variant<true, kFmtInt8F16>(plan, P, stream);
     case 8 | kFmtBf16Split: return launch_local_variant<false, kFmtBf16Split>(plan, P, stream);
     case 8 | kFmtInt4Bf16: return launch_local_variant<false, kFmtInt4Bf16>(plan, P, stream);
     case 8 | kFmtInt4F16Group: return launch_local_variant<false, kFmtInt4F16Group>(plan, P, stream);
     case 8 | kFmtFp8F16: return launch_local_variant<false, kFmtFp8F16>(plan, P, stream);
+    case 8 | kFmtInt8F16: return launch_local_variant<false, kFmtInt8F16>(plan, P, stream);
   }
   return cudaErrorInvalidValue;
 }
@@ -713,6 +720,9 @@ cudaError_t launch_gemm_local_batch(const GemmPlan& plan, const BatchDev& B, uin
     case kFmtFp8F16:
       return wide ? launch_local_batch_variant<kFmtFp8F16, true>(plan, B, grid, stream)
                   : launch_local_batch_variant<kFmtFp8F16, false>(plan, B, grid, stream);
+    case kFmtInt8F16:
+      return wide ? launch_local_batch_variant<kFmtInt8F16, true>(plan, B, grid, stream)
+                  : launch_local_batch_variant<kFmtInt8F16, false>(plan, B, grid, stream);
   }
   return cudaErrorInvalidValue;
 }

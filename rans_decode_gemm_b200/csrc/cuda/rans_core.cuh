@@ -49,7 +49,7 @@ constexpr uint32_t kStatusCorrupt = 0x1u;
 constexpr uint32_t kStatusTimeout = 0x2u;
 constexpr uint32_t kStatusBadOffsets = 0x4u;
 
-enum : uint32_t { kDtInt4 = 0, kDtBf16Split = 1, kDtFp8 = 2, kDtInt4Pairs = 3 };
+enum : uint32_t { kDtInt4 = 0, kDtBf16Split = 1, kDtFp8 = 2, kDtInt4Pairs = 3, kDtInt8 = 4 };
 
 
 // Abort-aware bounded wait.  Returns false if the wait ran out (then sets the
@@ -700,6 +700,18 @@ __device__ __forceinline__ void fmt_int4_f16_scaled(const uint32_t (&e)[8], __ha
     v |= 0x64006400u;
     __half2 h = *reinterpret_cast<__half2*>(&v);
     h = __hmul2(__hsub2(h, __floats2half2_rn(1032.0f, 1032.0f)), scale);
+    out[p] = *reinterpret_cast<uint32_t*>(&h);
+  }
+}
+
+// int8 codes (symbol q + 128) as exact f16: f16(1024 + s) has bits
+// 0x6400 | s for s < 1024; subtract 1152.
+__device__ __forceinline__ void fmt_int8_f16(const uint32_t (&e)[8], uint32_t (&out)[4]) {
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    uint32_t v = ((e[2 * p] >> 12) & 0xFFu) | ((e[2 * p + 1] << 4) & 0x00FF0000u) | 0x64006400u;
+    __half2 h = *reinterpret_cast<__half2*>(&v);
+    h = __hsub2(h, __floats2half2_rn(1152.0f, 1152.0f));
     out[p] = *reinterpret_cast<uint32_t*>(&h);
   }
 }

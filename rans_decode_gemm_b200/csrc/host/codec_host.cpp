@@ -101,6 +101,8 @@ bool code_tile(const TileJob& job, uint64_t t, std::vector<uint8_t>& out,
       raw_tile[(j >> 3) * 256 + l * 8 + (j & 7)] =
           static_cast<uint8_t>(((b >> 8) & 0x80) | (b & 0x7F));
     }
+  } else if (job.dtype == kInt8) {
+    for (size_t q = 0; q < S; ++q) sym[q] = static_cast<uint8_t>(job.w[origin + order[q]] ^ 0x80);
   } else {
     for (size_t q = 0; q < S; ++q) sym[q] = job.w[origin + order[q]];
   }
@@ -205,6 +207,9 @@ void histogram(uint32_t dtype, const void* w, uint64_t n_weights, uint64_t* hist
       } else if (dtype == kInt4Pairs) {
         const uint8_t* p = static_cast<const uint8_t*>(w);
         for (uint64_t i = a; i < b; ++i) h[p[i] ^ 0x88]++;
+      } else if (dtype == kInt8) {
+        const uint8_t* p = static_cast<const uint8_t*>(w);
+        for (uint64_t i = a; i < b; ++i) h[p[i] ^ 0x80]++;
       } else if (dtype == kBf16Split) {
         const uint16_t* p = static_cast<const uint16_t*>(w);
         for (uint64_t i = a; i < b; ++i) h[(p[i] >> 7) & 0xFF]++;
