@@ -48,6 +48,10 @@
 // one word is pushed first if x >= 2^40 f_a f_b.  Tile bytes: 32 little-endian
 // u64 final states, then the u32 words in decoder order, then zero padding.
 //
+// fp4 (dtype 5; [SB] s2.1 lists fp4 among the seven formats measured): e2m1
+// codes stored like int4 (two per byte, element k even in the low nibble),
+// symbol = the code (alphabet 16), value e2m1 times an optional per-row scale.
+//
 // int8 (dtype 4; [SB] s2.1 lists int8 among the seven formats measured): one byte per
 // weight, two's complement q in [-128, 127], symbol q + 128, alphabet 256;
 // value q times an optional per-row scale.
@@ -71,7 +75,7 @@
 
 namespace {
 
-enum { DT_INT4 = 0, DT_BF16_SPLIT = 1, DT_FP8_E4M3 = 2, DT_INT4_PAIRS = 3, DT_INT8 = 4 };
+enum { DT_INT4 = 0, DT_BF16_SPLIT = 1, DT_FP8_E4M3 = 2, DT_INT4_PAIRS = 3, DT_INT8 = 4, DT_FP4_E2M1 = 5 };
 enum { SC_NONE = 0, SC_ROW_BF16 = 1, SC_ROW_F32 = 2, SC_GROUP_BF16 = 3 };
 enum {
   OK = 0, ERR_ARG = 1, ERR_SHAPE = 2, ERR_ALPHABET = 3, ERR_BUFFER_TOO_SMALL = 4,
@@ -84,7 +88,9 @@ const uint32_t kWordBits = 16;       // renormalisation word width (b = 2^16)
 const uint64_t kLWide = 1ull << 32;  // wide variant: lower bound of the state interval
 const uint32_t kWideWordBits = 32;   // wide variant: renormalisation word width (b = 2^32)
 
-int alphabet_of(int dtype) { return dtype == DT_INT4 ? 16 : 256; }
+int alphabet_of(int dtype) { return (dtype == DT_INT4 || dtype == DT_FP4_E2M1) ? 16 : 256; }
+// packed two per byte, element k even in the low nibble
+bool is_nibble(int dtype) { return dtype == DT_INT4 || dtype == DT_INT4_PAIRS || dtype == DT_FP4_E2M1; }
 bool is_int4(int dtype) { return dtype == DT_INT4 || dtype == DT_INT4_PAIRS; }
 
 // ---- 1. Symbols: what is treated as "a sequence of discrete symbols" ---------
@@ -113,6 +119,11 @@ uint32_t pair_symbol_at(const void* w, uint64_t idx) {
 uint32_t symbol_at(int dtype, const void* w, uint64_t idx) {
   if (dtype == DT_INT4) return (uint32_t)(int4_code((const uint8_t*)w, idx) + 8);
   if (dtype == DT_INT4_PAIRS) return pair_symbol_at(w, idx);
+  // fp4 e2m1: the 4-bit code itself
+  if (dtype == DT_FP4_E2M1) {
+    const uint8_t byte = ((const uint8_t*)w)[idx / 2];
+    return (idx % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+  }
   // int8: two's complement code q in [-128, 127]; symbol q + 128 (the byte
   // with its top bit flipped)
   if (dtype == DT_INT8) return (uint32_t)((int)(int8_t)((const uint8_t*)w)[idx] + 128);
@@ -346,6 +357,16 @@ double e4m3_value(uint8_t code) {
   return sign ? -v : v;
 }
 
+// fp4 e2m1 value from the format definition: 1 sign, 2 exponent (bias 1),
+// 1 mantissa bit; exponent 0 is subnormal with value m * 0.5; no inf or NaN.
+double e2m1_value(uint8_t code) {
+  int sign = (code >> 3) & 1;
+  int E = (code >> 1) & 3;
+  int m = code & 1;
+  double v = (E == 0) ? 0.5 * m : std::ldexp(1.0 + m / 2.0, E - 1);
+  return sign ? -v : v;
+}
+
 double bf16_value(uint16_t bits) {
   uint32_t u = (uint32_t)bits << 16;
   float f;
@@ -366,6 +387,8 @@ extern "C" {
 int oracle_alphabet_size(int dtype) { return alphabet_of(dtype); }
 
 double oracle_e4m3_value(uint8_t code) { return e4m3_value(code); }
+
+double oracle_e2m1_value(uint8_t code) { return e2m1_value(code); }
 
 // ---- 2. Histogram and Shannon entropy ([SB s2.1], [DF11 实验方法]) -----------
 void oracle_histogram(int dtype, const void* w, uint64_t n_weights, uint64_t* counts) {
@@ -587,7 +610,7 @@ int oracle_encode(int dtype, const void* w, uint32_t N, uint32_t K, uint32_t til
                   uint32_t tile_k, const uint32_t* freq, int prob_bits, uint8_t* stream,
                   uint64_t cap, uint64_t* stream_bytes, uint64_t* offsets, uint8_t* raw,
                   int threads, int state_bits) {
-  if (dtype < 0 || dtype > 4) return ERR_ARG;
+  if (dtype < 0 || dtype > 5) return ERR_ARG;
   if (state_bits != 32 && state_bits != 64) return ERR_ARG;
   if (!layout_ok(N, K, tile_n, tile_k)) return ERR_SHAPE;
   if (state_bits == 64 && prob_bits != 12) return ERR_ARG;  // the pair bound assumes n = 12
@@ -625,7 +648,7 @@ int oracle_decode(int dtype, const uint8_t* stream, uint64_t stream_bytes,
                   uint32_t tile_n, uint32_t tile_k, const uint32_t* freq, int prob_bits,
                   void* w_out, uint64_t tile_begin, uint64_t tile_end, int threads,
                   int state_bits) {
-  if (dtype < 0 || dtype > 4) return ERR_ARG;
+  if (dtype < 0 || dtype > 5) return ERR_ARG;
   if (state_bits != 32 && state_bits != 64) return ERR_ARG;
   if (!layout_ok(N, K, tile_n, tile_k)) return ERR_SHAPE;
   if (state_bits == 64 && prob_bits != 12) return ERR_ARG;
@@ -681,9 +704,9 @@ int oracle_decode(int dtype, const uint8_t* stream, uint64_t stream_bytes,
         if (dtype == DT_INT4_PAIRS) {
           // idx is even: the pair is exactly one packed byte
           ((uint8_t*)w_out)[idx / 2] = (uint8_t)(s ^ 0x88);
-        } else if (dtype == DT_INT4) {
+        } else if (dtype == DT_INT4 || dtype == DT_FP4_E2M1) {
           uint8_t* out = (uint8_t*)w_out;
-          uint8_t nib = (uint8_t)((s - 8) & 0xF);
+          uint8_t nib = (uint8_t)((dtype == DT_INT4 ? s - 8 : s) & 0xF);
           if (idx % 2 == 0) out[idx / 2] = (uint8_t)((out[idx / 2] & 0xF0) | nib);
           else out[idx / 2] = (uint8_t)((out[idx / 2] & 0x0F) | (nib << 4));
         } else if (dtype == DT_INT8) {
@@ -715,11 +738,12 @@ int oracle_decode(int dtype, const uint8_t* stream, uint64_t stream_bytes,
 //   bf16 : the bf16 value (no scale)
 //   fp8  : e4m3_value(code) (SC_NONE) or e4m3_value(code) * s_n (SC_ROW_F32)
 //   int8 : q (SC_NONE) or q * s_n (SC_ROW_F32 or SC_ROW_BF16)
+//   fp4  : e2m1_value(code) (SC_NONE) or e2m1_value(code) * s_n (SC_ROW_F32 or SC_ROW_BF16)
 // Y is M x n_rows row-major doubles.
 int oracle_gemm(int dtype, const uint16_t* X, uint32_t M, uint32_t K, const void* W,
                 uint32_t N, int scale_kind, const void* scales, uint32_t group_k,
                 const uint32_t* rows, uint32_t n_rows, double* Y, int threads) {
-  if (dtype < 0 || dtype > 4) return ERR_ARG;
+  if (dtype < 0 || dtype > 5) return ERR_ARG;
   if (scale_kind == SC_GROUP_BF16 && (group_k == 0 || K % group_k != 0)) return ERR_ARG;
   if (scale_kind != SC_NONE && scales == nullptr) return ERR_ARG;
   if (rows == nullptr) n_rows = N;
@@ -737,6 +761,11 @@ int oracle_gemm(int dtype, const uint16_t* X, uint32_t M, uint32_t K, const void
         else if (scale_kind == SC_GROUP_BF16)
           v *= bf16_value(((const uint16_t*)scales)[n * (K / group_k) + k / group_k]);
         else if (scale_kind == SC_ROW_F32) v *= f32_value(scales, n);
+      } else if (dtype == DT_FP4_E2M1) {
+        const uint8_t byte = ((const uint8_t*)W)[idx / 2];
+        v = e2m1_value((idx % 2 == 0) ? (byte & 0xF) : (byte >> 4));
+        if (scale_kind == SC_ROW_F32) v *= f32_value(scales, n);
+        else if (scale_kind == SC_ROW_BF16) v *= bf16_value(((const uint16_t*)scales)[n]);
       } else if (dtype == DT_INT8) {
         v = (double)(int8_t)((const uint8_t*)W)[idx];
         if (scale_kind == SC_ROW_F32) v *= f32_value(scales, n);

@@ -27,7 +27,7 @@ from dataclasses import dataclass, field
 import numpy as np
 import torch
 
-INT4, BF16_SPLIT, FP8_E4M3, INT4_PAIRS, INT8 = 0, 1, 2, 3, 4
+INT4, BF16_SPLIT, FP8_E4M3, INT4_PAIRS, INT8, FP4_E2M1 = 0, 1, 2, 3, 4, 5
 SCALE_NONE, SCALE_ROW_BF16, SCALE_ROW_F32, SCALE_GROUP_BF16 = 0, 1, 2, 3
 
 
@@ -59,7 +59,12 @@ CONFIGS = {
                        [1, 4, 16, 64, 256, 2048], 4),
     # int8 (absmax per row) of a Llama-8B-shaped MLP projection
     "int8_8b": Config("int8_8b", INT8, 14336, 4096, 128, 64, SCALE_ROW_F32, 0, [1, 16, 128], 5),
+    # fp4 e2m1 (absmax per row, nearest grid value) of the same shape
+    "fp4_8b": Config("fp4_8b", FP4_E2M1, 14336, 4096, 128, 64, SCALE_ROW_F32, 0, [1, 16, 128], 6),
 }
+
+# e2m1 codes 0..7 in increasing value: 0, 0.5, 1, 1.5, 2, 3, 4, 6 (the sign is bit 3)
+_E2M1_GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], np.float32)
 
 
 def to_bf16_bits(a: np.ndarray) -> np.ndarray:
@@ -113,6 +118,19 @@ def make_weights(cfg: Config, matrix: int = 0, N: int | None = None, K: int | No
                 lo, hi = np.searchsorted(outliers, [r0 * K, r1 * K])
                 v[outliers[lo:hi] - r0 * K] *= 20.0
             w[r0 * K:r1 * K] = to_bf16_bits(v)
+    elif cfg.dtype == FP4_E2M1:
+        w = np.empty(N * K // 2, np.uint8)
+        scales = np.empty(N, np.float32)
+        for r0, r1 in _rows_chunks(N, K):
+            v = (rng.standard_normal((r1 - r0, K)) * 0.02).astype(np.float32)
+            s = (np.abs(v).max(axis=1) / 6.0).astype(np.float32)
+            scales[r0:r1] = s
+            a = np.abs(v / s[:, None])
+            mag = np.abs(a[..., None] - _E2M1_GRID).argmin(axis=-1).astype(np.uint8)
+            codes = mag | (np.signbit(v).astype(np.uint8) << 3)
+            codes[mag == 0] = 0                       # +0 for values that round to zero
+            c = codes.reshape(-1)
+            w[r0 * K // 2:r1 * K // 2] = c[0::2] | (c[1::2] << 4)
     elif cfg.dtype == INT8:
         w = np.empty(N * K, np.uint8)
         scales = np.empty(N, np.float32)

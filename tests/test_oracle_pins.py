@@ -581,6 +581,57 @@ def test_gemm_int8_exact_integers(oracle):
     assert np.array_equal(Ys, (xi @ q.T).astype(np.float64) * s.astype(np.float64)[None, :])
 
 
+# ---- fp4 e2m1 ----------------------------------------------------------------------
+# The e2m1 value table of the OCP Microscaling (MX) format specification: codes
+# 0-7 are 0, 0.5, 1, 1.5, 2, 3, 4, 6; bit 3 is the sign.
+E2M1_TABLE = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def test_e2m1_values_match_the_mx_table(oracle):
+    for c in range(16):
+        v = oracle.e2m1_value(c)
+        ref = E2M1_TABLE[c & 7]
+        assert v == (-ref if c & 8 else ref), c
+        assert math.copysign(1.0, v) == (-1.0 if c & 8 else 1.0)   # code 8 is -0
+
+
+def test_fp4_symbol_is_the_code_low_nibble_first(oracle):
+    c = oracle.histogram(WL.FP4_E2M1, np.array([0x21, 0xF7], np.uint8), 4)
+    assert c.size == 16 and list(np.nonzero(c)[0]) == [1, 2, 7, 15] and c.sum() == 4
+
+
+@pytest.mark.parametrize("state_bits,band", [(32, 0.15), (64, 0.25)])
+def test_fp4_encode_decode_identity_and_size(oracle, state_bits, band):
+    cfg, d = _small("fp4_8b", 512, 1024)
+    counts = oracle.histogram(WL.FP4_E2M1, d["w"], 512 * 1024)
+    H = oracle.entropy(counts)
+    _, freq = oracle.normalize(counts)
+    st, stream, offsets, raw = oracle.encode(WL.FP4_E2M1, d["w"], 512, 1024, cfg.tile_n,
+                                             cfg.tile_k, freq, state_bits=state_bits)
+    assert st == 0 and raw is None
+    st, out = oracle.decode(WL.FP4_E2M1, stream, offsets, None, 512, 1024, cfg.tile_n,
+                            cfg.tile_k, freq, state_bits=state_bits)
+    assert st == 0 and np.array_equal(out, d["w"])
+    gap = 8.0 * stream.size / (512 * 1024) - H
+    assert -0.01 < gap < band, gap
+
+
+def test_gemm_fp4_exact(oracle):
+    rng = np.random.default_rng(13)
+    M, N, K = 3, 32, 64
+    codes = rng.integers(0, 16, size=(N, K)).astype(np.uint8)
+    vals = np.array([(-1 if c & 8 else 1) * E2M1_TABLE[c & 7] for c in codes.reshape(-1)]).reshape(N, K)
+    xi = rng.integers(-9, 10, size=(M, K)).astype(np.int64)
+    Xb = WL.to_bf16_bits(xi.astype(np.float32))
+    c = codes.reshape(-1)
+    W = (c[0::2] | (c[1::2] << 4)).astype(np.uint8)
+    Y = oracle.gemm(WL.FP4_E2M1, Xb.reshape(M, K), M, K, W, N)
+    assert np.array_equal(Y, xi @ vals.T)
+    s = np.array([2.0 ** -(n % 3) for n in range(N)], np.float32)
+    Ys = oracle.gemm(WL.FP4_E2M1, Xb, M, K, W, N, WL.SCALE_ROW_F32, s)
+    assert np.array_equal(Ys, (xi @ vals.T) * s.astype(np.float64)[None, :])
+
+
 # ---- fp64 GEMM ------------------------------------------------------------------
 def test_gemm_int4_exact_integers(oracle):
     rng = np.random.default_rng(2)
