@@ -420,6 +420,13 @@ def dequant_bf16(torch, cfg, d, device):
         if s.dim() == 1:
             return (q * s[:, None]).to(torch.bfloat16)
         return (q * s.repeat_interleave(K // s.shape[1], dim=1)).to(torch.bfloat16)
+    if cfg.dtype == 5:  # e2m1 codes (packed like int4), fp32 row scales
+        b = torch.from_numpy(d["w"]).to(device)
+        c = torch.stack([b & 0xF, b >> 4], dim=1).view(N, K).long()
+        grid = torch.tensor([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], device=device)
+        v = grid[c & 7] * torch.where((c & 8) != 0, -1.0, 1.0)
+        s = torch.from_numpy(d["scales"]).to(device)
+        return (v * s[:, None]).to(torch.bfloat16)
     if cfg.dtype == 4:  # int8 codes, fp32 row scales
         q = torch.from_numpy(d["w"].view(np.int8)).to(device).view(N, K).float()
         s = torch.from_numpy(d["scales"]).to(device)
@@ -442,7 +449,7 @@ def sweep(args):
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
     peaks, peaks_src = load_peaks()
-    nominal = {0: 0.5, 1: 2.0, 2: 1.0, 4: 1.0}
+    nominal = {0: 0.5, 1: 2.0, 2: 1.0, 4: 1.0, 5: 0.5}
     st = torch.zeros(1, dtype=torch.int32, device=device)
     stream = torch.cuda.Stream(device=device)
     torch.cuda.set_stream(stream)
@@ -501,7 +508,7 @@ def sweep(args):
             Wb = dequant_bf16(torch, cfg, d, device)
             wcopies = max(1, min(copies, int(-(-256e6 // (N * K * 2)))))
             Wbs = [Wb] + [Wb.clone() for _ in range(wcopies - 1)]
-            dec = torch.empty(N * K * (2 if cfg.dtype == 1 else 1) // (2 if cfg.dtype == 0 else 1),
+            dec = torch.empty(N * K * (2 if cfg.dtype == 1 else 1) // (2 if cfg.dtype in (0, 5) else 1),
                               dtype=torch.uint8, device=device)
             rep_for = lambda us_est: max(3, min(200, int(20000 / max(us_est, 1.0))))
             t_dec = timed_graph([lambda l=l: ans.ans_decode_tiles(l.tiles, dec, st) for l in layers], 3)

@@ -50,6 +50,8 @@
  *                  complement code q in [-8, 7]; coded symbol q + 8 (A = 16).
  *   ANS_BF16_SPLIT uint16 bf16 bits; coded symbol = exponent byte (A = 256).
  *   ANS_FP8_E4M3   e4m3fn code bytes; coded symbol = the code (A = 256).
+ *   ANS_FP4_E2M1   e2m1 codes packed like ANS_INT4 (element k even in the low
+ *                  nibble); coded symbol = the code (A = 16).
  *   ANS_INT8       int8 code bytes q in [-128, 127]; coded symbol q + 128,
  *                  i.e. the byte XOR 0x80 (A = 256).
  *   ANS_INT4_PAIRS the same storage as ANS_INT4, coded one symbol per packed
@@ -105,7 +107,8 @@ typedef enum {
   ANS_BF16_SPLIT = 1,
   ANS_FP8_E4M3 = 2,
   ANS_INT4_PAIRS = 3,
-  ANS_INT8 = 4
+  ANS_INT8 = 4,
+  ANS_FP4_E2M1 = 5
 } ans_dtype;
 
 typedef enum {
@@ -119,7 +122,7 @@ typedef enum {
  * freq[s] > 0 exactly for the symbols present in the layer; the freq sum to
  * 2^prob_bits; cdf[s] = sum of freq[t] for t < s, cdf[alphabet] = 2^prob_bits. */
 typedef struct {
-  uint32_t alphabet;  /* 16 (ANS_INT4) or 256 */
+  uint32_t alphabet;  /* 16 (ANS_INT4, ANS_FP4_E2M1) or 256 */
   uint32_t prob_bits; /* 12 for the stream format; 1..15 accepted by ans_build_codebook */
   uint16_t freq[256];
   uint16_t cdf[257];
@@ -219,7 +222,8 @@ ans_status ans_gemm_workspace(const ans_layout* layout, uint32_t M, ans_scale_ki
  *   int4: q (NONE), q * s[n] (ROW_BF16 or ROW_F32), q * s[n][k/group_k]
  *         (GROUP_BF16, group_k a multiple of 16 dividing K);
  *   bf16: the bf16 value (NONE);  fp8: e4m3 value (NONE) or value * s[n] (ROW_F32);
- *   int8: q (NONE) or q * s[n] (ROW_BF16 or ROW_F32).
+ *   int8: q (NONE) or q * s[n] (ROW_BF16 or ROW_F32);
+ *   fp4: e2m1 value (NONE) or value * s[n] (ROW_BF16 or ROW_F32).
  * W's tiles are decoded by producer warps straight into shared memory in the
  * tensor-core operand layout and consumed by tcgen05 MMAs; they never reach
  * global memory.  Accumulation is fp32 in a fixed order, so the result is

@@ -20,13 +20,15 @@ ans_status cuda_fail(cudaError_t e, const char* where) {
   return ANS_ERR_CUDA;
 }
 
-uint32_t alphabet_of(uint32_t dtype) { return dtype == ANS_INT4 ? 16u : 256u; }
+uint32_t alphabet_of(uint32_t dtype) { return (dtype == ANS_INT4 || dtype == ANS_FP4_E2M1) ? 16u : 256u; }
 // packed-nibble storage (per-element or pair symbols)
 bool is_int4(uint32_t dtype) { return dtype == ANS_INT4 || dtype == ANS_INT4_PAIRS; }
+// two weights per byte
+bool is_nibble(uint32_t dtype) { return is_int4(dtype) || dtype == ANS_FP4_E2M1; }
 
 ans_status check_layout(const ans_layout* l) {
   if (!l) return ANS_ERR_ARG;
-  if (l->dtype > ANS_INT8) return ANS_ERR_ARG;
+  if (l->dtype > ANS_FP4_E2M1) return ANS_ERR_ARG;
   if (l->state_bits != 0 && l->state_bits != 32 && l->state_bits != 64) return ANS_ERR_ARG;
   if (!anshost::layout_valid(l->N, l->K, l->tile_n, l->tile_k)) return ANS_ERR_SHAPE;
   return ANS_OK;
@@ -177,15 +179,15 @@ ans_status ans_layout_check(const ans_layout* layout) { return check_layout(layo
 
 ans_status ans_histogram(const void* d_w, const ans_layout* layout, uint64_t* d_hist,
                          ans_stream_t stream) {
-  if (!layout || layout->dtype > ANS_INT8) return ANS_ERR_ARG;
+  if (!layout || layout->dtype > ANS_FP4_E2M1) return ANS_ERR_ARG;
   if (layout->N == 0 || layout->K == 0) return ANS_ERR_SHAPE;
-  if (is_int4(layout->dtype) && layout->K % 2 != 0) return ANS_ERR_SHAPE;
+  if (is_nibble(layout->dtype) && layout->K % 2 != 0) return ANS_ERR_SHAPE;
   if (!d_w || !d_hist || reinterpret_cast<uintptr_t>(d_w) % 16 != 0) return ANS_ERR_ARG;
   int sms = 0;
   ans_status st = device_info(&sms);
   if (st != ANS_OK) return st;
   const uint64_t n = static_cast<uint64_t>(layout->N) * layout->K;
-  const uint64_t bytes = is_int4(layout->dtype) ? n / 2 : (layout->dtype == ANS_BF16_SPLIT ? 2 * n : n);
+  const uint64_t bytes = is_nibble(layout->dtype) ? n / 2 : (layout->dtype == ANS_BF16_SPLIT ? 2 * n : n);
   cudaError_t e = ansdev::launch_histogram(d_w, bytes, layout->dtype, d_hist,
                                            reinterpret_cast<cudaStream_t>(stream), sms);
   if (e != cudaSuccess) return cuda_fail(e, "ans_histogram");
@@ -193,9 +195,9 @@ ans_status ans_histogram(const void* d_w, const ans_layout* layout, uint64_t* d_
 }
 
 ans_status ans_histogram_host(const void* h_w, const ans_layout* layout, uint64_t* hist) {
-  if (!layout || layout->dtype > ANS_INT8) return ANS_ERR_ARG;
+  if (!layout || layout->dtype > ANS_FP4_E2M1) return ANS_ERR_ARG;
   if (layout->N == 0 || layout->K == 0) return ANS_ERR_SHAPE;
-  if (is_int4(layout->dtype) && layout->K % 2 != 0) return ANS_ERR_SHAPE;
+  if (is_nibble(layout->dtype) && layout->K % 2 != 0) return ANS_ERR_SHAPE;
   if (!h_w || !hist) return ANS_ERR_ARG;
   anshost::histogram(layout->dtype, h_w, static_cast<uint64_t>(layout->N) * layout->K, hist);
   return ANS_OK;

@@ -29,10 +29,10 @@ __device__ __forceinline__ void store_group(void* out, uint64_t idx, const uint3
     uint32_t o[4];
     fmt_bf16_split(e, raw8, o);
     *reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + idx) = make_uint4(o[0], o[1], o[2], o[3]);
-  } else if (DT == kDtInt4) {
+  } else if (DT == kDtInt4 || DT == kDtFp4) {
     uint32_t w = 0;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) w |= (((e[k] >> 12) ^ 8u) & 0xFu) << (4 * k);
+    for (int k = 0; k < 8; ++k) w |= (((e[k] >> 12) ^ (DT == kDtInt4 ? 8u : 0u)) & 0xFu) << (4 * k);
     *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(out) + idx / 2) = w;
   } else {
     // one byte per symbol: the e4m3 code, the int8 code (symbol ^ 0x80) or the
@@ -173,9 +173,10 @@ __global__ void __launch_bounds__(kHistWarps * 32)
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       uint32_t u = words[k];
-      if (dtype == kDtInt4) {
+      if (dtype == kDtInt4 || dtype == kDtFp4) {
+        const uint32_t flip = dtype == kDtInt4 ? 8u : 0u;
 #pragma unroll
-        for (int n = 0; n < 8; ++n) atomicAdd(&mine[((u >> (4 * n)) & 0xFu) ^ 8u], 1u);
+        for (int n = 0; n < 8; ++n) atomicAdd(&mine[((u >> (4 * n)) & 0xFu) ^ flip], 1u);
       } else if (dtype == kDtInt4Pairs || dtype == kDtInt8) {
         const uint32_t flip = dtype == kDtInt8 ? 0x80u : 0x88u;
 #pragma unroll
@@ -193,9 +194,10 @@ __global__ void __launch_bounds__(kHistWarps * 32)
   if (blockIdx.x == 0) {
     for (uint64_t b = n16 * 16 + threadIdx.x * (dtype == kDtBf16Split ? 2 : 1); b < n_bytes;
          b += blockDim.x * (dtype == kDtBf16Split ? 2 : 1)) {
-      if (dtype == kDtInt4) {
-        atomicAdd(&mine[(w[b] & 0xFu) ^ 8u], 1u);
-        atomicAdd(&mine[((w[b] >> 4) & 0xFu) ^ 8u], 1u);
+      if (dtype == kDtInt4 || dtype == kDtFp4) {
+        const uint32_t flip = dtype == kDtInt4 ? 8u : 0u;
+        atomicAdd(&mine[(w[b] & 0xFu) ^ flip], 1u);
+        atomicAdd(&mine[((w[b] >> 4) & 0xFu) ^ flip], 1u);
       } else if (dtype == kDtInt4Pairs || dtype == kDtInt8) {
         atomicAdd(&mine[w[b] ^ (dtype == kDtInt8 ? 0x80u : 0x88u)], 1u);
       } else if (dtype == kDtBf16Split) {
@@ -207,7 +209,7 @@ __global__ void __launch_bounds__(kHistWarps * 32)
     }
   }
   __syncthreads();
-  const uint32_t A = dtype == kDtInt4 ? 16 : 256;
+  const uint32_t A = (dtype == kDtInt4 || dtype == kDtFp4) ? 16 : 256;
   for (uint32_t s = threadIdx.x; s < A; s += blockDim.x) {
     uint64_t sum = 0;
     for (uint32_t k = 0; k < kHistWarps; ++k) sum += h[k][s];
@@ -241,18 +243,20 @@ cudaError_t launch_decode_tiles(const LayerDev& L, void* out, uint32_t* status,
     if (L.dtype == kDtInt4) return launch_decode_variant<kDtInt4, true>(L, out, status, stream, blocks, warps);
     if (L.dtype == kDtInt4Pairs) return launch_decode_variant<kDtInt4Pairs, true>(L, out, status, stream, blocks, warps);
     if (L.dtype == kDtInt8) return launch_decode_variant<kDtInt8, true>(L, out, status, stream, blocks, warps);
+    if (L.dtype == kDtFp4) return launch_decode_variant<kDtFp4, true>(L, out, status, stream, blocks, warps);
     return launch_decode_variant<kDtFp8, true>(L, out, status, stream, blocks, warps);
   }
   if (L.dtype == kDtBf16Split) return launch_decode_variant<kDtBf16Split, false>(L, out, status, stream, blocks, warps);
   if (L.dtype == kDtInt4) return launch_decode_variant<kDtInt4, false>(L, out, status, stream, blocks, warps);
   if (L.dtype == kDtInt4Pairs) return launch_decode_variant<kDtInt4Pairs, false>(L, out, status, stream, blocks, warps);
   if (L.dtype == kDtInt8) return launch_decode_variant<kDtInt8, false>(L, out, status, stream, blocks, warps);
+  if (L.dtype == kDtFp4) return launch_decode_variant<kDtFp4, false>(L, out, status, stream, blocks, warps);
   return launch_decode_variant<kDtFp8, false>(L, out, status, stream, blocks, warps);
 }
 
 cudaError_t launch_histogram(const void* w, uint64_t n_bytes, uint32_t dtype, uint64_t* hist,
                              cudaStream_t stream, int num_sms) {
-  uint32_t A = dtype == kDtInt4 ? 16 : 256;
+  uint32_t A = (dtype == kDtInt4 || dtype == kDtFp4) ? 16 : 256;
   cudaError_t e = cudaMemsetAsync(hist, 0, A * sizeof(uint64_t), stream);
   if (e != cudaSuccess) return e;
   uint64_t n16 = n_bytes / 16;

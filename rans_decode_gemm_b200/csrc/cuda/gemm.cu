@@ -290,6 +290,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
             else if constexpr (kFmt == kFmtInt4F16Group)
               fmt_int4_f16_scaled(e, i == 0 ? gs0 : i == 1 ? gs1 : i == 2 ? gs2 : gs3, o);
             else if constexpr (kFmt == kFmtInt8F16) fmt_int8_f16(e, o);
+            else if constexpr (kFmt == kFmtFp4Bf16) fmt_fp4_bf16(e, o);
             else fmt_fp8_f16(e, o);
             if (zero_tile) {
 #pragma unroll
@@ -315,8 +316,9 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
                 else fmt_fp8_f16(e, o);
               } else {
 #pragma unroll
-                for (int k = 0; k < 8; ++k) e[k] = (((v.x >> (4 * k)) & 0xFu) ^ 8u) << 12;
-                if (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
+                for (int k = 0; k < 8; ++k) e[k] = (((v.x >> (4 * k)) & 0xFu) ^ (kFmt == kFmtFp4Bf16 ? 0u : 8u)) << 12;
+                if (kFmt == kFmtFp4Bf16) fmt_fp4_bf16(e, o);
+                else if (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
                 else fmt_int4_f16_scaled(e, i == 0 ? gs0 : i == 1 ? gs1 : i == 2 ? gs2 : gs3, o);
               }
             }
@@ -589,6 +591,7 @@ bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool dec
     p.fmt = decode ? ((scale_kind == 3) ? kFmtInt4PairF16Group : kFmtInt4PairBf16)
                    : ((scale_kind == 3) ? kFmtInt4F16Group : kFmtInt4Bf16);
   else if (L.dtype == 4) p.fmt = kFmtInt8F16;
+  else if (L.dtype == 5) p.fmt = kFmtFp4Bf16;
   else p.fmt = kFmtFp8F16;
   p.ab_f16 = (fmt_group(p.fmt) || p.fmt == kFmtFp8F16 || p.fmt == kFmtInt8F16) ? 1 : 0;
   p.M = M;
@@ -846,11 +849,15 @@ cudaError_t launch_gemm(const GemmPlan& plan, const LayerDev& L, bool decode, co
     case kFmtInt8F16:
       return P.L.wide ? launch_variant<true, kFmtInt8F16, true>(plan, P, stream)
                       : launch_variant<true, kFmtInt8F16>(plan, P, stream);
+    case kFmtFp4Bf16:
+      return P.L.wide ? launch_variant<true, kFmtFp4Bf16, true>(plan, P, stream)
+                      : launch_variant<true, kFmtFp4Bf16>(plan, P, stream);
     case 8 | kFmtBf16Split: return launch_variant<false, kFmtBf16Split>(plan, P, stream);
     case 8 | kFmtInt4Bf16: return launch_variant<false, kFmtInt4Bf16>(plan, P, stream);
     case 8 | kFmtInt4F16Group: return launch_variant<false, kFmtInt4F16Group>(plan, P, stream);
     case 8 | kFmtFp8F16: return launch_variant<false, kFmtFp8F16>(plan, P, stream);
     case 8 | kFmtInt8F16: return launch_variant<false, kFmtInt8F16>(plan, P, stream);
+    case 8 | kFmtFp4Bf16: return launch_variant<false, kFmtFp4Bf16>(plan, P, stream);
   }
   return cudaErrorInvalidValue;
 }

@@ -341,6 +341,7 @@ __device__ __forceinline__ void local_cta(const GemmDev& P) {
                 else if constexpr (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
                 else if constexpr (kFmt == kFmtInt4F16Group) fmt_int4_f16_scaled(e, gsc[i], o);
                 else if constexpr (kFmt == kFmtInt8F16) fmt_int8_f16(e, o);
+                else if constexpr (kFmt == kFmtFp4Bf16) fmt_fp4_bf16(e, o);
                 else fmt_fp8_f16(e, o);
                 if (kConst && zero_tile) {
 #pragma unroll
@@ -363,8 +364,9 @@ __device__ __forceinline__ void local_cta(const GemmDev& P) {
                     else fmt_fp8_f16(e, o);
                   } else {
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) e[k] = (((v.x >> (4 * k)) & 0xFu) ^ 8u) << 12;
-                    if (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
+                    for (int k = 0; k < 8; ++k) e[k] = (((v.x >> (4 * k)) & 0xFu) ^ (kFmt == kFmtFp4Bf16 ? 0u : 8u)) << 12;
+                    if (kFmt == kFmtFp4Bf16) fmt_fp4_bf16(e, o);
+                    else if (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
                     else fmt_int4_f16_scaled(e, gsc[i], o);
                   }
                 }
@@ -671,11 +673,15 @@ cudaError_t launch_gemm_local(const GemmPlan& plan, const GemmDev& P, bool decod
     case kFmtInt8F16:
       return P.L.wide ? launch_local_variant<true, kFmtInt8F16, true>(plan, P, stream)
                       : launch_local_variant<true, kFmtInt8F16>(plan, P, stream);
+    case kFmtFp4Bf16:
+      return P.L.wide ? launch_local_variant<true, kFmtFp4Bf16, true>(plan, P, stream)
+                      : launch_local_variant<true, kFmtFp4Bf16>(plan, P, stream);
     case 8 | kFmtBf16Split: return launch_local_variant<false, kFmtBf16Split>(plan, P, stream);
     case 8 | kFmtInt4Bf16: return launch_local_variant<false, kFmtInt4Bf16>(plan, P, stream);
     case 8 | kFmtInt4F16Group: return launch_local_variant<false, kFmtInt4F16Group>(plan, P, stream);
     case 8 | kFmtFp8F16: return launch_local_variant<false, kFmtFp8F16>(plan, P, stream);
     case 8 | kFmtInt8F16: return launch_local_variant<false, kFmtInt8F16>(plan, P, stream);
+    case 8 | kFmtFp4Bf16: return launch_local_variant<false, kFmtFp4Bf16>(plan, P, stream);
   }
   return cudaErrorInvalidValue;
 }
@@ -723,6 +729,9 @@ cudaError_t launch_gemm_local_batch(const GemmPlan& plan, const BatchDev& B, uin
     case kFmtInt8F16:
       return wide ? launch_local_batch_variant<kFmtInt8F16, true>(plan, B, grid, stream)
                   : launch_local_batch_variant<kFmtInt8F16, false>(plan, B, grid, stream);
+    case kFmtFp4Bf16:
+      return wide ? launch_local_batch_variant<kFmtFp4Bf16, true>(plan, B, grid, stream)
+                  : launch_local_batch_variant<kFmtFp4Bf16, false>(plan, B, grid, stream);
   }
   return cudaErrorInvalidValue;
 }

@@ -33,7 +33,8 @@ enum : uint32_t {
   kFmtFp8F16 = 3,      // e4m3 code -> exact f16 (row scale applied in the epilogue)
   kFmtInt4PairBf16 = 4,     // int4 pair symbol -> two exact bf16 (row scale in the epilogue)
   kFmtInt4PairF16Group = 5, // int4 pair symbol * group scale -> two exact f16
-  kFmtInt8F16 = 6           // int8 code -> exact f16 (row scale applied in the epilogue)
+  kFmtInt8F16 = 6,          // int8 code -> exact f16 (row scale applied in the epilogue)
+  kFmtFp4Bf16 = 7           // e2m1 code -> exact bf16 (row scale applied in the epilogue)
 };
 // int4 pair symbols: 8 symbols of a lane fill 16 columns of one slab row
 __host__ __device__ constexpr bool fmt_pair(uint32_t f) { return f == kFmtInt4PairBf16 || f == kFmtInt4PairF16Group; }

@@ -85,11 +85,12 @@ bool code_tile(const TileJob& job, uint64_t t, std::vector<uint8_t>& out,
   sym.resize(S);
   if (job.dtype == kInt4Pairs) {
     for (size_t q = 0; q < S; ++q) sym[q] = static_cast<uint8_t>(job.w[(origin + order[q]) >> 1] ^ 0x88);
-  } else if (job.dtype == kInt4) {
+  } else if (job.dtype == kInt4 || job.dtype == kFp4) {
+    const uint8_t flip = job.dtype == kInt4 ? 8 : 0;  // int4: q + 8; fp4: the code
     for (size_t q = 0; q < S; ++q) {
       const uint64_t e = origin + order[q];
       const uint8_t b = job.w[e >> 1];
-      sym[q] = static_cast<uint8_t>(((e & 1) ? (b >> 4) : (b & 15)) ^ 8);
+      sym[q] = static_cast<uint8_t>(((e & 1) ? (b >> 4) : (b & 15)) ^ flip);
     }
   } else if (job.dtype == kBf16Split) {
     const uint16_t* w16 = reinterpret_cast<const uint16_t*>(job.w);
@@ -192,8 +193,9 @@ bool layout_valid(uint32_t N, uint32_t K, uint32_t tile_n, uint32_t tile_k) {
 }
 
 void histogram(uint32_t dtype, const void* w, uint64_t n_weights, uint64_t* hist) {
-  const uint32_t A = dtype == kInt4 ? 16 : 256;
-  const uint64_t units = (dtype == kInt4 || dtype == kInt4Pairs) ? n_weights / 2 : n_weights;  // bytes or u16 words
+  const uint32_t A = (dtype == kInt4 || dtype == kFp4) ? 16 : 256;
+  const uint64_t units = (dtype == kInt4 || dtype == kInt4Pairs || dtype == kFp4)
+                             ? n_weights / 2 : n_weights;  // bytes or u16 words
   const unsigned nw = worker_count(units / 65536 + 1);
   std::vector<std::vector<uint64_t>> part(nw, std::vector<uint64_t>(256, 0));
   std::vector<std::thread> pool;
@@ -201,9 +203,10 @@ void histogram(uint32_t dtype, const void* w, uint64_t n_weights, uint64_t* hist
     pool.emplace_back([&, k]() {
       const uint64_t a = units * k / nw, b = units * (k + 1) / nw;
       uint64_t* h = part[k].data();
-      if (dtype == kInt4) {
+      if (dtype == kInt4 || dtype == kFp4) {
         const uint8_t* p = static_cast<const uint8_t*>(w);
-        for (uint64_t i = a; i < b; ++i) { h[(p[i] & 15) ^ 8]++; h[(p[i] >> 4) ^ 8]++; }
+        const uint8_t flip = dtype == kInt4 ? 8 : 0;
+        for (uint64_t i = a; i < b; ++i) { h[(p[i] & 15) ^ flip]++; h[(p[i] >> 4) ^ flip]++; }
       } else if (dtype == kInt4Pairs) {
         const uint8_t* p = static_cast<const uint8_t*>(w);
         for (uint64_t i = a; i < b; ++i) h[p[i] ^ 0x88]++;
@@ -324,7 +327,7 @@ int encode(uint32_t dtype, const void* w, uint32_t N, uint32_t K, uint32_t tile_
   job.tile_k = tile_k;
   job.n_kt = n_kt;
   job.order = &order;
-  const uint32_t A = dtype == kInt4 ? 16 : 256;
+  const uint32_t A = (dtype == kInt4 || dtype == kFp4) ? 16 : 256;
   uint32_t run = 0;
   for (uint32_t s = 0; s < 256; ++s) {
     job.freq[s] = s < A ? freq[s] : 0;

@@ -38,7 +38,8 @@ def test_status_strings_and_layout_checks(ans_lib):
     assert ans.ans_layout_check(ans.make_layout(0, 512, 520, 128, 40)) == 2    # tile_k % 16
     assert ans.ans_layout_check(ans.make_layout(0, 512, 512, 64, 32)) == 2     # tile_n
     assert ans.ans_layout_check(ans.make_layout(7, 512, 512, 128, 32)) == 1    # dtype
-    assert ans.ans_layout_check(ans.make_layout(5, 512, 512, 128, 32)) == 1    # dtype
+    assert ans.ans_layout_check(ans.make_layout(6, 512, 512, 128, 32)) == 1    # dtype
+    assert ans.ans_layout_check(ans.make_layout(5, 512, 512, 128, 32)) == 0    # fp4
     assert ans.ans_layout_check(ans.make_layout(4, 512, 512, 128, 32)) == 0    # int8
     assert ans.ans_layout_check(ans.make_layout(3, 512, 512, 128, 32)) == 0    # int4 pairs
     assert ans.ans_layout_check(ans.make_layout(1, 0, 512, 128, 32)) == 2      # empty
@@ -49,7 +50,8 @@ def test_status_strings_and_layout_checks(ans_lib):
 
 
 CASES = [("tiny_int4", 512, 512), ("bf16_4096", 512, 512), ("llama8b_mlp", 256, 1024),
-         ("int4_70b", 512, 512), ("fp8_405b", 256, 1024), ("int8_8b", 256, 1024)]
+         ("int4_70b", 512, 512), ("fp8_405b", 256, 1024), ("int8_8b", 256, 1024),
+         ("fp4_8b", 256, 1024)]
 
 
 @pytest.mark.parametrize("pairs", [False, True])
