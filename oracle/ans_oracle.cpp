@@ -52,6 +52,9 @@
 // codes stored like int4 (two per byte, element k even in the low nibble),
 // symbol = the code (alphabet 16), value e2m1 times an optional per-row scale.
 //
+// fp4 pairs (dtype 6): fp4 codes coded one symbol per packed byte, the byte
+// itself (alphabet 256), in the int4 pairs' lane map.
+//
 // int8 (dtype 4; [SB] s2.1 lists int8 among the seven formats measured): one byte per
 // weight, two's complement q in [-128, 127], symbol q + 128, alphabet 256;
 // value q times an optional per-row scale.
@@ -75,7 +78,15 @@
 
 namespace {
 
-enum { DT_INT4 = 0, DT_BF16_SPLIT = 1, DT_FP8_E4M3 = 2, DT_INT4_PAIRS = 3, DT_INT8 = 4, DT_FP4_E2M1 = 5 };
+enum {
+  DT_INT4 = 0,
+  DT_BF16_SPLIT = 1,
+  DT_FP8_E4M3 = 2,
+  DT_INT4_PAIRS = 3,
+  DT_INT8 = 4,
+  DT_FP4_E2M1 = 5,
+  DT_FP4_PAIRS = 6
+};
 enum { SC_NONE = 0, SC_ROW_BF16 = 1, SC_ROW_F32 = 2, SC_GROUP_BF16 = 3 };
 enum {
   OK = 0, ERR_ARG = 1, ERR_SHAPE = 2, ERR_ALPHABET = 3, ERR_BUFFER_TOO_SMALL = 4,
@@ -90,7 +101,12 @@ const uint32_t kWideWordBits = 32;   // wide variant: renormalisation word width
 
 int alphabet_of(int dtype) { return (dtype == DT_INT4 || dtype == DT_FP4_E2M1) ? 16 : 256; }
 // packed two per byte, element k even in the low nibble
-bool is_nibble(int dtype) { return dtype == DT_INT4 || dtype == DT_INT4_PAIRS || dtype == DT_FP4_E2M1; }
+bool is_nibble(int dtype) {
+  return dtype == DT_INT4 || dtype == DT_INT4_PAIRS || dtype == DT_FP4_E2M1 || dtype == DT_FP4_PAIRS;
+}
+// one symbol per packed byte (two consecutive K elements)
+bool is_pairs(int dtype) { return dtype == DT_INT4_PAIRS || dtype == DT_FP4_PAIRS; }
+bool is_fp4(int dtype) { return dtype == DT_FP4_E2M1 || dtype == DT_FP4_PAIRS; }
 bool is_int4(int dtype) { return dtype == DT_INT4 || dtype == DT_INT4_PAIRS; }
 
 // ---- 1. Symbols: what is treated as "a sequence of discrete symbols" ---------
@@ -119,6 +135,8 @@ uint32_t pair_symbol_at(const void* w, uint64_t idx) {
 uint32_t symbol_at(int dtype, const void* w, uint64_t idx) {
   if (dtype == DT_INT4) return (uint32_t)(int4_code((const uint8_t*)w, idx) + 8);
   if (dtype == DT_INT4_PAIRS) return pair_symbol_at(w, idx);
+  // fp4 pairs: the packed byte itself (low nibble: the even element's code)
+  if (dtype == DT_FP4_PAIRS) return ((const uint8_t*)w)[idx / 2];
   // fp4 e2m1: the 4-bit code itself
   if (dtype == DT_FP4_E2M1) {
     const uint8_t byte = ((const uint8_t*)w)[idx / 2];
@@ -255,7 +273,7 @@ struct Layout {
   uint32_t N, K, tile_n, tile_k;
   int state_bits;  // 32, or 64 for the wide-state variant
   uint64_t n_tiles() const { return (uint64_t)(N / tile_n) * (K / tile_k); }
-  uint64_t tile_symbols() const { return (uint64_t)tile_n * tile_k / (dtype == DT_INT4_PAIRS ? 2 : 1); }
+  uint64_t tile_symbols() const { return (uint64_t)tile_n * tile_k / (is_pairs(dtype) ? 2 : 1); }
   uint64_t tile_weights() const { return (uint64_t)tile_n * tile_k; }
 };
 
@@ -270,7 +288,7 @@ int encode_tile(const Layout& lay, const void* w, const Codebook& cb, uint64_t t
   const bool wide = lay.state_bits == 64;
   auto sym_of = [&](uint32_t l, uint32_t j) {
     uint32_t row, col;
-    if (lay.dtype == DT_INT4_PAIRS) lane_map_pairs(lay.tile_n, l, j, &row, &col);
+    if (is_pairs(lay.dtype)) lane_map_pairs(lay.tile_n, l, j, &row, &col);
     else lane_map(lay.tile_n, l, j, &row, &col);
     return symbol_at(lay.dtype, w, (n0 + row) * lay.K + (k0 + col));
   };
@@ -394,7 +412,7 @@ double oracle_e2m1_value(uint8_t code) { return e2m1_value(code); }
 void oracle_histogram(int dtype, const void* w, uint64_t n_weights, uint64_t* counts) {
   int A = alphabet_of(dtype);
   for (int s = 0; s < A; ++s) counts[s] = 0;
-  const uint64_t step = dtype == DT_INT4_PAIRS ? 2 : 1;  // one pair symbol per 2 weights
+  const uint64_t step = is_pairs(dtype) ? 2 : 1;  // one pair symbol per 2 weights
   for (uint64_t i = 0; i + step <= n_weights; i += step) counts[symbol_at(dtype, w, i)]++;
 }
 
@@ -610,7 +628,7 @@ int oracle_encode(int dtype, const void* w, uint32_t N, uint32_t K, uint32_t til
                   uint32_t tile_k, const uint32_t* freq, int prob_bits, uint8_t* stream,
                   uint64_t cap, uint64_t* stream_bytes, uint64_t* offsets, uint8_t* raw,
                   int threads, int state_bits) {
-  if (dtype < 0 || dtype > 5) return ERR_ARG;
+  if (dtype < 0 || dtype > 6) return ERR_ARG;
   if (state_bits != 32 && state_bits != 64) return ERR_ARG;
   if (!layout_ok(N, K, tile_n, tile_k)) return ERR_SHAPE;
   if (state_bits == 64 && prob_bits != 12) return ERR_ARG;  // the pair bound assumes n = 12
@@ -648,7 +666,7 @@ int oracle_decode(int dtype, const uint8_t* stream, uint64_t stream_bytes,
                   uint32_t tile_n, uint32_t tile_k, const uint32_t* freq, int prob_bits,
                   void* w_out, uint64_t tile_begin, uint64_t tile_end, int threads,
                   int state_bits) {
-  if (dtype < 0 || dtype > 5) return ERR_ARG;
+  if (dtype < 0 || dtype > 6) return ERR_ARG;
   if (state_bits != 32 && state_bits != 64) return ERR_ARG;
   if (!layout_ok(N, K, tile_n, tile_k)) return ERR_SHAPE;
   if (state_bits == 64 && prob_bits != 12) return ERR_ARG;
@@ -698,12 +716,12 @@ int oracle_decode(int dtype, const uint8_t* stream, uint64_t stream_bytes,
           x[l] = (x[l] << (8 * word_bytes)) | word;
         }
         uint32_t row, col;
-        if (dtype == DT_INT4_PAIRS) lane_map_pairs(tile_n, l, j, &row, &col);
+        if (is_pairs(dtype)) lane_map_pairs(tile_n, l, j, &row, &col);
         else lane_map(tile_n, l, j, &row, &col);
         uint64_t idx = (n0 + row) * K + (k0 + col);
-        if (dtype == DT_INT4_PAIRS) {
+        if (is_pairs(dtype)) {
           // idx is even: the pair is exactly one packed byte
-          ((uint8_t*)w_out)[idx / 2] = (uint8_t)(s ^ 0x88);
+          ((uint8_t*)w_out)[idx / 2] = (uint8_t)(dtype == DT_INT4_PAIRS ? s ^ 0x88 : s);
         } else if (dtype == DT_INT4 || dtype == DT_FP4_E2M1) {
           uint8_t* out = (uint8_t*)w_out;
           uint8_t nib = (uint8_t)((dtype == DT_INT4 ? s - 8 : s) & 0xF);
@@ -743,7 +761,7 @@ int oracle_decode(int dtype, const uint8_t* stream, uint64_t stream_bytes,
 int oracle_gemm(int dtype, const uint16_t* X, uint32_t M, uint32_t K, const void* W,
                 uint32_t N, int scale_kind, const void* scales, uint32_t group_k,
                 const uint32_t* rows, uint32_t n_rows, double* Y, int threads) {
-  if (dtype < 0 || dtype > 5) return ERR_ARG;
+  if (dtype < 0 || dtype > 6) return ERR_ARG;
   if (scale_kind == SC_GROUP_BF16 && (group_k == 0 || K % group_k != 0)) return ERR_ARG;
   if (scale_kind != SC_NONE && scales == nullptr) return ERR_ARG;
   if (rows == nullptr) n_rows = N;
@@ -761,7 +779,7 @@ int oracle_gemm(int dtype, const uint16_t* X, uint32_t M, uint32_t K, const void
         else if (scale_kind == SC_GROUP_BF16)
           v *= bf16_value(((const uint16_t*)scales)[n * (K / group_k) + k / group_k]);
         else if (scale_kind == SC_ROW_F32) v *= f32_value(scales, n);
-      } else if (dtype == DT_FP4_E2M1) {
+      } else if (is_fp4(dtype)) {
         const uint8_t byte = ((const uint8_t*)W)[idx / 2];
         v = e2m1_value((idx % 2 == 0) ? (byte & 0xF) : (byte >> 4));
         if (scale_kind == SC_ROW_F32) v *= f32_value(scales, n);

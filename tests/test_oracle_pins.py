@@ -632,6 +632,36 @@ def test_gemm_fp4_exact(oracle):
     assert np.array_equal(Ys, (xi @ vals.T) * s.astype(np.float64)[None, :])
 
 
+@pytest.mark.parametrize("state_bits", [32, 64])
+def test_fp4_pairs_identity_marginals_and_gemm(oracle, state_bits):
+    cfg, d = _small("fp4_8b", 512, 1024)
+    pc = oracle.histogram(WL.FP4_PAIRS, d["w"], 512 * 1024)
+    assert pc.size == 256 and pc.sum() == 512 * 1024 // 2
+    # the packed byte is the symbol: the marginals are the per-code histograms
+    # of the even and the odd elements
+    b = d["w"]
+    assert np.array_equal(pc.reshape(16, 16).sum(axis=0), np.bincount(b & 0xF, minlength=16))
+    assert np.array_equal(pc.reshape(16, 16).sum(axis=1), np.bincount(b >> 4, minlength=16))
+    _, freq = oracle.normalize(pc)
+    st, stream, offsets, _ = oracle.encode(WL.FP4_PAIRS, b, 512, 1024, cfg.tile_n, cfg.tile_k,
+                                           freq, state_bits=state_bits)
+    assert st == 0
+    st, out = oracle.decode(WL.FP4_PAIRS, stream, offsets, None, 512, 1024, cfg.tile_n,
+                            cfg.tile_k, freq, state_bits=state_bits)
+    assert st == 0 and np.array_equal(out, b)
+    # the same lane map as int4 pairs: the int4-pair symbol of the byte b ^ 0x88
+    # is b, so coding the bytes XOR 0x88 as int4 pairs gives the same stream
+    st, s_i4, o_i4, _ = oracle.encode(WL.INT4_PAIRS, b ^ 0x88, 512, 1024, cfg.tile_n, cfg.tile_k,
+                                      freq, state_bits=state_bits)
+    assert st == 0 and np.array_equal(s_i4, stream) and np.array_equal(o_i4, offsets)
+    rng = np.random.default_rng(2)
+    X = WL.to_bf16_bits(rng.standard_normal((2, 1024)))
+    rows = np.arange(0, 512, 41, dtype=np.uint32)
+    Yp = oracle.gemm(WL.FP4_PAIRS, X, 2, 1024, b, 512, cfg.scale_kind, d["scales"], rows=rows)
+    Y1 = oracle.gemm(WL.FP4_E2M1, X, 2, 1024, b, 512, cfg.scale_kind, d["scales"], rows=rows)
+    assert np.array_equal(Yp, Y1)
+
+
 # ---- fp64 GEMM ------------------------------------------------------------------
 def test_gemm_int4_exact_integers(oracle):
     rng = np.random.default_rng(2)
