@@ -66,9 +66,9 @@ def parse():
     ap.add_argument("--state-bits", type=int, default=64, choices=[32, 64],
                     help="stream format: 64 = wide lane states (32-bit words, one "
                          "renormalisation test per symbol pair), 32 = 32-bit states")
-    ap.add_argument("--int4-symbols", default="pairs", choices=["pairs", "element"],
-                    help="--sweep: code int4 weights one symbol per packed byte (two K "
-                         "elements) or one per element")
+    ap.add_argument("--nibble-symbols", default="pairs", choices=["pairs", "element"],
+                    help="--sweep: code int4 and fp4 weights one symbol per packed byte "
+                         "(two K elements) or one per element")
     ap.add_argument("--quick", action="store_true",
                     help="skip the context sweep and the CPU baseline (profiling runs)")
     return ap.parse_args()
@@ -482,8 +482,9 @@ def sweep(args):
         for mi, (mname, mN, mK) in enumerate(cfg.matrices):
             d = WL.make_weights(cfg, mi)
             N, K = d["N"], d["K"]
-            pairs = cfg.dtype == WL.INT4 and args.int4_symbols == "pairs"
-            coded = WL.INT4_PAIRS if pairs else cfg.dtype
+            pairs = cfg.dtype in (WL.INT4, WL.FP4_E2M1) and args.nibble_symbols == "pairs"
+            coded = ({WL.INT4: WL.INT4_PAIRS, WL.FP4_E2M1: WL.FP4_PAIRS}[cfg.dtype] if pairs
+                     else cfg.dtype)
             lay = ans.make_layout(coded, N, K, cfg.tile_n, cfg.tile_k, args.state_bits)
             dw = torch.from_numpy(d["w"].view(np.int16) if d["w"].dtype == np.uint16 else d["w"]).to(device)
             A = ans.ALPHABET[coded]
@@ -536,7 +537,8 @@ def sweep(args):
                 algo = layers[0].compressed_bytes + 2 * M * K + 4 * M * N
                 rec = {"workload": name, "matrix": mname, "N": N, "K": K, "M": M,
                        "state_bits": args.state_bits,
-                       **({"int4_symbols": args.int4_symbols} if cfg.dtype == WL.INT4 else {}),
+                       **({"nibble_symbols": args.nibble_symbols}
+                          if cfg.dtype in (WL.INT4, WL.FP4_E2M1) else {}),
                        "tile": f"{lay.tile_n}x{lay.tile_k}", "bits_per_weight": round(bpw, 4),
                        "entropy_bound_bits": round(bound, 4), "gap_bits": round(bpw - bound, 4),
                        "encode_s": round(encode_s, 2), "copies": copies,

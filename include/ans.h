@@ -52,6 +52,9 @@
  *   ANS_FP8_E4M3   e4m3fn code bytes; coded symbol = the code (A = 256).
  *   ANS_FP4_E2M1   e2m1 codes packed like ANS_INT4 (element k even in the low
  *                  nibble); coded symbol = the code (A = 16).
+ *   ANS_FP4_PAIRS  the same storage as ANS_FP4_E2M1, coded one symbol per packed
+ *                  byte (the byte itself, A = 256), in the lane map of
+ *                  ANS_INT4_PAIRS.
  *   ANS_INT8       int8 code bytes q in [-128, 127]; coded symbol q + 128,
  *                  i.e. the byte XOR 0x80 (A = 256).
  *   ANS_INT4_PAIRS the same storage as ANS_INT4, coded one symbol per packed
@@ -108,7 +111,8 @@ typedef enum {
   ANS_FP8_E4M3 = 2,
   ANS_INT4_PAIRS = 3,
   ANS_INT8 = 4,
-  ANS_FP4_E2M1 = 5
+  ANS_FP4_E2M1 = 5,
+  ANS_FP4_PAIRS = 6
 } ans_dtype;
 
 typedef enum {

@@ -17,10 +17,11 @@ import numpy as np
 
 from . import build as _build
 
-INT4, BF16_SPLIT, FP8_E4M3, INT4_PAIRS, INT8, FP4_E2M1 = 0, 1, 2, 3, 4, 5
+INT4, BF16_SPLIT, FP8_E4M3, INT4_PAIRS, INT8, FP4_E2M1, FP4_PAIRS = 0, 1, 2, 3, 4, 5, 6
 SCALE_NONE, SCALE_ROW_BF16, SCALE_ROW_F32, SCALE_GROUP_BF16 = 0, 1, 2, 3
 STATUS_CORRUPT, STATUS_TIMEOUT, STATUS_BAD_OFFSETS = 0x1, 0x2, 0x4
-ALPHABET = {INT4: 16, BF16_SPLIT: 256, FP8_E4M3: 256, INT4_PAIRS: 256, INT8: 256, FP4_E2M1: 16}
+ALPHABET = {INT4: 16, BF16_SPLIT: 256, FP8_E4M3: 256, INT4_PAIRS: 256, INT8: 256, FP4_E2M1: 16,
+            FP4_PAIRS: 256}
 
 # every symbol include/ans.h declares
 EXPORTS = ["ans_status_string", "ans_last_error", "ans_num_tiles", "ans_layout_check",

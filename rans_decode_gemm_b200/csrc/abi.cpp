@@ -24,11 +24,13 @@ uint32_t alphabet_of(uint32_t dtype) { return (dtype == ANS_INT4 || dtype == ANS
 // packed-nibble storage (per-element or pair symbols)
 bool is_int4(uint32_t dtype) { return dtype == ANS_INT4 || dtype == ANS_INT4_PAIRS; }
 // two weights per byte
-bool is_nibble(uint32_t dtype) { return is_int4(dtype) || dtype == ANS_FP4_E2M1; }
+bool is_nibble(uint32_t dtype) {
+  return is_int4(dtype) || dtype == ANS_FP4_E2M1 || dtype == ANS_FP4_PAIRS;
+}
 
 ans_status check_layout(const ans_layout* l) {
   if (!l) return ANS_ERR_ARG;
-  if (l->dtype > ANS_FP4_E2M1) return ANS_ERR_ARG;
+  if (l->dtype > ANS_FP4_PAIRS) return ANS_ERR_ARG;
   if (l->state_bits != 0 && l->state_bits != 32 && l->state_bits != 64) return ANS_ERR_ARG;
   if (!anshost::layout_valid(l->N, l->K, l->tile_n, l->tile_k)) return ANS_ERR_SHAPE;
   return ANS_OK;
@@ -179,7 +181,7 @@ ans_status ans_layout_check(const ans_layout* layout) { return check_layout(layo
 
 ans_status ans_histogram(const void* d_w, const ans_layout* layout, uint64_t* d_hist,
                          ans_stream_t stream) {
-  if (!layout || layout->dtype > ANS_FP4_E2M1) return ANS_ERR_ARG;
+  if (!layout || layout->dtype > ANS_FP4_PAIRS) return ANS_ERR_ARG;
   if (layout->N == 0 || layout->K == 0) return ANS_ERR_SHAPE;
   if (is_nibble(layout->dtype) && layout->K % 2 != 0) return ANS_ERR_SHAPE;
   if (!d_w || !d_hist || reinterpret_cast<uintptr_t>(d_w) % 16 != 0) return ANS_ERR_ARG;
@@ -195,7 +197,7 @@ ans_status ans_histogram(const void* d_w, const ans_layout* layout, uint64_t* d_
 }
 
 ans_status ans_histogram_host(const void* h_w, const ans_layout* layout, uint64_t* hist) {
-  if (!layout || layout->dtype > ANS_FP4_E2M1) return ANS_ERR_ARG;
+  if (!layout || layout->dtype > ANS_FP4_PAIRS) return ANS_ERR_ARG;
   if (layout->N == 0 || layout->K == 0) return ANS_ERR_SHAPE;
   if (is_nibble(layout->dtype) && layout->K % 2 != 0) return ANS_ERR_SHAPE;
   if (!h_w || !hist) return ANS_ERR_ARG;

@@ -49,7 +49,8 @@ __device__ __forceinline__ void store_group(void* out, uint64_t idx, const uint3
       hi ^= 0x80808080u;
     }
     // idx counts bytes for fp8 and K elements (two per byte) for int4 pairs
-    *reinterpret_cast<uint2*>(static_cast<uint8_t*>(out) + (DT == kDtInt4Pairs ? idx / 2 : idx)) =
+    *reinterpret_cast<uint2*>(static_cast<uint8_t*>(out) +
+                              ((DT == kDtInt4Pairs || DT == kDtFp4Pairs) ? idx / 2 : idx)) =
         make_uint2(lo, hi);
   }
 }
@@ -124,7 +125,7 @@ __global__ void __launch_bounds__(kDecMaxWarps * 32, 2)
     uint32_t g = 0;
     // group order (slab s, half h, chunk c, row i) matches the stream's lane
     // map; an int4 pair group covers both 8-column chunks of its row
-    constexpr uint32_t kGroups = DT == kDtInt4Pairs ? 4 : 8;
+    constexpr uint32_t kGroups = (DT == kDtInt4Pairs || DT == kDtFp4Pairs) ? 4 : 8;
     for (uint32_t s = 0; s < C; ++s) {
       for (uint32_t h = 0; h < H; ++h) {
 #pragma unroll
@@ -177,8 +178,8 @@ __global__ void __launch_bounds__(kHistWarps * 32)
         const uint32_t flip = dtype == kDtInt4 ? 8u : 0u;
 #pragma unroll
         for (int n = 0; n < 8; ++n) atomicAdd(&mine[((u >> (4 * n)) & 0xFu) ^ flip], 1u);
-      } else if (dtype == kDtInt4Pairs || dtype == kDtInt8) {
-        const uint32_t flip = dtype == kDtInt8 ? 0x80u : 0x88u;
+      } else if (dtype == kDtInt4Pairs || dtype == kDtInt8 || dtype == kDtFp4Pairs) {
+        const uint32_t flip = dtype == kDtInt8 ? 0x80u : (dtype == kDtInt4Pairs ? 0x88u : 0u);
 #pragma unroll
         for (int n = 0; n < 4; ++n) atomicAdd(&mine[((u >> (8 * n)) & 0xFFu) ^ flip], 1u);
       } else if (dtype == kDtBf16Split) {
@@ -198,8 +199,8 @@ __global__ void __launch_bounds__(kHistWarps * 32)
         const uint32_t flip = dtype == kDtInt4 ? 8u : 0u;
         atomicAdd(&mine[(w[b] & 0xFu) ^ flip], 1u);
         atomicAdd(&mine[((w[b] >> 4) & 0xFu) ^ flip], 1u);
-      } else if (dtype == kDtInt4Pairs || dtype == kDtInt8) {
-        atomicAdd(&mine[w[b] ^ (dtype == kDtInt8 ? 0x80u : 0x88u)], 1u);
+      } else if (dtype == kDtInt4Pairs || dtype == kDtInt8 || dtype == kDtFp4Pairs) {
+        atomicAdd(&mine[w[b] ^ (dtype == kDtInt8 ? 0x80u : (dtype == kDtInt4Pairs ? 0x88u : 0u))], 1u);
       } else if (dtype == kDtBf16Split) {
         uint32_t u = w[b] | (static_cast<uint32_t>(w[b + 1]) << 8);
         atomicAdd(&mine[(u >> 7) & 0xFFu], 1u);
@@ -244,6 +245,7 @@ cudaError_t launch_decode_tiles(const LayerDev& L, void* out, uint32_t* status,
     if (L.dtype == kDtInt4Pairs) return launch_decode_variant<kDtInt4Pairs, true>(L, out, status, stream, blocks, warps);
     if (L.dtype == kDtInt8) return launch_decode_variant<kDtInt8, true>(L, out, status, stream, blocks, warps);
     if (L.dtype == kDtFp4) return launch_decode_variant<kDtFp4, true>(L, out, status, stream, blocks, warps);
+    if (L.dtype == kDtFp4Pairs) return launch_decode_variant<kDtFp4Pairs, true>(L, out, status, stream, blocks, warps);
     return launch_decode_variant<kDtFp8, true>(L, out, status, stream, blocks, warps);
   }
   if (L.dtype == kDtBf16Split) return launch_decode_variant<kDtBf16Split, false>(L, out, status, stream, blocks, warps);
@@ -251,6 +253,7 @@ cudaError_t launch_decode_tiles(const LayerDev& L, void* out, uint32_t* status,
   if (L.dtype == kDtInt4Pairs) return launch_decode_variant<kDtInt4Pairs, false>(L, out, status, stream, blocks, warps);
   if (L.dtype == kDtInt8) return launch_decode_variant<kDtInt8, false>(L, out, status, stream, blocks, warps);
   if (L.dtype == kDtFp4) return launch_decode_variant<kDtFp4, false>(L, out, status, stream, blocks, warps);
+  if (L.dtype == kDtFp4Pairs) return launch_decode_variant<kDtFp4Pairs, false>(L, out, status, stream, blocks, warps);
   return launch_decode_variant<kDtFp8, false>(L, out, status, stream, blocks, warps);
 }
 

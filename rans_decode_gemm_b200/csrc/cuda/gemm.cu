@@ -283,6 +283,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
               decode_group<kWide>(tc, lut_s, pipe.ring_s, lt, e);
             }
             if constexpr (kFmt == kFmtInt4PairBf16) fmt_int4pair_bf16(e, o);
+            else if constexpr (kFmt == kFmtFp4PairBf16) fmt_fp4pair_bf16(e, o);
             else if constexpr (kFmt == kFmtInt4PairF16Group)
               fmt_int4pair_f16_scaled(e, i == 0 ? gs0 : i == 1 ? gs1 : i == 2 ? gs2 : gs3, o);
             else if constexpr (kFmt == kFmtBf16Split) fmt_bf16_split(e, raw8, o);
@@ -592,6 +593,7 @@ bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool dec
                    : ((scale_kind == 3) ? kFmtInt4F16Group : kFmtInt4Bf16);
   else if (L.dtype == 4) p.fmt = kFmtInt8F16;
   else if (L.dtype == 5) p.fmt = kFmtFp4Bf16;
+  else if (L.dtype == 6) p.fmt = decode ? kFmtFp4PairBf16 : kFmtFp4Bf16;  // same slabs
   else p.fmt = kFmtFp8F16;
   p.ab_f16 = (fmt_group(p.fmt) || p.fmt == kFmtFp8F16 || p.fmt == kFmtInt8F16) ? 1 : 0;
   p.M = M;
@@ -827,7 +829,7 @@ cudaError_t launch_gemm(const GemmPlan& plan, const LayerDev& L, bool decode, co
   }
   if (plan.local) return launch_gemm_local(plan, P, decode, stream);
 
-  switch (plan.fmt | (decode ? 0u : 8u)) {
+  switch (plan.fmt | (decode ? 0u : 16u)) {  // 16 | fmt: the copy variants
     case kFmtBf16Split:
       return P.L.wide ? launch_variant<true, kFmtBf16Split, true>(plan, P, stream)
                       : launch_variant<true, kFmtBf16Split>(plan, P, stream);
@@ -852,12 +854,15 @@ cudaError_t launch_gemm(const GemmPlan& plan, const LayerDev& L, bool decode, co
     case kFmtFp4Bf16:
       return P.L.wide ? launch_variant<true, kFmtFp4Bf16, true>(plan, P, stream)
                       : launch_variant<true, kFmtFp4Bf16>(plan, P, stream);
-    case 8 | kFmtBf16Split: return launch_variant<false, kFmtBf16Split>(plan, P, stream);
-    case 8 | kFmtInt4Bf16: return launch_variant<false, kFmtInt4Bf16>(plan, P, stream);
-    case 8 | kFmtInt4F16Group: return launch_variant<false, kFmtInt4F16Group>(plan, P, stream);
-    case 8 | kFmtFp8F16: return launch_variant<false, kFmtFp8F16>(plan, P, stream);
-    case 8 | kFmtInt8F16: return launch_variant<false, kFmtInt8F16>(plan, P, stream);
-    case 8 | kFmtFp4Bf16: return launch_variant<false, kFmtFp4Bf16>(plan, P, stream);
+    case kFmtFp4PairBf16:
+      return P.L.wide ? launch_variant<true, kFmtFp4PairBf16, true>(plan, P, stream)
+                      : launch_variant<true, kFmtFp4PairBf16>(plan, P, stream);
+    case 16 | kFmtBf16Split: return launch_variant<false, kFmtBf16Split>(plan, P, stream);
+    case 16 | kFmtInt4Bf16: return launch_variant<false, kFmtInt4Bf16>(plan, P, stream);
+    case 16 | kFmtInt4F16Group: return launch_variant<false, kFmtInt4F16Group>(plan, P, stream);
+    case 16 | kFmtFp8F16: return launch_variant<false, kFmtFp8F16>(plan, P, stream);
+    case 16 | kFmtInt8F16: return launch_variant<false, kFmtInt8F16>(plan, P, stream);
+    case 16 | kFmtFp4Bf16: return launch_variant<false, kFmtFp4Bf16>(plan, P, stream);
   }
   return cudaErrorInvalidValue;
 }

@@ -336,6 +336,7 @@ __device__ __forceinline__ void local_cta(const GemmDev& P) {
                   }
                 }
                 if constexpr (kFmt == kFmtInt4PairBf16) fmt_int4pair_bf16(e, o);
+                else if constexpr (kFmt == kFmtFp4PairBf16) fmt_fp4pair_bf16(e, o);
                 else if constexpr (kFmt == kFmtInt4PairF16Group) fmt_int4pair_f16_scaled(e, gsc[i], o);
                 else if constexpr (kFmt == kFmtBf16Split) fmt_bf16_split(e, raw8, o);
                 else if constexpr (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
@@ -651,7 +652,7 @@ static cudaError_t launch_local_variant(const GemmPlan& plan, const GemmDev& P, 
 
 cudaError_t launch_gemm_local(const GemmPlan& plan, const GemmDev& P, bool decode,
                               cudaStream_t stream) {
-  switch (plan.fmt | (decode ? 0u : 8u)) {
+  switch (plan.fmt | (decode ? 0u : 16u)) {  // 16 | fmt: the copy variants
     case kFmtBf16Split:
       return P.L.wide ? launch_local_variant<true, kFmtBf16Split, true>(plan, P, stream)
                       : launch_local_variant<true, kFmtBf16Split>(plan, P, stream);
@@ -676,12 +677,15 @@ cudaError_t launch_gemm_local(const GemmPlan& plan, const GemmDev& P, bool decod
     case kFmtFp4Bf16:
       return P.L.wide ? launch_local_variant<true, kFmtFp4Bf16, true>(plan, P, stream)
                       : launch_local_variant<true, kFmtFp4Bf16>(plan, P, stream);
-    case 8 | kFmtBf16Split: return launch_local_variant<false, kFmtBf16Split>(plan, P, stream);
-    case 8 | kFmtInt4Bf16: return launch_local_variant<false, kFmtInt4Bf16>(plan, P, stream);
-    case 8 | kFmtInt4F16Group: return launch_local_variant<false, kFmtInt4F16Group>(plan, P, stream);
-    case 8 | kFmtFp8F16: return launch_local_variant<false, kFmtFp8F16>(plan, P, stream);
-    case 8 | kFmtInt8F16: return launch_local_variant<false, kFmtInt8F16>(plan, P, stream);
-    case 8 | kFmtFp4Bf16: return launch_local_variant<false, kFmtFp4Bf16>(plan, P, stream);
+    case kFmtFp4PairBf16:
+      return P.L.wide ? launch_local_variant<true, kFmtFp4PairBf16, true>(plan, P, stream)
+                      : launch_local_variant<true, kFmtFp4PairBf16>(plan, P, stream);
+    case 16 | kFmtBf16Split: return launch_local_variant<false, kFmtBf16Split>(plan, P, stream);
+    case 16 | kFmtInt4Bf16: return launch_local_variant<false, kFmtInt4Bf16>(plan, P, stream);
+    case 16 | kFmtInt4F16Group: return launch_local_variant<false, kFmtInt4F16Group>(plan, P, stream);
+    case 16 | kFmtFp8F16: return launch_local_variant<false, kFmtFp8F16>(plan, P, stream);
+    case 16 | kFmtInt8F16: return launch_local_variant<false, kFmtInt8F16>(plan, P, stream);
+    case 16 | kFmtFp4Bf16: return launch_local_variant<false, kFmtFp4Bf16>(plan, P, stream);
   }
   return cudaErrorInvalidValue;
 }
@@ -732,6 +736,9 @@ cudaError_t launch_gemm_local_batch(const GemmPlan& plan, const BatchDev& B, uin
     case kFmtFp4Bf16:
       return wide ? launch_local_batch_variant<kFmtFp4Bf16, true>(plan, B, grid, stream)
                   : launch_local_batch_variant<kFmtFp4Bf16, false>(plan, B, grid, stream);
+    case kFmtFp4PairBf16:
+      return wide ? launch_local_batch_variant<kFmtFp4PairBf16, true>(plan, B, grid, stream)
+                  : launch_local_batch_variant<kFmtFp4PairBf16, false>(plan, B, grid, stream);
   }
   return cudaErrorInvalidValue;
 }

@@ -34,10 +34,13 @@ enum : uint32_t {
   kFmtInt4PairBf16 = 4,     // int4 pair symbol -> two exact bf16 (row scale in the epilogue)
   kFmtInt4PairF16Group = 5, // int4 pair symbol * group scale -> two exact f16
   kFmtInt8F16 = 6,          // int8 code -> exact f16 (row scale applied in the epilogue)
-  kFmtFp4Bf16 = 7           // e2m1 code -> exact bf16 (row scale applied in the epilogue)
+  kFmtFp4Bf16 = 7,          // e2m1 code -> exact bf16 (row scale applied in the epilogue)
+  kFmtFp4PairBf16 = 8       // e2m1 pair symbol (a packed byte) -> two exact bf16
 };
 // int4 pair symbols: 8 symbols of a lane fill 16 columns of one slab row
-__host__ __device__ constexpr bool fmt_pair(uint32_t f) { return f == kFmtInt4PairBf16 || f == kFmtInt4PairF16Group; }
+__host__ __device__ constexpr bool fmt_pair(uint32_t f) {
+  return f == kFmtInt4PairBf16 || f == kFmtInt4PairF16Group || f == kFmtFp4PairBf16;
+}
 // a per-(row, K group) scale is applied while the slab is written
 __host__ __device__ constexpr bool fmt_group(uint32_t f) { return f == kFmtInt4F16Group || f == kFmtInt4PairF16Group; }
 

@@ -49,7 +49,15 @@ constexpr uint32_t kStatusCorrupt = 0x1u;
 constexpr uint32_t kStatusTimeout = 0x2u;
 constexpr uint32_t kStatusBadOffsets = 0x4u;
 
-enum : uint32_t { kDtInt4 = 0, kDtBf16Split = 1, kDtFp8 = 2, kDtInt4Pairs = 3, kDtInt8 = 4, kDtFp4 = 5 };
+enum : uint32_t {
+  kDtInt4 = 0,
+  kDtBf16Split = 1,
+  kDtFp8 = 2,
+  kDtInt4Pairs = 3,
+  kDtInt8 = 4,
+  kDtFp4 = 5,
+  kDtFp4Pairs = 6
+};
 
 
 // Abort-aware bounded wait.  Returns false if the wait ran out (then sets the
@@ -720,15 +728,21 @@ __device__ __forceinline__ void fmt_int8_f16(const uint32_t (&e)[8], uint32_t (&
 // bf16 patterns 0x0000, 0x3F00, 0x3F80, 0x3FC0, 0x4000, 0x4040, 0x4080, 0x40C0,
 // looked up bytewise with two byte permutes (the low and the high byte of
 // both codes at once), interleaved with a third; bit 3 of a code is the sign.
+__device__ __forceinline__ uint32_t e2m1x2_bf16x2(uint32_t c0, uint32_t c1) {
+  const uint32_t sel = (c0 & 7u) | ((c1 & 7u) << 4);
+  const uint32_t lo = __byte_perm(0xC0800000u, 0xC0804000u, sel);  // low bytes, codes 0-7
+  const uint32_t hi = __byte_perm(0x3F3F3F00u, 0x40404040u, sel);  // high bytes
+  return __byte_perm(lo, hi, 0x5140u) | ((c0 & 8u) << 12) | ((c1 & 8u) << 28);
+}
 __device__ __forceinline__ void fmt_fp4_bf16(const uint32_t (&e)[8], uint32_t (&out)[4]) {
 #pragma unroll
-  for (int p = 0; p < 4; ++p) {
-    const uint32_t c0 = (e[2 * p] >> 12) & 0xFu, c1 = (e[2 * p + 1] >> 12) & 0xFu;
-    const uint32_t sel = (c0 & 7u) | ((c1 & 7u) << 4);
-    const uint32_t lo = __byte_perm(0xC0800000u, 0xC0804000u, sel);  // low bytes, codes 0-7
-    const uint32_t hi = __byte_perm(0x3F3F3F00u, 0x40404040u, sel);  // high bytes
-    out[p] = __byte_perm(lo, hi, 0x5140u) | ((c0 & 8u) << 12) | ((c1 & 8u) << 28);
-  }
+  for (int p = 0; p < 4; ++p) out[p] = e2m1x2_bf16x2((e[2 * p] >> 12) & 0xFu, (e[2 * p + 1] >> 12) & 0xFu);
+}
+// fp4 pair symbols (the packed byte, in bits 12..19 of the entry): 8 symbols ->
+// 16 consecutive K elements.
+__device__ __forceinline__ void fmt_fp4pair_bf16(const uint32_t (&e)[8], uint32_t (&out)[8]) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k) out[k] = e2m1x2_bf16x2((e[k] >> 12) & 0xFu, (e[k] >> 16) & 0xFu);
 }
 
 // e4m3 codes to exact f16 pairs with the hardware converter.

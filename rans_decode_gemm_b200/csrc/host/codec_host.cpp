@@ -80,11 +80,13 @@ bool code_tile(const TileJob& job, uint64_t t, std::vector<uint8_t>& out,
                std::vector<uint8_t>& sym, std::vector<uint16_t>& words,
                std::vector<uint32_t>& words32, uint8_t* raw_tile) {
   const uint64_t origin = (t / job.n_kt) * job.tile_n * job.K + (t % job.n_kt) * job.tile_k;
-  const size_t S = static_cast<size_t>(job.tile_n) * job.tile_k / (job.dtype == kInt4Pairs ? 2 : 1);
+  const bool pairs = job.dtype == kInt4Pairs || job.dtype == kFp4Pairs;
+  const size_t S = static_cast<size_t>(job.tile_n) * job.tile_k / (pairs ? 2 : 1);
   const std::vector<uint64_t>& order = *job.order;
   sym.resize(S);
-  if (job.dtype == kInt4Pairs) {
-    for (size_t q = 0; q < S; ++q) sym[q] = static_cast<uint8_t>(job.w[(origin + order[q]) >> 1] ^ 0x88);
+  if (pairs) {
+    const uint8_t flip = job.dtype == kInt4Pairs ? 0x88 : 0;  // fp4 pairs: the byte itself
+    for (size_t q = 0; q < S; ++q) sym[q] = static_cast<uint8_t>(job.w[(origin + order[q]) >> 1] ^ flip);
   } else if (job.dtype == kInt4 || job.dtype == kFp4) {
     const uint8_t flip = job.dtype == kInt4 ? 8 : 0;  // int4: q + 8; fp4: the code
     for (size_t q = 0; q < S; ++q) {
@@ -194,7 +196,7 @@ bool layout_valid(uint32_t N, uint32_t K, uint32_t tile_n, uint32_t tile_k) {
 
 void histogram(uint32_t dtype, const void* w, uint64_t n_weights, uint64_t* hist) {
   const uint32_t A = (dtype == kInt4 || dtype == kFp4) ? 16 : 256;
-  const uint64_t units = (dtype == kInt4 || dtype == kInt4Pairs || dtype == kFp4)
+  const uint64_t units = (dtype == kInt4 || dtype == kInt4Pairs || dtype == kFp4 || dtype == kFp4Pairs)
                              ? n_weights / 2 : n_weights;  // bytes or u16 words
   const unsigned nw = worker_count(units / 65536 + 1);
   std::vector<std::vector<uint64_t>> part(nw, std::vector<uint64_t>(256, 0));
@@ -207,9 +209,10 @@ void histogram(uint32_t dtype, const void* w, uint64_t n_weights, uint64_t* hist
         const uint8_t* p = static_cast<const uint8_t*>(w);
         const uint8_t flip = dtype == kInt4 ? 8 : 0;
         for (uint64_t i = a; i < b; ++i) { h[(p[i] & 15) ^ flip]++; h[(p[i] >> 4) ^ flip]++; }
-      } else if (dtype == kInt4Pairs) {
+      } else if (dtype == kInt4Pairs || dtype == kFp4Pairs) {
         const uint8_t* p = static_cast<const uint8_t*>(w);
-        for (uint64_t i = a; i < b; ++i) h[p[i] ^ 0x88]++;
+        const uint8_t flip = dtype == kInt4Pairs ? 0x88 : 0;
+        for (uint64_t i = a; i < b; ++i) h[p[i] ^ flip]++;
       } else if (dtype == kInt8) {
         const uint8_t* p = static_cast<const uint8_t*>(w);
         for (uint64_t i = a; i < b; ++i) h[p[i] ^ 0x80]++;
@@ -317,7 +320,8 @@ int encode(uint32_t dtype, const void* w, uint32_t N, uint32_t K, uint32_t tile_
   const uint32_t n_kt = K / tile_k;
   const uint64_t tiles = static_cast<uint64_t>(N / tile_n) * n_kt;
   const std::vector<uint64_t> order =
-      dtype == kInt4Pairs ? lane_order_pairs(tile_n, tile_k, K) : lane_order(tile_n, tile_k, K);
+      (dtype == kInt4Pairs || dtype == kFp4Pairs) ? lane_order_pairs(tile_n, tile_k, K)
+                                                  : lane_order(tile_n, tile_k, K);
   TileJob job;
   job.wide = wide;
   job.dtype = dtype;

@@ -4,7 +4,7 @@
 
 namespace anshost {
 
-enum : uint32_t { kInt4 = 0, kBf16Split = 1, kFp8 = 2, kInt4Pairs = 3, kInt8 = 4, kFp4 = 5 };
+enum : uint32_t { kInt4 = 0, kBf16Split = 1, kFp8 = 2, kInt4Pairs = 3, kInt8 = 4, kFp4 = 5, kFp4Pairs = 6 };
 
 bool layout_valid(uint32_t N, uint32_t K, uint32_t tile_n, uint32_t tile_k);
 void histogram(uint32_t dtype, const void* w, uint64_t n_weights, uint64_t* hist);

@@ -38,7 +38,8 @@ def test_status_strings_and_layout_checks(ans_lib):
     assert ans.ans_layout_check(ans.make_layout(0, 512, 520, 128, 40)) == 2    # tile_k % 16
     assert ans.ans_layout_check(ans.make_layout(0, 512, 512, 64, 32)) == 2     # tile_n
     assert ans.ans_layout_check(ans.make_layout(7, 512, 512, 128, 32)) == 1    # dtype
-    assert ans.ans_layout_check(ans.make_layout(6, 512, 512, 128, 32)) == 1    # dtype
+    assert ans.ans_layout_check(ans.make_layout(7, 512, 512, 128, 32)) == 1    # dtype
+    assert ans.ans_layout_check(ans.make_layout(6, 512, 512, 128, 32)) == 0    # fp4 pairs
     assert ans.ans_layout_check(ans.make_layout(5, 512, 512, 128, 32)) == 0    # fp4
     assert ans.ans_layout_check(ans.make_layout(4, 512, 512, 128, 32)) == 0    # int8
     assert ans.ans_layout_check(ans.make_layout(3, 512, 512, 128, 32)) == 0    # int4 pairs
@@ -60,9 +61,10 @@ CASES = [("tiny_int4", 512, 512), ("bf16_4096", 512, 512), ("llama8b_mlp", 256, 
 def test_host_codec_matches_oracle(oracle, ans_lib, name, N, K, state_bits, pairs):
     cfg = WL.CONFIGS[name]
     if pairs:
-        if cfg.dtype != WL.INT4:
-            pytest.skip("pair symbols are an int4 coding")
-        cfg = WL.Config(**{**cfg.__dict__, "dtype": WL.INT4_PAIRS})
+        if cfg.dtype not in (WL.INT4, WL.FP4_E2M1):
+            pytest.skip("pair symbols are a coding of packed nibbles")
+        cfg = WL.Config(**{**cfg.__dict__,
+                           "dtype": WL.INT4_PAIRS if cfg.dtype == WL.INT4 else WL.FP4_PAIRS})
     d = WL.make_weights(WL.CONFIGS[name], 0, N=N, K=K)
     lay = ans.make_layout(cfg.dtype, N, K, cfg.tile_n, cfg.tile_k, state_bits)
     hist = ans.ans_histogram_host(d["w"], lay)

@@ -57,6 +57,7 @@ def _sms():
 
 CASES = [("bf16_4096", 1024, 2048, 64, None), ("int4_70b", 512, 1024, 64, ans.INT4_PAIRS),
          ("int8_8b", 512, 1024, 64, None), ("fp4_8b", 512, 1024, 32, None),
+         ("fp4_8b", 512, 1024, 64, ans.FP4_PAIRS),
          ("int4_70b", 512, 1024, 32, None), ("fp8_405b", 256, 2048, 64, None),
          ("tiny_int4", 512, 512, 32, None), ("llama8b_mlp", 512, 1024, 64, None)]
 

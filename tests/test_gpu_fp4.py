@@ -23,10 +23,10 @@ def cases():
     return {}
 
 
-def _case(cases, N, K, state_bits):
-    key = (N, K, state_bits)
+def _case(cases, N, K, state_bits, dtype=ans.FP4_E2M1):
+    key = (N, K, state_bits, dtype)
     if key not in cases:
-        cases[key] = make_case("fp4_8b", N, K, state_bits=state_bits)
+        cases[key] = make_case("fp4_8b", N, K, state_bits=state_bits, dtype=dtype)
     return cases[key]
 
 
@@ -38,37 +38,44 @@ def _decode(layer, lay):
     return out.cpu().numpy(), int(st.item())
 
 
+@pytest.mark.parametrize("dtype", [ans.FP4_E2M1, ans.FP4_PAIRS])
 @pytest.mark.parametrize("N,K", [(512, 1024), (3, 38), (1, 16)])
-def test_fp4_histogram_gpu(cuda, oracle, N, K):
+def test_fp4_histogram_gpu(cuda, oracle, N, K, dtype):
     w = np.random.default_rng(N + K).integers(0, 256, size=N * K // 2).astype(np.uint8)
-    lay = ans.make_layout(ans.FP4_E2M1, N, K, 128, 64)
-    h = torch.zeros(16, dtype=torch.int64, device="cuda")
+    lay = ans.make_layout(dtype, N, K, 128, 64)
+    h = torch.zeros(ans.ALPHABET[dtype], dtype=torch.int64, device="cuda")
     ans.ans_histogram(to_dev(w), lay, h)
     torch.cuda.synchronize()
-    assert np.array_equal(h.cpu().numpy().astype(np.uint64), oracle.histogram(WL.FP4_E2M1, w, N * K))
+    assert np.array_equal(h.cpu().numpy().astype(np.uint64), oracle.histogram(dtype, w, N * K))
 
 
+@pytest.mark.parametrize("dtype", [ans.FP4_E2M1, ans.FP4_PAIRS])
 @pytest.mark.parametrize("state_bits", [32, 64])
 @pytest.mark.parametrize("N,K", SMALL)
-def test_fp4_decode_bit_exact(cuda, oracle, cases, N, K, state_bits):
-    cfg, d, lay, layer = _case(cases, N, K, state_bits)
+def test_fp4_decode_bit_exact(cuda, oracle, cases, N, K, state_bits, dtype):
+    cfg, d, lay, layer = _case(cases, N, K, state_bits, dtype)
     out, st = _decode(layer, lay)
     assert st == 0 and np.array_equal(out, d["w"])
-    sto, ref = oracle.decode(WL.FP4_E2M1, layer.h_stream, layer.h_offsets, None, N, K, cfg.tile_n,
+    sto, ref = oracle.decode(dtype, layer.h_stream, layer.h_offsets, None, N, K, cfg.tile_n,
                              cfg.tile_k, layer.codebook.freq_array(), state_bits=state_bits)
     assert sto == 0 and np.array_equal(out, ref)
 
 
+@pytest.mark.parametrize("dtype", [ans.FP4_E2M1, ans.FP4_PAIRS])
 @pytest.mark.parametrize("state_bits", [32, 64])
 @pytest.mark.parametrize("N,K", SMALL)
 @pytest.mark.parametrize("M", [1, 16, 17, 64, 128, 300])
-def test_fp4_gemm_parity(cuda, oracle, cases, N, K, M, state_bits):
-    cfg, d, lay, layer = _case(cases, N, K, state_bits)
+def test_fp4_gemm_parity(cuda, oracle, cases, N, K, M, state_bits, dtype):
+    cfg, d, lay, layer = _case(cases, N, K, state_bits, dtype)
     X = WL.make_x(cfg, M, K)
     Y, st, _ = run_gemm(cfg, d, lay, layer, X, compressed=True)
     Yu, stu, _ = run_gemm(cfg, d, lay, layer, X, compressed=False)
     assert st == 0 and stu == 0
     assert torch.equal(Y, Yu), "ans_gemm must be bit-identical to ans_gemm_uncompressed"
+    if dtype == ans.FP4_PAIRS:   # the per-code coding fills the same slabs
+        _, _, lay1, layer1 = _case(cases, N, K, state_bits)
+        Y1, st1, _ = run_gemm(cfg, d, lay1, layer1, X, compressed=True)
+        assert st1 == 0 and torch.equal(Y, Y1)
     Yref = oracle.gemm(WL.FP4_E2M1, X, M, K, d["w"], N, cfg.scale_kind, d["scales"])
     assert rel_fro(Y.cpu().numpy(), Yref) <= TOL
 
@@ -79,8 +86,8 @@ def test_fp4_gemm_schedules(cuda, oracle, cases, monkeypatch, schedule, ctas, pr
     monkeypatch.setenv("ANS_GEMM_SCHEDULE", schedule)
     monkeypatch.setenv("ANS_GEMM_MAX_CTAS", str(ctas))
     monkeypatch.setenv("ANS_GEMM_MAX_PRODUCERS", str(producers))
-    for state_bits in (32, 64):
-        cfg, d, lay, layer = _case(cases, 512, 1024, state_bits)
+    for state_bits, dtype in ((32, ans.FP4_E2M1), (64, ans.FP4_E2M1), (64, ans.FP4_PAIRS)):
+        cfg, d, lay, layer = _case(cases, 512, 1024, state_bits, dtype)
         X = WL.make_x(cfg, 16, 1024)
         Y, st, _ = run_gemm(cfg, d, lay, layer, X, compressed=True)
         Yu, stu, _ = run_gemm(cfg, d, lay, layer, X, compressed=False)
