@@ -347,6 +347,16 @@ def time_ours(args):
             "offline": {"host_encode_s": round(encode_s, 3)},
         }
         result.update(extra)
+        if "decode_tiles_Tsym_per_s" in extra:
+            # the second ceiling: the rate at which the fused kernel decodes
+            # symbols against the standalone decode kernel on the same layer
+            # (the per-tile rANS chain, not HBM or the tensor cores, bounds both)
+            fused_rate = N * K / (kern_ms * 1e-3) / 1e12
+            ceil = extra["decode_tiles_Tsym_per_s"]
+            result["decode_ceiling"] = {
+                "unit": "T symbols/s", "fused": round(fused_rate, 4),
+                "standalone_decode": ceil, "frac": round(fused_rate / ceil, 4),
+                "note": "ans_gemm symbol rate / ans_decode_tiles symbol rate, same layer, same run"}
         if not (args.no_cpu_baseline or args.quick):
             result["cpu_baseline"] = cpu_baseline(cfg, d, lay, layer, X_h, budget_s=20.0)
     if pg is not None:
