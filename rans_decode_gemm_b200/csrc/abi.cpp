@@ -382,8 +382,7 @@ void ansdev_set_trace(void* d_buf, size_t bytes) { ansdev::set_trace_buffer(d_bu
 namespace {
 
 // Shared checks of a batch; on success *sms is the device's SM count.
-ans_status check_batch(const ans_gemm_job* jobs, uint32_t n_jobs, uint32_t M,
-                       ans_scale_kind scale_kind, int* sms) {
+ans_status check_batch(const ans_gemm_job* jobs, uint32_t n_jobs, int* sms) {
   if (!jobs || n_jobs == 0 || n_jobs > ANS_MAX_BATCH) return ANS_ERR_ARG;
   for (uint32_t j = 0; j < n_jobs; ++j) {
     if (!jobs[j].W) return ANS_ERR_ARG;
@@ -395,8 +394,6 @@ ans_status check_batch(const ans_gemm_job* jobs, uint32_t n_jobs, uint32_t M,
         a.tile_k != b.tile_k || (a.state_bits == 64) != (b.state_bits == 64))
       return ANS_ERR_SHAPE;
   }
-  (void)M;
-  (void)scale_kind;
   return device_info(sms);
 }
 
@@ -425,7 +422,7 @@ ans_status ans_gemm_batched_workspace(const ans_gemm_job* jobs, uint32_t n_jobs,
                                       ans_scale_kind scale_kind, size_t* bytes) {
   if (!bytes) return ANS_ERR_ARG;
   int sms = 0;
-  ans_status st = check_batch(jobs, n_jobs, M, scale_kind, &sms);
+  ans_status st = check_batch(jobs, n_jobs, &sms);
   if (st != ANS_OK) return st;
   if (M == 0) { *bytes = 0; return ANS_OK; }
   ansdev::GemmPlan share, full;
@@ -440,7 +437,7 @@ ans_status ans_gemm_batched(const ans_gemm_job* jobs, uint32_t n_jobs, uint32_t 
                             ans_scale_kind scale_kind, uint32_t group_k, void* d_ws,
                             size_t ws_bytes, uint32_t* d_status, ans_stream_t stream) {
   int sms = 0;
-  ans_status st = check_batch(jobs, n_jobs, M, scale_kind, &sms);
+  ans_status st = check_batch(jobs, n_jobs, &sms);
   if (st != ANS_OK) return st;
   ansdev::LayerDev Ls[ANS_MAX_BATCH];
   const ansdev::LayerDev* Lp[ANS_MAX_BATCH];

@@ -20,8 +20,8 @@ constexpr uint32_t kDecLutBytes = kSlots * 4;
 // [lut 16 KB][align slack 2 KB][rings W x 2 KB][barriers W x 4 x 8 B]
 constexpr uint32_t kDecSmem = kDecLutBytes + 128 + kDecMaxWarps * kRingStride + kDecMaxWarps * 4 * 8;
 
-// 8 output elements of one lane (row, 8 consecutive columns) in the original
-// storage format.
+// The 8 symbols of one lane's group in the original storage format: 8
+// consecutive columns of one row, or 16 for pair symbols (one byte each).
 template <uint32_t DT>
 __device__ __forceinline__ void store_group(void* out, uint64_t idx, const uint32_t (&e)[8],
                                             uint64_t raw8) {
