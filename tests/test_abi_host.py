@@ -167,3 +167,38 @@ def test_batched_argument_checks(ans_lib):
     lib = ans.load()
     arr = ans._jobs([(None, ta, None, None), (None, wide, None, None)])
     assert lib.ans_gemm_batched(arr, 2, 16, 0, 0, None, 0, None, None) == 2   # state widths differ
+
+
+def test_host_codec_matches_oracle_fuzzed(oracle, ans_lib):
+    # random shapes, tile shapes, state widths and skews for every coded dtype:
+    # the library's encoder writes the oracle's bytes and its histogram is the oracle's
+    rng = np.random.default_rng(77)
+    for trial in range(24):
+        dtype = int(rng.choice([WL.INT4, WL.BF16_SPLIT, WL.FP8_E4M3, WL.INT4_PAIRS, WL.INT8,
+                                WL.FP4_E2M1, WL.FP4_PAIRS]))
+        tile_n = int(rng.choice([128, 256]))
+        tile_k = int(rng.choice([16, 32, 64, 128]))
+        N, K = tile_n * int(rng.integers(1, 3)), tile_k * int(rng.integers(1, 4))
+        state_bits = int(rng.choice([32, 64]))
+        scale = float(rng.choice([0.3, 1.0, 3.0]))
+        if dtype in (WL.INT4, WL.INT4_PAIRS, WL.FP4_E2M1, WL.FP4_PAIRS):
+            nib = np.clip(np.rint(rng.laplace(0, scale, size=N * K)), -8, 7).astype(np.int8) & 0xF
+            w = (nib[0::2] | (nib[1::2] << 4)).astype(np.uint8)
+        elif dtype == WL.BF16_SPLIT:
+            w = WL.to_bf16_bits(rng.standard_normal(N * K) * 0.02 * scale)
+        else:
+            w = np.clip(np.rint(rng.laplace(0, 8 * scale, size=N * K)), -128, 127).astype(np.int8).view(np.uint8)
+        lay = ans.make_layout(dtype, N, K, tile_n, tile_k, state_bits)
+        hist = ans.ans_histogram_host(w, lay)
+        assert np.array_equal(hist, oracle.histogram(dtype, w, N * K)), trial
+        cb = ans.ans_build_codebook(hist, ans.ALPHABET[dtype], 12)
+        stream, offsets, raw = ans.ans_encode_tiles(w, lay, cb)
+        st, s_or, off_or, raw_or = oracle.encode(dtype, w, N, K, tile_n, tile_k, cb.freq_array(),
+                                                 state_bits=state_bits)
+        assert st == 0, trial
+        assert np.array_equal(stream, s_or) and np.array_equal(offsets, off_or), trial
+        if raw is not None:
+            assert np.array_equal(raw, raw_or), trial
+        st, out = oracle.decode(dtype, stream, offsets, raw, N, K, tile_n, tile_k,
+                                cb.freq_array(), state_bits=state_bits)
+        assert st == 0 and np.array_equal(out, w), trial
