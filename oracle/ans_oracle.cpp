@@ -52,6 +52,12 @@
 // codes stored like int4 (two per byte, element k even in the low nibble),
 // symbol = the code (alphabet 16), value e2m1 times an optional per-row scale.
 //
+// bf16 whole (dtype 7; [SB] s4.1 implies bf16 coded as 16-bit symbols): the
+// 16-bit pattern is the symbol (alphabet 65536, probability precision up to
+// n = 16); the wide-state pair bound is 2^(64 - 2n) f_a f_b, so it holds for
+// n = 16 as well (two steps from x >= 2^32 leave x >= 1, and one 32-bit word
+// restores x >= 2^32).
+//
 // fp4 pairs (dtype 6): fp4 codes coded one symbol per packed byte, the byte
 // itself (alphabet 256), in the int4 pairs' lane map.
 //
@@ -85,7 +91,8 @@ enum {
   DT_INT4_PAIRS = 3,
   DT_INT8 = 4,
   DT_FP4_E2M1 = 5,
-  DT_FP4_PAIRS = 6
+  DT_FP4_PAIRS = 6,
+  DT_BF16_WHOLE = 7
 };
 enum { SC_NONE = 0, SC_ROW_BF16 = 1, SC_ROW_F32 = 2, SC_GROUP_BF16 = 3 };
 enum {
@@ -99,7 +106,10 @@ const uint32_t kWordBits = 16;       // renormalisation word width (b = 2^16)
 const uint64_t kLWide = 1ull << 32;  // wide variant: lower bound of the state interval
 const uint32_t kWideWordBits = 32;   // wide variant: renormalisation word width (b = 2^32)
 
-int alphabet_of(int dtype) { return (dtype == DT_INT4 || dtype == DT_FP4_E2M1) ? 16 : 256; }
+int alphabet_of(int dtype) {
+  if (dtype == DT_BF16_WHOLE) return 65536;
+  return (dtype == DT_INT4 || dtype == DT_FP4_E2M1) ? 16 : 256;
+}
 // packed two per byte, element k even in the low nibble
 bool is_nibble(int dtype) {
   return dtype == DT_INT4 || dtype == DT_INT4_PAIRS || dtype == DT_FP4_E2M1 || dtype == DT_FP4_PAIRS;
@@ -145,6 +155,7 @@ uint32_t symbol_at(int dtype, const void* w, uint64_t idx) {
   // int8: two's complement code q in [-128, 127]; symbol q + 128 (the byte
   // with its top bit flipped)
   if (dtype == DT_INT8) return (uint32_t)((int)(int8_t)((const uint8_t*)w)[idx] + 128);
+  if (dtype == DT_BF16_WHOLE) return ((const uint16_t*)w)[idx];  // the whole 16-bit pattern
   if (dtype == DT_BF16_SPLIT) {
     uint16_t bits = ((const uint16_t*)w)[idx];
     return (bits >> 7) & 0xFFu;
@@ -215,7 +226,7 @@ struct Codebook {
 };
 
 int make_codebook(const uint32_t* freq, int A, int prob_bits, Codebook* cb) {
-  if (prob_bits < 1 || prob_bits > 16 || A < 1 || A > 256) return ERR_ARG;
+  if (prob_bits < 1 || prob_bits > 16 || A < 1 || A > 65536) return ERR_ARG;
   cb->n = (uint32_t)prob_bits;
   cb->M = 1u << prob_bits;
   cb->f.assign(freq, freq + A);
@@ -254,11 +265,12 @@ uint64_t decode_symbol(uint64_t x, const Codebook& cb, int* sym) {
 }
 
 // Wide variant, one pair (a = the earlier symbol, b = the later one) coded in
-// reverse: push one 32-bit word if x >= 2^40 f_a f_b (compared in 128 bits:
-// the bound is 2^64 when f_a = f_b = 4096), then code b, then a.
+// reverse: push one 32-bit word if x >= 2^(64 - 2n) f_a f_b (2^40 f_a f_b for
+// n = 12; compared in 128 bits: the bound is 2^64 when f_a = f_b = M), then
+// code b, then a.
 uint64_t encode_pair_wide(uint64_t x, uint32_t fa, uint32_t ca, uint32_t fb, uint32_t cb_,
                           const Codebook& cb, std::vector<uint32_t>* pushed) {
-  unsigned __int128 x_max = ((unsigned __int128)fa * fb) << 40;
+  unsigned __int128 x_max = ((unsigned __int128)fa * fb) << (64 - 2 * cb.n);
   if ((unsigned __int128)x >= x_max) {
     pushed->push_back((uint32_t)(x & 0xFFFFFFFFull));
     x >>= kWideWordBits;
@@ -445,10 +457,14 @@ double oracle_entropy(const uint64_t* counts, int A) {
 // while a move still lowers the cost.  Ties go to the lower symbol index.
 // Gains are evaluated as c * log2l((f + 1.0L) / f) in long double.
 int oracle_normalize(const uint64_t* counts, int A, int prob_bits, uint32_t* freq) {
-  if (A < 1 || A > 256 || prob_bits < 1 || prob_bits > 16) return ERR_ARG;
+  if (A < 1 || A > 65536 || prob_bits < 1 || prob_bits > 16) return ERR_ARG;
   const uint64_t M = 1ull << prob_bits;
   uint64_t total = 0, present = 0;
   for (int s = 0; s < A; ++s) { total += counts[s]; present += counts[s] > 0; }
+  // the loops below visit the present symbols only, in increasing order
+  std::vector<int> live;
+  for (int s = 0; s < A; ++s)
+    if (counts[s] > 0) live.push_back(s);
   if (total == 0) return ERR_ARG;
   if (present > M) return ERR_ALPHABET;
   std::vector<uint64_t> f(A, 0);
@@ -467,25 +483,25 @@ int oracle_normalize(const uint64_t* counts, int A, int prob_bits, uint32_t* fre
   };
   while (sum < M) {
     int best = -1;
-    for (int s = 0; s < A; ++s)
-      if (counts[s] > 0 && (best < 0 || gain(s) > gain(best))) best = s;
+    for (int s : live)
+      if (best < 0 || gain(s) > gain(best)) best = s;
     f[best]++;
     sum++;
   }
   while (sum > M) {
     int best = -1;
-    for (int s = 0; s < A; ++s)
-      if (counts[s] > 0 && f[s] > 1 && (best < 0 || loss(s) < loss(best))) best = s;
+    for (int s : live)
+      if (f[s] > 1 && (best < 0 || loss(s) < loss(best))) best = s;
     f[best]--;
     sum--;
   }
   for (;;) {
     int up = -1;
-    for (int s = 0; s < A; ++s)
-      if (counts[s] > 0 && (up < 0 || gain(s) > gain(up))) up = s;
+    for (int s : live)
+      if (up < 0 || gain(s) > gain(up)) up = s;
     int down = -1;
-    for (int s = 0; s < A; ++s)
-      if (s != up && counts[s] > 0 && f[s] > 1 && (down < 0 || loss(s) < loss(down))) down = s;
+    for (int s : live)
+      if (s != up && f[s] > 1 && (down < 0 || loss(s) < loss(down))) down = s;
     if (up < 0 || down < 0 || !(gain(up) > loss(down))) break;
     f[up]++;
     f[down]--;
@@ -628,10 +644,10 @@ int oracle_encode(int dtype, const void* w, uint32_t N, uint32_t K, uint32_t til
                   uint32_t tile_k, const uint32_t* freq, int prob_bits, uint8_t* stream,
                   uint64_t cap, uint64_t* stream_bytes, uint64_t* offsets, uint8_t* raw,
                   int threads, int state_bits) {
-  if (dtype < 0 || dtype > 6) return ERR_ARG;
+  if (dtype < 0 || dtype > 7) return ERR_ARG;
   if (state_bits != 32 && state_bits != 64) return ERR_ARG;
   if (!layout_ok(N, K, tile_n, tile_k)) return ERR_SHAPE;
-  if (state_bits == 64 && prob_bits != 12) return ERR_ARG;  // the pair bound assumes n = 12
+  if (state_bits == 64 && prob_bits != 12 && prob_bits != 16) return ERR_ARG;  // pair bound: n = 12 or 16
   Codebook cb;
   int st = make_codebook(freq, alphabet_of(dtype), prob_bits, &cb);
   if (st != OK) return st;
@@ -666,10 +682,10 @@ int oracle_decode(int dtype, const uint8_t* stream, uint64_t stream_bytes,
                   uint32_t tile_n, uint32_t tile_k, const uint32_t* freq, int prob_bits,
                   void* w_out, uint64_t tile_begin, uint64_t tile_end, int threads,
                   int state_bits) {
-  if (dtype < 0 || dtype > 6) return ERR_ARG;
+  if (dtype < 0 || dtype > 7) return ERR_ARG;
   if (state_bits != 32 && state_bits != 64) return ERR_ARG;
   if (!layout_ok(N, K, tile_n, tile_k)) return ERR_SHAPE;
-  if (state_bits == 64 && prob_bits != 12) return ERR_ARG;
+  if (state_bits == 64 && prob_bits != 12 && prob_bits != 16) return ERR_ARG;
   Codebook cb;
   int st = make_codebook(freq, alphabet_of(dtype), prob_bits, &cb);
   if (st != OK) return st;
@@ -729,6 +745,8 @@ int oracle_decode(int dtype, const uint8_t* stream, uint64_t stream_bytes,
           else out[idx / 2] = (uint8_t)((out[idx / 2] & 0x0F) | (nib << 4));
         } else if (dtype == DT_INT8) {
           ((uint8_t*)w_out)[idx] = (uint8_t)(int8_t)(s - 128);
+        } else if (dtype == DT_BF16_WHOLE) {
+          ((uint16_t*)w_out)[idx] = (uint16_t)s;
         } else if (dtype == DT_BF16_SPLIT) {
           uint8_t r = raw[t * lay.tile_symbols() + (j / 8) * 256 + l * 8 + (j % 8)];
           ((uint16_t*)w_out)[idx] = bf16_from_parts((uint32_t)s, r);
@@ -761,7 +779,7 @@ int oracle_decode(int dtype, const uint8_t* stream, uint64_t stream_bytes,
 int oracle_gemm(int dtype, const uint16_t* X, uint32_t M, uint32_t K, const void* W,
                 uint32_t N, int scale_kind, const void* scales, uint32_t group_k,
                 const uint32_t* rows, uint32_t n_rows, double* Y, int threads) {
-  if (dtype < 0 || dtype > 6) return ERR_ARG;
+  if (dtype < 0 || dtype > 7) return ERR_ARG;
   if (scale_kind == SC_GROUP_BF16 && (group_k == 0 || K % group_k != 0)) return ERR_ARG;
   if (scale_kind != SC_NONE && scales == nullptr) return ERR_ARG;
   if (rows == nullptr) n_rows = N;
@@ -788,7 +806,7 @@ int oracle_gemm(int dtype, const uint16_t* X, uint32_t M, uint32_t K, const void
         v = (double)(int8_t)((const uint8_t*)W)[idx];
         if (scale_kind == SC_ROW_F32) v *= f32_value(scales, n);
         else if (scale_kind == SC_ROW_BF16) v *= bf16_value(((const uint16_t*)scales)[n]);
-      } else if (dtype == DT_BF16_SPLIT) {
+      } else if (dtype == DT_BF16_SPLIT || dtype == DT_BF16_WHOLE) {
         v = bf16_value(((const uint16_t*)W)[idx]);
         if (scale_kind == SC_ROW_BF16) v *= bf16_value(((const uint16_t*)scales)[n]);
         else if (scale_kind == SC_ROW_F32) v *= f32_value(scales, n);

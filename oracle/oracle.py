@@ -17,7 +17,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "ans_oracle.cpp")
 LIB = os.path.join(HERE, "liboracle.so")
 
-INT4, BF16_SPLIT, FP8_E4M3, INT4_PAIRS, INT8, FP4_E2M1, FP4_PAIRS = 0, 1, 2, 3, 4, 5, 6
+INT4, BF16_SPLIT, FP8_E4M3, INT4_PAIRS, INT8, FP4_E2M1, FP4_PAIRS, BF16_WHOLE = 0, 1, 2, 3, 4, 5, 6, 7
 SCALE_NONE, SCALE_ROW_BF16, SCALE_ROW_F32, SCALE_GROUP_BF16 = 0, 1, 2, 3
 OK, ERR_ARG, ERR_SHAPE, ERR_ALPHABET, ERR_BUFFER_TOO_SMALL, ERR_CORRUPT = 0, 1, 2, 3, 4, 6
 
@@ -199,7 +199,7 @@ def decode(dtype, stream, offsets, raw, N, K, tile_n, tile_k, freq, prob_bits=12
     if out is None:
         if dtype in (INT4, INT4_PAIRS, FP4_E2M1, FP4_PAIRS):
             out = np.zeros(N * K // 2, np.uint8)
-        elif dtype == BF16_SPLIT:
+        elif dtype in (BF16_SPLIT, BF16_WHOLE):
             out = np.zeros(N * K, np.uint16)
         else:
             out = np.zeros(N * K, np.uint8)

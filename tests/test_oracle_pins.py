@@ -662,6 +662,63 @@ def test_fp4_pairs_identity_marginals_and_gemm(oracle, state_bits):
     assert np.array_equal(Yp, Y1)
 
 
+# ---- bf16 as whole 16-bit symbols (probability precision 2^16) ---------------------
+def test_bf16_whole_symbol_is_the_pattern(oracle):
+    counts = oracle.histogram(WL.BF16_WHOLE, np.arange(65536, dtype=np.uint16), 65536)
+    assert counts.size == 65536 and (counts == 1).all()
+
+
+@pytest.mark.parametrize("state_bits", [32, 64])
+def test_bf16_whole_equiprobable_closed_form(oracle, state_bits):
+    # f = 1 for all 65536 symbols at n = 16: coding s is x -> x * 2^16 + s.
+    # Narrow states start at 2^16, always give up their low 16 bits first and
+    # end at 2^16 + s_0; wide states start at 2^32, give up their low 32 bits
+    # before each pair and end at 2^32 + s_1 * 2^16 + s_0: one word per symbol
+    # or per pair, 2 bytes per symbol either way.
+    N, K = 128, 64
+    rng = np.random.default_rng(21)
+    w = rng.integers(0, 65536, size=N * K).astype(np.uint16)
+    freq = np.ones(65536, np.uint32)
+    st, stream, offsets, _ = oracle.encode(WL.BF16_WHOLE, w, N, K, 128, 64, freq, prob_bits=16,
+                                           state_bits=state_bits)
+    assert st == 0
+    sb = state_bits // 8
+    assert int(offsets[1]) == 32 * sb + 2 * N * K
+    states = np.frombuffer(stream[:32 * sb].tobytes(), np.uint32 if sb == 4 else np.uint64)
+    w2 = w.reshape(N, K).astype(np.uint64)
+    # lane l's first two symbols are row l, columns 0 and 1
+    expect = (1 << 16) + w2[:32, 0] if sb == 4 else (1 << 32) + (w2[:32, 1] << 16) + w2[:32, 0]
+    assert np.array_equal(states.astype(np.uint64), expect)
+    st, out = oracle.decode(WL.BF16_WHOLE, stream, offsets, None, N, K, 128, 64, freq,
+                            prob_bits=16, state_bits=state_bits)
+    assert st == 0 and np.array_equal(out, w)
+
+
+@pytest.mark.parametrize("state_bits,band", [(32, 0.25), (64, 0.35)])
+def test_bf16_whole_identity_size_and_gemm(oracle, state_bits, band):
+    cfg, d = _small("bf16_4096", 512, 1024)
+    w = d["w"]
+    counts = oracle.histogram(WL.BF16_WHOLE, w, w.size)
+    H16 = oracle.entropy(counts)
+    st, freq = oracle.normalize(counts, 16)
+    assert st == 0 and freq.sum() == 65536 and ((freq > 0) == (counts > 0)).all()
+    st, stream, offsets, raw = oracle.encode(WL.BF16_WHOLE, w, 512, 1024, 128, 64, freq,
+                                             prob_bits=16, state_bits=state_bits)
+    assert st == 0 and raw is None
+    st, out = oracle.decode(WL.BF16_WHOLE, stream, offsets, None, 512, 1024, 128, 64, freq,
+                            prob_bits=16, state_bits=state_bits)
+    assert st == 0 and np.array_equal(out, w)
+    gap = 8.0 * stream.size / w.size - H16
+    assert -0.01 < gap < band, gap
+    # the whole-value entropy is at most the split bound H(exponent) + 8
+    He = oracle.entropy(oracle.histogram(WL.BF16_SPLIT, w, w.size))
+    assert H16 <= He + 8 + 1e-9
+    X = WL.to_bf16_bits(np.random.default_rng(3).standard_normal((2, 1024)))
+    rows = np.arange(0, 512, 53, dtype=np.uint32)
+    assert np.array_equal(oracle.gemm(WL.BF16_WHOLE, X, 2, 1024, w, 512, rows=rows),
+                          oracle.gemm(WL.BF16_SPLIT, X, 2, 1024, w, 512, rows=rows))
+
+
 # ---- fp64 GEMM ------------------------------------------------------------------
 def test_gemm_int4_exact_integers(oracle):
     rng = np.random.default_rng(2)
