@@ -202,3 +202,23 @@ def test_host_codec_matches_oracle_fuzzed(oracle, ans_lib):
         st, out = oracle.decode(dtype, stream, offsets, raw, N, K, tile_n, tile_k,
                                 cb.freq_array(), state_bits=state_bits)
         assert st == 0 and np.array_equal(out, w), trial
+
+
+def test_dtype_constants_agree_with_the_header():
+    # the binding's dtype, scale and status constants are the header's values
+    text = open(os.path.join(ROOT, "include", "ans.h")).read()
+    enum = dict((k, int(v)) for k, v in re.findall(r"\b(ANS_[A-Z0-9_]+)\s*=\s*(\d+)", text))
+    assert enum["ANS_INT4"] == ans.INT4 and enum["ANS_BF16_SPLIT"] == ans.BF16_SPLIT
+    assert enum["ANS_FP8_E4M3"] == ans.FP8_E4M3 and enum["ANS_INT4_PAIRS"] == ans.INT4_PAIRS
+    assert enum["ANS_INT8"] == ans.INT8 and enum["ANS_FP4_E2M1"] == ans.FP4_E2M1
+    assert enum["ANS_FP4_PAIRS"] == ans.FP4_PAIRS
+    assert enum["ANS_SCALE_GROUP_BF16"] == ans.SCALE_GROUP_BF16
+    assert enum["ANS_SCALE_ROW_F32"] == ans.SCALE_ROW_F32
+    flags = dict((k, int(v, 16)) for k, v in re.findall(r"#define\s+(ANS_STATUS_[A-Z_]+)\s+0x([0-9a-fA-F]+)u", text))
+    assert flags["ANS_STATUS_CORRUPT"] == ans.STATUS_CORRUPT
+    assert flags["ANS_STATUS_TIMEOUT"] == ans.STATUS_TIMEOUT
+    assert flags["ANS_STATUS_BAD_OFFSETS"] == ans.STATUS_BAD_OFFSETS
+    assert int(re.search(r"#define\s+ANS_MAX_BATCH\s+(\d+)", text).group(1)) == ans.MAX_BATCH
+    # the workload generators use the same dtype numbers
+    assert (WL.INT4, WL.BF16_SPLIT, WL.FP8_E4M3, WL.INT4_PAIRS, WL.INT8, WL.FP4_E2M1,
+            WL.FP4_PAIRS) == (0, 1, 2, 3, 4, 5, 6)
