@@ -377,6 +377,30 @@ ans_status ans_gemm_noalloc(const uint16_t* d_X, uint32_t M, const ans_tiles* W,
 // Internal profiling hook (not part of the public ABI in include/ans.h).
 void ansdev_set_trace(void* d_buf, size_t bytes) { ansdev::set_trace_buffer(d_buf, bytes); }
 
+// Internal test hook (not part of the public ABI): the launch plan that
+// ans_gemm (decode = 1) or ans_gemm_uncompressed (decode = 0) would use for a
+// layout, M and scale kind on a device with num_sms SMs, without touching a
+// device.  out[0..19] = local, grid, D, n_slots, tmem_cols, smem_bytes, T,
+// T_pass, n_pass, NT, n_bufs, fmt, ab_f16, H, C, x_stages, n_units,
+// n_segments, ws_bytes (low 32 bits), ws_bytes (high 32 bits).  Returns 1 if
+// the shape can be scheduled, 0 if not, -1 for a bad layout.
+int ansdev_gemm_plan(const ans_layout* layout, uint32_t M, uint32_t scale_kind, int decode,
+                     int num_sms, uint32_t* out) {
+  if (check_layout(layout) != ANS_OK || !out) return -1;
+  ansdev::LayerDev L;
+  fill_layer_plain(layout, &L);
+  L.wide = layout->state_bits == 64 ? 1u : 0u;
+  ansdev::GemmPlan p;
+  if (!ansdev::make_gemm_plan(L, M, scale_kind, decode != 0, num_sms, &p)) return 0;
+  const uint32_t v[20] = {p.local, p.grid, p.D, p.n_slots, p.tmem_cols, p.smem_bytes, p.T,
+                          p.T_pass, p.n_pass, p.NT, p.n_bufs, p.fmt, p.ab_f16, p.H, p.C,
+                          p.x_stages, static_cast<uint32_t>(p.n_units), p.n_segments,
+                          static_cast<uint32_t>(p.ws_bytes),
+                          static_cast<uint32_t>(static_cast<uint64_t>(p.ws_bytes) >> 32)};
+  for (int i = 0; i < 20; ++i) out[i] = v[i];
+  return 1;
+}
+
 }  // extern "C"
 
 namespace {
