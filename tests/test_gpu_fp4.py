@@ -1,8 +1,10 @@
-"""GPU parity of fp4 e2m1 weights (symbol = the code, per-row fp32 scale, MMA in bf16):
-GPU histogram equal to the oracle's, standalone decode bit-exact and equal to
-the oracle's decode of the same stream, fused GEMM bit-identical to the
-uncompressed variant and within 1e-3 relative Frobenius error of the fp64
-oracle, in both schedules and both stream formats, alone and batched."""
+"""GPU parity of fp4 e2m1 weights (per-row fp32 scale, MMA in bf16), coded one
+symbol per code or one per packed byte (pair symbols): GPU histogram equal to
+the oracle's, standalone decode bit-exact and equal to the oracle's decode of
+the same stream, fused GEMM bit-identical to the uncompressed variant (and,
+for pair symbols, to the per-code coding) and within 1e-3 relative Frobenius
+error of the fp64 oracle, in both schedules and both stream formats.  The
+batched launch of fp4 layers is tested in test_gpu_batched.py."""
 import numpy as np
 import pytest
 import torch

@@ -2,7 +2,8 @@
 GPU histogram equal to the oracle's, standalone decode bit-exact and equal to
 the oracle's decode of the same stream, fused GEMM bit-identical to the
 uncompressed variant and within 1e-3 relative Frobenius error of the fp64
-oracle, in both schedules and both stream formats, alone and batched."""
+oracle, in both schedules and both stream formats.  The batched launch of int8
+layers is tested in test_gpu_batched.py."""
 import numpy as np
 import pytest
 import torch
