@@ -1,14 +1,19 @@
 #!/usr/bin/env python3
 """Benchmark of the fused tile-rANS decode + GEMM on one B200 per rank.
 
-Workload (the layer the headline metric is quoted on): a 4096 x 4096 bf16
-weight matrix drawn from N(0, 0.02), coded as an rANS exponent stream (one
-12-bit codebook, 128 x 64 tiles, 32 lanes; by default the wide-state stream
-format, --state-bits 32 for 32-bit lane states) plus the raw sign/mantissa byte,
-multiplied by X (16 x 4096 bf16, N(0, 1)).  One step is one ans_gemm call
-(decode inside the GEMM, Y fp32).  Twelve copies of the compressed layer
-(together far larger than the 126 MB L2) rotate across steps, so every step
-reads its weights from HBM.
+Headline workload (the largest layer of the pages' workloads that fits one
+GPU): a 53248 x 16384 fp8 e4m3 weight matrix shaped like a Llama-405B
+projection (w ~ N(0, 0.02), per-row absmax scale amax/448 stored fp32),
+coded as one rANS stream of 8-bit symbols per 128 x 128 tile (one 12-bit
+codebook per layer, 32 lanes; by default the wide-state stream format,
+--state-bits 32 for 32-bit lane states), multiplied by X (16 x 16384 bf16,
+N(0, 1)).  One step is one ans_gemm call (decode inside the GEMM, fp32 Y).
+The compressed layer (~0.7 GB, two copies alternating) is far larger than
+the 126 MB L2, so every step reads its weights from HBM.
+
+A secondary entry times the bf16 4096 x 4096 split-stream layer at M = 16
+(exponent coded per 128 x 64 tile, raw sign/mantissa byte), twelve rotating
+copies in CUDA graphs of consecutive calls.
 
 Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle on
 the same workload instead.  Under torchrun every rank runs its own replica
@@ -18,6 +23,7 @@ over ranks.
 from __future__ import annotations
 
 import argparse
+import datetime
 import hashlib
 import json
 import os
@@ -32,45 +38,62 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-WORKLOAD = "bf16_4096"
+WORKLOAD = "fp8_405b"
 M_HEAD = 16
-N_COPIES = 12
+HEAD_COPIES = 2
+SECOND = "bf16_4096"
+SECOND_COPIES = 12
+METRIC = ("fused decode-GEMM effective weight GB/s (405B-shaped fp8 e4m3 layer "
+          "53248x16384, M=16)")
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
-# sources of the kernel the bench times at M=16 (the local schedule); the
+# nominal storage bytes per weight of the decompressed layer
+NOMINAL = {0: 0.5, 1: 2.0, 2: 1.0, 3: 0.5, 4: 1.0, 5: 0.5, 6: 0.5}
+# sources of the kernel the bench times at M = 16 (the local schedule); the
 # committed DRAM-traffic summary is only used while they are unchanged
 KERNEL_SOURCES = ["rans_decode_gemm_b200/csrc/cuda/gemm_local.cu",
                   "rans_decode_gemm_b200/csrc/cuda/gemm_common.cuh",
                   "rans_decode_gemm_b200/csrc/cuda/rans_core.cuh",
                   "rans_decode_gemm_b200/csrc/cuda/ptx.cuh",
                   "rans_decode_gemm_b200/csrc/cuda/launch.h"]
+TRAFFIC_PROFILE = "profiles/fused_gemm_local_fp8_405b_m16.json"
 
 
-def workload_name(state_bits):
+def workload_name(name, state_bits, M):
     fmt = ("64-bit lane states, 32-bit words, one renormalisation test per symbol pair"
            if state_bits == 64 else "32-bit lane states, 16-bit words")
+    if name == "fp8_405b":
+        return ("405B-shaped fp8 e4m3 53248x16384, w~N(0,0.02) / (row amax/448), fp32 row "
+                "scales, 8-bit symbols, 128x128 tiles, 32 lanes, 12-bit freqs, "
+                f"{fmt}; X {M}x16384 bf16 N(0,1); seed 4")
     return ("bf16 split-stream 4096x4096 N(0,0.02), 128x64 tiles, 32 lanes, 12-bit freqs, "
-            f"{fmt}; X 16x4096 bf16 N(0,1); seed 1")
+            f"{fmt}; X {M}x4096 bf16 N(0,1); seed 1")
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10000)
-    ap.add_argument("--warmup", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true",
                     help="every workload of the pages at full size, one JSON line per point "
                          "(instead of the benchmark line)")
     ap.add_argument("--sweep-configs", default="", help="comma-separated subset for --sweep")
+    ap.add_argument("--sweep-ms", default="", help="comma-separated token counts for --sweep "
+                                                   "(default: each workload's own)")
     ap.add_argument("--state-bits", type=int, default=64, choices=[32, 64],
                     help="stream format: 64 = wide lane states (32-bit words, one "
                          "renormalisation test per symbol pair), 32 = 32-bit states")
     ap.add_argument("--nibble-symbols", default="pairs", choices=["pairs", "element"],
                     help="--sweep: code int4 and fp4 weights one symbol per packed byte "
                          "(two K elements) or one per element")
+    ap.add_argument("--rows", type=int, default=0,
+                    help="profiling: the headline layer cut to its first ROWS rows (a "
+                         "multiple of 128); 0 = the whole layer")
     ap.add_argument("--quick", action="store_true",
-                    help="skip the context sweep and the CPU baseline (profiling runs)")
+                    help="only the headline timing: no context sweep, secondary entry or "
+                         "CPU baseline (profiling runs)")
     return ap.parse_args()
 
 
@@ -91,9 +114,9 @@ def kernel_source_hash() -> str:
 
 
 def profiled_traffic():
-    """dram read+write bytes per launch of the fused kernel from the committed
-    ncu summary, if it was taken on the current kernel source."""
-    path = os.path.join(ROOT, "profiles", "fused_gemm_bf16_4096_m16.json")
+    """dram read+write bytes per launch of the headline kernel from the
+    committed ncu summary, if it was taken on the current kernel source."""
+    path = os.path.join(ROOT, TRAFFIC_PROFILE)
     if not os.path.exists(path):
         return None
     with open(path) as fh:
@@ -103,29 +126,64 @@ def profiled_traffic():
     return d.get("dram_bytes_per_launch")
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling during the timed region."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi clock / throttle sampling (20 ms period, host timestamps),
+    started before the warm-up; the samples that fall inside the timed window
+    are reported separately from those of the whole loaded window."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
         self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.window = None
 
-    def start(self):
+    def start(self, wait_s: float = 3.0):
+        """Starts the sampler and returns once its first sample is written."""
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=self.file, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
+            return
+        t_end = time.time() + wait_s
+        while time.time() < t_end:
+            if os.path.getsize(self.file.name) > 0:
+                break
+            time.sleep(0.01)
+
+    def mark(self, t0: float, t1: float):
+        """Host-time bounds of the timed region."""
+        self.window = (t0, t1)
+
+    @staticmethod
+    def _ts(s: str):
+        for fmt in ("%Y/%m/%d %H:%M:%S.%f", "%Y/%m/%d %H:%M:%S"):
+            try:
+                return datetime.datetime.strptime(s, fmt).timestamp()
+            except ValueError:
+                pass
+        return None
 
     def stop(self):
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -136,19 +194,37 @@ class ClockSampler:
         with open(self.file.name) as fh:
             for line in fh:
                 parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9:
+                if len(parts) >= 10:
                     rows.append(parts)
         os.unlink(self.file.name)
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+
+        timed = []
+        if self.window is not None:
+            a, b = self.window
+            for r in rows:
+                t = self._ts(r[0])
+                if t is not None and a - 0.02 <= t <= b + 0.02:
+                    timed.append(r)
+        use = timed if timed else rows
+        sm = [v for v in (num(r[2]) for r in use) if v is not None]
+        smax = [v for v in (num(r[3]) for r in rows) if v is not None]
+        reasons = sorted({n for r in use for n, v in zip(self.REASONS, r[6:10])
+                          if v.lower() == "active"})
         under_load = sorted(sm)[len(sm) // 2:] if sm else []
         return {"sm_mhz": statistics.median(under_load) if under_load else None,
                 "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
-                "samples": len(rows)}
+                "samples": len(use), "samples_in_timed_region": len(timed),
+                "samples_total": len(rows), "period_ms": 20,
+                "window": "timed region" if timed else
+                          "warm-up and timed region (no sample fell inside the timed region)"}
 
 
 def dist_setup(args):
@@ -177,21 +253,51 @@ def replica_gbs(world, bytes_per_step, ms_per_step):
     return world * bytes_per_step / (ms_per_step * 1e-3) / 1e9
 
 
-def build_layers(torch, ans, WL, device, state_bits):
-    cfg = WL.CONFIGS[WORKLOAD]
-    d = WL.make_weights(cfg, 0)
+def percentiles(vals):
+    v = sorted(vals)
+    if not v:
+        return None
+
+    def q(p):
+        return v[min(len(v) - 1, max(0, int(round(p * (len(v) - 1)))))]
+    return {"p10": round(q(0.10), 6), "p50": round(q(0.50), 6), "p90": round(q(0.90), 6),
+            "n": len(v)}
+
+
+def build_layers(torch, ans, WL, name, device, state_bits, copies, rows=0):
+    """Offline path through the library (GPU histogram -> codebook -> host
+    encode), then `copies` device copies of the compressed layer (its first
+    `rows` rows when rows > 0)."""
+    cfg = WL.CONFIGS[name]
+    d = WL.make_weights(cfg, 0, N=rows if rows else None)
     lay = ans.make_layout(cfg.dtype, d["N"], d["K"], cfg.tile_n, cfg.tile_k, state_bits)
-    # offline path through the library: GPU histogram -> codebook -> host encode
-    dw = torch.from_numpy(d["w"].view(np.int16)).to(device)
-    hist = torch.zeros(256, dtype=torch.int64, device=device)
+    w = d["w"]
+    dw = torch.from_numpy(w.view(np.int16) if w.dtype == np.uint16 else w).to(device)
+    A = ans.ALPHABET[cfg.dtype]
+    hist = torch.zeros(A, dtype=torch.int64, device=device)
     ans.ans_histogram(dw, lay, hist)
     hist_h = hist.cpu().numpy().astype(np.uint64)
     t0 = time.perf_counter()
-    cb = ans.ans_build_codebook(hist_h, 256, 12)
-    stream, offsets, raw = ans.ans_encode_tiles(d["w"], lay, cb)
+    cb = ans.ans_build_codebook(hist_h, A, 12)
+    stream, offsets, raw = ans.ans_encode_tiles(w, lay, cb)
     encode_s = time.perf_counter() - t0
-    layers = [ans.CompressedLayer(lay, cb, stream, offsets, raw, device) for _ in range(N_COPIES)]
-    return cfg, d, lay, layers, hist_h, encode_s, dw
+    layers = [ans.CompressedLayer(lay, cb, stream, offsets, raw, device) for _ in range(copies)]
+    sc = None
+    if d["scales"] is not None:
+        s = np.ascontiguousarray(d["scales"])
+        sc = torch.from_numpy(s.view(np.int16) if s.dtype == np.uint16 else s).to(device)
+    return cfg, d, lay, layers, hist_h, encode_s, dw, sc
+
+
+def algo_bytes(layer, cfg, M, N, K):
+    """Bytes one ans_gemm call must move at the least: the compressed layer,
+    the scales, X in and Y out."""
+    sbytes = 0
+    if cfg.scale_kind in (1, 3):
+        sbytes = 2 * N * (K // cfg.group_k if cfg.scale_kind == 3 else 1)
+    elif cfg.scale_kind == 2:
+        sbytes = 4 * N
+    return layer.compressed_bytes + sbytes + 2 * M * K + 4 * M * N
 
 
 def time_ours(args):
@@ -204,25 +310,25 @@ def time_ours(args):
     device = torch.device("cuda", local)
     pg = None
     if world > 1:
-        import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=device)
         pg = dist
-    cfg, d, lay, layers, hist, encode_s, dw = build_layers(torch, ans, WL, device, args.state_bits)
+    cfg, d, lay, layers, hist, encode_s, dw, sc = build_layers(
+        torch, ans, WL, WORKLOAD, device, args.state_bits, HEAD_COPIES, args.rows)
     N, K, M = lay.N, lay.K, M_HEAD
     X_h = WL.make_x(cfg, M, K)
     X = torch.from_numpy(X_h.view(np.int16)).to(device)
     Y = torch.empty(M, N, dtype=torch.float32, device=device)
     ws_bytes = ans.ans_gemm_workspace(lay, M, cfg.scale_kind)
-    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=device)
+    ws = torch.zeros(max(ws_bytes, 256), dtype=torch.uint8, device=device)
     st = torch.zeros(1, dtype=torch.int32, device=device)
     stream = torch.cuda.Stream(device=device)
     torch.cuda.set_stream(stream)
 
     def step(i):
-        ans.ans_gemm(X, M, layers[i % N_COPIES].tiles, cfg.scale_kind, None, 0, Y, ws,
-                     ws_bytes, st, stream)
+        ans.ans_gemm(X, M, layers[i % HEAD_COPIES].tiles, cfg.scale_kind, sc, cfg.group_k, Y, ws,
+                     ws.numel(), st, stream)
 
     def barrier():
         torch.cuda.synchronize()
@@ -230,48 +336,29 @@ def time_ours(args):
             pg.barrier()
         torch.cuda.synchronize()
 
-    # The steps are captured as CUDA graphs of consecutive calls, one call per
-    # rotating layer copy (what an inference engine does with a stack of
-    # layers), so the timed region measures the GPU work rather than Python /
-    # ctypes launch cost, and consecutive kernels may overlap their prologue
-    # with the previous kernel's tail (programmatic dependent launch).  A
-    # second graph holds the remainder, so exactly `steps` calls are timed.
-    for i in range(N_COPIES):          # eager warm-up: first-call attributes
-        step(i)
-    torch.cuda.synchronize()
-
-    def capture(n):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for i in range(n):
-                step(i)
-        return g
-
-    g_full = capture(N_COPIES)
-    rem = args.steps % N_COPIES
-    g_rem = capture(rem) if rem else None
-    torch.cuda.synchronize()
-
+    # Each call is about a millisecond of GPU work, so plain stream launches
+    # keep the GPU busy; an event before every call gives the per-call
+    # spread, the first and last events bracket the timed region.
     sampler = ClockSampler(local)
     sampler.start()
-    for i in range(max(1, (args.warmup + N_COPIES - 1) // N_COPIES)):
-        g_full.replay()
+    for i in range(args.warmup):
+        step(i)
     barrier()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for i in range(args.steps // N_COPIES):
-        g_full.replay()
-    if g_rem is not None:
-        g_rem.replay()
-    t1.record(stream)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    h0 = time.time()
+    ev[0].record(stream)
+    for i in range(args.steps):
+        step(i)
+        ev[i + 1].record(stream)
     barrier()
+    h1 = time.time()
+    sampler.mark(h0, h1)
     clocks = sampler.stop()
-    total_ms = t0.elapsed_time(t1)
+    total_ms = ev[0].elapsed_time(ev[-1])
+    per_call = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
     kern_ms = total_ms / args.steps
     status = int(st.item())
     total_ms, = max_over_ranks(pg, [total_ms], device)
-    del g_full, g_rem
 
     # e2e through the same C ABI with host buffers: pinned X in, Y out per step
     Xp = torch.from_numpy(X_h.view(np.int16)).pin_memory()
@@ -280,8 +367,8 @@ def time_ours(args):
 
     def e2e_step(i):
         Xd.copy_(Xp, non_blocking=True)
-        ans.ans_gemm(Xd, M, layers[i % N_COPIES].tiles, cfg.scale_kind, None, 0, Y, ws,
-                     ws_bytes, st, stream)
+        ans.ans_gemm(Xd, M, layers[i % HEAD_COPIES].tiles, cfg.scale_kind, sc, cfg.group_k, Y,
+                     ws, ws.numel(), st, stream)
         Yp.copy_(Y, non_blocking=True)
 
     for i in range(min(args.warmup, 20)):
@@ -289,7 +376,7 @@ def time_ours(args):
     barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    n_e2e = max(1, min(args.steps, 500))
+    n_e2e = max(1, min(args.steps, 200))
     e0.record(stream)
     for i in range(n_e2e):
         e2e_step(i)
@@ -297,49 +384,50 @@ def time_ours(args):
     barrier()
     e2e_ms, = max_over_ranks(pg, [e0.elapsed_time(e1) / n_e2e], device)
 
-    # context numbers on rank 0: other M, the two-pass baseline, uncompressed
     extra = {}
     if rank == 0 and not args.quick:
-        extra = context_numbers(torch, ans, WL, cfg, d, lay, layers, dw, device)
+        extra = context_numbers(torch, ans, WL, cfg, d, lay, layers, dw, sc, device, stream)
+        del dw
+        torch.cuda.empty_cache()
+        extra["secondary"] = secondary_entry(torch, ans, WL, args, device, stream)
 
     result = None
     if rank == 0:
         peaks, peaks_src = load_peaks()
-        weight_bytes = N * K * 2  # nominal bf16 storage of the decompressed weights
+        weight_bytes = N * K * NOMINAL[cfg.dtype]  # nominal storage of the decompressed weights
         layer = layers[0]
-        algo_bytes = layer.compressed_bytes + 2 * M * K + 4 * M * N
-        # launches per ans_gemm call: the local schedule (M <= 32 tokens per
-        # 128-row half) is one kernel; the shared-accumulator schedule stages X
-        # in a second one first
-        launches_per_step = 1 if ((M + 15) // 16 * 16) * (lay.tile_n // 128) <= 32 else 2
+        ab = algo_bytes(layer, cfg, M, N, K)
+        # the local schedule (M <= 32 tokens per 128-row half) is one kernel
+        launches_per_step = 1
         ms_per_step = total_ms / args.steps
         value = replica_gbs(world, weight_bytes, ms_per_step)
-        achieved = algo_bytes / (kern_ms * 1e-3) / 1e9
+        achieved = ab / (kern_ms * 1e-3) / 1e9
         peak = float(peaks["hbm_gbs"])
-        H_exp = ans.ans_entropy(hist)
+        H = ans.ans_entropy(hist)
         bpw = 8.0 * layer.compressed_bytes / (N * K)
         result = {
-            "metric": "fused decode-GEMM effective weight GB/s (bf16 weights, M=16)",
+            "metric": METRIC,
             "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": workload_name(args.state_bits),
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+            "config": {"workload": workload_name(WORKLOAD, args.state_bits, M) +
+                                   (f" (first {N} rows only)" if args.rows else ""),
                        "state_bits": args.state_bits,
                        "M": M, "N": N, "K": K, "global_batch": M * world,
                        "parallelism": f"replicas x{world}",
-                       "l2": f"inputs larger than L2: {N_COPIES} rotating copies of the "
-                             f"compressed layer ({N_COPIES * layer.compressed_bytes / 1e6:.0f} MB)"},
+                       "l2": f"inputs larger than L2: {HEAD_COPIES} alternating copies of the "
+                             f"compressed layer ({layer.compressed_bytes / 1e6:.0f} MB each)"},
+            "per_call_ms": percentiles(per_call),
             "bits_per_weight": round(bpw, 4),
-            "entropy_bits": {"exponent": round(H_exp, 4), "split_bound": round(H_exp + 8, 4)},
+            "entropy_bits": round(H, 4), "gap_bits": round(bpw - H, 4),
             "status": status,
             "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "traffic": profiled_traffic(), "peak_source": peaks_src,
-                         "algorithmic_bytes_per_launch": algo_bytes,
+                         "algorithmic_bytes_per_launch": ab,
                          "kernel_ms_per_launch": round(kern_ms, 6),
-                         "timing": "per-step time of the ans_gemm launch(es): CUDA graphs of "
-                                   f"{N_COPIES} consecutive calls (one per layer copy), events on "
-                                   "the launch stream"},
+                         "timing": "CUDA events on the launch stream around each ans_gemm "
+                                   "call (one kernel launch per call)"},
             "e2e": {"value": round(replica_gbs(world, weight_bytes, e2e_ms), 2), "unit": "GB/s",
                     "h2d_bytes_per_step": 2 * M * K, "d2h_bytes_per_step": 4 * M * N},
             "gpu_launches": launches_per_step * args.steps,
@@ -350,7 +438,6 @@ def time_ours(args):
         if "decode_tiles_Tsym_per_s" in extra:
             # the second ceiling: the rate at which the fused kernel decodes
             # symbols against the standalone decode kernel on the same layer
-            # (the per-tile rANS chain, not HBM or the tensor cores, bounds both)
             fused_rate = N * K / (kern_ms * 1e-3) / 1e12
             ceil = extra["decode_tiles_Tsym_per_s"]
             result["decode_ceiling"] = {
@@ -358,63 +445,124 @@ def time_ours(args):
                 "standalone_decode": ceil, "frac": round(fused_rate / ceil, 4),
                 "note": "ans_gemm symbol rate / ans_decode_tiles symbol rate, same layer, same run"}
         if not (args.no_cpu_baseline or args.quick):
-            result["cpu_baseline"] = cpu_baseline(cfg, d, lay, layer, X_h, budget_s=20.0)
+            result["cpu_baseline"] = cpu_baseline(cfg, d, lay, layer, X_h)
     if pg is not None:
         pg.barrier()
         pg.destroy_process_group()
     return result
 
 
-def context_numbers(torch, ans, WL, cfg, d, lay, layers, dw, device):
-    """Single-GPU context: ans_gemm at the config's other M, the uncompressed
-    variant, cuBLAS on the decoded bf16 weights and the two-pass baseline
-    (ans_decode_tiles to HBM, then cuBLAS)."""
+def timed_events(torch, stream, fn, iters, warm):
+    """Average µs per call of fn(i) over `iters` calls after `warm` untimed
+    ones (CUDA events on `stream`)."""
+    for i in range(warm):
+        fn(i)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(iters):
+        fn(i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / iters * 1e3
+
+
+def context_numbers(torch, ans, WL, cfg, d, lay, layers, dw, sc, device, stream):
+    """Single-GPU context on the headline layer: ans_gemm at the workload's
+    token counts, the same kernel on uncompressed weights, cuBLAS on dense
+    bf16 weights, ans_decode_tiles and the two-pass baselines (decode to HBM,
+    then the uncompressed kernel or cuBLAS)."""
     N, K = lay.N, lay.K
     st = torch.zeros(1, dtype=torch.int32, device=device)
     peaks, _ = load_peaks()
-
-    def timed(fn, iters=100, warm=10):
-        for i in range(warm):
-            fn(i)
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        for i in range(iters):
-            fn(i)
-        b.record()
-        torch.cuda.synchronize()
-        return a.elapsed_time(b) / iters * 1e3  # us
-
-    W_copies = [torch.empty(N, K, dtype=torch.bfloat16, device=device) for _ in range(N_COPIES)]
-    for Wc in W_copies:
-        Wc.view(torch.int16).view(-1).copy_(dw)
+    nc = len(layers)
+    Wb = dequant_bf16(torch, cfg, d, device)
+    dec = torch.empty(dw.numel() * dw.element_size(), dtype=torch.uint8, device=device)
+    t_d = timed_events(torch, stream, lambda i: ans.ans_decode_tiles(layers[i % nc].tiles, dec, st),
+                       10, 2)
     out = {"sweep": []}
     for M in cfg.Ms:
         X = torch.from_numpy(WL.make_x(cfg, M, K).view(np.int16)).to(device)
         Y = torch.empty(M, N, dtype=torch.float32, device=device)
+        Yu = torch.empty(M, N, dtype=torch.float32, device=device)
         nb = ans.ans_gemm_workspace(lay, M, cfg.scale_kind)
-        ws = torch.zeros(nb, dtype=torch.uint8, device=device)
-        t_f = timed(lambda i: ans.ans_gemm(X, M, layers[i % N_COPIES].tiles, 0, None, 0, Y, ws, nb, st))
-        t_u = timed(lambda i: ans.ans_gemm_uncompressed(X, M, W_copies[i % N_COPIES].view(torch.int16),
-                                                        lay, 0, None, 0, Y, ws, nb, st))
+        ws = torch.zeros(max(nb, 256), dtype=torch.uint8, device=device)
+        it = max(3, min(50, int(40000 / (M + 100))))
+        t_f = timed_events(torch, stream, lambda i: ans.ans_gemm(
+            X, M, layers[i % nc].tiles, cfg.scale_kind, sc, cfg.group_k, Y, ws, ws.numel(), st),
+            it, 2)
+        t_u = timed_events(torch, stream, lambda i: ans.ans_gemm_uncompressed(
+            X, M, dw, lay, cfg.scale_kind, sc, cfg.group_k, Yu, ws, ws.numel(), st), it, 2)
+        same = bool(torch.equal(Y, Yu))
         Xb = X.view(torch.bfloat16)
-        t_c = timed(lambda i: torch.matmul(Xb, W_copies[i % N_COPIES].t()))
-        dec = torch.empty(N, K, dtype=torch.bfloat16, device=device)
-        t_d = timed(lambda i: ans.ans_decode_tiles(layers[i % N_COPIES].tiles, dec, st))
-        t_2 = timed(lambda i: (ans.ans_decode_tiles(layers[i % N_COPIES].tiles, dec, st),
-                               torch.matmul(Xb, dec.t())))
-        algo = layers[0].compressed_bytes + 2 * M * K + 4 * M * N
+        t_c = timed_events(torch, stream, lambda i: torch.matmul(Xb, Wb.t()), it, 2)
+        ab = algo_bytes(layers[0], cfg, M, N, K)
         flops = 2.0 * M * N * K
         out["sweep"].append({
             "M": M, "ans_gemm_us": round(t_f, 2),
-            "effective_weight_GBps": round(N * K * 2 / (t_f * 1e-6) / 1e9, 1),
-            "hbm_frac": round(algo / (t_f * 1e-6) / 1e9 / float(peaks["hbm_gbs"]), 4),
+            "effective_weight_GBps": round(N * K * NOMINAL[cfg.dtype] / (t_f * 1e-6) / 1e9, 1),
+            "hbm_frac": round(ab / (t_f * 1e-6) / 1e9 / float(peaks["hbm_gbs"]), 4),
             "tensor_frac": round(flops / (t_f * 1e-6) / 1e12 / float(peaks["bf16_tflops"]), 5),
-            "uncompressed_us": round(t_u, 2), "cublas_us": round(t_c, 2),
-            "decode_tiles_us": round(t_d, 2), "two_pass_us": round(t_2, 2),
-            "speedup_vs_two_pass": round(t_2 / t_f, 3)})
-    out["decode_tiles_Tsym_per_s"] = round(N * K / (out["sweep"][0]["decode_tiles_us"] * 1e-6) / 1e12, 4)
+            "uncompressed_us": round(t_u, 2), "bit_identical_to_uncompressed": same,
+            "cublas_bf16_us": round(t_c, 2), "decode_tiles_us": round(t_d, 2),
+            "two_pass_us": round(t_d + t_u, 2), "two_pass_cublas_us": round(t_d + t_c, 2),
+            "speedup_vs_two_pass": round((t_d + t_u) / t_f, 3),
+            "speedup_vs_two_pass_cublas": round((t_d + t_c) / t_f, 3),
+            "status": int(st.item())})
+        del X, Y, Yu, ws
+    out["decode_tiles_Tsym_per_s"] = round(N * K / (t_d * 1e-6) / 1e12, 4)
+    del Wb, dec
     return out
+
+
+def secondary_entry(torch, ans, WL, args, device, stream):
+    """The bf16 4096 x 4096 split-stream layer at M = 16: twelve rotating
+    copies, CUDA graphs of twelve consecutive calls, events per replay."""
+    cfg, d, lay, layers, hist, encode_s, dw, sc = build_layers(
+        torch, ans, WL, SECOND, device, args.state_bits, SECOND_COPIES)
+    N, K, M = lay.N, lay.K, 16
+    X = torch.from_numpy(WL.make_x(cfg, M, K).view(np.int16)).to(device)
+    Y = torch.empty(M, N, dtype=torch.float32, device=device)
+    nb = ans.ans_gemm_workspace(lay, M, 0)
+    ws = torch.zeros(max(nb, 256), dtype=torch.uint8, device=device)
+    st = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def step(i):
+        ans.ans_gemm(X, M, layers[i % SECOND_COPIES].tiles, 0, None, 0, Y, ws, ws.numel(), st,
+                     stream)
+    for i in range(SECOND_COPIES):
+        step(i)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(SECOND_COPIES):
+            step(i)
+    reps = 60
+    for _ in range(5):
+        g.replay()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+    ev[0].record(stream)
+    for r in range(reps):
+        g.replay()
+        ev[r + 1].record(stream)
+    torch.cuda.synchronize()
+    per = [ev[r].elapsed_time(ev[r + 1]) / SECOND_COPIES for r in range(reps)]
+    ms = ev[0].elapsed_time(ev[-1]) / (reps * SECOND_COPIES)
+    del g
+    peaks, _ = load_peaks()
+    ab = algo_bytes(layers[0], cfg, M, N, K)
+    return {"workload": workload_name(SECOND, args.state_bits, M),
+            "value": round(N * K * 2 / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "ms_per_call": round(ms, 6), "per_call_ms": percentiles(per),
+            "bits_per_weight": round(8.0 * layers[0].compressed_bytes / (N * K), 4),
+            "entropy_bits_split_bound": round(ans.ans_entropy(hist) + 8, 4),
+            "roofline": {"bound": "hbm", "achieved": round(ab / (ms * 1e-3) / 1e9, 2),
+                         "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                         "frac": round(ab / (ms * 1e-3) / 1e9 / float(peaks["hbm_gbs"]), 4),
+                         "algorithmic_bytes_per_launch": ab},
+            "status": int(st.item()),
+            "timing": f"CUDA graphs of {SECOND_COPIES} consecutive calls over rotating copies"}
 
 
 def dequant_bf16(torch, cfg, d, device):
@@ -441,9 +589,12 @@ def dequant_bf16(torch, cfg, d, device):
         q = torch.from_numpy(d["w"].view(np.int8)).to(device).view(N, K).float()
         s = torch.from_numpy(d["scales"]).to(device)
         return (q * s[:, None]).to(torch.bfloat16)
+    out = torch.empty(N, K, dtype=torch.bfloat16, device=device)
     codes = torch.from_numpy(d["w"]).to(device).view(torch.float8_e4m3fn).view(N, K)
     s = torch.from_numpy(d["scales"]).to(device)
-    return (codes.float() * s[:, None]).to(torch.bfloat16)
+    for r0 in range(0, N, 4096):  # in row chunks: the fp32 temporary stays small
+        out[r0:r0 + 4096] = (codes[r0:r0 + 4096].float() * s[r0:r0 + 4096, None]).to(torch.bfloat16)
+    return out
 
 
 def sweep(args):
@@ -459,7 +610,6 @@ def sweep(args):
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
     peaks, peaks_src = load_peaks()
-    nominal = {0: 0.5, 1: 2.0, 2: 1.0, 4: 1.0, 5: 0.5}
     st = torch.zeros(1, dtype=torch.int32, device=device)
     stream = torch.cuda.Stream(device=device)
     torch.cuda.set_stream(stream)
@@ -486,6 +636,7 @@ def sweep(args):
         return a.elapsed_time(b) * 1e3 / (reps * len(calls))
 
     only = set(args.sweep_configs.split(",")) if args.sweep_configs else None
+    ms_only = [int(m) for m in args.sweep_ms.split(",")] if args.sweep_ms else None
     for name, cfg in WL.CONFIGS.items():
         if only and name not in only:
             continue
@@ -525,7 +676,7 @@ def sweep(args):
             t_dec = timed_graph([lambda l=l: ans.ans_decode_tiles(l.tiles, dec, st) for l in layers], 3)
             t_dec = timed_graph([lambda l=l: ans.ans_decode_tiles(l.tiles, dec, st) for l in layers],
                                 rep_for(t_dec * copies))
-            for M in cfg.Ms:
+            for M in (ms_only or cfg.Ms):
                 X = torch.from_numpy(WL.make_x(cfg, M, K).view(np.int16)).to(device)
                 Y = torch.empty(M, N, dtype=torch.float32, device=device)
                 Yu = torch.empty(M, N, dtype=torch.float32, device=device)
@@ -544,7 +695,7 @@ def sweep(args):
                 cub = [lambda w=w: torch.matmul(Xb, w.t()) for w in Wbs]
                 t_c = timed_graph(cub, 2)
                 t_c = timed_graph(cub, rep_for(t_c * len(cub)))
-                algo = layers[0].compressed_bytes + 2 * M * K + 4 * M * N
+                ab = algo_bytes(layers[0], cfg, M, N, K)
                 rec = {"workload": name, "matrix": mname, "N": N, "K": K, "M": M,
                        "state_bits": args.state_bits,
                        **({"nibble_symbols": args.nibble_symbols}
@@ -553,8 +704,8 @@ def sweep(args):
                        "entropy_bound_bits": round(bound, 4), "gap_bits": round(bpw - bound, 4),
                        "encode_s": round(encode_s, 2), "copies": copies,
                        "ans_gemm_us": round(t_f, 2),
-                       "effective_weight_GBps": round(N * K * nominal[cfg.dtype] / (t_f * 1e-6) / 1e9, 1),
-                       "hbm_frac": round(algo / (t_f * 1e-6) / 1e9 / float(peaks["hbm_gbs"]), 4),
+                       "effective_weight_GBps": round(N * K * NOMINAL[cfg.dtype] / (t_f * 1e-6) / 1e9, 1),
+                       "hbm_frac": round(ab / (t_f * 1e-6) / 1e9 / float(peaks["hbm_gbs"]), 4),
                        "tensor_frac": round(2.0 * M * N * K / (t_f * 1e-6) / 1e12 / float(peaks["bf16_tflops"]), 4),
                        "uncompressed_us": round(t_u, 2), "bit_identical_to_uncompressed": same,
                        "decode_tiles_us": round(t_dec, 2),
@@ -611,34 +762,52 @@ def sweep_batched(args, torch, ans, WL, device, stream, st, timed_graph):
         print(json.dumps(rec), flush=True)
 
 
-def cpu_baseline(cfg, d, lay, layer, X_h, budget_s=20.0):
-    """The CPU oracle, as it stands, on the host cores: decode of a sample of
-    whole W row blocks plus the fp64 GEMM on their rows, scaled to the metric
-    (effective weight GB/s)."""
-    from oracle import oracle as O
-    O.build()
-    cores = os.cpu_count() or 1
+def oracle_rows_rate(O, cfg, d, lay, layer, X_h, budget_s, threads, max_rb=None):
+    """Oracle decode of whole W row blocks plus the fp64 GEMM of their rows,
+    until `budget_s` of CPU time is spent; returns (weights, seconds, blocks)."""
     N, K, M = lay.N, lay.K, X_h.shape[0]
     n_kt = K // lay.tile_k
     freq = layer.codebook.freq_array()
     rb_total = N // lay.tile_n
+    if max_rb is not None:
+        rb_total = min(rb_total, max_rb)
+    if cfg.dtype == 1:
+        out = np.zeros(N * K, np.uint16)
+    else:
+        out = np.zeros(int(N * K * NOMINAL[cfg.dtype]), np.uint8)
     done_rb, t_spent = 0, 0.0
-    out = np.zeros(N * K, np.uint16)
     while done_rb < rb_total and t_spent < budget_s:
         t0 = time.perf_counter()
         st, _ = O.decode(cfg.dtype, layer.h_stream, layer.h_offsets, layer.h_raw, N, K,
                          lay.tile_n, lay.tile_k, freq, tile_begin=done_rb * n_kt,
-                         tile_end=(done_rb + 1) * n_kt, out=out, threads=cores,
+                         tile_end=(done_rb + 1) * n_kt, out=out, threads=threads,
                          state_bits=lay.state_bits or 32)
         rows = np.arange(done_rb * lay.tile_n, (done_rb + 1) * lay.tile_n, dtype=np.uint32)
-        O.gemm(cfg.dtype, X_h, M, K, out, N, rows=rows, threads=cores)
+        O.gemm(cfg.dtype, X_h, M, K, out, N, cfg.scale_kind, d["scales"], cfg.group_k,
+               rows=rows, threads=threads)
         t_spent += time.perf_counter() - t0
         done_rb += 1
-    weights = done_rb * lay.tile_n * K
-    return {"value": round(weights * 2 / t_spent / 1e9, 4), "unit": "GB/s", "cores": cores,
-            "kind": "oracle",
-            "sample": f"{done_rb} of {rb_total} row blocks of 128 rows: oracle decode of their "
-                      f"{done_rb * n_kt} tiles + fp64 GEMM of their rows with X {M}x{K}"}
+    return done_rb * lay.tile_n * K, t_spent, done_rb
+
+
+def cpu_baseline(cfg, d, lay, layer, X_h, budget_s=15.0, budget_1core_s=8.0):
+    """The CPU oracle, as it stands, on the host cores (all of them, then one):
+    decode of a sample of whole W row blocks plus the fp64 GEMM on their rows,
+    scaled to the metric (effective weight GB/s)."""
+    from oracle import oracle as O
+    O.build()
+    cores = os.cpu_count() or 1
+    w_all, t_all, rb_all = oracle_rows_rate(O, cfg, d, lay, layer, X_h, budget_s, cores)
+    w_one, t_one, rb_one = oracle_rows_rate(O, cfg, d, lay, layer, X_h, budget_1core_s, 1)
+    M, K = X_h.shape
+    nb = NOMINAL[cfg.dtype]
+    return {"value": round(w_all * nb / t_all / 1e9, 4), "unit": "GB/s", "cores": cores,
+            "kind": "oracle", "cpu_model": cpu_model(),
+            "sample": f"{rb_all} of {lay.N // lay.tile_n} row blocks of {lay.tile_n} rows: "
+                      f"oracle decode of their {rb_all * (K // lay.tile_k)} tiles + fp64 GEMM of "
+                      f"their rows with X {M}x{K}, {cores} threads",
+            "one_core": {"value": round(w_one * nb / t_one / 1e9, 4), "unit": "GB/s", "cores": 1,
+                         "sample": f"{rb_one} row blocks, 1 thread"}}
 
 
 def time_reference(args):
@@ -646,7 +815,6 @@ def time_reference(args):
     if rank != 0:
         return None
     from oracle import oracle as O
-    from rans_decode_gemm_b200 import ans
     from rans_decode_gemm_b200 import workloads as WL
     O.build()
     cfg = WL.CONFIGS[WORKLOAD]
@@ -654,41 +822,47 @@ def time_reference(args):
     N, K, M = d["N"], d["K"], M_HEAD
     counts = O.histogram(cfg.dtype, d["w"], N * K)
     _, freq = O.normalize(counts)
-    st, stream, offsets, raw = O.encode(cfg.dtype, d["w"], N, K, cfg.tile_n, cfg.tile_k, freq,
-                                        state_bits=args.state_bits)
-    X_h = WL.make_x(cfg, M, K)
-    cores = os.cpu_count() or 1
+    # the oracle codes only the row blocks the timed steps decode
     n_kt = K // cfg.tile_k
     rb_total = N // cfg.tile_n
-    out = np.zeros(N * K, np.uint16)
+    n_rb = min(rb_total, max(1, args.warmup + args.steps))
+    rows_w = d["w"][:n_rb * cfg.tile_n * K]
+    st, stream, offsets, raw = O.encode(cfg.dtype, rows_w, n_rb * cfg.tile_n, K, cfg.tile_n,
+                                        cfg.tile_k, freq, state_bits=args.state_bits)
+    X_h = WL.make_x(cfg, M, K)
+    cores = os.cpu_count() or 1
+    out = np.zeros(n_rb * cfg.tile_n * K, np.uint8)
+    Nr = n_rb * cfg.tile_n
 
     def one(rb):
-        O.decode(cfg.dtype, stream, offsets, raw, N, K, cfg.tile_n, cfg.tile_k, freq,
+        O.decode(cfg.dtype, stream, offsets, raw, Nr, K, cfg.tile_n, cfg.tile_k, freq,
                  tile_begin=rb * n_kt, tile_end=(rb + 1) * n_kt, out=out, threads=cores,
                  state_bits=args.state_bits)
         rows = np.arange(rb * cfg.tile_n, (rb + 1) * cfg.tile_n, dtype=np.uint32)
-        O.gemm(cfg.dtype, X_h, M, K, out, N, rows=rows, threads=cores)
+        O.gemm(cfg.dtype, X_h, M, K, out, Nr, cfg.scale_kind, d["scales"][:Nr], cfg.group_k,
+               rows=rows, threads=cores)
 
     for i in range(args.warmup):
-        one(i % rb_total)
+        one(i % n_rb)
     t0 = time.perf_counter()
     for i in range(args.steps):
-        one(i % rb_total)
+        one((args.warmup + i) % n_rb)
     dt = time.perf_counter() - t0
     per_rb_s = dt / max(1, args.steps)
-    value = cfg.tile_n * K * 2 / per_rb_s / 1e9
-    sample = (f"each step: oracle decode of one 128-row block ({n_kt} tiles) + fp64 GEMM "
-              f"of its rows with X {M}x{K}")
-    return {"impl": "reference",
-            "metric": "fused decode-GEMM effective weight GB/s (bf16 weights, M=16)",
+    value = cfg.tile_n * K * NOMINAL[cfg.dtype] / per_rb_s / 1e9
+    sample = (f"each step: oracle decode of one {cfg.tile_n}-row block ({n_kt} tiles) + fp64 "
+              f"GEMM of its rows with X {M}x{K}, {cores} threads")
+    return {"impl": "reference", "metric": METRIC,
             "value": round(value, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(per_rb_s * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": workload_name(args.state_bits), "state_bits": args.state_bits,
-                       "M": M, "N": N, "K": K},
+            "config": {"workload": workload_name(WORKLOAD, args.state_bits, M),
+                       "state_bits": args.state_bits, "M": M, "N": N, "K": K,
+                       "global_batch": M * world, "parallelism": f"replicas x{world}",
+                       "l2": "host memory (CPU oracle)"},
             "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores,
-                             "kind": "oracle", "sample": sample},
+                             "kind": "oracle", "sample": sample, "cpu_model": cpu_model()},
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 

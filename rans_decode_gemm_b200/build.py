@@ -7,6 +7,7 @@ import glob
 import os
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
@@ -39,7 +40,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         return LIB
     build_dir = os.path.join(ROOT, "_build")
     os.makedirs(build_dir, exist_ok=True)
-    objs = []
+    jobs = []
     for src in sources():
         obj = os.path.join(build_dir, os.path.relpath(src, CSRC).replace(os.sep, "_") + ".o")
         cmd = [NVCC, *ARCH, "-lineinfo", "-O3", "-std=c++17", "-Xcompiler", "-fPIC,-pthread",
@@ -48,8 +49,12 @@ def build(force: bool = False, verbose: bool = False) -> str:
             cmd[1:1] = ["-Xptxas", "-v"] if verbose else []
         if verbose:
             print(" ".join(cmd), file=sys.stderr)
-        subprocess.check_call(cmd)
-        objs.append(obj)
+        jobs.append((cmd, obj))
+    # the translation units are independent: compile them side by side
+    with ThreadPoolExecutor(max_workers=max(1, min(len(jobs), os.cpu_count() or 1))) as ex:
+        for f in [ex.submit(subprocess.check_call, cmd) for cmd, _ in jobs]:
+            f.result()
+    objs = [obj for _, obj in jobs]
     tmp = LIB + f".tmp{os.getpid()}"
     subprocess.check_call([NVCC, *ARCH, "-shared", "-Xcompiler", "-fPIC", "-o", tmp, *objs,
                            "-lpthread"])
