@@ -104,6 +104,9 @@ typedef enum {
                                        its words did not end at its last byte */
 #define ANS_STATUS_TIMEOUT 0x2u     /* a bounded wait inside a kernel ran out */
 #define ANS_STATUS_BAD_OFFSETS 0x4u /* an offset was unaligned, decreasing or past the end */
+#define ANS_STATUS_SMEM_ALIGN 0x8u  /* a fused-GEMM CTA's dynamic shared memory did not start
+                                       on the 1024-byte boundary its tensor-core operand
+                                       layout assumes (its Y is not valid) */
 
 typedef enum {
   ANS_INT4 = 0,
@@ -248,16 +251,20 @@ ans_status ans_gemm(const uint16_t* d_X, uint32_t M, const ans_tiles* W,
  * while a CUDA graph is being captured, plug-ins whose host framework owns all
  * device memory, or latency-critical paths that may not take an allocation's
  * implicit synchronisation).  Same arguments and result as ans_gemm, without
- * the workspace: the scratch (split-K counters and partials, staged X) lives
- * in a fixed 16 MiB device array inside the library, which every GPU that
- * loads the library holds until the process exits.  A shape whose
- * ans_gemm_workspace exceeds 16 MiB returns ANS_ERR_BUFFER_TOO_SMALL (text via
- * ans_last_error).  The first call on a device looks the array's device
- * address up (cudaGetSymbolAddress with that device current); make that first
- * call before any stream capture.  Each call clears the split-K counters with
- * a memset on `stream`; it never allocates.  All calls share the one array,
- * which keeps the last call's contents: calls that overlap on the GPU (other
- * streams, other threads) race and must be serialised by the caller. */
+ * the workspace: the scratch (split-K counters and partials, the f16 copy of
+ * X for the f16 formats) lives in a fixed 16 MiB device array inside the
+ * library, which every GPU that loads the library holds until the process
+ * exits.  A shape whose ans_gemm_workspace exceeds 16 MiB returns
+ * ANS_ERR_BUFFER_TOO_SMALL (text via ans_last_error).  Every argument check of
+ * ans_gemm runs before anything is queued, so a refused call leaves the array
+ * untouched.  The first call on a device looks the array's device address up
+ * (cudaGetSymbolAddress with that device current) and keeps it for the life of
+ * the process; make that first call before any stream capture, and do not
+ * reset the device (cudaDeviceReset) while the library is loaded.  Each call
+ * clears the split-K counters with a memset on `stream`; it never allocates.
+ * All calls share the one array, which keeps the last call's contents: calls
+ * that overlap on the GPU (other streams, other threads) race and must be
+ * serialised by the caller. */
 ans_status ans_gemm_noalloc(const uint16_t* d_X, uint32_t M, const ans_tiles* W,
                             ans_scale_kind scale_kind, const void* d_scales, uint32_t group_k,
                             float* d_Y, uint32_t* d_status, ans_stream_t stream);
@@ -283,26 +290,31 @@ typedef struct {
 
 #define ANS_MAX_BATCH 8
 
-/* Bytes of device workspace for ans_gemm_batched over n_jobs layers of the
- * layout of jobs[0] (same conditions as ans_gemm_workspace). */
+/* Bytes of device workspace for ans_gemm_batched over these n_jobs layers
+ * (same conditions as ans_gemm_workspace, for each layer). */
 ans_status ans_gemm_batched_workspace(const ans_gemm_job* jobs, uint32_t n_jobs, uint32_t M,
                                       ans_scale_kind scale_kind, size_t* bytes);
 
-/* Several independent layers in one launch (the gate and up projections of
- * an MLP, say; "Approaching Shannon Bound", s3.1 applied to a list of
- * layers): Y_j = X_j * dequant(W_j)^T for j < n_jobs, with M, scale_kind and
- * group_k shared.  1 <= n_jobs <= ANS_MAX_BATCH; every W_j must have the same
- * layout (dtype, N, K, tile shape, state width; ANS_ERR_SHAPE otherwise) and
- * its own codebook.  When the shape takes the small-M schedule on an equal
- * share of the SMs (M up to 32 for 128-row tiles, 16 for 256-row tiles) the
- * layers share one kernel launch, each on its share, so one kernel tail
- * serves them all; otherwise they run as consecutive ans_gemm launches.  Each
- * Y_j is deterministic and within the error bound of ans_gemm; in one launch
- * it is bit-identical to ans_gemm on the same layer confined to the same
- * number of SMs (the split-K partition depends on the SM count, so it may
- * differ from ans_gemm's in the last bits).  d_ws: ans_gemm_batched_workspace
- * bytes, zero-filled once before first use (the kernels leave it that way);
- * d_status as for ans_gemm. */
+/* Several independent layers in one launch (the gate, up and down
+ * projections of an MLP, say: block-level batched decompression of several
+ * matrices, DFloat11's "两阶段Kernel"; "Approaching Shannon Bound", s3.1
+ * applied to a list of layers): Y_j = X_j * dequant(W_j)^T for j < n_jobs,
+ * with M, scale_kind and group_k shared.  1 <= n_jobs <= ANS_MAX_BATCH; every
+ * W_j must have the same coded dtype and stream format (state width;
+ * ANS_ERR_SHAPE otherwise) and its own codebook; N, K and the tile shape may
+ * differ.  Layer j takes a share of the SMs proportional to its weight count
+ * N_j * K_j: G_j = max(1, floor(SMs * w_j / sum w)), the largest share giving
+ * SMs back while the shares add up to more than the device has, the SMs left
+ * over going one each to the first layers.  When every layer takes the small-M
+ * schedule on its share (M up to 32 for 128-row tiles, 16 for 256-row tiles)
+ * the layers share one kernel launch, each on its share with its own launch
+ * plan, so one kernel tail serves them all; otherwise they run as consecutive
+ * ans_gemm launches.  Each Y_j is deterministic and within the error bound of
+ * ans_gemm; in one launch it is bit-identical to ans_gemm on the same layer
+ * confined to G_j SMs (the split-K partition depends on the SM count, so it
+ * may differ from ans_gemm's on the whole device in the last bits).  d_ws:
+ * ans_gemm_batched_workspace bytes, zero-filled once before first use (the
+ * kernels leave it that way); d_status as for ans_gemm. */
 ans_status ans_gemm_batched(const ans_gemm_job* jobs, uint32_t n_jobs, uint32_t M,
                             ans_scale_kind scale_kind, uint32_t group_k, void* d_ws,
                             size_t ws_bytes, uint32_t* d_status, ans_stream_t stream);

@@ -19,7 +19,7 @@ from . import build as _build
 
 INT4, BF16_SPLIT, FP8_E4M3, INT4_PAIRS, INT8, FP4_E2M1, FP4_PAIRS = 0, 1, 2, 3, 4, 5, 6
 SCALE_NONE, SCALE_ROW_BF16, SCALE_ROW_F32, SCALE_GROUP_BF16 = 0, 1, 2, 3
-STATUS_CORRUPT, STATUS_TIMEOUT, STATUS_BAD_OFFSETS = 0x1, 0x2, 0x4
+STATUS_CORRUPT, STATUS_TIMEOUT, STATUS_BAD_OFFSETS, STATUS_SMEM_ALIGN = 0x1, 0x2, 0x4, 0x8
 ALPHABET = {INT4: 16, BF16_SPLIT: 256, FP8_E4M3: 256, INT4_PAIRS: 256, INT8: 256, FP4_E2M1: 16,
             FP4_PAIRS: 256}
 
@@ -264,6 +264,37 @@ def ans_gemm_batched(jobs, M: int, scale_kind: int, group_k: int, d_ws, ws_bytes
     _check(load().ans_gemm_batched(arr, len(jobs), M, scale_kind, group_k, _ptr(d_ws), ws_bytes,
                                    _ptr(d_status), _stream(stream)),
            "ans_gemm_batched")
+
+
+def _set_plan_limits(max_ctas: int = 0, max_producers: int = 0, force_shared: bool = False):
+    """Internal test hook of libans.so (not part of include/ans.h): caps on the
+    CTAs and producer warps of every later fused-GEMM plan in this process,
+    and a switch that sends every token count to the shared-accumulator
+    schedule.  (0, 0, False) restores the defaults."""
+    fn = load().ansdev_set_plan_limits
+    fn.argtypes = [C.c_uint32, C.c_uint32, C.c_uint32]
+    fn.restype = None
+    fn(int(max_ctas), int(max_producers), 1 if force_shared else 0)
+
+
+def _set_wait_budget(cycles: int = 0):
+    """Internal test hook of libans.so: the budget (clock64 cycles) of every
+    wait in the kernels that the pipeline's own progress ends, on the current
+    device; 0 restores the default (about 1.5 s).  A wait that runs out sets
+    the TIMEOUT status bit and the kernel returns."""
+    fn = load().ansdev_set_wait_budget
+    fn.argtypes = [C.c_longlong]
+    fn.restype = C.c_int
+    _check(fn(int(cycles)), "ansdev_set_wait_budget")
+
+
+def _wait_probe(d_status, stream=None):
+    """Internal test hook: one bounded wait on a barrier nothing arrives on
+    (leaves the TIMEOUT bit in d_status)."""
+    fn = load().ansdev_wait_probe
+    fn.argtypes = [C.c_void_p, C.c_void_p]
+    fn.restype = C.c_int
+    _check(fn(_ptr(d_status), _stream(stream)), "ansdev_wait_probe")
 
 
 # ---- marshalling helper: a compressed layer resident on a device -----------------

@@ -129,26 +129,68 @@ ans_status check_scales(uint32_t dtype, ans_scale_kind kind, const void* scales,
   return ANS_ERR_ARG;
 }
 
+// Checks of the device buffers every fused-GEMM call takes (no device work).
+ans_status check_gemm_io(const uint16_t* d_X, float* d_Y, uint32_t* d_status, const void* d_scales) {
+  if (!d_X || !d_Y || !d_status) return ANS_ERR_ARG;
+  if (reinterpret_cast<uintptr_t>(d_X) % 16 != 0 || reinterpret_cast<uintptr_t>(d_Y) % 16 != 0 ||
+      (d_scales && reinterpret_cast<uintptr_t>(d_scales) % 16 != 0))
+    return ANS_ERR_ARG;
+  return ANS_OK;
+}
+
+// Checks of a compressed layer as ans_gemm takes it (no device work).
+ans_status check_gemm_tiles(const ans_tiles* W, ans_scale_kind scale_kind, const void* d_scales,
+                            uint32_t group_k) {
+  if (!W) return ANS_ERR_ARG;
+  ans_status st = check_layout(&W->layout);
+  if (st != ANS_OK) return st;
+  st = check_codebook(&W->codebook, W->layout.dtype);
+  if (st != ANS_OK) return st;
+  st = check_scales(W->layout.dtype, scale_kind, d_scales, group_k, W->layout);
+  if (st != ANS_OK) return st;
+  if (!W->stream || !W->offsets) return ANS_ERR_ARG;
+  if (W->layout.dtype == ANS_BF16_SPLIT && !W->raw) return ANS_ERR_ARG;
+  if (reinterpret_cast<uintptr_t>(W->stream) % 16 != 0 ||
+      reinterpret_cast<uintptr_t>(W->offsets) % 8 != 0 ||
+      (W->raw && reinterpret_cast<uintptr_t>(W->raw) % 16 != 0))
+    return ANS_ERR_ARG;
+  return ANS_OK;
+}
+
+// The launch plan of one call on the current device.
+ans_status plan_gemm(const ansdev::LayerDev& L, uint32_t M, ans_scale_kind kind, bool decode,
+                     ansdev::GemmPlan* plan) {
+  int sms = 0;
+  ans_status st = device_info(&sms);
+  if (st != ANS_OK) return st;
+  if (!ansdev::make_gemm_plan(L, M, kind, decode, sms, plan)) return ANS_ERR_UNSUPPORTED;
+  return ANS_OK;
+}
+
+ans_status launch_planned(const ansdev::GemmPlan& plan, const uint16_t* d_X,
+                          const ansdev::LayerDev& L, bool decode, const void* d_W,
+                          ans_scale_kind kind, const void* d_scales, uint32_t group_k, float* d_Y,
+                          void* d_ws, uint32_t* d_status, ans_stream_t stream) {
+  cudaError_t e = ansdev::launch_gemm(plan, L, decode, d_W, d_X, d_scales, kind, group_k, d_Y,
+                                      d_ws, d_status, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, decode ? "ans_gemm" : "ans_gemm_uncompressed");
+  return ANS_OK;
+}
+
 ans_status run_gemm(const uint16_t* d_X, uint32_t M, const ansdev::LayerDev& L, bool decode,
                     const void* d_W, ans_scale_kind kind, const void* d_scales, uint32_t group_k,
                     float* d_Y, void* d_ws, size_t ws_bytes, uint32_t* d_status,
                     ans_stream_t stream) {
   if (M == 0) return ANS_OK;
-  if (!d_X || !d_Y || !d_status || !d_ws) return ANS_ERR_ARG;
-  if (reinterpret_cast<uintptr_t>(d_X) % 16 != 0 || reinterpret_cast<uintptr_t>(d_Y) % 16 != 0 ||
-      reinterpret_cast<uintptr_t>(d_ws) % 256 != 0 ||
-      (d_scales && reinterpret_cast<uintptr_t>(d_scales) % 16 != 0))
-    return ANS_ERR_ARG;
-  int sms = 0;
-  ans_status st = device_info(&sms);
+  ans_status st = check_gemm_io(d_X, d_Y, d_status, d_scales);
   if (st != ANS_OK) return st;
+  if (!d_ws || reinterpret_cast<uintptr_t>(d_ws) % 256 != 0) return ANS_ERR_ARG;
   ansdev::GemmPlan plan;
-  if (!ansdev::make_gemm_plan(L, M, kind, decode, sms, &plan)) return ANS_ERR_UNSUPPORTED;
+  st = plan_gemm(L, M, kind, decode, &plan);
+  if (st != ANS_OK) return st;
   if (ws_bytes < plan.ws_bytes) return ANS_ERR_BUFFER_TOO_SMALL;
-  cudaError_t e = ansdev::launch_gemm(plan, L, decode, d_W, d_X, d_scales, kind, group_k, d_Y,
-                                      d_ws, d_status, reinterpret_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, decode ? "ans_gemm" : "ans_gemm_uncompressed");
-  return ANS_OK;
+  return launch_planned(plan, d_X, L, decode, d_W, kind, d_scales, group_k, d_Y, d_ws, d_status,
+                        stream);
 }
 
 }  // namespace
@@ -305,19 +347,8 @@ ans_status ans_gemm(const uint16_t* d_X, uint32_t M, const ans_tiles* W,
                     ans_scale_kind scale_kind, const void* d_scales, uint32_t group_k,
                     float* d_Y, void* d_ws, size_t ws_bytes, uint32_t* d_status,
                     ans_stream_t stream) {
-  if (!W) return ANS_ERR_ARG;
-  ans_status st = check_layout(&W->layout);
+  ans_status st = check_gemm_tiles(W, scale_kind, d_scales, group_k);
   if (st != ANS_OK) return st;
-  st = check_codebook(&W->codebook, W->layout.dtype);
-  if (st != ANS_OK) return st;
-  st = check_scales(W->layout.dtype, scale_kind, d_scales, group_k, W->layout);
-  if (st != ANS_OK) return st;
-  if (!W->stream || !W->offsets) return ANS_ERR_ARG;
-  if (W->layout.dtype == ANS_BF16_SPLIT && !W->raw) return ANS_ERR_ARG;
-  if (reinterpret_cast<uintptr_t>(W->stream) % 16 != 0 ||
-      reinterpret_cast<uintptr_t>(W->offsets) % 8 != 0 ||
-      (W->raw && reinterpret_cast<uintptr_t>(W->raw) % 16 != 0))
-    return ANS_ERR_ARG;
   ansdev::LayerDev L;
   fill_layer(W, &L);
   return run_gemm(d_X, M, L, true, nullptr, scale_kind, d_scales, group_k, d_Y, d_ws, ws_bytes,
@@ -342,48 +373,72 @@ ans_status ans_gemm_uncompressed(const uint16_t* d_X, uint32_t M, const void* d_
 ans_status ans_gemm_noalloc(const uint16_t* d_X, uint32_t M, const ans_tiles* W,
                             ans_scale_kind scale_kind, const void* d_scales, uint32_t group_k,
                             float* d_Y, uint32_t* d_status, ans_stream_t stream) {
-  if (!W) return ANS_ERR_ARG;
+  // every check of ans_gemm first: a refused call leaves the shared scratch
+  // (and any call still running on it) untouched
+  ans_status st = check_gemm_tiles(W, scale_kind, d_scales, group_k);
+  if (st != ANS_OK) return st;
   if (M == 0) return ANS_OK;
-  ans_status st = check_layout(&W->layout);
+  st = check_gemm_io(d_X, d_Y, d_status, d_scales);
   if (st != ANS_OK) return st;
-  size_t need = 0;
-  st = ans_gemm_workspace(&W->layout, M, scale_kind, &need);
+  ansdev::LayerDev L;
+  fill_layer(W, &L);
+  ansdev::GemmPlan plan;
+  st = plan_gemm(L, M, scale_kind, true, &plan);
   if (st != ANS_OK) return st;
-  if (need > ansdev::kNoAllocScratchBytes) {
+  if (plan.ws_bytes > ansdev::kNoAllocScratchBytes) {
     std::snprintf(g_last_error, sizeof(g_last_error),
                   "ans_gemm_noalloc: this shape needs %zu bytes of scratch, above the fixed "
                   "%zu-byte maximum; use ans_gemm with a caller workspace",
-                  need, ansdev::kNoAllocScratchBytes);
+                  plan.ws_bytes, ansdev::kNoAllocScratchBytes);
     return ANS_ERR_BUFFER_TOO_SMALL;
   }
   void* scratch = nullptr;
   cudaError_t e = ansdev::noalloc_scratch(&scratch);
   if (e != cudaSuccess) return cuda_fail(e, "ans_gemm_noalloc scratch");
-  // the split-K counters must start at zero: clear them on the caller's stream
-  // (a memset, not an allocation)
-  ansdev::LayerDev L;
-  fill_layer_plain(&W->layout, &L);
-  ansdev::GemmPlan plan;
-  int sms = 0;
-  st = device_info(&sms);
-  if (st != ANS_OK) return st;
-  if (!ansdev::make_gemm_plan(L, M, scale_kind, true, sms, &plan)) return ANS_ERR_UNSUPPORTED;
+  // the split-K counters must start at zero: clear them on the caller's
+  // stream (a memset, not an allocation)
   e = cudaMemsetAsync(scratch, 0, plan.ws_counters_bytes, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "ans_gemm_noalloc clear");
-  return ans_gemm(d_X, M, W, scale_kind, d_scales, group_k, d_Y, scratch,
-                  ansdev::kNoAllocScratchBytes, d_status, stream);
+  return launch_planned(plan, d_X, L, true, nullptr, scale_kind, d_scales, group_k, d_Y, scratch,
+                        d_status, stream);
 }
 
 // Internal profiling hook (not part of the public ABI in include/ans.h).
 void ansdev_set_trace(void* d_buf, size_t bytes) { ansdev::set_trace_buffer(d_buf, bytes); }
 
+// Internal test hooks (not part of the public ABI): the budget, in clock64
+// cycles, of every wait in the library's kernels that the pipeline's own
+// progress ends (0 restores the default of about 1.5 s), on the current
+// device; and one bounded wait on a barrier that nothing arrives on, which
+// leaves the TIMEOUT bit in *d_status.
+int ansdev_set_wait_budget(long long cycles) {
+  const long long c = cycles > 0 ? cycles : ansdev::kWaitBudgetCyclesHost;
+  cudaError_t e = ansdev::set_live_wait_budget_gemm(c);
+  if (e == cudaSuccess) e = ansdev::set_live_wait_budget_local(c);
+  if (e == cudaSuccess) e = ansdev::set_live_wait_budget_decode(c);
+  return e == cudaSuccess ? ANS_OK : cuda_fail(e, "ansdev_set_wait_budget");
+}
+
+int ansdev_wait_probe(uint32_t* d_status, ans_stream_t stream) {
+  if (!d_status) return ANS_ERR_ARG;
+  cudaError_t e = ansdev::launch_wait_probe(d_status, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ANS_OK : cuda_fail(e, "ansdev_wait_probe");
+}
+
+// Internal test hook (not part of the public ABI): caps on the CTAs and
+// producer warps of every later fused-GEMM plan in this process and a switch
+// that forces the shared-accumulator schedule; 0, 0, 0 restores the defaults.
+void ansdev_set_plan_limits(uint32_t max_ctas, uint32_t max_producers, uint32_t force_shared) {
+  ansdev::set_plan_limits(max_ctas, max_producers, force_shared);
+}
+
 // Internal test hook (not part of the public ABI): the launch plan that
 // ans_gemm (decode = 1) or ans_gemm_uncompressed (decode = 0) would use for a
 // layout, M and scale kind on a device with num_sms SMs, without touching a
-// device.  out[0..19] = local, grid, D, n_slots, tmem_cols, smem_bytes, T,
+// device.  out[0..20] = local, grid, D, n_slots, tmem_cols, smem_bytes, T,
 // T_pass, n_pass, NT, n_bufs, fmt, ab_f16, H, C, x_stages, n_units,
-// n_segments, ws_bytes (low 32 bits), ws_bytes (high 32 bits).  Returns 1 if
-// the shape can be scheduled, 0 if not, -1 for a bad layout.
+// n_segments, ws_bytes (low 32 bits), ws_bytes (high 32 bits), n_banks.
+// Returns 1 if the shape can be scheduled, 0 if not, -1 for a bad layout.
 int ansdev_gemm_plan(const ans_layout* layout, uint32_t M, uint32_t scale_kind, int decode,
                      int num_sms, uint32_t* out) {
   if (check_layout(layout) != ANS_OK || !out) return -1;
@@ -392,12 +447,13 @@ int ansdev_gemm_plan(const ans_layout* layout, uint32_t M, uint32_t scale_kind, 
   L.wide = layout->state_bits == 64 ? 1u : 0u;
   ansdev::GemmPlan p;
   if (!ansdev::make_gemm_plan(L, M, scale_kind, decode != 0, num_sms, &p)) return 0;
-  const uint32_t v[20] = {p.local, p.grid, p.D, p.n_slots, p.tmem_cols, p.smem_bytes, p.T,
+  const uint32_t v[21] = {p.local, p.grid, p.D, p.n_slots, p.tmem_cols, p.smem_bytes, p.T,
                           p.T_pass, p.n_pass, p.NT, p.n_bufs, p.fmt, p.ab_f16, p.H, p.C,
                           p.x_stages, static_cast<uint32_t>(p.n_units), p.n_segments,
                           static_cast<uint32_t>(p.ws_bytes),
-                          static_cast<uint32_t>(static_cast<uint64_t>(p.ws_bytes) >> 32)};
-  for (int i = 0; i < 20; ++i) out[i] = v[i];
+                          static_cast<uint32_t>(static_cast<uint64_t>(p.ws_bytes) >> 32),
+                          p.n_banks};
+  for (int i = 0; i < 21; ++i) out[i] = v[i];
   return 1;
 }
 
@@ -405,7 +461,9 @@ int ansdev_gemm_plan(const ans_layout* layout, uint32_t M, uint32_t scale_kind, 
 
 namespace {
 
-// Shared checks of a batch; on success *sms is the device's SM count.
+// Shared checks of a batch: every layout valid, one coded dtype and one
+// stream format (state width) for all jobs; shapes and tiles may differ.  On
+// success *sms is the device's SM count.
 ans_status check_batch(const ans_gemm_job* jobs, uint32_t n_jobs, int* sms) {
   if (!jobs || n_jobs == 0 || n_jobs > ANS_MAX_BATCH) return ANS_ERR_ARG;
   for (uint32_t j = 0; j < n_jobs; ++j) {
@@ -414,27 +472,59 @@ ans_status check_batch(const ans_gemm_job* jobs, uint32_t n_jobs, int* sms) {
     if (st != ANS_OK) return st;
     const ans_layout& a = jobs[0].W->layout;
     const ans_layout& b = jobs[j].W->layout;
-    if (a.dtype != b.dtype || a.N != b.N || a.K != b.K || a.tile_n != b.tile_n ||
-        a.tile_k != b.tile_k || (a.state_bits == 64) != (b.state_bits == 64))
-      return ANS_ERR_SHAPE;
+    if (a.dtype != b.dtype || (a.state_bits == 64) != (b.state_bits == 64)) return ANS_ERR_SHAPE;
   }
   return device_info(sms);
 }
 
-// Plans of a batch: *share for one job on its share of the SMs (used when
-// it takes the small-M schedule, all jobs in one launch), *full for one job
-// on all SMs (consecutive launches otherwise); *ws_job the workspace bytes of
-// one job, enough for either.
+// SM shares of a batch in one launch, proportional to the jobs' weight
+// counts: G_j = max(1, floor(sms * w_j / sum w)); while the shares add up to
+// more than sms the largest gives one back; what is left over goes one each
+// to the first jobs.
+void batch_shares(const ans_gemm_job* jobs, uint32_t n, int sms, uint32_t* G) {
+  double total = 0;
+  for (uint32_t j = 0; j < n; ++j)
+    total += static_cast<double>(jobs[j].W->layout.N) * jobs[j].W->layout.K;
+  uint32_t sum = 0;
+  for (uint32_t j = 0; j < n; ++j) {
+    const double w = static_cast<double>(jobs[j].W->layout.N) * jobs[j].W->layout.K;
+    G[j] = static_cast<uint32_t>(static_cast<double>(sms) * w / total);
+    if (G[j] < 1) G[j] = 1;
+    sum += G[j];
+  }
+  while (sum > static_cast<uint32_t>(sms)) {
+    uint32_t big = 0;
+    for (uint32_t j = 1; j < n; ++j)
+      if (G[j] > G[big]) big = j;
+    if (G[big] <= 1) break;
+    --G[big];
+    --sum;
+  }
+  for (uint32_t j = 0; sum < static_cast<uint32_t>(sms) && j < n; ++j, ++sum) ++G[j];
+}
+
+// Plans of a batch: share[j] for job j on its share of the SMs (used when
+// every job takes the small-M schedule there: all jobs in one launch),
+// full[j] for job j on all SMs (consecutive launches otherwise); ws_off[j]
+// the byte offset of job j's workspace, ws_off[n] the total, each job's part
+// large enough for either plan.
 ans_status batch_plan(const ans_gemm_job* jobs, uint32_t n_jobs, uint32_t M,
                       ans_scale_kind scale_kind, int sms, ansdev::GemmPlan* share,
-                      ansdev::GemmPlan* full, size_t* ws_job) {
-  ansdev::LayerDev L;
-  fill_layer_plain(&jobs[0].W->layout, &L);
-  const int part = sms / static_cast<int>(n_jobs) > 0 ? sms / static_cast<int>(n_jobs) : 1;
-  if (!ansdev::make_gemm_plan(L, M, scale_kind, true, part, share)) return ANS_ERR_UNSUPPORTED;
-  if (!ansdev::make_gemm_plan(L, M, scale_kind, true, sms, full)) return ANS_ERR_UNSUPPORTED;
-  const size_t a = share->ws_bytes > full->ws_bytes ? share->ws_bytes : full->ws_bytes;
-  *ws_job = ((a + 255) / 256) * 256;
+                      ansdev::GemmPlan* full, size_t* ws_off, bool* one_launch) {
+  uint32_t G[ANS_MAX_BATCH];
+  batch_shares(jobs, n_jobs, sms, G);
+  *one_launch = true;
+  ws_off[0] = 0;
+  for (uint32_t j = 0; j < n_jobs; ++j) {
+    ansdev::LayerDev L;
+    fill_layer_plain(&jobs[j].W->layout, &L);
+    if (!ansdev::make_gemm_plan(L, M, scale_kind, true, static_cast<int>(G[j]), &share[j]))
+      return ANS_ERR_UNSUPPORTED;
+    if (!ansdev::make_gemm_plan(L, M, scale_kind, true, sms, &full[j])) return ANS_ERR_UNSUPPORTED;
+    if (!share[j].local || share[j].fmt != share[0].fmt) *one_launch = false;
+    const size_t a = share[j].ws_bytes > full[j].ws_bytes ? share[j].ws_bytes : full[j].ws_bytes;
+    ws_off[j + 1] = ws_off[j] + ((a + 255) / 256) * 256;
+  }
   return ANS_OK;
 }
 
@@ -449,11 +539,12 @@ ans_status ans_gemm_batched_workspace(const ans_gemm_job* jobs, uint32_t n_jobs,
   ans_status st = check_batch(jobs, n_jobs, &sms);
   if (st != ANS_OK) return st;
   if (M == 0) { *bytes = 0; return ANS_OK; }
-  ansdev::GemmPlan share, full;
-  size_t ws_job = 0;
-  st = batch_plan(jobs, n_jobs, M, scale_kind, sms, &share, &full, &ws_job);
+  ansdev::GemmPlan share[ANS_MAX_BATCH], full[ANS_MAX_BATCH];
+  size_t ws_off[ANS_MAX_BATCH + 1];
+  bool one = false;
+  st = batch_plan(jobs, n_jobs, M, scale_kind, sms, share, full, ws_off, &one);
   if (st != ANS_OK) return st;
-  *bytes = n_jobs * ws_job;
+  *bytes = ws_off[n_jobs];
   return ANS_OK;
 }
 
@@ -470,22 +561,11 @@ ans_status ans_gemm_batched(const ans_gemm_job* jobs, uint32_t n_jobs, uint32_t 
   float* Ys[ANS_MAX_BATCH];
   for (uint32_t j = 0; j < n_jobs; ++j) {
     const ans_tiles* W = jobs[j].W;
-    st = check_codebook(&W->codebook, W->layout.dtype);
+    st = check_gemm_tiles(W, scale_kind, jobs[j].d_scales, group_k);
     if (st != ANS_OK) return st;
-    st = check_scales(W->layout.dtype, scale_kind, jobs[j].d_scales, group_k, W->layout);
-    if (st != ANS_OK) return st;
-    if (!W->stream || !W->offsets) return ANS_ERR_ARG;
-    if (W->layout.dtype == ANS_BF16_SPLIT && !W->raw) return ANS_ERR_ARG;
-    if (reinterpret_cast<uintptr_t>(W->stream) % 16 != 0 ||
-        reinterpret_cast<uintptr_t>(W->offsets) % 8 != 0 ||
-        (W->raw && reinterpret_cast<uintptr_t>(W->raw) % 16 != 0))
-      return ANS_ERR_ARG;
     if (M > 0) {
-      if (!jobs[j].d_X || !jobs[j].d_Y) return ANS_ERR_ARG;
-      if (reinterpret_cast<uintptr_t>(jobs[j].d_X) % 16 != 0 ||
-          reinterpret_cast<uintptr_t>(jobs[j].d_Y) % 16 != 0 ||
-          (jobs[j].d_scales && reinterpret_cast<uintptr_t>(jobs[j].d_scales) % 16 != 0))
-        return ANS_ERR_ARG;
+      st = check_gemm_io(jobs[j].d_X, jobs[j].d_Y, d_status, jobs[j].d_scales);
+      if (st != ANS_OK) return st;
     }
     fill_layer(W, &Ls[j]);
     Lp[j] = &Ls[j];
@@ -494,22 +574,23 @@ ans_status ans_gemm_batched(const ans_gemm_job* jobs, uint32_t n_jobs, uint32_t 
     Ys[j] = jobs[j].d_Y;
   }
   if (M == 0) return ANS_OK;
-  if (!d_status || !d_ws || reinterpret_cast<uintptr_t>(d_ws) % 256 != 0) return ANS_ERR_ARG;
-  ansdev::GemmPlan share, full;
-  size_t ws_job = 0;
-  st = batch_plan(jobs, n_jobs, M, scale_kind, sms, &share, &full, &ws_job);
+  if (!d_ws || reinterpret_cast<uintptr_t>(d_ws) % 256 != 0) return ANS_ERR_ARG;
+  ansdev::GemmPlan share[ANS_MAX_BATCH], full[ANS_MAX_BATCH];
+  size_t ws_off[ANS_MAX_BATCH + 1];
+  bool one = false;
+  st = batch_plan(jobs, n_jobs, M, scale_kind, sms, share, full, ws_off, &one);
   if (st != ANS_OK) return st;
-  if (ws_bytes < n_jobs * ws_job) return ANS_ERR_BUFFER_TOO_SMALL;
+  if (ws_bytes < ws_off[n_jobs]) return ANS_ERR_BUFFER_TOO_SMALL;
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (share.local) {
+  if (one) {
     cudaError_t e = ansdev::launch_gemm_batched(share, n_jobs, Lp, Xs, Ss, scale_kind, group_k, Ys,
-                                                d_ws, d_status, s);
+                                                d_ws, ws_off, d_status, s);
     if (e != cudaSuccess) return cuda_fail(e, "ans_gemm_batched");
     return ANS_OK;
   }
   for (uint32_t j = 0; j < n_jobs; ++j) {
-    cudaError_t e = ansdev::launch_gemm(full, Ls[j], true, nullptr, Xs[j], Ss[j], scale_kind,
-                                        group_k, Ys[j], static_cast<uint8_t*>(d_ws) + j * ws_job,
+    cudaError_t e = ansdev::launch_gemm(full[j], Ls[j], true, nullptr, Xs[j], Ss[j], scale_kind,
+                                        group_k, Ys[j], static_cast<uint8_t*>(d_ws) + ws_off[j],
                                         d_status, s);
     if (e != cudaSuccess) return cuda_fail(e, "ans_gemm_batched");
   }

@@ -272,4 +272,28 @@ cudaError_t launch_histogram(const void* w, uint64_t n_bytes, uint32_t dtype, ui
   return cudaGetLastError();
 }
 
+// Internal test kernel: one thread makes one bounded wait, as the kernels'
+// waits run (wait_live), on an mbarrier that nothing ever arrives on; when the
+// budget runs out the status word gets the TIMEOUT bit and the kernel returns.
+__global__ void wait_probe_kernel(uint32_t* status) {
+  __shared__ uint64_t bar;
+  __shared__ uint32_t abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) wait_live(&bar, 0, &abort_flag, status, 0);
+}
+
+cudaError_t launch_wait_probe(uint32_t* status, cudaStream_t stream) {
+  wait_probe_kernel<<<1, 32, 0, stream>>>(status);
+  return cudaGetLastError();
+}
+
+cudaError_t set_live_wait_budget_decode(long long cycles) {
+  return cudaMemcpyToSymbol(g_live_wait_budget, &cycles, sizeof(cycles));
+}
+
 }  // namespace ansdev

@@ -23,10 +23,15 @@
 //     depend on timing and matches ans_gemm_uncompressed exactly.
 //   * A W row block split over several CTAs is reduced by the last CTA to
 //     finish it, in ascending CTA order (deterministic, no float atomics).
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
+#include <atomic>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 
 #include "gemm_common.cuh"
 #include "kernels.h"
@@ -36,11 +41,21 @@
 namespace ansdev {
 
 constexpr uint32_t kFixedWarps = 6;
-constexpr uint32_t kMaxProducers = 16;
+// 6 fixed warps + 14 producers = 20 warps: about 100 registers a thread, so
+// that the issuing warp and the producers run without spills
+constexpr uint32_t kMaxProducers = 14;
 constexpr uint32_t kMaxThreads = (kFixedWarps + kMaxProducers) * 32;
 
+// Barriers of one CTA, one array in this order:
+//   w_full[2 D]   producer d's slot k holds a slab (count 1)
+//   w_empty[2 D]  the MMAs that read producer d's slot k are done (one
+//                 commit per slab)
+//   x_full[XS]    X stage holds its slab (TMA bytes)
+//   x_rel[XS]     X chunk k (xe consecutive stages) is free again (one commit
+//                 per chunk, after its last stage's MMAs)
+//   acc_full[2], acc_empty[2], mma_done, chunk[4 D] (compressed-stream rings)
 struct Bars {
-  uint64_t *w_full, *w_empty, *x_full, *x_empty, *acc_full, *acc_empty, *mma_done, *chunk;
+  uint64_t *w_full, *w_empty, *x_full, *x_rel, *acc_full, *acc_empty, *mma_done, *chunk;
 };
 
 __device__ __forceinline__ Bars carve_bars(uint8_t* base, uint32_t D, uint32_t XS) {
@@ -49,8 +64,8 @@ __device__ __forceinline__ Bars carve_bars(uint8_t* base, uint32_t D, uint32_t X
   r.w_full = b;
   r.w_empty = b + 2 * D;
   r.x_full = b + 4 * D;
-  r.x_empty = b + 4 * D + XS;
-  r.acc_full = b + 4 * D + 2 * XS;
+  r.x_rel = r.x_full + XS;
+  r.acc_full = r.x_rel + XS;
   r.acc_empty = r.acc_full + 2;
   r.mma_done = r.acc_empty + 2;
   r.chunk = r.mma_done + 1;
@@ -59,6 +74,28 @@ __device__ __forceinline__ Bars carve_bars(uint8_t* base, uint32_t D, uint32_t X
 
 __host__ __device__ inline uint32_t num_bars(uint32_t D, uint32_t XS) {
   return 4 * D + 2 * XS + 5 + 4 * D;
+}
+
+// X stages are released in chunks of xe consecutive stages (one commit per
+// chunk): 4 when the ring has 16 or more, else one at a time (a small ring
+// must not wait for a whole chunk); the ring uses xs_used = a multiple of xe
+// of its stages.
+__device__ __forceinline__ uint32_t x_chunk(uint32_t XS) { return XS >= 16 ? 4u : 1u; }
+
+// Units of round r of a CTA: [u0, u0 + nd).  With one accumulator set a round
+// that reaches into the next W row block is consumed in two parts (its units
+// of the first segment, then the rest); returns the units of the first part.
+__device__ __forceinline__ uint32_t round_part0(const GemmDev& P, uint32_t u0, uint32_t nd) {
+  return P.n_bufs == 2 ? nd : min(nd, P.L.n_kt - u0 % P.L.n_kt);
+}
+
+// Wait until the MMAs that read producer d's slab q - 2 (the slab before q in
+// the same slot) are done, before slab q is written into that slot.
+__device__ __forceinline__ bool wait_slot(const Bars& B, uint32_t d, uint32_t q,
+                                          volatile uint32_t* abort, uint32_t* status,
+                                          uint32_t backoff_ns = 0) {
+  return q < 2 || wait_live(&B.w_empty[2 * d + (q & 1u)], ((q >> 1) + 1) & 1u, abort, status, 1,
+                            backoff_ns);
 }
 
 // Where a unit sits: K tile, token pass and W row-block segment, plus
@@ -113,6 +150,51 @@ __device__ __forceinline__ void for_each_mma_step(const GemmDev& P, uint32_t u_b
 }
 
 // ---------------------------------------------------------------------------
+// Producer side of one W slab in copy mode (ans_gemm_uncompressed): the slab
+// (rows n0 + 128 h .. + 127, columns k0 + 16 s .. + 15) formatted like the
+// decoded one.  kCopyLoads: per-lane global loads of the packed nibbles.
+template <uint32_t kFmt>
+__device__ __forceinline__ void copy_loads(const GemmDev& P, uint32_t n0, uint32_t k0, uint32_t h,
+                                           uint32_t s, uint32_t lane, uint4 (&cp)[8]) {
+#pragma unroll
+  for (int gg = 0; gg < 8; ++gg) {
+    const uint32_t i = gg & 3, c = gg >> 2;
+    const uint64_t row = n0 + lane + 32 * (4 * h + i);
+    const uint64_t idx = row * P.L.K + k0 + 16 * s + 8 * c;
+    const uint32_t v =
+        __ldg(reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(P.w_plain) + idx / 2));
+    cp[gg] = make_uint4(v, 0, 0, 0);
+  }
+}
+
+// Eight packed-nibble codes (one 32-bit word, element k in bits 4k..4k+3) as
+// slot-table-like entries (symbol at bits 12..19), then the format's operand.
+template <uint32_t kFmt>
+__device__ __forceinline__ void copy_nibbles_fmt(uint32_t v, __half2 gs, uint32_t (&o)[4]) {
+  uint32_t e[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    e[k] = (((v >> (4 * k)) & 0xFu) ^ (kFmt == kFmtFp4Bf16 ? 0u : 8u)) << 12;
+  if constexpr (kFmt == kFmtFp4Bf16) fmt_fp4_bf16(e, o);
+  else if constexpr (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
+  else fmt_int4_f16_scaled(e, gs, o);
+}
+
+// Eight 1-byte codes (two 32-bit words) as the format's operand.
+template <uint32_t kFmt>
+__device__ __forceinline__ void copy_bytes_fmt(uint32_t lo, uint32_t hi, uint32_t (&o)[4]) {
+  const uint32_t flip = kFmt == kFmtInt8F16 ? 0x80u : 0u;  // int8: symbol = byte ^ 0x80
+  uint32_t e[8];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    e[k] = (((lo >> (8 * k)) & 0xFFu) ^ flip) << 12;
+    e[k + 4] = (((hi >> (8 * k)) & 0xFFu) ^ flip) << 12;
+  }
+  if constexpr (kFmt == kFmtInt8F16) fmt_int8_f16(e, o);
+  else fmt_fp8_f16(e, o);
+}
+
+// ---------------------------------------------------------------------------
 template <bool kDecode, uint32_t kFmt, bool kWide>
 __global__ void __launch_bounds__(kMaxThreads, 1)
     fused_gemm_kernel(const __grid_constant__ GemmDev P) {
@@ -145,6 +227,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     reduce_flag = 0;
   }
   {
+    // arrivals per phase: the epilogue's four warps on acc_empty, one otherwise
     uint64_t* b0 = B.w_full;  // the barriers are one array, in carve_bars order
     const uint32_t n_bars = num_bars(D, XS);
     for (uint32_t i = threadIdx.x; i < n_bars; i += blockDim.x)
@@ -156,6 +239,9 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     tmem_relinquish();
   } else if (kDecode && P.L.single_symbol == kNoSymbol) {
     build_lut(lut, P.L, warp - 1, blockDim.x / 32 - 1, lane);
+  } else if (warp == 5 && lane == 0) {
+    prefetch_tmap(&P.tmap_x);
+    if (!kDecode && copy_mode_of(kFmt) != kCopyLoads) prefetch_tmap(&P.tmap_w);
   }
   tc_fence_before();
   __syncthreads();
@@ -163,289 +249,385 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
   const uint32_t tmem_base = tmem_slot;
   volatile uint32_t* abort = &abort_flag;
   // the prologue above read only kernel parameters: from here on global
-  // memory, after the previous grid in the stream (X staging) has completed
+  // memory, after the previous grid in the stream has completed
   griddep_wait();
   griddep_launch_dependents();
+  check_smem_base(smem, P.status);
   if (threadIdx.x == 0) trace_mark(P, 0);
 
   if (warp >= kFixedWarps) {
     // ======================= producer warps =======================
     const uint32_t d = warp - kFixedWarps;
-    const uint32_t lt = lanemask_lt();
     const LayerDev& L = P.L;
-    const bool single = L.single_symbol != kNoSymbol;
     const uint32_t H = P.H;
-    const uint32_t n_slabs = P.H * P.C;
-    const uint32_t groups = n_slabs * 8;  // 8 groups of 8 symbols per lane fill one slab
-    const uint32_t lut_s = smem_u32(lut);
+    const uint32_t n_us = P.H * P.C;  // slabs per unit
     TileSeq seq{static_cast<uint32_t>(u_begin) + d, D, static_cast<uint32_t>(u_end), L.n_tiles};
-    ChunkPipe pipe;
-    pipe_init(pipe, chunks + d * kRingStride, B.chunk + 4 * d);
-    TileCursor tc;
-    tc.cb = 0;
-    uint32_t sc = 0;  // unit slabs produced
     const uint32_t swz = ((lane >> 2) & 1u) << 4;
     const uint32_t wslots_s = smem_u32(wring + 2 * d * kSlabBytes);
+    constexpr uint32_t kCopy = kDecode ? kCopyLoads : copy_mode_of(kFmt);
 
-    for (uint32_t r = 0; seq.has(r); ++r) {
-      const uint32_t t = seq.at(r);
-      const uint32_t n0 = (t / n_kt) * L.tile_n, k0 = (t % n_kt) * L.tile_k;
-      bool zero_tile = false;
-      if (kDecode) {
-        if (!tile_begin(pipe, L, seq, t, tc, lane, abort, P.status)) {
-          zero_tile = true;
-          if (lane == 0) atomicOr(P.status, kStatusBadOffsets);
-        }
-      }
-      __half2 gscale[8];
-      if (fmt_group(kFmt)) {
-        const uint32_t gk = k0 / P.group_k;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const uint32_t hh = q / 4, ii = q % 4;
-          float sv = 0.f;
-          if (hh < H) {
-            const uint32_t row = n0 + lane + 32 * (4 * hh + ii);
-            sv = bf16_to_f32(__ldg(static_cast<const uint16_t*>(P.scales) +
-                                   static_cast<uint64_t>(row) * P.n_groups_k + gk));
+    if constexpr (!kDecode && kCopy == kCopyTmaSlab) {
+      // ---- bf16 weights: one TMA box per slab, straight into the slot (the
+      // box's 32-byte swizzle is the slab layout); one lane works
+      if (lane == 0) {
+        uint32_t q = 0;  // slabs issued
+        for (uint32_t r = 0; seq.has(r) && !*abort; ++r) {
+          const uint32_t t = seq.at(r);
+          const uint32_t n0 = (t / n_kt) * L.tile_n, k0 = (t % n_kt) * L.tile_k;
+          for (uint32_t us = 0; us < n_us; ++us, ++q) {
+            const uint32_t h = us % H, s = us / H, slot = q & 1u;
+            if (!wait_slot(B, d, q, abort, P.status)) break;
+            const uint32_t bar = smem_u32(&B.w_full[2 * d + slot]);
+            mbar_arrive_expect_tx_s(bar, kSlabBytes);
+            tma_load_2d_hint_s(wslots_s + slot * kSlabBytes, &P.tmap_w,
+                               static_cast<int32_t>(k0 + 16 * s), static_cast<int32_t>(n0 + 128 * h),
+                               bar, l2_evict_first());
           }
-          gscale[q] = __float2half2_rn(sv);
+          if (*abort) break;
         }
+        // copies still in flight (only after an abort) land before exit
+        for (uint32_t k = q > 2 ? q - 2 : 0; k < q; ++k)
+          wait_drain(&B.w_full[2 * d + (k & 1u)], (k >> 1) & 1u, P.status);
       }
-      // raw sign/mantissa bytes of groups g, g+1, g+2 in flight (bf16, decode)
-      const unsigned long long* raw_tile = nullptr;
-      uint64_t r0 = 0, r1 = 0, r2 = 0;
-      if (kDecode && kFmt == kFmtBf16Split && !zero_tile) {
-        raw_tile = reinterpret_cast<const unsigned long long*>(
-                       L.raw + static_cast<uint64_t>(t) * (L.tile_n * L.tile_k)) + lane;
-        r0 = __ldg(raw_tile);
-        r1 = __ldg(raw_tile + 32);
-        r2 = __ldg(raw_tile + 64);
-      }
-
-      for (uint32_t us = 0; us < n_slabs; ++us) {
+      __syncwarp();
+    } else if constexpr (!kDecode && kCopy == kCopyTmaRaw) {
+      // ---- 1-byte codes: the raw 128 x 16-byte box of each slab lands in a
+      // two-stage ring (the decode variant's chunk ring), the lanes format it
+      // into the slot: lane l owns rows l, l + 32, l + 64, l + 96
+      const uint32_t raw_s = smem_u32(chunks + d * kRingStride);
+      uint64_t* raw_bar = B.chunk + 4 * d;
+      uint32_t n_slabs = 0;
+      for (uint32_t r = 0; seq.has(r); ++r) n_slabs += n_us;
+      auto issue_raw = [&](uint32_t q) {  // lane 0: the raw box of slab q into stage q & 1
+        const uint32_t r = q / n_us, us = q - r * n_us;
+        const uint32_t t = seq.at(r);
+        const uint32_t n0 = (t / n_kt) * L.tile_n, k0 = (t % n_kt) * L.tile_k;
         const uint32_t h = us % H, s = us / H;
-        const uint32_t slot = sc & 1u;
-        // group scales of this lane's four rows in half h (int4 x group scale)
-        __half2 gs0, gs1, gs2, gs3;
-        if (fmt_group(kFmt)) {
-          gs0 = h ? gscale[4] : gscale[0];
-          gs1 = h ? gscale[5] : gscale[1];
-          gs2 = h ? gscale[6] : gscale[2];
-          gs3 = h ? gscale[7] : gscale[3];
-        }
-        // copy mode: fetch the slab's 8 groups before waiting for the slot
-        uint4 cp[8];
-        if (!kDecode) {
+        const uint32_t bar = smem_u32(&raw_bar[q & 1u]);
+        mbar_arrive_expect_tx_s(bar, 128 * 16);
+        tma_load_2d_hint_s(raw_s + (q & 1u) * 2048, &P.tmap_w, static_cast<int32_t>(k0 + 16 * s),
+                           static_cast<int32_t>(n0 + 128 * h), bar, l2_evict_first());
+      };
+      uint32_t issued = 0;
+      if (lane == 0)
+        for (; issued < 2 && issued < n_slabs; ++issued) issue_raw(issued);
+      issued = __shfl_sync(0xFFFFFFFFu, issued, 0);
+      uint32_t q = 0;
+      for (; q < n_slabs; ++q) {
+        const uint32_t slot = q & 1u;
+        const bool got = wait_live(&raw_bar[slot], (q >> 1) & 1u, abort, P.status, 7);
+        if (__any_sync(0xFFFFFFFFu, !got)) break;  // warp-uniform exit
+        uint4 v[4];
 #pragma unroll
-          for (int gg = 0; gg < 8; ++gg) {
-            const uint32_t i = gg & 3, c = gg >> 2;
-            const uint64_t row = n0 + lane + 32 * (4 * h + i);
-            const uint64_t idx = row * L.K + k0 + 16 * s + 8 * c;
-            if (kFmt == kFmtBf16Split) {
-              cp[gg] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(P.w_plain) + idx));
-            } else if (kFmt == kFmtFp8F16 || kFmt == kFmtInt8F16) {
-              uint2 v = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(P.w_plain) + idx));
-              cp[gg] = make_uint4(v.x, v.y, 0, 0);
-            } else {
-              uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(P.w_plain) + idx / 2));
-              cp[gg] = make_uint4(v, 0, 0, 0);
-            }
-          }
-        }
-        if (sc >= 2) wait_live(&B.w_empty[2 * d + slot], ((sc >> 1) + 1) & 1u, abort, P.status, 1, 64);
-        const uint32_t slab_s = wslots_s + slot * kSlabBytes;
-        // a group is 8 columns of one row, or both 8-column halves of it for
-        // int4 pair symbols (4 groups per slab)
-        constexpr bool kPair = fmt_pair(kFmt);
-        constexpr uint32_t kGroups = kPair ? 4 : 8, kOut = kPair ? 8 : 4;
-#pragma unroll 1
-        for (uint32_t gg = 0; gg < kGroups; ++gg) {
-          const uint32_t g = us * 8 + gg;
-          const uint32_t i = gg & 3, c = gg >> 2;
-          uint32_t o[kOut];
-          if (kDecode) {
-            const uint64_t raw8 = r0;
-            if (kFmt == kFmtBf16Split && !zero_tile) {
-              r0 = r1;
-              r1 = r2;
-              if (g + 3 < groups) r2 = __ldg(raw_tile + 32 * (g + 3));
-            }
-            uint32_t e[8];
-            if (zero_tile) {
-#pragma unroll
-              for (int k = 0; k < 8; ++k) e[k] = 0;
-            } else if (single) {
-#pragma unroll
-              for (int k = 0; k < 8; ++k) e[k] = L.single_symbol << 12;
-            } else {
-              tile_group(pipe, L, seq, tc, lane, abort, P.status);
-              decode_group<kWide>(tc, lut_s, pipe.ring_s, lt, e);
-            }
-            if constexpr (kFmt == kFmtInt4PairBf16) fmt_int4pair_bf16(e, o);
-            else if constexpr (kFmt == kFmtFp4PairBf16) fmt_fp4pair_bf16(e, o);
-            else if constexpr (kFmt == kFmtInt4PairF16Group)
-              fmt_int4pair_f16_scaled(e, i == 0 ? gs0 : i == 1 ? gs1 : i == 2 ? gs2 : gs3, o);
-            else if constexpr (kFmt == kFmtBf16Split) fmt_bf16_split(e, raw8, o);
-            else if constexpr (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
-            else if constexpr (kFmt == kFmtInt4F16Group)
-              fmt_int4_f16_scaled(e, i == 0 ? gs0 : i == 1 ? gs1 : i == 2 ? gs2 : gs3, o);
-            else if constexpr (kFmt == kFmtInt8F16) fmt_int8_f16(e, o);
-            else if constexpr (kFmt == kFmtFp4Bf16) fmt_fp4_bf16(e, o);
-            else fmt_fp8_f16(e, o);
-            if (zero_tile) {
-#pragma unroll
-              for (uint32_t k = 0; k < kOut; ++k) o[k] = 0;
-            }
-          } else if constexpr (!kPair) {
-            uint4 v = cp[0];
-#pragma unroll
-            for (int q = 1; q < 8; ++q)
-              if (gg == static_cast<uint32_t>(q)) v = cp[q];
-            if (kFmt == kFmtBf16Split) {
-              o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
-            } else {
-              uint32_t e[8];
-              if (kFmt == kFmtFp8F16 || kFmt == kFmtInt8F16) {
-                  const uint32_t flip = kFmt == kFmtInt8F16 ? 0x80u : 0u;  // int8: symbol = byte ^ 0x80
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                  e[k] = (((v.x >> (8 * k)) & 0xFFu) ^ flip) << 12;
-                  e[k + 4] = (((v.y >> (8 * k)) & 0xFFu) ^ flip) << 12;
-                }
-                if constexpr (kFmt == kFmtInt8F16) fmt_int8_f16(e, o);
-                else fmt_fp8_f16(e, o);
-              } else {
-#pragma unroll
-                for (int k = 0; k < 8; ++k) e[k] = (((v.x >> (4 * k)) & 0xFu) ^ (kFmt == kFmtFp4Bf16 ? 0u : 8u)) << 12;
-                if (kFmt == kFmtFp4Bf16) fmt_fp4_bf16(e, o);
-                else if (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
-                else fmt_int4_f16_scaled(e, i == 0 ? gs0 : i == 1 ? gs1 : i == 2 ? gs2 : gs3, o);
-              }
-            }
-          }
-          const uint32_t row_s = slab_s + (32 * i + lane) * 32;
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row_s + ((c << 4) ^ swz)),
-                       "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3])
+        for (int i = 0; i < 4; ++i)
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(v[i].x), "=r"(v[i].y), "=r"(v[i].z), "=r"(v[i].w)
+                       : "r"(raw_s + slot * 2048 + (32 * i + lane) * 16)
                        : "memory");
-          if constexpr (kPair)
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row_s + (16u ^ swz)),
-                         "r"(o[kOut - 4]), "r"(o[kOut - 3]), "r"(o[kOut - 2]), "r"(o[kOut - 1])
+        // the stage is free once every lane has read it: refill it
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && q + 2 < n_slabs && !*abort) {
+          issue_raw(q + 2);
+          issued = q + 3;
+        }
+        issued = __shfl_sync(0xFFFFFFFFu, issued, 0);
+        uint32_t o[4][2][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          copy_bytes_fmt<kFmt>(v[i].x, v[i].y, o[i][0]);
+          copy_bytes_fmt<kFmt>(v[i].z, v[i].w, o[i][1]);
+        }
+        const bool free_slot = wait_slot(B, d, q, abort, P.status);
+        if (__any_sync(0xFFFFFFFFu, !free_slot)) break;
+        const uint32_t slab_s = wslots_s + slot * kSlabBytes;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t row_s = slab_s + (32 * i + lane) * 32;
+#pragma unroll
+          for (uint32_t c = 0; c < 2; ++c)
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row_s + ((c << 4) ^ swz)),
+                         "r"(o[i][c][0]), "r"(o[i][c][1]), "r"(o[i][c][2]), "r"(o[i][c][3])
                          : "memory");
         }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&B.w_full[2 * d + slot]);
-        if (lane == 0 && sc == 0) trace_mark(P, 2 + d);
-        ++sc;
       }
-      if (kDecode && !zero_tile) {
-        if (!tile_end(L, tc, single) && lane == 0) atomicOr(P.status, kStatusCorrupt);
+      // raw boxes still in flight (only after an abort) land before exit
+      if (lane == 0)
+        for (uint32_t k = q; k < issued; ++k) wait_drain(&raw_bar[k & 1u], (k >> 1) & 1u, P.status);
+      __syncwarp();
+    } else {
+      // ---- decode (ans_gemm), or per-lane loads of packed nibbles (copy)
+      const uint32_t lt = lanemask_lt();
+      const bool single = L.single_symbol != kNoSymbol;
+      const uint32_t n_slabs = P.H * P.C;
+      const uint32_t groups = n_slabs * 8;  // 8 groups of 8 symbols per lane fill one slab
+      const uint32_t lut_s = smem_u32(lut);
+      ChunkPipe pipe;
+      pipe_init(pipe, chunks + d * kRingStride, B.chunk + 4 * d);
+      TileCursor tc;
+      tc.cb = 0;
+      uint32_t sc = 0;  // unit slabs produced
+
+      for (uint32_t r = 0; seq.has(r); ++r) {
+        const uint32_t t = seq.at(r);
+        const uint32_t n0 = (t / n_kt) * L.tile_n, k0 = (t % n_kt) * L.tile_k;
+        bool zero_tile = false;
+        if (kDecode) {
+          if (!tile_begin(pipe, L, seq, t, tc, lane, abort, P.status)) {
+            zero_tile = true;
+            if (lane == 0) atomicOr(P.status, kStatusBadOffsets);
+          }
+        }
+        __half2 gscale[8];
+        if (fmt_group(kFmt)) {
+          const uint32_t gk = k0 / P.group_k;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const uint32_t hh = q / 4, ii = q % 4;
+            float sv = 0.f;
+            if (hh < H) {
+              const uint32_t row = n0 + lane + 32 * (4 * hh + ii);
+              sv = bf16_to_f32(__ldg(static_cast<const uint16_t*>(P.scales) +
+                                     static_cast<uint64_t>(row) * P.n_groups_k + gk));
+            }
+            gscale[q] = __float2half2_rn(sv);
+          }
+        }
+        // raw sign/mantissa bytes of groups g, g+1, g+2 in flight (bf16, decode)
+        const unsigned long long* raw_tile = nullptr;
+        uint64_t r0 = 0, r1 = 0, r2 = 0;
+        if (kDecode && kFmt == kFmtBf16Split && !zero_tile) {
+          raw_tile = reinterpret_cast<const unsigned long long*>(
+                         L.raw + static_cast<uint64_t>(t) * (L.tile_n * L.tile_k)) + lane;
+          r0 = __ldg(raw_tile);
+          r1 = __ldg(raw_tile + 32);
+          r2 = __ldg(raw_tile + 64);
+        }
+
+        for (uint32_t us = 0; us < n_slabs; ++us) {
+          const uint32_t h = us % H, s = us / H;
+          const uint32_t slot = sc & 1u;
+          // group scales of this lane's four rows in half h (int4 x group scale)
+          __half2 gs0, gs1, gs2, gs3;
+          if (fmt_group(kFmt)) {
+            gs0 = h ? gscale[4] : gscale[0];
+            gs1 = h ? gscale[5] : gscale[1];
+            gs2 = h ? gscale[6] : gscale[2];
+            gs3 = h ? gscale[7] : gscale[3];
+          }
+          // copy mode: fetch the slab's 8 groups before waiting for the slot
+          uint4 cp[8];
+          if constexpr (!kDecode) copy_loads<kFmt>(P, n0, k0, h, s, lane, cp);
+          wait_slot(B, d, sc, abort, P.status, 64);
+          const uint32_t slab_s = wslots_s + slot * kSlabBytes;
+          // a group is 8 columns of one row, or both 8-column halves of it for
+          // int4 pair symbols (4 groups per slab)
+          constexpr bool kPair = fmt_pair(kFmt);
+          constexpr uint32_t kGroups = kPair ? 4 : 8, kOut = kPair ? 8 : 4;
+#pragma unroll 1
+          for (uint32_t gg = 0; gg < kGroups; ++gg) {
+            const uint32_t g = us * 8 + gg;
+            const uint32_t i = gg & 3, c = gg >> 2;
+            uint32_t o[kOut];
+            if (kDecode) {
+              const uint64_t raw8 = r0;
+              if (kFmt == kFmtBf16Split && !zero_tile) {
+                r0 = r1;
+                r1 = r2;
+                if (g + 3 < groups) r2 = __ldg(raw_tile + 32 * (g + 3));
+              }
+              uint32_t e[8];
+              if (zero_tile) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) e[k] = 0;
+              } else if (single) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) e[k] = L.single_symbol << 12;
+              } else {
+                tile_group(pipe, L, seq, tc, lane, abort, P.status);
+                decode_group<kWide>(tc, lut_s, pipe.ring_s, lt, e);
+              }
+              if constexpr (kFmt == kFmtInt4PairBf16) fmt_int4pair_bf16(e, o);
+              else if constexpr (kFmt == kFmtFp4PairBf16) fmt_fp4pair_bf16(e, o);
+              else if constexpr (kFmt == kFmtInt4PairF16Group)
+                fmt_int4pair_f16_scaled(e, i == 0 ? gs0 : i == 1 ? gs1 : i == 2 ? gs2 : gs3, o);
+              else if constexpr (kFmt == kFmtBf16Split) fmt_bf16_split(e, raw8, o);
+              else if constexpr (kFmt == kFmtInt4Bf16) fmt_int4_bf16(e, o);
+              else if constexpr (kFmt == kFmtInt4F16Group)
+                fmt_int4_f16_scaled(e, i == 0 ? gs0 : i == 1 ? gs1 : i == 2 ? gs2 : gs3, o);
+              else if constexpr (kFmt == kFmtInt8F16) fmt_int8_f16(e, o);
+              else if constexpr (kFmt == kFmtFp4Bf16) fmt_fp4_bf16(e, o);
+              else fmt_fp8_f16(e, o);
+              if (zero_tile) {
+#pragma unroll
+                for (uint32_t k = 0; k < kOut; ++k) o[k] = 0;
+              }
+            } else if constexpr (!kPair) {
+              uint4 v = cp[0];
+#pragma unroll
+              for (int q = 1; q < 8; ++q)
+                if (gg == static_cast<uint32_t>(q)) v = cp[q];
+              copy_nibbles_fmt<kFmt>(v.x, i == 0 ? gs0 : i == 1 ? gs1 : i == 2 ? gs2 : gs3, o);
+            }
+            const uint32_t row_s = slab_s + (32 * i + lane) * 32;
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row_s + ((c << 4) ^ swz)),
+                         "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3])
+                         : "memory");
+            if constexpr (kPair)
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row_s + (16u ^ swz)),
+                           "r"(o[kOut - 4]), "r"(o[kOut - 3]), "r"(o[kOut - 2]), "r"(o[kOut - 1])
+                           : "memory");
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&B.w_full[2 * d + slot]);
+          if (lane == 0 && sc == 0) trace_mark(P, 2 + d);
+          ++sc;
+        }
+        if (kDecode && !zero_tile) {
+          if (!tile_end(L, tc, single) && lane == 0) atomicOr(P.status, kStatusCorrupt);
+        }
       }
+      if (kDecode) pipe_drain(pipe, P.status);
     }
-    if (kDecode) pipe_drain(pipe, P.status);
     if (lane == 0) trace_mark(P, 18 + d);
   } else if (warp == 4) {
-    // ======================= MMA issue (one thread) =======================
-    if (lane == 0) {
-      const uint32_t ub = static_cast<uint32_t>(u_begin), ue = static_cast<uint32_t>(u_end);
-      const uint32_t seg_begin = ub / n_kt;
-      // descriptor fields shared by every operand: LBO 16 B, SBO 256 B,
-      // version 1, 32-byte swizzle; only the start address varies
-      const uint64_t dhi = (1ull << 16) | (16ull << 32) | (1ull << 46) | (6ull << 61);
-      const uint32_t a_base = smem_u32(wring) >> 4, x_base = smem_u32(xring) >> 4;
-      const uint32_t slab16 = kSlabBytes >> 4, xstage16 = x_stage_bytes >> 4, t16 = (P.T * 32) >> 4;
-      uint32_t fresh = 0;  // bit (buf * 2 + h): next MMA into that accumulator starts it
-      uint32_t xs = 0, xpar = 0;
-      uint32_t r = 0;
-      for (uint32_t u0 = ub; u0 < ue; u0 += D, ++r) {
-        const uint32_t nd = min(D, ue - u0);
-        const uint32_t seg0 = u0 / n_kt, kt0 = u0 - seg0 * n_kt;
-        const uint32_t nA = P.n_bufs == 2 ? nd : min(nd, n_kt - kt0);
-        for (uint32_t part = 0; part < 2; ++part) {
-          const uint32_t d_lo = part == 0 ? 0 : nA, d_hi = part == 0 ? nA : nd;
-          for (uint32_t s = 0; s < P.C; ++s) {
+    // ======================= MMA issue =======================
+    // Slabs are consumed in a fixed order (round, part, slab, producer, half),
+    // so the accumulation order does not depend on timing.  For every (round,
+    // part, slab) group the warp's lanes first test the W barriers of all its
+    // producers at once (one round trip instead of one per producer), then
+    // lane 0 issues the group's MMAs.  Where TMEM has room the units are
+    // spread over accumulator banks -- unit u into bank (u - u_begin) % banks,
+    // each bank accumulated in unit order and the banks summed in bank order
+    // by the epilogue -- so consecutive MMAs go to different accumulators.
+    // Each W slot is released by a commit right after its MMAs (so its
+    // producer can write the next slab as early as possible), the X stages by
+    // one commit per chunk.
+    const uint32_t ub = static_cast<uint32_t>(u_begin), ue = static_cast<uint32_t>(u_end);
+    const uint32_t seg_begin = ub / n_kt;
+    const uint32_t H = P.H, NT = P.NT, NB = P.n_banks;
+    const uint32_t XE = x_chunk(XS), XSu = XS - XS % XE;
+    // descriptor fields shared by every operand: LBO 16 B, SBO 256 B,
+    // version 1, 32-byte swizzle; only the start address varies
+    const uint64_t dhi = (1ull << 16) | (16ull << 32) | (1ull << 46) | (6ull << 61);
+    const uint32_t a_base = smem_u32(wring) >> 4, x_base = smem_u32(xring) >> 4;
+    const uint32_t slab16 = kSlabBytes >> 4, xstage16 = x_stage_bytes >> 4, t16 = (P.T * 32) >> 4;
+    uint32_t n = 0;  // MMA steps (X stages) of the CTA before the current group
+    uint32_t g = 0;  // groups consumed
+    uint32_t r = 0;
+    bool live = true;
+    for (uint32_t u0 = ub; u0 < ue && live; u0 += D, ++r) {
+      const uint32_t nd = min(D, ue - u0);
+      const uint32_t seg0 = u0 / n_kt, kt0 = u0 - seg0 * n_kt;
+      const uint32_t nA = round_part0(P, u0, nd);
+      for (uint32_t part = 0; part < 2 && live; ++part) {
+        const uint32_t d_lo = part == 0 ? 0 : nA, d_hi = part == 0 ? nA : nd;
+        if (d_lo == d_hi) continue;
+        for (uint32_t s = 0; s < P.C && live; ++s, ++g) {
+          // readiness of every W slab of the group, one lane per (producer, half)
+          bool ok = true;
+          const uint32_t ng = (d_hi - d_lo) * H;
+          if (lane < ng) {
+            const uint32_t dd = d_lo + lane / H, hh = lane % H;
+            const uint32_t idx = (r * P.C + s) * H + hh;
+            ok = wait_live(&B.w_full[2 * dd + (idx & 1u)], (idx >> 1) & 1u, abort, P.status, 3);
+          }
+          if (__ballot_sync(0xFFFFFFFFu, !ok) != 0) live = false;
+          if (!live) break;
+          if (lane == 0) {
+            if (g == 0) trace_mark(P, 48);
+            tc_fence_after();
             for (uint32_t d = d_lo; d < d_hi; ++d) {
               const uint32_t kt = kt0 + d;
               const bool wrap = kt >= n_kt;
               const uint32_t ktw = wrap ? kt - n_kt : kt;
               const uint32_t lseg = seg0 + (wrap ? 1u : 0u) - seg_begin;
               const uint32_t buf = P.n_bufs == 2 ? (lseg & 1u) : 0u;
-              if (s == 0 && (u0 + d == ub || ktw == 0)) {
+              const uint32_t u = u0 + d;
+              const uint32_t bank = (u - ub) % NB;
+              const uint32_t step = n + (d - d_lo);
+              // the segment's units in this CTA start at u_first; its first
+              // NB units start one bank each (their first slab), and the first
+              // one waits until the epilogue has drained the buffer
+              const uint32_t u_first = max(ub, (seg_begin + lseg) * n_kt);
+              const bool start = s == 0 && u - u_first < NB;
+              if (start && u == u_first) {
                 const uint32_t k = P.n_bufs == 2 ? (lseg >> 1) : lseg;
-                if (k >= 1) wait_live(&B.acc_empty[buf], (k - 1) & 1u, abort, P.status, 4);
-                tc_fence_after();
-                fresh |= 3u << (2 * buf);
-              }
-              wait_live(&B.x_full[xs], xpar, abort, P.status, 2);
-              for (uint32_t h = 0; h < P.H; ++h) {
-                const uint32_t idx = (r * P.C + s) * P.H + h;
-                const uint32_t slot = idx & 1u;
-                wait_live(&B.w_full[2 * d + slot], (idx >> 1) & 1u, abort, P.status, 3);
-                tc_fence_after();
-                const uint64_t adesc = dhi | (a_base + (2 * d + slot) * slab16);
-                const uint32_t acc_bit = 1u << (2 * buf + h);
-                const uint32_t accumulate = (fresh & acc_bit) ? 0u : 1u;
-                for (uint32_t j = 0; j < P.NT; ++j) {
-                  const uint64_t bdesc = dhi | (x_base + xs * xstage16 + j * t16);
-                  const uint32_t col = ((buf * P.H + h) * P.NT + j) * P.T;
-                  umma_f16(tmem_base + col, adesc, bdesc, P.idesc, accumulate);
+                if (k >= 1 && !wait_live(&B.acc_empty[buf], (k - 1) & 1u, abort, P.status, 4)) {
+                  live = false;
+                  break;
                 }
-                fresh &= ~acc_bit;
-                umma_commit(&B.w_empty[2 * d + slot]);
+                tc_fence_after();
               }
-              umma_commit(&B.x_empty[xs]);
-              if (++xs == XS) { xs = 0; xpar ^= 1u; }
+              const uint32_t xs = step % XSu;
+              if (!wait_live(&B.x_full[xs], (step / XSu) & 1u, abort, P.status, 2)) {
+                live = false;
+                break;
+              }
+              for (uint32_t h = 0; h < H; ++h) {
+                const uint32_t idx = (r * P.C + s) * H + h;
+                const uint64_t adesc = dhi | (a_base + (2 * d + (idx & 1u)) * slab16);
+                for (uint32_t j = 0; j < NT; ++j) {
+                  const uint64_t bdesc = dhi | (x_base + xs * xstage16 + j * t16);
+                  const uint32_t col = (((buf * NB + bank) * H + h) * NT + j) * P.T;
+                  umma_f16(tmem_base + col, adesc, bdesc, P.idesc, start ? 0u : 1u);
+                }
+                // the slot is free for its producer once these MMAs are done
+                umma_commit(&B.w_empty[2 * d + (idx & 1u)]);
+              }
+              // the last stage of an X chunk: the chunk is free once these MMAs are done
+              if (step % XE == XE - 1) umma_commit(&B.x_rel[xs / XE]);
               if (s == P.C - 1 && (u0 + d + 1 == ue || ktw + 1 == n_kt))
                 umma_commit(&B.acc_full[buf]);
             }
           }
-          if (P.n_bufs == 2) break;  // one part: the whole round slab-major
+          live = __shfl_sync(0xFFFFFFFFu, live ? 1u : 0u, 0) != 0;
+          n += d_hi - d_lo;
         }
       }
+    }
+    if (lane == 0) {
       umma_commit(B.mma_done);
       trace_mark(P, 34);
     }
     __syncwarp();
   } else if (warp == 5) {
-    // ======================= X loader (TMA, one thread) =======================
+    // ============ X loader (TMA from the tensor map, one thread) ============
+    // X slab (token pass p, columns kx .. kx + 15) is the tensor map's box at
+    // (kx, p * T_pass + j * T) for j < NT; rows past M land as zeros.
     if (lane == 0) {
+      const uint32_t XE = x_chunk(XS), XSu = XS - XS % XE;
       uint32_t xc = 0;
       uint32_t n_issued = 0;  // loads issued: steps [0, n_issued) (none after an abort)
-      long long xw = 0, xi = 0;
-      const long long xb = clock64();
+      const uint32_t xring_s = smem_u32(xring);
       for_each_mma_step(P, static_cast<uint32_t>(u_begin), static_cast<uint32_t>(u_end),
                         [&](uint32_t, uint32_t s, uint32_t, uint32_t, const UnitInfo& I) {
-        const uint32_t xs = xc % XS;
-        long long c0 = clock64();
-        if (xc >= XS) wait_live(&B.x_empty[xs], ((xc / XS) + 1) & 1u, abort, P.status, 5);
-        xw += clock64() - c0;
-        c0 = clock64();
-        const uint32_t p = I.p;
-        const uint32_t kx = I.kt * P.L.tile_k + 16 * s;
+        const uint32_t xs = xc % XSu;
+        // the stage's chunk was released by its last use (one lap earlier)
+        if (xc >= XSu) wait_live(&B.x_rel[xs / XE], ((xc / XSu) - 1) & 1u, abort, P.status, 5, 32);
         if (!*abort && n_issued == xc) {
-          // X slab (pass p, 16-column slab kx/16) is T_pass x 32 contiguous,
-          // pre-swizzled bytes in the staged copy: one bulk copy
-          const uint64_t slab = static_cast<uint64_t>(p) * (P.L.K / 16) + kx / 16;
-          mbar_arrive_expect_tx(&B.x_full[xs], P.T_pass * 32);
-          bulk_g2s(xring + xs * x_stage_bytes, P.xs + slab * (P.T_pass * 32), P.T_pass * 32,
-                   &B.x_full[xs]);
+          const uint32_t kx = I.kt * P.L.tile_k + 16 * s;
+          const uint32_t bar = smem_u32(&B.x_full[xs]);
+          mbar_arrive_expect_tx_s(bar, x_stage_bytes);
+          // X slabs are read by every CTA working at their K columns: kept in L2
+          const uint64_t pol = l2_evict_last();
+          for (uint32_t j = 0; j < P.NT; ++j)
+            tma_load_2d_hint_s(xring_s + xs * x_stage_bytes + j * P.T * 32, &P.tmap_x,
+                               static_cast<int32_t>(kx), static_cast<int32_t>(I.p * P.T_pass + j * P.T),
+                               bar, pol);
           n_issued = xc + 1;
         }
-        xi += clock64() - c0;
         ++xc;
       });
-      if (P.trace) {
-        P.trace[blockIdx.x * 64 + 53] = xw;
-        P.trace[blockIdx.x * 64 + 54] = xi;
-        P.trace[blockIdx.x * 64 + 55] = clock64() - xb;
-        P.trace[blockIdx.x * 64 + 56] = xc;
-      }
       trace_mark(P, 42);
       // drain: the last load issued into every stage must have landed
-      const uint32_t first = n_issued > XS ? n_issued - XS : 0;
+      const uint32_t first = n_issued > XSu ? n_issued - XSu : 0;
       for (uint32_t q = first; q < n_issued; ++q)
-        wait_drain(&B.x_full[q % XS], (q / XS) & 1u, P.status);
+        wait_drain(&B.x_full[q % XSu], (q / XSu) & 1u, P.status);
       trace_mark(P, 35);
     }
     __syncwarp();
@@ -457,6 +639,8 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     for (uint32_t seg = seg_first; seg <= seg_last; ++seg) {
       const uint32_t lseg = static_cast<uint32_t>(seg - seg_first);
       const uint32_t buf = lseg % P.n_bufs;
+      // after an abort the accumulator holds no valid sum, but the epilogue
+      // still takes part in split-K so that the counters return to zero
       wait_live(&B.acc_full[buf], (lseg / P.n_bufs) & 1u, abort, P.status, 6, 256);
       tc_fence_after();
       if (e == 0 && lseg < 2) trace_mark(P, 36 + lseg);
@@ -466,19 +650,67 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
       const bool complete = u_begin <= s_lo && u_end >= s_hi;
       const uint32_t slot = (seg == seg_first) ? 0u : 1u;
       float* part = P.partials + (static_cast<uint64_t>(blockIdx.x) * 2 + slot) * P.H * P.T_pass * 128;
+      // banks that hold a part of the segment: unit u went to bank
+      // (u - u_begin) % banks, so the segment's first units in this CTA name them
+      const uint32_t NB = P.n_banks;
+      uint32_t bmask = 0;
+      {
+        const uint32_t a = max(u_begin, s_lo), b = min(u_end, s_hi);
+        for (uint32_t u = a; u < b && u < a + NB; ++u) bmask |= 1u << ((u - u_begin) % NB);
+      }
       for (uint32_t h = 0; h < P.H; ++h) {
         const uint32_t n = rb * P.L.tile_n + h * 128 + e;
         const float scale = complete ? row_scale(P, n) : 1.0f;
         for (uint32_t j = 0; j < P.NT; ++j) {
-          const uint32_t col0 = ((buf * P.H + h) * P.NT + j) * P.T;
-          for (uint32_t cc = 0; cc < P.T; cc += 16) {
-            uint32_t v[16];
-            tmem_ld16(tmem_base + ((32 * warp) << 16) + col0 + cc, v);
-            tmem_ld_wait();
-            float f[16];
+          // tokens past M are padding: stop at the last 16-column chunk holding one
+          const uint32_t m0 = p * P.T_pass + j * P.T;
+          const uint32_t t_end = P.M > m0 ? min(P.T, P.M - m0) : 0u;
+          auto col_of = [&](uint32_t bank) {
+            return tmem_base + ((32 * warp) << 16) + (((buf * NB + bank) * P.H + h) * P.NT + j) * P.T;
+          };
+          if (NB == 1) {
+            for (uint32_t cc = 0; cc < t_end; cc += 32) {
+              uint32_t v[2][16];
+              tmem_ld16(col_of(0) + cc, v[0]);
+              if (cc + 16 < t_end) tmem_ld16(col_of(0) + cc + 16, v[1]);
+              tmem_ld_wait();
 #pragma unroll
-            for (int q = 0; q < 16; ++q) f[q] = __uint_as_float(v[q]);
-            epi_emit16(P, f, complete, scale, part, p, h, j * P.T + cc, n, e);
+              for (uint32_t k = 0; k < 2; ++k) {
+                if (cc + 16 * k >= t_end) break;
+                float f[16];
+#pragma unroll
+                for (int q = 0; q < 16; ++q) f[q] = __uint_as_float(v[k][q]);
+                epi_emit16(P, f, complete, scale, part, p, h, j * P.T + cc + 16 * k, n, e);
+              }
+            }
+          } else {
+            // the banks' sums, added in bank order, eight columns at a time:
+            // the first bank loads into the sum, one more rides along with
+            // it, further ones one by one
+            for (uint32_t cc = 0; cc < t_end; cc += 8) {
+              uint32_t a[8], v[8];
+              uint32_t m = bmask;
+              tmem_ld8(col_of(__ffs(m) - 1) + cc, a);
+              m &= m - 1;
+              const bool two = m != 0;
+              if (two) {
+                tmem_ld8(col_of(__ffs(m) - 1) + cc, v);
+                m &= m - 1;
+              }
+              tmem_ld_wait();
+              float f[8];
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                f[q] = two ? __uint_as_float(a[q]) + __uint_as_float(v[q]) : __uint_as_float(a[q]);
+              while (m) {
+                tmem_ld8(col_of(__ffs(m) - 1) + cc, v);
+                m &= m - 1;
+                tmem_ld_wait();
+#pragma unroll
+                for (int q = 0; q < 8; ++q) f[q] += __uint_as_float(v[q]);
+              }
+              epi_emit<8>(P, f, complete, scale, part, p, h, j * P.T + cc, n, e);
+            }
           }
         }
       }
@@ -508,47 +740,30 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
   }
   // the split-K reductions this CTA arrived last for, on every thread
   if (reduce_flag) {
+    if (threadIdx.x == 0) trace_mark(P, 49);
     fence_acq_rel_gpu();  // acquire: the counter showed every contributor arrived
     for (uint32_t k = 0; k < red_n; ++k)
       if ((reduce_flag >> k) & 1u) splitk_reduce(P, G, red_seg[k], threadIdx.x, blockDim.x);
   }
 }
 
-// Stages X for the fused kernel: for every token pass p and 16-column slab
-// ks, a contiguous block of T_pass rows x 32 bytes holding X[p*T_pass + r]
-// [16 ks .. 16 ks + 15] (zero for rows >= M), its two 16-byte chunks placed
-// with the 32-byte swizzle the MMA descriptor expects (chunk c of row r at
-// c ^ ((r >> 2) & 1)); optionally converted to f16.  One thread per chunk.
-__global__ void x_stage_kernel(const uint16_t* __restrict__ X, uint8_t* __restrict__ xs,
-                               uint32_t M, uint32_t K, uint32_t T_pass, uint32_t n_pass,
-                               uint32_t to_f16) {
+// f16 copy of X for the formats whose MMA runs in f16 (X row-major M x K,
+// bf16 bits in, f16 out; 8 elements per thread step).
+__global__ void x_to_f16_kernel(const uint16_t* __restrict__ X, uint16_t* __restrict__ X16,
+                                uint64_t n8) {
   griddep_wait();
   griddep_launch_dependents();
-  const uint64_t n_chunks = static_cast<uint64_t>(n_pass) * (K / 16) * T_pass * 2;
-  for (uint64_t i = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_chunks;
+  for (uint64_t i = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
        i += static_cast<uint64_t>(gridDim.x) * blockDim.x) {
-    const uint32_t c = static_cast<uint32_t>(i & 1);
-    const uint64_t rest = i >> 1;
-    const uint32_t r = static_cast<uint32_t>(rest % T_pass);
-    const uint64_t slab = rest / T_pass;  // p * (K / 16) + ks
-    const uint32_t ks = static_cast<uint32_t>(slab % (K / 16));
-    const uint32_t p = static_cast<uint32_t>(slab / (K / 16));
-    const uint32_t m = p * T_pass + r;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (m < M) {
-      v = __ldg(reinterpret_cast<const uint4*>(X + static_cast<uint64_t>(m) * K + 16 * ks + 8 * c));
-      if (to_f16) {
-        uint32_t in[4] = {v.x, v.y, v.z, v.w}, out[4];
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(X) + i);
+    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+    uint32_t out[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          __half2 h = __floats2half2_rn(__uint_as_float(in[k] << 16), __uint_as_float(in[k] & 0xFFFF0000u));
-          out[k] = *reinterpret_cast<uint32_t*>(&h);
-        }
-        v = make_uint4(out[0], out[1], out[2], out[3]);
-      }
+    for (int k = 0; k < 4; ++k) {
+      __half2 hv = __floats2half2_rn(__uint_as_float(in[k] << 16), __uint_as_float(in[k] & 0xFFFF0000u));
+      out[k] = *reinterpret_cast<uint32_t*>(&hv);
     }
-    const uint64_t dst = slab * (static_cast<uint64_t>(T_pass) * 32) + r * 32 + ((c ^ ((r >> 2) & 1u)) << 4);
-    *reinterpret_cast<uint4*>(xs + dst) = v;
+    reinterpret_cast<uint4*>(X16)[i] = make_uint4(out[0], out[1], out[2], out[3]);
   }
 }
 
@@ -559,6 +774,17 @@ static uint32_t round_up(uint32_t a, uint32_t b) { return (a + b - 1) / b * b; }
 static unsigned long long* g_trace = nullptr;
 void set_trace_buffer(void* d_buf, size_t bytes) {
   g_trace = bytes >= 64 * sizeof(unsigned long long) ? static_cast<unsigned long long*>(d_buf) : nullptr;
+}
+
+cudaError_t set_live_wait_budget_gemm(long long cycles) {
+  return cudaMemcpyToSymbol(g_live_wait_budget, &cycles, sizeof(cycles));
+}
+
+static std::atomic<uint32_t> g_cap_ctas{0}, g_cap_producers{0}, g_force_shared{0};
+void set_plan_limits(uint32_t max_ctas, uint32_t max_producers, uint32_t force_shared) {
+  g_cap_ctas.store(max_ctas, std::memory_order_relaxed);
+  g_cap_producers.store(max_producers, std::memory_order_relaxed);
+  g_force_shared.store(force_shared ? 1u : 0u, std::memory_order_relaxed);
 }
 
 // Accumulator slots the local schedule needs in the busiest CTA: one per
@@ -601,23 +827,15 @@ bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool dec
   p.C = L.tile_k / 16;
   const uint32_t Mp = round_up(M < 1 ? 1 : M, 16);
   uint64_t sms = num_sms > 0 ? static_cast<uint64_t>(num_sms) : 148;
-  // Tuning / testing knobs: cap the CTA count and the producer warps per CTA,
-  // force one of the two schedules.
-  if (const char* v = std::getenv("ANS_GEMM_MAX_CTAS")) {
-    long cap = std::strtol(v, nullptr, 10);
-    if (cap > 0 && static_cast<uint64_t>(cap) < sms) sms = static_cast<uint64_t>(cap);
-  }
-  uint32_t D_cap = kMaxProducers;
-  if (const char* v = std::getenv("ANS_GEMM_MAX_PRODUCERS")) {
-    long cap = std::strtol(v, nullptr, 10);
-    if (cap > 0 && static_cast<uint32_t>(cap) < D_cap) D_cap = static_cast<uint32_t>(cap);
-  }
+  // test limits (set_plan_limits): cap the CTA count and the producer warps
+  // per CTA, force the shared-accumulator schedule
+  const uint32_t cap_ctas = g_cap_ctas.load(std::memory_order_relaxed);
+  if (cap_ctas > 0 && cap_ctas < sms) sms = cap_ctas;
+  const uint32_t cap_prod = g_cap_producers.load(std::memory_order_relaxed);
   // unit indices are 32-bit in the kernels
   if (static_cast<uint64_t>(L.n_tiles) * ((M + 15) / 16) >= (1ull << 31)) return false;
   bool want_local = p.H * Mp <= 32;
-  if (const char* v = std::getenv("ANS_GEMM_SCHEDULE")) {
-    if (std::strcmp(v, "central") == 0) want_local = false;
-  }
+  if (g_force_shared.load(std::memory_order_relaxed)) want_local = false;
   const uint32_t lut_bytes = kSlots * 4;
 
   if (want_local) {
@@ -630,7 +848,7 @@ bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool dec
     p.n_segments = L.N / L.tile_n;
     p.grid = static_cast<uint32_t>(p.n_units < sms ? p.n_units : sms);
     const uint64_t per_cta = (p.n_units + p.grid - 1) / p.grid;
-    uint32_t D = D_cap < kLocalProducersMax ? D_cap : kLocalProducersMax;
+    uint32_t D = (cap_prod > 0 && cap_prod < kLocalProducersMax) ? cap_prod : kLocalProducersMax;
     if (D > per_cta) D = static_cast<uint32_t>(per_cta);
     for (; D >= 1; --D) {
       const uint32_t slots = local_slots(static_cast<uint32_t>(p.n_units), p.grid, D, L.n_kt);
@@ -671,7 +889,7 @@ bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool dec
     // no fit: fall through to the shared-accumulator schedule
   }
 
-  // ---- shared-accumulator schedule: one MMA-issuing thread per CTA
+  // ---- shared-accumulator schedule: one MMA-issuing warp per CTA
   const uint32_t max_cols = 512;
   if (2 * p.H * Mp <= max_cols) {
     p.n_bufs = 2;
@@ -688,7 +906,14 @@ bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool dec
   p.T_pass = p.T * p.NT;
   p.n_pass = (M + p.T_pass - 1) / p.T_pass;
   if (p.n_pass == 0) p.n_pass = 1;
-  uint32_t cols = p.n_bufs * p.H * p.T_pass;
+  // Accumulator banks: where TMEM has room the units of a CTA are spread
+  // over 2 or 4 banks (unit u into bank (u - u_begin) % banks), summed in
+  // bank order by the epilogue, so that consecutive MMAs write different
+  // accumulators.
+  p.n_banks = 1;
+  for (uint32_t nb = 4; nb >= 2; nb /= 2)
+    if (nb * p.n_bufs * p.H * p.T_pass <= max_cols) { p.n_banks = nb; break; }
+  uint32_t cols = p.n_banks * p.n_bufs * p.H * p.T_pass;
   p.tmem_cols = 32;
   while (p.tmem_cols < cols) p.tmem_cols <<= 1;
   if (p.tmem_cols > 512) return false;
@@ -698,52 +923,98 @@ bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool dec
   p.grid = static_cast<uint32_t>(p.n_units < sms ? p.n_units : sms);
   uint64_t per_cta = (p.n_units + p.grid - 1) / p.grid;
 
-  // shared memory: [lut][w rings][chunk rings][x stages][barriers]
+  // Producers against X stages.  Every MMA step waits for its X slab, loaded
+  // by TMA from L2 a microsecond or more before; the decode variant consumes
+  // a slab about every 1,000 cycles (one per producer every ~13,000), so a
+  // few stages cover that latency: at least 3, and 32 KB of stages when they
+  // are small.  The producer count is the largest that leaves them room.
+  // Shared memory, decode variant: [slot table][W slots][chunk rings][X stages][barriers].
   const uint32_t x_stage = p.T_pass * 32;
-  uint32_t D = D_cap;
-  if (D > L.n_kt) D = L.n_kt;
+  const uint32_t xs_min = std::max(3u, std::min(8u, 32768u / x_stage));
+  uint32_t D = (cap_prod > 0 && cap_prod < kMaxProducers) ? cap_prod : kMaxProducers;
+  if (D > L.n_kt) D = L.n_kt;  // a round spans at most two W row-block segments
   if (D > per_cta) D = static_cast<uint32_t>(per_cta);
-  // X stages take whatever shared memory the producers leave (deep rings keep
-  // every X slab of a round in flight at small M), at least 2, at most 64.
-  uint32_t XS = 0;
-  for (;;) {
-    uint32_t off = lut_bytes;
-    off = round_up(off, 2048);
-    const uint32_t off_w = off;
-    off += D * 2 * kSlabBytes;
+  const uint32_t lut_bytes_c = lut_bytes;
+  auto layout = [&](uint32_t Dn, bool with_lut, bool with_rings, uint32_t* off_w, uint32_t* off_chunk,
+                    uint32_t* off_x) {
+    uint32_t off = with_lut ? round_up(lut_bytes_c, 2048) : 0;
+    *off_w = off;
+    off += Dn * 2 * kSlabBytes;
     off = round_up(off, 128);
-    const uint32_t off_chunk = off;
-    off += D * kRingStride + 128;
+    *off_chunk = off;
+    if (with_rings) off += Dn * kRingStride + 128;
     off = round_up(off, 1024);
-    const uint32_t off_x = off;
+    *off_x = off;
+    return off;
+  };
+  for (;; --D) {
+    if (D == 0) return false;
+    uint32_t ow, oc, ox;
+    const uint32_t off = layout(D, true, true, &ow, &oc, &ox);
     const uint32_t bars_max = num_bars(D, 64) * 8;
     const uint32_t room = kSmemLimit > off + bars_max ? kSmemLimit - off - bars_max : 0;
-    XS = room / x_stage;
-    if (XS > 64) XS = 64;
-    if (XS >= 2) {
-      off += XS * x_stage;
-      off = round_up(off, 8);
-      p.off_lut = 0;
-      p.off_w = off_w;
-      p.off_chunk = off_chunk;
-      p.off_x = off_x;
-      p.off_bars = off;
-      off += num_bars(D, XS) * 8;
-      p.smem_bytes = off;
-      break;
-    }
-    if (D > 1) { --D; continue; }
-    return false;
+    if (room / x_stage >= xs_min) break;
   }
   p.D = D;
-  p.x_stages = XS;
+  // the layout of the variant asked for: the decode variant as above; the copy
+  // variant has no slot table and (except for 1-byte codes, staged by TMA in
+  // the chunk area) no chunk rings, so its X ring is deeper -- it consumes a
+  // slab per MMA, not per decode
+  const uint32_t cmode = copy_mode_of(p.fmt);
+  const bool rings = decode || cmode == kCopyTmaRaw;
+  {
+    uint32_t ow, oc, ox;
+    uint32_t off = layout(D, decode, rings, &ow, &oc, &ox);
+    const uint32_t bars_max = num_bars(D, 64) * 8;
+    const uint32_t room = kSmemLimit > off + bars_max ? kSmemLimit - off - bars_max : 0;
+    uint32_t XS = room / x_stage;
+    if (XS > 64) XS = 64;
+    if (XS < 2) return false;
+    off += XS * x_stage;
+    off = round_up(off, 8);
+    p.off_lut = 0;
+    p.off_w = ow;
+    p.off_chunk = oc;
+    p.off_x = ox;
+    p.off_bars = off;
+    off += num_bars(D, XS) * 8;
+    p.smem_bytes = off;
+    p.x_stages = XS;
+  }
   p.ws_partials_bytes = static_cast<size_t>(p.grid) * 2 * p.H * p.T_pass * 128 * sizeof(float);
   p.ws_counters_bytes = round_up(p.n_segments * 4, 256);
-  p.ws_x16_bytes = static_cast<size_t>(p.n_pass) * p.T_pass * L.K * 2;  // staged X slabs
+  p.ws_x16_bytes = p.ab_f16 ? static_cast<size_t>(M) * L.K * 2 : 0;  // f16 copy of X
   p.ws_bytes = p.ws_counters_bytes + (p.ws_partials_bytes + 255) / 256 * 256 +
                (p.ws_x16_bytes + 255) / 256 * 256;
   *plan = p;
   return true;
+}
+
+// ---- tensor maps (2-D, tiled, no multicast), encoded through the driver
+// entry point the runtime hands out (no link-time dependence on libcuda)
+static cudaError_t encode_tmap(CUtensorMap* map, CUtensorMapDataType type, const void* base,
+                               uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_inner,
+                               uint32_t box_outer, CUtensorMapSwizzle swizzle) {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  static cudaError_t lookup = cudaSuccess;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    lookup = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q);
+    if (lookup == cudaSuccess && (q != cudaDriverEntryPointSuccess || f == nullptr))
+      lookup = cudaErrorSymbolNotFound;
+    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  if (lookup != cudaSuccess) return lookup;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, type, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 template <bool kDecode, uint32_t kFmt, bool kWide = false>
@@ -792,6 +1063,7 @@ static GemmDev make_gemm_dev(const GemmPlan& plan, const LayerDev& L, const void
   P.C = plan.C;
   P.D = plan.D;
   P.n_bufs = plan.n_bufs;
+  P.n_banks = plan.n_banks ? plan.n_banks : 1;
   P.x_stages = plan.x_stages;
   P.tmem_cols = plan.tmem_cols;
   P.n_rb = L.N / L.tile_n;
@@ -816,16 +1088,33 @@ cudaError_t launch_gemm(const GemmPlan& plan, const LayerDev& L, bool decode, co
                         uint32_t group_k, float* Y, void* ws, uint32_t* status,
                         cudaStream_t stream) {
   if (plan.M == 0) return cudaSuccess;
-  const GemmDev P = make_gemm_dev(plan, L, w_plain, X, scales, scale_kind, group_k, Y, ws, status);
+  GemmDev P = make_gemm_dev(plan, L, w_plain, X, scales, scale_kind, group_k, Y, ws, status);
   if (!plan.local) {
-    const uint64_t n_chunks = static_cast<uint64_t>(plan.n_pass) * (L.K / 16) * plan.T_pass * 2;
-    uint32_t blocks = static_cast<uint32_t>((n_chunks + 255) / 256);
-    if (blocks > 4096) blocks = 4096;
-    if (blocks == 0) blocks = 1;
-    cudaError_t e = launch_pdl(x_stage_kernel, dim3(blocks), dim3(256), 0, stream, X,
-                               const_cast<uint8_t*>(P.xs), plan.M, L.K, plan.T_pass,
-                               plan.n_pass, plan.ab_f16);
+    // X for the MMA as a tensor map: the caller's bf16 X, or its f16 copy
+    const void* xsrc = X;
+    if (plan.ab_f16) {
+      const uint64_t n8 = static_cast<uint64_t>(plan.M) * L.K / 8;
+      uint32_t blocks = static_cast<uint32_t>((n8 + 255) / 256);
+      if (blocks > 4096) blocks = 4096;
+      if (blocks == 0) blocks = 1;
+      cudaError_t e = launch_pdl(x_to_f16_kernel, dim3(blocks), dim3(256), 0, stream, X,
+                                 reinterpret_cast<uint16_t*>(const_cast<uint8_t*>(P.xs)), n8);
+      if (e != cudaSuccess) return e;
+      xsrc = P.xs;
+    }
+    cudaError_t e = encode_tmap(&P.tmap_x, CU_TENSOR_MAP_DATA_TYPE_UINT16, xsrc, L.K, plan.M,
+                                static_cast<uint64_t>(L.K) * 2, 16, plan.T, CU_TENSOR_MAP_SWIZZLE_32B);
     if (e != cudaSuccess) return e;
+    if (!decode) {
+      const uint32_t cm = copy_mode_of(plan.fmt);
+      if (cm == kCopyTmaSlab)
+        e = encode_tmap(&P.tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT16, w_plain, L.K, L.N,
+                        static_cast<uint64_t>(L.K) * 2, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B);
+      else if (cm == kCopyTmaRaw)
+        e = encode_tmap(&P.tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_plain, L.K, L.N, L.K, 16, 128,
+                        CU_TENSOR_MAP_SWIZZLE_NONE);
+      if (e != cudaSuccess) return e;
+    }
   }
   if (plan.local) return launch_gemm_local(plan, P, decode, stream);
 
@@ -867,23 +1156,28 @@ cudaError_t launch_gemm(const GemmPlan& plan, const LayerDev& L, bool decode, co
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_gemm_batched(const GemmPlan& plan, uint32_t n, const LayerDev* const* Ls,
+cudaError_t launch_gemm_batched(const GemmPlan* plans, uint32_t n, const LayerDev* const* Ls,
                                 const uint16_t* const* Xs, const void* const* scales,
                                 uint32_t scale_kind, uint32_t group_k, float* const* Ys, void* ws,
-                                uint32_t* status, cudaStream_t stream) {
-  if (plan.M == 0 || n == 0) return cudaSuccess;
-  if (!plan.local || n > kMaxBatch) return cudaErrorInvalidValue;
+                                const size_t* ws_off, uint32_t* status, cudaStream_t stream) {
+  if (n == 0 || plans[0].M == 0) return cudaSuccess;
+  if (n > kMaxBatch) return cudaErrorInvalidValue;
   static_assert(sizeof(BatchDev) <= 32000, "kernel parameter limit");
   BatchDev B;
   std::memset(&B, 0, sizeof(B));
   B.n_jobs = n;
-  const size_t ws_job = ((plan.ws_bytes + 255) / 256) * 256;
+  GemmPlan shape = plans[0];  // the launch: the largest producer count and shared memory
+  uint32_t cta = 0;
   for (uint32_t j = 0; j < n; ++j) {
-    B.job[j] = make_gemm_dev(plan, *Ls[j], nullptr, Xs[j], scales[j], scale_kind, group_k, Ys[j],
-                             static_cast<uint8_t*>(ws) + j * ws_job, status);
-    B.job[j].cta0 = j * plan.grid;
+    if (!plans[j].local || plans[j].fmt != plans[0].fmt) return cudaErrorInvalidValue;
+    B.job[j] = make_gemm_dev(plans[j], *Ls[j], nullptr, Xs[j], scales[j], scale_kind, group_k,
+                             Ys[j], static_cast<uint8_t*>(ws) + ws_off[j], status);
+    B.job[j].cta0 = cta;
+    cta += plans[j].grid;
+    shape.D = std::max(shape.D, plans[j].D);
+    shape.smem_bytes = std::max(shape.smem_bytes, plans[j].smem_bytes);
   }
-  return launch_gemm_local_batch(plan, B, n * plan.grid, stream);
+  return launch_gemm_local_batch(shape, B, cta, stream);
 }
 
 }  // namespace ansdev

@@ -55,29 +55,35 @@ __device__ __forceinline__ float row_scale(const GemmDev& P, uint32_t n) {
   return 1.0f;
 }
 
-// Epilogue output of 16 accumulator columns (tokens tok0 .. tok0 + 15 of
+// Epilogue output of NV accumulator columns (tokens tok0 .. tok0 + NV - 1 of
 // token pass p) for W row n = rb * tile_n + h * 128 + e.  A segment that this
 // CTA holds completely goes to Y (scaled); otherwise the values go to this
 // CTA's partial-sum slot for the split-K reduction.
-__device__ __forceinline__ void epi_emit16(const GemmDev& P, const float (&v)[16], bool complete,
-                                           float scale, float* part, uint32_t p, uint32_t h,
-                                           uint32_t tok0, uint32_t n, uint32_t e) {
+template <uint32_t NV>
+__device__ __forceinline__ void epi_emit(const GemmDev& P, const float (&v)[NV], bool complete,
+                                         float scale, float* part, uint32_t p, uint32_t h,
+                                         uint32_t tok0, uint32_t n, uint32_t e) {
   // tokens past M are padding: neither stored nor reduced
   const uint32_t m0 = p * P.T_pass + tok0;
-  const uint32_t nv = P.M > m0 ? min(16u, P.M - m0) : 0u;
+  const uint32_t nv = P.M > m0 ? min(NV, P.M - m0) : 0u;
   if (complete) {
     float* y = P.Y + static_cast<uint64_t>(m0) * P.L.N + n;
 #pragma unroll
-    for (uint32_t q = 0; q < 16; ++q) {
+    for (uint32_t q = 0; q < NV; ++q) {
       if (q < nv) *y = v[q] * scale;
       y += P.L.N;
     }
   } else {
     float* d = part + (static_cast<uint64_t>(h) * P.T_pass + tok0) * 128 + e;
 #pragma unroll
-    for (uint32_t q = 0; q < 16; ++q)
+    for (uint32_t q = 0; q < NV; ++q)
       if (q < nv) d[q * 128] = v[q];
   }
+}
+__device__ __forceinline__ void epi_emit16(const GemmDev& P, const float (&v)[16], bool complete,
+                                           float scale, float* part, uint32_t p, uint32_t h,
+                                           uint32_t tok0, uint32_t n, uint32_t e) {
+  epi_emit<16>(P, v, complete, scale, part, p, h, tok0, n, e);
 }
 
 // Split-K over CTAs.  A W row block's segment seg (token pass p, row block

@@ -137,9 +137,13 @@ __device__ __forceinline__ void local_cta(const GemmDev& P) {
   // memory, after the previous grid in the stream has completed
   griddep_wait();
   griddep_launch_dependents();
+  check_smem_base(smem, P.status);
   if (threadIdx.x == 0) trace_mark(P, 0);
 
-  if (warp >= kLocalFixedWarps) {
+  if (warp >= kLocalFixedWarps + D) {
+    // a batched launch is shaped for its job with the most producer warps;
+    // the warps beyond this job's producers have no work
+  } else if (warp >= kLocalFixedWarps) {
     // ============================ producer warps ============================
     const uint32_t d = warp - kLocalFixedWarps;
     uint32_t pb, pe;
@@ -442,7 +446,7 @@ __device__ __forceinline__ void local_cta(const GemmDev& P) {
       const uint32_t rmask = __ballot_sync(0xFFFFFFFFu, ready);
       if (rmask == 0) {
         if (*abort) break;
-        if (clock64() - idle_since > kWaitBudgetCycles) {
+        if (clock64() - idle_since > g_live_wait_budget) {
           if (lane == 0) {
             *abort = 1u;
             atomicOr(P.status, kStatusTimeout | (1u << (8 + 2)));
@@ -741,6 +745,10 @@ cudaError_t launch_gemm_local_batch(const GemmPlan& plan, const BatchDev& B, uin
                   : launch_local_batch_variant<kFmtFp4PairBf16, false>(plan, B, grid, stream);
   }
   return cudaErrorInvalidValue;
+}
+
+cudaError_t set_live_wait_budget_local(long long cycles) {
+  return cudaMemcpyToSymbol(g_live_wait_budget, &cycles, sizeof(cycles));
 }
 
 }  // namespace ansdev

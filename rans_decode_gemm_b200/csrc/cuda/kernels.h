@@ -1,6 +1,7 @@
 // kernels.h -- plain structs and launch entry points shared between the C-ABI
 // layer (host C++) and the CUDA kernels.  No device code here.
 #pragma once
+#include <cuda.h>  // CUtensorMap (the type only: maps are encoded through the runtime's driver entry point)
 #include <cuda_runtime.h>
 
 #include <cstddef>
@@ -9,6 +10,9 @@
 namespace ansdev {
 
 constexpr uint32_t kNoSymbolHost = 0xFFFFFFFFu;
+// Default budget of the kernels' bounded waits (about 1.5 s at 1.9 GHz; the
+// device side's kWaitBudgetCycles).
+constexpr long long kWaitBudgetCyclesHost = 3000000000LL;
 
 // A compressed layer as the kernels see it (passed by value as a kernel
 // parameter; the codebook travels with it).
@@ -52,7 +56,9 @@ struct GemmPlan {
   uint32_t H, C;       // 128-row halves per tile, 16-column slabs per tile
   uint32_t D;          // producer warps per CTA
   uint32_t n_bufs;     // TMEM accumulator sets (1 or 2)
-  uint32_t x_stages;
+  uint32_t n_banks;    // shared-accumulator schedule: accumulator banks per set (1, 2 or 4)
+  uint32_t x_stages;    // X stages of the shared-accumulator schedule (differs between the
+                        // decode and copy variants; the accumulation order does not depend on it)
   uint32_t tmem_cols;
   uint32_t local;      // 1: every producer warp issues its own MMAs (gemm_local.cu)
   uint32_t n_slots;    // local schedule: TMEM accumulators per CTA (max over CTAs)
@@ -63,6 +69,18 @@ struct GemmPlan {
   uint32_t off_lut, off_w, off_chunk, off_x, off_bars;
   size_t ws_partials_bytes, ws_counters_bytes, ws_x16_bytes, ws_bytes;
 };
+
+// How the producers of the shared-accumulator schedule fill W slabs from
+// uncompressed weights (ans_gemm_uncompressed).
+enum : uint32_t {
+  kCopyLoads = 0,    // per-lane global loads, formatted in registers (packed nibbles)
+  kCopyTmaSlab = 1,  // bf16: one TMA box per slab, straight into the slot (32-byte swizzle)
+  kCopyTmaRaw = 2    // 1-byte codes: TMA box of the raw bytes, formatted shared -> shared
+};
+__host__ __device__ constexpr uint32_t copy_mode_of(uint32_t fmt) {
+  return fmt == kFmtBf16Split ? kCopyTmaSlab
+         : (fmt == kFmtFp8F16 || fmt == kFmtInt8F16) ? kCopyTmaRaw : kCopyLoads;
+}
 
 struct GemmDev {
   LayerDev L;
@@ -75,22 +93,30 @@ struct GemmDev {
   uint32_t scale_kind, group_k, n_groups_k;
   uint32_t M, T, NT, T_pass, n_pass;
   uint32_t H, C, D, n_bufs, x_stages, tmem_cols;
+  uint32_t n_banks;
   uint32_t n_rb;
   uint64_t n_units;
   uint32_t idesc;
   uint32_t off_lut, off_w, off_chunk, off_x, off_bars;
   unsigned long long* trace;  // optional per-CTA event timestamps (internal profiling)
-  const uint8_t* xs;          // X staged as pre-swizzled 16-column slabs (workspace)
+  const uint8_t* xs;          // f16 copy of X (M x K row-major, workspace) for the f16 formats
   const uint16_t* X;          // local schedule: X as given (bf16, M x K row-major)
   uint32_t x_f16;             // local schedule: convert X to f16 for the MMA
   uint32_t n_slots;           // local schedule: accumulator slots (barriers) per CTA
   uint32_t n_cta;             // CTAs that share this layer's units (the grid, or a batch job's share)
   uint32_t cta0;              // first CTA of this layer in the grid (0 unless batched)
+  // shared-accumulator schedule: X (or its f16 copy) as a 2-D tensor map,
+  // box 16 columns x T rows, 32-byte swizzle; copy variant: W as a 2-D
+  // tensor map (bf16: box 16 x 128, 32-byte swizzle; 1-byte codes: box
+  // 16 bytes x 128 rows, no swizzle)
+  CUtensorMap tmap_x;
+  CUtensorMap tmap_w;
 };
 
-// Several layers of one shape in one launch of the local schedule: job j
-// owns CTAs [job[j].cta0, job[j].cta0 + job[j].n_cta).  Passed by value as
-// the kernel parameter (well under the 32 KB parameter limit).
+// Several layers in one launch of the local schedule (shapes may differ; one
+// operand format): job j owns CTAs [job[j].cta0, job[j].cta0 + job[j].n_cta)
+// and runs with its own plan's producers, slots and shared-memory layout.
+// Passed by value as the kernel parameter (under the 32 KB parameter limit).
 constexpr uint32_t kMaxBatch = 8;
 struct BatchDev {
   uint32_t n_jobs;
@@ -100,6 +126,22 @@ struct BatchDev {
 // Internal profiling hook: when set, every fused-GEMM CTA writes globaltimer
 // stamps of its phases to trace[cta * 64 + slot].
 void set_trace_buffer(void* d_buf, size_t bytes);
+
+// Internal test hook: caps on the CTAs and producer warps a fused-GEMM plan
+// may use, and a switch that sends every token count to the shared-
+// accumulator schedule (0 = no cap, default schedule).  Process-wide; the
+// tests use it to force many rounds, long producer runs and both schedules
+// on small shapes.
+void set_plan_limits(uint32_t max_ctas, uint32_t max_producers, uint32_t force_shared);
+
+// Internal test hooks: the budget (clock64 cycles) of the waits that the
+// pipeline's progress ends, per translation unit, on the current device
+// (kWaitBudgetCycles by default); and a kernel that makes one such wait on a
+// barrier nothing arrives on (status gets the TIMEOUT bit).
+cudaError_t set_live_wait_budget_gemm(long long cycles);
+cudaError_t set_live_wait_budget_local(long long cycles);
+cudaError_t set_live_wait_budget_decode(long long cycles);
+cudaError_t launch_wait_probe(uint32_t* status, cudaStream_t stream);
 
 // Scratch capacity of the allocation-free entry point (16 MiB per device).
 constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
@@ -132,12 +174,13 @@ cudaError_t launch_gemm(const GemmPlan& plan, const LayerDev& L, bool decode, co
                         const uint16_t* X, const void* scales, uint32_t scale_kind,
                         uint32_t group_k, float* Y, void* ws, uint32_t* status,
                         cudaStream_t stream);
-// n layers of one shape (plan made for one of them with a CTA cap of grid / n;
-// plan.local), each with its own X, scales and Y, in one launch; ws holds n
-// consecutive workspaces of round_up(plan.ws_bytes, 256) bytes.
-cudaError_t launch_gemm_batched(const GemmPlan& plan, uint32_t n, const LayerDev* const* Ls,
+// n layers in one launch of the small-M schedule: layer j runs plans[j]
+// (every plan local, one operand format) on CTAs [sum of the earlier grids,
+// + plans[j].grid), each with its own X, scales, Y and workspace
+// (ws + ws_off[j], round_up(plans[j].ws_bytes, 256) bytes at least).
+cudaError_t launch_gemm_batched(const GemmPlan* plans, uint32_t n, const LayerDev* const* Ls,
                                 const uint16_t* const* Xs, const void* const* scales,
                                 uint32_t scale_kind, uint32_t group_k, float* const* Ys, void* ws,
-                                uint32_t* status, cudaStream_t stream);
+                                const size_t* ws_off, uint32_t* status, cudaStream_t stream);
 
 }  // namespace ansdev

@@ -119,6 +119,29 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
+// L2 cache policies for the copies: data read once (the weight stream) is
+// evicted first, data read by many CTAs (X) last.
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t l2_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// 1-D bulk copy global -> this CTA's shared memory with an L2 cache policy.
+__device__ __forceinline__ void bulk_g2s_hint_s(uint32_t dst_s, const void* src, uint32_t bytes,
+                                                uint32_t bar_s, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1], %2, [%3], %4;" ::"r"(dst_s),
+      "l"(src), "r"(bytes), "r"(bar_s), "l"(policy)
+      : "memory");
+}
+
 // 1-D bulk copy global -> this CTA's shared memory, completing on `bar`.
 // src, dst 16-byte aligned; bytes a multiple of 16.  No multicast.
 __device__ __forceinline__ void bulk_g2s_s(uint32_t dst_s, const void* src, uint32_t bytes,
@@ -134,14 +157,28 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
   bulk_g2s_s(smem_u32(dst), src, bytes, smem_u32(bar));
 }
 
-// 2-D tiled tensor copy global -> shared (no multicast).  x is the innermost
-// coordinate in elements.
-__device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int32_t x, int32_t y,
-                                            uint64_t* bar) {
+// 2-D tiled tensor copy global -> this CTA's shared memory, completing on
+// the barrier at bar_s (no multicast).  tmap: a tensor map in kernel
+// parameter space; x is the innermost coordinate in elements and x * the
+// element size must be a multiple of 16 bytes; dst_s aligned to 128 bytes
+// (256 with the 32-byte swizzle).  Rows past the tensor's extent land as
+// zeros.
+__device__ __forceinline__ void tma_load_2d_s(uint32_t dst_s, const void* tmap, int32_t x,
+                                              int32_t y, uint32_t bar_s) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
-      "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
-      "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(bar))
+      "[%0], [%1, {%2, %3}], [%4];" ::"r"(dst_s),
+      "l"(tmap), "r"(x), "r"(y), "r"(bar_s)
+      : "memory");
+}
+
+// The same with an L2 cache policy.
+__device__ __forceinline__ void tma_load_2d_hint_s(uint32_t dst_s, const void* tmap, int32_t x,
+                                                   int32_t y, uint32_t bar_s, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst_s),
+      "l"(tmap), "r"(x), "r"(y), "r"(bar_s), "l"(policy)
       : "memory");
 }
 
@@ -217,6 +254,14 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
         "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
         "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7])
       : "r"(taddr)
       : "memory");
 }

@@ -48,6 +48,17 @@ constexpr uint32_t kNoSymbol = kNoSymbolHost;
 constexpr uint32_t kStatusCorrupt = 0x1u;
 constexpr uint32_t kStatusTimeout = 0x2u;
 constexpr uint32_t kStatusBadOffsets = 0x4u;
+constexpr uint32_t kStatusSmemAlign = 0x8u;
+
+// The fused kernels lay out W slabs and X stages at 1024-byte multiples of
+// the dynamic shared-memory base and describe them to the tensor cores (and
+// TMA) with 32-byte swizzle, whose pattern is taken from the absolute shared
+// address: the base must be 1024-byte aligned.  Checked once per CTA, after
+// griddepcontrol.wait (it writes global memory); a misaligned base is
+// reported, not trapped on.
+__device__ __forceinline__ void check_smem_base(const void* smem_base, uint32_t* status) {
+  if (threadIdx.x == 0 && (smem_u32(smem_base) & 1023u) != 0) atomicOr(status, kStatusSmemAlign);
+}
 
 enum : uint32_t {
   kDtInt4 = 0,
@@ -59,6 +70,14 @@ enum : uint32_t {
   kDtFp4Pairs = 6
 };
 
+
+// Budget of the waits that the pipeline's own progress ends (wait_live and
+// its variants), in clock64() cycles: kWaitBudgetCycles unless the internal
+// test hook shortened it (one copy per translation unit, set by the
+// set_live_wait_budget_* functions).  Drains of copies already in flight
+// always wait kWaitBudgetCycles: those copies land on their own, and a CTA
+// must not exit while one is still writing its shared memory.
+static __device__ long long g_live_wait_budget = kWaitBudgetCycles;
 
 // Abort-aware bounded wait.  Returns false if the wait ran out (then sets the
 // CTA's abort flag and the TIMEOUT status bit) or if the CTA already aborted.
@@ -72,7 +91,7 @@ __device__ __forceinline__ bool wait_live(uint64_t* bar, uint32_t parity, volati
   long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
     if (*abort) return false;
-    if (clock64() - t0 > kWaitBudgetCycles) {
+    if (clock64() - t0 > g_live_wait_budget) {
       *abort = 1u;
       atomicOr(status, kStatusTimeout | (1u << (8 + site)));
       return false;
@@ -89,7 +108,7 @@ __device__ __forceinline__ bool wait_live_s(uint32_t bar_s, uint32_t parity, vol
   long long t0 = clock64();
   while (!mbar_try_wait_s(bar_s, parity)) {
     if (*abort) return false;
-    if (clock64() - t0 > kWaitBudgetCycles) {
+    if (clock64() - t0 > g_live_wait_budget) {
       *abort = 1u;
       atomicOr(status, kStatusTimeout | (1u << (8 + site)));
       return false;
@@ -116,7 +135,7 @@ __device__ __forceinline__ bool wait_all_live(uint64_t* bars, uint32_t n, uint32
     if (all) return true;
     if (pass == 0) t0 = clock64();
     if (*abort) return false;
-    if (clock64() - t0 > kWaitBudgetCycles) {
+    if (clock64() - t0 > g_live_wait_budget) {
       *abort = 1u;
       atomicOr(status, kStatusTimeout | (1u << (8 + site)));
       return false;
@@ -252,10 +271,13 @@ __device__ __forceinline__ void pipe_issue(ChunkPipe& p, const LayerDev& L, cons
     uint32_t n = min(kChunkBytes, p.it_bytes - off);
     uint32_t slot = p.issued & 3u;
     if (lane == 0) {
+      // the stream is read once per token pass: evicted from L2 first
+      const uint64_t pol = l2_evict_first();
+      const uint32_t bar = smem_u32(&p.bars[slot]);
       const uint32_t nm = slot == 0 ? min(n, kRingMirror) : 0u;  // mirror of slot 0's head
-      mbar_arrive_expect_tx(&p.bars[slot], n + nm);
-      bulk_g2s(p.ring + slot * kChunkBytes, L.stream + p.it_start + off, n, &p.bars[slot]);
-      if (nm) bulk_g2s(p.ring + kRingBytes, L.stream + p.it_start + off, nm, &p.bars[slot]);
+      mbar_arrive_expect_tx_s(bar, n + nm);
+      bulk_g2s_hint_s(smem_u32(p.ring + slot * kChunkBytes), L.stream + p.it_start + off, n, bar, pol);
+      if (nm) bulk_g2s_hint_s(smem_u32(p.ring + kRingBytes), L.stream + p.it_start + off, nm, bar, pol);
     }
     p.it_chunk++;
     p.issued++;
@@ -385,11 +407,13 @@ __device__ __forceinline__ void rp_issue(RunPipe& p, uint32_t lim, uint32_t lane
     const uint32_t n = min(kChunkBytes, p.run_bytes - off);
     const uint32_t slot = p.issued & 3u;
     if (lane == 0) {
+      // the stream is read once per token pass: evicted from L2 first
+      const uint64_t pol = l2_evict_first();
       const uint32_t nm = slot == 0 ? min(n, kRingMirror) : 0u;  // mirror of slot 0's head
       const uint32_t bar = p.bars_s + 8 * slot;
       mbar_arrive_expect_tx_s(bar, n + nm);
-      bulk_g2s_s(p.ring_s + slot * kChunkBytes, p.src + off, n, bar);
-      if (nm) bulk_g2s_s(p.ring_s + kRingBytes, p.src + off, nm, bar);
+      bulk_g2s_hint_s(p.ring_s + slot * kChunkBytes, p.src + off, n, bar, pol);
+      if (nm) bulk_g2s_hint_s(p.ring_s + kRingBytes, p.src + off, nm, bar, pol);
     }
     p.issued++;
   }

@@ -34,3 +34,19 @@ def cuda():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return torch.device("cuda:0")
+
+
+@pytest.fixture
+def plan_limits():
+    """plan_limits(max_ctas=, max_producers=, schedule="local"|"central"):
+    limits on the fused-GEMM launch plans of this test (the library's internal
+    test hook), restored to the defaults afterwards."""
+    from rans_decode_gemm_b200 import ans
+    state = {"max_ctas": 0, "max_producers": 0, "schedule": "local"}
+
+    def set_limits(**kw):
+        state.update(kw)
+        ans._set_plan_limits(state["max_ctas"], state["max_producers"],
+                             state["schedule"] == "central")
+    yield set_limits
+    ans._set_plan_limits(0, 0, False)

@@ -150,7 +150,7 @@ def test_single_symbol_layer(oracle, ans_lib):
 def test_batched_argument_checks(ans_lib):
     # argument and layout errors are reported before any device is touched
     a = ans.make_layout(ans.BF16_SPLIT, 256, 128, 128, 64)
-    b = ans.make_layout(ans.BF16_SPLIT, 128, 128, 128, 64)
+    b = ans.make_layout(ans.FP8_E4M3, 128, 128, 128, 64)   # shapes may differ, dtypes may not
     cb = ans.AnsCodebook()
     ta, tb = ans.AnsTiles(a, cb, None, 0, None, None), ans.AnsTiles(b, cb, None, 0, None, None)
     with pytest.raises(ans.AnsError) as e:
@@ -218,6 +218,7 @@ def test_dtype_constants_agree_with_the_header():
     assert flags["ANS_STATUS_CORRUPT"] == ans.STATUS_CORRUPT
     assert flags["ANS_STATUS_TIMEOUT"] == ans.STATUS_TIMEOUT
     assert flags["ANS_STATUS_BAD_OFFSETS"] == ans.STATUS_BAD_OFFSETS
+    assert flags["ANS_STATUS_SMEM_ALIGN"] == ans.STATUS_SMEM_ALIGN
     assert int(re.search(r"#define\s+ANS_MAX_BATCH\s+(\d+)", text).group(1)) == ans.MAX_BATCH
     # the workload generators use the same dtype numbers
     assert (WL.INT4, WL.BF16_SPLIT, WL.FP8_E4M3, WL.INT4_PAIRS, WL.INT8, WL.FP4_E2M1,

@@ -1,8 +1,8 @@
-"""GPU parity of ans_gemm_batched (several layers of one layout in one call):
-each layer's Y is bit-identical to ans_gemm and to ans_gemm_uncompressed on
-the same layer confined to the same number of SMs (one launch, small M) or
-on the whole GPU (consecutive launches, larger M), and within 1e-3 relative
-Frobenius error of the fp64 oracle."""
+"""GPU parity of ans_gemm_batched (several layers in one call, of one layout or
+of different shapes): each layer's Y is bit-identical to ans_gemm and to
+ans_gemm_uncompressed on the same layer confined to the same number of SMs
+(one launch, small M) or on the whole GPU (consecutive launches, larger M),
+and within 1e-3 relative Frobenius error of the fp64 oracle."""
 import numpy as np
 import pytest
 import torch
@@ -55,6 +55,21 @@ def _sms():
     return torch.cuda.get_device_properties(0).multi_processor_count
 
 
+def _shares(layers, sms):
+    """The SM share of each layer in one launch, as include/ans.h states it:
+    proportional to the weight count, at least one, the largest giving back
+    while the sum is too large, the rest one each to the first layers."""
+    w = [lay.N * lay.K for (_, _, lay, _) in layers]
+    G = [max(1, int(sms * wj / sum(w))) for wj in w]
+    while sum(G) > sms and max(G) > 1:
+        G[G.index(max(G))] -= 1
+    for j in range(len(G)):
+        if sum(G) >= sms:
+            break
+        G[j] += 1
+    return G
+
+
 CASES = [("bf16_4096", 1024, 2048, 64, None), ("int4_70b", 512, 1024, 64, ans.INT4_PAIRS),
          ("int8_8b", 512, 1024, 64, None), ("fp4_8b", 512, 1024, 32, None),
          ("fp4_8b", 512, 1024, 64, ans.FP4_PAIRS),
@@ -65,13 +80,14 @@ CASES = [("bf16_4096", 1024, 2048, 64, None), ("int4_70b", 512, 1024, 64, ans.IN
 @pytest.mark.parametrize("name,N,K,state_bits,dtype", CASES)
 @pytest.mark.parametrize("n", [1, 2, 3, 8])
 @pytest.mark.parametrize("M", [1, 16])
-def test_batched_one_launch_parity(cuda, oracle, monkeypatch, name, N, K, state_bits, dtype, n, M):
+def test_batched_one_launch_parity(cuda, oracle, plan_limits, name, N, K, state_bits, dtype, n, M):
     layers = _layers(name, N, K, n, state_bits, dtype)
     Xs, Ys, st = _run_batched(layers, M)
     assert st == 0
     # the single-layer calls on the same share of the SMs add in the same order
-    monkeypatch.setenv("ANS_GEMM_MAX_CTAS", str(max(1, _sms() // n)))
+    G = _shares(layers, _sms())
     for j, (cfg, d, lay, layer) in enumerate(layers):
+        plan_limits(max_ctas=G[j])
         Y1, st1, _ = run_gemm(cfg, d, lay, layer, Xs[j], compressed=True)
         Yu, stu, _ = run_gemm(cfg, d, lay, layer, Xs[j], compressed=False)
         assert st1 == 0 and stu == 0
@@ -135,3 +151,84 @@ def test_batched_workspace_and_status(cuda):
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     assert all(torch.equal(a, j[3]) for a, j in zip(Y0, jobs))
+
+
+def _layer(name, N, K, tile_n=None, tile_k=None, state_bits=64, dtype=None, seed_off=0, matrix=0):
+    base = WL.CONFIGS[name]
+    cfg = WL.Config(**{**base.__dict__, "seed": base.seed + seed_off})
+    d = WL.make_weights(cfg, matrix, N=N, K=K)
+    lay = ans.make_layout(cfg.dtype if dtype is None else dtype, d["N"], d["K"],
+                          tile_n or cfg.tile_n, tile_k or cfg.tile_k, state_bits)
+    return cfg, d, lay, ans.CompressedLayer.from_weights(d["w"], lay, device="cuda")
+
+
+MIXED = [
+    # an MLP in miniature: gate and up (N x K) with down (K x N)
+    [("llama8b_mlp", 768, 512, None, None), ("llama8b_mlp", 768, 512, None, None),
+     ("llama8b_mlp", 512, 768, None, None)],
+    # different tile widths and shapes of one dtype
+    [("bf16_4096", 1024, 512, 128, 64), ("bf16_4096", 256, 2048, 128, 128),
+     ("bf16_4096", 512, 256, 128, 32)],
+    # 256-row tiles next to 128-row tiles, int4 pair symbols with group scales
+    [("int4_70b", 512, 1024, 256, 64), ("int4_70b", 384, 512, 128, 64)],
+    # very unequal weight counts: the small layer still gets one SM
+    [("fp8_405b", 2048, 2048, None, None), ("fp8_405b", 128, 128, None, None)],
+]
+
+
+@pytest.mark.parametrize("case", range(len(MIXED)))
+@pytest.mark.parametrize("state_bits", [32, 64])
+@pytest.mark.parametrize("M", [1, 16])
+def test_batched_mixed_layouts_one_launch(cuda, oracle, plan_limits, case, state_bits, M):
+    spec = MIXED[case]
+    dtype = ans.INT4_PAIRS if spec[0][0] == "int4_70b" else None
+    layers = [_layer(nm, N, K, tn, tk, state_bits, dtype, seed_off=100 * j)
+              for j, (nm, N, K, tn, tk) in enumerate(spec)]
+    Xs, Ys, st = _run_batched(layers, M)
+    assert st == 0
+    G = _shares(layers, _sms())
+    assert sum(G) <= _sms() and min(G) >= 1
+    for j, (cfg, d, lay, layer) in enumerate(layers):
+        plan_limits(max_ctas=G[j])
+        Y1, st1, _ = run_gemm(cfg, d, lay, layer, Xs[j], compressed=True)
+        Yu, stu, _ = run_gemm(cfg, d, lay, layer, Xs[j], compressed=False)
+        assert st1 == 0 and stu == 0
+        assert torch.equal(Ys[j], Y1) and torch.equal(Ys[j], Yu), j
+        Yref = oracle.gemm(cfg.dtype, Xs[j], M, lay.K, d["w"], lay.N, cfg.scale_kind, d["scales"],
+                           cfg.group_k)
+        assert rel_fro(Ys[j].cpu().numpy(), Yref) <= TOL
+
+
+def test_batched_mixed_layouts_consecutive_launches(cuda, oracle):
+    # past the small-M schedule the layers of different shapes run one after
+    # the other on the whole GPU: bit-identical to ans_gemm
+    layers = [_layer("llama8b_mlp", 768, 512), _layer("llama8b_mlp", 512, 768, seed_off=7)]
+    Xs, Ys, st = _run_batched(layers, 96)
+    assert st == 0
+    for j, (cfg, d, lay, layer) in enumerate(layers):
+        Y1, st1, _ = run_gemm(cfg, d, lay, layer, Xs[j], compressed=True)
+        assert st1 == 0 and torch.equal(Ys[j], Y1), j
+        Yref = oracle.gemm(cfg.dtype, Xs[j], 96, lay.K, d["w"], lay.N)
+        assert rel_fro(Ys[j].cpu().numpy(), Yref) <= TOL
+
+
+def test_batched_whole_llama_mlp_full_size(cuda, oracle, plan_limits):
+    # gate and up (14336 x 4096) and down (4096 x 14336) of the Llama-8B-shaped
+    # MLP in one launch at M = 16; each bit-identical to ans_gemm on its share
+    # of the SMs, fp64 check on 128 sampled W rows of each
+    base = WL.CONFIGS["llama8b_mlp"]
+    layers = []
+    for mi in (0, 1, 2):
+        d = WL.make_weights(base, mi)
+        lay = ans.make_layout(base.dtype, d["N"], d["K"], base.tile_n, base.tile_k, 64)
+        layers.append((base, d, lay, ans.CompressedLayer.from_weights(d["w"], lay, device="cuda")))
+    Xs, Ys, st = _run_batched(layers, 16)
+    assert st == 0
+    G = _shares(layers, _sms())
+    for j, (cfg, d, lay, layer) in enumerate(layers):
+        plan_limits(max_ctas=G[j])
+        Y1, st1, _ = run_gemm(cfg, d, lay, layer, Xs[j], compressed=True)
+        assert st1 == 0 and torch.equal(Ys[j], Y1), j
+        rows = np.random.default_rng(j).choice(lay.N, size=128, replace=False).astype(np.uint32)
+        Yref = oracle.gemm(cfg.dtype, Xs[j], 16, lay.K, d["w"], lay.N, rows=rows)
+        assert rel_fro(Ys[j].cpu().numpy()[:, rows], Yref) <= TOL

@@ -84,10 +84,8 @@ def test_fp4_gemm_parity(cuda, oracle, cases, N, K, M, state_bits, dtype):
 
 @pytest.mark.parametrize("schedule", ["local", "central"])
 @pytest.mark.parametrize("ctas,producers", [(8, 16), (3, 7)])
-def test_fp4_gemm_schedules(cuda, oracle, cases, monkeypatch, schedule, ctas, producers):
-    monkeypatch.setenv("ANS_GEMM_SCHEDULE", schedule)
-    monkeypatch.setenv("ANS_GEMM_MAX_CTAS", str(ctas))
-    monkeypatch.setenv("ANS_GEMM_MAX_PRODUCERS", str(producers))
+def test_fp4_gemm_schedules(cuda, oracle, cases, plan_limits, schedule, ctas, producers):
+    plan_limits(schedule=schedule, max_ctas=ctas, max_producers=producers)
     for state_bits, dtype in ((32, ans.FP4_E2M1), (64, ans.FP4_E2M1), (64, ans.FP4_PAIRS)):
         cfg, d, lay, layer = _case(cases, 512, 1024, state_bits, dtype)
         X = WL.make_x(cfg, 16, 1024)

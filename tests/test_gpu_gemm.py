@@ -121,15 +121,13 @@ def test_gemm_corrupt_stream_flags_status(cuda, cases):
                                         ("fp8_405b", 512, 1024, 300), ("tiny_int4", 512, 512, 130),
                                         ("int4_70b", 512, 2048, 16), ("fp8_405b", 512, 1024, 32),
                                         ("tiny_int4", 512, 512, 1)])
-def test_gemm_multi_round_schedules(cuda, oracle, cases, monkeypatch, schedule, ctas, producers,
+def test_gemm_multi_round_schedules(cuda, oracle, cases, plan_limits, schedule, ctas, producers,
                                     name, N, K, M):
     # few CTAs and few producer warps: many rounds (shared-accumulator
     # schedule) or long per-warp runs crossing W row blocks (local schedule,
     # M <= 32 only; larger M always takes the shared-accumulator schedule),
     # slab, chunk and X rings wrapping many times
-    monkeypatch.setenv("ANS_GEMM_SCHEDULE", schedule)
-    monkeypatch.setenv("ANS_GEMM_MAX_CTAS", str(ctas))
-    monkeypatch.setenv("ANS_GEMM_MAX_PRODUCERS", str(producers))
+    plan_limits(schedule=schedule, max_ctas=ctas, max_producers=producers)
     cfg, d, lay, layer = _case(cases, name, N, K)
     X = WL.make_x(cfg, M, K)
     Y, st, _ = run_gemm(cfg, d, lay, layer, X, compressed=True)
@@ -141,7 +139,7 @@ def test_gemm_multi_round_schedules(cuda, oracle, cases, monkeypatch, schedule, 
 
 @pytest.mark.parametrize("name,N,K,M", [("bf16_4096", 1024, 4096, 16), ("int4_70b", 512, 2048, 8),
                                         ("fp8_405b", 256, 2048, 32), ("tiny_int4", 512, 512, 1)])
-def test_gemm_both_schedules_small_m(cuda, oracle, cases, monkeypatch, name, N, K, M):
+def test_gemm_both_schedules_small_m(cuda, oracle, cases, plan_limits, name, N, K, M):
     # at M <= 32 the local schedule is the default; the shared-accumulator one
     # must agree with the fp64 oracle too (the two add in different orders, so
     # they agree to rounding, not bit for bit)
@@ -150,7 +148,7 @@ def test_gemm_both_schedules_small_m(cuda, oracle, cases, monkeypatch, name, N, 
     Yref = oracle.gemm(cfg.dtype, X, M, K, d["w"], N, cfg.scale_kind, d["scales"], cfg.group_k)
     out = {}
     for schedule in ["local", "central"]:
-        monkeypatch.setenv("ANS_GEMM_SCHEDULE", schedule)
+        plan_limits(schedule=schedule)
         Y, st, _ = run_gemm(cfg, d, lay, layer, X, compressed=True)
         Yu, stu, _ = run_gemm(cfg, d, lay, layer, X, compressed=False)
         assert st == 0 and stu == 0 and torch.equal(Y, Yu), schedule
@@ -160,10 +158,10 @@ def test_gemm_both_schedules_small_m(cuda, oracle, cases, monkeypatch, name, N, 
 
 
 @pytest.mark.parametrize("schedule", ["local", "central"])
-def test_gemm_bad_offsets_flag_status(cuda, cases, monkeypatch, schedule):
+def test_gemm_bad_offsets_flag_status(cuda, cases, plan_limits, schedule):
     # an offset table that points past the stream: the affected tiles are
     # skipped (treated as zero), the status says why, nothing reads outside
-    monkeypatch.setenv("ANS_GEMM_SCHEDULE", schedule)
+    plan_limits(schedule=schedule)
     cfg, d, lay, layer = _case(cases, "bf16_4096", 512, 1024)
     off = layer.h_offsets.copy()
     off[7] = off[-1] + 4096
@@ -178,12 +176,12 @@ def test_gemm_bad_offsets_flag_status(cuda, cases, monkeypatch, schedule):
 @pytest.mark.parametrize("name,N,K,M", [("bf16_4096", 1024, 2048, 16), ("int4_70b", 512, 2048, 16),
                                         ("fp8_405b", 512, 1024, 32), ("tiny_int4", 512, 512, 1),
                                         ("llama8b_mlp", 384, 2048, 5)])
-def test_gemm_local_long_producer_runs(cuda, oracle, cases, monkeypatch, ctas, name, N, K, M):
+def test_gemm_local_long_producer_runs(cuda, oracle, cases, plan_limits, ctas, name, N, K, M):
     # few CTAs: every producer warp of the local schedule owns a long run of
     # tiles crossing W row blocks (chunk rings wrap many times, several
     # accumulators per producer); bit-identical to the uncompressed variant
     # and within the bar of the fp64 oracle
-    monkeypatch.setenv("ANS_GEMM_MAX_CTAS", str(ctas))
+    plan_limits(max_ctas=ctas)
     cfg, d, lay, layer = _case(cases, name, N, K)
     X = WL.make_x(cfg, M, K)
     Y, st, _ = run_gemm(cfg, d, lay, layer, X, compressed=True)
@@ -193,9 +191,9 @@ def test_gemm_local_long_producer_runs(cuda, oracle, cases, monkeypatch, ctas, n
     assert rel_fro(Y.cpu().numpy(), Yref) <= TOL
 
 
-def test_gemm_long_runs_corrupt_and_bad_offsets(cuda, cases, monkeypatch):
+def test_gemm_long_runs_corrupt_and_bad_offsets(cuda, cases, plan_limits):
     # a corrupt or badly indexed tile in the middle of a producer's run
-    monkeypatch.setenv("ANS_GEMM_MAX_CTAS", "4")
+    plan_limits(max_ctas=4)
     cfg, d, lay, layer = _case(cases, "bf16_4096", 512, 1024)
     X = WL.make_x(cfg, 16, 1024)
     bad = layer.h_stream.copy()
@@ -272,6 +270,26 @@ def test_gemm_full_size_large_layers_sampled(cuda, oracle, cases, name, M):
     Yu, stu, _ = run_gemm(cfg, d, lay, layer, X, compressed=False)
     assert st == 0 and stu == 0 and torch.equal(Y, Yu)
     rows = np.random.default_rng(M).choice(lay.N, size=256, replace=False).astype(np.uint32)
+    Yref = oracle.gemm(cfg.dtype, X, M, lay.K, d["w"], lay.N, cfg.scale_kind, d["scales"],
+                       cfg.group_k, rows=rows)
+    assert rel_fro(Y.cpu().numpy()[:, rows], Yref) <= TOL
+
+
+@pytest.mark.parametrize("name,M,dtype", [("fp8_405b", 2048, None), ("fp8_405b", 256, None),
+                                          ("int4_70b", 1024, ans.INT4_PAIRS),
+                                          ("int4_70b", 1024, None), ("llama8b_mlp", 512, None)])
+def test_gemm_full_size_large_m_sampled(cuda, oracle, name, M, dtype):
+    # large token counts at full size, in the launch configuration the sweep
+    # times (several token passes of the shared-accumulator schedule for the
+    # 405B-shaped layer at M = 2048 and the 70B-shaped one at M = 1024):
+    # bit-identical to the uncompressed variant on all of Y, and within the
+    # bar of the fp64 oracle on 256 sampled W rows
+    cfg, d, lay, layer = make_case(name, state_bits=64, dtype=dtype)
+    X = WL.make_x(cfg, M)
+    Y, st, _ = run_gemm(cfg, d, lay, layer, X, compressed=True)
+    Yu, stu, _ = run_gemm(cfg, d, lay, layer, X, compressed=False)
+    assert st == 0 and stu == 0 and torch.equal(Y, Yu)
+    rows = np.random.default_rng(M + 7).choice(lay.N, size=256, replace=False).astype(np.uint32)
     Yref = oracle.gemm(cfg.dtype, X, M, lay.K, d["w"], lay.N, cfg.scale_kind, d["scales"],
                        cfg.group_k, rows=rows)
     assert rel_fro(Y.cpu().numpy()[:, rows], Yref) <= TOL

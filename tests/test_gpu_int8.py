@@ -76,10 +76,8 @@ def test_int8_gemm_parity(cuda, oracle, cases, N, K, M, state_bits):
 
 @pytest.mark.parametrize("schedule", ["local", "central"])
 @pytest.mark.parametrize("ctas,producers", [(8, 16), (3, 7)])
-def test_int8_gemm_schedules(cuda, oracle, cases, monkeypatch, schedule, ctas, producers):
-    monkeypatch.setenv("ANS_GEMM_SCHEDULE", schedule)
-    monkeypatch.setenv("ANS_GEMM_MAX_CTAS", str(ctas))
-    monkeypatch.setenv("ANS_GEMM_MAX_PRODUCERS", str(producers))
+def test_int8_gemm_schedules(cuda, oracle, cases, plan_limits, schedule, ctas, producers):
+    plan_limits(schedule=schedule, max_ctas=ctas, max_producers=producers)
     for state_bits in (32, 64):
         cfg, d, lay, layer = _case(cases, 512, 1024, state_bits)
         X = WL.make_x(cfg, 16, 1024)

@@ -148,11 +148,9 @@ def test_pairs_gemm_parity(cuda, oracle, cases, name, N, K, M, state_bits):
 @pytest.mark.parametrize("ctas,producers", [(8, 16), (3, 7)])
 @pytest.mark.parametrize("name,N,K,M", [("int4_70b", 512, 2048, 16), ("tiny_int4", 512, 512, 1),
                                         ("int4_70b", 1024, 1024, 130)])
-def test_pairs_gemm_schedules_and_long_runs(cuda, oracle, cases, monkeypatch, schedule, ctas,
+def test_pairs_gemm_schedules_and_long_runs(cuda, oracle, cases, plan_limits, schedule, ctas,
                                             producers, name, N, K, M):
-    monkeypatch.setenv("ANS_GEMM_SCHEDULE", schedule)
-    monkeypatch.setenv("ANS_GEMM_MAX_CTAS", str(ctas))
-    monkeypatch.setenv("ANS_GEMM_MAX_PRODUCERS", str(producers))
+    plan_limits(schedule=schedule, max_ctas=ctas, max_producers=producers)
     for state_bits in (32, 64):
         cfg, d, lay, layer = _case(cases, name, N, K, state_bits)
         X = WL.make_x(cfg, M, K)

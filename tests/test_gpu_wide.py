@@ -120,11 +120,9 @@ def test_wide_gemm_parity(cuda, oracle, cases, name, N, K, M):
 @pytest.mark.parametrize("name,N,K,M", [("bf16_4096", 1024, 2048, 16), ("int4_70b", 512, 2048, 16),
                                         ("fp8_405b", 512, 1024, 32), ("tiny_int4", 512, 512, 1),
                                         ("llama8b_mlp", 384, 2048, 130)])
-def test_wide_gemm_schedules_and_long_runs(cuda, oracle, cases, monkeypatch, schedule, ctas,
+def test_wide_gemm_schedules_and_long_runs(cuda, oracle, cases, plan_limits, schedule, ctas,
                                            producers, name, N, K, M):
-    monkeypatch.setenv("ANS_GEMM_SCHEDULE", schedule)
-    monkeypatch.setenv("ANS_GEMM_MAX_CTAS", str(ctas))
-    monkeypatch.setenv("ANS_GEMM_MAX_PRODUCERS", str(producers))
+    plan_limits(schedule=schedule, max_ctas=ctas, max_producers=producers)
     cfg, d, lay, layer = _case(cases, name, N, K)
     X = WL.make_x(cfg, M, K)
     Y, st, _ = run_gemm(cfg, d, lay, layer, X, compressed=True)

@@ -12,7 +12,7 @@ from rans_decode_gemm_b200 import workloads as WL
 
 FIELDS = ["local", "grid", "D", "n_slots", "tmem_cols", "smem_bytes", "T", "T_pass", "n_pass",
           "NT", "n_bufs", "fmt", "ab_f16", "H", "C", "x_stages", "n_units", "n_segments",
-          "ws_lo", "ws_hi"]
+          "ws_lo", "ws_hi", "n_banks"]
 SMEM_MAX = 232448          # sm_100 per-block dynamic shared memory
 FMT = {"bf16": 0, "int4_bf16": 1, "int4_group": 2, "fp8": 3, "int4_pair": 4,
        "int4_pair_group": 5, "int8": 6, "fp4": 7, "fp4_pair": 8}
@@ -23,7 +23,7 @@ def _plan(lay, M, kind, decode, sms):
     fn = lib.ansdev_gemm_plan
     fn.argtypes = [C.c_void_p, C.c_uint32, C.c_uint32, C.c_int, C.c_int, C.c_void_p]
     fn.restype = C.c_int
-    out = (C.c_uint32 * 20)()
+    out = (C.c_uint32 * 21)()
     r = fn(C.addressof(lay), M, kind, decode, sms, out)
     return r, dict(zip(FIELDS, list(out)))
 
@@ -64,9 +64,13 @@ def test_plans_fit_and_cover(ans_lib, name, dtype, state_bits):
             assert r == 1, (M, sms)
             ru, pu = _plan(lay, M, cfg.scale_kind, 0, sms)
             assert ru == 1
-            # the schedule does not depend on whether the weights are compressed
-            assert {k: v for k, v in p.items() if k != "fmt"} == \
-                   {k: v for k, v in pu.items() if k != "fmt"}, (M, sms)
+            # the schedule does not depend on whether the weights are compressed;
+            # the shared-accumulator schedule's copy variant lays out shared
+            # memory without the slot table and chunk rings (a deeper X ring),
+            # which does not change the order of the additions
+            layout = {"fmt"} | (set() if p["local"] else {"smem_bytes", "x_stages"})
+            assert {k: v for k, v in p.items() if k not in layout} == \
+                   {k: v for k, v in pu.items() if k not in layout}, (M, sms)
             assert p["fmt"] == _expected_fmt(dtype, cfg.scale_kind, True)
             assert pu["fmt"] == _expected_fmt(dtype, cfg.scale_kind, False)
             assert p["ab_f16"] == (1 if p["fmt"] in (2, 3, 5, 6) else 0)
@@ -83,8 +87,13 @@ def test_plans_fit_and_cover(ans_lib, name, dtype, state_bits):
                 assert p["n_slots"] * H * T <= tc
                 assert p["n_units"] == n_tiles and p["n_segments"] == N // cfg.tile_n
             else:
-                assert 1 <= p["D"] <= 16 and p["n_bufs"] in (1, 2)
-                assert p["n_bufs"] * H * p["T_pass"] <= 512
+                assert 1 <= p["D"] <= 14 and p["n_bufs"] in (1, 2)
+                # X stages: enough to cover the TMA latency of the X slabs
+                assert p["x_stages"] >= 3 and pu["x_stages"] >= p["x_stages"]
+                assert pu["smem_bytes"] <= SMEM_MAX
+                assert p["n_banks"] in (1, 2, 4)
+                assert p["n_banks"] * p["n_bufs"] * H * p["T_pass"] <= tc <= 512
+                assert p["n_banks"] * H * p["NT"] <= 32   # one issuing lane per accumulator
                 assert p["n_units"] == n_tiles * p["n_pass"]
                 assert p["n_segments"] == (N // cfg.tile_n) * p["n_pass"]
             assert p["ws_lo"] + (p["ws_hi"] << 32) > 0
