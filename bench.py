@@ -89,8 +89,8 @@ def parse():
                     help="--sweep: code int4 and fp4 weights one symbol per packed byte "
                          "(two K elements) or one per element")
     ap.add_argument("--rows", type=int, default=0,
-                    help="profiling: the headline layer cut to its first ROWS rows (a "
-                         "multiple of 128); 0 = the whole layer")
+                    help="profiling: the headline layer (or, with --sweep, every matrix) cut "
+                         "to its first ROWS rows (a multiple of the tile height); 0 = whole")
     ap.add_argument("--quick", action="store_true",
                     help="only the headline timing: no context sweep, secondary entry or "
                          "CPU baseline (profiling runs)")
@@ -641,7 +641,7 @@ def sweep(args):
         if only and name not in only:
             continue
         for mi, (mname, mN, mK) in enumerate(cfg.matrices):
-            d = WL.make_weights(cfg, mi)
+            d = WL.make_weights(cfg, mi, N=args.rows if args.rows else None)
             N, K = d["N"], d["K"]
             pairs = cfg.dtype in (WL.INT4, WL.FP4_E2M1) and args.nibble_symbols == "pairs"
             coded = ({WL.INT4: WL.INT4_PAIRS, WL.FP4_E2M1: WL.FP4_PAIRS}[cfg.dtype] if pairs

@@ -41,8 +41,9 @@
 namespace ansdev {
 
 constexpr uint32_t kFixedWarps = 6;
-// 6 fixed warps + 14 producers = 20 warps: about 100 registers a thread, so
-// that the issuing warp and the producers run without spills
+// 6 fixed warps + 14 producers = 20 warps (640 threads): about 100 registers
+// a thread, so that the issuing warp and the producers run without spills
+// (16 producers at 80 registers spill and run a few per cent slower)
 constexpr uint32_t kMaxProducers = 14;
 constexpr uint32_t kMaxThreads = (kFixedWarps + kMaxProducers) * 32;
 
@@ -51,53 +52,27 @@ constexpr uint32_t kMaxThreads = (kFixedWarps + kMaxProducers) * 32;
 //   w_empty[2 D]  the MMAs that read producer d's slot k are done (one
 //                 commit per slab)
 //   x_full[XS]    X stage holds its slab (TMA bytes)
-//   x_rel[XS]     X chunk k (xe consecutive stages) is free again (one commit
-//                 per chunk, after its last stage's MMAs)
+//   x_empty[XS]   the MMAs that read X stage k are done (one commit per stage)
 //   acc_full[2], acc_empty[2], mma_done, chunk[4 D] (compressed-stream rings)
 struct Bars {
-  uint64_t *w_full, *w_empty, *x_full, *x_rel, *acc_full, *acc_empty, *mma_done, *chunk;
+  uint64_t *w_full, *w_empty, *x_full, *x_empty, *acc_full, *acc_empty, *mma_done, *chunk;
 };
-
 __device__ __forceinline__ Bars carve_bars(uint8_t* base, uint32_t D, uint32_t XS) {
   uint64_t* b = reinterpret_cast<uint64_t*>(base);
   Bars r;
   r.w_full = b;
   r.w_empty = b + 2 * D;
   r.x_full = b + 4 * D;
-  r.x_rel = r.x_full + XS;
-  r.acc_full = r.x_rel + XS;
+  r.x_empty = b + 4 * D + XS;
+  r.acc_full = b + 4 * D + 2 * XS;
   r.acc_empty = r.acc_full + 2;
   r.mma_done = r.acc_empty + 2;
   r.chunk = r.mma_done + 1;
   return r;
 }
-
 __host__ __device__ inline uint32_t num_bars(uint32_t D, uint32_t XS) {
   return 4 * D + 2 * XS + 5 + 4 * D;
 }
-
-// X stages are released in chunks of xe consecutive stages (one commit per
-// chunk): 4 when the ring has 16 or more, else one at a time (a small ring
-// must not wait for a whole chunk); the ring uses xs_used = a multiple of xe
-// of its stages.
-__device__ __forceinline__ uint32_t x_chunk(uint32_t XS) { return XS >= 16 ? 4u : 1u; }
-
-// Units of round r of a CTA: [u0, u0 + nd).  With one accumulator set a round
-// that reaches into the next W row block is consumed in two parts (its units
-// of the first segment, then the rest); returns the units of the first part.
-__device__ __forceinline__ uint32_t round_part0(const GemmDev& P, uint32_t u0, uint32_t nd) {
-  return P.n_bufs == 2 ? nd : min(nd, P.L.n_kt - u0 % P.L.n_kt);
-}
-
-// Wait until the MMAs that read producer d's slab q - 2 (the slab before q in
-// the same slot) are done, before slab q is written into that slot.
-__device__ __forceinline__ bool wait_slot(const Bars& B, uint32_t d, uint32_t q,
-                                          volatile uint32_t* abort, uint32_t* status,
-                                          uint32_t backoff_ns = 0) {
-  return q < 2 || wait_live(&B.w_empty[2 * d + (q & 1u)], ((q >> 1) + 1) & 1u, abort, status, 1,
-                            backoff_ns);
-}
-
 // Where a unit sits: K tile, token pass and W row-block segment, plus
 // whether it opens / closes its segment within this CTA's range.
 struct UnitInfo {
@@ -149,6 +124,7 @@ __device__ __forceinline__ void for_each_mma_step(const GemmDev& P, uint32_t u_b
   }
 }
 
+// ---------------------------------------------------------------------------
 // ---------------------------------------------------------------------------
 // Producer side of one W slab in copy mode (ans_gemm_uncompressed): the slab
 // (rows n0 + 128 h .. + 127, columns k0 + 16 s .. + 15) formatted like the
@@ -227,7 +203,6 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     reduce_flag = 0;
   }
   {
-    // arrivals per phase: the epilogue's four warps on acc_empty, one otherwise
     uint64_t* b0 = B.w_full;  // the barriers are one array, in carve_bars order
     const uint32_t n_bars = num_bars(D, XS);
     for (uint32_t i = threadIdx.x; i < n_bars; i += blockDim.x)
@@ -276,12 +251,12 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
           const uint32_t n0 = (t / n_kt) * L.tile_n, k0 = (t % n_kt) * L.tile_k;
           for (uint32_t us = 0; us < n_us; ++us, ++q) {
             const uint32_t h = us % H, s = us / H, slot = q & 1u;
-            if (!wait_slot(B, d, q, abort, P.status)) break;
+            if (q >= 2 && !wait_live(&B.w_empty[2 * d + slot], ((q >> 1) + 1) & 1u, abort, P.status, 1))
+              break;
             const uint32_t bar = smem_u32(&B.w_full[2 * d + slot]);
             mbar_arrive_expect_tx_s(bar, kSlabBytes);
-            tma_load_2d_hint_s(wslots_s + slot * kSlabBytes, &P.tmap_w,
-                               static_cast<int32_t>(k0 + 16 * s), static_cast<int32_t>(n0 + 128 * h),
-                               bar, l2_evict_first());
+            tma_load_2d_s(wslots_s + slot * kSlabBytes, &P.tmap_w, static_cast<int32_t>(k0 + 16 * s),
+                          static_cast<int32_t>(n0 + 128 * h), bar);
           }
           if (*abort) break;
         }
@@ -305,8 +280,8 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         const uint32_t h = us % H, s = us / H;
         const uint32_t bar = smem_u32(&raw_bar[q & 1u]);
         mbar_arrive_expect_tx_s(bar, 128 * 16);
-        tma_load_2d_hint_s(raw_s + (q & 1u) * 2048, &P.tmap_w, static_cast<int32_t>(k0 + 16 * s),
-                           static_cast<int32_t>(n0 + 128 * h), bar, l2_evict_first());
+        tma_load_2d_s(raw_s + (q & 1u) * 2048, &P.tmap_w, static_cast<int32_t>(k0 + 16 * s),
+                      static_cast<int32_t>(n0 + 128 * h), bar);
       };
       uint32_t issued = 0;
       if (lane == 0)
@@ -338,7 +313,8 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
           copy_bytes_fmt<kFmt>(v[i].x, v[i].y, o[i][0]);
           copy_bytes_fmt<kFmt>(v[i].z, v[i].w, o[i][1]);
         }
-        const bool free_slot = wait_slot(B, d, q, abort, P.status);
+        const bool free_slot =
+            q < 2 || wait_live(&B.w_empty[2 * d + slot], ((q >> 1) + 1) & 1u, abort, P.status, 1);
         if (__any_sync(0xFFFFFFFFu, !free_slot)) break;
         const uint32_t slab_s = wslots_s + slot * kSlabBytes;
 #pragma unroll
@@ -421,7 +397,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
           // copy mode: fetch the slab's 8 groups before waiting for the slot
           uint4 cp[8];
           if constexpr (!kDecode) copy_loads<kFmt>(P, n0, k0, h, s, lane, cp);
-          wait_slot(B, d, sc, abort, P.status, 64);
+          if (sc >= 2) wait_live(&B.w_empty[2 * d + slot], ((sc >> 1) + 1) & 1u, abort, P.status, 1, 64);
           const uint32_t slab_s = wslots_s + slot * kSlabBytes;
           // a group is 8 columns of one row, or both 8-column halves of it for
           // int4 pair symbols (4 groups per slab)
@@ -500,34 +476,27 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     // so the accumulation order does not depend on timing.  For every (round,
     // part, slab) group the warp's lanes first test the W barriers of all its
     // producers at once (one round trip instead of one per producer), then
-    // lane 0 issues the group's MMAs.  Where TMEM has room the units are
-    // spread over accumulator banks -- unit u into bank (u - u_begin) % banks,
-    // each bank accumulated in unit order and the banks summed in bank order
-    // by the epilogue -- so consecutive MMAs go to different accumulators.
-    // Each W slot is released by a commit right after its MMAs (so its
-    // producer can write the next slab as early as possible), the X stages by
-    // one commit per chunk.
+    // lane 0 issues the group's MMAs, X stage by X stage.
     const uint32_t ub = static_cast<uint32_t>(u_begin), ue = static_cast<uint32_t>(u_end);
     const uint32_t seg_begin = ub / n_kt;
-    const uint32_t H = P.H, NT = P.NT, NB = P.n_banks;
-    const uint32_t XE = x_chunk(XS), XSu = XS - XS % XE;
+    const uint32_t H = P.H;
     // descriptor fields shared by every operand: LBO 16 B, SBO 256 B,
     // version 1, 32-byte swizzle; only the start address varies
     const uint64_t dhi = (1ull << 16) | (16ull << 32) | (1ull << 46) | (6ull << 61);
     const uint32_t a_base = smem_u32(wring) >> 4, x_base = smem_u32(xring) >> 4;
     const uint32_t slab16 = kSlabBytes >> 4, xstage16 = x_stage_bytes >> 4, t16 = (P.T * 32) >> 4;
-    uint32_t n = 0;  // MMA steps (X stages) of the CTA before the current group
-    uint32_t g = 0;  // groups consumed
+    uint32_t fresh = 0;  // bit (buf * 2 + h): next MMA into that accumulator starts it
+    uint32_t xs = 0, xpar = 0;
     uint32_t r = 0;
     bool live = true;
     for (uint32_t u0 = ub; u0 < ue && live; u0 += D, ++r) {
       const uint32_t nd = min(D, ue - u0);
       const uint32_t seg0 = u0 / n_kt, kt0 = u0 - seg0 * n_kt;
-      const uint32_t nA = round_part0(P, u0, nd);
+      const uint32_t nA = P.n_bufs == 2 ? nd : min(nd, n_kt - kt0);
       for (uint32_t part = 0; part < 2 && live; ++part) {
         const uint32_t d_lo = part == 0 ? 0 : nA, d_hi = part == 0 ? nA : nd;
         if (d_lo == d_hi) continue;
-        for (uint32_t s = 0; s < P.C && live; ++s, ++g) {
+        for (uint32_t s = 0; s < P.C && live; ++s) {
           // readiness of every W slab of the group, one lane per (producer, half)
           bool ok = true;
           const uint32_t ng = (d_hi - d_lo) * H;
@@ -539,7 +508,6 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
           if (__ballot_sync(0xFFFFFFFFu, !ok) != 0) live = false;
           if (!live) break;
           if (lane == 0) {
-            if (g == 0) trace_mark(P, 48);
             tc_fence_after();
             for (uint32_t d = d_lo; d < d_hi; ++d) {
               const uint32_t kt = kt0 + d;
@@ -547,46 +515,41 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
               const uint32_t ktw = wrap ? kt - n_kt : kt;
               const uint32_t lseg = seg0 + (wrap ? 1u : 0u) - seg_begin;
               const uint32_t buf = P.n_bufs == 2 ? (lseg & 1u) : 0u;
-              const uint32_t u = u0 + d;
-              const uint32_t bank = (u - ub) % NB;
-              const uint32_t step = n + (d - d_lo);
-              // the segment's units in this CTA start at u_first; its first
-              // NB units start one bank each (their first slab), and the first
-              // one waits until the epilogue has drained the buffer
-              const uint32_t u_first = max(ub, (seg_begin + lseg) * n_kt);
-              const bool start = s == 0 && u - u_first < NB;
-              if (start && u == u_first) {
+              if (s == 0 && (u0 + d == ub || ktw == 0)) {
                 const uint32_t k = P.n_bufs == 2 ? (lseg >> 1) : lseg;
                 if (k >= 1 && !wait_live(&B.acc_empty[buf], (k - 1) & 1u, abort, P.status, 4)) {
                   live = false;
                   break;
                 }
                 tc_fence_after();
+                fresh |= 3u << (2 * buf);
               }
-              const uint32_t xs = step % XSu;
-              if (!wait_live(&B.x_full[xs], (step / XSu) & 1u, abort, P.status, 2)) {
+              if (!wait_live(&B.x_full[xs], xpar, abort, P.status, 2)) {
                 live = false;
                 break;
               }
+              tc_fence_after();
               for (uint32_t h = 0; h < H; ++h) {
                 const uint32_t idx = (r * P.C + s) * H + h;
-                const uint64_t adesc = dhi | (a_base + (2 * d + (idx & 1u)) * slab16);
-                for (uint32_t j = 0; j < NT; ++j) {
+                const uint32_t slot = idx & 1u;
+                const uint64_t adesc = dhi | (a_base + (2 * d + slot) * slab16);
+                const uint32_t acc_bit = 1u << (2 * buf + h);
+                const uint32_t accumulate = (fresh & acc_bit) ? 0u : 1u;
+                for (uint32_t j = 0; j < P.NT; ++j) {
                   const uint64_t bdesc = dhi | (x_base + xs * xstage16 + j * t16);
-                  const uint32_t col = (((buf * NB + bank) * H + h) * NT + j) * P.T;
-                  umma_f16(tmem_base + col, adesc, bdesc, P.idesc, start ? 0u : 1u);
+                  const uint32_t col = ((buf * H + h) * P.NT + j) * P.T;
+                  umma_f16(tmem_base + col, adesc, bdesc, P.idesc, accumulate);
                 }
-                // the slot is free for its producer once these MMAs are done
-                umma_commit(&B.w_empty[2 * d + (idx & 1u)]);
+                fresh &= ~acc_bit;
+                umma_commit(&B.w_empty[2 * d + slot]);
               }
-              // the last stage of an X chunk: the chunk is free once these MMAs are done
-              if (step % XE == XE - 1) umma_commit(&B.x_rel[xs / XE]);
+              umma_commit(&B.x_empty[xs]);
+              if (++xs == XS) { xs = 0; xpar ^= 1u; }
               if (s == P.C - 1 && (u0 + d + 1 == ue || ktw + 1 == n_kt))
                 umma_commit(&B.acc_full[buf]);
             }
           }
           live = __shfl_sync(0xFFFFFFFFu, live ? 1u : 0u, 0) != 0;
-          n += d_hi - d_lo;
         }
       }
     }
@@ -600,34 +563,30 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     // X slab (token pass p, columns kx .. kx + 15) is the tensor map's box at
     // (kx, p * T_pass + j * T) for j < NT; rows past M land as zeros.
     if (lane == 0) {
-      const uint32_t XE = x_chunk(XS), XSu = XS - XS % XE;
       uint32_t xc = 0;
       uint32_t n_issued = 0;  // loads issued: steps [0, n_issued) (none after an abort)
       const uint32_t xring_s = smem_u32(xring);
       for_each_mma_step(P, static_cast<uint32_t>(u_begin), static_cast<uint32_t>(u_end),
                         [&](uint32_t, uint32_t s, uint32_t, uint32_t, const UnitInfo& I) {
-        const uint32_t xs = xc % XSu;
-        // the stage's chunk was released by its last use (one lap earlier)
-        if (xc >= XSu) wait_live(&B.x_rel[xs / XE], ((xc / XSu) - 1) & 1u, abort, P.status, 5, 32);
+        const uint32_t xs = xc % XS;
+        if (xc >= XS) wait_live(&B.x_empty[xs], ((xc / XS) + 1) & 1u, abort, P.status, 5, 32);
         if (!*abort && n_issued == xc) {
           const uint32_t kx = I.kt * P.L.tile_k + 16 * s;
           const uint32_t bar = smem_u32(&B.x_full[xs]);
           mbar_arrive_expect_tx_s(bar, x_stage_bytes);
-          // X slabs are read by every CTA working at their K columns: kept in L2
-          const uint64_t pol = l2_evict_last();
           for (uint32_t j = 0; j < P.NT; ++j)
-            tma_load_2d_hint_s(xring_s + xs * x_stage_bytes + j * P.T * 32, &P.tmap_x,
-                               static_cast<int32_t>(kx), static_cast<int32_t>(I.p * P.T_pass + j * P.T),
-                               bar, pol);
+            tma_load_2d_s(xring_s + xs * x_stage_bytes + j * P.T * 32, &P.tmap_x,
+                          static_cast<int32_t>(kx), static_cast<int32_t>(I.p * P.T_pass + j * P.T),
+                          bar);
           n_issued = xc + 1;
         }
         ++xc;
       });
       trace_mark(P, 42);
       // drain: the last load issued into every stage must have landed
-      const uint32_t first = n_issued > XSu ? n_issued - XSu : 0;
+      const uint32_t first = n_issued > XS ? n_issued - XS : 0;
       for (uint32_t q = first; q < n_issued; ++q)
-        wait_drain(&B.x_full[q % XSu], (q / XSu) & 1u, P.status);
+        wait_drain(&B.x_full[q % XS], (q / XS) & 1u, P.status);
       trace_mark(P, 35);
     }
     __syncwarp();
@@ -650,66 +609,26 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
       const bool complete = u_begin <= s_lo && u_end >= s_hi;
       const uint32_t slot = (seg == seg_first) ? 0u : 1u;
       float* part = P.partials + (static_cast<uint64_t>(blockIdx.x) * 2 + slot) * P.H * P.T_pass * 128;
-      // banks that hold a part of the segment: unit u went to bank
-      // (u - u_begin) % banks, so the segment's first units in this CTA name them
-      const uint32_t NB = P.n_banks;
-      uint32_t bmask = 0;
-      {
-        const uint32_t a = max(u_begin, s_lo), b = min(u_end, s_hi);
-        for (uint32_t u = a; u < b && u < a + NB; ++u) bmask |= 1u << ((u - u_begin) % NB);
-      }
       for (uint32_t h = 0; h < P.H; ++h) {
         const uint32_t n = rb * P.L.tile_n + h * 128 + e;
         const float scale = complete ? row_scale(P, n) : 1.0f;
         for (uint32_t j = 0; j < P.NT; ++j) {
+          const uint32_t col0 = ((buf * P.H + h) * P.NT + j) * P.T;
           // tokens past M are padding: stop at the last 16-column chunk holding one
           const uint32_t m0 = p * P.T_pass + j * P.T;
           const uint32_t t_end = P.M > m0 ? min(P.T, P.M - m0) : 0u;
-          auto col_of = [&](uint32_t bank) {
-            return tmem_base + ((32 * warp) << 16) + (((buf * NB + bank) * P.H + h) * P.NT + j) * P.T;
-          };
-          if (NB == 1) {
-            for (uint32_t cc = 0; cc < t_end; cc += 32) {
-              uint32_t v[2][16];
-              tmem_ld16(col_of(0) + cc, v[0]);
-              if (cc + 16 < t_end) tmem_ld16(col_of(0) + cc + 16, v[1]);
-              tmem_ld_wait();
+          for (uint32_t cc = 0; cc < t_end; cc += 32) {
+            uint32_t v[2][16];
+            tmem_ld16(tmem_base + ((32 * warp) << 16) + col0 + cc, v[0]);
+            if (cc + 16 < t_end) tmem_ld16(tmem_base + ((32 * warp) << 16) + col0 + cc + 16, v[1]);
+            tmem_ld_wait();
 #pragma unroll
-              for (uint32_t k = 0; k < 2; ++k) {
-                if (cc + 16 * k >= t_end) break;
-                float f[16];
+            for (uint32_t k = 0; k < 2; ++k) {
+              if (cc + 16 * k >= t_end) break;
+              float f[16];
 #pragma unroll
-                for (int q = 0; q < 16; ++q) f[q] = __uint_as_float(v[k][q]);
-                epi_emit16(P, f, complete, scale, part, p, h, j * P.T + cc + 16 * k, n, e);
-              }
-            }
-          } else {
-            // the banks' sums, added in bank order, eight columns at a time:
-            // the first bank loads into the sum, one more rides along with
-            // it, further ones one by one
-            for (uint32_t cc = 0; cc < t_end; cc += 8) {
-              uint32_t a[8], v[8];
-              uint32_t m = bmask;
-              tmem_ld8(col_of(__ffs(m) - 1) + cc, a);
-              m &= m - 1;
-              const bool two = m != 0;
-              if (two) {
-                tmem_ld8(col_of(__ffs(m) - 1) + cc, v);
-                m &= m - 1;
-              }
-              tmem_ld_wait();
-              float f[8];
-#pragma unroll
-              for (int q = 0; q < 8; ++q)
-                f[q] = two ? __uint_as_float(a[q]) + __uint_as_float(v[q]) : __uint_as_float(a[q]);
-              while (m) {
-                tmem_ld8(col_of(__ffs(m) - 1) + cc, v);
-                m &= m - 1;
-                tmem_ld_wait();
-#pragma unroll
-                for (int q = 0; q < 8; ++q) f[q] += __uint_as_float(v[q]);
-              }
-              epi_emit<8>(P, f, complete, scale, part, p, h, j * P.T + cc, n, e);
+              for (int q = 0; q < 16; ++q) f[q] = __uint_as_float(v[k][q]);
+              epi_emit16(P, f, complete, scale, part, p, h, j * P.T + cc + 16 * k, n, e);
             }
           }
         }
@@ -740,7 +659,6 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
   }
   // the split-K reductions this CTA arrived last for, on every thread
   if (reduce_flag) {
-    if (threadIdx.x == 0) trace_mark(P, 49);
     fence_acq_rel_gpu();  // acquire: the counter showed every contributor arrived
     for (uint32_t k = 0; k < red_n; ++k)
       if ((reduce_flag >> k) & 1u) splitk_reduce(P, G, red_seg[k], threadIdx.x, blockDim.x);
@@ -906,14 +824,7 @@ bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool dec
   p.T_pass = p.T * p.NT;
   p.n_pass = (M + p.T_pass - 1) / p.T_pass;
   if (p.n_pass == 0) p.n_pass = 1;
-  // Accumulator banks: where TMEM has room the units of a CTA are spread
-  // over 2 or 4 banks (unit u into bank (u - u_begin) % banks), summed in
-  // bank order by the epilogue, so that consecutive MMAs write different
-  // accumulators.
-  p.n_banks = 1;
-  for (uint32_t nb = 4; nb >= 2; nb /= 2)
-    if (nb * p.n_bufs * p.H * p.T_pass <= max_cols) { p.n_banks = nb; break; }
-  uint32_t cols = p.n_banks * p.n_bufs * p.H * p.T_pass;
+  const uint32_t cols = p.n_bufs * p.H * p.T_pass;
   p.tmem_cols = 32;
   while (p.tmem_cols < cols) p.tmem_cols <<= 1;
   if (p.tmem_cols > 512) return false;
@@ -1063,7 +974,6 @@ static GemmDev make_gemm_dev(const GemmPlan& plan, const LayerDev& L, const void
   P.C = plan.C;
   P.D = plan.D;
   P.n_bufs = plan.n_bufs;
-  P.n_banks = plan.n_banks ? plan.n_banks : 1;
   P.x_stages = plan.x_stages;
   P.tmem_cols = plan.tmem_cols;
   P.n_rb = L.N / L.tile_n;

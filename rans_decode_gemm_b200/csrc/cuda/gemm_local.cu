@@ -438,6 +438,7 @@ __device__ __forceinline__ void local_cta(const GemmDev& P) {
     const uint32_t a_s = smem_u32(wslots) + 2 * q * kSlabBytes;
     const uint32_t b_s = smem_u32(xslots) + 2 * q * T * 32;
     long long idle_since = clock64();
+    const long long idle_budget = g_live_wait_budget;
     for (;;) {
       const bool has = q < D && u < pe;
       if (__ballot_sync(0xFFFFFFFFu, has) == 0) break;
@@ -446,7 +447,7 @@ __device__ __forceinline__ void local_cta(const GemmDev& P) {
       const uint32_t rmask = __ballot_sync(0xFFFFFFFFu, ready);
       if (rmask == 0) {
         if (*abort) break;
-        if (clock64() - idle_since > g_live_wait_budget) {
+        if (clock64() - idle_since > idle_budget) {
           if (lane == 0) {
             *abort = 1u;
             atomicOr(P.status, kStatusTimeout | (1u << (8 + 2)));

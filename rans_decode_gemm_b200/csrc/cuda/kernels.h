@@ -56,7 +56,6 @@ struct GemmPlan {
   uint32_t H, C;       // 128-row halves per tile, 16-column slabs per tile
   uint32_t D;          // producer warps per CTA
   uint32_t n_bufs;     // TMEM accumulator sets (1 or 2)
-  uint32_t n_banks;    // shared-accumulator schedule: accumulator banks per set (1, 2 or 4)
   uint32_t x_stages;    // X stages of the shared-accumulator schedule (differs between the
                         // decode and copy variants; the accumulation order does not depend on it)
   uint32_t tmem_cols;
@@ -93,7 +92,6 @@ struct GemmDev {
   uint32_t scale_kind, group_k, n_groups_k;
   uint32_t M, T, NT, T_pass, n_pass;
   uint32_t H, C, D, n_bufs, x_stages, tmem_cols;
-  uint32_t n_banks;
   uint32_t n_rb;
   uint64_t n_units;
   uint32_t idesc;

@@ -77,7 +77,10 @@ enum : uint32_t {
 // set_live_wait_budget_* functions).  Drains of copies already in flight
 // always wait kWaitBudgetCycles: those copies land on their own, and a CTA
 // must not exit while one is still writing its shared memory.
-static __device__ long long g_live_wait_budget = kWaitBudgetCycles;
+// Constant memory (one copy per translation unit, filled with
+// cudaMemcpyToSymbol): a wait reads it once, before its spin loop, from the
+// constant cache -- a spin loop must not wait on a memory load between polls.
+static __constant__ long long g_live_wait_budget = kWaitBudgetCycles;
 
 // Abort-aware bounded wait.  Returns false if the wait ran out (then sets the
 // CTA's abort flag and the TIMEOUT status bit) or if the CTA already aborted.
@@ -88,10 +91,11 @@ __device__ __forceinline__ bool wait_live(uint64_t* bar, uint32_t parity, volati
                                           uint32_t* status, uint32_t site = 0,
                                           uint32_t backoff_ns = 0) {
   if (mbar_try_wait(bar, parity)) return true;
-  long long t0 = clock64();
+  const long long budget = g_live_wait_budget;
+  const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
     if (*abort) return false;
-    if (clock64() - t0 > g_live_wait_budget) {
+    if (clock64() - t0 > budget) {
       *abort = 1u;
       atomicOr(status, kStatusTimeout | (1u << (8 + site)));
       return false;
@@ -105,10 +109,11 @@ __device__ __forceinline__ bool wait_live(uint64_t* bar, uint32_t parity, volati
 __device__ __forceinline__ bool wait_live_s(uint32_t bar_s, uint32_t parity, volatile uint32_t* abort,
                                             uint32_t* status, uint32_t site = 0) {
   if (mbar_try_wait_s(bar_s, parity)) return true;
-  long long t0 = clock64();
+  const long long budget = g_live_wait_budget;
+  const long long t0 = clock64();
   while (!mbar_try_wait_s(bar_s, parity)) {
     if (*abort) return false;
-    if (clock64() - t0 > g_live_wait_budget) {
+    if (clock64() - t0 > budget) {
       *abort = 1u;
       atomicOr(status, kStatusTimeout | (1u << (8 + site)));
       return false;
@@ -126,6 +131,7 @@ __device__ __forceinline__ bool wait_all_live(uint64_t* bars, uint32_t n, uint32
                                               volatile uint32_t* abort, uint32_t* status,
                                               uint32_t site, uint32_t backoff_ns) {
   const uint32_t b0 = smem_u32(bars);
+  const long long budget = g_live_wait_budget;
   long long t0 = 0;
   for (uint32_t pass = 0;; ++pass) {
     bool all = true;
@@ -135,7 +141,7 @@ __device__ __forceinline__ bool wait_all_live(uint64_t* bars, uint32_t n, uint32
     if (all) return true;
     if (pass == 0) t0 = clock64();
     if (*abort) return false;
-    if (clock64() - t0 > g_live_wait_budget) {
+    if (clock64() - t0 > budget) {
       *abort = 1u;
       atomicOr(status, kStatusTimeout | (1u << (8 + site)));
       return false;
