@@ -416,6 +416,7 @@ int ansdev_set_wait_budget(long long cycles) {
   cudaError_t e = ansdev::set_live_wait_budget_gemm(c);
   if (e == cudaSuccess) e = ansdev::set_live_wait_budget_local(c);
   if (e == cudaSuccess) e = ansdev::set_live_wait_budget_decode(c);
+  if (e == cudaSuccess) e = ansdev::set_live_wait_budget_dense(c);
   return e == cudaSuccess ? ANS_OK : cuda_fail(e, "ansdev_set_wait_budget");
 }
 

@@ -170,6 +170,36 @@ __device__ __forceinline__ void copy_bytes_fmt(uint32_t lo, uint32_t hi, uint32_
   else fmt_fp8_f16(e, o);
 }
 
+// Uncompressed weights (N x K codes) into the 16-bit operand format, N x K
+// row-major (the same values the producers write into the slabs): thread i
+// formats the eight elements 8 i .. 8 i + 7.
+template <uint32_t kFmt>
+__global__ void format_w16_kernel(const void* w, const void* scales, uint32_t K, uint32_t group_k,
+                                  uint32_t n_groups_k, uint16_t* w16, uint64_t n8) {
+  griddep_wait();
+  griddep_launch_dependents();
+  for (uint64_t i = blockIdx.x * static_cast<uint64_t>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<uint64_t>(gridDim.x) * blockDim.x) {
+    uint32_t o[4];
+    if constexpr (kFmt == kFmtFp8F16 || kFmt == kFmtInt8F16) {
+      const uint2 v = __ldg(reinterpret_cast<const uint2*>(w) + i);
+      copy_bytes_fmt<kFmt>(v.x, v.y, o);
+    } else {
+      const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(w) + i);
+      __half2 gs = __float2half2_rn(0.f);
+      if constexpr (fmt_group(kFmt)) {
+        const uint64_t e0 = i * 8;
+        const uint64_t row = e0 / K;
+        const uint32_t g = static_cast<uint32_t>(e0 - row * K) / group_k;
+        gs = __float2half2_rn(bf16_to_f32(
+            __ldg(static_cast<const uint16_t*>(scales) + row * n_groups_k + g)));
+      }
+      copy_nibbles_fmt<kFmt>(v, gs, o);
+    }
+    reinterpret_cast<uint4*>(w16)[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
 // ---------------------------------------------------------------------------
 template <bool kDecode, uint32_t kFmt, bool kWide>
 __global__ void __launch_bounds__(kMaxThreads, 1)
@@ -398,6 +428,11 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
           uint4 cp[8];
           if constexpr (!kDecode) copy_loads<kFmt>(P, n0, k0, h, s, lane, cp);
           if (sc >= 2) wait_live(&B.w_empty[2 * d + slot], ((sc >> 1) + 1) & 1u, abort, P.status, 1, 64);
+          if (kDecode && P.store_w16) {
+            // the store of the slot's previous slab has read it
+            if (lane == 0) bulk_wait_read<1>();
+            __syncwarp();
+          }
           const uint32_t slab_s = wslots_s + slot * kSlabBytes;
           // a group is 8 columns of one row, or both 8-column halves of it for
           // int4 pair symbols (4 groups per slab)
@@ -460,6 +495,10 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive(&B.w_full[2 * d + slot]);
+          // first token pass of a large-M call: the slab also goes to W16
+          if (kDecode && P.store_w16 && lane == 0)
+            tma_store_2d_s(&P.tmap_w, static_cast<int32_t>(k0 + 16 * s),
+                           static_cast<int32_t>(n0 + 128 * h), slab_s);
           if (lane == 0 && sc == 0) trace_mark(P, 2 + d);
           ++sc;
         }
@@ -468,6 +507,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         }
       }
       if (kDecode) pipe_drain(pipe, P.status);
+      if (kDecode && P.store_w16 && lane == 0) bulk_wait_all();
     }
     if (lane == 0) trace_mark(P, 18 + d);
   } else if (warp == 4) {
@@ -749,6 +789,7 @@ bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool dec
   // per CTA, force the shared-accumulator schedule
   const uint32_t cap_ctas = g_cap_ctas.load(std::memory_order_relaxed);
   if (cap_ctas > 0 && cap_ctas < sms) sms = cap_ctas;
+  p.sms = static_cast<uint32_t>(sms);
   const uint32_t cap_prod = g_cap_producers.load(std::memory_order_relaxed);
   // unit indices are 32-bit in the kernels
   if (static_cast<uint64_t>(L.n_tiles) * ((M + 15) / 16) >= (1ull << 31)) return false;
@@ -828,6 +869,30 @@ bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool dec
   p.tmem_cols = 32;
   while (p.tmem_cols < cols) p.tmem_cols <<= 1;
   if (p.tmem_cols > 512) return false;
+  if (p.n_pass > 1 && L.K % 64 == 0) {
+    // More tokens than one pass: the first T_pass tokens run fused (the
+    // decode variant decodes every tile once and also stores the decoded
+    // weights, W16), the rest run as one dense GEMM on W16 (gemm_dense.cu).
+    // This plan is the first pass's, with the call's token count and the
+    // workspace of the whole call.
+    GemmPlan first;
+    if (!make_gemm_plan(L, p.T_pass, scale_kind, decode, num_sms, &first) || first.n_pass != 1)
+      return false;
+    const uint32_t n_pass = p.n_pass;
+    p = first;
+    p.M = M;
+    p.n_pass = n_pass;
+    p.n_units = static_cast<uint64_t>(n_pass) * L.n_tiles;
+    p.n_segments = n_pass * (L.N / L.tile_n);
+    p.ws_x16_bytes = p.ab_f16 ? static_cast<size_t>(M) * L.K * 2 : 0;
+    // W16: decoded by the first pass, or the uncompressed codes formatted
+    // (bf16 weights are used as they are)
+    p.ws_w16_bytes = (decode || p.fmt != kFmtBf16Split) ? static_cast<size_t>(L.N) * L.K * 2 : 0;
+    p.ws_bytes = p.ws_counters_bytes + (p.ws_partials_bytes + 255) / 256 * 256 +
+                 (p.ws_x16_bytes + 255) / 256 * 256 + p.ws_w16_bytes;
+    *plan = p;
+    return true;
+  }
 
   p.n_units = static_cast<uint64_t>(p.n_pass) * L.n_tiles;
   p.n_segments = p.n_pass * (L.N / L.tile_n);
@@ -993,28 +1058,51 @@ static GemmDev make_gemm_dev(const GemmPlan& plan, const LayerDev& L, const void
   return P;
 }
 
-cudaError_t launch_gemm(const GemmPlan& plan, const LayerDev& L, bool decode, const void* w_plain,
-                        const uint16_t* X, const void* scales, uint32_t scale_kind,
-                        uint32_t group_k, float* Y, void* ws, uint32_t* status,
-                        cudaStream_t stream) {
-  if (plan.M == 0) return cudaSuccess;
+// Grid for an elementwise pass over n items, 256 threads a block.
+static uint32_t stream_blocks(uint64_t n) {
+  uint64_t b = (n + 255) / 256;
+  if (b > 4096) b = 4096;
+  return b == 0 ? 1u : static_cast<uint32_t>(b);
+}
+
+// X (M x K bf16) as f16 into x16, for the formats whose MMA operands are f16.
+static cudaError_t convert_x(const uint16_t* X, uint32_t M, uint32_t K, uint8_t* x16,
+                             cudaStream_t stream) {
+  const uint64_t n8 = static_cast<uint64_t>(M) * K / 8;
+  return launch_pdl(x_to_f16_kernel, dim3(stream_blocks(n8)), dim3(256), 0, stream, X,
+                    reinterpret_cast<uint16_t*>(x16), n8);
+}
+
+// One launch of a single-pass plan.  x16_ready: this call's f16 copy of X,
+// already made (null: made here when the format wants it).  w16: when set,
+// the decode variant also stores every decoded slab there (N x K row-major).
+static cudaError_t launch_single(const GemmPlan& plan, const LayerDev& L, bool decode,
+                                 const void* w_plain, const uint16_t* X, const uint8_t* x16_ready,
+                                 const void* scales, uint32_t scale_kind, uint32_t group_k, float* Y,
+                                 void* ws, uint16_t* w16, uint32_t* status, cudaStream_t stream) {
   GemmDev P = make_gemm_dev(plan, L, w_plain, X, scales, scale_kind, group_k, Y, ws, status);
   if (!plan.local) {
     // X for the MMA as a tensor map: the caller's bf16 X, or its f16 copy
     const void* xsrc = X;
     if (plan.ab_f16) {
-      const uint64_t n8 = static_cast<uint64_t>(plan.M) * L.K / 8;
-      uint32_t blocks = static_cast<uint32_t>((n8 + 255) / 256);
-      if (blocks > 4096) blocks = 4096;
-      if (blocks == 0) blocks = 1;
-      cudaError_t e = launch_pdl(x_to_f16_kernel, dim3(blocks), dim3(256), 0, stream, X,
-                                 reinterpret_cast<uint16_t*>(const_cast<uint8_t*>(P.xs)), n8);
-      if (e != cudaSuccess) return e;
+      if (x16_ready) {
+        P.xs = x16_ready;
+      } else {
+        cudaError_t e = convert_x(X, plan.M, L.K, const_cast<uint8_t*>(P.xs), stream);
+        if (e != cudaSuccess) return e;
+      }
       xsrc = P.xs;
     }
     cudaError_t e = encode_tmap(&P.tmap_x, CU_TENSOR_MAP_DATA_TYPE_UINT16, xsrc, L.K, plan.M,
                                 static_cast<uint64_t>(L.K) * 2, 16, plan.T, CU_TENSOR_MAP_SWIZZLE_32B);
     if (e != cudaSuccess) return e;
+    if (decode && w16) {
+      // the decoded slabs' destination: W16 as 16 x 128 boxes, the slab layout
+      e = encode_tmap(&P.tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT16, w16, L.K, L.N,
+                      static_cast<uint64_t>(L.K) * 2, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B);
+      if (e != cudaSuccess) return e;
+      P.store_w16 = 1;
+    }
     if (!decode) {
       const uint32_t cm = copy_mode_of(plan.fmt);
       if (cm == kCopyTmaSlab)
@@ -1064,6 +1152,90 @@ cudaError_t launch_gemm(const GemmPlan& plan, const LayerDev& L, bool decode, co
     case 16 | kFmtFp4Bf16: return launch_variant<false, kFmtFp4Bf16>(plan, P, stream);
   }
   return cudaErrorInvalidValue;
+}
+
+static cudaError_t format_w16(uint32_t fmt, const void* w, const void* scales, const LayerDev& L,
+                              uint32_t group_k, uint16_t* w16, cudaStream_t stream) {
+  const uint64_t n8 = static_cast<uint64_t>(L.N) * L.K / 8;
+  const uint32_t ngk = group_k ? L.K / group_k : 0;
+  const dim3 g(stream_blocks(n8)), b(256);
+  switch (fmt) {
+    case kFmtInt4Bf16:
+      return launch_pdl(format_w16_kernel<kFmtInt4Bf16>, g, b, 0, stream, w, scales, L.K, group_k, ngk, w16, n8);
+    case kFmtInt4F16Group:
+      return launch_pdl(format_w16_kernel<kFmtInt4F16Group>, g, b, 0, stream, w, scales, L.K, group_k, ngk, w16, n8);
+    case kFmtFp8F16:
+      return launch_pdl(format_w16_kernel<kFmtFp8F16>, g, b, 0, stream, w, scales, L.K, group_k, ngk, w16, n8);
+    case kFmtInt8F16:
+      return launch_pdl(format_w16_kernel<kFmtInt8F16>, g, b, 0, stream, w, scales, L.K, group_k, ngk, w16, n8);
+    case kFmtFp4Bf16:
+      return launch_pdl(format_w16_kernel<kFmtFp4Bf16>, g, b, 0, stream, w, scales, L.K, group_k, ngk, w16, n8);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_gemm(const GemmPlan& plan, const LayerDev& L, bool decode, const void* w_plain,
+                        const uint16_t* X, const void* scales, uint32_t scale_kind,
+                        uint32_t group_k, float* Y, void* ws, uint32_t* status,
+                        cudaStream_t stream) {
+  if (plan.M == 0) return cudaSuccess;
+  if (plan.local || plan.n_pass == 1 || L.K % 64 != 0)
+    return launch_single(plan, L, decode, w_plain, X, nullptr, scales, scale_kind, group_k, Y, ws,
+                         nullptr, status, stream);
+  // Large M: the first T_pass tokens fused (the decode variant storing the
+  // decoded weights into W16), then every other token in one dense GEMM on
+  // W16 -- the uncompressed variant formats its codes into W16 the same way
+  // (bf16 weights are used as they are), so both variants feed the dense
+  // kernel the same operands.
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  uint8_t* x16 = wsb + plan.ws_counters_bytes + (plan.ws_partials_bytes + 255) / 256 * 256;
+  uint16_t* w16 = reinterpret_cast<uint16_t*>(x16 + (plan.ws_x16_bytes + 255) / 256 * 256);
+  cudaError_t e;
+  if (plan.ab_f16) {
+    e = convert_x(X, plan.M, L.K, x16, stream);
+    if (e != cudaSuccess) return e;
+  }
+  GemmPlan first;
+  if (!make_gemm_plan(L, plan.T_pass, scale_kind, decode, static_cast<int>(plan.sms), &first))
+    return cudaErrorInvalidValue;
+  e = launch_single(first, L, decode, w_plain, X, plan.ab_f16 ? x16 : nullptr, scales, scale_kind,
+                    group_k, Y, ws, decode ? w16 : nullptr, status, stream);
+  if (e != cudaSuccess) return e;
+  const void* wop = w16;
+  if (!decode) {
+    if (plan.fmt == kFmtBf16Split) {
+      wop = w_plain;
+    } else {
+      e = format_w16(plan.fmt, w_plain, scales, L, group_k, w16, stream);
+      if (e != cudaSuccess) return e;
+    }
+  }
+  const uint32_t M_rest = plan.M - plan.T_pass;
+  const void* xr = plan.ab_f16 ? static_cast<const void*>(x16 + static_cast<uint64_t>(plan.T_pass) * L.K * 2)
+                               : static_cast<const void*>(X + static_cast<uint64_t>(plan.T_pass) * L.K);
+  DenseDev D;
+  std::memset(&D, 0, sizeof(D));
+  e = encode_tmap(&D.tmap_a, CU_TENSOR_MAP_DATA_TYPE_UINT16, wop, L.K, L.N,
+                  static_cast<uint64_t>(L.K) * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e != cudaSuccess) return e;
+  // a box of at most M_rest rows; the MMA's token columns past it hold stale
+  // shared memory and are never stored
+  e = encode_tmap(&D.tmap_b, CU_TENSOR_MAP_DATA_TYPE_UINT16, xr, L.K, M_rest,
+                  static_cast<uint64_t>(L.K) * 2, 64, std::min(M_rest, 256u),
+                  CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e != cudaSuccess) return e;
+  D.Y = Y + static_cast<uint64_t>(plan.T_pass) * L.N;
+  D.scales = scales;
+  D.status = status;
+  D.scale_kind = scale_kind;
+  D.M = M_rest;
+  D.N = L.N;
+  D.K = L.K;
+  D.m_blocks = (M_rest + 255) / 256;
+  D.n_tiles = D.m_blocks * (L.N / 128);
+  D.b_box_rows = std::min(M_rest, 256u);
+  D.idesc = idesc_f16(plan.ab_f16 ? 0u : 1u, 128, 256);
+  return launch_dense_gemm(D, plan.sms, stream);
 }
 
 cudaError_t launch_gemm_batched(const GemmPlan* plans, uint32_t n, const LayerDev* const* Ls,

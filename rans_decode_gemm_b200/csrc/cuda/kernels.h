@@ -66,7 +66,11 @@ struct GemmPlan {
   uint32_t n_segments; // n_pass * (N / tile_n)
   uint32_t smem_bytes;
   uint32_t off_lut, off_w, off_chunk, off_x, off_bars;
-  size_t ws_partials_bytes, ws_counters_bytes, ws_x16_bytes, ws_bytes;
+  uint32_t sms;        // SMs the plan was made for
+  // workspace: [counters][partials][f16 copy of X][W16]; W16 (the weights
+  // decoded or formatted to the 16-bit operand format, N x K row-major) only
+  // when the call has several token passes (see launch_gemm)
+  size_t ws_partials_bytes, ws_counters_bytes, ws_x16_bytes, ws_w16_bytes, ws_bytes;
 };
 
 // How the producers of the shared-accumulator schedule fill W slabs from
@@ -109,7 +113,30 @@ struct GemmDev {
   // 16 bytes x 128 rows, no swizzle)
   CUtensorMap tmap_x;
   CUtensorMap tmap_w;
+  // first token pass of a large-M call (decode variant): every decoded slab
+  // is also stored, through tmap_w, into W16 (N x K row-major, the operand
+  // format) for the dense kernel that takes the remaining tokens
+  uint32_t store_w16;
 };
+
+// Dense GEMM on 16-bit weights that are already in the MMA operand format
+// (gemm_dense.cu): Y[m][n] = s_n * sum_k X[m][k] W[n][k] for m < M, fp32 Y
+// (M x N row-major).  W (N x K) and X (M x K) are 16-bit row-major and given
+// as 2-D tensor maps with 64 x 128 (W) and 64 x 256 (X) boxes, 128-byte
+// swizzle; tiles of 128 W rows x 256 tokens, W-row-block major.
+struct DenseDev {
+  CUtensorMap tmap_a;   // W
+  CUtensorMap tmap_b;   // X
+  float* Y;
+  const void* scales;   // scale_kind 1: bf16 per row, 2: fp32 per row, else none
+  uint32_t* status;
+  uint32_t scale_kind;
+  uint32_t M, N, K;
+  uint32_t m_blocks, n_tiles;
+  uint32_t b_box_rows;  // rows of X a box brings (256, or M when smaller)
+  uint32_t idesc;
+};
+cudaError_t launch_dense_gemm(const DenseDev& P, uint32_t sms, cudaStream_t stream);
 
 // Several layers in one launch of the local schedule (shapes may differ; one
 // operand format): job j owns CTAs [job[j].cta0, job[j].cta0 + job[j].n_cta)
@@ -139,6 +166,7 @@ void set_plan_limits(uint32_t max_ctas, uint32_t max_producers, uint32_t force_s
 cudaError_t set_live_wait_budget_gemm(long long cycles);
 cudaError_t set_live_wait_budget_local(long long cycles);
 cudaError_t set_live_wait_budget_decode(long long cycles);
+cudaError_t set_live_wait_budget_dense(long long cycles);
 cudaError_t launch_wait_probe(uint32_t* status, cudaStream_t stream);
 
 // Scratch capacity of the allocation-free entry point (16 MiB per device).

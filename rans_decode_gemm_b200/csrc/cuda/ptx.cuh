@@ -163,6 +163,26 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
 // element size must be a multiple of 16 bytes; dst_s aligned to 128 bytes
 // (256 with the 32-byte swizzle).  Rows past the tensor's extent land as
 // zeros.
+// TMA store of one 2-D box from this CTA's shared memory (laid out as the
+// tensor map's box, swizzle included) to the tensor at (x, y), committed as
+// one bulk group of the calling thread.  x, y >= 0; x * element size a
+// multiple of 16 bytes.
+__device__ __forceinline__ void tma_store_2d_s(const void* tmap, int32_t x, int32_t y, uint32_t src_s) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(tmap),
+               "r"(x), "r"(y), "r"(src_s)
+               : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until at most N of the calling thread's bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Wait until every bulk group of the calling thread has completed.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d_s(uint32_t dst_s, const void* tmap, int32_t x,
                                               int32_t y, uint32_t bar_s) {
   asm volatile(

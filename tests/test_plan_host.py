@@ -69,6 +69,13 @@ def test_plans_fit_and_cover(ans_lib, name, dtype, state_bits):
             # memory without the slot table and chunk rings (a deeper X ring),
             # which does not change the order of the additions
             layout = {"fmt"} | (set() if p["local"] else {"smem_bytes", "x_stages"})
+            # several token passes: the workspace holds the decoded weights
+            # for the dense GEMM of the later tokens (the uncompressed
+            # variant's own bf16 weights need no copy)
+            if p["n_pass"] > 1 and K % 64 == 0:
+                layout |= {"ws_lo", "ws_hi"}
+                ws, wsu = p["ws_lo"] + (p["ws_hi"] << 32), pu["ws_lo"] + (pu["ws_hi"] << 32)
+                assert ws - wsu == (N * K * 2 if dtype == WL.BF16_SPLIT else 0)
             assert {k: v for k, v in p.items() if k not in layout} == \
                    {k: v for k, v in pu.items() if k not in layout}, (M, sms)
             assert p["fmt"] == _expected_fmt(dtype, cfg.scale_kind, True)
