@@ -219,7 +219,10 @@ ans_status ans_decode_tiles(const ans_tiles* tiles, void* d_out, uint32_t* d_sta
 /* Bytes of device workspace ans_gemm / ans_gemm_uncompressed need for a
  * layout, M tokens and a scale kind.  The workspace must be zero-filled once
  * before its first use; the kernels return it to all-zero counters on
- * completion (after a run that set *d_status, zero it again). */
+ * completion (after a run that set *d_status, zero it again).  Above one
+ * token pass (M > 512 for 128-row tiles, M > 256 for 256-row tiles, with K a
+ * multiple of 64) it also holds a 16-bit copy of the decoded weights, 2 N K
+ * bytes (see ans_gemm). */
 ans_status ans_gemm_workspace(const ans_layout* layout, uint32_t M, ans_scale_kind scale_kind,
                               size_t* bytes);
 
@@ -232,9 +235,14 @@ ans_status ans_gemm_workspace(const ans_layout* layout, uint32_t M, ans_scale_ki
  *   int8: q (NONE) or q * s[n] (ROW_BF16 or ROW_F32);
  *   fp4: e2m1 value (NONE) or value * s[n] (ROW_BF16 or ROW_F32).
  * W's tiles are decoded by producer warps straight into shared memory in the
- * tensor-core operand layout and consumed by tcgen05 MMAs; they never reach
- * global memory.  Accumulation is fp32 in a fixed order, so the result is
- * bit-identical to ans_gemm_uncompressed on the same weights.  GROUP_BF16 runs
+ * tensor-core operand layout and consumed by tcgen05 MMAs.  Up to one token
+ * pass (512 tokens for 128-row tiles, 256 for 256-row tiles) the decoded
+ * weights never reach global memory.  Above it, the first pass runs fused
+ * and also stores every decoded tile into the workspace, and the remaining
+ * tokens run as one dense tensor-core GEMM on those stored weights.  Each
+ * tile is then decoded once per call, not once per pass.  Accumulation is
+ * fp32 in a fixed order, so the result is bit-identical to
+ * ans_gemm_uncompressed on the same weights.  GROUP_BF16 runs
  * the MMA in f16 (X and q*s are exact in f16 when |X| < 65504 and the scales
  * lie in [2^-14, 2^12]), and so do fp8 and int8 (their codes are exact in
  * f16, the row scale is applied to the fp32 accumulator); the other kinds run
@@ -271,7 +279,10 @@ ans_status ans_gemm_noalloc(const uint16_t* d_X, uint32_t M, const ans_tiles* W,
 
 /* The same kernel with the decoder warps replaced by a copy of the original
  * (uncompressed) weights d_W (format of layout->dtype, row-major N x K).
- * Bit-exact reference for ans_gemm and the uncompressed baseline. */
+ * Above one token pass the codes are formatted into the workspace's 16-bit
+ * copy for the dense GEMM, as ans_gemm's decoded ones are.  bf16 weights are
+ * read in place.  Bit-exact reference for ans_gemm and the uncompressed
+ * baseline. */
 ans_status ans_gemm_uncompressed(const uint16_t* d_X, uint32_t M, const void* d_W,
                                  const ans_layout* layout, ans_scale_kind scale_kind,
                                  const void* d_scales, uint32_t group_k, float* d_Y, void* d_ws,

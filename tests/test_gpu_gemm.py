@@ -293,3 +293,36 @@ def test_gemm_full_size_large_m_sampled(cuda, oracle, name, M, dtype):
     Yref = oracle.gemm(cfg.dtype, X, M, lay.K, d["w"], lay.N, cfg.scale_kind, d["scales"],
                        cfg.group_k, rows=rows)
     assert rel_fro(Y.cpu().numpy()[:, rows], Yref) <= TOL
+
+
+@pytest.mark.parametrize("name,N,K,M", [("bf16_4096", 512, 1024, 513), ("bf16_4096", 512, 1024, 812),
+                                        ("fp8_405b", 256, 2048, 1100), ("int4_70b", 512, 1024, 257),
+                                        ("int8_8b", 384, 1024, 700), ("fp4_8b", 384, 1024, 530),
+                                        ("tiny_int4", 128, 96, 600)])
+def test_gemm_large_m_dense_path_edges(cuda, oracle, cases, name, N, K, M):
+    # more tokens than one pass: the first pass fused, the rest through the
+    # dense GEMM on the decoded weights -- a single token left over (one row
+    # of X in the dense kernel's box), two token blocks with a ragged second,
+    # every coded format; K not a multiple of 64 keeps every pass fused
+    cfg, d, lay, layer = _case(cases, name, N, K)
+    X = WL.make_x(cfg, M, K)
+    Y, st, _ = run_gemm(cfg, d, lay, layer, X, compressed=True)
+    Yu, stu, _ = run_gemm(cfg, d, lay, layer, X, compressed=False)
+    assert st == 0 and stu == 0
+    assert torch.equal(Y, Yu), "ans_gemm must be bit-identical to ans_gemm_uncompressed"
+    Yref = oracle.gemm(cfg.dtype, X, M, K, d["w"], N, cfg.scale_kind, d["scales"], cfg.group_k)
+    assert rel_fro(Y.cpu().numpy(), Yref) <= TOL
+
+
+@pytest.mark.parametrize("dtype", [ans.INT4_PAIRS, ans.FP4_PAIRS])
+def test_gemm_large_m_pair_symbols(cuda, oracle, dtype):
+    # pair-symbol layouts store the same decoded weights as per-element ones
+    name = "int4_70b" if dtype == ans.INT4_PAIRS else "fp4_8b"
+    cfg, d, lay, layer = make_case(name, 512, 1024, state_bits=64, dtype=dtype)
+    M = 700
+    X = WL.make_x(cfg, M, 1024)
+    Y, st, _ = run_gemm(cfg, d, lay, layer, X, compressed=True)
+    Yu, stu, _ = run_gemm(cfg, d, lay, layer, X, compressed=False)
+    assert st == 0 and stu == 0 and torch.equal(Y, Yu)
+    Yref = oracle.gemm(cfg.dtype, X, M, 1024, d["w"], 512, cfg.scale_kind, d["scales"], cfg.group_k)
+    assert rel_fro(Y.cpu().numpy(), Yref) <= TOL

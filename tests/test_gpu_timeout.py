@@ -74,3 +74,21 @@ def test_decode_tiles_with_short_waits_is_exact_or_flagged(cuda, wait_budget):
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     assert np.array_equal(out.cpu().numpy(), d["w"])
+
+
+def test_large_m_waits_run_out_then_the_next_call_is_exact(cuda, oracle, wait_budget):
+    # the fused first pass and the dense GEMM of the remaining tokens both
+    # return on a run-out wait with the flag set; the next call is exact
+    cfg, d, lay, layer = make_case("bf16_4096", 512, 1024, state_bits=64)
+    M = 700
+    X = WL.make_x(cfg, M, 1024)
+    wait_budget(2000)
+    Y, st, ws = run_gemm(cfg, d, lay, layer, X, compressed=True)
+    assert st & ans.STATUS_TIMEOUT
+    wait_budget(0)
+    nseg = lay.N // lay.tile_n
+    assert int(ws[:4 * nseg].view(torch.int32).abs().sum().item()) == 0
+    Y, st, _ = run_gemm(cfg, d, lay, layer, X, compressed=True, ws=ws)
+    assert st == 0
+    Yref = oracle.gemm(cfg.dtype, X, M, 1024, d["w"], 512)
+    assert rel_fro(Y.cpu().numpy(), Yref) <= TOL
