@@ -260,7 +260,8 @@ ans_status ans_gemm(const uint16_t* d_X, uint32_t M, const ans_tiles* W,
  * device memory, or latency-critical paths that may not take an allocation's
  * implicit synchronisation).  Same arguments and result as ans_gemm, without
  * the workspace: the scratch (split-K counters and partials, the f16 copy of
- * X for the f16 formats) lives in a fixed 16 MiB device array inside the
+ * X for the f16 formats and, above one token pass, the decoded copy of W)
+ * lives in a fixed 16 MiB device array inside the
  * library, which every GPU that loads the library holds until the process
  * exits.  A shape whose ans_gemm_workspace exceeds 16 MiB returns
  * ANS_ERR_BUFFER_TOO_SMALL (text via ans_last_error).  Every argument check of

@@ -436,9 +436,11 @@ void ansdev_set_plan_limits(uint32_t max_ctas, uint32_t max_producers, uint32_t 
 // Internal test hook (not part of the public ABI): the launch plan that
 // ans_gemm (decode = 1) or ans_gemm_uncompressed (decode = 0) would use for a
 // layout, M and scale kind on a device with num_sms SMs, without touching a
-// device.  out[0..19] = local, grid, D, n_slots, tmem_cols, smem_bytes, T,
+// device.  out[0..20] = local, grid, D, n_slots, tmem_cols, smem_bytes, T,
 // T_pass, n_pass, NT, n_bufs, fmt, ab_f16, H, C, x_stages, n_units,
-// n_segments, ws_bytes (low 32 bits), ws_bytes (high 32 bits).
+// n_segments, ws_bytes (low 32 bits), ws_bytes (high 32 bits), dense (1: a
+// fused first pass of 16 tokens, then the dense GEMM; the other fields are
+// the first pass's).
 // Returns 1 if the shape can be scheduled, 0 if not, -1 for a bad layout.
 int ansdev_gemm_plan(const ans_layout* layout, uint32_t M, uint32_t scale_kind, int decode,
                      int num_sms, uint32_t* out) {
@@ -448,12 +450,12 @@ int ansdev_gemm_plan(const ans_layout* layout, uint32_t M, uint32_t scale_kind, 
   L.wide = layout->state_bits == 64 ? 1u : 0u;
   ansdev::GemmPlan p;
   if (!ansdev::make_gemm_plan(L, M, scale_kind, decode != 0, num_sms, &p)) return 0;
-  const uint32_t v[20] = {p.local, p.grid, p.D, p.n_slots, p.tmem_cols, p.smem_bytes, p.T,
+  const uint32_t v[21] = {p.local, p.grid, p.D, p.n_slots, p.tmem_cols, p.smem_bytes, p.T,
                           p.T_pass, p.n_pass, p.NT, p.n_bufs, p.fmt, p.ab_f16, p.H, p.C,
                           p.x_stages, static_cast<uint32_t>(p.n_units), p.n_segments,
                           static_cast<uint32_t>(p.ws_bytes),
-                          static_cast<uint32_t>(static_cast<uint64_t>(p.ws_bytes) >> 32)};
-  for (int i = 0; i < 20; ++i) out[i] = v[i];
+                          static_cast<uint32_t>(static_cast<uint64_t>(p.ws_bytes) >> 32), p.dense};
+  for (int i = 0; i < 21; ++i) out[i] = v[i];
   return 1;
 }
 

@@ -793,9 +793,43 @@ bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool dec
   const uint32_t cap_prod = g_cap_producers.load(std::memory_order_relaxed);
   // unit indices are 32-bit in the kernels
   if (static_cast<uint64_t>(L.n_tiles) * ((M + 15) / 16) >= (1ull << 31)) return false;
-  bool want_local = p.H * Mp <= 32;
+  // The small-M schedule keeps a private accumulator of H * T columns per
+  // producer and accumulator slot.  256-row tiles at 17-32 tokens (64
+  // columns: about 7 producers fit TMEM) take it only with pair symbols,
+  // whose cheaper decode keeps up with fewer producers; the choice depends on
+  // the layout alone, so both variants plan the same schedule.
+  const bool pair_layout = L.dtype == 3 || L.dtype == 6;
+  bool want_local = p.H * Mp <= 32 || (pair_layout && Mp <= 32 && p.H * Mp <= 64);
   if (g_force_shared.load(std::memory_order_relaxed)) want_local = false;
   const uint32_t lut_bytes = kSlots * 4;
+
+  // More tokens than one pass of the shared-accumulator schedule (512 / H):
+  // the first kDenseFirstTokens tokens run fused on the small-M schedule,
+  // whose decoders are the fastest, and store every decoded slab into W16;
+  // the other tokens run as one dense GEMM on W16 (gemm_dense.cu).  The plan
+  // is the first pass's, with the call's token count and the workspace of
+  // the whole call.
+  // (When the first pass does not fit the small-M schedule -- a device of
+  // very few SMs -- every pass runs on the shared-accumulator schedule.)
+  GemmPlan first;
+  if (M > 512 / p.H && L.K % 64 == 0 && !g_force_shared.load(std::memory_order_relaxed) &&
+      make_gemm_plan(L, kDenseFirstTokens, scale_kind, decode, num_sms, &first) && first.local) {
+    const uint32_t T_pass = 512 / p.H;
+    p = first;
+    p.M = M;
+    p.dense = 1;
+    p.M_first = kDenseFirstTokens;
+    p.T_pass = T_pass;
+    p.n_pass = (M + T_pass - 1) / T_pass;
+    p.ws_x16_bytes = p.ab_f16 ? static_cast<size_t>(M) * L.K * 2 : 0;
+    // W16: decoded by the first pass, or the uncompressed codes formatted
+    // (bf16 weights are used as they are)
+    p.ws_w16_bytes = (decode || p.fmt != kFmtBf16Split) ? static_cast<size_t>(L.N) * L.K * 2 : 0;
+    p.ws_bytes = p.ws_counters_bytes + (p.ws_partials_bytes + 255) / 256 * 256 +
+                 (p.ws_x16_bytes + 255) / 256 * 256 + p.ws_w16_bytes;
+    *plan = p;
+    return true;
+  }
 
   if (want_local) {
     // ---- local schedule: every producer issues its own MMAs (gemm_local.cu)
@@ -869,30 +903,6 @@ bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool dec
   p.tmem_cols = 32;
   while (p.tmem_cols < cols) p.tmem_cols <<= 1;
   if (p.tmem_cols > 512) return false;
-  if (p.n_pass > 1 && L.K % 64 == 0) {
-    // More tokens than one pass: the first T_pass tokens run fused (the
-    // decode variant decodes every tile once and also stores the decoded
-    // weights, W16), the rest run as one dense GEMM on W16 (gemm_dense.cu).
-    // This plan is the first pass's, with the call's token count and the
-    // workspace of the whole call.
-    GemmPlan first;
-    if (!make_gemm_plan(L, p.T_pass, scale_kind, decode, num_sms, &first) || first.n_pass != 1)
-      return false;
-    const uint32_t n_pass = p.n_pass;
-    p = first;
-    p.M = M;
-    p.n_pass = n_pass;
-    p.n_units = static_cast<uint64_t>(n_pass) * L.n_tiles;
-    p.n_segments = n_pass * (L.N / L.tile_n);
-    p.ws_x16_bytes = p.ab_f16 ? static_cast<size_t>(M) * L.K * 2 : 0;
-    // W16: decoded by the first pass, or the uncompressed codes formatted
-    // (bf16 weights are used as they are)
-    p.ws_w16_bytes = (decode || p.fmt != kFmtBf16Split) ? static_cast<size_t>(L.N) * L.K * 2 : 0;
-    p.ws_bytes = p.ws_counters_bytes + (p.ws_partials_bytes + 255) / 256 * 256 +
-                 (p.ws_x16_bytes + 255) / 256 * 256 + p.ws_w16_bytes;
-    *plan = p;
-    return true;
-  }
 
   p.n_units = static_cast<uint64_t>(p.n_pass) * L.n_tiles;
   p.n_segments = p.n_pass * (L.N / L.tile_n);
@@ -1081,6 +1091,13 @@ static cudaError_t launch_single(const GemmPlan& plan, const LayerDev& L, bool d
                                  const void* scales, uint32_t scale_kind, uint32_t group_k, float* Y,
                                  void* ws, uint16_t* w16, uint32_t* status, cudaStream_t stream) {
   GemmDev P = make_gemm_dev(plan, L, w_plain, X, scales, scale_kind, group_k, Y, ws, status);
+  if (decode && w16) {
+    // the decoded slabs' destination: W16 as 16 x 128 boxes, the slab layout
+    cudaError_t e = encode_tmap(&P.tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT16, w16, L.K, L.N,
+                                static_cast<uint64_t>(L.K) * 2, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B);
+    if (e != cudaSuccess) return e;
+    P.store_w16 = 1;
+  }
   if (!plan.local) {
     // X for the MMA as a tensor map: the caller's bf16 X, or its f16 copy
     const void* xsrc = X;
@@ -1096,13 +1113,6 @@ static cudaError_t launch_single(const GemmPlan& plan, const LayerDev& L, bool d
     cudaError_t e = encode_tmap(&P.tmap_x, CU_TENSOR_MAP_DATA_TYPE_UINT16, xsrc, L.K, plan.M,
                                 static_cast<uint64_t>(L.K) * 2, 16, plan.T, CU_TENSOR_MAP_SWIZZLE_32B);
     if (e != cudaSuccess) return e;
-    if (decode && w16) {
-      // the decoded slabs' destination: W16 as 16 x 128 boxes, the slab layout
-      e = encode_tmap(&P.tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT16, w16, L.K, L.N,
-                      static_cast<uint64_t>(L.K) * 2, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B);
-      if (e != cudaSuccess) return e;
-      P.store_w16 = 1;
-    }
     if (!decode) {
       const uint32_t cm = copy_mode_of(plan.fmt);
       if (cm == kCopyTmaSlab)
@@ -1179,10 +1189,10 @@ cudaError_t launch_gemm(const GemmPlan& plan, const LayerDev& L, bool decode, co
                         uint32_t group_k, float* Y, void* ws, uint32_t* status,
                         cudaStream_t stream) {
   if (plan.M == 0) return cudaSuccess;
-  if (plan.local || plan.n_pass == 1 || L.K % 64 != 0)
+  if (!plan.dense)
     return launch_single(plan, L, decode, w_plain, X, nullptr, scales, scale_kind, group_k, Y, ws,
                          nullptr, status, stream);
-  // Large M: the first T_pass tokens fused (the decode variant storing the
+  // Large M: the first M_first tokens fused (the decode variant storing the
   // decoded weights into W16), then every other token in one dense GEMM on
   // W16 -- the uncompressed variant formats its codes into W16 the same way
   // (bf16 weights are used as they are), so both variants feed the dense
@@ -1196,7 +1206,7 @@ cudaError_t launch_gemm(const GemmPlan& plan, const LayerDev& L, bool decode, co
     if (e != cudaSuccess) return e;
   }
   GemmPlan first;
-  if (!make_gemm_plan(L, plan.T_pass, scale_kind, decode, static_cast<int>(plan.sms), &first))
+  if (!make_gemm_plan(L, plan.M_first, scale_kind, decode, static_cast<int>(plan.sms), &first))
     return cudaErrorInvalidValue;
   e = launch_single(first, L, decode, w_plain, X, plan.ab_f16 ? x16 : nullptr, scales, scale_kind,
                     group_k, Y, ws, decode ? w16 : nullptr, status, stream);
@@ -1210,9 +1220,9 @@ cudaError_t launch_gemm(const GemmPlan& plan, const LayerDev& L, bool decode, co
       if (e != cudaSuccess) return e;
     }
   }
-  const uint32_t M_rest = plan.M - plan.T_pass;
-  const void* xr = plan.ab_f16 ? static_cast<const void*>(x16 + static_cast<uint64_t>(plan.T_pass) * L.K * 2)
-                               : static_cast<const void*>(X + static_cast<uint64_t>(plan.T_pass) * L.K);
+  const uint32_t M_rest = plan.M - plan.M_first;
+  const void* xr = plan.ab_f16 ? static_cast<const void*>(x16 + static_cast<uint64_t>(plan.M_first) * L.K * 2)
+                               : static_cast<const void*>(X + static_cast<uint64_t>(plan.M_first) * L.K);
   DenseDev D;
   std::memset(&D, 0, sizeof(D));
   e = encode_tmap(&D.tmap_a, CU_TENSOR_MAP_DATA_TYPE_UINT16, wop, L.K, L.N,
@@ -1224,7 +1234,7 @@ cudaError_t launch_gemm(const GemmPlan& plan, const LayerDev& L, bool decode, co
                   static_cast<uint64_t>(L.K) * 2, 64, std::min(M_rest, 256u),
                   CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
-  D.Y = Y + static_cast<uint64_t>(plan.T_pass) * L.N;
+  D.Y = Y + static_cast<uint64_t>(plan.M_first) * L.N;
   D.scales = scales;
   D.status = status;
   D.scale_kind = scale_kind;

@@ -297,8 +297,14 @@ __device__ __forceinline__ void local_cta(const GemmDev& P) {
 #pragma unroll
             for (uint32_t k = 0; k < kOut; ++k) o_prev[k] = 0;
             auto store_prev = [&](uint32_t gg) {
-              if (gg == 1 && nw >= 2)
+              if (gg == 1 && nw >= 2) {
                 wait_live(&w_empty[2 * d + slot], ((nw >> 1) + 1) & 1u, abort, P.status, 1);
+                if (kDecode && P.store_w16) {
+                  // the W16 store of the slot's previous slab has read it
+                  if (lane == 0) bulk_wait_read<1>();
+                  __syncwarp();
+                }
+              }
               const uint32_t row_s = w_s + (32 * ((gg - 1) & 3) + lane) * 32;
               if constexpr (kPair) {
                 sts128(row_s + swz, o_prev[0], o_prev[1], o_prev[2], o_prev[3]);
@@ -403,6 +409,10 @@ __device__ __forceinline__ void local_cta(const GemmDev& P) {
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&w_full[2 * d + slot]);
+            // first pass of a large-M call: the slab also goes to W16
+            if (kDecode && P.store_w16 && lane == 0)
+              tma_store_2d_s(&P.tmap_w, static_cast<int32_t>(k0 + 16 * s),
+                             static_cast<int32_t>(n0 + 128 * h), w_s);
             ++nw;
           }
         };
@@ -416,6 +426,7 @@ __device__ __forceinline__ void local_cta(const GemmDev& P) {
       }
     }
     if (kDecode) rp_drain(pipe, P.status);
+    if (kDecode && P.store_w16 && lane == 0) bulk_wait_all();
     if (lane == 0) trace_mark(P, 18 + d);
   } else if (warp == 4) {
     // ================== MMA issue (lane q follows producer q) ==================
@@ -518,7 +529,7 @@ __device__ __forceinline__ void local_cta(const GemmDev& P) {
   } else {
     // ===================== epilogue (warps 0-3, 128 threads) =====================
     const uint32_t e = threadIdx.x;   // TMEM lane = row within the 128-row half
-    const uint32_t nck = H * T / 16;  // 16-column chunks per accumulator (1 or 2)
+    const uint32_t nck = H * T / 16;  // 16-column chunks per accumulator (1, 2 or 4)
     const uint32_t seg_first = ub / n_kt;
     // W row-block segment of every accumulator slot, in slot (= unit) order
     if (e == 0) {
@@ -547,45 +558,52 @@ __device__ __forceinline__ void local_cta(const GemmDev& P) {
       wait_live(&acc_full[sa], 0, abort, P.status, 6, 64);
       wait_all_live(&acc_full[sa], sb - sa, 0, abort, P.status, 6, 32);
       tc_fence_after();
-      float acc[2][16];
-      for (uint32_t k = sa; k < sb;) {
-        const uint32_t nb = (nck == 1 && k + 1 < sb) ? 2u : 1u;
-        uint32_t v[2][16];
-        const uint32_t taddr = tmem_base + ((32 * warp) << 16) + k * H * T;
-        tmem_ld16(taddr, v[0]);
-        if (nb == 2 || nck == 2) tmem_ld16(taddr + 16, v[1]);
-        tmem_ld_wait();
-        if (nck == 1) {
-#pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            float x = __uint_as_float(v[0][q]);
-            if (k > sa) x = acc[0][q] + x;
-            if (nb == 2) x = x + __uint_as_float(v[1][q]);
-            acc[0][q] = x;
-          }
-        } else {
-#pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            acc[0][q] = (k > sa) ? acc[0][q] + __uint_as_float(v[0][q]) : __uint_as_float(v[0][q]);
-            acc[1][q] = (k > sa) ? acc[1][q] + __uint_as_float(v[1][q]) : __uint_as_float(v[1][q]);
-          }
-        }
-        k += nb;
-      }
       // store: Y for a segment this CTA holds whole, else split-K partials
       const uint32_t p = seg / P.n_rb, rb = seg % P.n_rb;
       const uint32_t s_lo = seg * n_kt, s_hi = s_lo + n_kt;
       const bool complete = ub <= s_lo && ue >= s_hi;
       const uint32_t pslot = (seg == seg_first) ? 0u : 1u;
       float* part = P.partials + (static_cast<uint64_t>(cta) * 2 + pslot) * H * P.T_pass * 128;
+      // the accumulators' 16-column chunks, two at a time (one pass unless a
+      // 256-row tile meets more than 16 tokens)
+      for (uint32_t c0 = 0; c0 < nck; c0 += 2) {
+        const uint32_t ncc = min(2u, nck - c0);
+        float acc[2][16];
+        for (uint32_t k = sa; k < sb;) {
+          // one chunk per accumulator: two accumulators per wait
+          const uint32_t nb = (ncc == 1 && k + 1 < sb) ? 2u : 1u;
+          uint32_t v[2][16];
+          const uint32_t taddr = tmem_base + ((32 * warp) << 16) + k * H * T + 16 * c0;
+          tmem_ld16(taddr, v[0]);
+          if (nb == 2) tmem_ld16(taddr + H * T, v[1]);
+          else if (ncc == 2) tmem_ld16(taddr + 16, v[1]);
+          tmem_ld_wait();
+          if (ncc == 1) {
 #pragma unroll
-      for (uint32_t ck = 0; ck < 2; ++ck) {
-        if (ck >= nck) break;
-        const uint32_t per_h = T / 16;
-        const uint32_t h = ck / per_h, tok0 = (ck % per_h) * 16;
-        const uint32_t n = rb * P.L.tile_n + h * 128 + e;
-        const float scale = complete ? row_scale(P, n) : 1.0f;
-        epi_emit16(P, acc[ck], complete, scale, part, p, h, tok0, n, e);
+            for (int q = 0; q < 16; ++q) {
+              float x = __uint_as_float(v[0][q]);
+              if (k > sa) x = acc[0][q] + x;
+              if (nb == 2) x = x + __uint_as_float(v[1][q]);
+              acc[0][q] = x;
+            }
+          } else {
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+              acc[0][q] = (k > sa) ? acc[0][q] + __uint_as_float(v[0][q]) : __uint_as_float(v[0][q]);
+              acc[1][q] = (k > sa) ? acc[1][q] + __uint_as_float(v[1][q]) : __uint_as_float(v[1][q]);
+            }
+          }
+          k += nb;
+        }
+#pragma unroll
+        for (uint32_t ck = 0; ck < 2; ++ck) {
+          if (ck >= ncc) break;
+          const uint32_t c = c0 + ck, per_h = T / 16;
+          const uint32_t h = c / per_h, tok0 = (c % per_h) * 16;
+          const uint32_t n = rb * P.L.tile_n + h * 128 + e;
+          const float scale = complete ? row_scale(P, n) : 1.0f;
+          epi_emit16(P, acc[ck], complete, scale, part, p, h, tok0, n, e);
+        }
       }
       if (e == 0) trace_mark(P, 60 + min(nflush, 1u));
       if (!complete) pend[npend++] = seg;

@@ -67,6 +67,10 @@ struct GemmPlan {
   uint32_t smem_bytes;
   uint32_t off_lut, off_w, off_chunk, off_x, off_bars;
   uint32_t sms;        // SMs the plan was made for
+  // large M: a fused first pass of M_first tokens (the small-M schedule,
+  // storing the decoded weights into W16), then a dense GEMM for the other
+  // M - M_first tokens; the other fields describe the first pass's launch
+  uint32_t dense, M_first;
   // workspace: [counters][partials][f16 copy of X][W16]; W16 (the weights
   // decoded or formatted to the 16-bit operand format, N x K row-major) only
   // when the call has several token passes (see launch_gemm)
@@ -174,6 +178,9 @@ constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
 // Device address of that scratch on the current device (looked up once per
 // device; see noalloc.cu).
 cudaError_t noalloc_scratch(void** ptr);
+
+// Tokens of the fused first pass of a large-M call (see GemmPlan::dense).
+constexpr uint32_t kDenseFirstTokens = 16;
 
 // Producer warps per CTA of the local schedule (gemm_local.cu).
 constexpr uint32_t kLocalProducersMax = 15;

@@ -58,9 +58,6 @@ __device__ __forceinline__ void mbar_arrive_expect_tx_s(uint32_t bar_s, uint32_t
       "r"(bytes)
       : "memory");
 }
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-  mbar_arrive_expect_tx_s(smem_u32(bar), bytes);
-}
 
 __device__ __forceinline__ bool mbar_try_wait_s(uint32_t bar_s, uint32_t parity) {
   uint32_t ok;
@@ -119,16 +116,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
-// L2 cache policies for the copies: data read once (the weight stream) is
-// evicted first, data read by many CTAs (X) last.
+// L2 cache policy for data read once (the compressed weight stream): evicted first.
 __device__ __forceinline__ uint64_t l2_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
-__device__ __forceinline__ uint64_t l2_evict_last() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
   return p;
 }
 
@@ -140,21 +131,6 @@ __device__ __forceinline__ void bulk_g2s_hint_s(uint32_t dst_s, const void* src,
       "[%0], [%1], %2, [%3], %4;" ::"r"(dst_s),
       "l"(src), "r"(bytes), "r"(bar_s), "l"(policy)
       : "memory");
-}
-
-// 1-D bulk copy global -> this CTA's shared memory, completing on `bar`.
-// src, dst 16-byte aligned; bytes a multiple of 16.  No multicast.
-__device__ __forceinline__ void bulk_g2s_s(uint32_t dst_s, const void* src, uint32_t bytes,
-                                           uint32_t bar_s) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(dst_s),
-      "l"(src), "r"(bytes), "r"(bar_s)
-      : "memory");
-}
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
-                                         uint64_t* bar) {
-  bulk_g2s_s(smem_u32(dst), src, bytes, smem_u32(bar));
 }
 
 // 2-D tiled tensor copy global -> this CTA's shared memory, completing on
@@ -189,16 +165,6 @@ __device__ __forceinline__ void tma_load_2d_s(uint32_t dst_s, const void* tmap, 
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
       "[%0], [%1, {%2, %3}], [%4];" ::"r"(dst_s),
       "l"(tmap), "r"(x), "r"(y), "r"(bar_s)
-      : "memory");
-}
-
-// The same with an L2 cache policy.
-__device__ __forceinline__ void tma_load_2d_hint_s(uint32_t dst_s, const void* tmap, int32_t x,
-                                                   int32_t y, uint32_t bar_s, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst_s),
-      "l"(tmap), "r"(x), "r"(y), "r"(bar_s), "l"(policy)
       : "memory");
 }
 
@@ -277,28 +243,8 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "r"(taddr)
       : "memory");
 }
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7])
-      : "r"(taddr)
-      : "memory");
-}
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-// Shared-memory matrix descriptor for tcgen05 (K-major operand, 32-byte
-// swizzle: 8-row x 32-byte atoms, rows 32 bytes apart, atoms `sbo` bytes apart).
-__device__ __forceinline__ uint64_t sdesc_sw32(uint32_t saddr, uint32_t sbo_bytes) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);          // bits 0-13: start address >> 4
-  d |= (uint64_t)1 << 16;                             // bits 16-29: LBO (unused for swizzled K-major)
-  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;  // bits 32-45: SBO >> 4
-  d |= (uint64_t)1 << 46;                             // bits 46-47: descriptor version 1 (sm_100)
-  d |= (uint64_t)6 << 61;                             // bits 61-63: layout = 32-byte swizzle
-  return d;
 }
 
 // Instruction descriptor, kind::f16, fp32 accumulator, both operands K-major.

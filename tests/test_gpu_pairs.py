@@ -128,7 +128,7 @@ def test_pairs_corrupt_stream_is_flagged(cuda, cases):
 
 @pytest.mark.parametrize("state_bits", [32, 64])
 @pytest.mark.parametrize("name,N,K", SMALL)
-@pytest.mark.parametrize("M", [1, 16, 17, 64, 128, 300])
+@pytest.mark.parametrize("M", [1, 16, 17, 24, 32, 64, 128, 300])
 def test_pairs_gemm_parity(cuda, oracle, cases, name, N, K, M, state_bits):
     cfg, d, lay, layer = _case(cases, name, N, K, state_bits)
     X = WL.make_x(cfg, M, K)
@@ -136,10 +136,17 @@ def test_pairs_gemm_parity(cuda, oracle, cases, name, N, K, M, state_bits):
     Yu, stu, _ = run_gemm(cfg, d, lay, layer, X, compressed=False)
     assert st == 0 and stu == 0
     assert torch.equal(Y, Yu), "ans_gemm must be bit-identical to ans_gemm_uncompressed"
-    # the per-element coding of the same weights fills the same slabs
+    # the per-element coding of the same weights fills the same slabs: the
+    # same result, bit for bit where both codings get the same schedule (on
+    # 256-row tiles at 17-32 tokens pair symbols take the small-M schedule,
+    # whose order of additions differs)
     _, _, lay1, layer1 = _case(cases, name, N, K, state_bits, dtype=ans.INT4)
     Y1, st1, _ = run_gemm(cfg, d, lay1, layer1, X, compressed=True)
-    assert st1 == 0 and torch.equal(Y, Y1)
+    assert st1 == 0
+    if lay.tile_n == 256 and 17 <= M <= 32:
+        assert rel_fro(Y.cpu().numpy(), Y1.cpu().numpy().astype(np.float64)) <= 1e-5
+    else:
+        assert torch.equal(Y, Y1)
     Yref = oracle.gemm(WL.INT4, X, M, K, d["w"], N, cfg.scale_kind, d["scales"], cfg.group_k)
     assert rel_fro(Y.cpu().numpy(), Yref) <= TOL
 
@@ -147,7 +154,8 @@ def test_pairs_gemm_parity(cuda, oracle, cases, name, N, K, M, state_bits):
 @pytest.mark.parametrize("schedule", ["local", "central"])
 @pytest.mark.parametrize("ctas,producers", [(8, 16), (3, 7)])
 @pytest.mark.parametrize("name,N,K,M", [("int4_70b", 512, 2048, 16), ("tiny_int4", 512, 512, 1),
-                                        ("int4_70b", 1024, 1024, 130)])
+                                        ("int4_70b", 1024, 1024, 130), ("int4_70b", 512, 2048, 32),
+                                        ("int4_70b", 512, 2048, 21)])
 def test_pairs_gemm_schedules_and_long_runs(cuda, oracle, cases, plan_limits, schedule, ctas,
                                             producers, name, N, K, M):
     plan_limits(schedule=schedule, max_ctas=ctas, max_producers=producers)

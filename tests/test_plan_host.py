@@ -12,7 +12,7 @@ from rans_decode_gemm_b200 import workloads as WL
 
 FIELDS = ["local", "grid", "D", "n_slots", "tmem_cols", "smem_bytes", "T", "T_pass", "n_pass",
           "NT", "n_bufs", "fmt", "ab_f16", "H", "C", "x_stages", "n_units", "n_segments",
-          "ws_lo", "ws_hi"]
+          "ws_lo", "ws_hi", "dense"]
 SMEM_MAX = 232448          # sm_100 per-block dynamic shared memory
 FMT = {"bf16": 0, "int4_bf16": 1, "int4_group": 2, "fp8": 3, "int4_pair": 4,
        "int4_pair_group": 5, "int8": 6, "fp4": 7, "fp4_pair": 8}
@@ -23,7 +23,7 @@ def _plan(lay, M, kind, decode, sms):
     fn = lib.ansdev_gemm_plan
     fn.argtypes = [C.c_void_p, C.c_uint32, C.c_uint32, C.c_int, C.c_int, C.c_void_p]
     fn.restype = C.c_int
-    out = (C.c_uint32 * 20)()
+    out = (C.c_uint32 * 21)()
     r = fn(C.addressof(lay), M, kind, decode, sms, out)
     return r, dict(zip(FIELDS, list(out)))
 
@@ -69,10 +69,16 @@ def test_plans_fit_and_cover(ans_lib, name, dtype, state_bits):
             # memory without the slot table and chunk rings (a deeper X ring),
             # which does not change the order of the additions
             layout = {"fmt"} | (set() if p["local"] else {"smem_bytes", "x_stages"})
-            # several token passes: the workspace holds the decoded weights
-            # for the dense GEMM of the later tokens (the uncompressed
-            # variant's own bf16 weights need no copy)
-            if p["n_pass"] > 1 and K % 64 == 0:
+            # more tokens than one pass: a fused first pass of 16 tokens on
+            # the small-M schedule, then the dense GEMM; the workspace holds
+            # the decoded weights (the uncompressed variant's own bf16 weights
+            # need no copy)
+            # (unless the first pass does not fit the small-M schedule, on a
+            # device of very few SMs)
+            assert p["dense"] == 0 or (M > 512 // H and K % 64 == 0)
+            if sms >= 18:
+                assert p["dense"] == (1 if M > 512 // H and K % 64 == 0 else 0)
+            if p["dense"]:
                 layout |= {"ws_lo", "ws_hi"}
                 ws, wsu = p["ws_lo"] + (p["ws_hi"] << 32), pu["ws_lo"] + (pu["ws_hi"] << 32)
                 assert ws - wsu == (N * K * 2 if dtype == WL.BF16_SPLIT else 0)
@@ -87,9 +93,16 @@ def test_plans_fit_and_cover(ans_lib, name, dtype, state_bits):
             tc = p["tmem_cols"]
             assert 32 <= tc <= 512 and tc & (tc - 1) == 0
             assert p["T_pass"] * p["n_pass"] >= M
-            if p["local"]:
+            if p["dense"]:
+                assert p["local"] == 1 and p["T"] == 16 and p["T_pass"] == 512 // H
+                assert p["n_units"] == n_tiles and p["n_segments"] == N // cfg.tile_n
+                assert p["D"] <= 15 and p["n_slots"] * H * 16 <= tc
+                assert p["ws_lo"] + (p["ws_hi"] << 32) >= 2 * N * K   # W16
+            elif p["local"]:
                 T = (M + 15) // 16 * 16
-                assert p["T"] == T and H * T <= 32 and p["n_pass"] == 1
+                pair = dtype in (WL.INT4_PAIRS, WL.FP4_PAIRS)
+                assert p["T"] == T and p["n_pass"] == 1
+                assert H * T <= 32 or (pair and T <= 32 and H * T <= 64)
                 assert 1 <= p["D"] <= 15 and 1 <= p["n_slots"] <= 32
                 assert p["n_slots"] * H * T <= tc
                 assert p["n_units"] == n_tiles and p["n_segments"] == N // cfg.tile_n

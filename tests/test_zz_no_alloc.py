@@ -49,11 +49,11 @@ def test_noalloc_matches_workspace_entry_point(cuda, name, N, K, M, state_bits):
 
 
 def test_noalloc_refuses_oversize_shape(cuda):
-    cfg, d, lay, layer = make_case("bf16_4096", 1024, 4096)
-    M = 2048                                  # needs far more than the 16 MiB scratch
+    cfg, d, lay, layer = make_case("bf16_4096", 4096, 4096)
+    M = 2048        # the decoded copy of W for the dense GEMM alone is 32 MiB
     assert ans.ans_gemm_workspace(lay, M, 0) > 16 << 20
     X = torch.zeros(M, 4096, dtype=torch.int16, device="cuda")
-    Y = torch.zeros(M, 1024, dtype=torch.float32, device="cuda")
+    Y = torch.zeros(M, 4096, dtype=torch.float32, device="cuda")
     with pytest.raises(ans.AnsError) as e:
         ans.ans_gemm_noalloc(X, M, layer.tiles, 0, None, 0, Y, status_tensor())
     assert e.value.status == 4
@@ -84,6 +84,23 @@ def test_noalloc_after_a_flagged_call_and_beside_a_refused_one(cuda):
     with pytest.raises(ans.AnsError) as e:            # no status word: refused
         ans.ans_gemm_noalloc(dX, M, layer.tiles, 0, None, 0, Y, None)
     assert e.value.status == 1
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert torch.equal(Y, Y_ref)
+
+
+def test_noalloc_large_m_within_the_scratch(cuda):
+    # a call above one token pass whose workspace (the decoded copy of W
+    # included) fits the fixed scratch runs there, same result as ans_gemm
+    cfg, d, lay, layer = make_case("bf16_4096", 1024, 4096)
+    M = 700
+    assert ans.ans_gemm_workspace(lay, M, 0) <= 16 << 20
+    X = WL.make_x(cfg, M, 4096)
+    Y_ref, st_ref, _ = run_gemm(cfg, d, lay, layer, X, compressed=True)
+    assert st_ref == 0
+    Y = torch.full((M, 1024), float("nan"), dtype=torch.float32, device="cuda")
+    st = status_tensor()
+    ans.ans_gemm_noalloc(x_dev(X), M, layer.tiles, 0, None, 0, Y, st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     assert torch.equal(Y, Y_ref)
