@@ -597,6 +597,33 @@ def dequant_bf16(torch, cfg, d, device):
     return out
 
 
+def whole16_row(args, torch, ans, name, mname, w, N, K, cfg, split_bpw, split_bound, split_dec_us,
+                st, timed_graph):
+    """bf16 coded as whole 16-bit symbols against the split stream on the same
+    layer: bits/weight, the entropy bound, and the standalone decode time."""
+    hist = ans.ans_histogram16_host(w)
+    freq = ans.ans_build_codebook16(hist, 16)
+    lay = ans.make_layout(ans.BF16_WHOLE, N, K, cfg.tile_n, cfg.tile_k, args.state_bits)
+    stream, offsets = ans.ans_encode_tiles16(w, lay, freq, 16)
+    table = ans.ans_decode_table16(freq, 16)
+    d_stream = torch.from_numpy(np.concatenate([stream, np.zeros(16, np.uint8)])).cuda()
+    d_off = torch.from_numpy(offsets.view(np.int64)).cuda()
+    d_table = torch.from_numpy(table).cuda()
+    out = torch.empty(N * K, dtype=torch.int16, device="cuda")
+    call = [lambda: ans.ans_decode_tiles16(lay, d_table, d_stream, stream.size, d_off, out, st)]
+    t = timed_graph(call, 3)
+    t = timed_graph(call, max(3, min(200, int(20000 / max(t, 1.0)))))
+    exact = bool(np.array_equal(out.cpu().numpy().view(np.uint16), w))
+    bpw = 8.0 * (stream.size + 8 * offsets.size) / (N * K)
+    return {"workload": name, "matrix": mname, "N": N, "K": K, "coding": "bf16 whole 16-bit symbols",
+            "state_bits": args.state_bits, "prob_bits": 16, "present_symbols": int((freq > 0).sum()),
+            "bits_per_weight": round(bpw, 4), "entropy_bound_bits": round(ans.ans_entropy(hist), 4),
+            "gap_bits": round(bpw - ans.ans_entropy(hist), 4), "decode_tiles16_us": round(t, 2),
+            "decode_Tsym_per_s": round(N * K / (t * 1e-6) / 1e12, 4), "bit_exact": exact,
+            "split_bits_per_weight": round(split_bpw, 4), "split_entropy_bound_bits": round(split_bound, 4),
+            "split_decode_tiles_us": round(split_dec_us, 2), "status": int(st.item())}
+
+
 def sweep(args):
     """Every workload of the pages at full size on one GPU: bits/weight against
     the entropy bound, ans_gemm at each M of the workload, the same kernel on
@@ -676,6 +703,9 @@ def sweep(args):
             t_dec = timed_graph([lambda l=l: ans.ans_decode_tiles(l.tiles, dec, st) for l in layers], 3)
             t_dec = timed_graph([lambda l=l: ans.ans_decode_tiles(l.tiles, dec, st) for l in layers],
                                 rep_for(t_dec * copies))
+            if cfg.dtype == WL.BF16_SPLIT:
+                print(json.dumps(whole16_row(args, torch, ans, name, mname, d["w"], N, K, cfg, bpw,
+                                             bound, t_dec, st, timed_graph)), flush=True)
             for M in (ms_only or cfg.Ms):
                 X = torch.from_numpy(WL.make_x(cfg, M, K).view(np.int16)).to(device)
                 Y = torch.empty(M, N, dtype=torch.float32, device=device)

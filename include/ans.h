@@ -57,6 +57,10 @@
  *                  ANS_INT4_PAIRS.
  *   ANS_INT8       int8 code bytes q in [-128, 127]; coded symbol q + 128,
  *                  i.e. the byte XOR 0x80 (A = 256).
+ *   ANS_BF16_WHOLE uint16 bf16 bits; coded symbol = the whole 16-bit pattern
+ *                  (A = 65536), probability precision up to 16 bits, the lane
+ *                  map of the one-symbol-per-element formats.  Only the
+ *                  16-bit-symbol entry points (ans_*16) take it.
  *   ANS_INT4_PAIRS the same storage as ANS_INT4, coded one symbol per packed
  *                  byte (two consecutive K elements): symbol = byte ^ 0x88,
  *                  i.e. (q_k + 8) | (q_{k+1} + 8) << 4 (A = 256), half as
@@ -115,7 +119,8 @@ typedef enum {
   ANS_INT4_PAIRS = 3,
   ANS_INT8 = 4,
   ANS_FP4_E2M1 = 5,
-  ANS_FP4_PAIRS = 6
+  ANS_FP4_PAIRS = 6,
+  ANS_BF16_WHOLE = 7  /* the 16-bit-symbol entry points only (ans_*16 below) */
 } ans_dtype;
 
 typedef enum {
@@ -181,8 +186,8 @@ ans_status ans_histogram(const void* d_w, const ans_layout* layout, uint64_t* d_
  * overwritten.  Multithreaded over rows; integer counts. */
 ans_status ans_histogram_host(const void* h_w, const ans_layout* layout, uint64_t* hist);
 
-/* Shannon entropy H = -sum p log2 p of a histogram, bits per symbol
- * (DFloat11 summary, section "实验方法").  Host. */
+/* Shannon entropy H = -sum p log2 p of a histogram of up to 65,536 bins,
+ * bits per symbol (DFloat11 summary, section "实验方法").  Host. */
 ans_status ans_entropy(const uint64_t* hist, uint32_t alphabet, double* bits_per_symbol);
 
 /* Normalises a histogram to integer frequencies summing to 2^prob_bits with
@@ -215,6 +220,46 @@ ans_status ans_encode_tiles(const void* h_w, const ans_layout* layout,
  * ("Approaching Shannon Bound", s2.2 and s4.2).  d_status: device uint32. */
 ans_status ans_decode_tiles(const ans_tiles* tiles, void* d_out, uint32_t* d_status,
                             ans_stream_t stream);
+
+/* ---- bf16 as whole 16-bit symbols ("Approaching Shannon Bound", s4.1:
+ * bf16's large symbol table makes the precision of the normalised
+ * frequencies cost more than for low-bit formats).  The stream format above
+ * with symbol = the bf16 bit pattern, 2^n slots (n <= 16; 16 is the reading
+ * used here), no raw side stream.  The codebook is a host array
+ * uint32 freq[65536] summing to 2^n.  Decode only: the fused GEMM takes the
+ * split format (ANS_BF16_SPLIT). */
+
+/* hist: uint64[65536], overwritten.  Host, multithreaded. */
+ans_status ans_histogram16_host(const uint16_t* h_w, uint64_t n_weights, uint64_t* hist);
+
+/* The normalisation of ans_build_codebook over 65,536 symbols: freq[65536]
+ * summing to 2^prob_bits (1..16), freq > 0 exactly for the present symbols.
+ * ANS_ERR_ALPHABET: more present symbols than 2^prob_bits. */
+ans_status ans_build_codebook16(const uint64_t* hist, uint32_t prob_bits, uint32_t* freq);
+
+/* Offline encoder for an ANS_BF16_WHOLE layout (either state width); the
+ * stream capacity from ans_encode_bound.  Same outputs and errors as
+ * ans_encode_tiles (no raw stream). */
+ans_status ans_encode_tiles16(const uint16_t* h_w, const ans_layout* layout, const uint32_t* freq,
+                              uint32_t prob_bits, uint8_t* h_stream, uint64_t cap,
+                              uint64_t* stream_bytes, uint64_t* h_offsets);
+
+/* The decoder's lookup table for a codebook (host image, to be copied to the
+ * device as is): *table_bytes receives its size (a multiple of 16); with
+ * h_table NULL only the size is returned.  prob_bits 12..16; at most 16,384
+ * present symbols (the table lives in shared memory), else
+ * ANS_ERR_UNSUPPORTED. */
+ans_status ans_decode_table16(const uint32_t* freq, uint32_t prob_bits, uint8_t* h_table,
+                              uint64_t cap, uint64_t* table_bytes);
+
+/* GPU decode of an ANS_BF16_WHOLE layer into its bf16 bits (uint16 N x K
+ * row-major, 16-byte aligned).  d_table: the ans_decode_table16 image on the
+ * device (16-byte aligned); d_stream / d_offsets as in ans_tiles.  Status
+ * bits as for ans_decode_tiles. */
+ans_status ans_decode_tiles16(const ans_layout* layout, const uint8_t* d_table, uint64_t table_bytes,
+                              const uint8_t* d_stream, uint64_t stream_bytes,
+                              const uint64_t* d_offsets, uint16_t* d_out, uint32_t* d_status,
+                              ans_stream_t stream);
 
 /* Bytes of device workspace ans_gemm / ans_gemm_uncompressed need for a
  * layout, M tokens and a scale kind.  The workspace must be zero-filled once

@@ -18,6 +18,7 @@ import numpy as np
 from . import build as _build
 
 INT4, BF16_SPLIT, FP8_E4M3, INT4_PAIRS, INT8, FP4_E2M1, FP4_PAIRS = 0, 1, 2, 3, 4, 5, 6
+BF16_WHOLE = 7   # bf16 as whole 16-bit symbols: the ans_*16 entry points only
 SCALE_NONE, SCALE_ROW_BF16, SCALE_ROW_F32, SCALE_GROUP_BF16 = 0, 1, 2, 3
 STATUS_CORRUPT, STATUS_TIMEOUT, STATUS_BAD_OFFSETS, STATUS_SMEM_ALIGN = 0x1, 0x2, 0x4, 0x8
 ALPHABET = {INT4: 16, BF16_SPLIT: 256, FP8_E4M3: 256, INT4_PAIRS: 256, INT8: 256, FP4_E2M1: 16,
@@ -26,7 +27,8 @@ ALPHABET = {INT4: 16, BF16_SPLIT: 256, FP8_E4M3: 256, INT4_PAIRS: 256, INT8: 256
 # every symbol include/ans.h declares
 EXPORTS = ["ans_status_string", "ans_last_error", "ans_num_tiles", "ans_layout_check",
            "ans_histogram", "ans_histogram_host", "ans_entropy", "ans_build_codebook", "ans_encode_bound",
-           "ans_encode_tiles", "ans_decode_tiles", "ans_gemm_workspace", "ans_gemm",
+           "ans_encode_tiles", "ans_decode_tiles", "ans_histogram16_host", "ans_build_codebook16",
+           "ans_encode_tiles16", "ans_decode_table16", "ans_decode_tiles16", "ans_gemm_workspace", "ans_gemm",
            "ans_gemm_noalloc", "ans_gemm_uncompressed", "ans_gemm_batched_workspace",
            "ans_gemm_batched"]
 MAX_BATCH = 8
@@ -88,6 +90,11 @@ def load():
             L.ans_encode_bound.argtypes = [P, P]
             L.ans_encode_tiles.argtypes = [P, P, P, P, u64, P, P, P]
             L.ans_decode_tiles.argtypes = [P, P, P, P]
+            L.ans_histogram16_host.argtypes = [P, u64, P]
+            L.ans_build_codebook16.argtypes = [P, u32, P]
+            L.ans_encode_tiles16.argtypes = [P, P, P, u32, P, u64, P, P]
+            L.ans_decode_table16.argtypes = [P, u32, P, u64, P]
+            L.ans_decode_tiles16.argtypes = [P, P, u64, P, u64, P, P, P, P]
             L.ans_gemm_workspace.argtypes = [P, u32, i32, P]
             L.ans_gemm.argtypes = [P, u32, P, i32, P, u32, P, P, sz, P, P]
             L.ans_gemm_noalloc.argtypes = [P, u32, P, i32, P, u32, P, P, P]
@@ -203,6 +210,57 @@ def ans_encode_tiles(h_w: np.ndarray, layout: AnsLayout, codebook: AnsCodebook):
 def ans_decode_tiles(tiles: AnsTiles, d_out, d_status, stream=None):
     _check(load().ans_decode_tiles(C.byref(tiles), _ptr(d_out), _ptr(d_status), _stream(stream)),
            "ans_decode_tiles")
+
+
+def ans_histogram16_host(h_w: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns -> uint64[65536] histogram of the whole 16-bit symbols."""
+    h_w = np.ascontiguousarray(h_w, dtype=np.uint16)
+    hist = np.zeros(65536, np.uint64)
+    _check(load().ans_histogram16_host(_ptr(h_w), h_w.size, _ptr(hist)), "ans_histogram16_host")
+    return hist
+
+
+def ans_build_codebook16(hist, prob_bits: int = 16) -> np.ndarray:
+    """uint32[65536] frequencies summing to 2^prob_bits."""
+    hist = np.ascontiguousarray(hist, dtype=np.uint64)
+    freq = np.zeros(65536, np.uint32)
+    _check(load().ans_build_codebook16(_ptr(hist), prob_bits, _ptr(freq)), "ans_build_codebook16")
+    return freq
+
+
+def ans_encode_tiles16(h_w: np.ndarray, layout: AnsLayout, freq, prob_bits: int = 16):
+    """Returns (stream uint8[], offsets uint64[n_tiles + 1])."""
+    h_w = np.ascontiguousarray(h_w, dtype=np.uint16)
+    freq = np.ascontiguousarray(freq, dtype=np.uint32)
+    cap = ans_encode_bound(layout)
+    stream = np.empty(max(cap, 16), np.uint8)
+    offsets = np.empty(ans_num_tiles(layout) + 1, np.uint64)
+    nbytes = C.c_uint64(0)
+    _check(load().ans_encode_tiles16(_ptr(h_w), C.byref(layout), _ptr(freq), prob_bits,
+                                     _ptr(stream), cap, C.byref(nbytes), _ptr(offsets)),
+           "ans_encode_tiles16")
+    return stream[:nbytes.value], offsets
+
+
+def ans_decode_table16(freq, prob_bits: int = 16) -> np.ndarray:
+    """The decoder's lookup-table image (uint8[], a multiple of 16 bytes)."""
+    freq = np.ascontiguousarray(freq, dtype=np.uint32)
+    nbytes = C.c_uint64(0)
+    L = load()
+    _check(L.ans_decode_table16(_ptr(freq), prob_bits, None, 0, C.byref(nbytes)),
+           "ans_decode_table16")
+    table = np.zeros(nbytes.value, np.uint8)
+    _check(L.ans_decode_table16(_ptr(freq), prob_bits, _ptr(table), table.size, C.byref(nbytes)),
+           "ans_decode_table16")
+    return table
+
+
+def ans_decode_tiles16(layout: AnsLayout, d_table, d_stream, stream_bytes: int, d_offsets, d_out,
+                       d_status, stream=None):
+    _check(load().ans_decode_tiles16(C.byref(layout), _ptr(d_table), d_table.numel(),
+                                     _ptr(d_stream), stream_bytes, _ptr(d_offsets), _ptr(d_out),
+                                     _ptr(d_status), _stream(stream)),
+           "ans_decode_tiles16")
 
 
 def ans_gemm_workspace(layout: AnsLayout, M: int, scale_kind: int = SCALE_NONE) -> int:

@@ -36,6 +36,29 @@ ans_status check_layout(const ans_layout* l) {
   return ANS_OK;
 }
 
+// Layout of the 16-bit-symbol entry points: dtype ANS_BF16_WHOLE.
+ans_status check_layout16(const ans_layout* l) {
+  if (!l) return ANS_ERR_ARG;
+  if (l->dtype != ANS_BF16_WHOLE) return ANS_ERR_ARG;
+  if (l->state_bits != 0 && l->state_bits != 32 && l->state_bits != 64) return ANS_ERR_ARG;
+  if (!anshost::layout_valid(l->N, l->K, l->tile_n, l->tile_k)) return ANS_ERR_SHAPE;
+  return ANS_OK;
+}
+
+// A 16-bit codebook: 65,536 frequencies summing to 2^prob_bits.
+ans_status check_freq16(const uint32_t* freq, uint32_t prob_bits) {
+  if (!freq || prob_bits < 1 || prob_bits > 16) return ANS_ERR_ARG;
+  uint64_t run = 0;
+  for (uint32_t s = 0; s < 65536; ++s) run += freq[s];
+  return run == (1ull << prob_bits) ? ANS_OK : ANS_ERR_ALPHABET;
+}
+
+// Either kind of layout: the one-byte-symbol formats, or the 16-bit-symbol
+// layout of the ans_*16 entry points.
+ans_status check_any_layout(const ans_layout* layout) {
+  return layout && layout->dtype == ANS_BF16_WHOLE ? check_layout16(layout) : check_layout(layout);
+}
+
 // Stream-format codebook: alphabet of the dtype, 12-bit precision, freq
 // summing to 4096, cdf consistent with freq.
 ans_status check_codebook(const ans_codebook* cb, uint32_t dtype) {
@@ -215,11 +238,11 @@ const char* ans_status_string(ans_status s) {
 const char* ans_last_error(void) { return g_last_error; }
 
 uint64_t ans_num_tiles(const ans_layout* layout) {
-  if (check_layout(layout) != ANS_OK) return 0;
+  if (check_any_layout(layout) != ANS_OK) return 0;
   return static_cast<uint64_t>(layout->N / layout->tile_n) * (layout->K / layout->tile_k);
 }
 
-ans_status ans_layout_check(const ans_layout* layout) { return check_layout(layout); }
+ans_status ans_layout_check(const ans_layout* layout) { return check_any_layout(layout); }
 
 ans_status ans_histogram(const void* d_w, const ans_layout* layout, uint64_t* d_hist,
                          ans_stream_t stream) {
@@ -248,7 +271,7 @@ ans_status ans_histogram_host(const void* h_w, const ans_layout* layout, uint64_
 }
 
 ans_status ans_entropy(const uint64_t* hist, uint32_t alphabet, double* bits_per_symbol) {
-  if (!hist || !bits_per_symbol || alphabet == 0 || alphabet > 256) return ANS_ERR_ARG;
+  if (!hist || !bits_per_symbol || alphabet == 0 || alphabet > 65536) return ANS_ERR_ARG;
   *bits_per_symbol = anshost::entropy_bits(hist, alphabet);
   return ANS_OK;
 }
@@ -274,7 +297,7 @@ ans_status ans_build_codebook(const uint64_t* hist, uint32_t alphabet, uint32_t 
 }
 
 ans_status ans_encode_bound(const ans_layout* layout, uint64_t* max_stream_bytes) {
-  ans_status st = check_layout(layout);
+  ans_status st = check_any_layout(layout);
   if (st != ANS_OK) return st;
   if (!max_stream_bytes) return ANS_ERR_ARG;
   *max_stream_bytes = anshost::encode_bound(layout->N, layout->K, layout->tile_n, layout->tile_k,
@@ -323,6 +346,87 @@ ans_status ans_decode_tiles(const ans_tiles* tiles, void* d_out, uint32_t* d_sta
   cudaError_t e = ansdev::launch_decode_tiles(L, d_out, d_status,
                                               reinterpret_cast<cudaStream_t>(stream), sms);
   if (e != cudaSuccess) return cuda_fail(e, "ans_decode_tiles");
+  return ANS_OK;
+}
+
+ans_status ans_histogram16_host(const uint16_t* h_w, uint64_t n_weights, uint64_t* hist) {
+  if (!h_w || !hist) return ANS_ERR_ARG;
+  anshost::histogram16(h_w, n_weights, hist);
+  return ANS_OK;
+}
+
+ans_status ans_build_codebook16(const uint64_t* hist, uint32_t prob_bits, uint32_t* freq) {
+  if (!hist || !freq) return ANS_ERR_ARG;
+  const int r = anshost::normalize16(hist, prob_bits, freq);
+  if (r == 3) return ANS_ERR_ALPHABET;
+  return r == 0 ? ANS_OK : ANS_ERR_ARG;
+}
+
+ans_status ans_encode_tiles16(const uint16_t* h_w, const ans_layout* layout, const uint32_t* freq,
+                              uint32_t prob_bits, uint8_t* h_stream, uint64_t cap,
+                              uint64_t* stream_bytes, uint64_t* h_offsets) {
+  ans_status st = check_layout16(layout);
+  if (st != ANS_OK) return st;
+  if (!h_w || !h_stream || !stream_bytes || !h_offsets) return ANS_ERR_ARG;
+  st = check_freq16(freq, prob_bits);
+  if (st != ANS_OK) return st;
+  const int r = anshost::encode16(h_w, layout->N, layout->K, layout->tile_n, layout->tile_k, freq,
+                                  prob_bits, h_stream, cap, stream_bytes, h_offsets,
+                                  layout->state_bits == 64);
+  if (r == 3) return ANS_ERR_ALPHABET;
+  if (r == 4) return ANS_ERR_BUFFER_TOO_SMALL;
+  return r == 0 ? ANS_OK : ANS_ERR_ARG;
+}
+
+ans_status ans_decode_table16(const uint32_t* freq, uint32_t prob_bits, uint8_t* h_table,
+                              uint64_t cap, uint64_t* table_bytes) {
+  if (!table_bytes) return ANS_ERR_ARG;
+  ans_status st = check_freq16(freq, prob_bits);
+  if (st != ANS_OK) return st;
+  if (prob_bits < 12) return ANS_ERR_UNSUPPORTED;
+  uint64_t present = 0;
+  for (uint32_t s = 0; s < 65536; ++s) present += freq[s] ? 1 : 0;
+  if (present > ansdev::kMaxPresent16) {
+    std::snprintf(g_last_error, sizeof(g_last_error),
+                  "ans_decode_table16: %llu present symbols, the decoder holds at most %u",
+                  static_cast<unsigned long long>(present), ansdev::kMaxPresent16);
+    return ANS_ERR_UNSUPPORTED;
+  }
+  *table_bytes = anshost::table16_bytes(freq);
+  if (!h_table) return ANS_OK;
+  const int r = anshost::table16(freq, prob_bits, h_table, cap);
+  if (r == 4) return ANS_ERR_BUFFER_TOO_SMALL;
+  return r == 0 ? ANS_OK : ANS_ERR_ALPHABET;
+}
+
+ans_status ans_decode_tiles16(const ans_layout* layout, const uint8_t* d_table, uint64_t table_bytes,
+                              const uint8_t* d_stream, uint64_t stream_bytes,
+                              const uint64_t* d_offsets, uint16_t* d_out, uint32_t* d_status,
+                              ans_stream_t stream) {
+  ans_status st = check_layout16(layout);
+  if (st != ANS_OK) return st;
+  if (!d_table || !d_stream || !d_offsets || !d_out || !d_status) return ANS_ERR_ARG;
+  if (table_bytes == 0 || table_bytes % 16 != 0 ||
+      table_bytes > 8 + 2 * 4096 + 6ull * ansdev::kMaxPresent16 + 15)
+    return ANS_ERR_ARG;
+  if (reinterpret_cast<uintptr_t>(d_out) % 16 != 0 ||
+      reinterpret_cast<uintptr_t>(d_table) % 16 != 0 ||
+      reinterpret_cast<uintptr_t>(d_stream) % 16 != 0 ||
+      reinterpret_cast<uintptr_t>(d_offsets) % 8 != 0)
+    return ANS_ERR_ARG;
+  int sms = 0;
+  st = device_info(&sms);
+  if (st != ANS_OK) return st;
+  ansdev::LayerDev L;
+  fill_layer_plain(layout, &L);
+  L.stream = d_stream;
+  L.stream_bytes = stream_bytes;
+  L.offsets = d_offsets;
+  L.wide = layout->state_bits == 64 ? 1u : 0u;
+  cudaError_t e = ansdev::launch_decode_tiles16(L, d_table, static_cast<uint32_t>(table_bytes),
+                                                d_out, d_status,
+                                                reinterpret_cast<cudaStream_t>(stream), sms);
+  if (e != cudaSuccess) return cuda_fail(e, "ans_decode_tiles16");
   return ANS_OK;
 }
 
@@ -417,6 +521,7 @@ int ansdev_set_wait_budget(long long cycles) {
   if (e == cudaSuccess) e = ansdev::set_live_wait_budget_local(c);
   if (e == cudaSuccess) e = ansdev::set_live_wait_budget_decode(c);
   if (e == cudaSuccess) e = ansdev::set_live_wait_budget_dense(c);
+  if (e == cudaSuccess) e = ansdev::set_live_wait_budget_decode16(c);
   return e == cudaSuccess ? ANS_OK : cuda_fail(e, "ansdev_set_wait_budget");
 }
 

@@ -1245,6 +1245,8 @@ cudaError_t launch_gemm(const GemmPlan& plan, const LayerDev& L, bool decode, co
   D.n_tiles = D.m_blocks * (L.N / 128);
   D.b_box_rows = std::min(M_rest, 256u);
   D.idesc = idesc_f16(plan.ab_f16 ? 0u : 1u, 128, 256);
+  const uint32_t tail = M_rest - (D.m_blocks - 1) * 256;
+  D.idesc_tail = idesc_f16(plan.ab_f16 ? 0u : 1u, 128, (tail + 15) / 16 * 16);
   return launch_dense_gemm(D, plan.sms, stream);
 }
 

@@ -130,6 +130,8 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
         if (acc >= 2 && !wait_live(&acc_empty[b], ((acc >> 1) + 1) & 1u, abort, P.status, 21)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + b * kDenseBN;
+        // the last token block is narrower when M is not a multiple of 256
+        const uint32_t idesc = (t % P.m_blocks == P.m_blocks - 1) ? P.idesc_tail : P.idesc;
         for (uint32_t kb = 0; kb < n_kb; ++kb, ++it) {
           const uint32_t s = it % kDenseStages;
           if (!wait_live(&full[s], (it / kDenseStages) & 1u, abort, P.status, 22)) {
@@ -140,7 +142,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
           const uint32_t a16 = (smem_s + s * kDenseStageBytes) >> 4, b16 = a16 + (kDenseABytes >> 4);
 #pragma unroll
           for (uint32_t j = 0; j < kDenseBK / 16; ++j)
-            umma_f16(d_tmem, dhi | (a16 + 2 * j), dhi | (b16 + 2 * j), P.idesc, (kb | j) != 0 ? 1u : 0u);
+            umma_f16(d_tmem, dhi | (a16 + 2 * j), dhi | (b16 + 2 * j), idesc, (kb | j) != 0 ? 1u : 0u);
           umma_commit(&empty[s]);
         }
         if (live) umma_commit(&acc_full[b]);

@@ -138,7 +138,8 @@ struct DenseDev {
   uint32_t M, N, K;
   uint32_t m_blocks, n_tiles;
   uint32_t b_box_rows;  // rows of X a box brings (256, or M when smaller)
-  uint32_t idesc;
+  uint32_t idesc;       // MMA 128 x 256 x 16
+  uint32_t idesc_tail;  // the last token block: N = its tokens rounded up to 16
 };
 cudaError_t launch_dense_gemm(const DenseDev& P, uint32_t sms, cudaStream_t stream);
 
@@ -171,6 +172,7 @@ cudaError_t set_live_wait_budget_gemm(long long cycles);
 cudaError_t set_live_wait_budget_local(long long cycles);
 cudaError_t set_live_wait_budget_decode(long long cycles);
 cudaError_t set_live_wait_budget_dense(long long cycles);
+cudaError_t set_live_wait_budget_decode16(long long cycles);
 cudaError_t launch_wait_probe(uint32_t* status, cudaStream_t stream);
 
 // Scratch capacity of the allocation-free entry point (16 MiB per device).
@@ -178,6 +180,12 @@ constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
 // Device address of that scratch on the current device (looked up once per
 // device; see noalloc.cu).
 cudaError_t noalloc_scratch(void** ptr);
+
+// bf16 as whole 16-bit symbols (decode16.cu): the decoder's table image
+// (built on the host) holds at most this many present symbols.
+constexpr uint32_t kMaxPresent16 = 16384;
+cudaError_t launch_decode_tiles16(const LayerDev& L, const uint8_t* table, uint32_t table_bytes,
+                                  uint16_t* out, uint32_t* status, cudaStream_t stream, int num_sms);
 
 // Tokens of the fused first pass of a large-M call (see GemmPlan::dense).
 constexpr uint32_t kDenseFirstTokens = 16;

@@ -19,4 +19,17 @@ int encode(uint32_t dtype, const void* w, uint32_t N, uint32_t K, uint32_t tile_
            uint32_t tile_k, const uint32_t* freq, uint8_t* stream, uint64_t cap,
            uint64_t* stream_bytes, uint64_t* offsets, uint8_t* raw, bool wide);
 
+// bf16 as whole 16-bit symbols (alphabet 65,536; codec16_host.cpp).
+void histogram16(const uint16_t* w, uint64_t n_weights, uint64_t* hist);
+// 0 ok, 1 bad argument, 3 too many present symbols.
+int normalize16(const uint64_t* hist, uint32_t prob_bits, uint32_t* freq);
+// 0 ok, 1 bad argument, 3 symbol with zero frequency or frequencies not
+// summing to 2^prob_bits, 4 capacity too small (size still reported).
+int encode16(const uint16_t* w, uint32_t N, uint32_t K, uint32_t tile_n, uint32_t tile_k,
+             const uint32_t* freq, uint32_t prob_bits, uint8_t* stream, uint64_t cap,
+             uint64_t* stream_bytes, uint64_t* offsets, bool wide);
+// Size and contents of the decoder's lookup-table image.
+uint64_t table16_bytes(const uint32_t* freq);
+int table16(const uint32_t* freq, uint32_t prob_bits, uint8_t* out, uint64_t bytes);
+
 }  // namespace anshost

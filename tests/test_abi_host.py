@@ -1,6 +1,7 @@
 """CPU tests of the C-ABI library: it loads, exports every entry point that
 include/ans.h declares, and its host codec (histogram, entropy, codebook,
 tile encoder) agrees with the CPU oracle byte for byte."""
+import ctypes as C
 import os
 import re
 
@@ -37,8 +38,13 @@ def test_status_strings_and_layout_checks(ans_lib):
     assert ans.ans_layout_check(ans.make_layout(0, 500, 512, 128, 32)) == 2    # N % tile_n
     assert ans.ans_layout_check(ans.make_layout(0, 512, 520, 128, 40)) == 2    # tile_k % 16
     assert ans.ans_layout_check(ans.make_layout(0, 512, 512, 64, 32)) == 2     # tile_n
-    assert ans.ans_layout_check(ans.make_layout(7, 512, 512, 128, 32)) == 1    # dtype
-    assert ans.ans_layout_check(ans.make_layout(7, 512, 512, 128, 32)) == 1    # dtype
+    assert ans.ans_layout_check(ans.make_layout(8, 512, 512, 128, 32)) == 1    # dtype
+    assert ans.ans_layout_check(ans.make_layout(7, 512, 512, 128, 32)) == 0    # 16-bit symbols
+    assert ans.ans_num_tiles(ans.make_layout(7, 512, 512, 128, 32)) == 64
+    # the one-byte-symbol entry points refuse the 16-bit-symbol layout
+    whole = ans.make_layout(7, 512, 512, 128, 32)
+    ws = C.c_size_t(0)
+    assert ans.load().ans_gemm_workspace(C.byref(whole), 16, 0, C.byref(ws)) == 1
     assert ans.ans_layout_check(ans.make_layout(6, 512, 512, 128, 32)) == 0    # fp4 pairs
     assert ans.ans_layout_check(ans.make_layout(5, 512, 512, 128, 32)) == 0    # fp4
     assert ans.ans_layout_check(ans.make_layout(4, 512, 512, 128, 32)) == 0    # int8
@@ -211,7 +217,7 @@ def test_dtype_constants_agree_with_the_header():
     assert enum["ANS_INT4"] == ans.INT4 and enum["ANS_BF16_SPLIT"] == ans.BF16_SPLIT
     assert enum["ANS_FP8_E4M3"] == ans.FP8_E4M3 and enum["ANS_INT4_PAIRS"] == ans.INT4_PAIRS
     assert enum["ANS_INT8"] == ans.INT8 and enum["ANS_FP4_E2M1"] == ans.FP4_E2M1
-    assert enum["ANS_FP4_PAIRS"] == ans.FP4_PAIRS
+    assert enum["ANS_FP4_PAIRS"] == ans.FP4_PAIRS and enum["ANS_BF16_WHOLE"] == ans.BF16_WHOLE
     assert enum["ANS_SCALE_GROUP_BF16"] == ans.SCALE_GROUP_BF16
     assert enum["ANS_SCALE_ROW_F32"] == ans.SCALE_ROW_F32
     flags = dict((k, int(v, 16)) for k, v in re.findall(r"#define\s+(ANS_STATUS_[A-Z_]+)\s+0x([0-9a-fA-F]+)u", text))
