@@ -51,6 +51,7 @@ NOMINAL = {0: 0.5, 1: 2.0, 2: 1.0, 3: 0.5, 4: 1.0, 5: 0.5, 6: 0.5}
 # sources of the kernel the bench times at M = 16 (the local schedule); the
 # committed DRAM-traffic summary is only used while they are unchanged
 KERNEL_SOURCES = ["rans_decode_gemm_b200/csrc/cuda/gemm_local.cu",
+                  "rans_decode_gemm_b200/csrc/cuda/kernels.h",
                   "rans_decode_gemm_b200/csrc/cuda/gemm_common.cuh",
                   "rans_decode_gemm_b200/csrc/cuda/rans_core.cuh",
                   "rans_decode_gemm_b200/csrc/cuda/ptx.cuh",
