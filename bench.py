@@ -761,10 +761,12 @@ def sweep(args):
 
 def sweep_batched(args, torch, ans, WL, device, stream, st, timed_graph):
     """The Llama MLP's gate and up projections (same layout, same X): two
-    ans_gemm calls against one ans_gemm_batched call, weights from HBM."""
+    ans_gemm calls against one ans_gemm_batched call; then the whole MLP
+    (gate, up and the 4096 x 14336 down projection, mixed shapes): three calls
+    against one batched launch.  Weights from HBM."""
     cfg = WL.CONFIGS["llama8b_mlp"]
     mats = []
-    for mi in (0, 1):
+    for mi in (0, 1, 2):
         d = WL.make_weights(cfg, mi)
         lay = ans.make_layout(cfg.dtype, d["N"], d["K"], cfg.tile_n, cfg.tile_k, args.state_bits)
         l0 = ans.CompressedLayer.from_weights(d["w"], lay, device=device)
@@ -789,6 +791,34 @@ def sweep_batched(args, torch, ans, WL, device, stream, st, timed_graph):
                "state_bits": args.state_bits, "two_ans_gemm_us": round(t2, 2),
                "ans_gemm_batched_us": round(t1, 2), "speedup": round(t2 / t1, 3),
                "effective_weight_GBps": round(2 * lay.N * lay.K * 2 / (t1 * 1e-6) / 1e9, 1),
+               "status": int(st.item())}
+        print(json.dumps(rec), flush=True)
+    # the whole MLP in one launch: gate and up read X (M x 4096), down reads an
+    # activation of M x 14336 (synthetic here)
+    lay_d = mats[2][0]
+    n_w = sum(m[0].N * m[0].K for m in mats)
+    for M in (1, 16):
+        X = torch.from_numpy(WL.make_x(cfg, M, lay.K).view(np.int16)).to(device)
+        Hx = torch.from_numpy(WL.make_x(cfg, M, lay_d.K).view(np.int16)).to(device)
+        Ys = [torch.empty(M, m[0].N, dtype=torch.float32, device=device) for m in mats]
+        ins = [X, X, Hx]
+        wss = []
+        for j in range(3):
+            nb = ans.ans_gemm_workspace(mats[j][0], M, 0)
+            wss.append((torch.zeros(max(nb, 256), dtype=torch.uint8, device=device), nb))
+        jobs = [[(ins[j], mats[j][1][c].tiles, None, Ys[j]) for j in range(3)] for c in range(4)]
+        nb3 = ans.ans_gemm_batched_workspace(jobs[0], M, 0)
+        ws3 = torch.zeros(max(nb3, 256), dtype=torch.uint8, device=device)
+        three = [lambda c=c, j=j: ans.ans_gemm(ins[j], M, mats[j][1][c].tiles, 0, None, 0, Ys[j],
+                                               wss[j][0], wss[j][1], st)
+                 for c in range(4) for j in range(3)]
+        one = [lambda c=c: ans.ans_gemm_batched(jobs[c], M, 0, 0, ws3, nb3, st) for c in range(4)]
+        t3 = timed_graph(three, 20) * 3   # per MLP
+        t1 = timed_graph(one, 20)
+        rec = {"workload": "llama8b_mlp", "matrix": "gate+up+down", "weights": n_w, "M": M,
+               "state_bits": args.state_bits, "three_ans_gemm_us": round(t3, 2),
+               "ans_gemm_batched_us": round(t1, 2), "speedup": round(t3 / t1, 3),
+               "effective_weight_GBps": round(n_w * 2 / (t1 * 1e-6) / 1e9, 1),
                "status": int(st.item())}
         print(json.dumps(rec), flush=True)
 
