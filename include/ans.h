@@ -325,10 +325,9 @@ ans_status ans_gemm_noalloc(const uint16_t* d_X, uint32_t M, const ans_tiles* W,
 
 /* The same kernel with the decoder warps replaced by a copy of the original
  * (uncompressed) weights d_W (format of layout->dtype, row-major N x K).
- * Above one token pass the codes are formatted into the workspace's 16-bit
- * copy for the dense GEMM, as ans_gemm's decoded ones are.  bf16 weights are
- * read in place.  Bit-exact reference for ans_gemm and the uncompressed
- * baseline. */
+ * Above one token pass the weights are formatted into the workspace's 16-bit
+ * copy for the dense GEMM, as ans_gemm's decoded ones are.  Bit-exact
+ * reference for ans_gemm and the uncompressed baseline. */
 ans_status ans_gemm_uncompressed(const uint16_t* d_X, uint32_t M, const void* d_W,
                                  const ans_layout* layout, ans_scale_kind scale_kind,
                                  const void* d_scales, uint32_t group_k, float* d_Y, void* d_ws,

@@ -170,18 +170,22 @@ __device__ __forceinline__ void copy_bytes_fmt(uint32_t lo, uint32_t hi, uint32_
   else fmt_fp8_f16(e, o);
 }
 
-// Uncompressed weights (N x K codes) into the 16-bit operand format, N x K
-// row-major (the same values the producers write into the slabs): thread i
-// formats the eight elements 8 i .. 8 i + 7.
+// Uncompressed weights (N x K codes) into W16, the slab images of the 16-bit
+// operand format (see GemmDev::w16; the same values and layout the producers
+// write into their slabs): thread i formats the eight elements 8 i .. 8 i + 7
+// of row-major W and stores them as one 16-byte piece of their slab.
 template <uint32_t kFmt>
 __global__ void format_w16_kernel(const void* w, const void* scales, uint32_t K, uint32_t group_k,
-                                  uint32_t n_groups_k, uint16_t* w16, uint64_t n8) {
+                                  uint32_t n_groups_k, uint8_t* w16, uint64_t n8) {
   griddep_wait();
   griddep_launch_dependents();
   for (uint64_t i = blockIdx.x * static_cast<uint64_t>(blockDim.x) + threadIdx.x; i < n8;
        i += static_cast<uint64_t>(gridDim.x) * blockDim.x) {
     uint32_t o[4];
-    if constexpr (kFmt == kFmtFp8F16 || kFmt == kFmtInt8F16) {
+    if constexpr (kFmt == kFmtBf16Split) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(w) + i);
+      o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+    } else if constexpr (kFmt == kFmtFp8F16 || kFmt == kFmtInt8F16) {
       const uint2 v = __ldg(reinterpret_cast<const uint2*>(w) + i);
       copy_bytes_fmt<kFmt>(v.x, v.y, o);
     } else {
@@ -196,7 +200,15 @@ __global__ void format_w16_kernel(const void* w, const void* scales, uint32_t K,
       }
       copy_nibbles_fmt<kFmt>(v, gs, o);
     }
-    reinterpret_cast<uint4*>(w16)[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    // row r, columns 8 c8 .. 8 c8 + 7 -> slab (r / 128, c8 / 2), row r % 128,
+    // 16-byte chunk c8 % 2 under the 32-byte swizzle
+    const uint64_t e0 = i * 8;
+    const uint64_t r = e0 / K;
+    const uint32_t col = static_cast<uint32_t>(e0 - r * K);
+    const uint32_t rr = static_cast<uint32_t>(r & 127), c = (col >> 3) & 1u;
+    const uint64_t slab = (r >> 7) * (K >> 4) + (col >> 4);
+    const uint32_t off = rr * 32 + ((c << 4) ^ (((rr >> 2) & 1u) << 4));
+    *reinterpret_cast<uint4*>(w16 + slab * kSlabBytes + off) = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 
@@ -428,7 +440,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
           uint4 cp[8];
           if constexpr (!kDecode) copy_loads<kFmt>(P, n0, k0, h, s, lane, cp);
           if (sc >= 2) wait_live(&B.w_empty[2 * d + slot], ((sc >> 1) + 1) & 1u, abort, P.status, 1, 64);
-          if (kDecode && P.store_w16) {
+          if (kDecode && P.w16 != nullptr) {
             // the store of the slot's previous slab has read it
             if (lane == 0) bulk_wait_read<1>();
             __syncwarp();
@@ -496,9 +508,10 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&B.w_full[2 * d + slot]);
           // first token pass of a large-M call: the slab also goes to W16
-          if (kDecode && P.store_w16 && lane == 0)
-            tma_store_2d_s(&P.tmap_w, static_cast<int32_t>(k0 + 16 * s),
-                           static_cast<int32_t>(n0 + 128 * h), slab_s);
+          if (kDecode && P.w16 != nullptr && lane == 0)
+            bulk_s2g_s(P.w16 + ((static_cast<uint64_t>((n0 >> 7) + h) * (L.K >> 4)) + (k0 >> 4) + s) *
+                                   kSlabBytes,
+                       slab_s, kSlabBytes);
           if (lane == 0 && sc == 0) trace_mark(P, 2 + d);
           ++sc;
         }
@@ -507,7 +520,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         }
       }
       if (kDecode) pipe_drain(pipe, P.status);
-      if (kDecode && P.store_w16 && lane == 0) bulk_wait_all();
+      if (kDecode && P.w16 != nullptr && lane == 0) bulk_wait_all();
     }
     if (lane == 0) trace_mark(P, 18 + d);
   } else if (warp == 4) {
@@ -822,9 +835,8 @@ bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool dec
     p.T_pass = T_pass;
     p.n_pass = (M + T_pass - 1) / T_pass;
     p.ws_x16_bytes = p.ab_f16 ? static_cast<size_t>(M) * L.K * 2 : 0;
-    // W16: decoded by the first pass, or the uncompressed codes formatted
-    // (bf16 weights are used as they are)
-    p.ws_w16_bytes = (decode || p.fmt != kFmtBf16Split) ? static_cast<size_t>(L.N) * L.K * 2 : 0;
+    // W16: decoded by the first pass, or the uncompressed weights formatted
+    p.ws_w16_bytes = static_cast<size_t>(L.N) * L.K * 2;
     p.ws_bytes = p.ws_counters_bytes + (p.ws_partials_bytes + 255) / 256 * 256 +
                  (p.ws_x16_bytes + 255) / 256 * 256 + p.ws_w16_bytes;
     *plan = p;
@@ -1091,13 +1103,7 @@ static cudaError_t launch_single(const GemmPlan& plan, const LayerDev& L, bool d
                                  const void* scales, uint32_t scale_kind, uint32_t group_k, float* Y,
                                  void* ws, uint16_t* w16, uint32_t* status, cudaStream_t stream) {
   GemmDev P = make_gemm_dev(plan, L, w_plain, X, scales, scale_kind, group_k, Y, ws, status);
-  if (decode && w16) {
-    // the decoded slabs' destination: W16 as 16 x 128 boxes, the slab layout
-    cudaError_t e = encode_tmap(&P.tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT16, w16, L.K, L.N,
-                                static_cast<uint64_t>(L.K) * 2, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B);
-    if (e != cudaSuccess) return e;
-    P.store_w16 = 1;
-  }
+  if (decode && w16) P.w16 = reinterpret_cast<uint8_t*>(w16);  // the decoded slabs' images
   if (!plan.local) {
     // X for the MMA as a tensor map: the caller's bf16 X, or its f16 copy
     const void* xsrc = X;
@@ -1165,11 +1171,13 @@ static cudaError_t launch_single(const GemmPlan& plan, const LayerDev& L, bool d
 }
 
 static cudaError_t format_w16(uint32_t fmt, const void* w, const void* scales, const LayerDev& L,
-                              uint32_t group_k, uint16_t* w16, cudaStream_t stream) {
+                              uint32_t group_k, uint8_t* w16, cudaStream_t stream) {
   const uint64_t n8 = static_cast<uint64_t>(L.N) * L.K / 8;
   const uint32_t ngk = group_k ? L.K / group_k : 0;
   const dim3 g(stream_blocks(n8)), b(256);
   switch (fmt) {
+    case kFmtBf16Split:
+      return launch_pdl(format_w16_kernel<kFmtBf16Split>, g, b, 0, stream, w, scales, L.K, group_k, ngk, w16, n8);
     case kFmtInt4Bf16:
       return launch_pdl(format_w16_kernel<kFmtInt4Bf16>, g, b, 0, stream, w, scales, L.K, group_k, ngk, w16, n8);
     case kFmtInt4F16Group:
@@ -1211,23 +1219,17 @@ cudaError_t launch_gemm(const GemmPlan& plan, const LayerDev& L, bool decode, co
   e = launch_single(first, L, decode, w_plain, X, plan.ab_f16 ? x16 : nullptr, scales, scale_kind,
                     group_k, Y, ws, decode ? w16 : nullptr, status, stream);
   if (e != cudaSuccess) return e;
-  const void* wop = w16;
   if (!decode) {
-    if (plan.fmt == kFmtBf16Split) {
-      wop = w_plain;
-    } else {
-      e = format_w16(plan.fmt, w_plain, scales, L, group_k, w16, stream);
-      if (e != cudaSuccess) return e;
-    }
+    e = format_w16(plan.fmt, w_plain, scales, L, group_k, reinterpret_cast<uint8_t*>(w16), stream);
+    if (e != cudaSuccess) return e;
   }
   const uint32_t M_rest = plan.M - plan.M_first;
   const void* xr = plan.ab_f16 ? static_cast<const void*>(x16 + static_cast<uint64_t>(plan.M_first) * L.K * 2)
                                : static_cast<const void*>(X + static_cast<uint64_t>(plan.M_first) * L.K);
   DenseDev D;
   std::memset(&D, 0, sizeof(D));
-  e = encode_tmap(&D.tmap_a, CU_TENSOR_MAP_DATA_TYPE_UINT16, wop, L.K, L.N,
-                  static_cast<uint64_t>(L.K) * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (e != cudaSuccess) return e;
+  D.w16 = reinterpret_cast<const uint8_t*>(w16);
+  D.k_slabs = L.K / 16;
   // a box of at most M_rest rows; the MMA's token columns past it hold stale
   // shared memory and are never stored
   e = encode_tmap(&D.tmap_b, CU_TENSOR_MAP_DATA_TYPE_UINT16, xr, L.K, M_rest,

@@ -13,10 +13,11 @@
 //   * Output tile 128 W rows x 256 tokens (swap-AB: A = W, B = X), full K per
 //     tile (no split-K), fp32 accumulators in TMEM, two accumulator sets so
 //     that the epilogue of one tile overlaps the MMAs of the next.
-//   * K stages of 64 columns, both operands brought by TMA as 128-byte
-//     swizzled K-major boxes (A 128 x 64, B 256 x 64: 48 KB a stage, 4
-//     stages); the MMA thread issues the stage's four K = 16 MMAs back to back
-//     and releases the stage with one commit.
+//   * K stages of 64 columns (48 KB a stage, 4 stages).  A is four consecutive
+//     W16 slab images (128 rows x 16 columns, 32-byte swizzle), contiguous in
+//     W16, so one 16 KB bulk copy brings them.  B is a TMA box of X, 256 x 64,
+//     128-byte swizzle.  The MMA thread issues the stage's four K = 16 MMAs
+//     back to back and releases the stage with one commit.
 //   * Warp roles: 0 TMA producer, 1 MMA issue (and TMEM owner), 2-5
 //     epilogue (warp w reads TMEM lanes 32 (w % 4) .. + 31).
 //   * Persistent CTAs take tiles t = blockIdx.x + i * gridDim.x, W row block
@@ -42,11 +43,6 @@ constexpr uint32_t kDenseBBytes = kDenseBN * kDenseBK * 2;  // 32 KB
 constexpr uint32_t kDenseStageBytes = kDenseABytes + kDenseBBytes;
 constexpr uint32_t kDenseThreads = 6 * 32;
 constexpr uint32_t kDenseSmem = kDenseStages * kDenseStageBytes + 1024;  // + alignment slack
-
-__device__ __forceinline__ void tma_load_2d_plain(uint32_t dst_s, const void* tmap, int32_t x, int32_t y,
-                                                  uint32_t bar_s) {
-  tma_load_2d_s(dst_s, tmap, x, y, bar_s);
-}
 
 __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __grid_constant__ DenseDev P) {
   extern __shared__ __align__(1024) uint8_t dsmem_raw[];
@@ -78,7 +74,6 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
     tmem_alloc(&tmem_slot, 512);
     tmem_relinquish();
   } else if (warp == 0 && lane == 0) {
-    prefetch_tmap(&P.tmap_a);
     prefetch_tmap(&P.tmap_b);
   }
   tc_fence_before();
@@ -104,10 +99,10 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
           const uint32_t bar = smem_u32(&full[s]);
           const uint32_t a_s = smem_s + s * kDenseStageBytes, b_s = a_s + kDenseABytes;
           mbar_arrive_expect_tx_s(bar, kDenseABytes + P.b_box_rows * kDenseBK * 2);
-          tma_load_2d_plain(a_s, &P.tmap_a, static_cast<int32_t>(kb * kDenseBK),
-                            static_cast<int32_t>(nb * kDenseBM), bar);
-          tma_load_2d_plain(b_s, &P.tmap_b, static_cast<int32_t>(kb * kDenseBK),
-                            static_cast<int32_t>(mb * kDenseBN), bar);
+          bulk_g2s_s(a_s, P.w16 + (static_cast<uint64_t>(nb) * P.k_slabs + 4 * kb) * kSlabBytes,
+                     kDenseABytes, bar);
+          tma_load_2d_s(b_s, &P.tmap_b, static_cast<int32_t>(kb * kDenseBK),
+                        static_cast<int32_t>(mb * kDenseBN), bar);
         }
       }
       // loads still in flight (only after an abort) land before exit
@@ -119,10 +114,12 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
   } else if (warp == 1) {
     // ======================= MMA issue =======================
     if (lane == 0) {
-      // descriptor fields: LBO (unused with swizzle) 16 B, SBO 1024 B (8 rows
-      // of 128 bytes), version 1, 128-byte swizzle; the K = 16 slice j of a
-      // stage starts 32 j bytes into each swizzled row
-      const uint64_t dhi = (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
+      // descriptor fields.  A: LBO 16 B, SBO 256 B (8 rows of 32 bytes),
+      // version 1, 32-byte swizzle; slab j of a stage is the K = 16 slice j.
+      // B: SBO 1024 B (8 rows of 128 bytes), 128-byte swizzle; the K = 16
+      // slice j starts 32 j bytes into each swizzled row.
+      const uint64_t da = (1ull << 16) | (16ull << 32) | (1ull << 46) | (6ull << 61);
+      const uint64_t db = (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
       uint32_t it = 0, acc = 0;
       bool live = true;
       for (uint32_t t = blockIdx.x; t < P.n_tiles && live; t += gridDim.x, ++acc) {
@@ -142,7 +139,8 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
           const uint32_t a16 = (smem_s + s * kDenseStageBytes) >> 4, b16 = a16 + (kDenseABytes >> 4);
 #pragma unroll
           for (uint32_t j = 0; j < kDenseBK / 16; ++j)
-            umma_f16(d_tmem, dhi | (a16 + 2 * j), dhi | (b16 + 2 * j), idesc, (kb | j) != 0 ? 1u : 0u);
+            umma_f16(d_tmem, da | (a16 + j * (kSlabBytes >> 4)), db | (b16 + 2 * j), idesc,
+                     (kb | j) != 0 ? 1u : 0u);
           umma_commit(&empty[s]);
         }
         if (live) umma_commit(&acc_full[b]);

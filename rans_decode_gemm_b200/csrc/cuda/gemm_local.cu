@@ -299,7 +299,7 @@ __device__ __forceinline__ void local_cta(const GemmDev& P) {
             auto store_prev = [&](uint32_t gg) {
               if (gg == 1 && nw >= 2) {
                 wait_live(&w_empty[2 * d + slot], ((nw >> 1) + 1) & 1u, abort, P.status, 1);
-                if (kDecode && P.store_w16) {
+                if (kDecode && P.w16 != nullptr) {
                   // the W16 store of the slot's previous slab has read it
                   if (lane == 0) bulk_wait_read<1>();
                   __syncwarp();
@@ -410,9 +410,10 @@ __device__ __forceinline__ void local_cta(const GemmDev& P) {
             __syncwarp();
             if (lane == 0) mbar_arrive(&w_full[2 * d + slot]);
             // first pass of a large-M call: the slab also goes to W16
-            if (kDecode && P.store_w16 && lane == 0)
-              tma_store_2d_s(&P.tmap_w, static_cast<int32_t>(k0 + 16 * s),
-                             static_cast<int32_t>(n0 + 128 * h), w_s);
+            if (kDecode && P.w16 != nullptr && lane == 0)
+              bulk_s2g_s(P.w16 + ((static_cast<uint64_t>((n0 >> 7) + h) * (L.K >> 4)) + (k0 >> 4) + s) *
+                                     kSlabBytes,
+                         w_s, kSlabBytes);
             ++nw;
           }
         };
@@ -426,7 +427,7 @@ __device__ __forceinline__ void local_cta(const GemmDev& P) {
       }
     }
     if (kDecode) rp_drain(pipe, P.status);
-    if (kDecode && P.store_w16 && lane == 0) bulk_wait_all();
+    if (kDecode && P.w16 != nullptr && lane == 0) bulk_wait_all();
     if (lane == 0) trace_mark(P, 18 + d);
   } else if (warp == 4) {
     // ================== MMA issue (lane q follows producer q) ==================

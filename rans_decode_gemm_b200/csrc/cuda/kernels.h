@@ -118,18 +118,21 @@ struct GemmDev {
   CUtensorMap tmap_x;
   CUtensorMap tmap_w;
   // first token pass of a large-M call (decode variant): every decoded slab
-  // is also stored, through tmap_w, into W16 (N x K row-major, the operand
-  // format) for the dense kernel that takes the remaining tokens
-  uint32_t store_w16;
+  // is also stored into W16 for the dense kernel that takes the remaining
+  // tokens, or null.  W16 holds the weights in the MMA operand format as 4 KB
+  // slab images (128 rows x 16 columns, 32-byte swizzle, the shared-memory
+  // layout): the image of rows 128 b .. + 127, columns 16 j .. + 15 at byte
+  // (b * K / 16 + j) * 4096.
+  uint8_t* w16;
 };
 
 // Dense GEMM on 16-bit weights that are already in the MMA operand format
 // (gemm_dense.cu): Y[m][n] = s_n * sum_k X[m][k] W[n][k] for m < M, fp32 Y
-// (M x N row-major).  W (N x K) and X (M x K) are 16-bit row-major and given
-// as 2-D tensor maps with 64 x 128 (W) and 64 x 256 (X) boxes, 128-byte
+// (M x N row-major).  W is W16 (slab images, see GemmDev::w16); X (M x K,
+// 16-bit row-major) is a 2-D tensor map with 64 x 256 boxes, 128-byte
 // swizzle; tiles of 128 W rows x 256 tokens, W-row-block major.
 struct DenseDev {
-  CUtensorMap tmap_a;   // W
+  const uint8_t* w16;   // W
   CUtensorMap tmap_b;   // X
   float* Y;
   const void* scales;   // scale_kind 1: bf16 per row, 2: fp32 per row, else none
@@ -137,6 +140,7 @@ struct DenseDev {
   uint32_t scale_kind;
   uint32_t M, N, K;
   uint32_t m_blocks, n_tiles;
+  uint32_t k_slabs;     // K / 16: W16 slab images per 128-row block
   uint32_t b_box_rows;  // rows of X a box brings (256, or M when smaller)
   uint32_t idesc;       // MMA 128 x 256 x 16
   uint32_t idesc_tail;  // the last token block: N = its tokens rounded up to 16

@@ -139,15 +139,23 @@ __device__ __forceinline__ void bulk_g2s_hint_s(uint32_t dst_s, const void* src,
 // element size must be a multiple of 16 bytes; dst_s aligned to 128 bytes
 // (256 with the 32-byte swizzle).  Rows past the tensor's extent land as
 // zeros.
-// TMA store of one 2-D box from this CTA's shared memory (laid out as the
-// tensor map's box, swizzle included) to the tensor at (x, y), committed as
-// one bulk group of the calling thread.  x, y >= 0; x * element size a
-// multiple of 16 bytes.
-__device__ __forceinline__ void tma_store_2d_s(const void* tmap, int32_t x, int32_t y, uint32_t src_s) {
-  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(tmap),
-               "r"(x), "r"(y), "r"(src_s)
+// Bulk copy of `bytes` (a multiple of 16; both addresses 16-byte aligned)
+// from this CTA's shared memory to global memory, committed as one bulk group
+// of the calling thread.
+__device__ __forceinline__ void bulk_s2g_s(void* dst, uint32_t src_s, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src_s),
+               "r"(bytes)
                : "memory");
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// 1-D bulk copy global -> this CTA's shared memory, completing on mbarrier bar_s.
+__device__ __forceinline__ void bulk_g2s_s(uint32_t dst_s, const void* src, uint32_t bytes,
+                                           uint32_t bar_s) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst_s),
+      "l"(src), "r"(bytes), "r"(bar_s)
+      : "memory");
 }
 // Wait until at most N of the calling thread's bulk groups still read shared memory.
 template <int N>
