@@ -628,7 +628,9 @@ ans_status batch_plan(const ans_gemm_job* jobs, uint32_t n_jobs, uint32_t M,
     if (!ansdev::make_gemm_plan(L, M, scale_kind, true, static_cast<int>(G[j]), &share[j]))
       return ANS_ERR_UNSUPPORTED;
     if (!ansdev::make_gemm_plan(L, M, scale_kind, true, sms, &full[j])) return ANS_ERR_UNSUPPORTED;
-    if (!share[j].local || share[j].fmt != share[0].fmt) *one_launch = false;
+    // one launch only when every job is a single pass of the small-M schedule
+    // on its share (a large-M plan's fields describe its first pass alone)
+    if (!share[j].local || share[j].dense || share[j].fmt != share[0].fmt) *one_launch = false;
     const size_t a = share[j].ws_bytes > full[j].ws_bytes ? share[j].ws_bytes : full[j].ws_bytes;
     ws_off[j + 1] = ws_off[j] + ((a + 255) / 256) * 256;
   }

@@ -988,7 +988,7 @@ bool make_gemm_plan(const LayerDev& L, uint32_t M, uint32_t scale_kind, bool dec
   return true;
 }
 
-// ---- tensor maps (2-D, tiled, no multicast), encoded through the driver
+// ---- tensor maps (2-D, tiled, one destination CTA), encoded through the driver
 // entry point the runtime hands out (no link-time dependence on libcuda)
 static cudaError_t encode_tmap(CUtensorMap* map, CUtensorMapDataType type, const void* base,
                                uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_inner,
@@ -1265,7 +1265,7 @@ cudaError_t launch_gemm_batched(const GemmPlan* plans, uint32_t n, const LayerDe
   GemmPlan shape = plans[0];  // the launch: the largest producer count and shared memory
   uint32_t cta = 0;
   for (uint32_t j = 0; j < n; ++j) {
-    if (!plans[j].local || plans[j].fmt != plans[0].fmt) return cudaErrorInvalidValue;
+    if (!plans[j].local || plans[j].dense || plans[j].fmt != plans[0].fmt) return cudaErrorInvalidValue;
     B.job[j] = make_gemm_dev(plans[j], *Ls[j], nullptr, Xs[j], scales[j], scale_kind, group_k,
                              Ys[j], static_cast<uint8_t*>(ws) + ws_off[j], status);
     B.job[j].cta0 = cta;

@@ -98,9 +98,12 @@ def test_batched_one_launch_parity(cuda, oracle, plan_limits, name, N, K, state_
 
 
 @pytest.mark.parametrize("name,N,K,M", [("bf16_4096", 512, 1024, 64), ("int4_70b", 512, 1024, 48),
-                                        ("fp8_405b", 256, 1024, 300)])
+                                        ("fp8_405b", 256, 1024, 300), ("bf16_4096", 512, 1024, 600),
+                                        ("int4_70b", 512, 1024, 300)])
 def test_batched_consecutive_launches_parity(cuda, oracle, name, N, K, M):
-    # shapes past the small-M schedule run one full-GPU launch per layer
+    # shapes past the small-M schedule run one full-GPU launch per layer --
+    # above one token pass (the last two cases) the fused first pass and the
+    # dense GEMM of each layer
     layers = _layers(name, N, K, 3)
     Xs, Ys, st = _run_batched(layers, M)
     assert st == 0
