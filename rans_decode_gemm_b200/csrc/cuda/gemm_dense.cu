@@ -1,11 +1,11 @@
 // gemm_dense.cu -- dense tcgen05 GEMM on 16-bit weights that are already
 // decoded: Y[m][n] = s_n * sum_k X[m][k] W[n][k], fp32 out.
 //
-// Used for the tokens past the first pass of a large-M call: the fused
-// kernel decodes every tile once while it computes the first token pass and
-// stores the decoded slabs (row-major, 16-bit) into the workspace; the
+// Used for the tokens past the first pass of a large-M call.  The fused
+// kernel decodes every tile once while it computes the first 16 tokens, and
+// stores each decoded slab's image (16-bit, W16) into the workspace.  The
 // remaining tokens meet those weights here, at tensor-core rate, instead of
-// decoding the layer again per pass.  The uncompressed variant runs the same
+// decoding the layer again per token pass.  The uncompressed variant runs the same
 // kernel on the same operands (its weights formatted the same way), so the
 // two variants stay bit-identical.
 //
@@ -18,7 +18,7 @@
 //     W16, so one 16 KB bulk copy brings them.  B is a TMA box of X, 256 x 64,
 //     128-byte swizzle.  The MMA thread issues the stage's four K = 16 MMAs
 //     back to back and releases the stage with one commit.
-//   * Warp roles: 0 TMA producer, 1 MMA issue (and TMEM owner), 2-5
+//   * Warp roles: 0 loads (bulk copy of A, TMA box of B), 1 MMA issue (and TMEM owner), 2-5
 //     epilogue (warp w reads TMEM lanes 32 (w % 4) .. + 31).
 //   * Persistent CTAs take tiles t = blockIdx.x + i * gridDim.x, W row block
 //     major (t / m_blocks), so the CTAs running at one time share W rows
@@ -86,7 +86,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_gemm_kernel(const __gr
   griddep_launch_dependents();
 
   if (warp == 0) {
-    // ======================= TMA producer =======================
+    // ======================= loads =======================
     if (lane == 0) {
       uint32_t it = 0;
       for (uint32_t t = blockIdx.x; t < P.n_tiles && !*abort; t += gridDim.x) {
