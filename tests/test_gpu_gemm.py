@@ -298,12 +298,13 @@ def test_gemm_full_size_large_m_sampled(cuda, oracle, name, M, dtype):
 @pytest.mark.parametrize("name,N,K,M", [("bf16_4096", 512, 1024, 513), ("bf16_4096", 512, 1024, 812),
                                         ("fp8_405b", 256, 2048, 1100), ("int4_70b", 512, 1024, 257),
                                         ("int8_8b", 384, 1024, 700), ("fp4_8b", 384, 1024, 530),
-                                        ("tiny_int4", 128, 96, 600)])
+                                        ("tiny_int4", 512, 512, 600), ("tiny_int4", 128, 96, 600)])
 def test_gemm_large_m_dense_path_edges(cuda, oracle, cases, name, N, K, M):
     # more tokens than one pass: the first pass fused, the rest through the
     # dense GEMM on the decoded weights -- a single token left over (one row
     # of X in the dense kernel's box), two token blocks with a ragged second,
-    # every coded format; K not a multiple of 64 keeps every pass fused
+    # every coded format and scale kind (row bf16: the tiny int4 layer); K not
+    # a multiple of 64 keeps every pass fused
     cfg, d, lay, layer = _case(cases, name, N, K)
     X = WL.make_x(cfg, M, K)
     Y, st, _ = run_gemm(cfg, d, lay, layer, X, compressed=True)
