@@ -237,7 +237,8 @@ ans_status ans_histogram16_host(const uint16_t* h_w, uint64_t n_weights, uint64_
  * ANS_ERR_ALPHABET: more present symbols than 2^prob_bits. */
 ans_status ans_build_codebook16(const uint64_t* hist, uint32_t prob_bits, uint32_t* freq);
 
-/* Offline encoder for an ANS_BF16_WHOLE layout (either state width); the
+/* Offline encoder for an ANS_BF16_WHOLE layout (either state width; the
+ * wide-state format only at prob_bits 12 or 16, else ANS_ERR_ARG); the
  * stream capacity from ans_encode_bound.  Same outputs and errors as
  * ans_encode_tiles (no raw stream). */
 ans_status ans_encode_tiles16(const uint16_t* h_w, const ans_layout* layout, const uint32_t* freq,

@@ -204,6 +204,8 @@ int encode16(const uint16_t* w, uint32_t N, uint32_t K, uint32_t tile_n, uint32_
              const uint32_t* freq, uint32_t prob_bits, uint8_t* stream, uint64_t cap,
              uint64_t* stream_bytes, uint64_t* offsets, bool wide) {
   if (prob_bits < 1 || prob_bits > 16) return 1;
+  // the wide-state format is defined at 12 and 16 bits of precision only
+  if (wide && prob_bits != 12 && prob_bits != 16) return 1;
   std::vector<uint32_t> cdf(kA16 + 1, 0);
   uint64_t run = 0;
   for (uint32_t s = 0; s < kA16; ++s) {

@@ -43,20 +43,20 @@ def test_codebook16_errors(ans_lib):
     assert e.value.status == 3
 
 
-@pytest.mark.parametrize("state_bits", [32, 64])
-def test_encode16_bytes_match_oracle(ans_lib, oracle, state_bits):
+@pytest.mark.parametrize("state_bits,prob_bits", [(32, 16), (64, 16), (32, 14), (64, 12)])
+def test_encode16_bytes_match_oracle(ans_lib, oracle, state_bits, prob_bits):
     N, K = 256, 512
     w = _weights(N, K)
-    freq = ans.ans_build_codebook16(ans.ans_histogram16_host(w), 16)
+    freq = ans.ans_build_codebook16(ans.ans_histogram16_host(w), prob_bits)
     lay = ans.make_layout(ans.BF16_WHOLE, N, K, 128, 64, state_bits)
-    stream, offsets = ans.ans_encode_tiles16(w, lay, freq, 16)
+    stream, offsets = ans.ans_encode_tiles16(w, lay, freq, prob_bits)
     st, ref_stream, ref_offsets, _ = oracle.encode(ans.BF16_WHOLE, w, N, K, 128, 64, freq,
-                                                   prob_bits=16, state_bits=state_bits)
+                                                   prob_bits=prob_bits, state_bits=state_bits)
     assert st == 0
     assert np.array_equal(offsets, ref_offsets)
     assert np.array_equal(stream, ref_stream)
     st, back = oracle.decode(ans.BF16_WHOLE, stream, offsets, None, N, K, 128, 64, freq,
-                             prob_bits=16, state_bits=state_bits)
+                             prob_bits=prob_bits, state_bits=state_bits)
     assert st == 0 and np.array_equal(back, w)
 
 
@@ -80,6 +80,10 @@ def test_encode16_rejects_bad_arguments(ans_lib):
     split = ans.make_layout(ans.BF16_SPLIT, 256, 256, 128, 64, 64)
     with pytest.raises(ans.AnsError) as e:
         ans.ans_encode_tiles16(w, split, freq, 16)    # not a 16-bit-symbol layout
+    assert e.value.status == 1
+    f14 = ans.ans_build_codebook16(ans.ans_histogram16_host(w), 14)
+    with pytest.raises(ans.AnsError) as e:
+        ans.ans_encode_tiles16(w, lay, f14, 14)       # wide states: 12 or 16 bits only
     assert e.value.status == 1
 
 

@@ -14,11 +14,11 @@ from _gpu_util import status_tensor, to_dev
 pytestmark = pytest.mark.gpu
 
 
-def _coded(w, N, K, tile_n, tile_k, state_bits):
-    freq = ans.ans_build_codebook16(ans.ans_histogram16_host(w), 16)
+def _coded(w, N, K, tile_n, tile_k, state_bits, prob_bits=16):
+    freq = ans.ans_build_codebook16(ans.ans_histogram16_host(w), prob_bits)
     lay = ans.make_layout(ans.BF16_WHOLE, N, K, tile_n, tile_k, state_bits)
-    stream, offsets = ans.ans_encode_tiles16(w, lay, freq, 16)
-    table = ans.ans_decode_table16(freq, 16)
+    stream, offsets = ans.ans_encode_tiles16(w, lay, freq, prob_bits)
+    table = ans.ans_decode_table16(freq, prob_bits)
     return lay, freq, stream, offsets, table
 
 
@@ -44,6 +44,17 @@ def test_decode16_bit_exact(cuda, name, N, K, tile_n, tile_k, state_bits):
     out, st = _decode(lay, stream, offsets, table)
     assert st == 0
     assert np.array_equal(out, w)
+
+
+@pytest.mark.parametrize("state_bits,prob_bits", [(32, 14), (32, 13), (64, 12)])
+def test_decode16_lower_precision(cuda, state_bits, prob_bits):
+    # 2^14, 2^13 or 2^12 slots: buckets of 4, 2 or 1 slot in the first-level
+    # table (the wide-state format is defined at 12 and 16 bits)
+    w = WL.make_weights(WL.CONFIGS["bf16_4096"], 0, N=512, K=1024)["w"]
+    lay, freq, stream, offsets, table = _coded(w, 512, 1024, 128, 64, state_bits, prob_bits)
+    assert int(freq.sum()) == 1 << prob_bits
+    out, st = _decode(lay, stream, offsets, table)
+    assert st == 0 and np.array_equal(out, w)
 
 
 @pytest.mark.parametrize("state_bits", [32, 64])
