@@ -27,20 +27,29 @@
  *   columns [kt*tile_k, +tile_k).  Lane l's j-th symbol is element
  *     row = l + 32*(4h + i), col = 16s + 8c + kk   where  g = j/8, kk = j%8,
  *     i = g%4, c = (g/4)%2, h = (g/8)%(tile_n/128), s = g/(8*(tile_n/128)).
- *   Tile bytes: 32 little-endian u32 final encoder states (lane order), then
- *   the u16 words in decoder order (step by step; within a step, lanes that
- *   need a word take the next one in increasing lane order), then zero bytes
- *   to a 16-byte boundary.  offsets[t] = byte start of tile t (16-byte
- *   aligned), offsets[n_tiles] = total stream bytes.
+ *   Tile bytes: the final-state block, then the u16 words in decoder order
+ *   (step by step; within a step, lanes that need a word take the next one in
+ *   increasing lane order), then zero bytes to a 16-byte boundary.
+ *   offsets[t] = byte start of tile t (16-byte aligned), offsets[n_tiles] =
+ *   total stream bytes.
+ *   Final-state block (a variable-length flush): a length table, one
+ *   little-endian u32 whose bit l is set when lane l's state takes 4 bytes
+ *   (else 3; states are >= 2^16), then the 32 final encoder states in lane
+ *   order, each little-endian in its byte count, then zero bytes up to an
+ *   even offset.  A single-symbol tile is 112 bytes: a zero table, 32 states
+ *   2^16 (00 00 01) and 12 bytes of padding.
  *   Wide-state variant (ans_layout.state_bits = 64): 64-bit lane states in
  *   [2^32, 2^64), 32-bit renormalisation words, and the renormalisation test
  *   made once per pair of symbols (steps 2i, 2i+1) instead of after every
  *   symbol: the decoder decodes both symbols of a pair, then a lane with
  *   x < 2^32 takes one word (x = x << 32 | w).  The encoder pushes a word
- *   before coding a pair (a, b) if x >= 2^40 * f_a * f_b.  Tile bytes: 32
- *   little-endian u64 states, then the u32 words in decoder order, then zero
- *   padding.  About 23 more bits per lane and tile than the default format,
- *   in exchange for half as many renormalisation steps.
+ *   before coding a pair (a, b) if x >= 2^40 * f_a * f_b.  Tile bytes: the
+ *   final-state block with states of 5 to 8 bytes (states are >= 2^32) and a
+ *   length table of two little-endian u32 bit planes (lane l takes 5 + bit l
+ *   of the first + 2 * bit l of the second bytes), zero bytes up to a multiple
+ *   of 4, then the u32 words in decoder order, then zero padding.  About 16
+ *   more bits per lane and tile than the default format (the initial state
+ *   2^32 instead of 2^16), in exchange for half as many renormalisation steps.
  *   bf16 raw side stream: tile_n*tile_k bytes per tile at t*tile_n*tile_k,
  *   the raw byte (sign << 7 | 7-bit mantissa) of lane l's j-th symbol at
  *   (j/8)*256 + l*8 + j%8.

@@ -33,9 +33,13 @@
 //   32-bit state x kept in [L, L*b) with L = 2^16 and renormalisation base
 //   b = 2^16 (16-bit words), 32 lanes per tile, one state per lane, all lanes
 //   sharing one interleaved word stream consumed in increasing lane order.
-// Byte format of one tile: 32 little-endian u32 final encoder states (lane
-// order), then the u16 words in decoder consumption order, then zero bytes up
-// to a 16-byte boundary.
+// Byte format of one tile (the final-state flush is left open by the pages;
+// the reading taken is a variable-length one): a length table, then each
+// lane's final encoder state in lane order, little-endian, in the fewest whole
+// bytes that hold it (x >= L = 2^16, so 3 or 4 bytes), then zero bytes up to a
+// word boundary (2 bytes), then the u16 words in decoder consumption order,
+// then zero bytes up to a 16-byte boundary.  The length table is one
+// little-endian u32 whose bit l is set when lane l's state takes 4 bytes.
 //
 // Wide-state variant (state_bits = 64; the same pages leave the state width
 // open): 64-bit state x in [L, L*b) with L = 2^32 and b = 2^32 (32-bit words),
@@ -45,8 +49,10 @@
 // 32-bit word always restores x >= L.  Encoder side, for a pair (a, b) coded
 // in reverse (b first, then a): the state must lie in
 // [(L >> 2n) f_a f_b, (L >> 2n) b f_a f_b) = [2^8 f_a f_b, 2^40 f_a f_b), so
-// one word is pushed first if x >= 2^40 f_a f_b.  Tile bytes: 32 little-endian
-// u64 final states, then the u32 words in decoder order, then zero padding.
+// one word is pushed first if x >= 2^40 f_a f_b.  Tile bytes as above with
+// states of 5 to 8 bytes (x >= 2^32), a length table of two little-endian u32
+// bit planes (lane l takes 5 + bit l of the first + 2 x bit l of the second
+// bytes), word boundary and words of 4 bytes.
 //
 // fp4 (dtype 5; [SB] s2.1 lists fp4 among the seven formats measured): e2m1
 // codes stored like int4 (two per byte, element k even in the low nibble),
@@ -289,6 +295,55 @@ struct Layout {
   uint64_t tile_weights() const { return (uint64_t)tile_n * tile_k; }
 };
 
+// ---- Final-state flush --------------------------------------------------------
+// Byte count of a final state: the fewest whole bytes that hold x (x >= L, so
+// at least 3 for 32-bit states and 5 for 64-bit ones).
+uint32_t flush_bytes(uint64_t x) {
+  uint32_t n = 0;
+  while (x != 0) { ++n; x >>= 8; }
+  return n;
+}
+
+// Appends the length table, the 32 final states and the zero bytes up to the
+// word boundary to an empty `out`.
+void put_final_states(const uint64_t* x, bool wide, std::vector<uint8_t>* out) {
+  const uint32_t least = wide ? 5 : 3, planes = wide ? 2 : 1, word = wide ? 4 : 2;
+  uint32_t plane[2] = {0, 0};
+  for (uint32_t l = 0; l < kLanes; ++l) {
+    const uint32_t extra = flush_bytes(x[l]) - least;  // 0..1 or 0..3
+    plane[0] |= (extra & 1u) << l;
+    plane[1] |= (extra >> 1) << l;
+  }
+  for (uint32_t p = 0; p < planes; ++p)
+    for (int b = 0; b < 4; ++b) out->push_back((uint8_t)(plane[p] >> (8 * b)));
+  for (uint32_t l = 0; l < kLanes; ++l)
+    for (uint32_t b = 0; b < flush_bytes(x[l]); ++b) out->push_back((uint8_t)(x[l] >> (8 * b)));
+  while (out->size() % word != 0) out->push_back(0);
+}
+
+// Reads the length table and the final states of a tile of `len` bytes.
+// Returns the offset of the first word, or 0 when the table points past the
+// tile or the word-boundary bytes are not zero.
+uint64_t get_final_states(const uint8_t* tile, uint64_t len, bool wide, uint64_t* x) {
+  const uint32_t least = wide ? 5 : 3, planes = wide ? 2 : 1, word = wide ? 4 : 2;
+  if (len < 4 * planes) return 0;
+  uint32_t plane[2] = {0, 0};
+  for (uint32_t p = 0; p < planes; ++p)
+    for (int b = 0; b < 4; ++b) plane[p] |= (uint32_t)tile[4 * p + b] << (8 * b);
+  uint64_t pos = 4 * planes;
+  for (uint32_t l = 0; l < kLanes; ++l) {
+    const uint32_t n = least + ((plane[0] >> l) & 1u) + 2 * ((plane[1] >> l) & 1u);
+    if (pos + n > len) return 0;
+    uint64_t v = 0;
+    for (uint32_t b = 0; b < n; ++b) v |= (uint64_t)tile[pos + b] << (8 * b);
+    x[l] = v;
+    pos += n;
+  }
+  for (; pos % word != 0; ++pos)
+    if (pos >= len || tile[pos] != 0) return 0;
+  return pos;
+}
+
 // Encode one tile into `out` (states, words, padding).  Returns OK or
 // ERR_ALPHABET when a symbol has no frequency in the codebook.
 int encode_tile(const Layout& lay, const void* w, const Codebook& cb, uint64_t t,
@@ -331,9 +386,7 @@ int encode_tile(const Layout& lay, const void* w, const Codebook& cb, uint64_t t
     }
   }
   out->clear();
-  const int state_bytes = wide ? 8 : 4;
-  for (uint32_t l = 0; l < kLanes; ++l)
-    for (int b = 0; b < state_bytes; ++b) out->push_back((uint8_t)((x[l] >> (8 * b)) & 0xFF));
+  put_final_states(x, wide, out);
   for (size_t q = pushed.size(); q-- > 0;) {
     out->push_back((uint8_t)(pushed[q] & 0xFF));
     out->push_back((uint8_t)(pushed[q] >> 8));
@@ -623,8 +676,8 @@ int oracle_rans64_decode_message(uint64_t state, const uint32_t* words, int n_wo
   return OK;
 }
 
-// Worst-case stream size: every symbol may push one word, plus states and
-// padding per tile.
+// Worst-case stream size: every symbol may push one word, plus the length
+// table, full-width states, the word boundary and padding per tile.
 // (Wide variant: 8-byte states and at most one 4-byte word per pair of
 // symbols, so the same 2 bytes per symbol.)
 uint64_t oracle_encode_bound(uint32_t N, uint32_t K, uint32_t tile_n, uint32_t tile_k,
@@ -633,7 +686,8 @@ uint64_t oracle_encode_bound(uint32_t N, uint32_t K, uint32_t tile_n, uint32_t t
   if (state_bits != 32 && state_bits != 64) return 0;
   uint64_t S = (uint64_t)tile_n * tile_k;
   uint64_t n_tiles = (uint64_t)(N / tile_n) * (K / tile_k);
-  return n_tiles * ((uint64_t)(state_bits / 8) * kLanes + 2 * S + 16);
+  const uint64_t table = state_bits == 64 ? 8 : 4;
+  return n_tiles * (table + (uint64_t)(state_bits / 8) * kLanes + 4 + 2 * S + 16);
 }
 
 // ---- Layer encode ([SB s3.1]): tiles, one shared codebook, offset index -----
@@ -692,7 +746,7 @@ int oracle_decode(int dtype, const uint8_t* stream, uint64_t stream_bytes,
   Layout lay{dtype, N, K, tile_n, tile_k, state_bits};
   const bool wide = state_bits == 64;
   const uint64_t L = wide ? kLWide : kL;
-  const uint32_t state_bytes = wide ? 8 : 4, word_bytes = wide ? 4 : 2;
+  const uint32_t word_bytes = wide ? 4 : 2;
   const uint64_t T = lay.n_tiles();
   if (tile_end > T) tile_end = T;
   if (tile_begin > tile_end) return ERR_ARG;
@@ -703,20 +757,17 @@ int oracle_decode(int dtype, const uint8_t* stream, uint64_t stream_bytes,
   parallel_for(tile_begin, tile_end, threads, [&](uint64_t t) {
     int& result = status[t - tile_begin];
     uint64_t a = offsets[t], b = offsets[t + 1];
-    if (b < a || b > stream_bytes || b - a < state_bytes * kLanes || a % 16 != 0) {
+    if (b < a || b > stream_bytes || a % 16 != 0) {
       result = ERR_CORRUPT;
       return;
     }
     const uint8_t* tile = stream + a;
     const uint64_t len = b - a;
     uint64_t x[kLanes];
-    for (uint32_t l = 0; l < kLanes; ++l) {
-      uint64_t v = 0;
-      for (uint32_t q = 0; q < state_bytes; ++q) v |= (uint64_t)tile[state_bytes * l + q] << (8 * q);
-      x[l] = v;
+    uint64_t cursor = get_final_states(tile, len, wide, x);
+    if (cursor == 0) { result = ERR_CORRUPT; return; }
+    for (uint32_t l = 0; l < kLanes; ++l)
       if (x[l] < L) { result = ERR_CORRUPT; return; }
-    }
-    uint64_t cursor = (uint64_t)state_bytes * kLanes;
     const uint64_t n0 = (t / kt_count) * tile_n, k0 = (t % kt_count) * tile_k;
     for (uint32_t j = 0; j < steps; ++j) {
       for (uint32_t l = 0; l < kLanes; ++l) {

@@ -210,17 +210,35 @@ __device__ __forceinline__ void lut_fill(uint32_t* lut, const uint32_t* cdf_s, u
   }
 }
 
-// Byte extent of tile t, validated against the format's rules.
-// Bytes of a tile's 32 lane states: u32 or (wide-state variant) u64 each.
-__device__ __forceinline__ uint32_t state_bytes(const LayerDev& L) { return L.wide ? 8u : 4u; }
+// A tile opens with its final-state block: a table of the lanes' state byte
+// counts (one u32 bit plane; two for the wide-state variant, whose counts are
+// 5 + plane0 bit + 2 x plane1 bit), the 32 lane states in lane order, each
+// little-endian in the fewest whole bytes that hold it (3..4, or 5..8), and
+// zero bytes up to the word boundary.  Its least size (every state at L) and
+// its greatest (every state at full width, before the word boundary):
+__device__ __forceinline__ uint32_t flush_min_bytes(const LayerDev& L) {
+  return L.wide ? 8u + 5u * kLanes : 4u + 3u * kLanes;
+}
+__device__ __forceinline__ uint32_t flush_max_bytes(const LayerDev& L) {
+  return L.wide ? 8u + 8u * kLanes : 4u + 4u * kLanes;
+}
+// Greatest size of a tile: block, word boundary, at most 2 bytes of words a
+// symbol, padding.
+__device__ __forceinline__ uint64_t tile_max_bytes(const LayerDev& L) {
+  return flush_max_bytes(L) + 4ull + 2ull * L.tile_n * L.tile_k + 16ull;
+}
+// A tile of a single-symbol codebook is its block with every state at L.
+__device__ __forceinline__ uint32_t single_tile_bytes(const LayerDev& L) {
+  return (flush_min_bytes(L) + 15u) & ~15u;
+}
 
+// Byte extent of tile t, validated against the format's rules.
 __device__ __forceinline__ bool tile_extent(const LayerDev& L, uint32_t t, uint64_t* start,
                                             uint32_t* bytes) {
   uint64_t a = __ldg(reinterpret_cast<const unsigned long long*>(L.offsets) + t);
   uint64_t b = __ldg(reinterpret_cast<const unsigned long long*>(L.offsets) + t + 1);
-  uint64_t max_bytes = state_bytes(L) * kLanes + 2ull * L.tile_n * L.tile_k + 16ull;
-  bool ok = (a % 16 == 0) && (b % 16 == 0) && b >= a + state_bytes(L) * kLanes && b <= L.stream_bytes &&
-            (b - a) <= max_bytes;
+  bool ok = (a % 16 == 0) && (b % 16 == 0) && b >= a + flush_min_bytes(L) && b <= L.stream_bytes &&
+            (b - a) <= tile_max_bytes(L);
   *start = a;
   *bytes = ok ? static_cast<uint32_t>(b - a) : 0u;
   return ok;
@@ -333,25 +351,40 @@ struct TileCursor {
   uint32_t bytes;  // tile bytes (padded)
 };
 
-// Lane states at ring position pos (the state bytes must be resident): the
-// lane's u32, or its two u32 halves for the wide-state variant.  Each load
-// wraps on its own.  Returns the position after the states.
+// Lane states from the final-state block at ring position pos (a tile start,
+// 16-byte aligned; the block must be resident).  Every lane reads the table,
+// finds its byte count and, by popcounts of the table below its bit, its
+// offset, then reads its bytes one by one; each load wraps on its own.
+// Returns the position of the first word.
 __device__ __forceinline__ uint32_t load_states(const LayerDev& L, uint32_t ring_s, uint32_t pos,
                                                 uint32_t lane, TileCursor& tc) {
-  const uint32_t sb = state_bytes(L);
-  uint32_t lo, hi = 0;
-  asm volatile("ld.shared.u32 %0, [%1];"
-               : "=r"(lo)
-               : "r"(((pos + sb * lane) & (kRingBytes - 1)) + ring_s)
-               : "memory");
+  uint32_t p0, p1 = 0;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(p0) : "r"((pos & (kRingBytes - 1)) + ring_s) : "memory");
   if (L.wide)
     asm volatile("ld.shared.u32 %0, [%1];"
-                 : "=r"(hi)
-                 : "r"(((pos + sb * lane + 4) & (kRingBytes - 1)) + ring_s)
+                 : "=r"(p1)
+                 : "r"(((pos + 4) & (kRingBytes - 1)) + ring_s)
                  : "memory");
-  tc.x = lo;
-  tc.xw = (static_cast<uint64_t>(hi) << 32) | lo;
-  return pos + sb * kLanes;
+  const uint32_t least = L.wide ? 5u : 3u, table = L.wide ? 8u : 4u, word = L.wide ? 4u : 2u;
+  const uint32_t below = (1u << lane) - 1u;
+  const uint32_t n = least + ((p0 >> lane) & 1u) + 2u * ((p1 >> lane) & 1u);
+  const uint32_t at = pos + table + least * lane + __popc(p0 & below) + 2u * __popc(p1 & below);
+  uint64_t v = 0;
+#pragma unroll
+  for (uint32_t b = 0; b < 8; ++b) {
+    if (b < n) {
+      uint32_t byte;
+      asm volatile("ld.shared.u8 %0, [%1];"
+                   : "=r"(byte)
+                   : "r"(((at + b) & (kRingBytes - 1)) + ring_s)
+                   : "memory");
+      v |= static_cast<uint64_t>(byte) << (8 * b);
+    }
+  }
+  tc.x = static_cast<uint32_t>(v);
+  tc.xw = v;
+  const uint32_t block = table + least * kLanes + __popc(p0) + 2u * __popc(p1);
+  return pos + ((block + word - 1u) & ~(word - 1u));
 }
 
 // A tile ends well when every lane is back at L and the cursor sits in the
@@ -472,8 +505,8 @@ __device__ __forceinline__ bool run_extent(const LayerDev& L, uint32_t t0, uint3
                                            uint64_t* start, uint32_t* bytes) {
   const unsigned long long* off = reinterpret_cast<const unsigned long long*>(L.offsets);
   const uint64_t a = __ldg(off + t0), b = __ldg(off + t1 + 1);
-  const uint64_t max_tile = state_bytes(L) * kLanes + 2ull * L.tile_n * L.tile_k + 16ull;
-  const bool ok = (a % 16 == 0) && (b % 16 == 0) && b >= a + 1ull * state_bytes(L) * kLanes * (t1 - t0 + 1) &&
+  const uint64_t max_tile = tile_max_bytes(L);
+  const bool ok = (a % 16 == 0) && (b % 16 == 0) && b >= a + 1ull * flush_min_bytes(L) * (t1 - t0 + 1) &&
                   b <= L.stream_bytes && (b - a) <= max_tile * (t1 - t0 + 1) &&
                   (b - a) < (1ull << 31);
   *start = a;
@@ -490,8 +523,8 @@ __device__ __forceinline__ bool run_tile_begin(RunPipe& p, const LayerDev& L, ui
                                                uint64_t b, uint64_t run_start, uint32_t base,
                                                TileCursor& tc, uint32_t lane,
                                                volatile uint32_t* abort, uint32_t* status) {
-  const uint64_t max_tile = state_bytes(L) * kLanes + 2ull * L.tile_n * L.tile_k + 16ull;
-  if (b % 16 != 0 || b < a + state_bytes(L) * kLanes || b - a > max_tile || a < run_start ||
+  const uint64_t max_tile = tile_max_bytes(L);
+  if (b % 16 != 0 || b < a + flush_min_bytes(L) || b - a > max_tile || a < run_start ||
       b > run_start + p.run_bytes)
     return false;
   tc.bytes = static_cast<uint32_t>(b - a);
@@ -506,7 +539,7 @@ __device__ __forceinline__ bool run_tile_begin(RunPipe& p, const LayerDev& L, ui
 __device__ __forceinline__ bool run_tile_end(const LayerDev& L, const TileCursor& tc, bool single) {
   const uint32_t used = tc.pos - tc.cb;
   bool bad = !lanes_at_start(L, tc) || used > tc.bytes || tc.bytes - used >= 16;
-  if (single) bad = !lanes_at_start(L, tc) || tc.bytes != state_bytes(L) * kLanes;
+  if (single) bad = !lanes_at_start(L, tc) || tc.bytes != single_tile_bytes(L);
   return !__any_sync(0xFFFFFFFFu, bad);
 }
 
@@ -545,7 +578,7 @@ __device__ __forceinline__ void tile_group(ChunkPipe& p, const LayerDev& L, cons
 __device__ __forceinline__ bool tile_end(const LayerDev& L, TileCursor& tc, bool single) {
   const uint32_t used = tc.pos - tc.cb * kChunkBytes;
   bool bad = !lanes_at_start(L, tc) || used > tc.bytes || tc.bytes - used >= 16;
-  if (single) bad = !lanes_at_start(L, tc) || tc.bytes != state_bytes(L) * kLanes;
+  if (single) bad = !lanes_at_start(L, tc) || tc.bytes != single_tile_bytes(L);
   tc.cb = tc.last + 1;
   return !__any_sync(0xFFFFFFFFu, bad);
 }

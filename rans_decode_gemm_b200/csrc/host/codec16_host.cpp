@@ -62,14 +62,9 @@ bool tile16_narrow(const std::vector<uint16_t>& sym, const uint32_t* freq, const
     }
     x[l] = static_cast<uint32_t>((static_cast<uint64_t>(v / f) << n) + v % f + cdf[s]);
   }
-  const size_t base = out.size(), len = 4 * kLanes + 2 * words.size();
-  out.resize(base + ((len + 15) & ~size_t(15)), 0);
-  uint8_t* p = out.data() + base;
-  std::memcpy(p, x, 4 * kLanes);  // little-endian host
-  for (size_t k = 0; k < words.size(); ++k) {
-    const uint16_t w = words[words.size() - 1 - k];
-    std::memcpy(p + 4 * kLanes + 2 * k, &w, 2);
-  }
+  uint64_t x64[kLanes];
+  for (uint32_t l = 0; l < kLanes; ++l) x64[l] = x[l];
+  append_tile(out, x64, words);
   return true;
 }
 
@@ -99,14 +94,7 @@ bool tile16_wide(const std::vector<uint16_t>& sym, const uint32_t* freq, const u
       x[l] = v;
     }
   }
-  const size_t base = out.size(), len = 8 * kLanes + 4 * words.size();
-  out.resize(base + ((len + 15) & ~size_t(15)), 0);
-  uint8_t* q = out.data() + base;
-  std::memcpy(q, x, 8 * kLanes);
-  for (size_t k = 0; k < words.size(); ++k) {
-    const uint32_t w = words[words.size() - 1 - k];
-    std::memcpy(q + 8 * kLanes + 4 * k, &w, 4);
-  }
+  append_tile(out, x, words);
   return true;
 }
 

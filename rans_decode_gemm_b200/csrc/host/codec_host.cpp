@@ -126,17 +126,9 @@ bool code_tile(const TileJob& job, uint64_t t, std::vector<uint8_t>& out,
     }
     x[l] = (v / f) * 4096u + (v % f) + job.cdf[s];
   }
-  const size_t base = out.size();
-  const size_t len = 4 * kLanes + 2 * words.size();
-  out.resize(base + ((len + 15) & ~static_cast<size_t>(15)), 0);
-  uint8_t* p = out.data() + base;
-  for (uint32_t l = 0; l < kLanes; ++l) std::memcpy(p + 4 * l, &x[l], 4);  // little-endian host
-  p += 4 * kLanes;
-  for (size_t k = 0; k < words.size(); ++k) {
-    const uint16_t wv = words[words.size() - 1 - k];
-    p[2 * k] = static_cast<uint8_t>(wv);
-    p[2 * k + 1] = static_cast<uint8_t>(wv >> 8);
-  }
+  uint64_t x64[kLanes];
+  for (uint32_t l = 0; l < kLanes; ++l) x64[l] = x[l];
+  append_tile(out, x64, words);
   return true;
 }
 
@@ -167,17 +159,42 @@ bool code_tile_wide(const TileJob& job, const std::vector<uint8_t>& sym, size_t 
       x[l] = v;
     }
   }
-  const size_t base = out.size();
-  const size_t len = 8 * kLanes + 4 * words.size();
-  out.resize(base + ((len + 15) & ~static_cast<size_t>(15)), 0);
-  uint8_t* q = out.data() + base;
-  for (uint32_t l = 0; l < kLanes; ++l) std::memcpy(q + 8 * l, &x[l], 8);  // little-endian host
-  q += 8 * kLanes;
-  for (size_t k = 0; k < words.size(); ++k) {
-    const uint32_t wv = words[words.size() - 1 - k];
-    std::memcpy(q + 4 * k, &wv, 4);
-  }
+  append_tile(out, x, words);
   return true;
+}
+
+// Tile bytes for either state width (Word = the renormalisation word).  A
+// state x >= L needs (bit length + 7) / 8 bytes: 3..4 for 32-bit states
+// (x >= 2^16), 5..8 for wide ones (x >= 2^32); the table stores that count
+// minus the least, bit b of it in plane b.
+template <typename Word>
+void append_tile_impl(std::vector<uint8_t>& out, const uint64_t* x, const std::vector<Word>& pushed) {
+  constexpr bool kWide = sizeof(Word) == 4;
+  constexpr uint32_t kLeast = kWide ? 5 : 3, kTable = kWide ? 8 : 4;
+  uint32_t len[kLanes], planes[2] = {0, 0};
+  size_t states = 0;
+  for (uint32_t l = 0; l < kLanes; ++l) {
+    len[l] = (64u - static_cast<uint32_t>(__builtin_clzll(x[l])) + 7u) / 8u;
+    const uint32_t extra = len[l] - kLeast;
+    planes[0] |= (extra & 1u) << l;
+    planes[1] |= (extra >> 1) << l;
+    states += len[l];
+  }
+  const size_t head = (kTable + states + sizeof(Word) - 1) & ~(sizeof(Word) - 1);
+  const size_t body = head + sizeof(Word) * pushed.size();
+  const size_t base = out.size();
+  out.resize(base + ((body + 15) & ~static_cast<size_t>(15)), 0);
+  uint8_t* p = out.data() + base;
+  std::memcpy(p, planes, kTable);  // little-endian host
+  size_t at = kTable;
+  for (uint32_t l = 0; l < kLanes; ++l) {
+    std::memcpy(p + at, &x[l], len[l]);
+    at += len[l];
+  }
+  for (size_t k = 0; k < pushed.size(); ++k) {
+    const Word wv = pushed[pushed.size() - 1 - k];
+    std::memcpy(p + head + sizeof(Word) * k, &wv, sizeof(Word));
+  }
 }
 
 unsigned worker_count(uint64_t jobs) {
@@ -188,6 +205,14 @@ unsigned worker_count(uint64_t jobs) {
 }
 
 }  // namespace
+
+void append_tile(std::vector<uint8_t>& out, const uint64_t* x, const std::vector<uint16_t>& pushed) {
+  append_tile_impl(out, x, pushed);
+}
+
+void append_tile(std::vector<uint8_t>& out, const uint64_t* x, const std::vector<uint32_t>& pushed) {
+  append_tile_impl(out, x, pushed);
+}
 
 bool layout_valid(uint32_t N, uint32_t K, uint32_t tile_n, uint32_t tile_k) {
   return N > 0 && K > 0 && (tile_n == 128 || tile_n == 256) && tile_k > 0 && tile_k % 16 == 0 &&
@@ -310,8 +335,9 @@ int normalize(const uint64_t* hist, uint32_t alphabet, uint32_t prob_bits, uint3
 uint64_t encode_bound(uint32_t N, uint32_t K, uint32_t tile_n, uint32_t tile_k, bool wide) {
   if (!layout_valid(N, K, tile_n, tile_k)) return 0;
   const uint64_t tiles = static_cast<uint64_t>(N / tile_n) * (K / tile_k);
-  // at most one word per symbol (2 bytes) or per pair (4 bytes): 2 bytes a symbol
-  return tiles * ((wide ? 8ull : 4ull) * kLanes + 2ull * tile_n * tile_k + 16ull);
+  // length table, full-width states, word boundary; at most one word per
+  // symbol (2 bytes) or per pair (4 bytes): 2 bytes a symbol; padding
+  return tiles * ((wide ? 8ull : 4ull) * (kLanes + 1) + 4ull + 2ull * tile_n * tile_k + 16ull);
 }
 
 int encode(uint32_t dtype, const void* w, uint32_t N, uint32_t K, uint32_t tile_n,

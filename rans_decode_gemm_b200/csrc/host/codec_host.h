@@ -1,6 +1,7 @@
 // codec_host.h -- internal interface of the host-side codec (no CUDA).
 #pragma once
 #include <cstdint>
+#include <vector>
 
 namespace anshost {
 
@@ -18,6 +19,15 @@ uint64_t encode_bound(uint32_t N, uint32_t K, uint32_t tile_n, uint32_t tile_k, 
 int encode(uint32_t dtype, const void* w, uint32_t N, uint32_t K, uint32_t tile_n,
            uint32_t tile_k, const uint32_t* freq, uint8_t* stream, uint64_t cap,
            uint64_t* stream_bytes, uint64_t* offsets, uint8_t* raw, bool wide);
+
+// Appends one tile's bytes to `out`: the final-state block (the byte count of
+// every lane's state as a table of bit planes, the 32 states in the fewest
+// whole bytes that hold each, zero bytes up to the word boundary), then the
+// pushed words in decoder order (the reverse of `pushed`), then zero bytes up
+// to a 16-byte boundary.  The u16 form is the 32-bit-state format, the u32
+// form the wide-state one.
+void append_tile(std::vector<uint8_t>& out, const uint64_t* x, const std::vector<uint16_t>& pushed);
+void append_tile(std::vector<uint8_t>& out, const uint64_t* x, const std::vector<uint32_t>& pushed);
 
 // bf16 as whole 16-bit symbols (alphabet 65,536; codec16_host.cpp).
 void histogram16(const uint16_t* w, uint64_t n_weights, uint64_t* hist);

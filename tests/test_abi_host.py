@@ -140,15 +140,18 @@ def test_host_error_paths(ans_lib):
 
 
 def test_single_symbol_layer(oracle, ans_lib):
-    # a constant layer codes to 128 bytes per tile (states only) and decodes
+    # a constant layer codes to 112 bytes per tile and decodes: a zero length
+    # table (every state at L = 2^16 takes the least 3 bytes), 32 states 00 00 01,
+    # 12 bytes of padding
     N, K = 256, 64
     w = np.full(N * K, 0x3C, np.uint8)
     lay = ans.make_layout(ans.FP8_E4M3, N, K, 128, 64)
     cb = ans.ans_build_codebook(ans.ans_histogram_host(w, lay), 256)
     assert cb.freq[0x3C] == 4096
     stream, offsets, _ = ans.ans_encode_tiles(w, lay, cb)
-    assert list(offsets) == [0, 128, 256]
-    assert (np.frombuffer(stream.tobytes(), np.uint32) == 65536).all()
+    assert list(offsets) == [0, 112, 224]
+    tile = bytes(4) + bytes([0, 0, 1]) * 32 + bytes(12)
+    assert stream.tobytes() == tile * 2
     st, out = oracle.decode(ans.FP8_E4M3, stream, offsets, None, N, K, 128, 64, cb.freq_array())
     assert st == 0 and np.array_equal(out, w)
 
