@@ -385,6 +385,54 @@ ans_status ans_gemm_batched(const ans_gemm_job* jobs, uint32_t n_jobs, uint32_t 
                             ans_scale_kind scale_kind, uint32_t group_k, void* d_ws,
                             size_t ws_bytes, uint32_t* d_status, ans_stream_t stream);
 
+/* ---- Versioned on-disk container of a compressed layer ---------------------
+ * "Approaching Shannon Bound", s3.1: the offline stage yields per layer a
+ * shared codebook, a tile offset index and the tile stream (and, for the bf16
+ * split, the raw side stream); the container holds them with the layout they
+ * were coded for, so a layer is compressed once and loaded many times.
+ * Bytes, all little-endian:
+ *   [0, 96)  header: magic "RANSTILE", u32 version (1), u32 header size (96),
+ *            u32 dtype, N, K, tile_n, tile_k, state_bits, prob_bits, alphabet,
+ *            u64 n_tiles, stream bytes, raw bytes, payload bytes, checksum,
+ *            reserved (0);
+ *   payload: freq (alphabet x u32), offsets ((n_tiles + 1) x u64), stream,
+ *            raw, each section starting on a 16-byte boundary of the
+ *            container (zero bytes between them).
+ * The checksum is 64-bit FNV-1a over the header (checksum field zero) and the
+ * payload.  All of it is host memory; nothing is allocated. */
+typedef struct {
+  ans_layout layout;       /* state_bits 0 is written as 32 */
+  uint32_t prob_bits;      /* 12; ANS_BF16_WHOLE: 12..16 (12 or 16 with 64-bit states) */
+  uint32_t alphabet;       /* 16 or 256 as the dtype has it; 65,536 for ANS_BF16_WHOLE */
+  uint64_t stream_bytes;
+  uint64_t raw_bytes;      /* N*K for ANS_BF16_SPLIT, else 0 */
+  const uint32_t* freq;    /* alphabet entries summing to 2^prob_bits */
+  const uint64_t* offsets; /* n_tiles + 1 entries: 0, 16-byte aligned, non-decreasing,
+                              the last = stream_bytes */
+  const uint8_t* stream;
+  const uint8_t* raw;      /* NULL when raw_bytes == 0 */
+  ans_codebook codebook;   /* output of ans_container_read (one-byte formats; zero for
+                              ANS_BF16_WHOLE); ignored by ans_container_write */
+} ans_container;
+
+/* Writes the container of `layer` to h_out (capacity `cap`); *bytes receives
+ * its size (h_out NULL: only the size).  ANS_ERR_ARG / ANS_ERR_SHAPE for a bad
+ * layout, a missing array, a raw size that does not match the dtype or
+ * offsets that break their rule; ANS_ERR_ALPHABET for an alphabet or a
+ * precision the dtype does not take or freq not summing to 2^prob_bits;
+ * ANS_ERR_BUFFER_TOO_SMALL when cap < *bytes. */
+ans_status ans_container_write(const ans_container* layer, uint8_t* h_out, uint64_t cap,
+                               uint64_t* bytes);
+
+/* Reads a container of exactly `bytes` bytes at h_buf (16-byte aligned, kept
+ * alive by the caller while `layer` is used): checks the magic, the version,
+ * the sizes, the checksum, the layout, the codebook and the offsets, then fills
+ * `layer` with the header's fields, views into h_buf (stream and raw 16-byte
+ * aligned) and, for the one-byte formats, the ans_codebook of freq.
+ * ANS_ERR_ARG for a NULL or misaligned argument, ANS_ERR_UNSUPPORTED for
+ * another version, ANS_ERR_CORRUPT for anything else that does not hold. */
+ans_status ans_container_read(const uint8_t* h_buf, uint64_t bytes, ans_container* layer);
+
 #ifdef __cplusplus
 }
 #endif

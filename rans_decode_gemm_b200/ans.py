@@ -30,7 +30,7 @@ EXPORTS = ["ans_status_string", "ans_last_error", "ans_num_tiles", "ans_layout_c
            "ans_encode_tiles", "ans_decode_tiles", "ans_histogram16_host", "ans_build_codebook16",
            "ans_encode_tiles16", "ans_decode_table16", "ans_decode_tiles16", "ans_gemm_workspace", "ans_gemm",
            "ans_gemm_noalloc", "ans_gemm_uncompressed", "ans_gemm_batched_workspace",
-           "ans_gemm_batched"]
+           "ans_gemm_batched", "ans_container_write", "ans_container_read"]
 MAX_BATCH = 8
 
 
@@ -57,6 +57,13 @@ class AnsLayout(C.Structure):
 class AnsTiles(C.Structure):
     _fields_ = [("layout", AnsLayout), ("codebook", AnsCodebook), ("stream", C.c_void_p),
                 ("stream_bytes", C.c_uint64), ("offsets", C.c_void_p), ("raw", C.c_void_p)]
+
+
+class AnsContainer(C.Structure):
+    _fields_ = [("layout", AnsLayout), ("prob_bits", C.c_uint32), ("alphabet", C.c_uint32),
+                ("stream_bytes", C.c_uint64), ("raw_bytes", C.c_uint64), ("freq", C.c_void_p),
+                ("offsets", C.c_void_p), ("stream", C.c_void_p), ("raw", C.c_void_p),
+                ("codebook", AnsCodebook)]
 
 
 class AnsGemmJob(C.Structure):
@@ -101,6 +108,8 @@ def load():
             L.ans_gemm_uncompressed.argtypes = [P, u32, P, P, i32, P, u32, P, P, sz, P, P]
             L.ans_gemm_batched_workspace.argtypes = [P, u32, u32, i32, P]
             L.ans_gemm_batched.argtypes = [P, u32, u32, i32, u32, P, sz, P, P]
+            L.ans_container_write.argtypes = [P, P, u64, P]
+            L.ans_container_read.argtypes = [P, u64, P]
             for name in EXPORTS:
                 if name not in ("ans_status_string", "ans_last_error", "ans_num_tiles"):
                     getattr(L, name).restype = i32
@@ -324,6 +333,70 @@ def ans_gemm_batched(jobs, M: int, scale_kind: int, group_k: int, d_ws, ws_bytes
            "ans_gemm_batched")
 
 
+def ans_container_write(layout: AnsLayout, prob_bits: int, freq, stream: np.ndarray,
+                        offsets: np.ndarray, raw: np.ndarray | None = None) -> np.ndarray:
+    """The versioned container of a compressed layer (host arrays) as uint8[]."""
+    freq = np.ascontiguousarray(freq, dtype=np.uint32)
+    stream = np.ascontiguousarray(stream, dtype=np.uint8)
+    offsets = np.ascontiguousarray(offsets, dtype=np.uint64)
+    raw = None if raw is None else np.ascontiguousarray(raw, dtype=np.uint8)
+    c = AnsContainer(layout, prob_bits, freq.size, stream.size, 0 if raw is None else raw.size,
+                     _ptr(freq).value, _ptr(offsets).value, _ptr(stream).value,
+                     None if raw is None else _ptr(raw).value, AnsCodebook())
+    L = load()
+    nbytes = C.c_uint64(0)
+    _check(L.ans_container_write(C.byref(c), None, 0, C.byref(nbytes)), "ans_container_write")
+    out = np.empty(nbytes.value, np.uint8)
+    _check(L.ans_container_write(C.byref(c), _ptr(out), out.size, C.byref(nbytes)),
+           "ans_container_write")
+    return out
+
+
+def _aligned_bytes(n: int) -> np.ndarray:
+    """uint8[n] starting on a 16-byte boundary (ans_container_read's rule)."""
+    block = np.empty(n + 16, np.uint8)
+    skip = (-block.ctypes.data) % 16
+    return block[skip:skip + n]
+
+
+def ans_container_read(buf) -> dict:
+    """A container's layer: layout, prob_bits, freq, offsets, stream, raw (views
+    into the container's bytes) and, for the one-byte formats, the codebook."""
+    buf = np.asarray(buf, dtype=np.uint8)
+    if buf.ctypes.data % 16 != 0 or not buf.flags["C_CONTIGUOUS"]:
+        aligned = _aligned_bytes(buf.size)
+        aligned[:] = buf
+        buf = aligned
+    c = AnsContainer()
+    _check(load().ans_container_read(_ptr(buf), buf.size, C.byref(c)), "ans_container_read")
+    base = buf.ctypes.data
+
+    def view(addr, nbytes):
+        return buf[addr - base:addr - base + nbytes]
+    n_tiles = ans_num_tiles(c.layout)
+    return {"layout": c.layout, "prob_bits": c.prob_bits,
+            "freq": view(c.freq, 4 * c.alphabet).view(np.uint32),
+            "offsets": view(c.offsets, 8 * (n_tiles + 1)).view(np.uint64),
+            "stream": view(c.stream, c.stream_bytes),
+            "raw": view(c.raw, c.raw_bytes) if c.raw_bytes else None,
+            "codebook": c.codebook if c.alphabet <= 256 else None}
+
+
+def save_layer(path: str, layout: AnsLayout, prob_bits: int, freq, stream, offsets, raw=None):
+    """Writes a compressed layer's container to a file."""
+    ans_container_write(layout, prob_bits, freq, stream, offsets, raw).tofile(path)
+
+
+def load_layer(path: str) -> dict:
+    """Reads a container file (into 16-byte aligned memory) -> ans_container_read."""
+    size = os.path.getsize(path)
+    buf = _aligned_bytes(size)
+    with open(path, "rb") as fh:
+        if fh.readinto(memoryview(buf)) != size:
+            raise AnsError(6, "load_layer", f"{path}: short read")
+    return ans_container_read(buf)
+
+
 def _set_plan_limits(max_ctas: int = 0, max_producers: int = 0, force_shared: bool = False):
     """Internal test hook of libans.so (not part of include/ans.h): caps on the
     CTAs and producer warps of every later fused-GEMM plan in this process,
@@ -382,6 +455,19 @@ class CompressedLayer:
         cb = 2 * self.codebook.alphabet
         return int(self.h_stream.size + self.h_offsets.size * 8 + cb +
                    (self.h_raw.size if self.h_raw is not None else 0))
+
+    def save(self, path: str):
+        """Writes the layer's container file (ans_container_write)."""
+        save_layer(path, self.layout, self.codebook.prob_bits, self.codebook.freq_array(),
+                   self.h_stream, self.h_offsets, self.h_raw)
+
+    @classmethod
+    def load(cls, path: str, device="cuda"):
+        """A layer from its container file (ans_container_read), uploaded to `device`."""
+        d = load_layer(path)
+        if d["codebook"] is None:
+            raise AnsError(1, "CompressedLayer.load", "a 16-bit-symbol layer has no ans_tiles form")
+        return cls(d["layout"], d["codebook"], d["stream"], d["offsets"], d["raw"], device)
 
     @classmethod
     def from_weights(cls, h_w: np.ndarray, layout: AnsLayout, hist=None, device="cuda"):

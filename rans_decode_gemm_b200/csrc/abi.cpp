@@ -216,6 +216,46 @@ ans_status run_gemm(const uint16_t* d_X, uint32_t M, const ansdev::LayerDev& L, 
                         stream);
 }
 
+// Layout, alphabet, precision and raw size of a container's layer: ANS_OK,
+// or the status that ans_container_write reports.
+ans_status check_container_fields(const ans_container* c) {
+  ans_status st = check_any_layout(&c->layout);
+  if (st != ANS_OK) return st;
+  const uint32_t dtype = c->layout.dtype;
+  const bool whole = dtype == ANS_BF16_WHOLE;
+  if (c->alphabet != (whole ? 65536u : alphabet_of(dtype))) return ANS_ERR_ALPHABET;
+  if (whole ? (c->prob_bits < 12 || c->prob_bits > 16 ||
+               (c->layout.state_bits == 64 && c->prob_bits != 12 && c->prob_bits != 16))
+            : c->prob_bits != 12)
+    return ANS_ERR_ALPHABET;
+  const uint64_t raw = dtype == ANS_BF16_SPLIT ? static_cast<uint64_t>(c->layout.N) * c->layout.K : 0;
+  if (c->raw_bytes != raw) return ANS_ERR_ARG;
+  const uint64_t bound = anshost::encode_bound(c->layout.N, c->layout.K, c->layout.tile_n,
+                                               c->layout.tile_k, c->layout.state_bits == 64);
+  if (c->stream_bytes > bound) return ANS_ERR_ARG;
+  return ANS_OK;
+}
+
+anshost::ContainerLayer to_host_layer(const ans_container* c) {
+  anshost::ContainerLayer h;
+  h.dtype = c->layout.dtype;
+  h.N = c->layout.N;
+  h.K = c->layout.K;
+  h.tile_n = c->layout.tile_n;
+  h.tile_k = c->layout.tile_k;
+  h.state_bits = c->layout.state_bits == 64 ? 64u : 32u;
+  h.prob_bits = c->prob_bits;
+  h.alphabet = c->alphabet;
+  h.n_tiles = static_cast<uint64_t>(c->layout.N / c->layout.tile_n) * (c->layout.K / c->layout.tile_k);
+  h.stream_bytes = c->stream_bytes;
+  h.raw_bytes = c->raw_bytes;
+  h.freq = c->freq;
+  h.offsets = c->offsets;
+  h.stream = c->stream;
+  h.raw = c->raw;
+  return h;
+}
+
 }  // namespace
 
 extern "C" {
@@ -703,6 +743,57 @@ ans_status ans_gemm_batched(const ans_gemm_job* jobs, uint32_t n_jobs, uint32_t 
                                         d_status, s);
     if (e != cudaSuccess) return cuda_fail(e, "ans_gemm_batched");
   }
+  return ANS_OK;
+}
+
+ans_status ans_container_write(const ans_container* layer, uint8_t* h_out, uint64_t cap,
+                               uint64_t* bytes) {
+  if (!layer || !bytes) return ANS_ERR_ARG;
+  ans_status st = check_container_fields(layer);
+  if (st != ANS_OK) return st;
+  const anshost::ContainerLayer h = to_host_layer(layer);
+  const int r = anshost::container_check(h);
+  if (r == 3) return ANS_ERR_ALPHABET;
+  if (r != 0) return ANS_ERR_ARG;
+  const int w = anshost::container_write(h, h_out, cap, bytes);
+  if (w == 4) return ANS_ERR_BUFFER_TOO_SMALL;
+  return w == 0 ? ANS_OK : ANS_ERR_ARG;
+}
+
+ans_status ans_container_read(const uint8_t* h_buf, uint64_t bytes, ans_container* layer) {
+  if (!h_buf || !layer || reinterpret_cast<uintptr_t>(h_buf) % 16 != 0) return ANS_ERR_ARG;
+  anshost::ContainerLayer h;
+  const int r = anshost::container_read(h_buf, bytes, &h);
+  if (r == 8) return ANS_ERR_UNSUPPORTED;
+  if (r != 0) return ANS_ERR_CORRUPT;
+  ans_container c;
+  std::memset(&c, 0, sizeof(c));
+  c.layout = ans_layout{h.dtype, h.N, h.K, h.tile_n, h.tile_k, h.state_bits};
+  c.prob_bits = h.prob_bits;
+  c.alphabet = h.alphabet;
+  c.stream_bytes = h.stream_bytes;
+  c.raw_bytes = h.raw_bytes;
+  c.freq = h.freq;
+  c.offsets = h.offsets;
+  c.stream = h.stream;
+  c.raw = h.raw;
+  // a header that passed its checksum may still describe an impossible layer
+  if ((h.state_bits != 32 && h.state_bits != 64) || check_container_fields(&c) != ANS_OK)
+    return ANS_ERR_CORRUPT;
+  if (to_host_layer(&c).n_tiles != h.n_tiles || anshost::container_check(h) != 0)
+    return ANS_ERR_CORRUPT;
+  if (c.alphabet <= 256) {
+    c.codebook.alphabet = c.alphabet;
+    c.codebook.prob_bits = c.prob_bits;
+    uint32_t run = 0;
+    for (uint32_t s = 0; s < c.alphabet; ++s) {
+      c.codebook.freq[s] = static_cast<uint16_t>(c.freq[s]);
+      c.codebook.cdf[s] = static_cast<uint16_t>(run);
+      run += c.freq[s];
+    }
+    c.codebook.cdf[c.alphabet] = static_cast<uint16_t>(run);
+  }
+  *layer = c;
   return ANS_OK;
 }
 

@@ -42,4 +42,27 @@ int encode16(const uint16_t* w, uint32_t N, uint32_t K, uint32_t tile_n, uint32_
 uint64_t table16_bytes(const uint32_t* freq);
 int table16(const uint32_t* freq, uint32_t prob_bits, uint8_t* out, uint64_t bytes);
 
+// A compressed layer as the on-disk container holds it (container_host.cpp).
+// Pointers are host memory; after container_read they point into the buffer.
+struct ContainerLayer {
+  uint32_t dtype, N, K, tile_n, tile_k, state_bits, prob_bits, alphabet;
+  uint64_t n_tiles, stream_bytes, raw_bytes;
+  const uint32_t* freq;
+  const uint64_t* offsets;
+  const uint8_t* stream;
+  const uint8_t* raw;
+};
+// Arrays of a layer to be written: 0 ok, 1 missing array, 3 freq not summing
+// to 2^prob_bits, 6 offsets not 0, 16-byte aligned, non-decreasing, ending at
+// the stream size.
+int container_check(const ContainerLayer& c);
+// Size of the container of a layer (0 when a size is out of range).
+uint64_t container_bytes(const ContainerLayer& c);
+// 0 ok (*written = size; out may be NULL to query it), 1 size out of range,
+// 4 capacity too small.
+int container_write(const ContainerLayer& c, uint8_t* out, uint64_t cap, uint64_t* written);
+// 0 ok, 6 not a container or damaged (magic, sizes, checksum), 8 another
+// version.  Fills c with the header's fields and views into buf.
+int container_read(const uint8_t* buf, uint64_t bytes, ContainerLayer* c);
+
 }  // namespace anshost
