@@ -232,3 +232,33 @@ def test_dtype_constants_agree_with_the_header():
     # the workload generators use the same dtype numbers
     assert (WL.INT4, WL.BF16_SPLIT, WL.FP8_E4M3, WL.INT4_PAIRS, WL.INT8, WL.FP4_E2M1,
             WL.FP4_PAIRS) == (0, 1, 2, 3, 4, 5, 6)
+
+
+@pytest.mark.parametrize("state_bits", [32, 64])
+def test_encode_bound_holds_for_the_costliest_layer(oracle, ans_lib, state_bits):
+    # every symbol of the layer has f = 1 (12 bits each, the most a symbol can
+    # cost): the stream comes close to the bound (2 bytes a symbol, plus the
+    # full-width state block, the word boundary and the padding of every tile)
+    # and stays under it; host bytes equal the oracle's
+    N, K = 256, 128
+    freq = np.zeros(256, np.uint64)
+    freq[0] = 4096 - 255
+    freq[1:] = 1
+    rng = np.random.default_rng(41)
+    w = rng.integers(1, 256, size=N * K).astype(np.uint8)
+    lay = ans.make_layout(ans.FP8_E4M3, N, K, 128, 64, state_bits)
+    cb = ans.AnsCodebook()
+    cb.alphabet, cb.prob_bits = 256, 12
+    run = 0
+    for s in range(256):
+        cb.freq[s], cb.cdf[s] = int(freq[s]), run
+        run += int(freq[s])
+    cb.cdf[256] = run
+    stream, offsets, _ = ans.ans_encode_tiles(w, lay, cb)
+    bound = ans.ans_encode_bound(lay)
+    assert stream.size <= bound
+    assert stream.size > 0.7 * bound
+    st, ref, ref_off, _ = oracle.encode(ans.FP8_E4M3, w, N, K, 128, 64, freq.astype(np.uint32),
+                                        state_bits=state_bits)
+    assert st == 0 and np.array_equal(stream, ref) and np.array_equal(offsets, ref_off)
+    assert bound == oracle.encode_bound(N, K, 128, 64, state_bits)
