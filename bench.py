@@ -61,7 +61,8 @@ TRAFFIC_PROFILE = "profiles/fused_gemm_local_fp8_405b_m16.json"
 
 def workload_name(name, state_bits, M):
     fmt = ("64-bit lane states, 32-bit words, one renormalisation test per symbol pair"
-           if state_bits == 64 else "32-bit lane states, 16-bit words")
+           if state_bits == 64 else "32-bit lane states, 16-bit words") + \
+        ", final states flushed in whole bytes"
     if name == "fp8_405b":
         return ("405B-shaped fp8 e4m3 53248x16384, w~N(0,0.02) / (row amax/448), fp32 row "
                 "scales, 8-bit symbols, 128x128 tiles, 32 lanes, 12-bit freqs, "
